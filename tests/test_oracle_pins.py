@@ -1,0 +1,389 @@
+"""Pins for the CPU oracle: hand-worked examples from the paper's equations,
+closed forms, invariants and brute force on tiny inputs -- never the oracle's
+own formula retyped.  CPU only."""
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from conftest import read_golden
+
+EPS = 1e-5
+
+
+def bf16(vals):
+    return synth.f32_to_bf16_bits(np.asarray(vals, np.float32))
+
+
+def bf16_val(bits):
+    return synth.bf16_bits_to_f32(bits)
+
+
+# ----------------------------------------------------------------------------
+# INT4 absmean (Eq. 6-7)
+# ----------------------------------------------------------------------------
+def test_int4_hand_examples():
+    g = read_golden("int4_hand.txt")
+    for xs, codes, beta in zip(g["x"], g["codes"], g["beta"]):
+        c, b, s = oracle.quant_int4(bf16([xs]))
+        assert c[0].tolist() == [int(v) for v in codes]
+        assert abs(float(b[0]) - beta[0]) < 1e-6
+        assert abs(float(s[0]) - beta[0] / math.sqrt(7)) < 1e-6
+
+
+def test_int4_constant_row_closed_form():
+    # x = c everywhere: beta = |c| exactly, sqrt7*c/(|c|+eps) ~ +-2.6457 -> +-3
+    for c in (0.75, -3.0, 1e-3, 96.0):
+        codes, beta, _ = oracle.quant_int4(bf16([[c] * 64]))
+        assert float(beta[0]) == float(bf16_val(bf16([c]))[0].__abs__())
+        assert set(codes[0].tolist()) == {3 if c > 0 else -3}
+
+
+def test_int4_zero_row():
+    codes, beta, scale = oracle.quant_int4(np.zeros((1, 32), np.uint16))
+    assert not codes.any() and beta[0] == 0 and scale[0] == 0
+
+
+def test_int4_brute_force_nearest_code():
+    # Each code is the nearest of the 16 INT4 values to x*sqrt7/(beta+eps),
+    # ties to the even one (brute force over the code set).
+    x = synth.gaussian_bf16(synth.rng(11), (8, 96), outlier_channels=(3,), outlier_scale=9.0)
+    codes, beta, _ = oracle.quant_int4(x)
+    xf = bf16_val(x).astype(np.float32)
+    for m in range(x.shape[0]):
+        mult = np.float32(np.float32(math.sqrt(7)) / (np.float32(beta[m]) + np.float32(EPS)))
+        for k in range(x.shape[1]):
+            v = float(np.float32(xf[m, k] * mult))
+            best = min(range(-8, 8), key=lambda c: (abs(v - c), c % 2))
+            assert codes[m, k] == best
+    assert codes.min() >= -8 and codes.max() <= 7
+
+
+def test_int4_beta_is_correctly_rounded_mean():
+    x = synth.gaussian_bf16(synth.rng(5), (4, 4096))
+    _, beta, _ = oracle.quant_int4(x)
+    for m in range(4):
+        mean = math.fsum(abs(float(v)) for v in bf16_val(x[m])) / 4096
+        assert abs(float(beta[m]) - mean) <= abs(mean) * 2 ** -24
+
+
+def test_int4_rejects_inexact_sums():
+    # a row whose |x| sum cannot be held exactly in fp64
+    row = bf16([[1e30, 1e-30] + [0.0] * 30])
+    with pytest.raises(ValueError):
+        oracle.quant_int4(row)
+
+
+# ----------------------------------------------------------------------------
+# FP4 E2M1 (Eq. 8-9)
+# ----------------------------------------------------------------------------
+def test_fp4_hand_example():
+    g = read_golden("fp4_hand.txt")
+    code4, tv, p, scale = oracle.quant_fp4(bf16(g["x"]))
+    assert p[0] == int(g["p"][0][0])
+    assert (tv[0] / 2.0).tolist() == g["values"][0]
+    assert code4[0].tolist() == [int(v) for v in g["codes"][0]]
+    assert scale[0] == 1.0
+
+
+@pytest.mark.parametrize("gmax,p", [(6.0, 0), (6.03125, 1), (3.0, -1), (3.015625, 0),
+                                    (12.0, 1), (0.75, -3), (1.5, -2), (1e-3, -12)])
+def test_fp4_scale_exponent_closed_form(gmax, p):
+    # p = ceil(log2(max|x| / 6)): the smallest power of two that covers the max
+    row = bf16([[gmax, -gmax / 4, 0.0, gmax / 3]])
+    g = float(bf16_val(row)[0, 0])
+    _, _, pp, scale = oracle.quant_fp4(row)
+    assert pp[0] == p
+    assert g <= 6 * 2.0 ** p and g > 6 * 2.0 ** (p - 1)
+    assert scale[0] == np.float32(2.0 ** p)
+
+
+def test_fp4_exhaustive_bf16_against_midpoint_table():
+    # Every positive and negative finite bf16 below 6 at p = 0, against a rounding
+    # written from the grid midpoints and the even-encoding tie rule.
+    mids = [(0.25, 0, 0), (0.75, 1, 2), (1.25, 2, 2), (1.75, 3, 4), (2.5, 4, 4),
+            (3.5, 5, 6), (5.0, 6, 6)]       # (midpoint, code below, code at tie)
+
+    def table_code(v):
+        a = abs(v)
+        code = 7
+        for mid, below, tie in mids:
+            if a < mid:
+                code = below
+                break
+            if a == mid:
+                code = tie
+                break
+        return code
+
+    bits = np.arange(0, 0x8000, dtype=np.uint16)
+    vals = bf16_val(bits)
+    keep = np.isfinite(vals) & (vals <= 6.0)
+    bits = bits[keep]
+    for sign in (0, 0x8000):
+        b = (bits | sign).astype(np.uint16)
+        row = np.concatenate([b, bf16([6.0])]).reshape(1, -1)   # pin max |x| = 6 -> p = 0
+        code4, tv, p, _ = oracle.quant_fp4(row)
+        assert p[0] == 0
+        v = bf16_val(row[0])
+        for j in range(row.shape[1]):
+            mag_code = table_code(float(v[j]))
+            expect = mag_code | (8 if (v[j] < 0 and mag_code != 0) else 0)
+            assert code4[0, j] == expect, (float(v[j]), code4[0, j], expect)
+        grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6])
+        assert np.array_equal(np.abs(tv[0]) / 2.0, grid[code4[0] & 7])
+
+
+# ----------------------------------------------------------------------------
+# Top-K + INT8 (Eq. 1)
+# ----------------------------------------------------------------------------
+def test_topk_int8_hand_example():
+    g = read_golden("topk_int8_hand.txt")
+    codes, mask, gamma, scale = oracle.sparsify_a8(bf16(g["x"]), int(g["keep"][0][0]))
+    assert mask[0].tolist() == [int(v) for v in g["mask"][0]]
+    assert codes[0].tolist() == [int(v) for v in g["codes"][0]]
+    assert gamma[0] == g["gamma"][0][0]
+    assert abs(scale[0] - 3 / 127) < 1e-8
+    assert oracle.pack_mask_bits(mask)[0, 0] == int(g["mask_word"][0][0])
+
+
+def _check_topk_invariants(mag, mask, keep):
+    """Exactly keep survivors; every survivor's magnitude >= every dropped one's;
+    at the threshold magnitude, survivors precede the dropped by index."""
+    kept = np.flatnonzero(mask)
+    dropped = np.flatnonzero(mask == 0)
+    assert kept.size == keep
+    if dropped.size and kept.size:
+        thr = mag[kept].min()
+        assert thr >= mag[dropped].max()
+        tk = kept[mag[kept] == thr]
+        td = dropped[mag[dropped] == thr]
+        if td.size:
+            assert tk.max() < td.min()
+
+
+def test_topk_invariants_heavy_tailed_and_ties():
+    g = synth.rng(3)
+    x = synth.student_t_bf16(g, (6, 512))
+    x[1, ::3] = 0                      # many tied zeros
+    x[2, :] = bf16([[0.5] * 512])[0]   # all tied
+    for keep in (1, 128, 256, 511, 512):
+        codes, mask, gamma, _ = oracle.sparsify_a8(x, keep)
+        mag = np.abs(bf16_val(x).astype(np.float64))
+        for m in range(6):
+            _check_topk_invariants(mag[m], mask[m], keep)
+            assert gamma[m] == mag[m].max()
+            assert np.all(codes[m][mask[m] == 0] == 0)
+            assert codes[m].min() >= -127 and codes[m].max() <= 127
+
+
+def test_topk_brute_force_tiny():
+    # all subsets of size keep: the chosen one is the unique lexicographic maximum
+    # of (sorted magnitudes desc, then smaller indices)
+    import itertools
+    g = synth.rng(9)
+    for trial in range(20):
+        x = bf16(np.round(g.standard_normal(7) * 2) / 2)       # many ties
+        mag = np.abs(bf16_val(x).astype(np.float64))
+        keep = 1 + trial % 6
+        _, mask, _, _ = oracle.sparsify_a8(x.reshape(1, -1), keep)
+        best = max(itertools.combinations(range(7), keep),
+                   key=lambda s: (sorted(mag[list(s)], reverse=True), [-i for i in s]))
+        assert sorted(np.flatnonzero(mask[0]).tolist()) == list(best)
+
+
+def test_int8_codes_bruteforce_nearest():
+    x = synth.student_t_bf16(synth.rng(4), (3, 200))
+    codes, mask, gamma, _ = oracle.sparsify_a8(x, 200)
+    xf = bf16_val(x)
+    for m in range(3):
+        mult = np.float32(np.float32(127.0) / (np.float32(gamma[m]) + np.float32(EPS)))
+        for k in range(200):
+            v = float(np.float32(xf[m, k] * mult))
+            assert abs(v - codes[m, k]) <= 0.5
+            if abs(v - codes[m, k]) == 0.5:
+                assert codes[m, k] % 2 == 0
+
+
+# ----------------------------------------------------------------------------
+# ReLU^2-GLU (Eq. 5)
+# ----------------------------------------------------------------------------
+def test_relu2_glu_hand_example():
+    g = read_golden("relu2glu_hand.txt")
+    gate, up = bf16(g["gate"]), bf16(g["up"])
+    for keep, mask_e, codes_e in zip(g["keep"], g["mask"], g["codes"]):
+        codes, mask, gamma, _, h = oracle.relu2_glu(gate, up, int(keep[0]), want_h=True)
+        assert h[0].tolist() == g["h"][0]
+        assert mask[0].tolist() == [int(v) for v in mask_e]
+        assert codes[0].tolist() == [int(v) for v in codes_e]
+        assert gamma[0] == 4.5
+
+
+def test_relu2_glu_closed_form():
+    g = synth.rng(21)
+    gate = synth.gaussian_bf16(g, (4, 300))
+    up = synth.gaussian_bf16(g, (4, 300))
+    _, mask, _, _, h = oracle.relu2_glu(gate, up, 150, want_h=True)
+    gf = bf16_val(gate).astype(np.float64)
+    uf = bf16_val(up).astype(np.float64)
+    exact = uf * np.maximum(gf, 0) ** 2
+    assert np.all(h[gf <= 0] == 0)                       # gate <= 0 gives exactly 0
+    assert np.all(np.abs(h - exact) <= np.abs(exact) * 2 ** -22)   # two fp32 roundings
+    for m in range(4):
+        _check_topk_invariants(np.abs(h[m].astype(np.float64)), mask[m], 150)
+
+
+# ----------------------------------------------------------------------------
+# Ternary weights (Eq. 2)
+# ----------------------------------------------------------------------------
+def test_ternary_hand_example():
+    g = read_golden("ternary_hand.txt")
+    w = np.array(g["w"], np.float32)
+    t, alpha = oracle.ternary_quantize(w)
+    assert abs(float(alpha) - g["alpha"][0][0]) < 1e-9
+    assert t.tolist() == [[int(v) for v in r] for r in g["codes"]]
+    assert oracle.pack_ternary2(t)[0, 0] == int(g["packed_row0"][0][0])
+
+
+def test_ternary_alpha_exact_cases():
+    # means that are exactly representable must come out exactly
+    w = np.array([[1, -2], [3, -4]], np.float32) * np.float32(0.125)
+    assert oracle.ternary_alpha(w) == np.float32(0.3125)
+    w = np.full((7, 33), -0.0213, np.float32)
+    assert oracle.ternary_alpha(w) == np.float32(0.0213)
+    assert oracle.ternary_alpha(np.zeros((3, 8), np.float32)) == 0.0
+    # subnormal entries are summed too
+    tiny = np.float32(2.0 ** -140)
+    assert oracle.ternary_alpha(np.full((2, 2), tiny, np.float32)) == tiny
+
+
+def test_ternary_alpha_against_fsum():
+    w = synth.latent_weights_f32(synth.rng(8), 64, 96)
+    a = float(oracle.ternary_alpha(w))
+    mean = math.fsum(abs(float(v)) for v in w.ravel()) / w.size
+    assert abs(a - mean) <= mean * 2 ** -24
+
+
+def test_round_fraction_to_f32_matches_numpy_single_rounding():
+    g = synth.rng(1)
+    vals = np.concatenate([g.standard_normal(2000) * 10.0 ** g.integers(-40, 38, 2000),
+                           [2.0 ** -149, 2.0 ** -149 * 1.5, 2.0 ** -126 * 0.75, 1.0 + 2.0 ** -24]])
+    for v in np.abs(vals):
+        if v == 0 or v >= 3.4e38:
+            continue
+        assert oracle.round_fraction_to_f32(Fraction(float(v))) == np.float32(v)
+
+
+def test_ternary_codes_bruteforce():
+    w = synth.latent_weights_f32(synth.rng(6), 16, 64)
+    t, alpha = oracle.ternary_quantize(w)
+    d = np.float32(np.float32(alpha) + np.float32(EPS))
+    for n in range(16):
+        for k in range(64):
+            q = float(np.float32(w[n, k] / d))
+            best = min((-1, 0, 1), key=lambda c: (abs(q - c), c % 2))
+            assert t[n, k] == best
+    # about 31% of Gaussian weights land on 0 (|w| < alpha/2, alpha ~ 0.8 sigma)
+    frac0 = np.mean(t == 0)
+    assert 0.2 < frac0 < 0.45
+
+
+# ----------------------------------------------------------------------------
+# GEMM (Y = Q_x(X) Q_w(W)^T)
+# ----------------------------------------------------------------------------
+def test_gemm_hand_example():
+    gi = read_golden("int4_hand.txt")
+    gt = read_golden("ternary_hand.txt")
+    gg = read_golden("gemm_hand.txt")
+    c, _, s = oracle.quant_int4(bf16([gi["x"][0]]))
+    t, alpha = oracle.ternary_quantize(np.array(gt["w"], np.float32))
+    acc, y = oracle.gemm(c, s, t, alpha)
+    assert acc[0].tolist() == [int(v) for v in gg["acc"][0]]
+    yv = bf16_val(y[0])
+    for a, b in zip(yv, gg["y"][0]):
+        assert abs(a - b) <= abs(b) * 2 ** -8
+
+
+def test_gemm_bruteforce_tiny_nonsquare():
+    g = synth.rng(2)
+    M, N, K = 5, 7, 33
+    a = g.integers(-128, 128, (M, K)).astype(np.int8)
+    t = g.integers(-1, 2, (N, K)).astype(np.int8)
+    s = (g.random(M) + 0.1).astype(np.float32)
+    alpha = np.float32(0.0173)
+    acc, y = oracle.gemm(a, s, t, alpha)
+    for m in range(M):
+        for n in range(N):
+            ref = sum(int(a[m, k]) * int(t[n, k]) for k in range(K))
+            assert acc[m, n] == ref
+            exact = Fraction(ref) * Fraction(float(s[m])) * Fraction(float(alpha))
+            yv = Fraction(float(bf16_val(y[m:m + 1, n])[0]))
+            assert abs(yv - exact) <= abs(exact) * Fraction(1, 256)   # half a bf16 ulp
+    # row selection returns the same rows
+    acc2, _ = oracle.gemm(a, s, t, alpha, rows=[4, 0])
+    assert np.array_equal(acc2, acc[[4, 0]])
+
+
+def test_gemm_alpha_groups():
+    g = synth.rng(12)
+    a = g.integers(-8, 8, (3, 16)).astype(np.int8)
+    t = g.integers(-1, 2, (6, 16)).astype(np.int8)
+    s = np.ones(3, np.float32)
+    _, y = oracle.gemm(a, s, t, np.array([1.0, 2.0], np.float32), alpha_group=3)
+    acc, y1 = oracle.gemm(a, s, t, np.float32(1.0))
+    assert np.array_equal(bf16_val(y[:, :3]), bf16_val(y1[:, :3]))
+    assert np.array_equal(bf16_val(y[:, 3:]), 2 * bf16_val(y1[:, 3:]))
+
+
+def test_gemm_end_to_end_dequant_matches_fp64():
+    # y ~ (dequantized X) . (dequantized W)^T in fp64, the product the method defines
+    x, w = synth.tiny_inputs(0)
+    c, _, s = oracle.quant_int4(x)
+    t, alpha = oracle.ternary_quantize(w)
+    _, y = oracle.gemm(c, s, t, alpha)
+    ref = (c.astype(np.float64) * s[:, None]) @ (t.astype(np.float64) * float(alpha)).T
+    err = np.abs(bf16_val(y).astype(np.float64) - ref).max(axis=1) / np.linalg.norm(ref, axis=1)
+    assert err.max() < 1e-2
+
+
+# ----------------------------------------------------------------------------
+# KV cache
+# ----------------------------------------------------------------------------
+def test_kv_hand_example():
+    g = read_golden("kv_hand.txt")
+    kv = bf16(g["x"]).reshape(1, 1, 8)
+    codes, scale = oracle.kv_quant(kv, bits=3, bos_pos=-1)
+    assert codes[0, 0].tolist() == [int(v) for v in g["codes3"][0]]
+    assert abs(scale[0, 0] - g["scale3"][0][0]) < 1e-6
+    assert oracle.pack_kv3(codes)[0, 0].tolist() == [int(v) for v in g["packed3"][0]]
+    codes4, scale4 = oracle.kv_quant(kv, bits=3, bos_pos=0)       # BOS row at 4 bits
+    assert codes4[0, 0].tolist() == [int(v) for v in g["codes4"][0]]
+    assert abs(scale4[0, 0] - g["scale4"][0][0]) < 1e-6
+
+
+def test_kv_ranges_and_roundtrip_bound():
+    k, _ = synth.kv_inputs(0, positions=9, heads=3, head_dim=128)
+    codes, scale = oracle.kv_quant(k, bits=3, bos_pos=0)
+    x = bf16_val(k).astype(np.float64)
+    for t in range(9):
+        b = 4 if t == 0 else 3
+        q = 2 ** (b - 1) - 1
+        c = codes[t].astype(np.int64)
+        assert c.min() >= 1 and c.max() <= 2 ** b - 1        # symmetric: code 0 unused
+        deq = (c - 2 ** (b - 1)) * scale[t][:, None].astype(np.float64)
+        gamma = np.abs(x[t]).max(axis=1)
+        assert np.all(np.abs(deq - x[t]) <= (gamma / (2 * q))[:, None] * (1 + 1e-4))
+
+
+# ----------------------------------------------------------------------------
+# Storage layouts
+# ----------------------------------------------------------------------------
+def test_pack_layouts():
+    assert oracle.pack_nibbles(np.array([1, -2], np.int8)).tolist() == [0xE1]
+    assert oracle.pack_ternary2(np.array([1, -1, 0, 1], np.int8)).tolist() == [0x4D]
+    m = np.zeros((1, 40), np.uint8)
+    m[0, [0, 31, 32, 39]] = 1
+    assert oracle.pack_mask_bits(m).tolist() == [[0x80000001, 0x81]]
