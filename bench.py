@@ -1,0 +1,527 @@
+"""Benchmark: one BitNet a4.8 decoder layer's BitLinear forward path, 7B shapes.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--afmt int4|fp4]
+
+A step is one pass of the whole hot path over one batch of M = 8 x 4096 tokens
+(hidden 4096, 32 heads x 128, FFN 11008), all on the GPU through the C ABI:
+
+  pack_ternary x5      latent fp32 W -> ternary int8 operand + alpha (Eq. 2),
+                       re-ternarized every pass as in the paper's forward
+  quant_a4(X_attn)     INT4 absmean (Eq. 6-7) or FP4 E2M1 (Eq. 8-9)
+  gemm  QKV            [M x 4096] x [12288 x 4096]^T
+  kv_quant3  K, V      3-bit post-RoPE KV, position 0 at 4 bits
+  sparsify_a8(X_o)     Top-K 50% + INT8 (Eq. 1)
+  gemm  O              [M x 4096] x [4096 x 4096]^T
+  quant_a4(X_ffn)
+  gemm  Up|Gate        [M x 4096] x [22016 x 4096]^T, one alpha per tensor
+  relu2_glu            up * relu(gate)^2 (Eq. 5) + Top-K 50% + INT8
+  gemm  Down           [M x 11008] x [4096 x 11008]^T
+
+Attention itself is outside the path; its output (the O-projection input) is a
+seeded heavy-tailed tensor.  Inputs are seeded synthetic data larger than L2.
+With --gpus N (torchrun) every rank runs an independent replica on its own
+tokens (weak scaling, no data-path collective); the time is the max over ranks.
+
+--impl reference times the CPU oracle on the host (rank 0 only) on a bounded
+token sample of the same workload, scaled to tokens/s.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "BitLinear GEMM TOPS & tokens/s (7B layer shapes) vs B200 INT8/FP4 peak; quant GB/s"
+SHAPE = synth.L7B
+EPS = 1e-5
+# measured B200 peaks of this machine (generated file), else the documented fallback
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+INT8_PER_BF16 = 2.0   # nominal dense int8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def workload_config(afmt: str, m: int):
+    s = SHAPE
+    return {
+        "workload": f"BitNet a4.8 7B-shape decoder layer, BitLinear forward, prefill 8x4096 tokens",
+        "hidden": s.hidden, "heads": s.heads, "head_dim": s.head_dim, "ffn": s.ffn, "tokens_per_gpu": m,
+        "activations": ("INT4 absmean" if afmt == "int4" else "FP4 E2M1 MinMax") +
+                       " for QKV/Up/Gate inputs; Top-K 50% + INT8 for O and Down inputs",
+        "weights": "ternary, re-quantized from fp32 latent weights every step",
+        "kv_cache": "3-bit, BOS position at 4 bits",
+        "l2": "inputs larger than L2 (each activation tensor 268 MB)",
+    }
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str | None):
+        self.bus_id = bus_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.bus_id:
+            cmd.insert(1, f"--id={self.bus_id}")
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.reader.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# multi-rank timing: every rank runs its own replica; the job's time is the
+# slowest rank's, and the job's throughput counts every rank's tokens
+# ---------------------------------------------------------------------------
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings (a collective used for timing only)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def weak_scaling_throughput(world: int, tokens_per_rank: int, steps: int, elapsed_ms: float) -> float:
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (elapsed_ms / 1e3)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+class Layer:
+    """Device buffers and the launch sequence of one layer step."""
+
+    def __init__(self, torch, tba, dev, m: int, afmt: str, seed: int):
+        self.torch, self.tba, self.dev = torch, tba, dev
+        s = SHAPE
+        d, f, H, Dh = s.hidden, s.ffn, s.heads, s.head_dim
+        self.m, self.d, self.f, self.H, self.Dh = m, d, f, H, Dh
+        self.afmt = afmt
+        T = torch
+        u8, i8, f32, i16, i32 = T.uint8, T.int8, T.float32, T.int16, T.int32
+
+        def dev_from(a):
+            a = np.ascontiguousarray(a)
+            if a.dtype == np.uint16:
+                a = a.view(np.int16)
+            return T.from_numpy(a).to(dev)
+
+        # latent weights (fp32, resident) and their ternary int8 operands
+        wts = synth.layer_weights(SHAPE, seed=3)
+        self.w_lat = {k: dev_from(v) for k, v in wts.items()}
+        del wts
+        self.w8 = {"qkv": T.empty((3 * d, d), dtype=u8, device=dev), "o": T.empty((d, d), dtype=u8, device=dev),
+                   "upgate": T.empty((2 * f, d), dtype=u8, device=dev), "down": T.empty((d, f), dtype=u8, device=dev)}
+        self.alpha = T.zeros((8,), dtype=f32, device=dev)   # qkv, o, up, gate, down
+        self.ws = T.empty((tba.workspace_size("pack_ternary") // 8,), dtype=T.int64, device=dev)
+
+        # activations: host copies (pinned, for the end-to-end leg) and device copies
+        x_attn, x_o, x_ffn = synth.layer_activations(SHAPE, seed=seed, tokens=m)
+        self.h_in = [T.from_numpy(a.view(np.int16)).pin_memory() for a in (x_attn, x_o, x_ffn)]
+        del x_attn, x_o, x_ffn
+        self.x = [h.to(dev) for h in self.h_in]
+
+        qbytes = 1  # BL_STORE_BYTES: one int8 per element for the tensor-core operand
+        self.qa = T.empty((m, d * qbytes), dtype=u8, device=dev)
+        self.qa_s = T.empty((m,), dtype=f32, device=dev)
+        self.qf = T.empty((m, d * qbytes), dtype=u8, device=dev)
+        self.qf_s = T.empty((m,), dtype=f32, device=dev)
+        self.o8 = T.empty((m, d), dtype=i8, device=dev)
+        self.o8_s = T.empty((m,), dtype=f32, device=dev)
+        self.h8 = T.empty((m, f), dtype=i8, device=dev)
+        self.h8_s = T.empty((m,), dtype=f32, device=dev)
+        self.y_qkv = T.empty((m, 3 * d), dtype=i16, device=dev)
+        self.y_o = T.empty((m, d), dtype=i16, device=dev)
+        self.y_ug = T.empty((m, 2 * f), dtype=i16, device=dev)
+        self.y_down = T.empty((m, d), dtype=i16, device=dev)
+        self.kv_codes = T.empty((2, m, H, Dh * 3 // 8), dtype=u8, device=dev)
+        self.kv_scale = T.empty((2, m, H), dtype=f32, device=dev)
+        self.kv_bos = T.empty((2, H, Dh // 2), dtype=u8, device=dev)
+        self.outputs = [self.y_o, self.y_down, self.kv_codes, self.kv_scale, self.kv_bos]
+        self.h_out = [T.empty(o.shape, dtype=o.dtype).pin_memory() for o in self.outputs]
+
+        # algorithmic work per step
+        N_K = {"qkv": (3 * d, d), "o": (d, d), "upgate": (2 * f, d), "down": (d, f)}
+        self.gemm_ops = {k: 2.0 * m * n * kk for k, (n, kk) in N_K.items()}
+        self.weights = sum(n * kk for n, kk in N_K.values())
+        self.launches_per_step = 5 * 3 + 2 + 4 + 2 + 1 + 1
+
+    # kernel-by-kernel bytes each launch must move (algorithmic, per the formulas
+    # of the path: read inputs once, write outputs once)
+    def kernel_bytes(self):
+        m, d, f, H, Dh = self.m, self.d, self.f, self.H, self.Dh
+        kv_one = m * H * (2 * Dh + Dh * 3 // 8 + 4)
+        return {
+            "quant_a4": 2 * (m * d * 2 + m * d + 4 * m),
+            "sparsify_a8": m * d * 2 + m * d + 4 * m,
+            "relu2_glu": m * f * 4 + m * f + 4 * m,
+            "kv_quant3": 2 * kv_one,
+            "pack_ternary": sum(n * kk * 5 for n, kk in [(3 * d, d), (d, d), (2 * f, d), (d, f)]),
+        }
+
+    def step(self, ev=None):
+        """Enqueue one step on the current stream; ev (optional) collects
+        (name, start_event, end_event) around every library call."""
+        tba, T = self.tba, self.torch
+        d, f, m, H, Dh = self.d, self.f, self.m, self.H, self.Dh
+        fp4 = self.afmt == "fp4"
+
+        def timed(name, fn):
+            if ev is None:
+                fn()
+                return
+            a = T.cuda.Event(enable_timing=True)
+            b = T.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            ev.append((name, a, b))
+
+        W, w8, al = self.w_lat, self.w8, self.alpha
+        ws = self.ws
+        timed("pack_ternary", lambda: tba.pack_ternary(W["qkv"], al[0:1], w8["qkv"], tba.BL_W_I8, ws, eps=EPS))
+        timed("pack_ternary", lambda: tba.pack_ternary(W["o"], al[1:2], w8["o"], tba.BL_W_I8, ws, eps=EPS))
+        timed("pack_ternary", lambda: tba.pack_ternary(W["up"], al[2:3], w8["upgate"][:f], tba.BL_W_I8, ws, eps=EPS))
+        timed("pack_ternary", lambda: tba.pack_ternary(W["gate"], al[3:4], w8["upgate"][f:], tba.BL_W_I8, ws,
+                                                       eps=EPS))
+        timed("pack_ternary", lambda: tba.pack_ternary(W["down"], al[4:5], w8["down"], tba.BL_W_I8, ws, eps=EPS))
+        q = tba.BL_QUANT_FP4_E2M1 if fp4 else tba.BL_QUANT_INT4
+        x_attn, x_o, x_ffn = self.x
+        # attention block
+        timed("quant_a4", lambda: tba.bitlinear_quant_a4(x_attn, self.qa, self.qa_s, q, tba.BL_STORE_BYTES, EPS))
+        timed("gemm_qkv", lambda: tba.bitlinear_gemm(self.qa, self.qa_s, w8["qkv"], al[0:1], m, 3 * d, d,
+                                                     y=self.y_qkv))
+        for i, off in enumerate((d, 2 * d)):     # K and V slices of the QKV output
+            timed("kv_quant3", lambda off=off, i=i: tba.kv_quant3(self.y_qkv[:, off:], m, H, Dh, self.kv_codes[i],
+                                                                  self.kv_scale[i], self.kv_bos[i], bits=3,
+                                                                  bos_pos=0, eps=EPS, ldt=3 * d))
+        timed("sparsify_a8", lambda: tba.bitlinear_sparsify_a8(x_o, synth.k_keep(d, SHAPE.topk_pct_o), self.o8,
+                                                               self.o8_s, None, EPS))
+        timed("gemm_o", lambda: tba.bitlinear_gemm(self.o8, self.o8_s, w8["o"], al[1:2], m, d, d, y=self.y_o))
+        # FFN block
+        timed("quant_a4", lambda: tba.bitlinear_quant_a4(x_ffn, self.qf, self.qf_s, q, tba.BL_STORE_BYTES, EPS))
+        timed("gemm_upgate", lambda: tba.bitlinear_gemm(self.qf, self.qf_s, w8["upgate"], al[2:4], m, 2 * f, d,
+                                                        y=self.y_ug, alpha_group=f))
+        timed("relu2_glu", lambda: tba.relu2_glu(self.y_ug[:, f:], self.y_ug[:, :f],
+                                                 synth.k_keep(f, SHAPE.topk_pct_down), self.h8, self.h8_s, None,
+                                                 EPS, M=m, F=f, ld=2 * f))
+        timed("gemm_down", lambda: tba.bitlinear_gemm(self.h8, self.h8_s, w8["down"], al[4:5], m, d, f,
+                                                      y=self.y_down))
+
+    def h2d(self):
+        for h, dv in zip(self.h_in, self.x):
+            dv.copy_(h, non_blocking=True)
+
+    def d2h(self):
+        for o, h in zip(self.outputs, self.h_out):
+            h.copy_(o, non_blocking=True)
+
+    def io_bytes(self):
+        return (sum(h.numel() * h.element_size() for h in self.h_in),
+                sum(h.numel() * h.element_size() for h in self.h_out))
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import ternary_bit_activation_b200 as tba
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    distributed = world > 1
+    if distributed:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    tba.lib()
+    m = SHAPE.tokens
+    layer = Layer(torch, tba, dev, m, args.afmt, seed=SHAPE.tokens + 17 * rank)
+    tba.sync_status()
+
+    def barrier():
+        if distributed:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        layer.step()
+    tba.sync_status()
+
+    props = torch.cuda.get_device_properties(dev)
+    bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    clocks = ClockSampler(bus)
+    clocks.start()
+    time.sleep(0.3)
+    events = []
+    barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        layer.step(events)
+    t1.record()
+    barrier()
+    clk = clocks.stop()
+    tba.sync_status()
+    elapsed_ms = t0.elapsed_time(t1)
+    per_kernel = {}
+    for name, a, b in events:
+        per_kernel.setdefault(name, []).append(a.elapsed_time(b))
+
+    # end to end through the C ABI with host buffers: H2D of the step's inputs,
+    # the step, D2H of its outputs -- every step
+    for _ in range(max(1, args.warmup // 2)):
+        layer.h2d(); layer.step(); layer.d2h()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        layer.h2d()
+        layer.step()
+        layer.d2h()
+    e1.record()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+
+    if distributed:
+        elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], dev)
+
+    if rank == 0:
+        peaks = load_peaks()
+        ms_step = elapsed_ms / args.steps
+        value = weak_scaling_throughput(world, m, args.steps, elapsed_ms)
+        gemm_names = [k for k in per_kernel if k.startswith("gemm_")]
+        gemm_ms = sum(sum(per_kernel[k]) for k in gemm_names)
+        gemm_ops = sum(layer.gemm_ops[k[5:]] for k in gemm_names) * args.steps
+        tops = gemm_ops / (gemm_ms / 1e3) / 1e12
+        peak_int8 = peaks["bf16_tflops_sustained"] * INT8_PER_BF16
+        kb = layer.kernel_bytes()
+        kernels = {}
+        for k, v in per_kernel.items():
+            per_step = sum(v) / args.steps
+            entry = {"ms_per_step": round(per_step, 4), "launches_per_step": len(v) // args.steps}
+            if k.startswith("gemm_"):
+                entry["tops_dense"] = round(layer.gemm_ops[k[5:]] / (per_step / 1e3) / 1e12, 1)
+            elif k in kb:
+                entry["gbs"] = round(kb[k] / (per_step / 1e3) / 1e9, 1)
+                entry["hbm_frac"] = round(entry["gbs"] / peaks["hbm_gbs"], 3)
+            kernels[k] = entry
+        # algorithmic TOPS: the Top-K-50% inputs (O, Down) carry half the nonzeros
+        alg_ops = (layer.gemm_ops["qkv"] + layer.gemm_ops["upgate"] +
+                   0.5 * (layer.gemm_ops["o"] + layer.gemm_ops["down"])) * args.steps
+        h2d, d2h = layer.io_bytes()
+        line = {
+            "metric": METRIC,
+            "value": round(value, 1),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "int8",
+            "data": "synthetic (seeded; Gaussian QKV/FFN inputs, Student-t nu=3 O input, N(0,0.02) latent weights)",
+            "config": dict(workload_config(args.afmt, m), parallelism=f"replicas x{world}"),
+            "roofline": {
+                "bound": "tensor",
+                "kernel": "gemm_tc_kernel (tcgen05 kind::i8)",
+                "achieved": round(tops, 1),
+                "peak": round(peak_int8, 1),
+                "unit": "TFLOP/s",
+                "frac": round(tops / peak_int8, 4),
+                "traffic": None,
+                "peak_note": f"int8 = 2 x {peaks['source']} sustained bf16 cuBLAS ({peaks['bf16_tflops_sustained']})",
+                "work": "dense-equivalent 2*M*N*K over the 4 GEMM launches of a step / their summed event time",
+            },
+            "gemm": {"tops_dense": round(tops, 1), "tops_algorithmic": round(alg_ops / (gemm_ms / 1e3) / 1e12, 1),
+                     "ms_per_step": round(gemm_ms / args.steps, 4)},
+            "kernels": kernels,
+            "e2e": {"value": round(world * m * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms / args.steps, 4)},
+            "gpu_launches": layer.launches_per_step * args.steps,
+            "clocks": clk,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(args.afmt, tokens_sample=args.cpu_tokens)
+        print(json.dumps(line), flush=True)
+    if distributed:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle arm
+# ---------------------------------------------------------------------------
+def oracle_sample_seconds(afmt: str, tokens: int, pack: bool = True):
+    """Time the CPU oracle over the same step on `tokens` rows: per-token work
+    (quantizers, the four products, ReLU^2-GLU, KV) plus, if `pack`, the
+    once-per-step ternary quantization of all latent weights."""
+    import oracle
+    s = SHAPE
+    d, f = s.hidden, s.ffn
+    wts = synth.layer_weights(s, seed=3)
+    x_attn, x_o, x_ffn = synth.layer_activations(s, seed=99, tokens=tokens)
+    t_pack = 0.0
+    t0 = time.perf_counter()
+    tq = {}
+    al = {}
+    for k, w in wts.items():
+        tq[k], al[k] = oracle.ternary_quantize(w, EPS)
+    t_pack = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    if afmt == "fp4":
+        _, qa, _, s_a = oracle.quant_fp4(x_attn)
+        s_a = (s_a / 2).astype(np.float32)
+    else:
+        qa, _, s_a = oracle.quant_int4(x_attn, EPS)
+    _, y_qkv = oracle.gemm(qa, s_a, tq["qkv"], al["qkv"])
+    kvin = np.ascontiguousarray(y_qkv[:, d:].reshape(tokens, 2, s.heads, s.head_dim).transpose(1, 0, 2, 3))
+    for i in range(2):
+        oracle.kv_quant(kvin[i], bits=3, bos_pos=0, eps=EPS)
+    c8, _, _, s8 = oracle.sparsify_a8(x_o, synth.k_keep(d, s.topk_pct_o), EPS)
+    oracle.gemm(c8, s8, tq["o"], al["o"])
+    if afmt == "fp4":
+        _, qf, _, s_f = oracle.quant_fp4(x_ffn)
+        s_f = (s_f / 2).astype(np.float32)
+    else:
+        qf, _, s_f = oracle.quant_int4(x_ffn, EPS)
+    _, y_up = oracle.gemm(qf, s_f, tq["up"], al["up"])
+    _, y_gate = oracle.gemm(qf, s_f, tq["gate"], al["gate"])
+    h8, _, _, sh = oracle.relu2_glu(y_gate, y_up, synth.k_keep(f, s.topk_pct_down), EPS)
+    oracle.gemm(h8, sh, tq["down"], al["down"])
+    t_tok = time.perf_counter() - t0
+    return t_pack, t_tok
+
+
+def cpu_baseline(afmt: str, tokens_sample: int):
+    t_pack, t_tok = oracle_sample_seconds(afmt, tokens_sample)
+    m = SHAPE.tokens
+    step_s = t_pack + t_tok * (m / tokens_sample)
+    return {"value": round(m / step_s, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{tokens_sample} tokens of the 7B-shape layer through every step of the path, plus the "
+                      f"once-per-step ternary quantization of all 202M latent weights; per-token time scaled "
+                      f"linearly to {m} tokens (pack {t_pack:.2f} s, sample {t_tok:.2f} s, single-threaded C)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    m = SHAPE.tokens
+    for _ in range(args.warmup):
+        oracle_sample_seconds(args.afmt, args.cpu_tokens_ref, pack=True)
+    total = 0.0
+    for _ in range(args.steps):
+        t_pack, t_tok = oracle_sample_seconds(args.afmt, args.cpu_tokens_ref, pack=True)
+        total += t_pack + t_tok * (m / args.cpu_tokens_ref)
+    value = args.steps * m / total
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded)",
+        "config": dict(workload_config(args.afmt, m), parallelism="host CPU, rank 0 only"),
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: {args.cpu_tokens_ref} tokens of the 7B-shape layer through the "
+                                   f"whole path plus the ternary quantization of all latent weights, per-token time "
+                                   f"scaled to {m} tokens; single-threaded C oracle"},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--afmt", choices=["int4", "fp4"], default="int4")
+    ap.add_argument("--cpu-tokens", type=int, default=32, help="token sample of the CPU baseline")
+    ap.add_argument("--cpu-tokens-ref", type=int, default=8, help="token sample per step of --impl reference")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

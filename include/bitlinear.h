@@ -1,0 +1,216 @@
+/*
+ * bitlinear.h -- C ABI of libbitlinear, the sm_100a (B200) implementation of the
+ * BitLinear forward path of BitNet a4.8 ("BitNet a4.8: 4-bit Activations for
+ * 1-bit LLMs", arXiv 2411.04965).
+ *
+ * Conventions for every entry point
+ *   - All tensor arguments are DEVICE pointers owned by the caller.  The library
+ *     allocates no device memory, keeps no per-call state and never frees
+ *     caller memory.  Work is enqueued on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and is asynchronous: outputs are valid once the
+ *     stream has reached that point.
+ *   - bf16 tensors are IEEE bfloat16, row-major.  "ld" arguments are row
+ *     strides in elements.  Pointers must be 16-byte aligned and row strides
+ *     must keep every row 16-byte aligned (noted per call).
+ *   - Arguments are validated on the host before anything is launched; a bad
+ *     argument returns a status without touching the GPU.  A launch failure
+ *     returns BL_ERR_CUDA.  Kernels bound every wait; a wait that runs out sets
+ *     a device status word instead of hanging, and bitlinear_sync_status()
+ *     reports it (BL_ERR_TIMEOUT).  No C++ exception crosses this boundary.
+ *   - Quantizers work per token (one row of X).  NaN/Inf inputs are outside the
+ *     contract (results unspecified).
+ *   - eps is the paper's "small constant" (1e-5 in the tests).
+ */
+#ifndef BITLINEAR_H_
+#define BITLINEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BL_API __attribute__((visibility("default")))
+#else
+#define BL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BL_OK = 0,
+    BL_ERR_NULL = 1,          /* a required pointer is NULL */
+    BL_ERR_ALIGN = 2,         /* a pointer or row stride breaks the 16-byte rule */
+    BL_ERR_SHAPE = 3,         /* a size is out of range for this call */
+    BL_ERR_ARG = 4,           /* an enum or scalar argument is invalid */
+    BL_ERR_UNSUPPORTED = 5,   /* valid, but this build has no kernel for it */
+    BL_ERR_CUDA = 6,          /* the CUDA runtime reported an error */
+    BL_ERR_TIMEOUT = 7,       /* a kernel gave up on a bounded wait */
+    BL_ERR_WORKSPACE = 8      /* workspace too small */
+} bl_status;
+
+/* Quantizer choice for the 4-bit activation path. */
+typedef enum {
+    BL_QUANT_INT4 = 0,        /* absmean INT4, Eq. 6-7 */
+    BL_QUANT_FP4_E2M1 = 1     /* MinMax FP4 E2M1, Eq. 8-9 */
+} bl_quant;
+
+/* How 4-bit codes are stored. */
+typedef enum {
+    BL_STORE_PACKED = 0,      /* two codes per byte: element 2i in bits 0-3, 2i+1 in bits 4-7 */
+    BL_STORE_BYTES = 1        /* one signed byte per element (tensor-core operand layout) */
+} bl_store;
+
+/* Activation operand formats accepted by bitlinear_gemm. */
+typedef enum {
+    BL_A_I8 = 0,              /* int8 per element: INT8 codes, INT4 codes in bytes, or FP4 as 2*value */
+    BL_A_I4 = 1,              /* packed two's-complement INT4 nibbles (BL_STORE_PACKED of INT4) */
+    BL_A_E2M1 = 2             /* packed E2M1 nibbles (BL_STORE_PACKED of FP4) */
+} bl_afmt;
+
+/* Ternary weight formats (both K-major: row n holds the K codes of output n). */
+typedef enum {
+    BL_W_T2 = 0,              /* 2-bit codes, 4 per byte, element 4i in bits 0-1: 0->00, +1->01, -1->11 */
+    BL_W_I8 = 1               /* one int8 in {-1,0,1} per element (tensor-core operand layout) */
+} bl_wfmt;
+
+/*
+ * bitlinear_quant_a4 -- 4-bit activation quantizer for the Gaussian-like inputs
+ * (attention QKV and FFN Up/Gate inputs).
+ * Paper: §3.4 "4-Bit Activation Quantization for Gaussian-Like Inputs".
+ *   BL_QUANT_INT4 (Eq. 6-7): beta = mean|x| over the row (summed exactly in
+ *     fp64 -- the contract covers rows whose |x| sum is exact in fp64, true for
+ *     ordinary data), mult = fp32(sqrt7) / (beta + eps) in fp32,
+ *     code = RoundClip(x * mult, -8, 7) with round-half-even.
+ *     scale[m] = beta / fp32(sqrt7) (the dequant factor).
+ *   BL_QUANT_FP4_E2M1 (Eq. 8-9, garbled on the page; reading used): p = the
+ *     smallest integer with max|x| <= 6 * 2^p (p = 0 for a zero row); each
+ *     x * 2^-p is rounded to the nearest E2M1 value {0,.5,1,1.5,2,3,4,6}, ties
+ *     to the even encoding; codes are sign bit 3 + value bits 0-2, a zero
+ *     magnitude is always +0.  scale[m] = 2^p.
+ * Storage: BL_STORE_PACKED writes M x K/2 bytes; BL_STORE_BYTES writes M x K
+ *   int8 (INT4: the code itself; FP4: 2 * value, an exact integer in [-12, 12],
+ *   with scale[m] = 2^(p-1) so that value * 2^p = byte * scale).
+ * x: [M x K] bf16 with row stride ldx.  codes: contiguous rows.  scale: [M] fp32.
+ * Requires K % 8 == 0, 8 <= K <= 16384, ldx % 8 == 0, 16-byte aligned pointers.
+ */
+BL_API bl_status bitlinear_quant_a4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                             bl_quant quant, bl_store store, float eps,
+                             void* codes, float* scale, void* stream);
+
+/*
+ * bitlinear_sparsify_a8 -- Top-K sparsification then INT8 absmax quantization
+ * for the outlier-heavy inputs (attention-output and FFN-down inputs).
+ * Paper: §3.4 "Sparsification Pipeline for Outlier-Heavy Intermediate States",
+ * Eq. 1 with Q_INT8:  codes = RoundClip(127/(gamma+eps) * x, -128, 127) * M,
+ * gamma = max|x| over the row, M = Top_k(|x|).
+ * Top-K reading: exactly k_keep survivors per row, ranked by |x| (the bf16
+ * magnitude) descending; equal magnitudes are taken in increasing index order.
+ * x: [M x K] bf16, row stride ldx.  codes: [M x K] int8 (0 where masked).
+ * scale: [M] fp32 = gamma / 127.  mask (nullable): [M x ceil(K/32)] uint32,
+ * bit j of word w is element 32w + j; bits past K are 0.
+ * Requires 1 <= k_keep <= K, K % 8 == 0, K <= 16384, ldx % 8 == 0.
+ */
+BL_API bl_status bitlinear_sparsify_a8(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                                int64_t k_keep, float eps, int8_t* codes, float* scale,
+                                uint32_t* mask, void* stream);
+
+/*
+ * pack_ternary -- absmean ternary weight quantizer and packer.
+ * Paper: §3.4 "Ternary Weight Quantization (BitLinear)", Eq. 2:
+ *   alpha = mean|W| over the whole tensor, t = RoundClip(W / (alpha + eps), -1, 1).
+ * alpha is the exact mean rounded once to fp32 (round-half-even): |w| values are
+ * summed exactly in integer bins per fp32 exponent, then divided and rounded
+ * with multi-word integer arithmetic on the device.  The division W/(alpha+eps)
+ * is an IEEE fp32 division.
+ * w: [N x K] fp32, row stride ldw.  alpha: one device float; read as the
+ * input when alpha_given != 0, written otherwise.  w_out: BL_W_T2 -> N x K/4
+ * bytes, BL_W_I8 -> N x K bytes (layouts in bl_wfmt).
+ * workspace: device scratch of bitlinear_workspace_size("pack_ternary", N, K, 0)
+ * bytes (2 KiB; cleared by the call itself).  Not needed when alpha_given != 0.
+ * Requires K % 16 == 0, ldw % 4 == 0, N * K < 2^40.
+ */
+BL_API bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float eps,
+                       int alpha_given, float* alpha, bl_wfmt wfmt, void* w_out,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * bitlinear_gemm -- BitLinear product with integer accumulation and the
+ * per-token x per-tensor dequant epilogue.
+ * Paper: §3.4, Y = Q_x(X) . Q_w(W)^T (the equation above Eq. 6, and Eq. 1).
+ *   acc[m,n] = sum_k a[m,k] * t[n,k]          exact int32
+ *   y[m,n]   = bf16( acc[m,n] * a_scale[m] * alpha[n / alpha_group] )
+ * For BL_A_E2M1 the codes' values are summed (exact: multiples of 0.5), and
+ * acc_out holds 2 * the sum.
+ * a: [M x K] in `afmt` (contiguous rows), a_scale: [M] fp32 (the scale the
+ * quantizer wrote), w: [N x K] in `wfmt` (pack_ternary's output), alpha: fp32
+ * array with one entry per group of alpha_group consecutive outputs
+ * (alpha_group = N for one tensor; e.g. F for stacked Up|Gate weights).
+ * y: [M x N] bf16 with row stride ldy (nullable).  acc_out: [M x N] int32,
+ * row stride N (nullable; a test aid).
+ * Kernels: BL_A_I8 x BL_W_I8 runs on the tcgen05 tensor cores (kind::i8,
+ * TMA-fed, TMEM accumulators); other operand formats run on a CUDA-core kernel
+ * that reads packed operands directly (the decode path).
+ * Requires K % 64 == 0, ldy % 8 == 0, 1 <= alpha_group.
+ */
+BL_API bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale,
+                         const void* w, bl_wfmt wfmt, const float* alpha, int64_t alpha_group,
+                         int64_t M, int64_t N, int64_t K,
+                         void* y_bf16, int64_t ldy, int32_t* acc_out, void* stream);
+
+/*
+ * relu2_glu -- squared-ReLU GLU fused with the down projection's
+ * sparsify-then-quantize step.
+ * Paper: §3.4 "Squared ReLU Gating and Conditional Computation in the FFN",
+ * Eq. 5:  h = up (.) max(0, gate)^2, computed in fp32 as g2 = g*g, h = up*g2;
+ * then Eq. 1 on h: gamma = max|h|, Top-K over |h| (fp32 magnitude, ties to
+ * the lower index), codes = RoundClip(127/(gamma+eps) * h, -128, 127) * M.
+ * k_keep = F keeps every entry (INT8 only).
+ * gate, up: [M x F] bf16 with the shared row stride ld (e.g. the two halves of
+ * a stacked Up|Gate output).  codes: [M x F] int8.  scale: [M] fp32 =
+ * gamma / 127.  mask (nullable): [M x ceil(F/32)] uint32 as in sparsify_a8.
+ * Requires 1 <= k_keep <= F, F % 8 == 0, F <= 16384, ld % 8 == 0.
+ */
+BL_API bl_status relu2_glu(const void* gate_bf16, const void* up_bf16, int64_t M, int64_t F, int64_t ld,
+                    int64_t k_keep, float eps, int8_t* codes, float* scale, uint32_t* mask,
+                    void* stream);
+
+/*
+ * kv_quant3 -- post-RoPE low-bit KV-cache quantizer.
+ * Paper: §3.4 "Low-Bit KV Cache Quantization" (absmax to unsigned integers;
+ * for 3-bit caches the beginning-of-sequence heads stay at 4 bits).
+ * Reading: per (position t, head h) vector of D values, gamma = max|x|,
+ * Q = 2^(b-1) - 1, c = RoundClip(Q/(gamma+eps) * x, -Q-1, Q), stored unsigned
+ * as c + 2^(b-1); scale = gamma / Q.
+ * kv: [T x H x D] bf16, stride ldt elements between positions (ldt >= H*D).
+ * codes: [T x H x D*bits/8] bytes.  bits = 3: eight codes per 3 bytes, code j
+ * of a group in bits 3j..3j+2 of a little-endian 24-bit word.  bits = 4: the
+ * nibble layout of BL_STORE_PACKED.  scale: [T x H] fp32.
+ * When bits == 3 and 0 <= bos_pos < T, position bos_pos is quantized at 4 bits
+ * into bos_codes ([H x D/2] bytes, nibble layout), its scale is gamma/7, and
+ * its 3-bit slot in `codes` is zero-filled.  bos_pos = -1: no BOS row.
+ * Requires D % 32 == 0, 32 <= D <= 256, ldt % 8 == 0.
+ */
+BL_API bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D, int64_t ldt, int bits,
+                    int64_t bos_pos, float eps, uint8_t* codes, float* scale, uint8_t* bos_codes,
+                    void* stream);
+
+/* Bytes of device workspace an operation needs ("pack_ternary"; 0 for the others). */
+BL_API size_t bitlinear_workspace_size(const char* op, int64_t M, int64_t N, int64_t K);
+
+/* Synchronizes `stream`, then reads and clears the calling device's status
+ * word.  Returns BL_ERR_TIMEOUT if a kernel gave up on a bounded wait since the
+ * last call, BL_ERR_CUDA on a runtime error, BL_OK otherwise. */
+BL_API bl_status bitlinear_sync_status(void* stream);
+
+/* Human-readable name of a status code (static storage). */
+BL_API const char* bitlinear_status_string(bl_status status);
+
+/* Library version string (static storage). */
+BL_API const char* bitlinear_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H_ */

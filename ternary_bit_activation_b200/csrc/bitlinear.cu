@@ -1,0 +1,394 @@
+// libbitlinear: C ABI over the sm_100a kernels of the BitNet a4.8 BitLinear
+// forward path (arXiv 2411.04965, §3.4).  One translation unit: the kernels
+// live in the headers included below; this file validates arguments, encodes
+// TMA descriptors and launches.  The declarations and their contracts are in
+// include/bitlinear.h.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "bitlinear.h"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "kv.cuh"
+#include "pack.cuh"
+#include "quant.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bl_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) return -1;
+  return d;
+}
+
+int sm_count() {
+  static int cached[kMaxDevices] = {0};
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return 148;
+  if (cached[d] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0) n = 148;
+    cached[d] = n;
+  }
+  return cached[d];
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors through the driver entry point (no link-time libcuda).
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D int8 tensor [rows x cols] (cols contiguous), box of box_cols x box_rows, 128B swizzle.
+bool make_i8_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                 uint32_t box_cols) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool tc_kernel_ready() {
+  static bool done[kMaxDevices] = {false};
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return false;
+  if (!done[d]) {
+    if (cudaFuncSetAttribute(bl::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bl::kTcSmemBytes)) != cudaSuccess)
+      return false;
+    done[d] = true;
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// launch helpers
+// ---------------------------------------------------------------------------
+template <int C>
+void launch_quant_a4_c(const uint16_t* x, int64_t M, int K, int64_t ldx, bool fp4, bool packed, float eps,
+                       uint8_t* codes, float* scale, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>((M + 1) / 2));
+  if (!fp4 && packed) bl::quant_a4_kernel<C, false, true><<<grid, 256, 0, s>>>(x, M, K, ldx, eps, codes, scale);
+  if (!fp4 && !packed) bl::quant_a4_kernel<C, false, false><<<grid, 256, 0, s>>>(x, M, K, ldx, eps, codes, scale);
+  if (fp4 && packed) bl::quant_a4_kernel<C, true, true><<<grid, 256, 0, s>>>(x, M, K, ldx, eps, codes, scale);
+  if (fp4 && !packed) bl::quant_a4_kernel<C, true, false><<<grid, 256, 0, s>>>(x, M, K, ldx, eps, codes, scale);
+}
+
+template <int C>
+void launch_sparsify_c(const uint16_t* x, int64_t M, int K, int64_t ldx, int keep, float eps, int8_t* codes,
+                       float* scale, uint32_t* mask, cudaStream_t s) {
+  bl::sparsify_a8_kernel<C><<<static_cast<unsigned>(M), bl::kTkThreads, 0, s>>>(x, K, ldx, keep, eps, codes, scale,
+                                                                                  mask);
+}
+
+template <int C>
+void launch_relu2_c(const uint16_t* g, const uint16_t* u, int64_t M, int F, int64_t ld, int keep, float eps,
+                    int8_t* codes, float* scale, uint32_t* mask, cudaStream_t s) {
+  bl::relu2_glu_kernel<C><<<static_cast<unsigned>(M), bl::kTkThreads, 0, s>>>(g, u, F, ld, keep, eps, codes, scale,
+                                                                                mask);
+}
+
+bool topk_chunks(int64_t K, int* chunks) {
+  const int64_t c = (K / 8 + bl::kTkThreads - 1) / bl::kTkThreads;
+  if (c < 1 || c > 8) return false;
+  *chunks = static_cast<int>(c);
+  return true;
+}
+
+template <int AF, bool WT2>
+void launch_simt(const uint8_t* a, const float* sc, const uint8_t* w, const float* al, int64_t g, int M, int N,
+                 int K, uint16_t* y, int64_t ldy, int32_t* acc, cudaStream_t s) {
+  const int64_t blocks_needed = (static_cast<int64_t>(N) + 7) / 8;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+  const unsigned grid = static_cast<unsigned>(blocks_needed < cap ? blocks_needed : cap);
+  if (M <= 1)
+    bl::gemm_simt_kernel<AF, WT2, 1><<<grid, 256, 0, s>>>(a, sc, w, al, g, M, N, K, y, ldy, acc);
+  else if (M <= 2)
+    bl::gemm_simt_kernel<AF, WT2, 2><<<grid, 256, 0, s>>>(a, sc, w, al, g, M, N, K, y, ldy, acc);
+  else if (M <= 4)
+    bl::gemm_simt_kernel<AF, WT2, 4><<<grid, 256, 0, s>>>(a, sc, w, al, g, M, N, K, y, ldy, acc);
+  else
+    bl::gemm_simt_kernel<AF, WT2, 8><<<grid, 256, 0, s>>>(a, sc, w, al, g, M, N, K, y, ldy, acc);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* bitlinear_version(void) { return "libbitlinear 0.1 (sm_100a)"; }
+
+const char* bitlinear_status_string(bl_status st) {
+  switch (st) {
+    case BL_OK: return "BL_OK";
+    case BL_ERR_NULL: return "BL_ERR_NULL";
+    case BL_ERR_ALIGN: return "BL_ERR_ALIGN";
+    case BL_ERR_SHAPE: return "BL_ERR_SHAPE";
+    case BL_ERR_ARG: return "BL_ERR_ARG";
+    case BL_ERR_UNSUPPORTED: return "BL_ERR_UNSUPPORTED";
+    case BL_ERR_CUDA: return "BL_ERR_CUDA";
+    case BL_ERR_TIMEOUT: return "BL_ERR_TIMEOUT";
+    case BL_ERR_WORKSPACE: return "BL_ERR_WORKSPACE";
+  }
+  return "BL_UNKNOWN";
+}
+
+size_t bitlinear_workspace_size(const char* op, int64_t M, int64_t N, int64_t K) {
+  (void)M; (void)N; (void)K;
+  if (op != nullptr && strcmp(op, "pack_ternary") == 0) return 256 * sizeof(unsigned long long);
+  return 0;
+}
+
+bl_status bitlinear_sync_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return BL_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, bl::g_status, sizeof(int)) != cudaSuccess) return BL_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(bl::g_status, &zero, sizeof(int)) != cudaSuccess) return BL_ERR_CUDA;
+    return static_cast<bl_status>(v);
+  }
+  return BL_OK;
+}
+
+bl_status bitlinear_quant_a4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, bl_quant quant, bl_store store,
+                             float eps, void* codes, float* scale, void* stream) {
+  if (quant != BL_QUANT_INT4 && quant != BL_QUANT_FP4_E2M1) return BL_ERR_ARG;
+  if (store != BL_STORE_PACKED && store != BL_STORE_BYTES) return BL_ERR_ARG;
+  if (M < 0 || K < 8 || K > 16384 || (K & 7) || ldx < K || (ldx & 7) || M > 0x7FFFFFFELL) return BL_ERR_SHAPE;
+  if (M == 0) return BL_OK;
+  if (x_bf16 == nullptr || codes == nullptr || scale == nullptr) return BL_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scale)) return BL_ERR_ALIGN;
+  if (!(eps >= 0.f)) return BL_ERR_ARG;
+  const int64_t c = (K / 8 + bl::kQ4ThreadsPerRow - 1) / bl::kQ4ThreadsPerRow;
+  const bool fp4 = quant == BL_QUANT_FP4_E2M1, packed = store == BL_STORE_PACKED;
+  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+  uint8_t* out = static_cast<uint8_t*>(codes);
+  cudaStream_t s = as_stream(stream);
+  const int k = static_cast<int>(K);
+  if (c <= 1) launch_quant_a4_c<1>(x, M, k, ldx, fp4, packed, eps, out, scale, s);
+  else if (c <= 2) launch_quant_a4_c<2>(x, M, k, ldx, fp4, packed, eps, out, scale, s);
+  else if (c <= 4) launch_quant_a4_c<4>(x, M, k, ldx, fp4, packed, eps, out, scale, s);
+  else if (c <= 8) launch_quant_a4_c<8>(x, M, k, ldx, fp4, packed, eps, out, scale, s);
+  else launch_quant_a4_c<16>(x, M, k, ldx, fp4, packed, eps, out, scale, s);
+  return launch_status();
+}
+
+bl_status bitlinear_sparsify_a8(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, int64_t k_keep, float eps,
+                                int8_t* codes, float* scale, uint32_t* mask, void* stream) {
+  if (M < 0 || K < 8 || K > 16384 || (K & 7) || ldx < K || (ldx & 7) || M > 0x7FFFFFFFLL) return BL_ERR_SHAPE;
+  if (k_keep < 1 || k_keep > K) return BL_ERR_ARG;
+  if (!(eps >= 0.f)) return BL_ERR_ARG;
+  if (M == 0) return BL_OK;
+  if (x_bf16 == nullptr || codes == nullptr || scale == nullptr) return BL_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scale) || (mask && !aligned16(mask))) return BL_ERR_ALIGN;
+  int c = 0;
+  if (!topk_chunks(K, &c)) return BL_ERR_SHAPE;
+  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
+  const int k = static_cast<int>(K), kk = static_cast<int>(k_keep);
+  cudaStream_t s = as_stream(stream);
+  switch (c) {
+    case 1: launch_sparsify_c<1>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
+    case 2: launch_sparsify_c<2>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
+    case 3: launch_sparsify_c<3>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
+    case 4: launch_sparsify_c<4>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
+    case 5: launch_sparsify_c<5>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
+    case 6: launch_sparsify_c<6>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
+    case 7: launch_sparsify_c<7>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
+    default: launch_sparsify_c<8>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
+  }
+  return launch_status();
+}
+
+bl_status relu2_glu(const void* gate_bf16, const void* up_bf16, int64_t M, int64_t F, int64_t ld, int64_t k_keep,
+                    float eps, int8_t* codes, float* scale, uint32_t* mask, void* stream) {
+  if (M < 0 || F < 8 || F > 16384 || (F & 7) || ld < F || (ld & 7) || M > 0x7FFFFFFFLL) return BL_ERR_SHAPE;
+  if (k_keep < 1 || k_keep > F) return BL_ERR_ARG;
+  if (!(eps >= 0.f)) return BL_ERR_ARG;
+  if (M == 0) return BL_OK;
+  if (gate_bf16 == nullptr || up_bf16 == nullptr || codes == nullptr || scale == nullptr) return BL_ERR_NULL;
+  if (!aligned16(gate_bf16) || !aligned16(up_bf16) || !aligned16(codes) || !aligned16(scale) ||
+      (mask && !aligned16(mask)))
+    return BL_ERR_ALIGN;
+  int c = 0;
+  if (!topk_chunks(F, &c)) return BL_ERR_SHAPE;
+  const uint16_t* g = static_cast<const uint16_t*>(gate_bf16);
+  const uint16_t* u = static_cast<const uint16_t*>(up_bf16);
+  const int f = static_cast<int>(F), kk = static_cast<int>(k_keep);
+  cudaStream_t s = as_stream(stream);
+  switch (c) {
+    case 1: launch_relu2_c<1>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
+    case 2: launch_relu2_c<2>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
+    case 3: launch_relu2_c<3>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
+    case 4: launch_relu2_c<4>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
+    case 5: launch_relu2_c<5>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
+    case 6: launch_relu2_c<6>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
+    case 7: launch_relu2_c<7>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
+    default: launch_relu2_c<8>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
+  }
+  return launch_status();
+}
+
+bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float eps, int alpha_given, float* alpha,
+                       bl_wfmt wfmt, void* w_out, void* workspace, size_t ws_bytes, void* stream) {
+  if (wfmt != BL_W_T2 && wfmt != BL_W_I8) return BL_ERR_ARG;
+  if (N < 0 || K < 16 || (K & 15) || ldw < K || (ldw & 3)) return BL_ERR_SHAPE;
+  if (N > 0 && (N * K >= (int64_t(1) << 40) || K > 0x7FFFFFFF)) return BL_ERR_SHAPE;
+  if (!(eps >= 0.f)) return BL_ERR_ARG;
+  if (N == 0) return BL_OK;
+  if (w == nullptr || alpha == nullptr || w_out == nullptr) return BL_ERR_NULL;
+  if (!aligned16(w) || !aligned16(w_out) || (reinterpret_cast<uintptr_t>(alpha) & 3u)) return BL_ERR_ALIGN;
+  cudaStream_t s = as_stream(stream);
+  const int k = static_cast<int>(K);
+  if (!alpha_given) {
+    if (workspace == nullptr) return BL_ERR_NULL;
+    if (ws_bytes < 256 * sizeof(unsigned long long)) return BL_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 7u) return BL_ERR_ALIGN;
+    unsigned long long* bins = static_cast<unsigned long long*>(workspace);
+    if (cudaMemsetAsync(bins, 0, 256 * sizeof(unsigned long long), s) != cudaSuccess) return BL_ERR_CUDA;
+    const int64_t total = N * (K / 4);
+    int64_t blocks = (total + bl::kBinThreads - 1) / bl::kBinThreads;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    if (blocks > cap) blocks = cap;
+    bl::ternary_bins_kernel<<<static_cast<unsigned>(blocks), bl::kBinThreads, 0, s>>>(w, N, k, ldw, bins);
+    if (launch_status() != BL_OK) return BL_ERR_CUDA;
+    bl::ternary_alpha_kernel<<<1, 32, 0, s>>>(bins, static_cast<unsigned long long>(N * K), alpha);
+    if (launch_status() != BL_OK) return BL_ERR_CUDA;
+  }
+  const int64_t total16 = N * (K / 16);
+  int64_t blocks = (total16 + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+  if (blocks > cap) blocks = cap;
+  uint8_t* out = static_cast<uint8_t*>(w_out);
+  if (wfmt == BL_W_T2)
+    bl::ternary_pack_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+  else
+    bl::ternary_pack_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+  return launch_status();
+}
+
+bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, const void* w, bl_wfmt wfmt,
+                         const float* alpha, int64_t alpha_group, int64_t M, int64_t N, int64_t K, void* y_bf16,
+                         int64_t ldy, int32_t* acc_out, void* stream) {
+  if (afmt != BL_A_I8 && afmt != BL_A_I4 && afmt != BL_A_E2M1) return BL_ERR_ARG;
+  if (wfmt != BL_W_T2 && wfmt != BL_W_I8) return BL_ERR_ARG;
+  if (alpha_group < 1) return BL_ERR_ARG;
+  if (M < 0 || N < 1 || K < 64 || (K & 63) || K > (1 << 20) || M > 0x7FFFFFFFLL || N > 0x7FFFFFFFLL)
+    return BL_ERR_SHAPE;
+  if (y_bf16 != nullptr && (ldy < N || (ldy & 7))) return BL_ERR_SHAPE;
+  if (M == 0) return BL_OK;
+  if (a == nullptr || a_scale == nullptr || w == nullptr || alpha == nullptr) return BL_ERR_NULL;
+  if (y_bf16 == nullptr && acc_out == nullptr) return BL_ERR_NULL;
+  if (!aligned16(a) || !aligned16(w) || (y_bf16 && !aligned16(y_bf16)) || (acc_out && !aligned16(acc_out)) ||
+      (reinterpret_cast<uintptr_t>(a_scale) & 3u) || (reinterpret_cast<uintptr_t>(alpha) & 3u))
+    return BL_ERR_ALIGN;
+  cudaStream_t s = as_stream(stream);
+  const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+  const uint8_t* A = static_cast<const uint8_t*>(a);
+  const uint8_t* W = static_cast<const uint8_t*>(w);
+  uint16_t* Y = static_cast<uint16_t*>(y_bf16);
+
+  if (afmt == BL_A_I8 && wfmt == BL_W_I8) {
+    if (!tc_kernel_ready()) return BL_ERR_CUDA;
+    CUtensorMap ta, tb;
+    if (!make_i8_map(&ta, A, static_cast<uint64_t>(M), static_cast<uint64_t>(K), bl::kTcBM, bl::kTcBK) ||
+        !make_i8_map(&tb, W, static_cast<uint64_t>(N), static_cast<uint64_t>(K), bl::kTcBN, bl::kTcBK))
+      return BL_ERR_CUDA;
+    bl::TcParams p;
+    p.a_scale = a_scale;
+    p.alpha = alpha;
+    p.alpha_group = alpha_group;
+    p.M = m;
+    p.N = n;
+    p.K = k;
+    p.y = Y;
+    p.ldy = ldy;
+    p.acc = acc_out;
+    p.num_m_blocks = (m + bl::kTcBM - 1) / bl::kTcBM;
+    p.num_n_blocks = (n + bl::kTcBN - 1) / bl::kTcBN;
+    p.num_tiles = p.num_m_blocks * p.num_n_blocks;
+    p.num_kb = (k + bl::kTcBK - 1) / bl::kTcBK;
+    const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
+    bl::gemm_tc_kernel<<<grid, bl::kTcThreads, bl::kTcSmemBytes, s>>>(ta, tb, p);
+    return launch_status();
+  }
+  const bool t2 = wfmt == BL_W_T2;
+  switch (afmt) {
+    case BL_A_I8:
+      if (t2) launch_simt<bl::kSimtA_I8, true>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+      else launch_simt<bl::kSimtA_I8, false>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+      break;
+    case BL_A_I4:
+      if (t2) launch_simt<bl::kSimtA_I4, true>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+      else launch_simt<bl::kSimtA_I4, false>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+      break;
+    default:
+      if (t2) launch_simt<bl::kSimtA_E2M1, true>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+      else launch_simt<bl::kSimtA_E2M1, false>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+      break;
+  }
+  return launch_status();
+}
+
+bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D, int64_t ldt, int bits, int64_t bos_pos,
+                    float eps, uint8_t* codes, float* scale, uint8_t* bos_codes, void* stream) {
+  if (bits != 3 && bits != 4) return BL_ERR_ARG;
+  if (T < 0 || H < 1 || D < 32 || D > 256 || (D & 31) || ldt < H * D || (ldt & 7)) return BL_ERR_SHAPE;
+  if (bos_pos < -1) return BL_ERR_ARG;
+  if (!(eps >= 0.f)) return BL_ERR_ARG;
+  if (T * H * (D / 8) > (int64_t(1) << 40) || H > 0x7FFFFFFF) return BL_ERR_SHAPE;
+  if (T == 0) return BL_OK;
+  const bool has_bos = bits == 3 && bos_pos >= 0 && bos_pos < T;
+  if (kv_bf16 == nullptr || codes == nullptr || scale == nullptr || (has_bos && bos_codes == nullptr))
+    return BL_ERR_NULL;
+  if (!aligned16(kv_bf16) || !aligned16(codes) || !aligned16(scale) || (has_bos && !aligned16(bos_codes)))
+    return BL_ERR_ALIGN;
+  const int tpv = static_cast<int>(D / 8);
+  const int64_t threads = T * H * tpv;
+  const unsigned grid = static_cast<unsigned>((threads + 255) / 256);
+  const uint16_t* kv = static_cast<const uint16_t*>(kv_bf16);
+  cudaStream_t s = as_stream(stream);
+  const int64_t bos = has_bos ? bos_pos : -1;
+  const int h = static_cast<int>(H);
+  switch (tpv) {
+    case 4: bl::kv_quant_kernel<4><<<grid, 256, 0, s>>>(kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
+    case 8: bl::kv_quant_kernel<8><<<grid, 256, 0, s>>>(kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
+    case 16: bl::kv_quant_kernel<16><<<grid, 256, 0, s>>>(kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
+    case 32: bl::kv_quant_kernel<32><<<grid, 256, 0, s>>>(kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
+    default: return BL_ERR_SHAPE;
+  }
+  return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,414 @@
+// BitLinear product (BitNet a4.8, §3.4: Y = Q_x(X) . Q_w(W)^T with integer
+// accumulation, then the per-token x per-tensor dequant):
+//   acc[m,n] = sum_k a[m,k] * t[n,k],   y[m,n] = bf16(acc * a_scale[m] * alpha[n / group])
+//
+// gemm_tc_kernel   -- int8 x int8 on the 5th-generation tensor cores
+//                     (tcgen05.mma kind::i8, s32 accumulators in TMEM), operands
+//                     streamed by TMA into a 128B-swizzled shared-memory ring,
+//                     persistent over output tiles with a double-buffered
+//                     accumulator so the epilogue overlaps the next tile.
+// gemm_simt_kernel -- CUDA-core kernel that reads packed operands directly
+//                     (2-bit ternary weights, INT4 / E2M1 nibbles); the decode
+//                     path, where the packed weight bytes set the time.
+#pragma once
+
+#include "common.cuh"
+
+namespace bl {
+
+// ---------------------------------------------------------------------------
+// tcgen05 kernel
+// ---------------------------------------------------------------------------
+constexpr int kTcBM = 128;      // tile rows (TMEM lanes)
+constexpr int kTcBN = 256;      // tile columns (TMEM columns per accumulator)
+constexpr int kTcBK = 128;      // K bytes per stage = one 128-byte swizzle atom row
+constexpr int kTcStages = 4;
+constexpr int kTcThreads = 192; // warp 0: TMA producer, warp 1: MMA issuer, warps 2-5: epilogue
+constexpr uint32_t kTcStageA = kTcBM * kTcBK;
+constexpr uint32_t kTcStageB = kTcBN * kTcBK;
+constexpr uint32_t kTcTmemCols = 2 * kTcBN;
+constexpr int kTcGroupM = 16;   // m-blocks per rasterisation group (L2 reuse of B)
+constexpr size_t kTcSmemBytes = 1024 /*align slack*/ + kTcStages * (kTcStageA + kTcStageB) + 256;
+
+struct TcParams {
+  const float* a_scale;
+  const float* alpha;
+  int64_t alpha_group;
+  int M, N, K;
+  uint16_t* y;
+  int64_t ldy;
+  int32_t* acc;
+  int num_m_blocks, num_n_blocks, num_tiles, num_kb;
+};
+
+// Shared-memory matrix descriptor for a K-major operand tile written by TMA
+// with 128-byte swizzling: rows of 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4)    // start address, 16-byte units
+         | (static_cast<uint64_t>(1) << 16)                 // leading offset (unused for this layout)
+         | (static_cast<uint64_t>(1024 >> 4) << 32)         // stride offset between 8-row groups
+         | (static_cast<uint64_t>(1) << 46)                 // descriptor version for sm_100
+         | (static_cast<uint64_t>(2) << 61);                // 128-byte swizzle
+}
+
+// Instruction descriptor: s32 accumulate, signed int8 A and B, both K-major,
+// N = 256, M = 128.
+constexpr uint32_t kTcIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(kTcBN) >> 3) << 17) |
+                              ((static_cast<uint32_t>(kTcBM) >> 4) << 24);
+
+__device__ __forceinline__ void tc_tile_coords(int tile, int nmb, int nnb, int& mb, int& nb) {
+  const int group = tile / (kTcGroupM * nnb);
+  const int first_m = group * kTcGroupM;
+  const int gsize = min(nmb - first_m, kTcGroupM);
+  const int in = tile - group * kTcGroupM * nnb;
+  mb = first_m + in % gsize;
+  nb = in / gsize;
+}
+
+// Lane 0 waits (bounded) and the result is shared with the warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+  const int lane = threadIdx.x & 31;
+  uint32_t ok = 1;
+  if (lane == 0) ok = mbar_wait_bounded(bar, parity) ? 1u : 0u;
+  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kTcStages * kTcStageA;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kTcStages * kTcStageB);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kTcStages;
+  uint64_t* tfull = bars + 2 * kTcStages;
+  uint64_t* tempty = bars + 2 * kTcStages + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kTcStages + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTcTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  bool aborted = false;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int tile = blockIdx.x; tile < p.num_tiles && !aborted; tile += gridDim.x) {
+        int mb, nb;
+        tc_tile_coords(tile, p.num_m_blocks, p.num_n_blocks, mb, nb);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait_bounded(&empty[s], ph ^ 1u)) {
+            aborted = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], kTcStageA + kTcStageB);
+          tma_load_2d(&tmA, &full[s], sA + s * kTcStageA, kb * kTcBK, mb * kTcBM);
+          tma_load_2d(&tmB, &full[s], sB + s * kTcStageB, kb * kTcBK, nb * kTcBN);
+          if (++s == kTcStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (one thread) ----------------
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int local = 0;
+      for (int tile = blockIdx.x; tile < p.num_tiles && !aborted; tile += gridDim.x, ++local) {
+        const int buf = local & 1;
+        const uint32_t tph = (local >> 1) & 1;
+        if (!mbar_wait_bounded(&tempty[buf], tph ^ 1u)) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kTcBN);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait_bounded(&full[s], ph)) {
+            aborted = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * kTcStageA);
+          const uint32_t b0 = smem_u32(sB + s * kTcStageB);
+#pragma unroll
+          for (int kk = 0; kk < kTcBK / 32; ++kk) {
+            mma_i8(d_tmem, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), kTcIdesc,
+                   (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);  // frees the stage once these MMAs have read it
+          if (++s == kTcStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (aborted) break;
+        mma_commit(&tfull[buf]);  // accumulator ready for the epilogue
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2-5) ----------------
+    const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad + 32) belong to this warp
+    int local = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
+      const int buf = local & 1;
+      const uint32_t tph = (local >> 1) & 1;
+      if (!warp_wait(&tfull[buf], tph)) {
+        aborted = true;
+        break;
+      }
+      tc_fence_after();
+      int mb, nb;
+      tc_tile_coords(tile, p.num_m_blocks, p.num_n_blocks, mb, nb);
+      const int row = mb * kTcBM + quad * 32 + lane;
+      const bool row_ok = row < p.M;
+      const float rs = row_ok ? p.a_scale[row] : 0.f;
+#pragma unroll 1
+      for (int c = 0; c < kTcBN / 32; ++c) {
+        uint32_t r[32];
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                               static_cast<uint32_t>(buf * kTcBN + c * 32);
+        tmem_ld_32x32b_x32(taddr, r);
+        tmem_wait_ld();
+        const int n0 = nb * kTcBN + c * 32;
+        if (!row_ok || n0 >= p.N) continue;
+        const int64_t ga = n0 / p.alpha_group;
+        const bool one_alpha = ((n0 + 31) / p.alpha_group) == ga;
+        const float cs_uniform = __fmul_rn(rs, p.alpha[one_alpha ? ga : 0]);
+        float yv[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float cs = one_alpha ? cs_uniform
+                                     : __fmul_rn(rs, p.alpha[min(static_cast<int64_t>(n0 + j), static_cast<int64_t>(p.N - 1)) / p.alpha_group]);
+          yv[j] = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), cs);
+        }
+        const bool full_chunk = n0 + 32 <= p.N;
+        if (p.y != nullptr) {
+          uint16_t* yr = p.y + static_cast<int64_t>(row) * p.ldy + n0;
+          if (full_chunk) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 o;
+              o.x = pack_bf16x2(yv[8 * q + 0], yv[8 * q + 1]);
+              o.y = pack_bf16x2(yv[8 * q + 2], yv[8 * q + 3]);
+              o.z = pack_bf16x2(yv[8 * q + 4], yv[8 * q + 5]);
+              o.w = pack_bf16x2(yv[8 * q + 6], yv[8 * q + 7]);
+              reinterpret_cast<uint4*>(yr)[q] = o;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (n0 + j < p.N) {
+                const __nv_bfloat16 b = __float2bfloat16_rn(yv[j]);
+                yr[j] = *reinterpret_cast<const uint16_t*>(&b);
+              }
+            }
+          }
+        }
+        if (p.acc != nullptr) {
+          int32_t* ar = p.acc + static_cast<int64_t>(row) * p.N + n0;
+          if (full_chunk && (p.N & 3) == 0) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              reinterpret_cast<uint4*>(ar)[q] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n0 + j < p.N) ar[j] = static_cast<int32_t>(r[j]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+    }
+  }
+
+  __syncthreads();
+  if (aborted) {
+    // let any copies or MMAs still in flight land before the CTA's memory goes away
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) {
+    }
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTcTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-core kernel for packed operands.  One warp per output column n (a row
+// of W); lanes split K in units of 64 codes; MT rows of A per pass share the
+// expanded weight unit.  dp4a on int8x4 words.
+// ---------------------------------------------------------------------------
+enum : int { kSimtA_I8 = 0, kSimtA_I4 = 1, kSimtA_E2M1 = 2 };
+
+// four 2-bit ternary codes (one byte) -> four int8 {-1,0,1} (two's-complement sign extension)
+__device__ __forceinline__ uint32_t expand_t2_byte(uint32_t b) {
+  const uint32_t spread = (b & 0x3u) | ((b & 0xCu) << 6) | ((b & 0x30u) << 12) | ((b & 0xC0u) << 18);
+  return __vsub4(spread ^ 0x02020202u, 0x02020202u);
+}
+
+// eight nibbles of a word -> two words of four bytes each, in element order
+__device__ __forceinline__ void split_nibbles(uint32_t p, uint32_t& w0, uint32_t& w1) {
+  const uint32_t lo = p & 0x0F0F0F0Fu;
+  const uint32_t hi = (p >> 4) & 0x0F0F0F0Fu;
+  w0 = __byte_perm(lo, hi, 0x5140);
+  w1 = __byte_perm(lo, hi, 0x7362);
+}
+
+__device__ __forceinline__ uint32_t sext_nibble_bytes(uint32_t x) { return __vsub4(x ^ 0x08080808u, 0x08080808u); }
+
+// E2M1 codes in bytes -> twice their value as int8: magnitudes {0,1,2,3,4,6,8,12}
+__device__ __forceinline__ uint32_t e2m1_bytes_to_twice(uint32_t x) {
+  const uint32_t idx = x & 0x07070707u;
+  const uint32_t sel = (idx & 0x7u) | ((idx >> 4) & 0x70u) | ((idx >> 8) & 0x700u) | ((idx >> 12) & 0x7000u);
+  const uint32_t mag = __byte_perm(0x03020100u, 0x0C080604u, sel);
+  const uint32_t m = ((x & 0x08080808u) >> 3) * 0xFFu;
+  return (mag & ~m) | (__vsub4(0u, mag) & m);
+}
+
+template <int AF>
+__device__ __forceinline__ void load_a_unit(const uint8_t* a_row, int u, uint32_t (&out)[16]) {
+  if constexpr (AF == kSimtA_I8) {
+    const uint4* p = reinterpret_cast<const uint4*>(a_row + static_cast<int64_t>(u) * 64);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = p[i];
+      out[4 * i] = v.x; out[4 * i + 1] = v.y; out[4 * i + 2] = v.z; out[4 * i + 3] = v.w;
+    }
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(a_row + static_cast<int64_t>(u) * 32);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint4 v = p[i];
+      const uint32_t pk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t w0, w1;
+        split_nibbles(pk[j], w0, w1);
+        if constexpr (AF == kSimtA_I4) {
+          out[8 * i + 2 * j] = sext_nibble_bytes(w0);
+          out[8 * i + 2 * j + 1] = sext_nibble_bytes(w1);
+        } else {
+          out[8 * i + 2 * j] = e2m1_bytes_to_twice(w0);
+          out[8 * i + 2 * j + 1] = e2m1_bytes_to_twice(w1);
+        }
+      }
+    }
+  }
+}
+
+template <bool WT2>
+__device__ __forceinline__ void load_w_unit(const uint8_t* w_row, int u, uint32_t (&out)[16]) {
+  if constexpr (WT2) {
+    const uint4 v = ld_global_nc_v4(w_row + static_cast<int64_t>(u) * 16);
+    const uint32_t pk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) out[4 * j + b] = expand_t2_byte((pk[j] >> (8 * b)) & 0xFFu);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = ld_global_nc_v4(w_row + static_cast<int64_t>(u) * 64 + 16 * i);
+      out[4 * i] = v.x; out[4 * i + 1] = v.y; out[4 * i + 2] = v.z; out[4 * i + 3] = v.w;
+    }
+  }
+}
+
+template <int AF, bool WT2, int MT>
+__global__ void __launch_bounds__(256) gemm_simt_kernel(const uint8_t* __restrict__ a, const float* __restrict__ a_scale,
+                                                        const uint8_t* __restrict__ w, const float* __restrict__ alpha,
+                                                        int64_t alpha_group, int M, int N, int K,
+                                                        uint16_t* __restrict__ y, int64_t ldy,
+                                                        int32_t* __restrict__ acc_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gwarp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int units = K >> 6;
+  const int64_t a_row_bytes = (AF == kSimtA_I8) ? K : (K >> 1);
+  const int64_t w_row_bytes = WT2 ? (K >> 2) : K;
+  const float unit_scale = (AF == kSimtA_E2M1) ? 0.5f : 1.0f;
+
+  for (int64_t n = gwarp; n < N; n += nwarps) {
+    const uint8_t* w_row = w + n * w_row_bytes;
+    const float al = alpha[n / alpha_group];
+    for (int m0 = 0; m0 < M; m0 += MT) {
+      int acc[MT];
+#pragma unroll
+      for (int r = 0; r < MT; ++r) acc[r] = 0;
+      for (int u = lane; u < units; u += 32) {
+        uint32_t wu[16];
+        load_w_unit<WT2>(w_row, u, wu);
+#pragma unroll
+        for (int r = 0; r < MT; ++r) {
+          if (m0 + r < M) {
+            uint32_t au[16];
+            load_a_unit<AF>(a + static_cast<int64_t>(m0 + r) * a_row_bytes, u, au);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[r] = __dp4a(static_cast<int>(au[i]), static_cast<int>(wu[i]), acc[r]);
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < MT; ++r) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[r] += __shfl_xor_sync(0xFFFFFFFFu, acc[r], o);
+      }
+      if (lane < MT) {
+        int mine = 0;
+#pragma unroll
+        for (int r = 0; r < MT; ++r)
+          if (r == lane) mine = acc[r];
+        const int m = m0 + lane;
+        if (m < M) {
+          if (acc_out != nullptr) acc_out[static_cast<int64_t>(m) * N + n] = mine;
+          if (y != nullptr) {
+            const float cs = __fmul_rn(__fmul_rn(a_scale[m], unit_scale), al);
+            const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__int2float_rn(mine), cs));
+            y[static_cast<int64_t>(m) * ldy + n] = *reinterpret_cast<const uint16_t*>(&b);
+          }
+        }
+      }
+    }
+  }
+}
+
+}  // namespace bl

@@ -1,0 +1,199 @@
+// Absmean ternary weight quantizer and packer (BitNet a4.8, §3.4 "Ternary
+// Weight Quantization (BitLinear)", Eq. 2):
+//   alpha = mean|W| (per tensor),  t = RoundClip(W / (alpha + eps), -1, 1).
+//
+// alpha is the exact mean rounded once to fp32.  |w| = m * 2^(max(E,1) - 150)
+// with m the 24-bit significand and E the biased exponent, so the exact sum is
+// held as one unsigned 64-bit integer per exponent (bins[E] += m); integer adds
+// are exact and order-free.  A single thread then forms
+//   Z = sum_E bins[E] << (max(E,1) - 1)          (the sum in units of 2^-149)
+// as a multi-word integer, divides by N*K and rounds to nearest-even fp32.
+#pragma once
+
+#include "common.cuh"
+
+namespace bl {
+
+constexpr int kBinThreads = 256;
+constexpr int kBinWarps = kBinThreads / 32;
+
+// Per-CTA: a private bin set per warp in shared memory, merged into the 256
+// global bins with one atomic per non-empty bin.
+__global__ void __launch_bounds__(kBinThreads) ternary_bins_kernel(const float* __restrict__ w, int64_t N, int K,
+                                                                   int64_t ldw,
+                                                                   unsigned long long* __restrict__ gbins) {
+  __shared__ unsigned long long sb[kBinWarps][256];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kBinWarps * 256; i += kBinThreads) (&sb[0][0])[i] = 0ull;
+  __syncthreads();
+  const int per_row = K >> 2;  // float4 per row
+  const int64_t total = N * static_cast<int64_t>(per_row);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * kBinThreads + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * kBinThreads) {
+    const int64_t n = i / per_row;
+    const int q = static_cast<int>(i - n * per_row);
+    const uint4 v = ld_global_nc_v4(w + n * ldw + static_cast<int64_t>(q) * 4);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t a = u[j] & 0x7FFFFFFFu;
+      const uint32_t e = a >> 23;
+      const uint32_t m = (a & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+      if (m) atomicAdd(&sb[warp][e], static_cast<unsigned long long>(m));
+    }
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < 256; b += kBinThreads) {
+    unsigned long long s = 0;
+#pragma unroll
+    for (int wv = 0; wv < kBinWarps; ++wv) s += sb[wv][b];
+    if (s) atomicAdd(&gbins[b], s);
+  }
+  (void)lane;
+}
+
+// Multi-word unsigned integer, little-endian 32-bit limbs.
+constexpr int kLimbs = 12;  // 384 bits: bins < 2^64 shifted by <= 253 bits
+
+__device__ __forceinline__ void big_add_shifted(uint32_t (&z)[kLimbs], unsigned long long v, int shift) {
+  const int li = shift >> 5, bo = shift & 31;
+  // v << bo spans up to three limbs
+  const uint32_t p0 = static_cast<uint32_t>(v << bo);
+  const uint32_t p1 = static_cast<uint32_t>((bo ? (v >> (32 - bo)) : (v >> 32)));
+  const uint32_t p2 = static_cast<uint32_t>(bo ? (v >> (64 - bo)) : 0ull);
+  const uint32_t parts[3] = {p0, p1, p2};
+  unsigned long long carry = 0;
+  for (int i = li; i < kLimbs; ++i) {
+    const unsigned long long add = (i - li < 3) ? parts[i - li] : 0u;
+    const unsigned long long s = static_cast<unsigned long long>(z[i]) + add + carry;
+    z[i] = static_cast<uint32_t>(s);
+    carry = s >> 32;
+    if (i - li >= 2 && carry == 0) break;
+  }
+}
+
+__device__ __forceinline__ int big_bitlen(const uint32_t (&z)[kLimbs]) {
+  for (int i = kLimbs - 1; i >= 0; --i)
+    if (z[i]) return 32 * i + (32 - __clz(z[i]));
+  return 0;
+}
+
+__device__ __forceinline__ uint32_t big_bit(const uint32_t (&z)[kLimbs], int b) {
+  return (b < 0 || b >= 32 * kLimbs) ? 0u : (z[b >> 5] >> (b & 31)) & 1u;
+}
+
+// Any bit set strictly below position b?
+__device__ __forceinline__ bool big_any_below(const uint32_t (&z)[kLimbs], int b) {
+  if (b <= 0) return false;
+  const int full = b >> 5;
+  for (int i = 0; i < full && i < kLimbs; ++i)
+    if (z[i]) return true;
+  const int rem = b & 31;
+  return rem && full < kLimbs && (z[full] & ((1u << rem) - 1u));
+}
+
+// 64-bit window of z starting at bit `sh` (sh >= 0).
+__device__ __forceinline__ unsigned long long big_window64(const uint32_t (&z)[kLimbs], int sh) {
+  unsigned long long r = 0;
+  for (int j = 0; j < 64; ++j) r |= static_cast<unsigned long long>(big_bit(z, sh + j)) << j;
+  return r;
+}
+
+// alpha = RN_fp32( (Z * 2^-149) / D ), single thread.
+__global__ void ternary_alpha_kernel(const unsigned long long* __restrict__ gbins, unsigned long long D,
+                                     float* __restrict__ alpha) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  uint32_t z[kLimbs];
+  for (int i = 0; i < kLimbs; ++i) z[i] = 0;
+  for (int e = 0; e < 256; ++e) {
+    const unsigned long long b = gbins[e];
+    if (b) big_add_shifted(z, b, (e > 0 ? e : 1) - 1);
+  }
+  // Long division Q = floor(Z / D), R = Z mod D.
+  uint32_t q[kLimbs];
+  unsigned __int128 rem = 0;
+  for (int i = kLimbs - 1; i >= 0; --i) {
+    const unsigned __int128 cur = (rem << 32) | z[i];
+    q[i] = static_cast<uint32_t>(cur / D);
+    rem = cur % D;
+  }
+  const unsigned long long R = static_cast<unsigned long long>(rem);
+  const int L = big_bitlen(q);
+  float result;
+  if (L == 0) {
+    // value * 2^149 = R/D < 1: rounds to 0 or to the smallest subnormal
+    result = (2 * static_cast<unsigned __int128>(R) > D) ? __uint_as_float(1u) : 0.f;
+  } else {
+    // value = (Q + R/D) * 2^-149, top bit of Q at L-1 -> exponent L-1-149.
+    // Keep 24 significant bits, or all bits down to 2^-149 when subnormal.
+    const int shift = (L - 1 - 23 > 0) ? (L - 1 - 23) : 0;
+    unsigned long long mant = big_window64(q, shift) & ((1ull << 25) - 1ull);
+    bool up;
+    if (shift == 0) {
+      const unsigned __int128 twoR = 2 * static_cast<unsigned __int128>(R);
+      up = twoR > D || (twoR == D && (mant & 1ull));
+    } else {
+      const uint32_t half = big_bit(q, shift - 1);
+      const bool below = big_any_below(q, shift - 1) || R != 0;
+      up = half && (below || (mant & 1ull));
+    }
+    mant += up ? 1ull : 0ull;
+    int lsb_exp = shift - 149;  // value = mant * 2^lsb_exp
+    if (mant >> 24) {           // carried into a new binade
+      mant >>= 1;
+      lsb_exp += 1;
+    }
+    if (mant >> 23) {
+      const int biased = lsb_exp + 23 + 127;
+      result = biased >= 255 ? __uint_as_float(0x7F800000u)
+                             : __uint_as_float((static_cast<uint32_t>(biased) << 23) |
+                                               static_cast<uint32_t>(mant & 0x7FFFFFu));
+    } else {
+      result = __uint_as_float(static_cast<uint32_t>(mant));  // subnormal: lsb_exp == -149
+    }
+  }
+  *alpha = result;
+}
+
+// t = RoundClip(w / (alpha + eps), -1, 1); 16 weights per thread-step.
+//   T2: 4 bytes out (2-bit codes, element 4i in bits 0-1; 0->00, +1->01, -1->11)
+//   I8: 16 bytes out
+template <bool T2>
+__global__ void __launch_bounds__(256) ternary_pack_kernel(const float* __restrict__ w, int64_t N, int K,
+                                                           int64_t ldw, const float* __restrict__ alpha,
+                                                           float eps, uint8_t* __restrict__ out) {
+  const float d = __fadd_rn(*alpha, eps);
+  const int per_row = K >> 4;
+  const int64_t total = N * static_cast<int64_t>(per_row);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = i / per_row;
+    const int q = static_cast<int>(i - n * per_row);
+    const float* src = w + n * ldw + static_cast<int64_t>(q) * 16;
+    int c[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 v = ld_global_nc_v4(src + 4 * j);
+      c[4 * j + 0] = round_clip(__fdiv_rn(__uint_as_float(v.x), d), -1.f, 1.f);
+      c[4 * j + 1] = round_clip(__fdiv_rn(__uint_as_float(v.y), d), -1.f, 1.f);
+      c[4 * j + 2] = round_clip(__fdiv_rn(__uint_as_float(v.z), d), -1.f, 1.f);
+      c[4 * j + 3] = round_clip(__fdiv_rn(__uint_as_float(v.w), d), -1.f, 1.f);
+    }
+    if constexpr (T2) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) word |= (static_cast<uint32_t>(c[j]) & 3u) << (2 * j);
+      reinterpret_cast<uint32_t*>(out + n * static_cast<int64_t>(K >> 2))[q] = word;
+    } else {
+      uint32_t wd[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        wd[j] = (static_cast<uint32_t>(c[4 * j]) & 0xFFu) | ((static_cast<uint32_t>(c[4 * j + 1]) & 0xFFu) << 8) |
+                ((static_cast<uint32_t>(c[4 * j + 2]) & 0xFFu) << 16) | (static_cast<uint32_t>(c[4 * j + 3]) << 24);
+      reinterpret_cast<uint4*>(out + n * static_cast<int64_t>(K))[q] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+    }
+  }
+}
+
+}  // namespace bl

@@ -1,0 +1,121 @@
+"""The C ABI library: loads, exports every symbol the public header declares,
+and validates arguments on the host (these calls return before any CUDA work,
+so they need no GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import ternary_bit_activation_b200 as tba
+from ternary_bit_activation_b200 import build as tba_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    tba_build.build()
+    return tba.lib()
+
+
+def declared_symbols():
+    hdr = open(os.path.join(ROOT, "include", "bitlinear.h")).read()
+    return re.findall(r"BL_API\s+[\w\s\*]+?\b(\w+)\s*\(", hdr)
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for required in ("bitlinear_quant_a4", "bitlinear_sparsify_a8", "pack_ternary", "bitlinear_gemm",
+                     "relu2_glu", "kv_quant3"):
+        assert required in names
+    assert sorted(names) == sorted(tba.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+    assert "sm_100a" in tba.version()
+
+
+def test_status_strings(L):
+    for code, name in enumerate(tba.STATUS_NAMES):
+        assert tba.status_string(code) == name
+
+
+def test_workspace_size(L):
+    assert tba.workspace_size("pack_ternary", 0, 4096, 4096) == 2048
+    assert tba.workspace_size("bitlinear_gemm", 128, 128, 128) == 0
+
+
+# fake device addresses: validation rejects before anything dereferences them
+A16 = 0x10000
+MIS = 0x10001
+P = ctypes.c_void_p
+
+
+def test_gemm_validation(L):
+    g = L.bitlinear_gemm
+    ok = dict(a=A16, afmt=0, s=A16, w=A16, wfmt=1, al=A16, grp=256, M=128, N=256, K=256, y=A16, ldy=256, acc=None)
+
+    def call(**kw):
+        d = dict(ok, **kw)
+        return g(P(d["a"]), d["afmt"], P(d["s"]), P(d["w"]), d["wfmt"], P(d["al"]), d["grp"], d["M"], d["N"],
+                 d["K"], P(d["y"]), d["ldy"], P(d["acc"]), None)
+
+    assert call(K=100) == 3            # K % 64
+    assert call(K=0) == 3
+    assert call(N=0) == 3
+    assert call(ldy=100) == 3          # ldy < N
+    assert call(ldy=260) == 3          # ldy % 8
+    assert call(afmt=7) == 4
+    assert call(wfmt=9) == 4
+    assert call(grp=0) == 4
+    assert call(M=0) == 0              # empty: no-op
+    assert call(a=None) == 1
+    assert call(y=None, acc=None) == 1
+    assert call(a=MIS) == 2
+    assert call(w=MIS) == 2
+
+
+def test_quant_validation(L):
+    q = L.bitlinear_quant_a4
+    assert q(P(A16), 4, 100, 100, 0, 0, 1e-5, P(A16), P(A16), None) == 3    # K % 8
+    assert q(P(A16), 4, 64, 60, 0, 0, 1e-5, P(A16), P(A16), None) == 3      # ldx < K
+    assert q(P(A16), 4, 32768, 32768, 0, 0, 1e-5, P(A16), P(A16), None) == 3  # K too large
+    assert q(P(A16), 4, 64, 64, 5, 0, 1e-5, P(A16), P(A16), None) == 4
+    assert q(P(A16), 4, 64, 64, 0, 3, 1e-5, P(A16), P(A16), None) == 4
+    assert q(P(A16), 4, 64, 64, 0, 0, -1.0, P(A16), P(A16), None) == 4
+    assert q(None, 4, 64, 64, 0, 0, 1e-5, P(A16), P(A16), None) == 1
+    assert q(P(MIS), 4, 64, 64, 0, 0, 1e-5, P(A16), P(A16), None) == 2
+    assert q(P(A16), 0, 64, 64, 0, 0, 1e-5, P(A16), P(A16), None) == 0
+
+
+def test_topk_validation(L):
+    s = L.bitlinear_sparsify_a8
+    assert s(P(A16), 4, 64, 64, 0, 1e-5, P(A16), P(A16), None, None) == 4      # k_keep < 1
+    assert s(P(A16), 4, 64, 64, 65, 1e-5, P(A16), P(A16), None, None) == 4     # k_keep > K
+    assert s(P(A16), 4, 20000, 20000, 5, 1e-5, P(A16), P(A16), None, None) == 3
+    assert s(P(A16), 4, 64, 64, 5, 1e-5, P(A16), P(A16), P(MIS), None) == 2
+    r = L.relu2_glu
+    assert r(P(A16), P(A16), 4, 64, 32, 5, 1e-5, P(A16), P(A16), None, None) == 3   # ld < F
+    assert r(P(A16), None, 4, 64, 64, 5, 1e-5, P(A16), P(A16), None, None) == 1
+
+
+def test_pack_and_kv_validation(L):
+    pk = L.pack_ternary
+    assert pk(P(A16), 8, 24, 24, 1e-5, 0, P(A16), 0, P(A16), P(A16), 2048, None) == 3   # K % 16
+    assert pk(P(A16), 8, 64, 64, 1e-5, 0, P(A16), 0, P(A16), P(A16), 1024, None) == 8   # workspace too small
+    assert pk(P(A16), 8, 64, 64, 1e-5, 0, P(A16), 0, P(A16), None, 0, None) == 1
+    assert pk(P(A16), 8, 64, 64, 1e-5, 0, P(A16), 5, P(A16), P(A16), 2048, None) == 4
+    kv = L.kv_quant3
+    assert kv(P(A16), 8, 4, 100, 400, 3, 0, 1e-5, P(A16), P(A16), P(A16), None) == 3     # D % 32
+    assert kv(P(A16), 8, 4, 128, 512, 5, 0, 1e-5, P(A16), P(A16), P(A16), None) == 4     # bits
+    assert kv(P(A16), 8, 4, 128, 512, 3, 0, 1e-5, P(A16), P(A16), None, None) == 1       # BOS buffer needed
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(tba, "_lib", None)
+    monkeypatch.setattr(tba, "LIB_PATH", str(tmp_path / "nope.so"))
+    with pytest.raises(RuntimeError):
+        tba.lib()

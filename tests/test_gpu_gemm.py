@@ -1,0 +1,190 @@
+"""GPU parity of the ternary packer and the BitLinear GEMM (tcgen05 and
+CUDA-core kernels) against the CPU oracle, through the C ABI.  alpha, packed
+codes and int32 accumulators are compared bit for bit; bf16 outputs per row
+within 1e-2 of the fp64 product (max |err| over the row's norm)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import ternary_bit_activation_b200 as tba
+from gpu_util import BF16_ROW_TOL, bf16_rows_rel_err, empty, host, to_dev
+
+pytestmark = pytest.mark.gpu
+
+EPS = 1e-5
+
+
+def run_pack(w, wfmt, alpha_in=None):
+    N, K = w.shape
+    wd = to_dev(w)
+    out = empty((N, K // 4 if wfmt == tba.BL_W_T2 else K), torch.uint8)
+    ws = empty((tba.workspace_size("pack_ternary", 0, N, K) // 8,), torch.int64)
+    alpha = empty((1,), torch.float32)
+    if alpha_in is not None:
+        alpha.fill_(float(alpha_in))
+    tba.pack_ternary(wd, alpha, out, wfmt=wfmt, workspace=ws, alpha_given=alpha_in is not None, eps=EPS)
+    tba.sync_status()
+    return host(out), host(alpha)[0]
+
+
+PACK_CASES = [
+    ("tiny_256x256", lambda: synth.tiny_inputs(0)[1]),
+    ("700M_qkv", lambda: synth.latent_weights_f32(synth.rng(21), 4608, 1536)),
+    ("odd_rows_K3200", lambda: synth.latent_weights_f32(synth.rng(22), 33, 3200)),
+    ("tiny_values", lambda: (synth.latent_weights_f32(synth.rng(23), 16, 64) * np.float32(1e-36))),
+    ("constant", lambda: np.full((8, 64), -0.0213, np.float32)),
+    ("zeros", lambda: np.zeros((4, 64), np.float32)),
+]
+
+
+@pytest.mark.parametrize("name,make", PACK_CASES, ids=[c[0] for c in PACK_CASES])
+@pytest.mark.parametrize("wfmt", [tba.BL_W_T2, tba.BL_W_I8], ids=["t2", "i8"])
+def test_pack_ternary_parity(name, make, wfmt):
+    w = make()
+    out, alpha = run_pack(w, wfmt)
+    t_ref, a_ref = oracle.ternary_quantize(w, EPS)
+    assert np.float32(alpha).view(np.uint32) == np.float32(a_ref).view(np.uint32), (alpha, a_ref)
+    if wfmt == tba.BL_W_T2:
+        assert np.array_equal(out, oracle.pack_ternary2(t_ref))
+    else:
+        assert np.array_equal(out.view(np.int8), t_ref)
+
+
+def test_pack_ternary_alpha_given():
+    w = synth.latent_weights_f32(synth.rng(24), 64, 256)
+    for a in (0.011, 0.016, 0.05):
+        out, alpha = run_pack(w, tba.BL_W_I8, alpha_in=a)
+        assert alpha == np.float32(a)
+        assert np.array_equal(out.view(np.int8), oracle.ternary_codes(w, np.float32(a), EPS))
+
+
+def exact_y(a_codes, a_scale, t_codes, alpha, group, rows):
+    al = np.atleast_1d(np.asarray(alpha, np.float64))
+    N = t_codes.shape[0]
+    acc = a_codes[rows].astype(np.int64) @ t_codes.astype(np.int64).T
+    col_alpha = al[np.arange(N) // group]
+    return acc, acc.astype(np.float64) * a_scale[rows, None].astype(np.float64) * col_alpha[None, :]
+
+
+def run_gemm(a_dev, afmt, scale, w_dev, wfmt, alpha, M, N, K, group=None, want_acc=True, ldy=None):
+    ldy = (N + 7) // 8 * 8 if ldy is None else ldy     # rows of y stay 16-byte aligned
+    y = empty((M, ldy), torch.int16)
+    acc = empty((M, N), torch.int32) if want_acc else None
+    al = to_dev(np.atleast_1d(np.asarray(alpha, np.float32)))
+    tba.bitlinear_gemm(a_dev, to_dev(scale), w_dev, al, M, N, K, y=y, acc=acc, afmt=afmt, wfmt=wfmt,
+                       alpha_group=group, ldy=ldy)
+    tba.sync_status()
+    return (host(acc) if want_acc else None), host(y, np.uint16)[:, :N]
+
+
+GEMM_TC_CASES = [
+    ("tiny_16x256x256", 16, 256, 256),
+    ("one_row", 1, 256, 128),
+    ("K_tail_200x300x320", 200, 300, 320),
+    ("multi_tile_384x768x1536", 384, 768, 1536),
+    ("ragged_257x520x3200", 257, 520, 3200),
+    ("many_tiles_1300x2304x1024", 1300, 2304, 1024),
+]
+
+
+@pytest.mark.parametrize("name,M,N,K", GEMM_TC_CASES, ids=[c[0] for c in GEMM_TC_CASES])
+def test_gemm_tc_parity(name, M, N, K):
+    g = synth.rng(M * 7 + N + K)
+    a = g.integers(-128, 128, (M, K)).astype(np.int8)
+    t = g.integers(-1, 2, (N, K)).astype(np.int8)
+    scale = (g.random(M) * 0.1 + 1e-3).astype(np.float32)
+    alpha = np.float32(0.0173)
+    acc, y = run_gemm(to_dev(a), tba.BL_A_I8, scale, to_dev(t), tba.BL_W_I8, alpha, M, N, K)
+    acc_ref, _ = oracle.gemm(a, scale, t, alpha, want_y=False)
+    assert np.array_equal(acc, acc_ref)
+    _, ex = exact_y(a, scale, t, alpha, N, np.arange(M))
+    assert bf16_rows_rel_err(y, ex) <= BF16_ROW_TOL
+    _, y_or = oracle.gemm(a, scale, t, alpha, rows=np.arange(min(M, 8)))
+    yo = synth.bf16_bits_to_f32(y_or).astype(np.float64)
+    yg = synth.bf16_bits_to_f32(y[:min(M, 8)]).astype(np.float64)
+    assert np.all(np.abs(yg - yo) <= np.abs(yo) * 2.0 ** -7 + 1e-30)   # within one bf16 ulp
+
+
+def test_gemm_tc_alpha_groups_and_ldy():
+    # stacked Up|Gate weights with one alpha per tensor; output written into a wider row
+    M, F, K = 130, 384, 512
+    g = synth.rng(31)
+    a = g.integers(-8, 8, (M, K)).astype(np.int8)
+    t = g.integers(-1, 2, (2 * F, K)).astype(np.int8)
+    scale = (g.random(M) + 0.5).astype(np.float32)
+    alpha = np.array([0.0151, 0.0213], np.float32)
+    acc, y = run_gemm(to_dev(a), tba.BL_A_I8, scale, to_dev(t), tba.BL_W_I8, alpha, M, 2 * F, K, group=F,
+                      ldy=2 * F + 64)
+    acc_ref, _ = oracle.gemm(a, scale, t, alpha, alpha_group=F, want_y=False)
+    assert np.array_equal(acc, acc_ref)
+    _, ex = exact_y(a, scale, t, alpha, F, np.arange(M))
+    assert bf16_rows_rel_err(y, ex) <= BF16_ROW_TOL
+
+
+def test_bitlinear_end_to_end_tiny():
+    # the tiny configuration end to end: quantize X (INT4 and Top-K/INT8),
+    # pack W, multiply -- all on the GPU -- against the oracle chain
+    x, w = synth.tiny_inputs(0)
+    M, K = x.shape
+    N = w.shape[0]
+    xd = to_dev(x)
+    w8, alpha = run_pack(w, tba.BL_W_I8)
+    t_ref, a_ref = oracle.ternary_quantize(w, EPS)
+    codes = empty((M, K), torch.uint8)
+    scale = empty((M,), torch.float32)
+    tba.bitlinear_quant_a4(xd, codes, scale, quant=tba.BL_QUANT_INT4, store=tba.BL_STORE_BYTES, eps=EPS)
+    al = to_dev(np.array([alpha], np.float32))
+    y = empty((M, N), torch.int16)
+    acc = empty((M, N), torch.int32)
+    tba.bitlinear_gemm(codes, scale, to_dev(w8), al, M, N, K, y=y, acc=acc)
+    tba.sync_status()
+    c_ref, _, s_ref = oracle.quant_int4(x, EPS)
+    acc_ref, y_ref = oracle.gemm(c_ref, s_ref, t_ref, a_ref)
+    assert np.array_equal(host(acc), acc_ref)
+    _, ex = exact_y(c_ref, s_ref, t_ref, a_ref, N, np.arange(M))
+    assert bf16_rows_rel_err(host(y, np.uint16), ex) <= BF16_ROW_TOL
+    # Top-K 50% + INT8 path
+    keep = synth.k_keep(K, 50)
+    c8 = empty((M, K), torch.int8)
+    s8 = empty((M,), torch.float32)
+    tba.bitlinear_sparsify_a8(xd, keep, c8, s8, None, eps=EPS)
+    tba.bitlinear_gemm(c8, s8, to_dev(w8), al, M, N, K, y=y, acc=acc)
+    tba.sync_status()
+    c8_ref, _, _, s8_ref = oracle.sparsify_a8(x, keep, EPS)
+    acc_ref, _ = oracle.gemm(c8_ref, s8_ref, t_ref, a_ref, want_y=False)
+    assert np.array_equal(host(acc), acc_ref)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 17])
+@pytest.mark.parametrize("afmt", ["i8", "i4", "e2m1"])
+@pytest.mark.parametrize("wfmt", [tba.BL_W_T2, tba.BL_W_I8], ids=["t2", "i8w"])
+def test_gemm_simt_parity(M, afmt, wfmt):
+    N, K = 96, 640
+    g = synth.rng(M + 100)
+    x = synth.gaussian_bf16(g, (M, K))
+    w = synth.latent_weights_f32(g, N, K)
+    t_ref, a_ref = oracle.ternary_quantize(w, EPS)
+    wq = oracle.pack_ternary2(t_ref) if wfmt == tba.BL_W_T2 else t_ref.view(np.uint8)
+    if afmt == "i8":
+        a_codes, _, _, scale = oracle.sparsify_a8(x, K // 2, EPS)
+        a_dev, af, acc_codes = to_dev(a_codes), tba.BL_A_I8, a_codes
+        acc_scale = scale
+    elif afmt == "i4":
+        c, _, scale = oracle.quant_int4(x, EPS)
+        a_dev, af, acc_codes = to_dev(oracle.pack_nibbles(c)), tba.BL_A_I4, c
+        acc_scale = scale
+    else:
+        code4, twice, _, scale = oracle.quant_fp4(x)
+        a_dev, af, acc_codes = to_dev(oracle.pack_nibbles(code4)), tba.BL_A_E2M1, twice
+        acc_scale = (scale.astype(np.float64) / 2).astype(np.float32)
+    acc, y = run_gemm(a_dev, af, scale, to_dev(wq), wfmt, a_ref, M, N, K)
+    acc_ref, _ = oracle.gemm(acc_codes, acc_scale, t_ref, a_ref, want_y=False)
+    assert np.array_equal(acc, acc_ref)
+    _, ex = exact_y(acc_codes, acc_scale, t_ref, a_ref, N, np.arange(M))
+    assert bf16_rows_rel_err(y, ex) <= BF16_ROW_TOL
+
+
+def test_sync_status_clean():
+    tba.sync_status()
