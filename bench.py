@@ -504,6 +504,86 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# single-kernel cases for profiler captures (small enough for ncu's replays;
+# inputs still larger than L2)
+# ---------------------------------------------------------------------------
+PROFILE_CASES = {
+    "gemm": "tcgen05 GEMM, int8 A [16384 x 4096] x ternary int8 W [12288 x 4096]",
+    "quant_a4": "INT4 quantizer, X bf16 [32768 x 4096]",
+    "sparsify_a8": "Top-K 50% + INT8, X bf16 [32768 x 4096]",
+    "relu2_glu": "ReLU^2-GLU + Top-K 50% + INT8, gate/up bf16 [16384 x 11008]",
+    "kv_quant3": "3-bit KV, K bf16 [32768 x 32 x 128]",
+    "pack_ternary": "ternary pack to int8, W fp32 [22016 x 4096]",
+    "gemm_decode": "CUDA-core GEMM, 2-bit W [12288 x 4096], 1 token",
+}
+
+
+def run_profile_case(name: str, launches: int):
+    import torch
+
+    import ternary_bit_activation_b200 as tba
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+
+    def bf16(m, k, scale=1.0):
+        return (torch.randn((m, k), generator=g, device=dev) * scale).to(torch.bfloat16).view(torch.int16)
+
+    if name == "gemm":
+        M, N, K = 16384, 12288, 4096
+        a = torch.randint(-8, 8, (M, K), generator=g, device=dev, dtype=torch.int8)
+        w = torch.randint(-1, 2, (N, K), generator=g, device=dev, dtype=torch.int8)
+        s = torch.rand((M,), generator=g, device=dev)
+        al = torch.full((1,), 0.0173, device=dev)
+        y = torch.empty((M, N), dtype=torch.int16, device=dev)
+        fn = lambda: tba.bitlinear_gemm(a, s, w, al, M, N, K, y=y)
+    elif name == "gemm_decode":
+        M, N, K = 1, 12288, 4096
+        a = torch.randint(-8, 8, (M, K), generator=g, device=dev, dtype=torch.int8)
+        w = torch.randint(0, 256, (N, K // 4), generator=g, device=dev, dtype=torch.int32).to(torch.uint8)
+        s = torch.rand((M,), generator=g, device=dev)
+        al = torch.full((1,), 0.0173, device=dev)
+        y = torch.empty((M, N), dtype=torch.int16, device=dev)
+        fn = lambda: tba.bitlinear_gemm(a, s, w, al, M, N, K, y=y, wfmt=tba.BL_W_T2)
+    elif name == "quant_a4":
+        x = bf16(32768, 4096)
+        c = torch.empty((32768, 4096), dtype=torch.uint8, device=dev)
+        s = torch.empty((32768,), device=dev)
+        fn = lambda: tba.bitlinear_quant_a4(x, c, s, tba.BL_QUANT_INT4, tba.BL_STORE_BYTES)
+    elif name == "sparsify_a8":
+        x = bf16(32768, 4096)
+        c = torch.empty((32768, 4096), dtype=torch.int8, device=dev)
+        s = torch.empty((32768,), device=dev)
+        fn = lambda: tba.bitlinear_sparsify_a8(x, 2048, c, s, None)
+    elif name == "relu2_glu":
+        M, F = 16384, 11008
+        ug = bf16(M, 2 * F)
+        c = torch.empty((M, F), dtype=torch.int8, device=dev)
+        s = torch.empty((M,), device=dev)
+        fn = lambda: tba.relu2_glu(ug[:, F:], ug[:, :F], F // 2, c, s, None, M=M, F=F, ld=2 * F)
+    elif name == "kv_quant3":
+        T, H, D = 32768, 32, 128
+        kv = bf16(T, H * D)
+        c = torch.empty((T, H, D * 3 // 8), dtype=torch.uint8, device=dev)
+        s = torch.empty((T, H), device=dev)
+        b = torch.empty((H, D // 2), dtype=torch.uint8, device=dev)
+        fn = lambda: tba.kv_quant3(kv, T, H, D, c, s, b, bits=3, bos_pos=0)
+    elif name == "pack_ternary":
+        w = torch.randn((22016, 4096), generator=g, device=dev) * 0.02
+        o = torch.empty((22016, 4096), dtype=torch.uint8, device=dev)
+        al = torch.empty((1,), device=dev)
+        ws = torch.empty((256,), dtype=torch.int64, device=dev)
+        fn = lambda: tba.pack_ternary(w, al, o, tba.BL_W_I8, ws)
+    else:
+        raise SystemExit(f"unknown profile case {name}; one of {sorted(PROFILE_CASES)}")
+    for _ in range(launches):
+        fn()
+    tba.sync_status()
+    print(f"profile case {name}: {PROFILE_CASES[name]}, {launches} launches OK")
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -514,7 +594,12 @@ def main(argv=None):
     ap.add_argument("--cpu-tokens", type=int, default=32, help="token sample of the CPU baseline")
     ap.add_argument("--cpu-tokens-ref", type=int, default=8, help="token sample per step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), help="run one kernel's small case and exit")
+    ap.add_argument("--launches", type=int, default=3, help="launches of --profile-case")
     args = ap.parse_args(argv)
+    if args.profile_case:
+        run_profile_case(args.profile_case, args.launches)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
