@@ -135,6 +135,29 @@ BL_API bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw,
                        void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * pack_ternary_noalloc -- pack_ternary for callers that cannot allocate device
+ * memory.  The paper has no counterpart: this is an interface convenience.
+ * Some callers may not allocate at all while they run -- an inference engine
+ * that owns every byte of device memory and forbids allocation inside its
+ * execute step (plugin interfaces, fixed-budget serving loops), or a C host
+ * with no device allocator of its own.  This variant needs no workspace
+ * argument: its scratch (the 256 exponent bins of the exact |W| sum) is a
+ * 2 KiB array inside the library, one per GPU that has loaded the library,
+ * held until the process exits.  The caller still passes w, alpha and w_out.
+ * Same arguments, layouts and results as pack_ternary (alpha and codes are
+ * bit-identical); the scratch is cleared at the start of every call.
+ * Limits: N * K < 2^40, so no 64-bit bin can overflow; larger tensors are
+ * rejected with BL_ERR_SHAPE.  The first call on a device looks up the
+ * array's device address (once per device); make that first call before any
+ * stream capture.  Every call on a device shares the one array, so calls that
+ * can overlap on that GPU (different streams, no ordering between them) race
+ * and must be serialized by the caller.  Allocates nothing.
+ */
+BL_API bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int64_t ldw, float eps,
+                                      int alpha_given, float* alpha, bl_wfmt wfmt, void* w_out,
+                                      void* stream);
+
+/*
  * bitlinear_gemm -- BitLinear product with integer accumulation and the
  * per-token x per-tensor dequant epilogue.
  * Paper: §3.4, Y = Q_x(X) . Q_w(W)^T (the equation above Eq. 6, and Eq. 1).

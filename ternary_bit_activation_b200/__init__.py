@@ -26,7 +26,8 @@ BL_STORE_PACKED, BL_STORE_BYTES = 0, 1
 BL_A_I8, BL_A_I4, BL_A_E2M1 = 0, 1, 2
 BL_W_T2, BL_W_I8 = 0, 1
 
-EXPORTED = ["bitlinear_quant_a4", "bitlinear_sparsify_a8", "pack_ternary", "bitlinear_gemm", "relu2_glu",
+EXPORTED = ["bitlinear_quant_a4", "bitlinear_sparsify_a8", "pack_ternary", "pack_ternary_noalloc", "bitlinear_gemm",
+            "relu2_glu",
             "kv_quant3", "bitlinear_workspace_size", "bitlinear_sync_status", "bitlinear_status_string",
             "bitlinear_version"]
 
@@ -52,6 +53,7 @@ def lib():
             "bitlinear_quant_a4": [P, I64, I64, I64, I, I, F, P, P, P],
             "bitlinear_sparsify_a8": [P, I64, I64, I64, I64, F, P, P, P, P],
             "pack_ternary": [P, I64, I64, I64, F, I, P, I, P, P, ctypes.c_size_t, P],
+            "pack_ternary_noalloc": [P, I64, I64, I64, F, I, P, I, P, P],
             "bitlinear_gemm": [P, I, P, P, I, P, I64, I64, I64, I64, P, I64, P, P],
             "relu2_glu": [P, P, I64, I64, I64, I64, F, P, P, P, P],
             "kv_quant3": [P, I64, I64, I64, I64, I, I64, F, P, P, P, P],
@@ -113,6 +115,16 @@ def pack_ternary(w, alpha, w_out, wfmt=BL_W_T2, workspace=None, alpha_given=Fals
     ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("pack_ternary", lib().pack_ternary(_ptr(w), N, K, w.stride(0), eps, 1 if alpha_given else 0, _ptr(alpha),
                                               wfmt, _ptr(w_out), _ptr(workspace), ws, _stream(stream)))
+
+
+def pack_ternary_noalloc(w, alpha, w_out, wfmt=BL_W_T2, alpha_given=False, eps=1e-5, stream=None):
+    """pack_ternary without a workspace argument, for callers that cannot
+    allocate device memory: the scratch lives in the library (one 2 KiB array
+    per GPU).  Calls that may overlap on one GPU must be serialized."""
+    N, K = w.shape
+    _check("pack_ternary_noalloc", lib().pack_ternary_noalloc(_ptr(w), N, K, w.stride(0), eps,
+                                                              1 if alpha_given else 0, _ptr(alpha), wfmt,
+                                                              _ptr(w_out), _stream(stream)))
 
 
 def bitlinear_gemm(a, a_scale, w, alpha, M, N, K, y=None, acc=None, afmt=BL_A_I8, wfmt=BL_W_I8, alpha_group=None,

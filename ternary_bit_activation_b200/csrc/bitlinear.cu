@@ -143,9 +143,65 @@ void launch_simt(const uint8_t* a, const float* sc, const uint8_t* w, const floa
     bl::gemm_simt_kernel<AF, WT2, 8><<<grid, 256, 0, s>>>(a, sc, w, al, g, M, N, K, y, ldy, acc);
 }
 
+// Scratch of pack_ternary_noalloc: the 256 exponent bins of the exact |W|
+// sum, one array per device that loads the library.  Host code only ever uses
+// the device address looked up below, never the symbol itself.
+static __device__ __align__(256) unsigned long long g_noalloc_bins[256];
+constexpr int64_t kNoallocMaxElems = int64_t(1) << 40;  // keeps every 64-bit bin below overflow
+
+// Device address of g_noalloc_bins on the current device, looked up once per
+// device (with that device current) and cached.
+unsigned long long* noalloc_bins_ptr() {
+  static unsigned long long* cached[kMaxDevices] = {nullptr};
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return nullptr;
+  if (cached[d] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_bins) != cudaSuccess) return nullptr;
+    cached[d] = static_cast<unsigned long long*>(p);
+  }
+  return cached[d];
+}
+
 }  // namespace
 
 extern "C" {
+
+bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int64_t ldw, float eps, int alpha_given,
+                               float* alpha, bl_wfmt wfmt, void* w_out, void* stream) {
+  if (wfmt != BL_W_T2 && wfmt != BL_W_I8) return BL_ERR_ARG;
+  if (N < 0 || K < 16 || (K & 15) || ldw < K || (ldw & 3) || K > 0x7FFFFFFF) return BL_ERR_SHAPE;
+  if (N > 0 && N * K >= kNoallocMaxElems) return BL_ERR_SHAPE;
+  if (!(eps >= 0.f)) return BL_ERR_ARG;
+  if (N == 0) return BL_OK;
+  if (w == nullptr || alpha == nullptr || w_out == nullptr) return BL_ERR_NULL;
+  if (!aligned16(w) || !aligned16(w_out) || (reinterpret_cast<uintptr_t>(alpha) & 3u)) return BL_ERR_ALIGN;
+  cudaStream_t s = as_stream(stream);
+  const int k = static_cast<int>(K);
+  if (!alpha_given) {
+    unsigned long long* bins = noalloc_bins_ptr();
+    if (bins == nullptr) return BL_ERR_CUDA;
+    if (cudaMemsetAsync(bins, 0, sizeof(g_noalloc_bins), s) != cudaSuccess) return BL_ERR_CUDA;
+    const int64_t total = N * (K / 4);
+    int64_t blocks = (total + bl::kBinThreads - 1) / bl::kBinThreads;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    if (blocks > cap) blocks = cap;
+    bl::ternary_bins_kernel<<<static_cast<unsigned>(blocks), bl::kBinThreads, 0, s>>>(w, N, k, ldw, bins);
+    if (launch_status() != BL_OK) return BL_ERR_CUDA;
+    bl::ternary_alpha_kernel<<<1, 32, 0, s>>>(bins, static_cast<unsigned long long>(N * K), alpha);
+    if (launch_status() != BL_OK) return BL_ERR_CUDA;
+  }
+  const int64_t total16 = N * (K / 16);
+  int64_t blocks = (total16 + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+  if (blocks > cap) blocks = cap;
+  uint8_t* out = static_cast<uint8_t*>(w_out);
+  if (wfmt == BL_W_T2)
+    bl::ternary_pack_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+  else
+    bl::ternary_pack_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+  return launch_status();
+}
 
 const char* bitlinear_version(void) { return "libbitlinear 0.1 (sm_100a)"; }
 

@@ -108,6 +108,10 @@ def test_pack_and_kv_validation(L):
     assert pk(P(A16), 8, 64, 64, 1e-5, 0, P(A16), 0, P(A16), P(A16), 1024, None) == 8   # workspace too small
     assert pk(P(A16), 8, 64, 64, 1e-5, 0, P(A16), 0, P(A16), None, 0, None) == 1
     assert pk(P(A16), 8, 64, 64, 1e-5, 0, P(A16), 5, P(A16), P(A16), 2048, None) == 4
+    pn = L.pack_ternary_noalloc
+    assert pn(P(A16), 1 << 21, 1 << 19, 1 << 19, 1e-5, 0, P(A16), 0, P(A16), None) == 3   # N*K >= 2^40
+    assert pn(P(A16), 8, 24, 24, 1e-5, 0, P(A16), 0, P(A16), None) == 3                   # K % 16
+    assert pn(P(A16), 8, 64, 64, 1e-5, 0, None, 0, P(A16), None) == 1
     kv = L.kv_quant3
     assert kv(P(A16), 8, 4, 100, 400, 3, 0, 1e-5, P(A16), P(A16), P(A16), None) == 3     # D % 32
     assert kv(P(A16), 8, 4, 128, 512, 5, 0, 1e-5, P(A16), P(A16), P(A16), None) == 4     # bits
