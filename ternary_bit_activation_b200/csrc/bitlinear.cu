@@ -88,6 +88,9 @@ bool tc_kernel_ready() {
     if (cudaFuncSetAttribute(bl::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(bl::kTcSmemBytes)) != cudaSuccess)
       return false;
+    if (cudaFuncSetAttribute(bl::gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bl::kT2SmemBytes)) != cudaSuccess)
+      return false;
     done[d] = true;
   }
   return true;
@@ -143,11 +146,11 @@ void launch_simt(const uint8_t* a, const float* sc, const uint8_t* w, const floa
     bl::gemm_simt_kernel<AF, WT2, 8><<<grid, 256, 0, s>>>(a, sc, w, al, g, M, N, K, y, ldy, acc);
 }
 
-// Scratch of pack_ternary_noalloc: the 256 exponent bins of the exact |W|
-// sum, one array per device that loads the library.  Host code only ever uses
-// the device address looked up below, never the symbol itself.
-static __device__ __align__(256) unsigned long long g_noalloc_bins[256];
-constexpr int64_t kNoallocMaxElems = int64_t(1) << 40;  // keeps every 64-bit bin below overflow
+// Scratch of pack_ternary_noalloc: the exponent bins of the exact |W| sum, one
+// array per device that loads the library.  Host code only ever uses the device
+// address looked up below, never the symbol itself.
+static __device__ __align__(256) unsigned long long g_noalloc_bins[bl::kBins];
+constexpr int64_t kNoallocMaxElems = bl::kMaxPackElems;  // keeps every 64-bit bin below overflow
 
 // Device address of g_noalloc_bins on the current device, looked up once per
 // device (with that device current) and cached.
@@ -222,7 +225,7 @@ const char* bitlinear_status_string(bl_status st) {
 
 size_t bitlinear_workspace_size(const char* op, int64_t M, int64_t N, int64_t K) {
   (void)M; (void)N; (void)K;
-  if (op != nullptr && strcmp(op, "pack_ternary") == 0) return 256 * sizeof(unsigned long long);
+  if (op != nullptr && strcmp(op, "pack_ternary") == 0) return bl::kBins * sizeof(unsigned long long);
   return 0;
 }
 
@@ -320,7 +323,7 @@ bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float 
                        bl_wfmt wfmt, void* w_out, void* workspace, size_t ws_bytes, void* stream) {
   if (wfmt != BL_W_T2 && wfmt != BL_W_I8) return BL_ERR_ARG;
   if (N < 0 || K < 16 || (K & 15) || ldw < K || (ldw & 3)) return BL_ERR_SHAPE;
-  if (N > 0 && (N * K >= (int64_t(1) << 40) || K > 0x7FFFFFFF)) return BL_ERR_SHAPE;
+  if (N > 0 && (N * K >= bl::kMaxPackElems || K > 0x7FFFFFFF)) return BL_ERR_SHAPE;
   if (!(eps >= 0.f)) return BL_ERR_ARG;
   if (N == 0) return BL_OK;
   if (w == nullptr || alpha == nullptr || w_out == nullptr) return BL_ERR_NULL;
@@ -329,10 +332,10 @@ bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float 
   const int k = static_cast<int>(K);
   if (!alpha_given) {
     if (workspace == nullptr) return BL_ERR_NULL;
-    if (ws_bytes < 256 * sizeof(unsigned long long)) return BL_ERR_WORKSPACE;
+    if (ws_bytes < bl::kBins * sizeof(unsigned long long)) return BL_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 7u) return BL_ERR_ALIGN;
     unsigned long long* bins = static_cast<unsigned long long*>(workspace);
-    if (cudaMemsetAsync(bins, 0, 256 * sizeof(unsigned long long), s) != cudaSuccess) return BL_ERR_CUDA;
+    if (cudaMemsetAsync(bins, 0, bl::kBins * sizeof(unsigned long long), s) != cudaSuccess) return BL_ERR_CUDA;
     const int64_t total = N * (K / 4);
     int64_t blocks = (total + bl::kBinThreads - 1) / bl::kBinThreads;
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
@@ -375,6 +378,31 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
   const uint8_t* W = static_cast<const uint8_t*>(w);
   uint16_t* Y = static_cast<uint16_t*>(y_bf16);
 
+  if (afmt == BL_A_I8 && wfmt == BL_W_I8 && M > bl::kTcBM) {
+    // CTA-pair kernel: 256 x 256 tiles over clusters of two CTAs
+    if (!tc_kernel_ready()) return BL_ERR_CUDA;
+    CUtensorMap ta, tb;
+    if (!make_i8_map(&ta, A, static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128, bl::kTcBK) ||
+        !make_i8_map(&tb, W, static_cast<uint64_t>(N), static_cast<uint64_t>(K), 128, bl::kTcBK))
+      return BL_ERR_CUDA;
+    bl::TcParams p;
+    p.a_scale = a_scale;
+    p.alpha = alpha;
+    p.alpha_group = alpha_group;
+    p.M = m;
+    p.N = n;
+    p.K = k;
+    p.y = Y;
+    p.ldy = ldy;
+    p.acc = acc_out;
+    p.num_m_blocks = (m + bl::kT2BM - 1) / bl::kT2BM;
+    p.num_n_blocks = (n + bl::kT2BN - 1) / bl::kT2BN;
+    p.num_tiles = p.num_m_blocks * p.num_n_blocks;
+    p.num_kb = (k + bl::kTcBK - 1) / bl::kTcBK;
+    const int pairs = p.num_tiles < sm_count() / 2 ? p.num_tiles : sm_count() / 2;
+    bl::gemm_tc2_kernel<<<2 * pairs, bl::kTcThreads, bl::kT2SmemBytes, s>>>(ta, tb, p);
+    return launch_status();
+  }
   if (afmt == BL_A_I8 && wfmt == BL_W_I8) {
     if (!tc_kernel_ready()) return BL_ERR_CUDA;
     CUtensorMap ta, tb;
@@ -431,8 +459,8 @@ bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D, int64_
   if (!aligned16(kv_bf16) || !aligned16(codes) || !aligned16(scale) || (has_bos && !aligned16(bos_codes)))
     return BL_ERR_ALIGN;
   const int tpv = static_cast<int>(D / 8);
-  const int64_t threads = T * H * tpv;
-  const unsigned grid = static_cast<unsigned>((threads + 255) / 256);
+  const int64_t groups = (T * H + bl::kKvItems - 1) / bl::kKvItems;
+  const unsigned grid = static_cast<unsigned>((groups * tpv + 255) / 256);
   const uint16_t* kv = static_cast<const uint16_t*>(kv_bf16);
   cudaStream_t s = as_stream(stream);
   const int64_t bos = has_bos ? bos_pos : -1;

@@ -273,6 +273,235 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// tcgen05 kernel on CTA pairs (cluster of 2, cta_group::2): a 256 x 256 tile
+// per pair, each CTA holding 128 rows of A and 128 rows (half the columns) of
+// B per stage, so every CTA streams half the B bytes of the 1-CTA kernel and
+// the 6-stage ring prefetches deeper in the same shared memory.  The leader
+// CTA (rank 0) issues the MMAs for both; both CTAs' TMA loads complete on the
+// leader's full barrier; every commit is sent to each CTA's barrier by its
+// cluster address; each CTA's epilogue reads its own 128 TMEM lanes and
+// releases the accumulator on the leader's barrier.
+// ---------------------------------------------------------------------------
+constexpr int kT2BM = 256;       // pair tile rows (128 per CTA)
+constexpr int kT2BN = 256;       // pair tile columns (128 B rows per CTA)
+constexpr int kT2Stages = 6;
+constexpr uint32_t kT2StageA = 128 * kTcBK;
+constexpr uint32_t kT2StageB = 128 * kTcBK;
+constexpr int kT2GroupM = 8;     // pair m-blocks per rasterisation group
+constexpr size_t kT2SmemBytes = 1024 + kT2Stages * (kT2StageA + kT2StageB) + 256;
+constexpr uint32_t kT2Idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(kT2BN) >> 3) << 17) |
+                              ((static_cast<uint32_t>(kT2BM) >> 4) << 24);
+
+__device__ __forceinline__ void t2_tile_coords(int tile, int nmb, int nnb, int& mb, int& nb) {
+  const int group = tile / (kT2GroupM * nnb);
+  const int first_m = group * kT2GroupM;
+  const int gsize = min(nmb - first_m, kT2GroupM);
+  const int in = tile - group * kT2GroupM * nnb;
+  mb = first_m + in % gsize;
+  nb = in / gsize;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kT2Stages * kT2StageA;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kT2Stages * kT2StageB);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kT2Stages;
+  uint64_t* tfull = bars + 2 * kT2Stages;
+  uint64_t* tempty = bars + 2 * kT2Stages + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kT2Stages + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kT2Stages; ++s) {
+      mbar_init(&full[s], 1);    // the leader's arrive.expect_tx; both CTAs' bytes
+      mbar_init(&empty[s], 1);   // one commit from the leader's MMA thread
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);  // 4 epilogue warps in each CTA
+    }
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTcTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();   // barriers initialised and TMEM allocated in both CTAs
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  bool aborted = false;
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs) ----------------
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int tile = pair; tile < p.num_tiles && !aborted; tile += npairs) {
+        int mb, nb;
+        t2_tile_coords(tile, p.num_m_blocks, p.num_n_blocks, mb, nb);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait_bounded(&empty[s], ph ^ 1u)) {
+            aborted = true;
+            break;
+          }
+          const uint32_t leader_full = mapa_shared(smem_u32(&full[s]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kT2StageA + kT2StageB));
+          tma_load_2d_pair(&tmA, leader_full, sA + s * kT2StageA, kb * kTcBK, mb * kT2BM + rank * 128);
+          tma_load_2d_pair(&tmB, leader_full, sB + s * kT2StageB, kb * kTcBK, nb * kT2BN + rank * 128);
+          if (++s == kT2Stages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (leader CTA, one thread) ----------------
+    if (leader && lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int local = 0;
+      for (int tile = pair; tile < p.num_tiles && !aborted; tile += npairs, ++local) {
+        const int buf = local & 1;
+        const uint32_t tph = (local >> 1) & 1;
+        if (!mbar_wait_bounded(&tempty[buf], tph ^ 1u)) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kT2BN);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait_bounded(&full[s], ph)) {
+            aborted = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * kT2StageA);
+          const uint32_t b0 = smem_u32(sB + s * kT2StageB);
+#pragma unroll
+          for (int kk = 0; kk < kTcBK / 32; ++kk) {
+            mma_i8_pair(d_tmem, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), kT2Idesc,
+                        (kb | kk) != 0 ? 1u : 0u);
+          }
+          // free stage s in both CTAs once these MMAs have read it
+          mma_commit_pair(mapa_shared(smem_u32(&empty[s]), 0));
+          mma_commit_pair(mapa_shared(smem_u32(&empty[s]), 1));
+          if (++s == kT2Stages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (aborted) break;
+        mma_commit_pair(mapa_shared(smem_u32(&tfull[buf]), 0));   // accumulator ready in both CTAs
+        mma_commit_pair(mapa_shared(smem_u32(&tfull[buf]), 1));
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2-5 of both CTAs) ----------------
+    const int quad = warp & 3;
+    int local = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs, ++local) {
+      const int buf = local & 1;
+      const uint32_t tph = (local >> 1) & 1;
+      if (!warp_wait(&tfull[buf], tph)) {
+        aborted = true;
+        break;
+      }
+      tc_fence_after();
+      int mb, nb;
+      t2_tile_coords(tile, p.num_m_blocks, p.num_n_blocks, mb, nb);
+      const int row = mb * kT2BM + static_cast<int>(rank) * 128 + quad * 32 + lane;
+      const bool row_ok = row < p.M;
+      const float rs = row_ok ? p.a_scale[row] : 0.f;
+#pragma unroll 1
+      for (int c = 0; c < kT2BN / 32; ++c) {
+        uint32_t r[32];
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                               static_cast<uint32_t>(buf * kT2BN + c * 32);
+        tmem_ld_32x32b_x32(taddr, r);
+        tmem_wait_ld();
+        const int n0 = nb * kT2BN + c * 32;
+        if (!row_ok || n0 >= p.N) continue;
+        const int64_t ga = n0 / p.alpha_group;
+        const bool one_alpha = ((n0 + 31) / p.alpha_group) == ga;
+        const float cs_uniform = __fmul_rn(rs, p.alpha[one_alpha ? ga : 0]);
+        float yv[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float cs = one_alpha ? cs_uniform
+                                     : __fmul_rn(rs, p.alpha[min(static_cast<int64_t>(n0 + j), static_cast<int64_t>(p.N - 1)) / p.alpha_group]);
+          yv[j] = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), cs);
+        }
+        const bool full_chunk = n0 + 32 <= p.N;
+        if (p.y != nullptr) {
+          uint16_t* yr = p.y + static_cast<int64_t>(row) * p.ldy + n0;
+          if (full_chunk) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 o;
+              o.x = pack_bf16x2(yv[8 * q + 0], yv[8 * q + 1]);
+              o.y = pack_bf16x2(yv[8 * q + 2], yv[8 * q + 3]);
+              o.z = pack_bf16x2(yv[8 * q + 4], yv[8 * q + 5]);
+              o.w = pack_bf16x2(yv[8 * q + 6], yv[8 * q + 7]);
+              reinterpret_cast<uint4*>(yr)[q] = o;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (n0 + j < p.N) {
+                const __nv_bfloat16 b = __float2bfloat16_rn(yv[j]);
+                yr[j] = *reinterpret_cast<const uint16_t*>(&b);
+              }
+            }
+          }
+        }
+        if (p.acc != nullptr) {
+          int32_t* ar = p.acc + static_cast<int64_t>(row) * p.N + n0;
+          if (full_chunk && (p.N & 3) == 0) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              reinterpret_cast<uint4*>(ar)[q] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n0 + j < p.N) ar[j] = static_cast<int32_t>(r[j]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
+    }
+  }
+
+  __syncthreads();
+  if (aborted) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) {
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();   // no CTA leaves while its peer may still signal its barriers
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, kTcTmemCols);
+}
+
+// ---------------------------------------------------------------------------
 // CUDA-core kernel for packed operands.  One warp per output column n (a row
 // of W); lanes split K in units of 64 codes; MT rows of A per pass share the
 // expanded weight unit.  dp4a on int8x4 words.

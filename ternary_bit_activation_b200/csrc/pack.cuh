@@ -4,9 +4,9 @@
 //
 // alpha is the exact mean rounded once to fp32.  |w| = m * 2^(max(E,1) - 150)
 // with m the 24-bit significand and E the biased exponent, so the exact sum is
-// held as one unsigned 64-bit integer per exponent (bins[E] += m); integer adds
-// are exact and order-free.  A single thread then forms
-//   Z = sum_E bins[E] << (max(E,1) - 1)          (the sum in units of 2^-149)
+// held as unsigned 64-bit integer coefficients of powers of two (bins); integer
+// adds are exact and order-free.  A single thread then forms
+//   Z = sum_e bins[e] << (e - 1)                 (the sum in units of 2^-149)
 // as a multi-word integer, divides by N*K and rounds to nearest-even fp32.
 #pragma once
 
@@ -15,54 +15,84 @@
 namespace bl {
 
 constexpr int kBinThreads = 256;
-constexpr int kBinWarps = kBinThreads / 32;
+// bins[e] is the integer coefficient of 2^(e - 150), e >= 1 (fp32 subnormals use
+// e = 1, the same scale).  A window base is at most 254 - 31, so the high half
+// of a window sum (index base + 32) still fits in 256 entries.
+constexpr int kBins = 256;
+// Each bin receives at most one 32-bit half per 128 weights (plus 24-bit
+// significands), so N*K < 2^38 keeps every 64-bit bin below overflow.
+constexpr int64_t kMaxPackElems = int64_t(1) << 38;
 
-// Per-CTA: a private bin set per warp in shared memory, merged into the 256
-// global bins with one atomic per non-empty bin.
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// Exact sum of |w| into exponent bins.  Each warp takes 128 weights at a time
+// (a float4 per lane), finds their largest exponent Ew, and adds every
+// significand shifted into a window of 32 exponents below Ew:
+//   |w| = m * 2^(e-150) = (m << (e - base)) * 2^(base-150),  base = max(Ew - 31, 1),
+// so each term is < 2^55 and the warp's 128-term sum < 2^62 is exact in 64 bits.
+// The sum goes into bins[base] (low 32 bits) and bins[base+32] (high bits).
+// Weights more than 2^31 below the group's largest go straight to their own bin.
 __global__ void __launch_bounds__(kBinThreads) ternary_bins_kernel(const float* __restrict__ w, int64_t N, int K,
                                                                    int64_t ldw,
                                                                    unsigned long long* __restrict__ gbins) {
-  __shared__ unsigned long long sb[kBinWarps][256];
-  const int warp = threadIdx.x >> 5;
+  __shared__ unsigned long long sb[kBins];
   const int lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < kBinWarps * 256; i += kBinThreads) (&sb[0][0])[i] = 0ull;
+  for (int i = threadIdx.x; i < kBins; i += kBinThreads) sb[i] = 0ull;
   __syncthreads();
   const int per_row = K >> 2;  // float4 per row
   const int64_t total = N * static_cast<int64_t>(per_row);
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * kBinThreads + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * kBinThreads) {
-    const int64_t n = i / per_row;
-    const int q = static_cast<int>(i - n * per_row);
-    const uint4 v = ld_global_nc_v4(w + n * ldw + static_cast<int64_t>(q) * 4);
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  const int64_t gwarp = (static_cast<int64_t>(blockIdx.x) * kBinThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kBinThreads) >> 5;
+  for (int64_t g = gwarp * 32; g < total; g += nwarps * 32) {   // warp-uniform trip count
+    const int64_t i = g + lane;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (i < total) {
+      const int64_t n = i / per_row;
+      const int q = static_cast<int>(i - n * per_row);
+      v = ld_global_nc_v4(w + n * ldw + static_cast<int64_t>(q) * 4);
+    }
+    const uint32_t u[4] = {v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu, v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu};
+    uint32_t e[4], m[4], emax = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t a = u[j] & 0x7FFFFFFFu;
-      const uint32_t e = a >> 23;
-      const uint32_t m = (a & 0x7FFFFFu) | (e ? 0x800000u : 0u);
-      if (m) atomicAdd(&sb[warp][e], static_cast<unsigned long long>(m));
+      const uint32_t E = u[j] >> 23;
+      m[j] = (u[j] & 0x7FFFFFu) | (E ? 0x800000u : 0u);
+      e[j] = E ? E : 1u;
+      if (m[j]) emax = max(emax, e[j]);
+    }
+    const uint32_t ew = __reduce_max_sync(0xFFFFFFFFu, emax);
+    if (ew == 0) continue;  // the whole group is zero
+    const uint32_t base = ew > 32 ? ew - 31 : 1u;
+    unsigned long long acc = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (m[j] == 0) continue;
+      if (e[j] >= base) acc += static_cast<unsigned long long>(m[j]) << (e[j] - base);
+      else atomicAdd(&sb[e[j]], static_cast<unsigned long long>(m[j]));
+    }
+    acc = warp_sum_u64(acc);
+    if (lane == 0) {
+      atomicAdd(&sb[base], acc & 0xFFFFFFFFull);
+      atomicAdd(&sb[base + 32], acc >> 32);
     }
   }
   __syncthreads();
-  for (int b = threadIdx.x; b < 256; b += kBinThreads) {
-    unsigned long long s = 0;
-#pragma unroll
-    for (int wv = 0; wv < kBinWarps; ++wv) s += sb[wv][b];
-    if (s) atomicAdd(&gbins[b], s);
-  }
-  (void)lane;
+  for (int b = threadIdx.x; b < kBins; b += kBinThreads)
+    if (sb[b]) atomicAdd(&gbins[b], sb[b]);
 }
 
 // Multi-word unsigned integer, little-endian 32-bit limbs.
-constexpr int kLimbs = 12;  // 384 bits: bins < 2^64 shifted by <= 253 bits
+constexpr int kLimbs = 12;  // 384 bits: bins < 2^64 shifted by <= 254 bits
 
 __device__ __forceinline__ void big_add_shifted(uint32_t (&z)[kLimbs], unsigned long long v, int shift) {
   const int li = shift >> 5, bo = shift & 31;
   // v << bo spans up to three limbs
-  const uint32_t p0 = static_cast<uint32_t>(v << bo);
-  const uint32_t p1 = static_cast<uint32_t>((bo ? (v >> (32 - bo)) : (v >> 32)));
-  const uint32_t p2 = static_cast<uint32_t>(bo ? (v >> (64 - bo)) : 0ull);
-  const uint32_t parts[3] = {p0, p1, p2};
+  const uint32_t parts[3] = {static_cast<uint32_t>(v << bo), static_cast<uint32_t>(bo ? (v >> (32 - bo)) : (v >> 32)),
+                             static_cast<uint32_t>(bo ? (v >> (64 - bo)) : 0ull)};
   unsigned long long carry = 0;
   for (int i = li; i < kLimbs; ++i) {
     const unsigned long long add = (i - li < 3) ? parts[i - li] : 0u;
@@ -79,8 +109,12 @@ __device__ __forceinline__ int big_bitlen(const uint32_t (&z)[kLimbs]) {
   return 0;
 }
 
+__device__ __forceinline__ uint32_t big_limb(const uint32_t (&z)[kLimbs], int i) {
+  return (i >= 0 && i < kLimbs) ? z[i] : 0u;
+}
+
 __device__ __forceinline__ uint32_t big_bit(const uint32_t (&z)[kLimbs], int b) {
-  return (b < 0 || b >= 32 * kLimbs) ? 0u : (z[b >> 5] >> (b & 31)) & 1u;
+  return (b < 0) ? 0u : (big_limb(z, b >> 5) >> (b & 31)) & 1u;
 }
 
 // Any bit set strictly below position b?
@@ -90,35 +124,48 @@ __device__ __forceinline__ bool big_any_below(const uint32_t (&z)[kLimbs], int b
   for (int i = 0; i < full && i < kLimbs; ++i)
     if (z[i]) return true;
   const int rem = b & 31;
-  return rem && full < kLimbs && (z[full] & ((1u << rem) - 1u));
+  return rem && (big_limb(z, full) & ((1u << rem) - 1u));
 }
 
-// 64-bit window of z starting at bit `sh` (sh >= 0).
+// 64-bit window of z starting at bit sh >= 0.
 __device__ __forceinline__ unsigned long long big_window64(const uint32_t (&z)[kLimbs], int sh) {
-  unsigned long long r = 0;
-  for (int j = 0; j < 64; ++j) r |= static_cast<unsigned long long>(big_bit(z, sh + j)) << j;
-  return r;
+  const int li = sh >> 5, bo = sh & 31;
+  const unsigned long long lo =
+      static_cast<unsigned long long>(big_limb(z, li)) | (static_cast<unsigned long long>(big_limb(z, li + 1)) << 32);
+  const unsigned long long hi = big_limb(z, li + 2);
+  return bo ? ((lo >> bo) | (hi << (64 - bo))) : lo;
 }
 
-// alpha = RN_fp32( (Z * 2^-149) / D ), single thread.
+// alpha = RN_fp32( (Z * 2^-149) / D ),  Z = sum_e bins[e] << (e - 1); single thread.
 __global__ void ternary_alpha_kernel(const unsigned long long* __restrict__ gbins, unsigned long long D,
                                      float* __restrict__ alpha) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   uint32_t z[kLimbs];
   for (int i = 0; i < kLimbs; ++i) z[i] = 0;
-  for (int e = 0; e < 256; ++e) {
+  for (int e = 0; e < kBins; ++e) {
     const unsigned long long b = gbins[e];
     if (b) big_add_shifted(z, b, (e > 0 ? e : 1) - 1);
   }
   // Long division Q = floor(Z / D), R = Z mod D.
   uint32_t q[kLimbs];
-  unsigned __int128 rem = 0;
-  for (int i = kLimbs - 1; i >= 0; --i) {
-    const unsigned __int128 cur = (rem << 32) | z[i];
-    q[i] = static_cast<uint32_t>(cur / D);
-    rem = cur % D;
+  unsigned long long R;
+  if (D <= 0xFFFFFFFFull) {
+    unsigned long long rem = 0;
+    for (int i = kLimbs - 1; i >= 0; --i) {
+      const unsigned long long cur = (rem << 32) | z[i];
+      q[i] = static_cast<uint32_t>(cur / D);
+      rem = cur % D;
+    }
+    R = rem;
+  } else {
+    unsigned __int128 rem = 0;
+    for (int i = kLimbs - 1; i >= 0; --i) {
+      const unsigned __int128 cur = (rem << 32) | z[i];
+      q[i] = static_cast<uint32_t>(cur / D);
+      rem = cur % D;
+    }
+    R = static_cast<unsigned long long>(rem);
   }
-  const unsigned long long R = static_cast<unsigned long long>(rem);
   const int L = big_bitlen(q);
   float result;
   if (L == 0) {

@@ -171,10 +171,13 @@ __global__ void __launch_bounds__(256) quant_a4_kernel(const uint16_t* __restric
 
 // ---------------------------------------------------------------------------
 // Top-K + INT8 (Eq. 1).  One 256-thread CTA per row; thread t holds chunks
-// c*256 + t (8 elements each) for c < CHUNKS, as fp32 values.  The keep-th
-// largest magnitude key is found by an MSD radix select over shared-memory
-// histograms; elements tied at that key are taken in index order with a
-// block-wide prefix count.
+// c*256 + t (8 elements each) for c < CHUNKS, as fp32 values.
+// Threshold search: if the row has at most `keep` nonzero magnitudes, the
+// threshold is 0 (every nonzero survives, zeros fill the rest in index order).
+// Otherwise the keep-th largest magnitude key is found by an MSD radix select
+// over the nonzero keys (zeros can no longer be the threshold), with one
+// private shared-memory histogram per warp merged by warp 0.  Elements tied
+// at the threshold key are taken in index order with a block prefix count.
 //   F32KEY = false: values came from bf16, key = 15-bit bf16 magnitude.
 //   F32KEY = true : values are fp32 (relu2_glu's h), key = 31-bit magnitude.
 // ---------------------------------------------------------------------------
@@ -182,10 +185,11 @@ constexpr int kTkThreads = 256;
 constexpr int kTkWarps = kTkThreads / 32;
 
 struct TopkSmem {
-  uint32_t hist[256];
+  uint32_t whist[kTkWarps][256];   // per-warp histograms, zero between passes
   uint32_t wmax[kTkWarps];
+  uint32_t wnz[kTkWarps];
   uint32_t sel_digit, sel_above, sel_count;
-  int32_t tie_off[8][kTkWarps];  // exclusive tie prefix per (chunk, warp)
+  int32_t tie_off[8][kTkWarps];    // exclusive tie prefix per (chunk, warp)
   int32_t tie_cnt[8][kTkWarps];
 };
 
@@ -194,16 +198,25 @@ __device__ __forceinline__ uint32_t mag_key(float v) {
   return F32KEY ? (__float_as_uint(v) & 0x7FFFFFFFu) : ((__float_as_uint(v) >> 16) & 0x7FFFu);
 }
 
-// Warp 0: find the digit d with  above(d) < r <= above(d) + hist[d], where
-// above(d) counts the candidates whose digit is greater than d.
-__device__ __forceinline__ void select_digit(TopkSmem& sm, int nbins, uint32_t r) {
+// Warp 0: merge the per-warp histograms (and zero them for the next pass),
+// then find the digit d with  above(d) < r <= above(d) + hist[d], where above(d)
+// counts the candidates whose digit is greater than d.
+__device__ __forceinline__ void merge_select_digit(TopkSmem& sm, int nbins, uint32_t r) {
   const int lane = threadIdx.x & 31;
   const int per = nbins / 32;  // 8 or 4 bins per lane
   uint32_t h[8];
   uint32_t s = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    h[i] = (i < per) ? sm.hist[lane * per + i] : 0u;
+    h[i] = 0;
+    if (i < per) {
+      const int b = lane * per + i;
+#pragma unroll
+      for (int w = 0; w < kTkWarps; ++w) {
+        h[i] += sm.whist[w][b];
+        sm.whist[w][b] = 0;
+      }
+    }
     s += h[i];
   }
   uint32_t inc = s;  // inclusive suffix sum over lanes >= lane
@@ -236,52 +249,73 @@ __device__ __forceinline__ void topk_int8_row(const float (&val)[CHUNKS][8], int
   const int warp = t >> 5;
   const int nchunk = K >> 3;
 
-  // gamma = max |x| as the largest key
-  uint32_t mk = 0;
+  // each warp clears its own histogram; the barrier below orders it
+  for (int i = lane; i < 256; i += 32) sm.whist[warp][i] = 0;
+
+  // gamma = max |x| (largest key) and the number of nonzero magnitudes
+  uint32_t mk = 0, nz = 0;
 #pragma unroll
   for (int c = 0; c < CHUNKS; ++c)
     if (c * kTkThreads + t < nchunk)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mk = max(mk, mag_key<F32KEY>(val[c][e]));
-  mk = warp_max_u32(mk);
-  if (lane == 0) sm.wmax[warp] = mk;
-
-  // MSD radix select of the keep-th largest key.
-  constexpr int kPasses = F32KEY ? 4 : 2;
-  uint32_t prefix = 0, fixed = 0, r = static_cast<uint32_t>(keep), tie_total = 0;
-#pragma unroll
-  for (int pass = 0; pass < kPasses; ++pass) {
-    const int shift = F32KEY ? (pass == 0 ? 23 : pass == 1 ? 15 : pass == 2 ? 7 : 0) : (pass == 0 ? 7 : 0);
-    const int width = (shift == 0) ? 7 : 8;
-    const uint32_t dmask = (1u << width) - 1u;
-    for (int i = t; i < 256; i += kTkThreads) sm.hist[i] = 0;
-    __syncthreads();
-#pragma unroll
-    for (int c = 0; c < CHUNKS; ++c) {
-      const bool chunk_ok = c * kTkThreads + t < nchunk;
-#pragma unroll
       for (int e = 0; e < 8; ++e) {
         const uint32_t key = mag_key<F32KEY>(val[c][e]);
-        const bool act = chunk_ok && ((key & fixed) == prefix);
-        const uint32_t am = __ballot_sync(0xFFFFFFFFu, act);
-        if (act) {
-          const uint32_t bin = (key >> shift) & dmask;
-          const uint32_t peers = __match_any_sync(am, bin);
-          if (lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], static_cast<uint32_t>(__popc(peers)));
+        mk = max(mk, key);
+        nz += key != 0u;
+      }
+  mk = warp_max_u32(mk);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) nz += __shfl_xor_sync(0xFFFFFFFFu, nz, o);
+  if (lane == 0) {
+    sm.wmax[warp] = mk;
+    sm.wnz[warp] = nz;
+  }
+  __syncthreads();
+  uint32_t gk = 0, nnz = 0;
+#pragma unroll
+  for (int w = 0; w < kTkWarps; ++w) {
+    gk = max(gk, sm.wmax[w]);
+    nnz += sm.wnz[w];
+  }
+
+  uint32_t thr, take, tie_total;
+  if (nnz <= static_cast<uint32_t>(keep)) {
+    thr = 0;                                   // every nonzero survives; zeros fill in index order
+    take = static_cast<uint32_t>(keep) - nnz;
+    tie_total = static_cast<uint32_t>(K) - nnz;
+  } else {
+    // MSD radix select of the keep-th largest nonzero key.
+    constexpr int kPasses = F32KEY ? 4 : 2;
+    uint32_t prefix = 0, fixed = 0, r = static_cast<uint32_t>(keep);
+    tie_total = 0;
+#pragma unroll
+    for (int pass = 0; pass < kPasses; ++pass) {
+      const int shift = F32KEY ? (pass == 0 ? 23 : pass == 1 ? 15 : pass == 2 ? 7 : 0) : (pass == 0 ? 7 : 0);
+      const int width = (shift == 0) ? 7 : 8;
+      const uint32_t dmask = (1u << width) - 1u;
+      uint32_t* hist = sm.whist[warp];
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) {
+        if (c * kTkThreads + t < nchunk) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t key = mag_key<F32KEY>(val[c][e]);
+            if (key != 0u && (key & fixed) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+          }
         }
       }
+      __syncthreads();
+      if (warp == 0) merge_select_digit(sm, 1 << width, r);
+      __syncthreads();
+      const uint32_t d = sm.sel_digit;
+      r -= sm.sel_above;
+      tie_total = sm.sel_count;
+      prefix |= d << shift;
+      fixed |= dmask << shift;
     }
-    __syncthreads();
-    if (warp == 0) select_digit(sm, 1 << width, r);
-    __syncthreads();
-    const uint32_t d = sm.sel_digit;
-    r -= sm.sel_above;
-    tie_total = sm.sel_count;
-    prefix |= d << shift;
-    fixed |= dmask << shift;
+    thr = prefix;   // key of the keep-th largest element
+    take = r;       // how many elements with key == thr survive (in index order)
   }
-  const uint32_t thr = prefix;   // key of the keep-th largest element
-  const uint32_t take = r;       // how many elements with key == thr survive (in index order)
 
   // Index-ordered rank among the ties, needed only when some ties are dropped.
   int tie_base[CHUNKS];
@@ -320,9 +354,6 @@ __device__ __forceinline__ void topk_int8_row(const float (&val)[CHUNKS][8], int
     for (int c = 0; c < CHUNKS; ++c) tie_base[c] = 0;
   }
 
-  uint32_t gk = 0;
-#pragma unroll
-  for (int w = 0; w < kTkWarps; ++w) gk = max(gk, sm.wmax[w]);
   const float gamma = F32KEY ? __uint_as_float(gk) : __uint_as_float(gk << 16);
   const float mult = __fdiv_rn(127.f, __fadd_rn(gamma, eps));
   if (t == 0) scale[row] = __fdiv_rn(gamma, 127.f);
