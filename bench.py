@@ -183,7 +183,10 @@ class Layer:
         x_attn, x_o, x_ffn = synth.layer_activations(SHAPE, seed=seed, tokens=m)
         self.h_in = [T.from_numpy(a.view(np.int16)).pin_memory() for a in (x_attn, x_o, x_ffn)]
         del x_attn, x_o, x_ffn
-        self.x = [h.to(dev) for h in self.h_in]
+        # two device sets of the step's inputs and outputs, so the end-to-end
+        # leg can copy one step's data while another step computes
+        self.x_sets = [[h.to(dev) for h in self.h_in] for _ in range(2)]
+        self.x = self.x_sets[0]
 
         qbytes = 1  # BL_STORE_BYTES: one int8 per element for the tensor-core operand
         self.qa = T.empty((m, d * qbytes), dtype=u8, device=dev)
@@ -195,13 +198,15 @@ class Layer:
         self.h8 = T.empty((m, f), dtype=i8, device=dev)
         self.h8_s = T.empty((m,), dtype=f32, device=dev)
         self.y_qkv = T.empty((m, 3 * d), dtype=i16, device=dev)
-        self.y_o = T.empty((m, d), dtype=i16, device=dev)
         self.y_ug = T.empty((m, 2 * f), dtype=i16, device=dev)
-        self.y_down = T.empty((m, d), dtype=i16, device=dev)
-        self.kv_codes = T.empty((2, m, H, Dh * 3 // 8), dtype=u8, device=dev)
-        self.kv_scale = T.empty((2, m, H), dtype=f32, device=dev)
-        self.kv_bos = T.empty((2, H, Dh // 2), dtype=u8, device=dev)
-        self.outputs = [self.y_o, self.y_down, self.kv_codes, self.kv_scale, self.kv_bos]
+        self.out_sets = []
+        for _ in range(2):
+            self.out_sets.append([T.empty((m, d), dtype=i16, device=dev),                 # O projection output
+                                  T.empty((m, d), dtype=i16, device=dev),                 # down projection output
+                                  T.empty((2, m, H, Dh * 3 // 8), dtype=u8, device=dev),  # 3-bit K and V codes
+                                  T.empty((2, m, H), dtype=f32, device=dev),              # their scales
+                                  T.empty((2, H, Dh // 2), dtype=u8, device=dev)])        # 4-bit BOS rows
+        self.use_set(0)
         self.h_out = [T.empty(o.shape, dtype=o.dtype).pin_memory() for o in self.outputs]
 
         # algorithmic work per step
@@ -272,6 +277,12 @@ class Layer:
         timed("gemm_down", lambda: tba.bitlinear_gemm(self.h8, self.h8_s, w8["down"], al[4:5], m, d, f,
                                                       y=self.y_down))
 
+    def use_set(self, i: int):
+        """Point the step at input/output buffer set i."""
+        self.x = self.x_sets[i]
+        self.outputs = self.out_sets[i]
+        self.y_o, self.y_down, self.kv_codes, self.kv_scale, self.kv_bos = self.outputs
+
     def h2d(self):
         for h, dv in zip(self.h_in, self.x):
             dv.copy_(h, non_blocking=True)
@@ -279,6 +290,48 @@ class Layer:
     def d2h(self):
         for o, h in zip(self.outputs, self.h_out):
             h.copy_(o, non_blocking=True)
+
+    def run_e2e(self, steps: int):
+        """`steps` end-to-end steps: per step, H2D of the inputs from pinned host
+        memory, the step, D2H of the outputs.  Copies run on their own streams
+        and overlap the neighbouring steps' compute; buffer sets alternate, and
+        events keep each set's copy-in, compute and copy-out in order.
+        Returns (start_event, end_event)."""
+        T = self.torch
+        comp = T.cuda.current_stream()
+        s_in = T.cuda.Stream()
+        s_out = T.cuda.Stream()
+        ev = lambda: T.cuda.Event()
+        inputs_free = [ev(), ev()]     # compute finished reading set i's inputs
+        inputs_ready = [ev(), ev()]
+        outputs_ready = [ev(), ev()]
+        outputs_free = [ev(), ev()]    # set i's outputs copied out
+        start = T.cuda.Event(enable_timing=True)
+        end = T.cuda.Event(enable_timing=True)
+        for e in inputs_free + outputs_free:
+            e.record(comp)
+        start.record(comp)
+        s_in.wait_event(start)
+        for i in range(steps):
+            p = i & 1
+            self.use_set(p)
+            with T.cuda.stream(s_in):
+                s_in.wait_event(inputs_free[p])
+                self.h2d()
+                inputs_ready[p].record(s_in)
+            comp.wait_event(inputs_ready[p])
+            comp.wait_event(outputs_free[p])
+            self.step()
+            inputs_free[p].record(comp)
+            outputs_ready[p].record(comp)
+            with T.cuda.stream(s_out):
+                s_out.wait_event(outputs_ready[p])
+                self.d2h()
+                outputs_free[p].record(s_out)
+        comp.wait_stream(s_out)
+        end.record(comp)
+        self.use_set(0)
+        return start, end
 
     def io_bytes(self):
         return (sum(h.numel() * h.element_size() for h in self.h_in),
@@ -337,19 +390,11 @@ def run_gpu(args):
     for name, a, b in events:
         per_kernel.setdefault(name, []).append(a.elapsed_time(b))
 
-    # end to end through the C ABI with host buffers: H2D of the step's inputs,
-    # the step, D2H of its outputs -- every step
-    for _ in range(max(1, args.warmup // 2)):
-        layer.h2d(); layer.step(); layer.d2h()
+    # end to end through the C ABI with host buffers: every step copies its
+    # inputs in from pinned host memory and its outputs back out
+    layer.run_e2e(max(2, args.warmup))
     barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        layer.h2d()
-        layer.step()
-        layer.d2h()
-    e1.record()
+    e0, e1 = layer.run_e2e(args.steps)
     barrier()
     e2e_ms = e0.elapsed_time(e1)
 
@@ -505,6 +550,121 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+# decode: the same layer for a few tokens at a time; 2-bit weights packed once
+# (inference), activations INT4-packed / Top-K INT8, CUDA-core GEMM kernel
+# ---------------------------------------------------------------------------
+def run_decode(args):
+    import torch
+
+    import ternary_bit_activation_b200 as tba
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    s = SHAPE
+    d, f = s.hidden, s.ffn
+    T = torch
+    wts = synth.layer_weights(s, seed=3)
+    shapes = {"qkv": (3 * d, d), "o": (d, d), "upgate": (2 * f, d), "down": (d, f)}
+    w2 = {k: T.empty((n, kk // 4), dtype=T.uint8, device=dev) for k, (n, kk) in shapes.items()}
+    alpha = T.zeros((8,), dtype=T.float32, device=dev)
+    ws = T.empty((tba.workspace_size("pack_ternary") // 8,), dtype=T.int64, device=dev)
+    for key, dst, ai in (("qkv", w2["qkv"], 0), ("o", w2["o"], 1), ("up", w2["upgate"][:f], 2),
+                         ("gate", w2["upgate"][f:], 3), ("down", w2["down"], 4)):
+        tba.pack_ternary(T.from_numpy(wts[key]).to(dev), alpha[ai:ai + 1], dst, tba.BL_W_T2, ws)
+    del wts
+    weight_bytes = sum(n * kk // 4 for n, kk in shapes.values())
+    results = []
+    for m in args.decode_tokens:
+        x_attn, x_o, x_ffn = [T.from_numpy(a.view(np.int16)).to(dev)
+                              for a in synth.layer_activations(s, seed=500 + m, tokens=m)]
+        qa = T.empty((m, d // 2), dtype=T.uint8, device=dev)
+        qa_s = T.empty((m,), dtype=T.float32, device=dev)
+        o8 = T.empty((m, d), dtype=T.int8, device=dev)
+        o8_s = T.empty((m,), dtype=T.float32, device=dev)
+        h8 = T.empty((m, f), dtype=T.int8, device=dev)
+        h8_s = T.empty((m,), dtype=T.float32, device=dev)
+        y_qkv = T.empty((m, 3 * d), dtype=T.int16, device=dev)
+        y_o = T.empty((m, d), dtype=T.int16, device=dev)
+        y_ug = T.empty((m, 2 * f), dtype=T.int16, device=dev)
+        y_down = T.empty((m, d), dtype=T.int16, device=dev)
+        gemm_ev = []
+
+        def step(record=False):
+            def g(fn):
+                if not record:
+                    fn()
+                    return
+                a_, b_ = T.cuda.Event(enable_timing=True), T.cuda.Event(enable_timing=True)
+                a_.record(); fn(); b_.record()
+                gemm_ev.append((a_, b_))
+            tba.bitlinear_quant_a4(x_attn, qa, qa_s, tba.BL_QUANT_INT4, tba.BL_STORE_PACKED, EPS)
+            g(lambda: tba.bitlinear_gemm(qa, qa_s, w2["qkv"], alpha[0:1], m, 3 * d, d, y=y_qkv,
+                                         afmt=tba.BL_A_I4, wfmt=tba.BL_W_T2))
+            tba.bitlinear_sparsify_a8(x_o, synth.k_keep(d, s.topk_pct_o), o8, o8_s, None, EPS)
+            g(lambda: tba.bitlinear_gemm(o8, o8_s, w2["o"], alpha[1:2], m, d, d, y=y_o, wfmt=tba.BL_W_T2))
+            tba.bitlinear_quant_a4(x_ffn, qa, qa_s, tba.BL_QUANT_INT4, tba.BL_STORE_PACKED, EPS)
+            g(lambda: tba.bitlinear_gemm(qa, qa_s, w2["upgate"], alpha[2:4], m, 2 * f, d, y=y_ug,
+                                         afmt=tba.BL_A_I4, wfmt=tba.BL_W_T2, alpha_group=f))
+            tba.relu2_glu(y_ug[:, f:], y_ug[:, :f], synth.k_keep(f, s.topk_pct_down), h8, h8_s, None, EPS,
+                          M=m, F=f, ld=2 * f)
+            g(lambda: tba.bitlinear_gemm(h8, h8_s, w2["down"], alpha[4:5], m, d, f, y=y_down, wfmt=tba.BL_W_T2))
+
+        for _ in range(args.warmup):
+            step()
+        tba.sync_status()
+        torch.cuda.synchronize()
+
+        # decode launches are a few microseconds each: capture one step (and
+        # its four GEMMs alone) in CUDA graphs and time graph replays
+        def capture(fn):
+            side = T.cuda.Stream()
+            side.wait_stream(T.cuda.current_stream())
+            with T.cuda.stream(side):
+                fn()
+            T.cuda.current_stream().wait_stream(side)
+            graph = T.cuda.CUDAGraph()
+            with T.cuda.graph(graph):
+                fn()
+            return graph
+
+        def gemms_only():
+            tba.bitlinear_gemm(qa, qa_s, w2["qkv"], alpha[0:1], m, 3 * d, d, y=y_qkv, afmt=tba.BL_A_I4,
+                               wfmt=tba.BL_W_T2)
+            tba.bitlinear_gemm(o8, o8_s, w2["o"], alpha[1:2], m, d, d, y=y_o, wfmt=tba.BL_W_T2)
+            tba.bitlinear_gemm(qa, qa_s, w2["upgate"], alpha[2:4], m, 2 * f, d, y=y_ug, afmt=tba.BL_A_I4,
+                               wfmt=tba.BL_W_T2, alpha_group=f)
+            tba.bitlinear_gemm(h8, h8_s, w2["down"], alpha[4:5], m, d, f, y=y_down, wfmt=tba.BL_W_T2)
+
+        g_step = capture(step)
+        g_gemm = capture(gemms_only)
+
+        def time_graph(graph):
+            for _ in range(3):
+                graph.replay()
+            torch.cuda.synchronize()
+            a_, b_ = T.cuda.Event(enable_timing=True), T.cuda.Event(enable_timing=True)
+            a_.record()
+            for _ in range(args.steps):
+                graph.replay()
+            b_.record()
+            torch.cuda.synchronize()
+            return a_.elapsed_time(b_) / args.steps
+
+        ms = time_graph(g_step)
+        gemm_ms = time_graph(g_gemm)
+        tba.sync_status()
+        del g_step, g_gemm
+        results.append({"tokens": m, "ms_per_layer": round(ms, 4), "tokens_per_s": round(m / (ms / 1e3), 1),
+                        "gemm_ms": round(gemm_ms, 4),
+                        "weight_stream_gbs": round(weight_bytes / (gemm_ms / 1e3) / 1e9, 1),
+                        "hbm_frac": round(weight_bytes / (gemm_ms / 1e3) / 1e9 / load_peaks()["hbm_gbs"], 3)})
+    line = {"metric": "decode BitLinear layer latency (7B shapes, 2-bit weights; CUDA-graph replay)",
+            "unit": "ms per layer",
+            "workload": "7B-shape layer, decode of M tokens against all four BitLinear matrices",
+            "weight_bytes": weight_bytes, "steps": args.steps, "warmup": args.warmup, "results": results}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
 # single-kernel cases for profiler captures (small enough for ncu's replays;
 # inputs still larger than L2)
 # ---------------------------------------------------------------------------
@@ -594,6 +754,9 @@ def main(argv=None):
     ap.add_argument("--cpu-tokens", type=int, default=32, help="token sample of the CPU baseline")
     ap.add_argument("--cpu-tokens-ref", type=int, default=8, help="token sample per step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["prefill", "decode"], default="prefill",
+                    help="prefill: the headline step; decode: per-token-batch latency sweep")
+    ap.add_argument("--decode-tokens", type=int, nargs="+", default=synth.DECODE_TOKENS)
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), help="run one kernel's small case and exit")
     ap.add_argument("--launches", type=int, default=3, help="launches of --profile-case")
     args = ap.parse_args(argv)
@@ -604,6 +767,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "decode":
+        run_decode(args)
     else:
         run_gpu(args)
 

@@ -119,8 +119,25 @@ void launch_sparsify_c(const uint16_t* x, int64_t M, int K, int64_t ldx, int kee
 template <int C>
 void launch_relu2_c(const uint16_t* g, const uint16_t* u, int64_t M, int F, int64_t ld, int keep, float eps,
                     int8_t* codes, float* scale, uint32_t* mask, cudaStream_t s) {
-  bl::relu2_glu_kernel<C><<<static_cast<unsigned>(M), bl::kTkThreads, 0, s>>>(g, u, F, ld, keep, eps, codes, scale,
-                                                                                mask);
+  // persistent: as many CTAs as fit (registers and the row buffer), rows strided over them
+  const size_t smem = 2 * static_cast<size_t>(C) * bl::kTkThreads * sizeof(uint4);
+  auto kern = bl::relu2_glu_persistent_kernel<C>;
+  // opt-in shared-memory limit and resident CTAs per SM, looked up once per device
+  static int per_sm_cache[kMaxDevices] = {};
+  const int d = current_device();
+  int per_sm = 1;
+  if (d >= 0 && d < kMaxDevices) {
+    if (per_sm_cache[d] == 0) {
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      int n = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, bl::kTkThreads, smem) != cudaSuccess || n < 1) n = 1;
+      per_sm_cache[d] = n;
+    }
+    per_sm = per_sm_cache[d];
+  }
+  const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
+  const unsigned grid = static_cast<unsigned>(M < cap ? M : cap);
+  kern<<<grid, bl::kTkThreads, smem, s>>>(g, u, M, F, ld, keep, eps, codes, scale, mask);
 }
 
 bool topk_chunks(int64_t K, int* chunks) {
@@ -130,20 +147,51 @@ bool topk_chunks(int64_t K, int* chunks) {
   return true;
 }
 
-template <int AF, bool WT2>
-void launch_simt(const uint8_t* a, const float* sc, const uint8_t* w, const float* al, int64_t g, int M, int N,
-                 int K, uint16_t* y, int64_t ldy, int32_t* acc, cudaStream_t s) {
-  const int64_t blocks_needed = (static_cast<int64_t>(N) + 7) / 8;
-  const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+template <int AF, bool WT2, int MT, int UPL>
+bool launch_simt_mu(const uint8_t* a, const float* sc, const uint8_t* w, const float* al, int64_t g, int M, int N,
+                    int K, uint16_t* y, int64_t ldy, int32_t* acc, cudaStream_t s) {
+  constexpr int R = bl::SimtShape<WT2, UPL>::R;
+  const int units_hi = ((K >> 6) + 31) >> 5;
+  const size_t smem = static_cast<size_t>(MT) * units_hi * 32 * 16 * sizeof(uint32_t);
+  auto kern = bl::gemm_simt_kernel<AF, WT2, MT, UPL>;
+  // the largest tile (K up to 2^20) needs the opt-in shared-memory limit; set it once per device
+  static bool attr_done[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return false;
+  if (!attr_done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+      return false;
+    attr_done[dev] = true;
+  }
+  if (smem > 227 * 1024) return false;
+  const int64_t warps_needed = (static_cast<int64_t>(N) + R - 1) / R;
+  const int64_t blocks_needed = (warps_needed + 7) / 8;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   const unsigned grid = static_cast<unsigned>(blocks_needed < cap ? blocks_needed : cap);
-  if (M <= 1)
-    bl::gemm_simt_kernel<AF, WT2, 1><<<grid, 256, 0, s>>>(a, sc, w, al, g, M, N, K, y, ldy, acc);
-  else if (M <= 2)
-    bl::gemm_simt_kernel<AF, WT2, 2><<<grid, 256, 0, s>>>(a, sc, w, al, g, M, N, K, y, ldy, acc);
-  else if (M <= 4)
-    bl::gemm_simt_kernel<AF, WT2, 4><<<grid, 256, 0, s>>>(a, sc, w, al, g, M, N, K, y, ldy, acc);
-  else
-    bl::gemm_simt_kernel<AF, WT2, 8><<<grid, 256, 0, s>>>(a, sc, w, al, g, M, N, K, y, ldy, acc);
+  kern<<<grid, 256, smem, s>>>(a, sc, w, al, g, M, N, K, y, ldy, acc);
+  return true;
+}
+
+// Units per lane per round (UPL, a power of two up to 8 for 2-bit weights and
+// up to 2 for int8 weights): enough to cover K in one round where possible.
+template <int AF, bool WT2, int MT>
+bool launch_simt_m(const uint8_t* a, const float* sc, const uint8_t* w, const float* al, int64_t g, int M, int N,
+                   int K, uint16_t* y, int64_t ldy, int32_t* acc, cudaStream_t s) {
+  const int per_lane = ((K >> 6) + 31) >> 5;
+  if (per_lane <= 1) return launch_simt_mu<AF, WT2, MT, 1>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
+  if (per_lane <= 2 || !WT2) return launch_simt_mu<AF, WT2, MT, 2>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
+  if (per_lane <= 4) return launch_simt_mu<AF, WT2, MT, 4>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
+  return launch_simt_mu<AF, WT2, MT, 8>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
+}
+
+// Rows of A per staged tile (MT): up to 8 tokens share each streamed weight unit.
+template <int AF, bool WT2>
+bool launch_simt(const uint8_t* a, const float* sc, const uint8_t* w, const float* al, int64_t g, int M, int N,
+                 int K, uint16_t* y, int64_t ldy, int32_t* acc, cudaStream_t s) {
+  if (M <= 1) return launch_simt_m<AF, WT2, 1>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
+  if (M <= 2) return launch_simt_m<AF, WT2, 2>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
+  if (M <= 4) return launch_simt_m<AF, WT2, 4>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
+  return launch_simt_m<AF, WT2, 8>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
 }
 
 // Scratch of pack_ternary_noalloc: the exponent bins of the exact |W| sum, one
@@ -191,7 +239,7 @@ bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int64_t ldw
     if (blocks > cap) blocks = cap;
     bl::ternary_bins_kernel<<<static_cast<unsigned>(blocks), bl::kBinThreads, 0, s>>>(w, N, k, ldw, bins);
     if (launch_status() != BL_OK) return BL_ERR_CUDA;
-    bl::ternary_alpha_kernel<<<1, 32, 0, s>>>(bins, static_cast<unsigned long long>(N * K), alpha);
+    bl::ternary_alpha_kernel<<<1, bl::kBins, 0, s>>>(bins, static_cast<unsigned long long>(N * K), alpha);
     if (launch_status() != BL_OK) return BL_ERR_CUDA;
   }
   const int64_t total16 = N * (K / 16);
@@ -342,7 +390,7 @@ bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float 
     if (blocks > cap) blocks = cap;
     bl::ternary_bins_kernel<<<static_cast<unsigned>(blocks), bl::kBinThreads, 0, s>>>(w, N, k, ldw, bins);
     if (launch_status() != BL_OK) return BL_ERR_CUDA;
-    bl::ternary_alpha_kernel<<<1, 32, 0, s>>>(bins, static_cast<unsigned long long>(N * K), alpha);
+    bl::ternary_alpha_kernel<<<1, bl::kBins, 0, s>>>(bins, static_cast<unsigned long long>(N * K), alpha);
     if (launch_status() != BL_OK) return BL_ERR_CUDA;
   }
   const int64_t total16 = N * (K / 16);
@@ -362,7 +410,7 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
                          int64_t ldy, int32_t* acc_out, void* stream) {
   if (afmt != BL_A_I8 && afmt != BL_A_I4 && afmt != BL_A_E2M1) return BL_ERR_ARG;
   if (wfmt != BL_W_T2 && wfmt != BL_W_I8) return BL_ERR_ARG;
-  if (alpha_group < 1) return BL_ERR_ARG;
+  if (alpha_group < 1 || alpha_group > 0x7FFFFFFFLL) return BL_ERR_ARG;
   if (M < 0 || N < 1 || K < 64 || (K & 63) || K > (1 << 20) || M > 0x7FFFFFFFLL || N > 0x7FFFFFFFLL)
     return BL_ERR_SHAPE;
   if (y_bf16 != nullptr && (ldy < N || (ldy & 7))) return BL_ERR_SHAPE;
@@ -400,7 +448,7 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
     p.num_tiles = p.num_m_blocks * p.num_n_blocks;
     p.num_kb = (k + bl::kTcBK - 1) / bl::kTcBK;
     const int pairs = p.num_tiles < sm_count() / 2 ? p.num_tiles : sm_count() / 2;
-    bl::gemm_tc2_kernel<<<2 * pairs, bl::kTcThreads, bl::kT2SmemBytes, s>>>(ta, tb, p);
+    bl::gemm_tc2_kernel<<<2 * pairs, bl::kT2Threads, bl::kT2SmemBytes, s>>>(ta, tb, p);
     return launch_status();
   }
   if (afmt == BL_A_I8 && wfmt == BL_W_I8) {
@@ -428,20 +476,22 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
     return launch_status();
   }
   const bool t2 = wfmt == BL_W_T2;
+  bool ok;
   switch (afmt) {
     case BL_A_I8:
-      if (t2) launch_simt<bl::kSimtA_I8, true>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
-      else launch_simt<bl::kSimtA_I8, false>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+      ok = t2 ? launch_simt<bl::kSimtA_I8, true>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s)
+              : launch_simt<bl::kSimtA_I8, false>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
       break;
     case BL_A_I4:
-      if (t2) launch_simt<bl::kSimtA_I4, true>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
-      else launch_simt<bl::kSimtA_I4, false>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+      ok = t2 ? launch_simt<bl::kSimtA_I4, true>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s)
+              : launch_simt<bl::kSimtA_I4, false>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
       break;
     default:
-      if (t2) launch_simt<bl::kSimtA_E2M1, true>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
-      else launch_simt<bl::kSimtA_E2M1, false>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+      ok = t2 ? launch_simt<bl::kSimtA_E2M1, true>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s)
+              : launch_simt<bl::kSimtA_E2M1, false>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
       break;
   }
+  if (!ok) return BL_ERR_CUDA;
   return launch_status();
 }
 
@@ -451,7 +501,7 @@ bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D, int64_
   if (T < 0 || H < 1 || D < 32 || D > 256 || (D & 31) || ldt < H * D || (ldt & 7)) return BL_ERR_SHAPE;
   if (bos_pos < -1) return BL_ERR_ARG;
   if (!(eps >= 0.f)) return BL_ERR_ARG;
-  if (T * H * (D / 8) > (int64_t(1) << 40) || H > 0x7FFFFFFF) return BL_ERR_SHAPE;
+  if (T * H > 0x7FFFFFFFLL / 4 || H > 0x7FFFFFFF) return BL_ERR_SHAPE;   // 32-bit vector indices in the kernel
   if (T == 0) return BL_OK;
   const bool has_bos = bits == 3 && bos_pos >= 0 && bos_pos < T;
   if (kv_bf16 == nullptr || codes == nullptr || scale == nullptr || (has_bos && bos_codes == nullptr))

@@ -287,7 +287,7 @@ constexpr int kT2BN = 256;       // pair tile columns (128 B rows per CTA)
 constexpr int kT2Stages = 6;
 constexpr uint32_t kT2StageA = 128 * kTcBK;
 constexpr uint32_t kT2StageB = 128 * kTcBK;
-constexpr int kT2GroupM = 8;     // pair m-blocks per rasterisation group
+constexpr int kT2GroupM = 16;    // pair m-blocks per rasterisation group (4096 rows of A share each B tile)
 constexpr size_t kT2SmemBytes = 1024 + kT2Stages * (kT2StageA + kT2StageB) + 256;
 constexpr uint32_t kT2Idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(kT2BN) >> 3) << 17) |
                               ((static_cast<uint32_t>(kT2BM) >> 4) << 24);
@@ -301,7 +301,58 @@ __device__ __forceinline__ void t2_tile_coords(int tile, int nmb, int nnb, int& 
   nb = in / gsize;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
+// One row's 32 consecutive accumulators -> y (bf16, scaled) and/or acc (int32).
+__device__ __forceinline__ void epilogue_chunk(const TcParams& p, int row, int n0, float rs, const uint32_t (&r)[32]) {
+  const int group = static_cast<int>(p.alpha_group);   // host keeps alpha_group < 2^31
+  const int ga = n0 / group;
+  const bool one_alpha = (n0 + 31) / group == ga;
+  const float cs_uniform = __fmul_rn(rs, p.alpha[ga]);
+  float yv[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float cs = one_alpha ? cs_uniform : __fmul_rn(rs, p.alpha[min(n0 + j, p.N - 1) / group]);
+    yv[j] = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), cs);
+  }
+  const bool full_chunk = n0 + 32 <= p.N;
+  if (p.y != nullptr) {
+    uint16_t* yr = p.y + static_cast<int64_t>(row) * p.ldy + n0;
+    if (full_chunk) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 o;
+        o.x = pack_bf16x2(yv[8 * q + 0], yv[8 * q + 1]);
+        o.y = pack_bf16x2(yv[8 * q + 2], yv[8 * q + 3]);
+        o.z = pack_bf16x2(yv[8 * q + 4], yv[8 * q + 5]);
+        o.w = pack_bf16x2(yv[8 * q + 6], yv[8 * q + 7]);
+        st_global_stream_v4(reinterpret_cast<uint4*>(yr) + q, o);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (n0 + j < p.N) {
+          const __nv_bfloat16 b = __float2bfloat16_rn(yv[j]);
+          yr[j] = *reinterpret_cast<const uint16_t*>(&b);
+        }
+      }
+    }
+  }
+  if (p.acc != nullptr) {
+    int32_t* ar = p.acc + static_cast<int64_t>(row) * p.N + n0;
+    if (full_chunk && (p.N & 3) == 0) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        reinterpret_cast<uint4*>(ar)[q] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (n0 + j < p.N) ar[j] = static_cast<int32_t>(r[j]);
+    }
+  }
+}
+
+constexpr int kT2Threads = 320;  // warp 0: TMA, warp 1: MMA (leader), warps 2-9: epilogue
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT2Threads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -328,7 +379,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 8);  // 4 epilogue warps in each CTA
+      mbar_init(&tempty[b], 16);  // 8 epilogue warps in each CTA
     }
     fence_mbarrier_init();
   }
@@ -412,8 +463,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
       }
     }
   } else {
-    // ---------------- epilogue (warps 2-5 of both CTAs) ----------------
+    // ---------------- epilogue (warps 2-9 of both CTAs) ----------------
+    // Two warps per TMEM lane quadrant, 128 columns (4 chunks of 32) each; the
+    // TMEM load of the next chunk is in flight while the current one is stored.
     const int quad = warp & 3;
+    const int c0 = ((warp - 2) >> 2) * 4;
     int local = 0;
     for (int tile = pair; tile < p.num_tiles; tile += npairs, ++local) {
       const int buf = local & 1;
@@ -428,60 +482,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
       const int row = mb * kT2BM + static_cast<int>(rank) * 128 + quad * 32 + lane;
       const bool row_ok = row < p.M;
       const float rs = row_ok ? p.a_scale[row] : 0.f;
-#pragma unroll 1
-      for (int c = 0; c < kT2BN / 32; ++c) {
-        uint32_t r[32];
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                               static_cast<uint32_t>(buf * kT2BN + c * 32);
-        tmem_ld_32x32b_x32(taddr, r);
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * kT2BN);
+      uint32_t ra[32], rb[32];
+      tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(c0 * 32), ra);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t(&r)[32] = (i & 1) ? rb : ra;
+        if (i + 1 < 4) tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((c0 + i + 1) * 32), (i & 1) ? ra : rb);
+        const int n0 = nb * kT2BN + (c0 + i) * 32;
+        if (row_ok && n0 < p.N) epilogue_chunk(p, row, n0, rs, r);
         tmem_wait_ld();
-        const int n0 = nb * kT2BN + c * 32;
-        if (!row_ok || n0 >= p.N) continue;
-        const int64_t ga = n0 / p.alpha_group;
-        const bool one_alpha = ((n0 + 31) / p.alpha_group) == ga;
-        const float cs_uniform = __fmul_rn(rs, p.alpha[one_alpha ? ga : 0]);
-        float yv[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float cs = one_alpha ? cs_uniform
-                                     : __fmul_rn(rs, p.alpha[min(static_cast<int64_t>(n0 + j), static_cast<int64_t>(p.N - 1)) / p.alpha_group]);
-          yv[j] = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), cs);
-        }
-        const bool full_chunk = n0 + 32 <= p.N;
-        if (p.y != nullptr) {
-          uint16_t* yr = p.y + static_cast<int64_t>(row) * p.ldy + n0;
-          if (full_chunk) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 o;
-              o.x = pack_bf16x2(yv[8 * q + 0], yv[8 * q + 1]);
-              o.y = pack_bf16x2(yv[8 * q + 2], yv[8 * q + 3]);
-              o.z = pack_bf16x2(yv[8 * q + 4], yv[8 * q + 5]);
-              o.w = pack_bf16x2(yv[8 * q + 6], yv[8 * q + 7]);
-              reinterpret_cast<uint4*>(yr)[q] = o;
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (n0 + j < p.N) {
-                const __nv_bfloat16 b = __float2bfloat16_rn(yv[j]);
-                yr[j] = *reinterpret_cast<const uint16_t*>(&b);
-              }
-            }
-          }
-        }
-        if (p.acc != nullptr) {
-          int32_t* ar = p.acc + static_cast<int64_t>(row) * p.N + n0;
-          if (full_chunk && (p.N & 3) == 0) {
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              reinterpret_cast<uint4*>(ar)[q] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (n0 + j < p.N) ar[j] = static_cast<int32_t>(r[j]);
-          }
-        }
       }
       tc_fence_before();
       __syncwarp();
@@ -582,60 +593,130 @@ __device__ __forceinline__ void load_w_unit(const uint8_t* w_row, int u, uint32_
   }
 }
 
-template <int AF, bool WT2, int MT>
+// A tile in shared memory: MT rows of K codes widened to int8, stored as words
+// so that, for a fixed word i of a unit, the 32 lanes of a warp (units
+// u = 32*uh + lane) read 32 consecutive words:  word(m, u, i) at
+// ((m * units_hi + u / 32) * 16 + i) * 32 + u % 32.
+__device__ __forceinline__ int simt_a_word(int m, int u, int i, int units_hi) {
+  return ((m * units_hi + (u >> 5)) * 16 + i) * 32 + (u & 31);
+}
+
+// Rows per warp for a round of UPL units per lane: 2-bit weight units are 16 B,
+// so a lane keeps UPL * R = 8 of them in flight; int8 units are 64 B (one row).
+template <bool WT2, int UPL>
+struct SimtShape {
+  static constexpr int R = WT2 ? (UPL >= 8 ? 1 : 8 / UPL) : 1;
+  static constexpr int Q = WT2 ? 1 : 4;  // 16-byte words per weight unit
+};
+
+template <int AF, bool WT2, int MT, int UPL>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const uint8_t* __restrict__ a, const float* __restrict__ a_scale,
                                                         const uint8_t* __restrict__ w, const float* __restrict__ alpha,
                                                         int64_t alpha_group, int M, int N, int K,
                                                         uint16_t* __restrict__ y, int64_t ldy,
                                                         int32_t* __restrict__ acc_out) {
+  constexpr int R = SimtShape<WT2, UPL>::R;
+  constexpr int Q = SimtShape<WT2, UPL>::Q;
+  extern __shared__ uint32_t sa[];
   const int lane = threadIdx.x & 31;
-  const int64_t gwarp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int units = K >> 6;
+  const int warp = threadIdx.x >> 5;
+  const int units = K >> 6;                 // 64 codes per unit
+  const int units_hi = (units + 31) >> 5;
   const int64_t a_row_bytes = (AF == kSimtA_I8) ? K : (K >> 1);
   const int64_t w_row_bytes = WT2 ? (K >> 2) : K;
   const float unit_scale = (AF == kSimtA_E2M1) ? 0.5f : 1.0f;
 
-  for (int64_t n = gwarp; n < N; n += nwarps) {
-    const uint8_t* w_row = w + n * w_row_bytes;
-    const float al = alpha[n / alpha_group];
-    for (int m0 = 0; m0 < M; m0 += MT) {
-      int acc[MT];
+  for (int m0 = 0; m0 < M; m0 += MT) {
+    __syncthreads();  // the previous tile's readers are done with sa
+    for (int i = threadIdx.x; i < MT * units_hi * 32; i += blockDim.x) {
+      const int m = i / (units_hi * 32);
+      const int u = i - m * units_hi * 32;
+      uint32_t wv[16];
+      if (m0 + m < M && u < units) {
+        load_a_unit<AF>(a + static_cast<int64_t>(m0 + m) * a_row_bytes, u, wv);
+      } else {
 #pragma unroll
-      for (int r = 0; r < MT; ++r) acc[r] = 0;
-      for (int u = lane; u < units; u += 32) {
-        uint32_t wu[16];
-        load_w_unit<WT2>(w_row, u, wu);
+        for (int j = 0; j < 16; ++j) wv[j] = 0;
+      }
 #pragma unroll
-        for (int r = 0; r < MT; ++r) {
-          if (m0 + r < M) {
-            uint32_t au[16];
-            load_a_unit<AF>(a + static_cast<int64_t>(m0 + r) * a_row_bytes, u, au);
+      for (int j = 0; j < 16; ++j) sa[simt_a_word(m, u, j, units_hi)] = wv[j];
+    }
+    __syncthreads();
+
+    for (int64_t n0 = (static_cast<int64_t>(blockIdx.x) * 8 + warp) * R; n0 < N;
+         n0 += static_cast<int64_t>(gridDim.x) * 8 * R) {
+      int acc[R][MT];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) acc[r] = __dp4a(static_cast<int>(au[i]), static_cast<int>(wu[i]), acc[r]);
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[r][m] = 0;
+      for (int u0 = 0; u0 < units; u0 += 32 * UPL) {
+        // every weight load of the round first, so they are in flight together
+        uint4 raw[UPL][R][Q];
+#pragma unroll
+        for (int j = 0; j < UPL; ++j) {
+          const int u = u0 + j * 32 + lane;
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            const bool ok = u < units && n0 + r < N;
+            const uint8_t* wr = w + (n0 + r < N ? n0 + r : n0) * w_row_bytes + static_cast<int64_t>(u) * (WT2 ? 16 : 64);
+#pragma unroll
+            for (int q = 0; q < Q; ++q) raw[j][r][q] = ok ? ld_global_nc_v4(wr + 16 * q) : make_uint4(0, 0, 0, 0);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < UPL; ++j) {
+          const int u = u0 + j * 32 + lane;
+          if (u >= units) continue;
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            uint32_t wx[16];
+            if constexpr (WT2) {
+              const uint32_t pk[4] = {raw[j][r][0].x, raw[j][r][0].y, raw[j][r][0].z, raw[j][r][0].w};
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) wx[4 * jj + b] = expand_t2_byte((pk[jj] >> (8 * b)) & 0xFFu);
+            } else {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                wx[4 * q] = raw[j][r][q].x; wx[4 * q + 1] = raw[j][r][q].y;
+                wx[4 * q + 2] = raw[j][r][q].z; wx[4 * q + 3] = raw[j][r][q].w;
+              }
+            }
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                acc[r][m] = __dp4a(static_cast<int>(sa[simt_a_word(m, u, i, units_hi)]), static_cast<int>(wx[i]), acc[r][m]);
           }
         }
       }
 #pragma unroll
-      for (int r = 0; r < MT; ++r) {
+      for (int r = 0; r < R; ++r)
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc[r] += __shfl_xor_sync(0xFFFFFFFFu, acc[r], o);
-      }
-      if (lane < MT) {
-        int mine = 0;
+        for (int m = 0; m < MT; ++m)
 #pragma unroll
-        for (int r = 0; r < MT; ++r)
-          if (r == lane) mine = acc[r];
-        const int m = m0 + lane;
-        if (m < M) {
-          if (acc_out != nullptr) acc_out[static_cast<int64_t>(m) * N + n] = mine;
-          if (y != nullptr) {
-            const float cs = __fmul_rn(__fmul_rn(a_scale[m], unit_scale), al);
-            const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__int2float_rn(mine), cs));
-            y[static_cast<int64_t>(m) * ldy + n] = *reinterpret_cast<const uint16_t*>(&b);
+          for (int o = 16; o > 0; o >>= 1) acc[r][m] += __shfl_xor_sync(0xFFFFFFFFu, acc[r][m], o);
+      // every lane holds every reduced sum; output (r, m) is written by lane (r * MT + m) % 32
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          if (lane == ((r * MT + m) & 31)) {
+            const int64_t n = n0 + r;
+            const int mm = m0 + m;
+            if (n < N && mm < M) {
+              const int v = acc[r][m];
+              if (acc_out != nullptr) acc_out[static_cast<int64_t>(mm) * N + n] = v;
+              if (y != nullptr) {
+                const float cs = __fmul_rn(__fmul_rn(a_scale[mm], unit_scale), alpha[n / alpha_group]);
+                const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__int2float_rn(v), cs));
+                y[static_cast<int64_t>(mm) * ldy + n] = *reinterpret_cast<const uint16_t*>(&b);
+              }
+            }
           }
         }
-      }
     }
   }
 }

@@ -22,30 +22,32 @@ __global__ void __launch_bounds__(256) kv_quant_kernel(const uint16_t* __restric
   constexpr int D = TPV * 8;
   const int lane = threadIdx.x & 31;
   const int sub = lane % TPV;  // position inside the vector's thread group
-  const int64_t group = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / TPV;
-  const int64_t ngroups = static_cast<int64_t>(gridDim.x) * blockDim.x / TPV;
-  const int64_t nvec = T * H;
+  // the host keeps T * H below 2^31, so vector indices fit 32-bit arithmetic
+  const uint32_t group = (blockIdx.x * blockDim.x + threadIdx.x) / TPV;
+  const uint32_t ngroups = gridDim.x * blockDim.x / TPV;
+  const uint32_t nvec = static_cast<uint32_t>(T) * static_cast<uint32_t>(H);
+  const uint32_t uh = static_cast<uint32_t>(H);
 
   // group g handles vectors g, g + ngroups, ... so neighbouring groups read
   // neighbouring vectors in every round
   uint4 v[kKvItems];
 #pragma unroll
   for (int it = 0; it < kKvItems; ++it) {
-    const int64_t vec = group + it * ngroups;
+    const uint32_t vec = group + it * ngroups;
     v[it] = make_uint4(0, 0, 0, 0);
     if (vec < nvec) {
-      const int64_t t = vec / H;
-      const int h = static_cast<int>(vec - t * H);
-      v[it] = ld_global_nc_v4(kv + t * ldt + static_cast<int64_t>(h) * D + sub * 8);
+      const uint32_t t = vec / uh;
+      const uint32_t h = vec - t * uh;
+      v[it] = ld_global_nc_v4(kv + static_cast<int64_t>(t) * ldt + static_cast<int64_t>(h) * D + sub * 8);
     }
   }
 
 #pragma unroll
   for (int it = 0; it < kKvItems; ++it) {
-    const int64_t vec = group + it * ngroups;
+    const uint32_t vec = group + it * ngroups;
     const bool ok = vec < nvec;
-    const int64_t t = ok ? vec / H : 0;
-    const int h = ok ? static_cast<int>(vec - t * H) : 0;
+    const uint32_t t = ok ? vec / uh : 0u;
+    const uint32_t h = ok ? vec - t * uh : 0u;
 
     uint32_t k[8];
     bf16x8_mag_keys(v[it], k);
@@ -56,7 +58,7 @@ __global__ void __launch_bounds__(256) kv_quant_kernel(const uint16_t* __restric
     for (int o = TPV / 2; o > 0; o >>= 1) mk = max(mk, __shfl_xor_sync(0xFFFFFFFFu, mk, o));
     const float gamma = __uint_as_float(mk << 16);
 
-    const bool is_bos = (bits == 3) && (t == bos_pos);
+    const bool is_bos = (bits == 3) && (static_cast<int64_t>(t) == bos_pos);
     const int b = is_bos ? 4 : bits;
     const float qmax = static_cast<float>((1 << (b - 1)) - 1);
     const float mult = __fdiv_rn(qmax, __fadd_rn(gamma, eps));
@@ -77,7 +79,7 @@ __global__ void __launch_bounds__(256) kv_quant_kernel(const uint16_t* __restric
         if (is_bos) {
           reinterpret_cast<uint32_t*>(bos_codes + static_cast<int64_t>(h) * (D / 2))[sub] = word;
         } else {
-          reinterpret_cast<uint32_t*>(codes + vec * (D / 2))[sub] = word;
+          reinterpret_cast<uint32_t*>(codes + static_cast<int64_t>(vec) * (D / 2))[sub] = word;
         }
       }
     }
@@ -93,7 +95,7 @@ __global__ void __launch_bounds__(256) kv_quant_kernel(const uint16_t* __restric
       const uint32_t w2 = __shfl_down_sync(0xFFFFFFFFu, w24, 2);
       const uint32_t w3 = __shfl_down_sync(0xFFFFFFFFu, w24, 3);
       if (ok && (sub & 3) == 0) {
-        uint32_t* dst = reinterpret_cast<uint32_t*>(codes + vec * (D * 3 / 8) + (sub / 4) * 12);
+        uint32_t* dst = reinterpret_cast<uint32_t*>(codes + static_cast<int64_t>(vec) * (D * 3 / 8) + (sub / 4) * 12);
         dst[0] = w24 | (w1 << 24);
         dst[1] = (w1 >> 8) | (w2 << 16);
         dst[2] = (w2 >> 16) | (w3 << 8);

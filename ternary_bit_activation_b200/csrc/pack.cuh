@@ -44,17 +44,23 @@ __global__ void __launch_bounds__(kBinThreads) ternary_bins_kernel(const float* 
   for (int i = threadIdx.x; i < kBins; i += kBinThreads) sb[i] = 0ull;
   __syncthreads();
   const int per_row = K >> 2;  // float4 per row
-  const int64_t total = N * static_cast<int64_t>(per_row);
   const int64_t gwarp = (static_cast<int64_t>(blockIdx.x) * kBinThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kBinThreads) >> 5;
-  for (int64_t g = gwarp * 32; g < total; g += nwarps * 32) {   // warp-uniform trip count
-    const int64_t i = g + lane;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (i < total) {
-      const int64_t n = i / per_row;
-      const int q = static_cast<int>(i - n * per_row);
-      v = ld_global_nc_v4(w + n * ldw + static_cast<int64_t>(q) * 4);
+  // a warp walks (row, 128-weight group) pairs without integer division: rows
+  // n = gwarp, gwarp + nwarps, ...; within a row, kGroups groups per round
+  constexpr int kGroups = 4;   // groups whose loads are issued together
+  for (int64_t n = gwarp; n < N; n += nwarps) {
+   const float* wrow = w + n * ldw;
+   for (int q0 = 0; q0 < per_row; q0 += 32 * kGroups) {   // warp-uniform
+    uint4 vv[kGroups];
+#pragma unroll
+    for (int gi = 0; gi < kGroups; ++gi) {
+      const int q = q0 + gi * 32 + lane;
+      vv[gi] = q < per_row ? ld_global_nc_v4(wrow + static_cast<int64_t>(q) * 4) : make_uint4(0, 0, 0, 0);
     }
+#pragma unroll
+   for (int gi = 0; gi < kGroups; ++gi) {
+    const uint4 v = vv[gi];
     const uint32_t u[4] = {v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu, v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu};
     uint32_t e[4], m[4], emax = 0;
 #pragma unroll
@@ -65,7 +71,7 @@ __global__ void __launch_bounds__(kBinThreads) ternary_bins_kernel(const float* 
       if (m[j]) emax = max(emax, e[j]);
     }
     const uint32_t ew = __reduce_max_sync(0xFFFFFFFFu, emax);
-    if (ew == 0) continue;  // the whole group is zero
+    if (ew == 0) continue;  // the whole group is zero (warp-uniform)
     const uint32_t base = ew > 32 ? ew - 31 : 1u;
     unsigned long long acc = 0;
 #pragma unroll
@@ -79,6 +85,8 @@ __global__ void __launch_bounds__(kBinThreads) ternary_bins_kernel(const float* 
       atomicAdd(&sb[base], acc & 0xFFFFFFFFull);
       atomicAdd(&sb[base + 32], acc >> 32);
     }
+   }
+   }
   }
   __syncthreads();
   for (int b = threadIdx.x; b < kBins; b += kBinThreads)
@@ -137,13 +145,16 @@ __device__ __forceinline__ unsigned long long big_window64(const uint32_t (&z)[k
 }
 
 // alpha = RN_fp32( (Z * 2^-149) / D ),  Z = sum_e bins[e] << (e - 1); single thread.
-__global__ void ternary_alpha_kernel(const unsigned long long* __restrict__ gbins, unsigned long long D,
-                                     float* __restrict__ alpha) {
+__global__ void __launch_bounds__(kBins) ternary_alpha_kernel(const unsigned long long* __restrict__ gbins,
+                                                               unsigned long long D, float* __restrict__ alpha) {
+  __shared__ unsigned long long sb[kBins];
+  for (int e = threadIdx.x; e < kBins; e += blockDim.x) sb[e] = gbins[e];   // one round trip for all bins
+  __syncthreads();
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   uint32_t z[kLimbs];
   for (int i = 0; i < kLimbs; ++i) z[i] = 0;
   for (int e = 0; e < kBins; ++e) {
-    const unsigned long long b = gbins[e];
+    const unsigned long long b = sb[e];
     if (b) big_add_shifted(z, b, (e > 0 ? e : 1) - 1);
   }
   // Long division Q = floor(Z / D), R = Z mod D.
@@ -211,12 +222,13 @@ __global__ void __launch_bounds__(256) ternary_pack_kernel(const float* __restri
                                                            int64_t ldw, const float* __restrict__ alpha,
                                                            float eps, uint8_t* __restrict__ out) {
   const float d = __fadd_rn(*alpha, eps);
-  const int per_row = K >> 4;
-  const int64_t total = N * static_cast<int64_t>(per_row);
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t n = i / per_row;
-    const int q = static_cast<int>(i - n * per_row);
+  const int per_row = K >> 4;   // 16 weights per thread-step
+  // rows strided over the grid's warps, 16-weight steps strided over lanes: no integer division
+  const int lane = threadIdx.x & 31;
+  const int64_t gwarp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t n = gwarp; n < N; n += nwarps)
+  for (int q = lane; q < per_row; q += 32) {
     const float* src = w + n * ldw + static_cast<int64_t>(q) * 16;
     int c[16];
 #pragma unroll
