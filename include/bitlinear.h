@@ -128,7 +128,7 @@ BL_API bl_status bitlinear_sparsify_a8(const void* x_bf16, int64_t M, int64_t K,
  * bytes, BL_W_I8 -> N x K bytes (layouts in bl_wfmt).
  * workspace: device scratch of bitlinear_workspace_size("pack_ternary", N, K, 0)
  * bytes (2 KiB; cleared by the call itself).  Not needed when alpha_given != 0.
- * Requires K % 16 == 0, ldw % 4 == 0, N * K < 2^38.
+ * Requires K % 16 == 0, ldw % 4 == 0, N * K < 2^31.
  */
 BL_API bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float eps,
                        int alpha_given, float* alpha, bl_wfmt wfmt, void* w_out,
@@ -146,7 +146,7 @@ BL_API bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw,
  * held until the process exits.  The caller still passes w, alpha and w_out.
  * Same arguments, layouts and results as pack_ternary (alpha and codes are
  * bit-identical); the scratch is cleared at the start of every call.
- * Limits: N * K < 2^38, so no 64-bit bin can overflow; larger tensors are
+ * Limits: N * K < 2^31, so no 64-bit bin can overflow; larger tensors are
  * rejected with BL_ERR_SHAPE.  The first call on a device looks up the
  * array's device address (once per device); make that first call before any
  * stream capture.  Every call on a device shares the one array, so calls that

@@ -15,6 +15,7 @@
 #include "kv.cuh"
 #include "pack.cuh"
 #include "quant.cuh"
+#include "topk.cuh"
 
 namespace {
 
@@ -109,43 +110,44 @@ void launch_quant_a4_c(const uint16_t* x, int64_t M, int K, int64_t ldx, bool fp
   if (fp4 && !packed) bl::quant_a4_kernel<C, true, false><<<grid, 256, 0, s>>>(x, M, K, ldx, eps, codes, scale);
 }
 
-template <int C>
-void launch_sparsify_c(const uint16_t* x, int64_t M, int K, int64_t ldx, int keep, float eps, int8_t* codes,
-                       float* scale, uint32_t* mask, cudaStream_t s) {
-  bl::sparsify_a8_kernel<C><<<static_cast<unsigned>(M), bl::kTkThreads, 0, s>>>(x, K, ldx, keep, eps, codes, scale,
-                                                                                  mask);
-}
-
-template <int C>
-void launch_relu2_c(const uint16_t* g, const uint16_t* u, int64_t M, int F, int64_t ld, int keep, float eps,
-                    int8_t* codes, float* scale, uint32_t* mask, cudaStream_t s) {
-  // persistent: as many CTAs as fit (registers and the row buffer), rows strided over them
-  const size_t smem = 2 * static_cast<size_t>(C) * bl::kTkThreads * sizeof(uint4);
-  auto kern = bl::relu2_glu_persistent_kernel<C>;
-  // opt-in shared-memory limit and resident CTAs per SM, looked up once per device
-  static int per_sm_cache[kMaxDevices] = {};
+// Top-K rows: groups of G warps per row (shared-memory row buffer), persistent
+// grid sized by the occupancy the buffer allows.
+template <int G, bool RELU2>
+bl_status launch_topk_rows_g(const uint16_t* x, const uint16_t* up, int64_t M, int K, int64_t ldx, int keep,
+                             float eps, int8_t* codes, float* scale, uint32_t* mask, cudaStream_t s) {
+  constexpr int kGroups = bl::kRowThreads / (G * 32);
+  const int row_words = (K / 8) * (RELU2 ? 2 : 1);
+  const size_t smem = static_cast<size_t>(kGroups) *
+                      (sizeof(bl::GroupSmem) + static_cast<size_t>(row_words) * 16 + (RELU2 ? bl::kRowListCap * 4 : 0));
+  if (smem > 227 * 1024) return BL_ERR_SHAPE;
+  auto kern = bl::topk_rows_kernel<G, RELU2>;
+  static bool attr_done[kMaxDevices] = {};
   const int d = current_device();
-  int per_sm = 1;
-  if (d >= 0 && d < kMaxDevices) {
-    if (per_sm_cache[d] == 0) {
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      int n = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, bl::kTkThreads, smem) != cudaSuccess || n < 1) n = 1;
-      per_sm_cache[d] = n;
-    }
-    per_sm = per_sm_cache[d];
+  if (d < 0 || d >= kMaxDevices) return BL_ERR_CUDA;
+  if (!attr_done[d]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+      return BL_ERR_CUDA;
+    attr_done[d] = true;
   }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, bl::kRowThreads, smem) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const int64_t need = (M + kGroups - 1) / kGroups;
   const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
-  const unsigned grid = static_cast<unsigned>(M < cap ? M : cap);
-  kern<<<grid, bl::kTkThreads, smem, s>>>(g, u, M, F, ld, keep, eps, codes, scale, mask);
+  const unsigned grid = static_cast<unsigned>(need < cap ? need : cap);
+  kern<<<grid, bl::kRowThreads, smem, s>>>(x, up, M, K, ldx, keep, eps, codes, scale, mask, row_words);
+  return launch_status();
 }
 
-bool topk_chunks(int64_t K, int* chunks) {
-  const int64_t c = (K / 8 + bl::kTkThreads - 1) / bl::kTkThreads;
-  if (c < 1 || c > 8) return false;
-  *chunks = static_cast<int>(c);
-  return true;
+template <bool RELU2>
+bl_status launch_topk_rows(const uint16_t* x, const uint16_t* up, int64_t M, int K, int64_t ldx, int keep,
+                           float eps, int8_t* codes, float* scale, uint32_t* mask, cudaStream_t s) {
+  if (K <= 4096) return launch_topk_rows_g<1, RELU2>(x, up, M, K, ldx, keep, eps, codes, scale, mask, s);
+  if (K <= 8192) return launch_topk_rows_g<2, RELU2>(x, up, M, K, ldx, keep, eps, codes, scale, mask, s);
+  return launch_topk_rows_g<4, RELU2>(x, up, M, K, ldx, keep, eps, codes, scale, mask, s);
 }
+
 
 template <int AF, bool WT2, int MT, int UPL>
 bool launch_simt_mu(const uint8_t* a, const float* sc, const uint8_t* w, const float* al, int64_t g, int M, int N,
@@ -320,22 +322,8 @@ bl_status bitlinear_sparsify_a8(const void* x_bf16, int64_t M, int64_t K, int64_
   if (M == 0) return BL_OK;
   if (x_bf16 == nullptr || codes == nullptr || scale == nullptr) return BL_ERR_NULL;
   if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scale) || (mask && !aligned16(mask))) return BL_ERR_ALIGN;
-  int c = 0;
-  if (!topk_chunks(K, &c)) return BL_ERR_SHAPE;
-  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
-  const int k = static_cast<int>(K), kk = static_cast<int>(k_keep);
-  cudaStream_t s = as_stream(stream);
-  switch (c) {
-    case 1: launch_sparsify_c<1>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
-    case 2: launch_sparsify_c<2>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
-    case 3: launch_sparsify_c<3>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
-    case 4: launch_sparsify_c<4>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
-    case 5: launch_sparsify_c<5>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
-    case 6: launch_sparsify_c<6>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
-    case 7: launch_sparsify_c<7>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
-    default: launch_sparsify_c<8>(x, M, k, ldx, kk, eps, codes, scale, mask, s); break;
-  }
-  return launch_status();
+  return launch_topk_rows<false>(static_cast<const uint16_t*>(x_bf16), nullptr, M, static_cast<int>(K), ldx,
+                                 static_cast<int>(k_keep), eps, codes, scale, mask, as_stream(stream));
 }
 
 bl_status relu2_glu(const void* gate_bf16, const void* up_bf16, int64_t M, int64_t F, int64_t ld, int64_t k_keep,
@@ -348,23 +336,10 @@ bl_status relu2_glu(const void* gate_bf16, const void* up_bf16, int64_t M, int64
   if (!aligned16(gate_bf16) || !aligned16(up_bf16) || !aligned16(codes) || !aligned16(scale) ||
       (mask && !aligned16(mask)))
     return BL_ERR_ALIGN;
-  int c = 0;
-  if (!topk_chunks(F, &c)) return BL_ERR_SHAPE;
-  const uint16_t* g = static_cast<const uint16_t*>(gate_bf16);
-  const uint16_t* u = static_cast<const uint16_t*>(up_bf16);
-  const int f = static_cast<int>(F), kk = static_cast<int>(k_keep);
-  cudaStream_t s = as_stream(stream);
-  switch (c) {
-    case 1: launch_relu2_c<1>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
-    case 2: launch_relu2_c<2>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
-    case 3: launch_relu2_c<3>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
-    case 4: launch_relu2_c<4>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
-    case 5: launch_relu2_c<5>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
-    case 6: launch_relu2_c<6>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
-    case 7: launch_relu2_c<7>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
-    default: launch_relu2_c<8>(g, u, M, f, ld, kk, eps, codes, scale, mask, s); break;
-  }
-  return launch_status();
+  // gate and up share the row stride ld; the kernel reads gate through x
+  return launch_topk_rows<true>(static_cast<const uint16_t*>(gate_bf16), static_cast<const uint16_t*>(up_bf16), M,
+                                static_cast<int>(F), ld, static_cast<int>(k_keep), eps, codes, scale, mask,
+                                as_stream(stream));
 }
 
 bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float eps, int alpha_given, float* alpha,

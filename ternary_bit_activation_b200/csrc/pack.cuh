@@ -16,12 +16,13 @@ namespace bl {
 
 constexpr int kBinThreads = 256;
 // bins[e] is the integer coefficient of 2^(e - 150), e >= 1 (fp32 subnormals use
-// e = 1, the same scale).  A window base is at most 254 - 31, so the high half
-// of a window sum (index base + 32) still fits in 256 entries.
+// e = 1, the same scale).  A window base is clamped to at most 223, so the high
+// half of a window sum (index base + 32) stays below 256.
 constexpr int kBins = 256;
-// Each bin receives at most one 32-bit half per 128 weights (plus 24-bit
-// significands), so N*K < 2^38 keeps every 64-bit bin below overflow.
-constexpr int64_t kMaxPackElems = int64_t(1) << 38;
+// Each bin receives at most one 32-bit half per flushed window (>= 1 weight)
+// or one 24-bit significand per weight, so N*K < 2^31 keeps every 64-bit bin
+// below overflow (2^31 * 2^32).
+constexpr int64_t kMaxPackElems = int64_t(1) << 31;
 
 __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
 #pragma unroll
@@ -29,13 +30,23 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
   return v;
 }
 
-// Exact sum of |w| into exponent bins.  Each warp takes 128 weights at a time
-// (a float4 per lane), finds their largest exponent Ew, and adds every
-// significand shifted into a window of 32 exponents below Ew:
-//   |w| = m * 2^(e-150) = (m << (e - base)) * 2^(base-150),  base = max(Ew - 31, 1),
-// so each term is < 2^55 and the warp's 128-term sum < 2^62 is exact in 64 bits.
-// The sum goes into bins[base] (low 32 bits) and bins[base+32] (high bits).
-// Weights more than 2^31 below the group's largest go straight to their own bin.
+// Exact sum of |w| into exponent bins.  Each lane keeps a 64-bit fixed-point
+// accumulator whose unit is 2^(base-150): |w| = m * 2^(e-150) adds m << (e - base)
+// (exact while 0 <= e - base <= 31, a term < 2^55).  The window is anchored on
+// the lane's first nonzero weight (base = its exponent - 24, clamped to
+// [1, 223], so it spans about 2^-24 to 2^7 of that weight); weights outside it
+// go straight to their own bin.
+// Every 256 terms (< 2^63 in total) and at the end, the accumulator is flushed
+// into bins[base] (low 32 bits) and bins[base + 32] (high bits).  Lanes walk
+// (row, float4) positions without integer division.
+__device__ __forceinline__ void bins_flush(unsigned long long* sb, uint32_t base, unsigned long long& acc) {
+  if (acc) {
+    atomicAdd(&sb[base], acc & 0xFFFFFFFFull);
+    atomicAdd(&sb[base + 32], acc >> 32);
+    acc = 0;
+  }
+}
+
 __global__ void __launch_bounds__(kBinThreads) ternary_bins_kernel(const float* __restrict__ w, int64_t N, int K,
                                                                    int64_t ldw,
                                                                    unsigned long long* __restrict__ gbins) {
@@ -46,55 +57,52 @@ __global__ void __launch_bounds__(kBinThreads) ternary_bins_kernel(const float* 
   const int per_row = K >> 2;  // float4 per row
   const int64_t gwarp = (static_cast<int64_t>(blockIdx.x) * kBinThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kBinThreads) >> 5;
-  // a warp walks (row, 128-weight group) pairs without integer division: rows
-  // n = gwarp, gwarp + nwarps, ...; within a row, kGroups groups per round
-  constexpr int kGroups = 4;   // groups whose loads are issued together
+  constexpr int kLoads = 4;   // float4 loads per lane issued together
+  uint32_t base = 0;          // 0: not anchored yet
+  unsigned long long acc = 0;
+  int terms = 0;
   for (int64_t n = gwarp; n < N; n += nwarps) {
-   const float* wrow = w + n * ldw;
-   for (int q0 = 0; q0 < per_row; q0 += 32 * kGroups) {   // warp-uniform
-    uint4 vv[kGroups];
+    const float* wrow = w + n * ldw;
+    for (int q0 = 0; q0 < per_row; q0 += 32 * kLoads) {
+      uint4 vv[kLoads];
 #pragma unroll
-    for (int gi = 0; gi < kGroups; ++gi) {
-      const int q = q0 + gi * 32 + lane;
-      vv[gi] = q < per_row ? ld_global_nc_v4(wrow + static_cast<int64_t>(q) * 4) : make_uint4(0, 0, 0, 0);
-    }
+      for (int j = 0; j < kLoads; ++j) {
+        const int q = q0 + j * 32 + lane;
+        vv[j] = q < per_row ? ld_global_nc_v4(wrow + static_cast<int64_t>(q) * 4) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-   for (int gi = 0; gi < kGroups; ++gi) {
-    const uint4 v = vv[gi];
-    const uint32_t u[4] = {v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu, v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu};
-    uint32_t e[4], m[4], emax = 0;
+      for (int j = 0; j < kLoads; ++j) {
+        const uint32_t u[4] = {vv[j].x, vv[j].y, vv[j].z, vv[j].w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t E = u[j] >> 23;
-      m[j] = (u[j] & 0x7FFFFFu) | (E ? 0x800000u : 0u);
-      e[j] = E ? E : 1u;
-      if (m[j]) emax = max(emax, e[j]);
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t a = u[k] & 0x7FFFFFFFu;
+          if (a == 0) continue;
+          const uint32_t E = a >> 23;
+          const uint32_t m = (a & 0x7FFFFFu) | (E ? 0x800000u : 0u);
+          const uint32_t e = E ? E : 1u;
+          if (base == 0) base = e > 25 ? min(e - 24, 223u) : 1u;   // window [base, base + 31] holds e
+          const uint32_t sh = e - base;   // wraps to a large value when e < base
+          if (sh <= 31u) {
+            acc += static_cast<unsigned long long>(m) << sh;
+            if (++terms == 256) {
+              bins_flush(sb, base, acc);
+              terms = 0;
+            }
+          } else {
+            atomicAdd(&sb[e], static_cast<unsigned long long>(m));
+          }
+        }
+      }
     }
-    const uint32_t ew = __reduce_max_sync(0xFFFFFFFFu, emax);
-    if (ew == 0) continue;  // the whole group is zero (warp-uniform)
-    const uint32_t base = ew > 32 ? ew - 31 : 1u;
-    unsigned long long acc = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (m[j] == 0) continue;
-      if (e[j] >= base) acc += static_cast<unsigned long long>(m[j]) << (e[j] - base);
-      else atomicAdd(&sb[e[j]], static_cast<unsigned long long>(m[j]));
-    }
-    acc = warp_sum_u64(acc);
-    if (lane == 0) {
-      atomicAdd(&sb[base], acc & 0xFFFFFFFFull);
-      atomicAdd(&sb[base + 32], acc >> 32);
-    }
-   }
-   }
   }
+  bins_flush(sb, base, acc);
   __syncthreads();
   for (int b = threadIdx.x; b < kBins; b += kBinThreads)
     if (sb[b]) atomicAdd(&gbins[b], sb[b]);
 }
 
 // Multi-word unsigned integer, little-endian 32-bit limbs.
-constexpr int kLimbs = 12;  // 384 bits: bins < 2^64 shifted by <= 254 bits
+constexpr int kLimbs = 12;  // 384 bits: bins < 2^64 shifted by <= 262 bits
 
 __device__ __forceinline__ void big_add_shifted(uint32_t (&z)[kLimbs], unsigned long long v, int shift) {
   const int li = shift >> 5, bo = shift & 31;

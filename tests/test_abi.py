@@ -109,7 +109,7 @@ def test_pack_and_kv_validation(L):
     assert pk(P(A16), 8, 64, 64, 1e-5, 0, P(A16), 0, P(A16), None, 0, None) == 1
     assert pk(P(A16), 8, 64, 64, 1e-5, 0, P(A16), 5, P(A16), P(A16), 2048, None) == 4
     pn = L.pack_ternary_noalloc
-    assert pn(P(A16), 1 << 20, 1 << 18, 1 << 18, 1e-5, 0, P(A16), 0, P(A16), None) == 3   # N*K >= 2^38
+    assert pn(P(A16), 1 << 16, 1 << 15, 1 << 15, 1e-5, 0, P(A16), 0, P(A16), None) == 3   # N*K >= 2^31
     assert pn(P(A16), 8, 24, 24, 1e-5, 0, P(A16), 0, P(A16), None) == 3                   # K % 16
     assert pn(P(A16), 8, 64, 64, 1e-5, 0, None, 0, P(A16), None) == 1
     kv = L.kv_quant3

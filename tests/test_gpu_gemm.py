@@ -29,12 +29,31 @@ def run_pack(w, wfmt, alpha_in=None):
     return host(out), host(alpha)[0]
 
 
+def _wide_range_weights():
+    # magnitudes from 2^-140 (subnormal) to 2^120, both signs
+    g = synth.rng(26)
+    e = g.integers(-140, 121, (64, 512))
+    m = 1.0 + g.random((64, 512))
+    sgn = np.where(g.random((64, 512)) < 0.5, -1.0, 1.0)
+    return (sgn * m * np.exp2(e.astype(np.float64))).astype(np.float32)
+
+
+def _tiny_first_weights():
+    # every lane's first weight is tiny, so its window sits far below the rest
+    w = synth.latent_weights_f32(synth.rng(27), 64, 1024)
+    w[:, ::4] = np.float32(1e-30)
+    return w
+
+
 PACK_CASES = [
     ("tiny_256x256", lambda: synth.tiny_inputs(0)[1]),
     ("700M_qkv", lambda: synth.latent_weights_f32(synth.rng(21), 4608, 1536)),
     ("odd_rows_K3200", lambda: synth.latent_weights_f32(synth.rng(22), 33, 3200)),
     ("tiny_values", lambda: (synth.latent_weights_f32(synth.rng(23), 16, 64) * np.float32(1e-36))),
     ("constant", lambda: np.full((8, 64), -0.0213, np.float32)),
+    ("wide_exponent_range", lambda: _wide_range_weights()),
+    ("tiny_first_then_normal", lambda: _tiny_first_weights()),
+    ("near_max_magnitude", lambda: (synth.latent_weights_f32(synth.rng(25), 8, 256) * np.float32(1e38))),
     ("zeros", lambda: np.zeros((4, 64), np.float32)),
 ]
 
