@@ -229,6 +229,12 @@ BL_API bl_status bitlinear_sync_status(void* stream);
 /* Human-readable name of a status code (static storage). */
 BL_API const char* bitlinear_status_string(bl_status status);
 
+/* Name of the CUDA runtime error (static storage, e.g. "cudaErrorInvalidValue")
+ * behind the last BL_ERR_CUDA that an entry point returned on the calling host
+ * thread; "cudaSuccess" if there was none.  Not reset by later successful calls.
+ * No counterpart in the paper: a diagnostic of this library. */
+BL_API const char* bitlinear_last_cuda_error(void);
+
 /* Library version string (static storage). */
 BL_API const char* bitlinear_version(void);
 

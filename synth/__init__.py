@@ -32,11 +32,13 @@ import numpy as np
 # ----------------------------------------------------------------------------
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """fp32 array -> bf16 bit patterns (uint16), round-to-nearest-even."""
-    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    a = np.ascontiguousarray(a, dtype=np.float32)
     if np.isnan(a).any():
         raise ValueError("NaN inputs are not generated")
-    rounding_bias = 0x7FFF + ((u >> 16) & 1)
-    return ((u + rounding_bias) >> 16).astype(np.uint16)
+    u = a.view(np.uint32)
+    rounding_bias = np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
+    # u + bias stays below 2^32 for every finite value (the top exponent is 0xFE)
+    return ((u + rounding_bias) >> np.uint32(16)).astype(np.uint16)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -50,10 +52,12 @@ def rng(seed: int) -> np.random.Generator:
 
 def gaussian_bf16(g: np.random.Generator, shape, sigma: float = 1.0,
                   outlier_channels=(), outlier_scale: float = 1.0) -> np.ndarray:
-    x = g.standard_normal(size=shape, dtype=np.float64) * sigma
+    x = g.standard_normal(size=shape, dtype=np.float32)
+    if sigma != 1.0:
+        x *= np.float32(sigma)
     for c in outlier_channels:
-        x[..., c] *= outlier_scale
-    return f32_to_bf16_bits(x.astype(np.float32))
+        x[..., c] *= np.float32(outlier_scale)
+    return f32_to_bf16_bits(x)
 
 
 def student_t_bf16(g: np.random.Generator, shape, nu: float = 3.0) -> np.ndarray:
@@ -62,7 +66,9 @@ def student_t_bf16(g: np.random.Generator, shape, nu: float = 3.0) -> np.ndarray
 
 
 def latent_weights_f32(g: np.random.Generator, n: int, k: int, sigma: float = 0.02) -> np.ndarray:
-    return (g.standard_normal(size=(n, k), dtype=np.float64) * sigma).astype(np.float32)
+    w = g.standard_normal(size=(n, k), dtype=np.float32)
+    w *= np.float32(sigma)
+    return w
 
 
 # ----------------------------------------------------------------------------
@@ -144,7 +150,10 @@ def glu_inputs(m: int, f: int, seed: int, gate_shift: float = 0.0):
     optional negative shift of the gate raises the fraction of zero ReLU^2
     outputs toward the paper's reported gate sparsity)."""
     g = rng(seed + 2000)
-    gate = f32_to_bf16_bits((g.standard_normal(size=(m, f)) + gate_shift).astype(np.float32))
+    gate = g.standard_normal(size=(m, f), dtype=np.float32)
+    if gate_shift:
+        gate += np.float32(gate_shift)
+    gate = f32_to_bf16_bits(gate)
     up = gaussian_bf16(g, (m, f))
     return gate, up
 

@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libbitlinear.so")
 BL_OK = 0
 STATUS_NAMES = ["BL_OK", "BL_ERR_NULL", "BL_ERR_ALIGN", "BL_ERR_SHAPE", "BL_ERR_ARG", "BL_ERR_UNSUPPORTED",
                 "BL_ERR_CUDA", "BL_ERR_TIMEOUT", "BL_ERR_WORKSPACE"]
+BL_ERR_CUDA = STATUS_NAMES.index("BL_ERR_CUDA")
 BL_QUANT_INT4, BL_QUANT_FP4_E2M1 = 0, 1
 BL_STORE_PACKED, BL_STORE_BYTES = 0, 1
 BL_A_I8, BL_A_I4, BL_A_E2M1 = 0, 1, 2
@@ -29,16 +30,18 @@ BL_W_T2, BL_W_I8 = 0, 1
 EXPORTED = ["bitlinear_quant_a4", "bitlinear_sparsify_a8", "pack_ternary", "pack_ternary_noalloc", "bitlinear_gemm",
             "relu2_glu",
             "kv_quant3", "bitlinear_workspace_size", "bitlinear_sync_status", "bitlinear_status_string",
-            "bitlinear_version"]
+            "bitlinear_last_cuda_error", "bitlinear_version"]
 
 _lib = None
 
 
 class BitLinearError(RuntimeError):
-    def __init__(self, fn: str, status: int):
+    def __init__(self, fn: str, status: int, cuda_error: str = ""):
         name = STATUS_NAMES[status] if 0 <= status < len(STATUS_NAMES) else f"status {status}"
-        super().__init__(f"{fn} failed: {name}")
+        detail = f" ({cuda_error})" if cuda_error else ""
+        super().__init__(f"{fn} failed: {name}{detail}")
         self.status = status
+        self.cuda_error = cuda_error
 
 
 def lib():
@@ -67,6 +70,8 @@ def lib():
         L.bitlinear_workspace_size.restype = ctypes.c_size_t
         L.bitlinear_status_string.argtypes = [I]
         L.bitlinear_status_string.restype = ctypes.c_char_p
+        L.bitlinear_last_cuda_error.argtypes = []
+        L.bitlinear_last_cuda_error.restype = ctypes.c_char_p
         L.bitlinear_version.argtypes = []
         L.bitlinear_version.restype = ctypes.c_char_p
         _lib = L
@@ -86,7 +91,7 @@ def _stream(stream=None) -> Optional[int]:
 
 def _check(fn: str, rc: int):
     if rc != BL_OK:
-        raise BitLinearError(fn, rc)
+        raise BitLinearError(fn, rc, last_cuda_error() if rc == BL_ERR_CUDA else "")
 
 
 # ---------------------------------------------------------------------------
@@ -163,6 +168,11 @@ def sync_status(stream=None):
 
 def status_string(status: int) -> str:
     return lib().bitlinear_status_string(status).decode()
+
+
+def last_cuda_error() -> str:
+    """Name of the CUDA error behind the last BL_ERR_CUDA on this thread."""
+    return lib().bitlinear_last_cuda_error().decode()
 
 
 def version() -> str:

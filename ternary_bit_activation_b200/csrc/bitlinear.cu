@@ -25,10 +25,18 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
-bl_status launch_status() {
-  const cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+// The last CUDA runtime error that made an entry point of this thread return
+// BL_ERR_CUDA (bitlinear_last_cuda_error reports its name).
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+// true on success; a failure is recorded for bitlinear_last_cuda_error
+bool cuda_ok(cudaError_t e) {
+  if (e == cudaSuccess) return true;
+  t_last_cuda_error = e;
+  return false;
 }
+
+bl_status launch_status() { return cuda_ok(cudaGetLastError()) ? BL_OK : BL_ERR_CUDA; }
 
 int current_device() {
   int d = 0;
@@ -86,11 +94,11 @@ bool tc_kernel_ready() {
   const int d = current_device();
   if (d < 0 || d >= kMaxDevices) return false;
   if (!done[d]) {
-    if (cudaFuncSetAttribute(bl::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(bl::kTcSmemBytes)) != cudaSuccess)
+    if (!cuda_ok(cudaFuncSetAttribute(bl::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(bl::kTcSmemBytes))))
       return false;
-    if (cudaFuncSetAttribute(bl::gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(bl::kT2SmemBytes)) != cudaSuccess)
+    if (!cuda_ok(cudaFuncSetAttribute(bl::gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(bl::kT2SmemBytes))))
       return false;
     done[d] = true;
   }
@@ -125,7 +133,7 @@ bl_status launch_topk_rows_g(const uint16_t* x, const uint16_t* up, int64_t M, i
   const int d = current_device();
   if (d < 0 || d >= kMaxDevices) return BL_ERR_CUDA;
   if (!attr_done[d]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+    if (!cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)))
       return BL_ERR_CUDA;
     attr_done[d] = true;
   }
@@ -156,16 +164,17 @@ bool launch_simt_mu(const uint8_t* a, const float* sc, const uint8_t* w, const f
   const int units_hi = ((K >> 6) + 31) >> 5;
   const size_t smem = static_cast<size_t>(MT) * units_hi * 32 * 16 * sizeof(uint32_t);
   auto kern = bl::gemm_simt_kernel<AF, WT2, MT, UPL>;
-  // the largest tile (K up to 2^20) needs the opt-in shared-memory limit; set it once per device
-  static bool attr_done[kMaxDevices] = {};
+  // Raise the kernel's dynamic shared-memory limit to what this tile needs (once
+  // per size and device).  The default limit counts static shared memory too, and
+  // the kernel holds a 1 KiB static table, so a 48 KiB tile already needs it.
+  static size_t attr_set[kMaxDevices] = {};
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return false;
-  if (!attr_done[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+  if (smem > attr_set[dev]) {
+    if (!cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))))
       return false;
-    attr_done[dev] = true;
+    attr_set[dev] = smem;
   }
-  if (smem > 227 * 1024) return false;
   const int64_t warps_needed = (static_cast<int64_t>(N) + R - 1) / R;
   const int64_t blocks_needed = (warps_needed + 7) / 8;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
@@ -210,7 +219,7 @@ unsigned long long* noalloc_bins_ptr() {
   if (d < 0 || d >= kMaxDevices) return nullptr;
   if (cached[d] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_bins) != cudaSuccess) return nullptr;
+    if (!cuda_ok(cudaGetSymbolAddress(&p, g_noalloc_bins))) return nullptr;
     cached[d] = static_cast<unsigned long long*>(p);
   }
   return cached[d];
@@ -234,7 +243,7 @@ bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int64_t ldw
   if (!alpha_given) {
     unsigned long long* bins = noalloc_bins_ptr();
     if (bins == nullptr) return BL_ERR_CUDA;
-    if (cudaMemsetAsync(bins, 0, sizeof(g_noalloc_bins), s) != cudaSuccess) return BL_ERR_CUDA;
+    if (!cuda_ok(cudaMemsetAsync(bins, 0, sizeof(g_noalloc_bins), s))) return BL_ERR_CUDA;
     const int64_t total = N * (K / 4);
     int64_t blocks = (total + bl::kBinThreads - 1) / bl::kBinThreads;
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
@@ -255,6 +264,8 @@ bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int64_t ldw
     bl::ternary_pack_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
   return launch_status();
 }
+
+const char* bitlinear_last_cuda_error(void) { return cudaGetErrorName(t_last_cuda_error); }
 
 const char* bitlinear_version(void) { return "libbitlinear 0.1 (sm_100a)"; }
 
@@ -280,12 +291,12 @@ size_t bitlinear_workspace_size(const char* op, int64_t M, int64_t N, int64_t K)
 }
 
 bl_status bitlinear_sync_status(void* stream) {
-  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return BL_ERR_CUDA;
+  if (!cuda_ok(cudaStreamSynchronize(as_stream(stream)))) return BL_ERR_CUDA;
   int v = 0;
-  if (cudaMemcpyFromSymbol(&v, bl::g_status, sizeof(int)) != cudaSuccess) return BL_ERR_CUDA;
+  if (!cuda_ok(cudaMemcpyFromSymbol(&v, bl::g_status, sizeof(int)))) return BL_ERR_CUDA;
   if (v != 0) {
     const int zero = 0;
-    if (cudaMemcpyToSymbol(bl::g_status, &zero, sizeof(int)) != cudaSuccess) return BL_ERR_CUDA;
+    if (!cuda_ok(cudaMemcpyToSymbol(bl::g_status, &zero, sizeof(int)))) return BL_ERR_CUDA;
     return static_cast<bl_status>(v);
   }
   return BL_OK;
@@ -358,7 +369,7 @@ bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float 
     if (ws_bytes < bl::kBins * sizeof(unsigned long long)) return BL_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 7u) return BL_ERR_ALIGN;
     unsigned long long* bins = static_cast<unsigned long long*>(workspace);
-    if (cudaMemsetAsync(bins, 0, bl::kBins * sizeof(unsigned long long), s) != cudaSuccess) return BL_ERR_CUDA;
+    if (!cuda_ok(cudaMemsetAsync(bins, 0, bl::kBins * sizeof(unsigned long long), s))) return BL_ERR_CUDA;
     const int64_t total = N * (K / 4);
     int64_t blocks = (total + bl::kBinThreads - 1) / bl::kBinThreads;
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;

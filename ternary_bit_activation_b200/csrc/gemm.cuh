@@ -618,6 +618,9 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const uint8_t* __restric
   constexpr int R = SimtShape<WT2, UPL>::R;
   constexpr int Q = SimtShape<WT2, UPL>::Q;
   extern __shared__ uint32_t sa[];
+  // byte of four 2-bit codes -> four int8 {-1,0,1}: one table read instead of bit arithmetic
+  __shared__ uint32_t t2_table[256];
+  if (WT2) t2_table[threadIdx.x & 255] = expand_t2_byte(threadIdx.x & 255);
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int units = K >> 6;                 // 64 codes per unit
@@ -676,7 +679,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const uint8_t* __restric
 #pragma unroll
               for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
-                for (int b = 0; b < 4; ++b) wx[4 * jj + b] = expand_t2_byte((pk[jj] >> (8 * b)) & 0xFFu);
+                for (int b = 0; b < 4; ++b) wx[4 * jj + b] = t2_table[(pk[jj] >> (8 * b)) & 0xFFu];
             } else {
 #pragma unroll
               for (int q = 0; q < 4; ++q) {

@@ -222,6 +222,17 @@ __global__ void __launch_bounds__(kBins) ternary_alpha_kernel(const unsigned lon
   *alpha = result;
 }
 
+// t = RoundClip(w / (alpha + eps), -1, 1) without the division.  With d = alpha + eps
+// and h = d / 2 (exact while d >= 2^-125): rint(RN(|w|/d)) clipped to 1 is nonzero
+// iff RN(|w|/d) > 1/2, iff |w|/d > 1/2 + 2^-25 (the tie at that midpoint rounds to
+// the even 1/2), iff |w| > h * (1 + 2^-24).  Since h * 2^-24 < ulp(h), for an
+// fp32 |w| that is the same as |w| > h.  So t = sign(w) * [|w| > h].  Smaller d
+// (or an infinite one) keeps the IEEE division.
+__device__ __forceinline__ int ternary_code(float w, float d, float h, bool fast) {
+  if (fast) return fabsf(w) > h ? (w > 0.f ? 1 : -1) : 0;
+  return round_clip(__fdiv_rn(w, d), -1.f, 1.f);
+}
+
 // t = RoundClip(w / (alpha + eps), -1, 1); 16 weights per thread-step.
 //   T2: 4 bytes out (2-bit codes, element 4i in bits 0-1; 0->00, +1->01, -1->11)
 //   I8: 16 bytes out
@@ -230,6 +241,8 @@ __global__ void __launch_bounds__(256) ternary_pack_kernel(const float* __restri
                                                            int64_t ldw, const float* __restrict__ alpha,
                                                            float eps, uint8_t* __restrict__ out) {
   const float d = __fadd_rn(*alpha, eps);
+  const bool fast = d >= 0x1p-125f && d <= 0x1p+127f;   // d/2 exact and normal
+  const float h = __fmul_rn(d, 0.5f);
   const int per_row = K >> 4;   // 16 weights per thread-step
   // rows strided over the grid's warps, 16-weight steps strided over lanes: no integer division
   const int lane = threadIdx.x & 31;
@@ -242,10 +255,10 @@ __global__ void __launch_bounds__(256) ternary_pack_kernel(const float* __restri
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const uint4 v = ld_global_nc_v4(src + 4 * j);
-      c[4 * j + 0] = round_clip(__fdiv_rn(__uint_as_float(v.x), d), -1.f, 1.f);
-      c[4 * j + 1] = round_clip(__fdiv_rn(__uint_as_float(v.y), d), -1.f, 1.f);
-      c[4 * j + 2] = round_clip(__fdiv_rn(__uint_as_float(v.z), d), -1.f, 1.f);
-      c[4 * j + 3] = round_clip(__fdiv_rn(__uint_as_float(v.w), d), -1.f, 1.f);
+      c[4 * j + 0] = ternary_code(__uint_as_float(v.x), d, h, fast);
+      c[4 * j + 1] = ternary_code(__uint_as_float(v.y), d, h, fast);
+      c[4 * j + 2] = ternary_code(__uint_as_float(v.z), d, h, fast);
+      c[4 * j + 3] = ternary_code(__uint_as_float(v.w), d, h, fast);
     }
     if constexpr (T2) {
       uint32_t word = 0;

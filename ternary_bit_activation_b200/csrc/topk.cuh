@@ -245,7 +245,9 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_kernel(
       thr = prefix;
       take = r;
     }
-    const bool partial = take < tie_total;
+    // Ranks among the ties are needed only when some are dropped -- and not when
+    // the tied key is 0 without a mask: a kept zero and a dropped one both get code 0.
+    const bool partial = take < tie_total && (thr != 0u || mask != nullptr);
 
     // ---- codes and mask; ties at the threshold ranked in index order ----
     // chunk q = tid + c*GT, so index order is slot c first, then thread.  When
