@@ -118,42 +118,30 @@ void launch_quant_a4_c(const uint16_t* x, int64_t M, int K, int64_t ldx, bool fp
   if (fp4 && !packed) bl::quant_a4_kernel<C, true, false><<<grid, 256, 0, s>>>(x, M, K, ldx, eps, codes, scale);
 }
 
-// Top-K rows: groups of G warps per row (shared-memory row buffer), persistent
-// grid sized by the occupancy the buffer allows.
-template <int G, bool RELU2>
-bl_status launch_topk_rows_g(const uint16_t* x, const uint16_t* up, int64_t M, int K, int64_t ldx, int keep,
-                             float eps, int8_t* codes, float* scale, uint32_t* mask, cudaStream_t s) {
-  constexpr int kGroups = bl::kRowThreads / (G * 32);
-  const int row_words = (K / 8) * (RELU2 ? 2 : 1);
-  const size_t smem = static_cast<size_t>(kGroups) *
-                      (sizeof(bl::GroupSmem) + static_cast<size_t>(row_words) * 16 + (RELU2 ? bl::kRowListCap * 4 : 0));
-  if (smem > 227 * 1024) return BL_ERR_SHAPE;
-  auto kern = bl::topk_rows_kernel<G, RELU2>;
-  static bool attr_done[kMaxDevices] = {};
-  const int d = current_device();
-  if (d < 0 || d >= kMaxDevices) return BL_ERR_CUDA;
-  if (!attr_done[d]) {
-    if (!cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)))
-      return BL_ERR_CUDA;
-    attr_done[d] = true;
-  }
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, bl::kRowThreads, smem) != cudaSuccess ||
-      per_sm < 1)
-    per_sm = 1;
-  const int64_t need = (M + kGroups - 1) / kGroups;
-  const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
-  const unsigned grid = static_cast<unsigned>(need < cap ? need : cap);
-  kern<<<grid, bl::kRowThreads, smem, s>>>(x, up, M, K, ldx, keep, eps, codes, scale, mask, row_words);
-  return launch_status();
-}
-
+// Top-K rows: one 256-thread CTA per row, persistent grid sized by the occupancy
+// that the shared-memory row stages allow.
 template <bool RELU2>
 bl_status launch_topk_rows(const uint16_t* x, const uint16_t* up, int64_t M, int K, int64_t ldx, int keep,
                            float eps, int8_t* codes, float* scale, uint32_t* mask, cudaStream_t s) {
-  if (K <= 4096) return launch_topk_rows_g<1, RELU2>(x, up, M, K, ldx, keep, eps, codes, scale, mask, s);
-  if (K <= 8192) return launch_topk_rows_g<2, RELU2>(x, up, M, K, ldx, keep, eps, codes, scale, mask, s);
-  return launch_topk_rows_g<4, RELU2>(x, up, M, K, ldx, keep, eps, codes, scale, mask, s);
+  const size_t smem = bl::tk_smem_bytes<RELU2>(K);
+  if (smem > 227 * 1024) return BL_ERR_SHAPE;
+  auto kern = bl::topk_rows_kernel<RELU2>;
+  static size_t attr_set[kMaxDevices] = {};
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return BL_ERR_CUDA;
+  if (smem > attr_set[d]) {
+    if (!cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))))
+      return BL_ERR_CUDA;
+    attr_set[d] = smem;
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, bl::kTkThreads, smem) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
+  const unsigned grid = static_cast<unsigned>(M < cap ? M : cap);
+  kern<<<grid, bl::kTkThreads, smem, s>>>(x, up, M, K, ldx, keep, eps, codes, scale, mask);
+  return launch_status();
 }
 
 

@@ -2,287 +2,352 @@
 // §3.4, Eq. 1 with Q_INT8), for the raw bf16 inputs (sparsify_a8) and for the
 // ReLU^2-GLU output h = up * max(0, gate)^2 in fp32 (Eq. 5, relu2_glu).
 //
-// One group of G warps handles one row; a 256-thread CTA holds 8/G groups that
-// share nothing but the CTA.  The row is copied once from HBM into the group's
-// shared memory (bf16 for sparsify, the fp32 h for relu2), so the selection
-// passes read shared memory, registers stay few and many rows are in flight per
-// SM.  Groups synchronize with their own named barrier (or a warp barrier).
+// One 256-thread CTA owns one row at a time (persistent over rows).  Rows stream
+// through a double-buffered shared-memory stage (cp.async, 16 B per copy): the
+// next row is in flight while the current one is ranked and quantized, so HBM is
+// read once per element and stays busy.  For ReLU^2 rows the first sweep writes
+// h over the staged gate/up values of its own chunk, so later sweeps read h.
 //
 // Selection: exactly `keep` survivors ranked by magnitude, ties to the lower
-// index.  If at most `keep` magnitudes are nonzero the threshold is 0 (every
-// nonzero survives, zeros fill the rest in index order).  Otherwise an MSD
-// radix select over the nonzero keys finds the keep-th largest key; with fp32
-// keys the candidates left after the first digit are compacted into a short
-// list that the remaining passes read.
+// index.  The keep-th largest magnitude key is found by an MSD radix select:
+// bf16 keys (15 bits) take an 8-bit then a 7-bit digit (the first counted in the
+// same sweep that finds the row maximum); fp32 keys (31 bits) take 8, 8, 8 and
+// 7 bits, and once two digits are fixed the few candidates left go to a short
+// list that the last passes read.  A full-row pass counts digits with shared
+// atomics into lane-private counter words (word bin*32 + lane for bf16, two
+// 16-bit bins per word for fp32), so a warp's 32 lanes always hit 32 different
+// banks; thread t then sums bin t over the 32 lane columns.  ReLU^2 rows with
+// at most `keep` nonzero values need no pass: every nonzero survives and zeros
+// fill the rest in index order.
 #pragma once
 
 #include "common.cuh"
 
 namespace bl {
 
-constexpr int kRowThreads = 256;          // threads per CTA
-constexpr int kRowListCap = 1024;         // compacted candidates (fp32 keys)
+constexpr int kTkThreads = 256;            // one row per CTA
+constexpr int kTkMaxSlots = 8;             // chunks of 8 values per thread and row (K <= 16384)
+constexpr int kTkListCap = 1024;           // fp32 candidates once two digits are fixed
 
 template <bool F32>
-struct RowTraits {
-  static constexpr int kElemBytes = F32 ? 4 : 2;
-  static constexpr int kPasses = F32 ? 4 : 2;
+struct __align__(16) TkShared {
+  uint32_t cnt[F32 ? 2048 : 4096];         // 256 bins x 16 columns (u32, or u16 pairs for fp32)
+  uint32_t tot[256];                       // bin totals of the current pass
+  uint32_t red[8][2];                      // per-warp max key / nonzero count
+  int32_t ties[8][kTkMaxSlots];            // ties at the threshold per (warp, slot)
+  uint32_t sel[4];                         // selected digit, count above it, its count
+  uint32_t hist[2][F32 ? 256 : 1];         // list passes (fp32 keys)
+  uint32_t list_n;
+  uint32_t list[F32 ? kTkListCap : 1];
 };
 
-// Per-group shared state, followed in memory by the row values.
-struct GroupSmem {
-  uint32_t hist[256];
-  uint32_t red[8];          // per-warp partials (max key / nonzero count / tie totals)
-  uint32_t red2[8];
-  uint32_t sel_digit, sel_above, sel_count, list_n;
-  int32_t tie_tot[64];      // ties per (warp in group, chunk slot): [warp * slots + slot]; G * slots <= 64
-};
-
-template <int G>
-__device__ __forceinline__ void group_sync(int gid) {
-  if constexpr (G == 1) {
-    __syncwarp();
-  } else {
-    asm volatile("bar.sync %0, %1;" ::"r"(1 + gid), "r"(G * 32) : "memory");
-  }
-}
-
+// Bytes of dynamic shared memory for rows of K values.
 template <bool F32>
-__device__ __forceinline__ void chunk_keys(const uint4* vals, uint32_t (&k)[8]) {
-  if constexpr (F32) {
-    const uint4 a = vals[0], b = vals[1];
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int e = 0; e < 8; ++e) k[e] = w[e] & 0x7FFFFFFFu;
-  } else {
-    bf16x8_mag_keys(vals[0], k);
-  }
+inline size_t tk_smem_bytes(int K) {
+  return sizeof(TkShared<F32>) + 2 * static_cast<size_t>(F32 ? 2 : 1) * static_cast<size_t>(K) * 2;
 }
 
+// Counter update: `inc` (0 or 1) for digit `bin`.  Lanes l and l+16 share a
+// counter column; a warp's other lanes hit 16 different banks.
 template <bool F32>
-__device__ __forceinline__ void chunk_values(const uint4* vals, float (&f)[8]) {
+__device__ __forceinline__ void tk_count(uint32_t* cnt, uint32_t bin, int col, uint32_t inc) {
   if constexpr (F32) {
-    const uint4 a = vals[0], b = vals[1];
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(w[e]);
+    atomicAdd(&cnt[((bin >> 1) << 4) + col], inc << ((bin & 1u) << 4));   // two 16-bit bins per word
   } else {
-    unpack_bf16x8(vals[0], f);
+    atomicAdd(&cnt[(bin << 4) + col], inc);
   }
 }
 
-// Within one warp: digit d with above(d) < r <= above(d) + hist[d], counting
-// from the top (above(d) = candidates with a larger digit); zeroes the
-// histogram.  Lane l owns bins l, l+32, ... (conflict-free).
-__device__ __forceinline__ void warp_select_digit(uint32_t* hist, int nbins, uint32_t r, GroupSmem& gs) {
-  const int lane = threadIdx.x & 31;
-  const int slots = nbins / 32;
-  uint32_t h[8];
+// Sum of bin b over the 16 counter columns, the column order rotated so that
+// the 32 lanes of a warp read 32 banks (lanes 2m and 2m+1 share words for fp32).
+template <bool F32>
+__device__ __forceinline__ uint32_t tk_bin_total(const uint32_t* cnt, uint32_t b, int lane) {
+  uint32_t s = 0;
+  const int rot = lane >> 1;
+  if constexpr (F32) {
+    const uint32_t* w = cnt + ((b >> 1) << 4);
+    const int sh = (b & 1u) ? 16 : 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    h[i] = 0;
-    if (i < slots) {
-      h[i] = hist[32 * i + lane];
-      hist[32 * i + lane] = 0;
-    }
+    for (int j = 0; j < 16; ++j) s += (w[(rot + j) & 15] >> sh) & 0xFFFFu;
+  } else {
+    const uint32_t* w = cnt + (b << 4);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) s += w[(rot + j) & 15];
   }
-  uint32_t above_slots = 0;
+  return s;
+}
+
+// Within one warp: the digit d with above(d) < r <= above(d) + count(d),
+// counting from the largest digit; t[i] = count of bin 8*lane + i.
+// Lane 0 of the warp returns the result in out[0..2].
+__device__ __forceinline__ void tk_select(const uint32_t (&t)[8], uint32_t r, int lane, uint32_t* out) {
+  uint32_t s = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s += t[i];
+  uint32_t incl = s;                       // sum over lanes >= lane
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, incl, o);
+    if (lane + o < 32) incl += v;
+  }
+  uint32_t above = incl - s;
 #pragma unroll
   for (int i = 7; i >= 0; --i) {
-    if (i >= slots) continue;
-    uint32_t inc = h[i];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t other = __shfl_down_sync(0xFFFFFFFFu, inc, o);
-      if (lane + o < 32) inc += other;
+    if (above < r && r <= above + t[i]) {
+      out[0] = static_cast<uint32_t>(8 * lane + i);
+      out[1] = above;
+      out[2] = t[i];
     }
-    const uint32_t above = above_slots + inc - h[i];
-    if (above < r && r <= above + h[i]) {
-      gs.sel_digit = static_cast<uint32_t>(32 * i + lane);
-      gs.sel_above = above;
-      gs.sel_count = h[i];
-    }
-    above_slots += __shfl_sync(0xFFFFFFFFu, inc, 0);
+    above += t[i];
   }
 }
 
-// G warps per row.  RELU2: values are h computed from gate/up; otherwise the
-// bf16 input row.  Chunk q (8 consecutive values) of a row belongs to thread
-// q % (32G); the row lives in shared memory as chunk-major 16-byte words.
-template <int G, bool RELU2>
-__global__ void __launch_bounds__(kRowThreads) topk_rows_kernel(
+// Low byte of the bits of RN(RN(v*mult) + 1.5*2^23): the code RoundClip(v*mult)
+// for |v*mult| <= 127 (the sum's ulp is 1, so it rounds half to even; the
+// product is rounded first, as the quantizer prescribes).
+__device__ __forceinline__ uint32_t tk_code_bits(float v, float mult) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(v, mult), 12582912.0f));
+}
+
+// Bytes e of lo/hi = code of value e when bit e of `bits` is set, else 0.
+__device__ __forceinline__ uint2 tk_pack_codes(const uint32_t (&cb)[8], uint32_t bits) {
+  const uint32_t lo = __byte_perm(__byte_perm(cb[0], cb[1], 0x0040), __byte_perm(cb[2], cb[3], 0x0040), 0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(cb[4], cb[5], 0x0040), __byte_perm(cb[6], cb[7], 0x0040), 0x5410);
+  // spread 4 mask bits to 4 bytes of 0x01, then to 0xFF
+  const uint32_t ml = ((((bits & 0xFu) * 0x00204081u) & 0x01010101u) * 0xFFu);
+  const uint32_t mh = (((((bits >> 4) & 0xFu) * 0x00204081u) & 0x01010101u) * 0xFFu);
+  return make_uint2(lo & ml, hi & mh);
+}
+
+template <bool F32>
+__device__ __forceinline__ void tk_keys(const uint4* st, int q, int row_words, uint32_t (&k)[8], float (&f)[8]) {
+  if constexpr (F32) {
+    const uint4 a = st[q], b = st[row_words + q];   // h written in place: values 0-3, then 4-7
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      f[e] = __uint_as_float(w[e]);
+      k[e] = w[e] & 0x7FFFFFFFu;
+    }
+  } else {
+    const uint4 v = st[q];
+    unpack_bf16x8(v, f);
+    bf16x8_mag_keys(v, k);
+  }
+}
+
+template <bool F32>
+__global__ void __launch_bounds__(kTkThreads, F32 ? 2 : 4) topk_rows_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ up, int64_t M, int K, int64_t ldx, int keep,
-    float eps, int8_t* __restrict__ codes, float* __restrict__ scale, uint32_t* __restrict__ mask,
-    int row_words /* 16-byte words of one row's values in shared memory */) {
-  constexpr bool F32 = RELU2;
-  constexpr int GT = G * 32;
-  constexpr int kWpc = F32 ? 2 : 1;                    // 16-byte words per chunk
-  constexpr int kGroups = kRowThreads / GT;
-  extern __shared__ uint4 dyn[];
-  const int gid = threadIdx.x / GT;
-  const int tid = threadIdx.x % GT;
-  const int lane = threadIdx.x & 31;
-  const int wig = tid >> 5;                            // warp in group
-  GroupSmem* gsm = reinterpret_cast<GroupSmem*>(dyn);
-  GroupSmem& gs = gsm[gid];
-  uint4* vals = reinterpret_cast<uint4*>(gsm + kGroups) + static_cast<int64_t>(gid) * row_words;
-  uint32_t* list = reinterpret_cast<uint32_t*>(reinterpret_cast<uint4*>(gsm + kGroups) +
-                                               static_cast<int64_t>(kGroups) * row_words) +
-                   gid * kRowListCap;
+    float eps, int8_t* __restrict__ codes, float* __restrict__ scale, uint32_t* __restrict__ mask) {
+  extern __shared__ __align__(16) uint8_t tk_dyn[];
+  TkShared<F32>& sm = *reinterpret_cast<TkShared<F32>*>(tk_dyn);
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int wig = tid >> 5;
+  const int nchunk = K >> 3;                       // 16-byte bf16 words per input row
+  const int row_words = nchunk;
+  const int stage_words = F32 ? 2 * row_words : row_words;
+  uint4* stages = reinterpret_cast<uint4*>(tk_dyn + sizeof(TkShared<F32>));
+  const int slots = (nchunk + kTkThreads - 1) / kTkThreads;
+  const int mwords = (K + 31) >> 5;
+  constexpr int kCntWords = F32 ? 2048 : 4096;
+  const int col = lane & 15;
 
-  const int nchunk = K >> 3;
-  const int my_chunks = (nchunk - tid + GT - 1) / GT;   // chunks q = tid + c*GT, c < my_chunks
+  auto prefetch = [&](int64_t r, int buf) {
+    if (r < M) {
+      uint4* dst = stages + buf * stage_words;
+      const uint16_t* src = x + r * ldx;
+      for (int i = tid; i < row_words; i += kTkThreads) cp_async_16(dst + i, src + static_cast<int64_t>(i) * 8);
+      if constexpr (F32) {
+        const uint16_t* usrc = up + r * ldx;
+        for (int i = tid; i < row_words; i += kTkThreads)
+          cp_async_16(dst + row_words + i, usrc + static_cast<int64_t>(i) * 8);
+      }
+    }
+    cp_async_commit();
+  };
+  auto zero_counters = [&]() {
+    for (int i = tid; i < kCntWords / 4; i += kTkThreads) reinterpret_cast<uint4*>(sm.cnt)[i] = make_uint4(0, 0, 0, 0);
+  };
 
-  for (int i = tid; i < 256; i += GT) gs.hist[i] = 0;
+  zero_counters();
+  int64_t row = blockIdx.x;
+  prefetch(row, 0);
+  int buf = 0;
+  for (; row < M; row += gridDim.x, buf ^= 1) {
+    prefetch(row + gridDim.x, buf ^ 1);
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+    __syncthreads();
+    uint4* st = stages + buf * stage_words;
 
-  for (int64_t row = static_cast<int64_t>(blockIdx.x) * kGroups + gid; row < M;
-       row += static_cast<int64_t>(gridDim.x) * kGroups) {
-    // ---- copy the row into shared memory; max key and nonzero count ----
+    // ---- sweep 1: max key; bf16 counts its first digit, fp32 writes h and counts nonzeros ----
     uint32_t mk = 0, nz = 0;
-    {
-      const uint16_t* xr = x + row * ldx;
-      const uint16_t* ur = RELU2 ? up + row * ldx : nullptr;
-#pragma unroll 4
-      for (int c = 0; c < my_chunks; ++c) {
-        const int q = tid + c * GT;
-        if constexpr (RELU2) {
-          const uint4 gv = ld_global_nc_v4(xr + static_cast<int64_t>(q) * 8);
-          const uint4 uv = ld_global_nc_v4(ur + static_cast<int64_t>(q) * 8);
-          float g[8], u[8];
-          unpack_bf16x8(gv, g);
-          unpack_bf16x8(uv, u);
-          uint32_t hb[8];
+    for (int q = tid; q < nchunk; q += kTkThreads) {
+      if constexpr (F32) {
+        const uint4 gv = st[q], uv = st[row_words + q];
+        float g[8], u[8];
+        unpack_bf16x8(gv, g);
+        unpack_bf16x8(uv, u);
+        uint32_t hb[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float rg = g[e] > 0.f ? g[e] : 0.f;
-            hb[e] = __float_as_uint(__fmul_rn(u[e], __fmul_rn(rg, rg)));
-            const uint32_t key = hb[e] & 0x7FFFFFFFu;
-            mk = max(mk, key);
-            nz += key != 0u;
-          }
-          vals[q * 2] = make_uint4(hb[0], hb[1], hb[2], hb[3]);
-          vals[q * 2 + 1] = make_uint4(hb[4], hb[5], hb[6], hb[7]);
-        } else {
-          const uint4 v = ld_global_nc_v4(xr + static_cast<int64_t>(q) * 8);
-          uint32_t k[8];
-          bf16x8_mag_keys(v, k);
+        for (int e = 0; e < 8; ++e) {
+          const float rg = fmaxf(g[e], 0.f);
+          hb[e] = __float_as_uint(__fmul_rn(u[e], __fmul_rn(rg, rg)));
+          const uint32_t key = hb[e] & 0x7FFFFFFFu;
+          mk = max(mk, key);
+          nz += key != 0u ? 1u : 0u;
+        }
+        st[q] = make_uint4(hb[0], hb[1], hb[2], hb[3]);
+        st[row_words + q] = make_uint4(hb[4], hb[5], hb[6], hb[7]);
+      } else {
+        const uint4 v = st[q];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            mk = max(mk, k[e]);
-            nz += k[e] != 0u;
-          }
-          vals[q] = v;
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t klo = w[i] & 0x7FFFu, khi = (w[i] >> 16) & 0x7FFFu;
+          mk = max(mk, max(klo, khi));
+          tk_count<false>(sm.cnt, klo >> 7, col, 1u);
+          tk_count<false>(sm.cnt, khi >> 7, col, 1u);
         }
       }
     }
     mk = __reduce_max_sync(0xFFFFFFFFu, mk);
     nz = __reduce_add_sync(0xFFFFFFFFu, nz);
     if (lane == 0) {
-      gs.red[wig] = mk;
-      gs.red2[wig] = nz;
+      sm.red[wig][0] = mk;
+      sm.red[wig][1] = nz;
     }
-    if (tid == 0) gs.list_n = 0;
-    group_sync<G>(gid);
-    uint32_t gk = 0, nnz = 0;
+    __syncthreads();
+    mk = 0;
+    nz = 0;
 #pragma unroll
-    for (int w = 0; w < G; ++w) {
-      gk = max(gk, gs.red[w]);
-      nnz += gs.red2[w];
+    for (int w = 0; w < 8; ++w) {
+      mk = max(mk, sm.red[w][0]);
+      nz += sm.red[w][1];
     }
 
-    // ---- threshold key `thr`; `take` elements equal to it survive ----
-    uint32_t thr, take, tie_total;
-    if (nnz <= static_cast<uint32_t>(keep)) {
-      thr = 0;
-      take = static_cast<uint32_t>(keep) - nnz;
-      tie_total = static_cast<uint32_t>(K) - nnz;
+    // ---- threshold key `thr`; the first `take` (index order) of its ties survive ----
+    uint32_t thr = 0, take = 0, tie_total = 0;
+    const bool all_kept = keep >= K;
+    bool counted = !F32;                         // counters hold this row's first digit
+    if (all_kept) {
+      // every element survives
+    } else if (F32 && nz <= static_cast<uint32_t>(keep)) {
+      take = static_cast<uint32_t>(keep) - nz;
+      tie_total = static_cast<uint32_t>(K) - nz;
     } else {
       uint32_t prefix = 0, fixed = 0, r = static_cast<uint32_t>(keep);
+      constexpr int kPasses = F32 ? 4 : 2;
       bool listed = false;
-      tie_total = 0;
 #pragma unroll 1
-      for (int pass = 0; pass < RowTraits<F32>::kPasses; ++pass) {
-        const int shift = F32 ? max(23 - 8 * pass, 0) : 7 - 7 * pass;
-        const int width = shift == 0 ? 7 : 8;
-        const uint32_t dmask = (1u << width) - 1u;
-        if (listed) {
-          const int n = static_cast<int>(gs.list_n);
-          for (int i = tid; i < n; i += GT) {
-            const uint32_t key = list[i];
-            if ((key & fixed) == prefix) atomicAdd(&gs.hist[(key >> shift) & dmask], 1u);
-          }
-        } else {
-#pragma unroll 2
-          for (int c = 0; c < my_chunks; ++c) {
-            uint32_t k[8];
-            chunk_keys<F32>(vals + (tid + c * GT) * kWpc, k);
+      for (int pass = 0; pass < kPasses; ++pass) {
+        const int shift = F32 ? (pass == 3 ? 0 : 23 - 8 * pass) : (pass == 0 ? 7 : 0);
+        const uint32_t dmask = shift == 0 ? 0x7Fu : 0xFFu;
+        if (!listed) {
+          if (!counted) {
+            for (int q = tid; q < nchunk; q += kTkThreads) {
+              uint32_t k[8];
+              float f[8];
+              tk_keys<F32>(st, q, row_words, k, f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              if (k[e] != 0u && (k[e] & fixed) == prefix) atomicAdd(&gs.hist[(k[e] >> shift) & dmask], 1u);
+              for (int e = 0; e < 8; ++e)
+                tk_count<F32>(sm.cnt, (k[e] >> shift) & dmask, col, (k[e] & fixed) == prefix ? 1u : 0u);
+            }
+            __syncthreads();
+          }
+          sm.tot[tid] = tk_bin_total<F32>(sm.cnt, static_cast<uint32_t>(tid), lane);
+          __syncthreads();
+          // warp 0 picks the digit while the others clear the counters
+          if (wig == 0) {
+            uint32_t t[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) t[i] = sm.tot[8 * lane + i];
+            tk_select(t, r, lane, sm.sel);
+          } else {
+            for (int i = tid - 32; i < kCntWords / 4; i += kTkThreads - 32)
+              reinterpret_cast<uint4*>(sm.cnt)[i] = make_uint4(0, 0, 0, 0);
+          }
+          counted = false;
+        } else {
+          // candidates in the list: a shared histogram
+          uint32_t* h = sm.hist[pass & 1];
+          const int n = static_cast<int>(sm.list_n);
+          for (int i = tid; i < n; i += kTkThreads) {
+            const uint32_t key = sm.list[i];
+            if ((key & fixed) == prefix) atomicAdd(&h[(key >> shift) & dmask], 1u);
+          }
+          __syncthreads();
+          if (wig == 0) {
+            uint32_t t[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) t[i] = h[8 * lane + i];
+            tk_select(t, r, lane, sm.sel);
           }
         }
-        group_sync<G>(gid);
-        if (wig == 0) warp_select_digit(gs.hist, 1 << width, r, gs);
-        group_sync<G>(gid);
-        r -= gs.sel_above;
-        tie_total = gs.sel_count;
-        prefix |= gs.sel_digit << shift;
+        __syncthreads();
+        r -= sm.sel[1];
+        tie_total = sm.sel[2];
+        prefix |= sm.sel[0] << shift;
         fixed |= dmask << shift;
-        if (F32 && pass == 0 && tie_total <= static_cast<uint32_t>(kRowListCap)) {
-          // candidates left after the top digit -> list (read by the remaining passes)
-#pragma unroll 2
-          for (int c = 0; c < my_chunks; ++c) {
+        if (F32 && pass == 1 && tie_total <= static_cast<uint32_t>(kTkListCap)) {
+          // two digits fixed: the remaining candidates go to the list
+          if (tid == 0) sm.list_n = 0;
+          for (int i = tid; i < 512; i += kTkThreads) (&sm.hist[0][0])[i] = 0;
+          __syncthreads();
+          for (int q = tid; q < nchunk; q += kTkThreads) {
             uint32_t k[8];
-            chunk_keys<F32>(vals + (tid + c * GT) * kWpc, k);
+            float f[8];
+            tk_keys<F32>(st, q, row_words, k, f);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-              if (k[e] != 0u && (k[e] & fixed) == prefix) list[atomicAdd(&gs.list_n, 1u)] = k[e];
+              if ((k[e] & fixed) == prefix) sm.list[atomicAdd(&sm.list_n, 1u)] = k[e];
           }
-          group_sync<G>(gid);
+          __syncthreads();
           listed = true;
         }
       }
       thr = prefix;
       take = r;
     }
+    if (counted) {
+      // a bf16 row that needed no selection: its first-digit counts are discarded
+      __syncthreads();
+      zero_counters();
+    }
     // Ranks among the ties are needed only when some are dropped -- and not when
     // the tied key is 0 without a mask: a kept zero and a dropped one both get code 0.
-    const bool partial = take < tie_total && (thr != 0u || mask != nullptr);
+    const bool partial = !all_kept && take < tie_total && (thr != 0u || mask != nullptr);
 
-    // ---- codes and mask; ties at the threshold ranked in index order ----
-    // chunk q = tid + c*GT, so index order is slot c first, then thread.  When
-    // some ties are dropped, pass A publishes each warp's tie count per slot;
-    // pass B re-scans its lanes to rank them.
-    const float gamma = F32 ? __uint_as_float(gk) : __uint_as_float(gk << 16);
-    const float mult = __fdiv_rn(127.f, __fadd_rn(gamma, eps));
+    // ---- codes and mask ----
+    const float gamma = F32 ? __uint_as_float(mk) : __uint_as_float(mk << 16);
+    const float denom = __fadd_rn(gamma, eps);
+    const float mult = denom > 0.f ? __fdiv_rn(127.f, denom) : 0.f;
     if (tid == 0) scale[row] = __fdiv_rn(gamma, 127.f);
-    const int slots = (nchunk + GT - 1) / GT;
-    const int mwords = (K + 31) >> 5;
     if (partial) {
-#pragma unroll 1
       for (int c = 0; c < slots; ++c) {
-        int cnt = 0;
-        if (c < my_chunks) {
+        const int q = tid + c * kTkThreads;
+        int n = 0;
+        if (q < nchunk) {
           uint32_t k[8];
-          chunk_keys<F32>(vals + (tid + c * GT) * kWpc, k);
+          float f[8];
+          tk_keys<F32>(st, q, row_words, k, f);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) cnt += k[e] == thr;
+          for (int e = 0; e < 8; ++e) n += k[e] == thr ? 1 : 0;
         }
-        cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
-        if (lane == 0) gs.tie_tot[wig * slots + c] = cnt;
+        n = __reduce_add_sync(0xFFFFFFFFu, n);
+        if (lane == 0) sm.ties[wig][c] = n;
       }
-      group_sync<G>(gid);
+      __syncthreads();
     }
-    int slot_base = 0;   // ties in earlier slots, all threads of the group
-#pragma unroll 1
+    uint32_t before = 0;   // ties in earlier slots, over the whole row
     for (int c = 0; c < slots; ++c) {
-      const int q = tid + c * GT;
-      const bool ok = c < my_chunks;
+      const int q = tid + c * kTkThreads;
+      const bool ok = q < nchunk;
       uint32_t k[8];
       float f[8];
       if (ok) {
-        chunk_keys<F32>(vals + q * kWpc, k);
-        chunk_values<F32>(vals + q * kWpc, f);
+        tk_keys<F32>(st, q, row_words, k, f);
       } else {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -290,43 +355,52 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_kernel(
           f[e] = 0.f;
         }
       }
-      int rank = 0;
-      if (partial) {
-        int cnt = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) cnt += ok && k[e] == thr;
-        int inc = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int other = __shfl_up_sync(0xFFFFFFFFu, inc, o);
-          if (lane >= o) inc += other;
-        }
-        int before = 0, total = 0;
-#pragma unroll
-        for (int w = 0; w < G; ++w) {
-          const int tw = gs.tie_tot[w * slots + c];
-          before += w < wig ? tw : 0;
-          total += tw;
-        }
-        rank = slot_base + before + inc - cnt;
-        slot_base += total;
-      }
       uint32_t bits = 0;
-      uint2 w2 = make_uint2(0, 0);
+      if (!partial) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        bool keepit = k[e] > thr;
-        if (k[e] == thr) {
-          keepit = !partial || rank < static_cast<int>(take);
-          ++rank;
+        for (int e = 0; e < 8; ++e) bits |= (k[e] >= thr ? 1u : 0u) << e;
+      } else {
+        // ties in this chunk: all kept, all dropped, or ranked (the slot holding the cut)
+        uint32_t slot_total = 0, warps_before = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          const uint32_t tw = static_cast<uint32_t>(sm.ties[w][c]);
+          slot_total += tw;
+          warps_before += w < wig ? tw : 0u;
         }
-        keepit = keepit && ok;
-        const int code = keepit ? round_clip(__fmul_rn(f[e], mult), -128.f, 127.f) : 0;
-        bits |= (keepit ? 1u : 0u) << e;
-        const uint32_t b = static_cast<uint32_t>(code) & 0xFFu;
-        if (e < 4) w2.x |= b << (8 * e); else w2.y |= b << (8 * (e - 4));
+        const bool keep_all = before + slot_total <= take;
+        const bool drop_all = before >= take;
+        int rank = 0;
+        if (!keep_all && !drop_all) {
+          int mine = 0;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mine += (ok && k[e] == thr) ? 1 : 0;
+          int inc = mine;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int other = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+            if (lane >= o) inc += other;
+          }
+          rank = static_cast<int>(before + warps_before) + inc - mine;
+        }
+        const uint32_t tie_ok = keep_all ? 1u : 0u;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t eq = k[e] == thr ? 1u : 0u;
+          const uint32_t ranked = (!drop_all && rank < static_cast<int>(take)) ? 1u : 0u;
+          const uint32_t kp = (k[e] > thr ? 1u : 0u) | (eq & (tie_ok | ranked));
+          rank += static_cast<int>(eq);
+          bits |= kp << e;
+        }
+        before += slot_total;
       }
-      if (ok) reinterpret_cast<uint2*>(codes + row * static_cast<int64_t>(K))[q] = w2;
+      if (!ok) bits = 0;
+      if (ok) {
+        uint32_t cb[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) cb[e] = tk_code_bits(f[e], mult);
+        reinterpret_cast<uint2*>(codes + row * static_cast<int64_t>(K))[q] = tk_pack_codes(cb, bits);
+      }
       if (mask != nullptr) {
         // chunks q..q+3 (lanes 4i..4i+3 of one slot) form one 32-bit mask word
         const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, bits, 1);
@@ -335,8 +409,9 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_kernel(
         if (ok && (lane & 3) == 0) mask[row * mwords + (q >> 2)] = bits | (b1 << 8) | (b2 << 16) | (b3 << 24);
       }
     }
-    group_sync<G>(gid);   // the row buffer and group state are reused by the next row
+    __syncthreads();   // the stage and the shared state are reused
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 }  // namespace bl

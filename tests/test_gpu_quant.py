@@ -111,6 +111,10 @@ TOPK_CASES = [
     ("keep1", lambda: synth.student_t_bf16(synth.rng(15), (6, 512)), 1),
     ("keep_all", lambda: synth.student_t_bf16(synth.rng(16), (6, 512)), 512),
     ("K40_ragged_mask_word", lambda: synth.student_t_bf16(synth.rng(17), (9, 40)), 13),
+    ("K4096_7B_O", lambda: synth.student_t_bf16(synth.rng(19), (12, 4096)), 2048),
+    ("K4104_two_warps", lambda: synth.student_t_bf16(synth.rng(20), (5, 4104)), 2052),
+    ("K16384_four_warps", lambda: synth.student_t_bf16(synth.rng(21), (3, 16384)), 8192),
+    ("gaussian_keep_small", lambda: synth.gaussian_bf16(synth.rng(22), (9, 1024)), 37),
 ]
 
 
@@ -129,6 +133,16 @@ def test_sparsify_a8_heavy_ties():
     x[2, :] = synth.f32_to_bf16_bits(np.round(synth.bf16_bits_to_f32(x[2]) * 2) / 2)   # coarse grid
     x[3, :1500] = 0x8000                                                           # -0 and +0 tie
     for keep in (1, 700, 1024, 1500, 2047):
+        codes, scale, mask = run_sparsify(x, keep)
+        check_topk(codes, scale, mask, oracle.sparsify_a8(x, keep, EPS))
+
+
+def test_sparsify_a8_zero_and_constant_rows():
+    x = synth.student_t_bf16(synth.rng(23), (4, 4096))
+    x[0] = 0                                                  # gamma = 0: every code 0
+    x[1] = synth.f32_to_bf16_bits(np.full(4096, -3.0, np.float32))
+    x[2, 100:] = 0
+    for keep in (1, 50, 100, 2048, 4095, 4096):
         codes, scale, mask = run_sparsify(x, keep)
         check_topk(codes, scale, mask, oracle.sparsify_a8(x, keep, EPS))
 
@@ -156,6 +170,11 @@ RELU_CASES = [
     ("7B_F11008", 6, 11008, 5504, -0.454),
     ("keep_all", 8, 1024, 1024, 0.0),
     ("F40_ragged", 5, 40, 7, 0.0),
+    ("F2048_one_warp_select", 7, 2048, 300, 0.0),
+    ("F11008_select_nonzero", 5, 11008, 2000, 0.0),
+    ("F11008_half", 6, 11008, 5504, 0.0),
+    ("F12296_eight_warps", 3, 12296, 6148, 0.0),
+    ("F16384_max", 3, 16384, 8192, -0.454),
 ]
 
 
@@ -164,6 +183,31 @@ def test_relu2_glu_parity(name, M, F, keep, shift):
     gate, up = synth.glu_inputs(M, F, seed=F + M, gate_shift=shift)
     codes, scale, mask = run_relu2(gate, up, keep, ld_pad=8)
     check_topk(codes, scale, mask, oracle.relu2_glu(gate, up, keep, EPS))
+
+
+def test_relu2_glu_ties_and_no_mask():
+    M, F = 6, 4096
+    gate, up = synth.glu_inputs(M, F, seed=99, gate_shift=0.0)
+    one = synth.f32_to_bf16_bits(np.full(F, 1.0, np.float32))
+    gate[0], up[0] = one, one                                  # every h equal: no list, all ties
+    up[1] = synth.f32_to_bf16_bits(np.round(synth.bf16_bits_to_f32(up[1]) * 4) / 4)   # coarse: many ties
+    gate[2] = 0                                                # all h zero
+    gate[3, ::3] = one[::3]                                    # a third equal to up
+    for keep in (1, 1000, 2048, 3000, 4095):
+        ref = oracle.relu2_glu(gate, up, keep, EPS)
+        codes, scale, mask = run_relu2(gate, up, keep)
+        check_topk(codes, scale, mask, ref)
+        # without a mask the codes and scales must not change
+        both = np.zeros((M, 2 * F), np.uint16)
+        both[:, :F] = up
+        both[:, F:] = gate
+        d = to_dev(both)
+        c2 = empty((M, F), torch.int8)
+        s2 = empty((M,), torch.float32)
+        tba.relu2_glu(d[:, F:], d[:, :F], keep, c2, s2, None, eps=EPS, M=M, F=F, ld=2 * F)
+        tba.sync_status()
+        assert np.array_equal(host(c2), ref[0])
+        assert np.array_equal(host(s2).view(np.uint32), ref[3].view(np.uint32))
 
 
 def run_kv(kv, bits, bos_pos, ldt_pad=0):
