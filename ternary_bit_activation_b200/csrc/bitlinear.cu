@@ -111,7 +111,10 @@ bool tc_kernel_ready() {
 template <int C>
 void launch_quant_a4_c(const uint16_t* x, int64_t M, int K, int64_t ldx, bool fp4, bool packed, float eps,
                        uint8_t* codes, float* scale, cudaStream_t s) {
-  const dim3 grid(static_cast<unsigned>((M + 1) / 2));
+  // persistent: two rows per CTA and iteration, eight CTAs per SM
+  const int64_t need = (M + 1) / 2;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  const dim3 grid(static_cast<unsigned>(need < cap ? need : cap));
   if (!fp4 && packed) bl::quant_a4_kernel<C, false, true><<<grid, 256, 0, s>>>(x, M, K, ldx, eps, codes, scale);
   if (!fp4 && !packed) bl::quant_a4_kernel<C, false, false><<<grid, 256, 0, s>>>(x, M, K, ldx, eps, codes, scale);
   if (fp4 && packed) bl::quant_a4_kernel<C, true, true><<<grid, 256, 0, s>>>(x, M, K, ldx, eps, codes, scale);
@@ -482,18 +485,21 @@ bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D, int64_
     return BL_ERR_NULL;
   if (!aligned16(kv_bf16) || !aligned16(codes) || !aligned16(scale) || (has_bos && !aligned16(bos_codes)))
     return BL_ERR_ALIGN;
-  const int tpv = static_cast<int>(D / 8);
+  const int tpv = static_cast<int>(D / 16);
+  // persistent grid: eight CTAs per SM at most, each thread group kKvItems vectors per round
   const int64_t groups = (T * H + bl::kKvItems - 1) / bl::kKvItems;
-  const unsigned grid = static_cast<unsigned>((groups * tpv + 255) / 256);
+  const int64_t need = (groups * tpv + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  const unsigned grid = static_cast<unsigned>(need < cap ? need : cap);
   const uint16_t* kv = static_cast<const uint16_t*>(kv_bf16);
   cudaStream_t s = as_stream(stream);
   const int64_t bos = has_bos ? bos_pos : -1;
   const int h = static_cast<int>(H);
   switch (tpv) {
+    case 2: bl::kv_quant_kernel<2><<<grid, 256, 0, s>>>(kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
     case 4: bl::kv_quant_kernel<4><<<grid, 256, 0, s>>>(kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
     case 8: bl::kv_quant_kernel<8><<<grid, 256, 0, s>>>(kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
     case 16: bl::kv_quant_kernel<16><<<grid, 256, 0, s>>>(kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
-    case 32: bl::kv_quant_kernel<32><<<grid, 256, 0, s>>>(kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
     default: return BL_ERR_SHAPE;
   }
   return launch_status();

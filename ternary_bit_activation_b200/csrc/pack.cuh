@@ -5,9 +5,9 @@
 // alpha is the exact mean rounded once to fp32.  |w| = m * 2^(max(E,1) - 150)
 // with m the 24-bit significand and E the biased exponent, so the exact sum is
 // held as unsigned 64-bit integer coefficients of powers of two (bins); integer
-// adds are exact and order-free.  A single thread then forms
+// adds are exact and order-free.  Twelve threads then form the 32-bit limbs of
 //   Z = sum_e bins[e] << (e - 1)                 (the sum in units of 2^-149)
-// as a multi-word integer, divides by N*K and rounds to nearest-even fp32.
+// and one thread divides it by N*K and rounds to nearest-even fp32.
 #pragma once
 
 #include "common.cuh"
@@ -17,7 +17,7 @@ namespace bl {
 constexpr int kBinThreads = 256;
 // bins[e] is the integer coefficient of 2^(e - 150), e >= 1 (fp32 subnormals use
 // e = 1, the same scale).  A window base is clamped to at most 223, so the high
-// half of a window sum (index base + 32) stays below 256.
+// half of a flushed window sum (index base + 32) stays below 256.
 constexpr int kBins = 256;
 // Each bin receives at most one 32-bit half per flushed window (>= 1 weight)
 // or one 24-bit significand per weight, so N*K < 2^31 keeps every 64-bit bin
@@ -30,20 +30,26 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
   return v;
 }
 
-// Exact sum of |w| into exponent bins.  Each lane keeps a 64-bit fixed-point
-// accumulator whose unit is 2^(base-150): |w| = m * 2^(e-150) adds m << (e - base)
-// (exact while 0 <= e - base <= 31, a term < 2^55).  The window is anchored on
-// the lane's first nonzero weight (base = its exponent - 24, clamped to
-// [1, 223], so it spans about 2^-24 to 2^7 of that weight); weights outside it
-// go straight to their own bin.
-// Every 256 terms (< 2^63 in total) and at the end, the accumulator is flushed
-// into bins[base] (low 32 bits) and bins[base + 32] (high bits).  Lanes walk
-// (row, float4) positions without integer division.
-__device__ __forceinline__ void bins_flush(unsigned long long* sb, uint32_t base, unsigned long long& acc) {
-  if (acc) {
-    atomicAdd(&sb[base], acc & 0xFFFFFFFFull);
-    atomicAdd(&sb[base + 32], acc >> 32);
-    acc = 0;
+// Exact sum of |w| into exponent bins.  Each lane keeps an fp64 accumulator
+// holding an integer multiple of 2^(ub-150) below 2^(ub-150+53): weights with
+// biased exponent E in the window [ub, ub + kWin - 1] are multiples of that unit
+// and below 2^(ub-150+45), so up to 256 of them add exactly (every partial sum
+// is representable).  The window is anchored 12 exponents below the largest
+// weight of the lane's first nonzero load batch (ub clamped to [1, 223]);
+// weights outside it, and fp32 subnormals, add their integer significand to
+// their own bin.  Every 16 load batches (256 weights per lane) and at the end,
+// the accumulator is flushed as an integer n < 2^53 into bins[ub] (low 32 bits)
+// and bins[ub + 32] (high bits).
+constexpr uint32_t kWin = 22;
+
+__device__ __forceinline__ void bins_flush(unsigned long long* sb, uint32_t ub, double& acc) {
+  if (acc != 0.0) {
+    // n = acc * 2^(150 - ub), exact: 150 - ub is in [-73, 149]
+    const double unit_inv = __hiloint2double(static_cast<int>((1023 + 150 - ub) << 20), 0);
+    const unsigned long long n = __double2ull_rn(acc * unit_inv);
+    atomicAdd(&sb[ub], n & 0xFFFFFFFFull);
+    atomicAdd(&sb[ub + 32], n >> 32);
+    acc = 0.0;
   }
 }
 
@@ -57,45 +63,52 @@ __global__ void __launch_bounds__(kBinThreads) ternary_bins_kernel(const float* 
   const int per_row = K >> 2;  // float4 per row
   const int64_t gwarp = (static_cast<int64_t>(blockIdx.x) * kBinThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kBinThreads) >> 5;
-  constexpr int kLoads = 4;   // float4 loads per lane issued together
-  uint32_t base = 0;          // 0: not anchored yet
-  unsigned long long acc = 0;
-  int terms = 0;
+  constexpr int kLoads = 4;   // float4 loads per lane issued together (16 weights)
+  uint32_t ub = 0;            // 0: not anchored yet
+  uint32_t lo_bits = 0;       // ub << 23
+  double acc = 0.0;
+  int batches = 0;
   for (int64_t n = gwarp; n < N; n += nwarps) {
     const float* wrow = w + n * ldw;
     for (int q0 = 0; q0 < per_row; q0 += 32 * kLoads) {
-      uint4 vv[kLoads];
+      uint32_t u[4 * kLoads];
 #pragma unroll
       for (int j = 0; j < kLoads; ++j) {
         const int q = q0 + j * 32 + lane;
-        vv[j] = q < per_row ? ld_global_nc_v4(wrow + static_cast<int64_t>(q) * 4) : make_uint4(0, 0, 0, 0);
+        const uint4 v = q < per_row ? ld_global_nc_v4(wrow + static_cast<int64_t>(q) * 4) : make_uint4(0, 0, 0, 0);
+        u[4 * j] = v.x & 0x7FFFFFFFu;
+        u[4 * j + 1] = v.y & 0x7FFFFFFFu;
+        u[4 * j + 2] = v.z & 0x7FFFFFFFu;
+        u[4 * j + 3] = v.w & 0x7FFFFFFFu;
+      }
+      if (ub == 0) {
+        uint32_t amax = 0;
+#pragma unroll
+        for (int i = 0; i < 4 * kLoads; ++i) amax = max(amax, u[i]);
+        if (amax != 0) {
+          const int E = static_cast<int>(amax >> 23);
+          ub = static_cast<uint32_t>(min(max(E - 12, 1), 223));
+          lo_bits = ub << 23;
+        }
       }
 #pragma unroll
-      for (int j = 0; j < kLoads; ++j) {
-        const uint32_t u[4] = {vv[j].x, vv[j].y, vv[j].z, vv[j].w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t a = u[k] & 0x7FFFFFFFu;
-          if (a == 0) continue;
+      for (int i = 0; i < 4 * kLoads; ++i) {
+        const uint32_t a = u[i];
+        if (a - lo_bits < (kWin << 23)) {
+          acc += static_cast<double>(__uint_as_float(a));   // exact; 0 before the anchor
+        } else if (a != 0) {
           const uint32_t E = a >> 23;
           const uint32_t m = (a & 0x7FFFFFu) | (E ? 0x800000u : 0u);
-          const uint32_t e = E ? E : 1u;
-          if (base == 0) base = e > 25 ? min(e - 24, 223u) : 1u;   // window [base, base + 31] holds e
-          const uint32_t sh = e - base;   // wraps to a large value when e < base
-          if (sh <= 31u) {
-            acc += static_cast<unsigned long long>(m) << sh;
-            if (++terms == 256) {
-              bins_flush(sb, base, acc);
-              terms = 0;
-            }
-          } else {
-            atomicAdd(&sb[e], static_cast<unsigned long long>(m));
-          }
+          atomicAdd(&sb[E ? E : 1u], static_cast<unsigned long long>(m));
         }
+      }
+      if (++batches == 16) {
+        bins_flush(sb, ub, acc);
+        batches = 0;
       }
     }
   }
-  bins_flush(sb, base, acc);
+  bins_flush(sb, ub, acc);
   __syncthreads();
   for (int b = threadIdx.x; b < kBins; b += kBinThreads)
     if (sb[b]) atomicAdd(&gbins[b], sb[b]);
@@ -103,21 +116,6 @@ __global__ void __launch_bounds__(kBinThreads) ternary_bins_kernel(const float* 
 
 // Multi-word unsigned integer, little-endian 32-bit limbs.
 constexpr int kLimbs = 12;  // 384 bits: bins < 2^64 shifted by <= 262 bits
-
-__device__ __forceinline__ void big_add_shifted(uint32_t (&z)[kLimbs], unsigned long long v, int shift) {
-  const int li = shift >> 5, bo = shift & 31;
-  // v << bo spans up to three limbs
-  const uint32_t parts[3] = {static_cast<uint32_t>(v << bo), static_cast<uint32_t>(bo ? (v >> (32 - bo)) : (v >> 32)),
-                             static_cast<uint32_t>(bo ? (v >> (64 - bo)) : 0ull)};
-  unsigned long long carry = 0;
-  for (int i = li; i < kLimbs; ++i) {
-    const unsigned long long add = (i - li < 3) ? parts[i - li] : 0u;
-    const unsigned long long s = static_cast<unsigned long long>(z[i]) + add + carry;
-    z[i] = static_cast<uint32_t>(s);
-    carry = s >> 32;
-    if (i - li >= 2 && carry == 0) break;
-  }
-}
 
 __device__ __forceinline__ int big_bitlen(const uint32_t (&z)[kLimbs]) {
   for (int i = kLimbs - 1; i >= 0; --i)
@@ -156,14 +154,30 @@ __device__ __forceinline__ unsigned long long big_window64(const uint32_t (&z)[k
 __global__ void __launch_bounds__(kBins) ternary_alpha_kernel(const unsigned long long* __restrict__ gbins,
                                                                unsigned long long D, float* __restrict__ alpha) {
   __shared__ unsigned long long sb[kBins];
+  __shared__ unsigned long long limb_sum[kLimbs];
   for (int e = threadIdx.x; e < kBins; e += blockDim.x) sb[e] = gbins[e];   // one round trip for all bins
+  __syncthreads();
+  // thread l < kLimbs sums the 32-bit pieces of every shifted bin that fall in
+  // limb l (at most 256 pieces < 2^32, so the sum stays below 2^40)
+  if (threadIdx.x < kLimbs) {
+    const int l = threadIdx.x;
+    unsigned long long acc = 0;
+    for (int e = 0; e < kBins; ++e) {
+      const unsigned long long v = sb[e];
+      const int r = (e > 0 ? e : 1) - 1 - 32 * l;   // bit of v that lands on the limb's bit 0 is -r
+      if (v == 0 || r >= 32 || r <= -64) continue;
+      acc += (r >= 0 ? (v << r) : (v >> -r)) & 0xFFFFFFFFull;
+    }
+    limb_sum[l] = acc;
+  }
   __syncthreads();
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   uint32_t z[kLimbs];
-  for (int i = 0; i < kLimbs; ++i) z[i] = 0;
-  for (int e = 0; e < kBins; ++e) {
-    const unsigned long long b = sb[e];
-    if (b) big_add_shifted(z, b, (e > 0 ? e : 1) - 1);
+  unsigned long long carry = 0;
+  for (int i = 0; i < kLimbs; ++i) {
+    const unsigned long long t = limb_sum[i] + carry;
+    z[i] = static_cast<uint32_t>(t);
+    carry = t >> 32;
   }
   // Long division Q = floor(Z / D), R = Z mod D.
   uint32_t q[kLimbs];
@@ -248,30 +262,43 @@ __global__ void __launch_bounds__(256) ternary_pack_kernel(const float* __restri
   const int lane = threadIdx.x & 31;
   const int64_t gwarp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t n = gwarp; n < N; n += nwarps)
-  for (int q = lane; q < per_row; q += 32) {
-    const float* src = w + n * ldw + static_cast<int64_t>(q) * 16;
-    int c[16];
+  for (int64_t n = gwarp; n < N; n += nwarps) {
+    // two 16-weight steps per lane and iteration: eight 16-byte loads in flight
+    for (int q0 = lane; q0 < per_row; q0 += 64) {
+      uint4 v[2][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint4 v = ld_global_nc_v4(src + 4 * j);
-      c[4 * j + 0] = ternary_code(__uint_as_float(v.x), d, h, fast);
-      c[4 * j + 1] = ternary_code(__uint_as_float(v.y), d, h, fast);
-      c[4 * j + 2] = ternary_code(__uint_as_float(v.z), d, h, fast);
-      c[4 * j + 3] = ternary_code(__uint_as_float(v.w), d, h, fast);
-    }
-    if constexpr (T2) {
-      uint32_t word = 0;
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int q = q0 + 32 * h2;
+        const float* src = w + n * ldw + static_cast<int64_t>(q) * 16;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) word |= (static_cast<uint32_t>(c[j]) & 3u) << (2 * j);
-      reinterpret_cast<uint32_t*>(out + n * static_cast<int64_t>(K >> 2))[q] = word;
-    } else {
-      uint32_t wd[4];
+        for (int j = 0; j < 4; ++j) v[h2][j] = q < per_row ? ld_global_nc_v4(src + 4 * j) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        wd[j] = (static_cast<uint32_t>(c[4 * j]) & 0xFFu) | ((static_cast<uint32_t>(c[4 * j + 1]) & 0xFFu) << 8) |
-                ((static_cast<uint32_t>(c[4 * j + 2]) & 0xFFu) << 16) | (static_cast<uint32_t>(c[4 * j + 3]) << 24);
-      reinterpret_cast<uint4*>(out + n * static_cast<int64_t>(K))[q] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int q = q0 + 32 * h2;
+        if (q >= per_row) continue;
+        int c[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          c[4 * j + 0] = ternary_code(__uint_as_float(v[h2][j].x), d, h, fast);
+          c[4 * j + 1] = ternary_code(__uint_as_float(v[h2][j].y), d, h, fast);
+          c[4 * j + 2] = ternary_code(__uint_as_float(v[h2][j].z), d, h, fast);
+          c[4 * j + 3] = ternary_code(__uint_as_float(v[h2][j].w), d, h, fast);
+        }
+        if constexpr (T2) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) word |= (static_cast<uint32_t>(c[j]) & 3u) << (2 * j);
+          reinterpret_cast<uint32_t*>(out + n * static_cast<int64_t>(K >> 2))[q] = word;
+        } else {
+          uint32_t wd[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            wd[j] = (static_cast<uint32_t>(c[4 * j]) & 0xFFu) | ((static_cast<uint32_t>(c[4 * j + 1]) & 0xFFu) << 8) |
+                    ((static_cast<uint32_t>(c[4 * j + 2]) & 0xFFu) << 16) | (static_cast<uint32_t>(c[4 * j + 3]) << 24);
+          reinterpret_cast<uint4*>(out + n * static_cast<int64_t>(K))[q] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        }
+      }
     }
   }
 }

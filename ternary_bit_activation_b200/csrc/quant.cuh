@@ -54,115 +54,157 @@ __device__ __forceinline__ int e2m1_index(float a) {
 }
 
 // ---------------------------------------------------------------------------
-// quant_a4: 128 threads per row, 2 rows per 256-thread CTA.  Thread t of a row
-// holds chunks c*128 + t (8 bf16 each) for c < CHUNKS.
+// quant_a4: 128 threads per row, two row slots per 256-thread CTA, persistent
+// over rows.  Thread t of a row holds chunks c*128 + t (8 bf16 each) for
+// c < CHUNKS; the next row's chunks are loaded before the current row is
+// reduced and written, so every thread keeps a row's loads in flight.
 // ---------------------------------------------------------------------------
 constexpr int kQ4ThreadsPerRow = 128;
+
+// Low bits of RN(RN(p) + 1.5*2^23) hold rint_even(p) for |p| < 2^22 (the sum's
+// ulp is 1); p is clamped to the code range first.
+__device__ __forceinline__ uint32_t q4_code_bits(float x, float mult) {
+  const float p = fminf(fmaxf(__fmul_rn(x, mult), -8.f), 7.f);
+  return __float_as_uint(__fadd_rn(p, 12582912.0f));
+}
+
+// Barrier of one row slot (128 threads); literal ids keep the CTA at two barriers.
+__device__ __forceinline__ void q4_row_sync(int sub) {
+  if (sub == 0) {
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+  } else {
+    asm volatile("bar.sync 2, 128;" ::: "memory");
+  }
+}
+
+template <int CHUNKS>
+__device__ __forceinline__ void q4_load(const uint16_t* x, int64_t row, int64_t M, int64_t ldx, int nchunk, int t,
+                                        uint4 (&v)[CHUNKS]) {
+  const bool ok = row < M;
+  const uint16_t* xr = x + (ok ? row : 0) * ldx;
+#pragma unroll
+  for (int c = 0; c < CHUNKS; ++c) {
+    const int idx = c * kQ4ThreadsPerRow + t;
+    v[c] = (ok && idx < nchunk) ? ld_global_nc_v4(xr + static_cast<int64_t>(idx) * 8) : make_uint4(0, 0, 0, 0);
+  }
+}
 
 template <int CHUNKS, bool FP4, bool PACKED>
 __global__ void __launch_bounds__(256) quant_a4_kernel(const uint16_t* __restrict__ x, int64_t M, int K,
                                                        int64_t ldx, float eps, uint8_t* __restrict__ codes,
                                                        float* __restrict__ scale) {
-  __shared__ double s_sum[2][4];
-  __shared__ uint32_t s_max[2][4];
+  __shared__ double s_sum[2][2][4];
+  __shared__ uint32_t s_max[2][2][4];
   const int sub = threadIdx.x >> 7;
   const int t = threadIdx.x & 127;
   const int warp = t >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * 2 + sub;
-  const bool row_ok = row < M;
   const int nchunk = K >> 3;
-  const uint16_t* xr = x + (row_ok ? row : 0) * ldx;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * 2;
+  int64_t row = static_cast<int64_t>(blockIdx.x) * 2 + sub;
 
+  // rows of up to 4096 values prefetch the next row; longer rows would need too
+  // many registers for two rows, so they load at the top of each iteration
+  constexpr bool kPrefetch = CHUNKS <= 4;
   uint4 v[CHUNKS];
-#pragma unroll
-  for (int c = 0; c < CHUNKS; ++c) {
-    const int idx = c * kQ4ThreadsPerRow + t;
-    v[c] = (row_ok && idx < nchunk) ? ld_global_nc_v4(xr + static_cast<int64_t>(idx) * 8) : make_uint4(0, 0, 0, 0);
-  }
+  if (kPrefetch) q4_load<CHUNKS>(x, row, M, ldx, nchunk, t, v);
+  for (int it = 0; row < M; row += stride, ++it) {
+    uint4 nx[kPrefetch ? CHUNKS : 1];
+    if constexpr (kPrefetch) {
+      q4_load<CHUNKS>(x, row + stride, M, ldx, nchunk, t, nx);
+    } else {
+      q4_load<CHUNKS>(x, row, M, ldx, nchunk, t, v);
+    }
+    const int par = it & 1;
 
-  if constexpr (!FP4) {
-    // beta = mean|x|: the fp64 sum of bf16 magnitudes is exact for in-contract
-    // rows, so the reduction order does not change it.
-    double acc = 0.0;
+    if constexpr (!FP4) {
+      // beta = mean|x|: the fp64 sum of bf16 magnitudes is exact for in-contract
+      // rows, so the reduction order does not change it.
+      double acc = 0.0;
 #pragma unroll
-    for (int c = 0; c < CHUNKS; ++c) {
-      float f[8];
-      unpack_bf16x8(v[c], f);
+      for (int c = 0; c < CHUNKS; ++c) {
+        float f[8];
+        unpack_bf16x8(v[c], f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc += static_cast<double>(fabsf(f[e]));
-    }
-    acc = warp_sum_f64(acc);
-    if (lane == 0) s_sum[sub][warp] = acc;
-    __syncthreads();
-    const double S = (s_sum[sub][0] + s_sum[sub][1]) + (s_sum[sub][2] + s_sum[sub][3]);
-    const float beta = __double2float_rn(S / static_cast<double>(K));
-    const float mult = __fdiv_rn(sqrt7_f32(), __fadd_rn(beta, eps));
-    if (row_ok && t == 0) scale[row] = __fdiv_rn(beta, sqrt7_f32());
-#pragma unroll
-    for (int c = 0; c < CHUNKS; ++c) {
-      const int idx = c * kQ4ThreadsPerRow + t;
-      if (!row_ok || idx >= nchunk) continue;
-      float f[8];
-      unpack_bf16x8(v[c], f);
-      int q[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) q[e] = round_clip(__fmul_rn(f[e], mult), -8.f, 7.f);
-      if constexpr (PACKED) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) word |= (static_cast<uint32_t>(q[e]) & 0xFu) << (4 * e);
-        reinterpret_cast<uint32_t*>(codes + row * (K >> 1))[idx] = word;
-      } else {
-        uint2 w2;
-        w2.x = (q[0] & 0xFF) | ((q[1] & 0xFF) << 8) | ((q[2] & 0xFF) << 16) | (static_cast<uint32_t>(q[3]) << 24);
-        w2.y = (q[4] & 0xFF) | ((q[5] & 0xFF) << 8) | ((q[6] & 0xFF) << 16) | (static_cast<uint32_t>(q[7]) << 24);
-        reinterpret_cast<uint2*>(codes + row * static_cast<int64_t>(K))[idx] = w2;
+        for (int e = 0; e < 8; ++e) acc += static_cast<double>(fabsf(f[e]));
       }
-    }
-  } else {
-    // MinMax FP4: max|x| as the largest 15-bit bf16 magnitude.
-    uint32_t mk = 0;
+      acc = warp_sum_f64(acc);
+      if (lane == 0) s_sum[par][sub][warp] = acc;
+      q4_row_sync(sub);
+      const double S = (s_sum[par][sub][0] + s_sum[par][sub][1]) + (s_sum[par][sub][2] + s_sum[par][sub][3]);
+      const float beta = __double2float_rn(S / static_cast<double>(K));
+      const float mult = __fdiv_rn(sqrt7_f32(), __fadd_rn(beta, eps));
+      if (t == 0) scale[row] = __fdiv_rn(beta, sqrt7_f32());
 #pragma unroll
-    for (int c = 0; c < CHUNKS; ++c) {
-      uint32_t k[8];
-      bf16x8_mag_keys(v[c], k);
+      for (int c = 0; c < CHUNKS; ++c) {
+        const int idx = c * kQ4ThreadsPerRow + t;
+        if (idx >= nchunk) continue;
+        float f[8];
+        unpack_bf16x8(v[c], f);
+        uint32_t q[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mk = max(mk, k[e]);
-    }
-    mk = warp_max_u32(mk);
-    if (lane == 0) s_max[sub][warp] = mk;
-    __syncthreads();
-    mk = max(max(s_max[sub][0], s_max[sub][1]), max(s_max[sub][2], s_max[sub][3]));
-    const int p = fp4_scale_exponent(mk << 16);
-    if (row_ok && t == 0) scale[row] = exact_pow2(PACKED ? p : p - 1);
-#pragma unroll
-    for (int c = 0; c < CHUNKS; ++c) {
-      const int idx = c * kQ4ThreadsPerRow + t;
-      if (!row_ok || idx >= nchunk) continue;
-      float f[8];
-      unpack_bf16x8(v[c], f);
-      uint32_t word = 0;
-      uint2 w2 = make_uint2(0, 0);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float s = mul_pow2(f[e], -p);
-        const int i = e2m1_index(fabsf(s));
-        const bool neg = (s < 0.f) && (i != 0);
+        for (int e = 0; e < 8; ++e) q[e] = q4_code_bits(f[e], mult);
         if constexpr (PACKED) {
-          word |= (static_cast<uint32_t>(i) | (neg ? 8u : 0u)) << (4 * e);
+          uint32_t word = 0;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) word |= (q[e] & 0xFu) << (4 * e);
+          reinterpret_cast<uint32_t*>(codes + row * (K >> 1))[idx] = word;
         } else {
-          // twice the E2M1 value: {0,1,2,3,4,6,8,12}[i]
-          const int tv = (i <= 4) ? i : (i == 5 ? 6 : (i == 6 ? 8 : 12));
-          const uint32_t b = static_cast<uint32_t>(neg ? -tv : tv) & 0xFFu;
-          if (e < 4) w2.x |= b << (8 * e); else w2.y |= b << (8 * (e - 4));
+          uint2 w2;
+          // the low byte of each sum's bits is the code as a two's-complement int8
+          w2.x = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+          w2.y = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
+          reinterpret_cast<uint2*>(codes + row * static_cast<int64_t>(K))[idx] = w2;
         }
       }
-      if constexpr (PACKED) {
-        reinterpret_cast<uint32_t*>(codes + row * (K >> 1))[idx] = word;
-      } else {
-        reinterpret_cast<uint2*>(codes + row * static_cast<int64_t>(K))[idx] = w2;
+    } else {
+      // MinMax FP4: max|x| as the largest 15-bit bf16 magnitude.
+      uint32_t mk = 0;
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) {
+        uint32_t k[8];
+        bf16x8_mag_keys(v[c], k);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mk = max(mk, k[e]);
       }
+      mk = __reduce_max_sync(0xFFFFFFFFu, mk);
+      if (lane == 0) s_max[par][sub][warp] = mk;
+      q4_row_sync(sub);
+      mk = max(max(s_max[par][sub][0], s_max[par][sub][1]), max(s_max[par][sub][2], s_max[par][sub][3]));
+      const int p = fp4_scale_exponent(mk << 16);
+      if (t == 0) scale[row] = exact_pow2(PACKED ? p : p - 1);
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) {
+        const int idx = c * kQ4ThreadsPerRow + t;
+        if (idx >= nchunk) continue;
+        float f[8];
+        unpack_bf16x8(v[c], f);
+        uint32_t word = 0;
+        uint2 w2 = make_uint2(0, 0);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float s = mul_pow2(f[e], -p);
+          const int i = e2m1_index(fabsf(s));
+          const bool neg = (s < 0.f) && (i != 0);
+          if constexpr (PACKED) {
+            word |= (static_cast<uint32_t>(i) | (neg ? 8u : 0u)) << (4 * e);
+          } else {
+            // twice the E2M1 value: {0,1,2,3,4,6,8,12}[i]
+            const int tv = (i <= 4) ? i : (i == 5 ? 6 : (i == 6 ? 8 : 12));
+            const uint32_t b = static_cast<uint32_t>(neg ? -tv : tv) & 0xFFu;
+            if (e < 4) w2.x |= b << (8 * e); else w2.y |= b << (8 * (e - 4));
+          }
+        }
+        if constexpr (PACKED) {
+          reinterpret_cast<uint32_t*>(codes + row * (K >> 1))[idx] = word;
+        } else {
+          reinterpret_cast<uint2*>(codes + row * static_cast<int64_t>(K))[idx] = w2;
+        }
+      }
+    }
+    if constexpr (kPrefetch) {
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) v[c] = nx[c];
     }
   }
 }
