@@ -172,8 +172,10 @@ BL_API bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int6
  * y: [M x N] bf16 with row stride ldy (nullable).  acc_out: [M x N] int32,
  * row stride N (nullable; a test aid).
  * Kernels: BL_A_I8 x BL_W_I8 runs on the tcgen05 tensor cores (kind::i8,
- * TMA-fed, TMEM accumulators); other operand formats run on a CUDA-core kernel
- * that reads packed operands directly (the decode path).
+ * TMA-fed, TMEM accumulators); BL_A_I8 x BL_W_T2 with M >= 8 runs on the
+ * tensor cores too, the 2-bit weights widened to int8 into tensor memory as the
+ * MMA's A operand (the tokens are the MMA's N side); other operand formats and
+ * fewer tokens run on a CUDA-core kernel that reads packed operands directly.
  * Requires K % 64 == 0, ldy % 8 == 0, 1 <= alpha_group.
  */
 BL_API bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale,

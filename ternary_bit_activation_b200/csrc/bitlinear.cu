@@ -89,6 +89,21 @@ bool make_i8_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t col
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Unswizzled map over a row-major byte matrix viewed in 8-byte elements
+// (cols_bytes % 16 == 0); a box row carries box_bytes of one matrix row.
+bool make_u64_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols_bytes, uint32_t box_rows,
+                  uint32_t box_bytes) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols_bytes / 8, rows};
+  const cuuint64_t strides[1] = {cols_bytes};
+  const cuuint32_t box[2] = {box_bytes / 8, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool tc_kernel_ready() {
   static bool done[kMaxDevices] = {false};
   const int d = current_device();
@@ -99,6 +114,13 @@ bool tc_kernel_ready() {
       return false;
     if (!cuda_ok(cudaFuncSetAttribute(bl::gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(bl::kT2SmemBytes))))
+      return false;
+    if (!cuda_ok(cudaFuncSetAttribute(bl::gemm_t2tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      227 * 1024)) ||
+        !cuda_ok(cudaFuncSetAttribute(bl::gemm_t2tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      227 * 1024)) ||
+        !cuda_ok(cudaFuncSetAttribute(bl::gemm_t2tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      227 * 1024)))
       return false;
     done[d] = true;
   }
@@ -450,6 +472,45 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
     p.num_kb = (k + bl::kTcBK - 1) / bl::kTcBK;
     const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
     bl::gemm_tc_kernel<<<grid, bl::kTcThreads, bl::kTcSmemBytes, s>>>(ta, tb, p);
+    return launch_status();
+  }
+  if (afmt == BL_A_I8 && wfmt == BL_W_T2 && M >= bl::kTsMinTokens) {
+    // 2-bit weights widened into tensor memory; tokens on the MMA's N side
+    if (!tc_kernel_ready()) return BL_ERR_CUDA;
+    const int nt = m <= 8 ? 8 : (m >= 256 ? 256 : ((m + 15) & ~15));
+    const int sub = nt <= 32 ? 4 : (nt <= 96 ? 2 : 1);          // 256-code sub-stages per TMA stage
+    CUtensorMap tx, tw;
+    if (!make_i8_map(&tx, A, static_cast<uint64_t>(M), static_cast<uint64_t>(K), static_cast<uint32_t>(nt), 128) ||
+        !make_u64_map(&tw, W, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4), bl::kTsBN,
+                      static_cast<uint32_t>(sub * bl::kTsSubK / 4)))
+      return BL_ERR_CUDA;
+    bl::TsParams p;
+    p.a_scale = a_scale;
+    p.alpha = alpha;
+    p.alpha_group = alpha_group;
+    p.M = m;
+    p.N = n;
+    p.K = k;
+    p.y = Y;
+    p.ldy = ldy;
+    p.acc = acc_out;
+    p.nt = nt;
+    p.num_n_tiles = (n + bl::kTsBN - 1) / bl::kTsBN;
+    p.num_units = p.num_n_tiles * ((m + nt - 1) / nt);
+    p.num_kb = (k + sub * bl::kTsSubK - 1) / (sub * bl::kTsSubK);
+    p.stage_x = static_cast<uint32_t>(nt * sub * bl::kTsSubK);
+    const uint32_t per_stage = p.stage_x + static_cast<uint32_t>(bl::kTsBN * sub * bl::kTsSubK / 4);
+    int stages = static_cast<int>((208u * 1024u) / per_stage);
+    p.stages = stages < 2 ? 2 : (stages > bl::kTsMaxStages ? bl::kTsMaxStages : stages);
+    // the whole TMEM: up to four accumulators of nt columns, and as many 64-column A buffers as fit
+    p.dslots = nt <= 32 ? 4u : (nt <= 64 ? 2u : 1u);
+    const uint32_t ab = (512u - p.dslots * static_cast<uint32_t>(nt)) / bl::kTsACols;
+    p.abufs = ab > static_cast<uint32_t>(bl::kTsMaxABufs) ? static_cast<uint32_t>(bl::kTsMaxABufs) : ab;
+    const size_t smem = 1024 + static_cast<size_t>(p.stages) * per_stage + 512;   // + barriers
+    const int grid = p.num_units < sm_count() ? p.num_units : sm_count();
+    if (sub == 4) bl::gemm_t2tc_kernel<4><<<grid, bl::kTsThreads, smem, s>>>(tx, tw, p);
+    else if (sub == 2) bl::gemm_t2tc_kernel<2><<<grid, bl::kTsThreads, smem, s>>>(tx, tw, p);
+    else bl::gemm_t2tc_kernel<1><<<grid, bl::kTsThreads, smem, s>>>(tx, tw, p);
     return launch_status();
   }
   const bool t2 = wfmt == BL_W_T2;

@@ -7,9 +7,14 @@
 //                     streamed by TMA into a 128B-swizzled shared-memory ring,
 //                     persistent over output tiles with a double-buffered
 //                     accumulator so the epilogue overlaps the next tile.
+// gemm_tc2_kernel  -- the same on CTA pairs (cta_group::2), 256 x 256 tiles.
+// gemm_t2tc_kernel -- 2-bit ternary weights x int8 activations for 8..256
+//                     tokens (decode): weights widened to int8 in registers
+//                     and stored into tensor memory as the MMA's A operand.
 // gemm_simt_kernel -- CUDA-core kernel that reads packed operands directly
-//                     (2-bit ternary weights, INT4 / E2M1 nibbles); the decode
-//                     path, where the packed weight bytes set the time.
+//                     (2-bit ternary weights, INT4 / E2M1 nibbles); decode of
+//                     fewer than 8 tokens, where the packed weight bytes and
+//                     the latency of a few tiles set the time.
 #pragma once
 
 #include "common.cuh"
@@ -510,6 +515,305 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT2Threads, 1)
   cluster_sync_all();   // no CTA leaves while its peer may still signal its barriers
   tc_fence_after();
   if (warp == 1) tmem_dealloc_pair(tmem_base, kTcTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// gemm_t2tc_kernel -- 2-bit ternary weights x int8 activations on the tensor
+// cores, for few tokens (decode).  The product is taken transposed,
+//   D[n, m] = sum_k t[n, k] * a[m, k],
+// so 128 weight rows form the MMA's M side and the tokens its N side (8, or a
+// multiple of 16 up to 256).  The weights stay 2-bit in HBM and shared memory:
+// widen warps turn each 16-code word into int8 in registers (5 bit operations
+// and 8 byte permutes) and store the rows into tensor memory, which the MMA
+// reads as its A operand; the activations reach shared memory by TMA in the
+// 128-byte-swizzled layout of the B operand.
+//   warp 0: TMA producer    warp 1: MMA issuer (one thread)
+//   warps 2-9: widen (warp w owns TMEM lanes 32*(w%4).. and half of every
+//              64-byte piece of its rows), then the epilogue of each tile
+// A TMA stage carries SUB sub-stages of 256 codes (SUB*64 bytes of each of the
+// tile's 128 weight rows): the TMA engine moves a box row at a time, so longer
+// rows move more bytes per SM.  Each sub-stage is widened into one of several
+// TMEM A buffers, so the widen warps run ahead of the MMA.  Consecutive MMAs go
+// to up to four accumulators in turn (summed in the epilogue).  A work unit is
+// one 128-row weight tile against one block of tokens, over all of K; the grid
+// is persistent over units.
+// ---------------------------------------------------------------------------
+constexpr int kTsBN = 128;                 // weight rows per tile (MMA M)
+constexpr int kTsSubK = 256;               // codes per sub-stage: 64 bytes of 2-bit weights per row
+constexpr int kTsWidenWarps = 8;
+constexpr int kTsThreads = 32 * (2 + kTsWidenWarps);
+constexpr uint32_t kTsACols = kTsSubK / 4; // TMEM columns of one widened sub-stage (4 codes per column)
+constexpr int kTsMaxStages = 16;
+constexpr int kTsMaxABufs = 6;             // widened sub-stages held in TMEM
+// Below this many tokens the CUDA-core kernel is faster: every tcgen05.mma
+// (M = 128, K = 32) costs about a hundred cycles of issue whatever N is, while
+// the CUDA-core kernel's work grows with the token count.
+constexpr int kTsMinTokens = 8;
+
+struct TsParams {
+  const float* a_scale;
+  const float* alpha;
+  int64_t alpha_group;
+  int M, N, K;
+  uint16_t* y;
+  int64_t ldy;
+  int32_t* acc;
+  int nt;                 // tokens per MMA (N side)
+  int num_n_tiles, num_units, num_kb, stages;
+  uint32_t stage_x;       // activation bytes per stage (nt * 256 * SUB)
+  uint32_t abufs;         // TMEM A buffers (2..kTsMaxABufs)
+  uint32_t dslots;        // accumulators (1, 2 or 4)
+};
+
+// int8 of a 2-bit code {00 -> 0, 01 -> 1, 11 -> -1}, as byte permute table.
+constexpr uint32_t kT2Lut = 0xFF000100u;
+
+// 16 codes (element e in bits 2e..2e+1) -> 4 words of int8, element order kept.
+__device__ __forceinline__ void widen_t2_word(uint32_t x, uint32_t* out) {
+  const uint32_t m1 = x & 0x33333333u;           // nibble i: code 2i
+  const uint32_t m2 = (x >> 2) & 0x33333333u;    // nibble i: code 2i+1
+  const uint32_t e0 = __byte_perm(kT2Lut, kT2Lut, m1);          // codes 0, 2, 4, 6
+  const uint32_t e1 = __byte_perm(kT2Lut, kT2Lut, m2);          // codes 1, 3, 5, 7
+  const uint32_t e2 = __byte_perm(kT2Lut, kT2Lut, m1 >> 16);    // codes 8, 10, 12, 14
+  const uint32_t e3 = __byte_perm(kT2Lut, kT2Lut, m2 >> 16);    // codes 9, 11, 13, 15
+  out[0] = __byte_perm(e0, e1, 0x5140);
+  out[1] = __byte_perm(e0, e1, 0x7362);
+  out[2] = __byte_perm(e2, e3, 0x5140);
+  out[3] = __byte_perm(e2, e3, 0x7362);
+}
+
+template <int SUB>
+__global__ void __launch_bounds__(kTsThreads, 1)
+    gemm_t2tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TsParams p) {
+  constexpr uint32_t kStageW = kTsBN * SUB * (kTsSubK / 4);   // weight bytes per stage
+  constexpr int kRowBytes = SUB * (kTsSubK / 4);              // bytes of one weight row per stage
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sX = smem;
+  uint8_t* sW = smem + static_cast<size_t>(p.stages) * p.stage_x;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sW + static_cast<size_t>(p.stages) * kStageW);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kTsMaxStages;
+  uint64_t* afull = bars + 2 * kTsMaxStages;
+  uint64_t* aempty = afull + kTsMaxABufs;
+  uint64_t* dfull = aempty + kTsMaxABufs;
+  uint64_t* dempty = dfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dempty + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + kTsWidenWarps);   // MMA commit (activations read) + widen warps (weights read)
+    }
+    for (int b = 0; b < static_cast<int>(p.abufs); ++b) {
+      mbar_init(&afull[b], kTsWidenWarps);
+      mbar_init(&aempty[b], 1);
+    }
+    mbar_init(dfull, 1);
+    mbar_init(dempty, kTsWidenWarps);
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmX);
+    prefetch_tmap(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t d_col = p.abufs * kTsACols;  // accumulators follow the A buffers
+  bool aborted = false;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int unit = blockIdx.x; unit < p.num_units && !aborted; unit += gridDim.x) {
+        const int nb = unit % p.num_n_tiles, mb = unit / p.num_n_tiles;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait_bounded(&empty[s], ph ^ 1u)) {
+            aborted = true;
+            break;
+          }
+          uint8_t* xs = sX + static_cast<size_t>(s) * p.stage_x;
+          mbar_arrive_expect_tx(&full[s], p.stage_x + kStageW);
+          tma_load_2d(&tmW, &full[s], sW + static_cast<size_t>(s) * kStageW, kb * (kRowBytes / 8), nb * kTsBN);
+#pragma unroll
+          for (int q = 0; q < 2 * SUB; ++q)
+            tma_load_2d(&tmX, &full[s], xs + q * p.nt * 128, kb * SUB * kTsSubK + 128 * q, mb * p.nt);
+          if (++s == p.stages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (one thread) ----------------
+    if (lane == 0) {
+      const uint32_t idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(p.nt) >> 3) << 17) |
+                             ((static_cast<uint32_t>(kTsBN) >> 4) << 24);
+      int s = 0;
+      uint32_t ph = 0, abuf = 0, aph = 0;
+      int local = 0;
+      for (int unit = blockIdx.x; unit < p.num_units && !aborted; unit += gridDim.x, ++local) {
+        if (!mbar_wait_bounded(dempty, (static_cast<uint32_t>(local) & 1u) ^ 1u)) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < p.num_kb && !aborted; ++kb) {
+          if (!mbar_wait_bounded(&full[s], ph)) {
+            aborted = true;
+            break;
+          }
+          const uint32_t xs = smem_u32(sX + static_cast<size_t>(s) * p.stage_x);
+          for (int j = 0; j < SUB; ++j) {
+            if (!mbar_wait_bounded(&afull[abuf], aph)) {
+              aborted = true;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kTsSubK / 32; ++kk) {
+              const uint32_t slot = static_cast<uint32_t>(kk) & (p.dslots - 1u);
+              const uint32_t a_tmem = tmem_base + abuf * kTsACols + static_cast<uint32_t>(kk * 8);
+              const uint32_t b_addr = xs + static_cast<uint32_t>((2 * j + (kk >> 2)) * p.nt * 128 + (kk & 3) * 32);
+              mma_i8_ts(tmem_base + d_col + slot * static_cast<uint32_t>(p.nt), a_tmem, sw128_kmajor_desc(b_addr),
+                        idesc, (kb != 0 || j != 0 || static_cast<uint32_t>(kk) >= p.dslots) ? 1u : 0u);
+            }
+            mma_commit(&aempty[abuf]);    // widened weights of this sub-stage read
+            if (++abuf == p.abufs) {
+              abuf = 0;
+              aph ^= 1u;
+            }
+          }
+          if (aborted) break;
+          mma_commit(&empty[s]);          // activations of this stage read
+          if (++s == p.stages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (aborted) break;
+        mma_commit(dfull);                // accumulators ready
+      }
+    }
+  } else if (warp < 2 + kTsWidenWarps) {
+    // ---------------- widen + epilogue (warps 2-9) ----------------
+    const int wi = warp - 2;
+    const int quad = warp & 3;
+    const int half = wi >> 2;
+    const int trow = quad * 32 + lane;                    // weight row within the tile = TMEM lane
+    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    int s = 0;
+    uint32_t ph = 0, abuf = 0, aph = 0;
+    int local = 0;
+    for (int unit = blockIdx.x; unit < p.num_units && !aborted; unit += gridDim.x, ++local) {
+      const int nb = unit % p.num_n_tiles, mb = unit / p.num_n_tiles;
+      for (int kb = 0; kb < p.num_kb && !aborted; ++kb) {
+        if (!warp_wait(&full[s], ph)) {
+          aborted = true;
+          break;
+        }
+        // this thread's bytes of the stage: SUB pieces of 64 bytes, it widens 32 of each
+        const uint8_t* row = sW + static_cast<size_t>(s) * kStageW + trow * kRowBytes + half * 32;
+        uint4 w[SUB][2];
+#pragma unroll
+        for (int j = 0; j < SUB; ++j) {
+          w[j][0] = reinterpret_cast<const uint4*>(row + j * 64)[0];
+          w[j][1] = reinterpret_cast<const uint4*>(row + j * 64)[1];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);            // this warp is done with the stage's weights
+#pragma unroll
+        for (int j = 0; j < SUB; ++j) {
+          if (!warp_wait(&aempty[abuf], aph ^ 1u)) {
+            aborted = true;
+            break;
+          }
+          const uint32_t x[8] = {w[j][0].x, w[j][0].y, w[j][0].z, w[j][0].w,
+                                 w[j][1].x, w[j][1].y, w[j][1].z, w[j][1].w};
+          uint32_t a[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) widen_t2_word(x[i], a + 4 * i);
+          tc_fence_after();
+          tmem_st_32x32b_x32(tmem_base + lane_addr + abuf * kTsACols + static_cast<uint32_t>(half * 32), a);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afull[abuf]);
+          if (++abuf == p.abufs) {
+            abuf = 0;
+            aph ^= 1u;
+          }
+        }
+        if (++s == p.stages) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (aborted) break;
+      // epilogue: lane = weight row n, columns = tokens; the two warps of a
+      // quadrant take alternate 8-column chunks
+      if (!warp_wait(dfull, static_cast<uint32_t>(local) & 1u)) {
+        aborted = true;
+        break;
+      }
+      tc_fence_after();
+      const int n = nb * kTsBN + trow;
+      const bool n_ok = n < p.N;
+      const float al = n_ok ? p.alpha[n / p.alpha_group] : 0.f;
+      for (int c = half; c < p.nt / 8; c += 2) {
+        uint32_t r[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (uint32_t slot = 0; slot < p.dslots; ++slot) {
+          uint32_t t[8];
+          tmem_ld_32x32b_x8(tmem_base + lane_addr + d_col + slot * static_cast<uint32_t>(p.nt) +
+                                static_cast<uint32_t>(c * 8),
+                            t);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) r[j] += t[j];
+        }
+        if (!n_ok) continue;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int m = mb * p.nt + c * 8 + j;
+          if (m >= p.M) break;
+          const int v = static_cast<int>(r[j]);
+          if (p.acc != nullptr) p.acc[static_cast<int64_t>(m) * p.N + n] = v;
+          if (p.y != nullptr) {
+            const float cs = __fmul_rn(p.a_scale[m], al);
+            const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__int2float_rn(v), cs));
+            p.y[static_cast<int64_t>(m) * p.ldy + n] = *reinterpret_cast<const uint16_t*>(&b);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dempty);
+    }
+  }
+
+  __syncthreads();
+  if (aborted) {
+    // let any copies or MMAs still in flight land before the CTA's memory goes away
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) {
+    }
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
 }
 
 // ---------------------------------------------------------------------------

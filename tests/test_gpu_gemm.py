@@ -205,5 +205,52 @@ def test_gemm_simt_parity(M, afmt, wfmt):
     assert bf16_rows_rel_err(y, ex) <= BF16_ROW_TOL
 
 
+# 2-bit weights x int8 activations on the tensor cores for M >= 8 (weights
+# widened into tensor memory; tokens on the MMA's N side: 8 for M = 8, else a
+# multiple of 16 up to 256 per token block); fewer tokens take the CUDA-core
+# kernel (test_gemm_simt_parity)
+GEMM_T2TC_CASES = [
+    ("M8_min_K", 8, 128, 64),
+    ("M8_ragged_N_K_tail", 8, 300, 320),
+    ("M8_two_tiles", 8, 256, 4096),
+    ("M12_K_tail_1088", 12, 136, 1088),
+    ("M9_nt16", 9, 130, 832),
+    ("M33_nt48", 33, 384, 768),
+    ("M100_nt112", 100, 200, 2048),
+    ("M256_nt256", 256, 129, 512),
+    ("M300_two_token_blocks", 300, 256, 256),
+    ("M64_K11008_down", 64, 160, 11008),
+]
+
+
+@pytest.mark.parametrize("name,M,N,K", GEMM_T2TC_CASES, ids=[c[0] for c in GEMM_T2TC_CASES])
+def test_gemm_t2_tensor_core_parity(name, M, N, K):
+    g = synth.rng(M * 13 + N + K)
+    a = g.integers(-128, 128, (M, K)).astype(np.int8)
+    t = g.integers(-1, 2, (N, K)).astype(np.int8)
+    scale = (g.random(M) * 0.1 + 1e-3).astype(np.float32)
+    alpha = np.float32(0.0173)
+    acc, y = run_gemm(to_dev(a), tba.BL_A_I8, scale, to_dev(oracle.pack_ternary2(t)), tba.BL_W_T2, alpha, M, N, K)
+    acc_ref, _ = oracle.gemm(a, scale, t, alpha, want_y=False)
+    assert np.array_equal(acc, acc_ref)
+    _, ex = exact_y(a, scale, t, alpha, N, np.arange(M))
+    assert bf16_rows_rel_err(y, ex) <= BF16_ROW_TOL
+
+
+def test_gemm_t2_tensor_core_alpha_groups_and_ldy():
+    M, F, K = 24, 192, 1024
+    g = synth.rng(33)
+    a = g.integers(-8, 8, (M, K)).astype(np.int8)
+    t = g.integers(-1, 2, (2 * F, K)).astype(np.int8)
+    scale = (g.random(M) + 0.5).astype(np.float32)
+    alpha = np.array([0.0151, 0.0213], np.float32)
+    acc, y = run_gemm(to_dev(a), tba.BL_A_I8, scale, to_dev(oracle.pack_ternary2(t)), tba.BL_W_T2, alpha, M,
+                      2 * F, K, group=F, ldy=2 * F + 64)
+    acc_ref, _ = oracle.gemm(a, scale, t, alpha, alpha_group=F, want_y=False)
+    assert np.array_equal(acc, acc_ref)
+    _, ex = exact_y(a, scale, t, alpha, F, np.arange(M))
+    assert bf16_rows_rel_err(y, ex) <= BF16_ROW_TOL
+
+
 def test_sync_status_clean():
     tba.sync_status()
