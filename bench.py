@@ -50,6 +50,11 @@ EPS = 1e-5
 # measured B200 peaks of this machine (generated file), else the documented fallback
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 INT8_PER_BF16 = 2.0   # nominal dense int8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
+# DRAM bytes (read + write) of the four GEMM launches of one step, from a one-pass ncu
+# capture of this benchmark (profiles/gemm_tc2_kernel__int8_16384x12288x4096.md gives the
+# command); algorithmic bytes of the same launches: 3.75 GB (A and W read once, Y written once)
+GEMM_STEP_DRAM_BYTES = 549892096 + 763724544 + 196653568 + 224203520 + 962767872 + 1400955648 + \
+    1338792960 + 251956480
 
 
 def load_peaks():
@@ -445,12 +450,14 @@ def run_gpu(args):
             "config": dict(workload_config(args.afmt, m), parallelism=f"replicas x{world}"),
             "roofline": {
                 "bound": "tensor",
-                "kernel": "gemm_tc_kernel (tcgen05 kind::i8)",
+                "kernel": "gemm_tc2_kernel (tcgen05 kind::i8, CTA pairs)",
                 "achieved": round(tops, 1),
                 "peak": round(peak_int8, 1),
                 "unit": "TFLOP/s",
                 "frac": round(tops / peak_int8, 4),
-                "traffic": None,
+                "traffic": GEMM_STEP_DRAM_BYTES if args.afmt == "int4" else None,
+                "traffic_note": "DRAM read+write bytes of the 4 GEMM launches of one step (ncu, one pass); "
+                                "algorithmic 3.75e9",
                 "peak_note": f"int8 = {INT8_PER_BF16:g} x {peaks['source']} {'burst' if burst else 'sustained'} "
                              f"bf16 cuBLAS ({peaks[basis]} TFLOP/s; nominal dense int8:bf16 ratio)",
                 "work": "dense-equivalent 2*M*N*K over the 4 GEMM launches of a step / their summed event time",
@@ -693,6 +700,7 @@ PROFILE_CASES = {
     "kv_quant3": "3-bit KV, K bf16 [32768 x 32 x 128]",
     "pack_ternary": "ternary pack to int8, W fp32 [22016 x 4096]",
     "gemm_decode": "CUDA-core GEMM, 2-bit W [12288 x 4096], 1 token",
+    "gemm_decode_tc": "tcgen05 GEMM, 2-bit W [12288 x 4096] widened into TMEM, 16 tokens",
 }
 
 
@@ -718,6 +726,14 @@ def run_profile_case(name: str, launches: int):
         fn = lambda: tba.bitlinear_gemm(a, s, w, al, M, N, K, y=y)
     elif name == "gemm_decode":
         M, N, K = 1, 12288, 4096
+        a = torch.randint(-8, 8, (M, K), generator=g, device=dev, dtype=torch.int8)
+        w = torch.randint(0, 256, (N, K // 4), generator=g, device=dev, dtype=torch.int32).to(torch.uint8)
+        s = torch.rand((M,), generator=g, device=dev)
+        al = torch.full((1,), 0.0173, device=dev)
+        y = torch.empty((M, N), dtype=torch.int16, device=dev)
+        fn = lambda: tba.bitlinear_gemm(a, s, w, al, M, N, K, y=y, wfmt=tba.BL_W_T2)
+    elif name == "gemm_decode_tc":
+        M, N, K = 16, 12288, 4096
         a = torch.randint(-8, 8, (M, K), generator=g, device=dev, dtype=torch.int8)
         w = torch.randint(0, 256, (N, K // 4), generator=g, device=dev, dtype=torch.int32).to(torch.uint8)
         s = torch.rand((M,), generator=g, device=dev)
