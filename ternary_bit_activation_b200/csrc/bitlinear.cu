@@ -261,9 +261,7 @@ bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int64_t ldw
     int64_t blocks = (total + bl::kBinThreads - 1) / bl::kBinThreads;
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
     if (blocks > cap) blocks = cap;
-    bl::ternary_bins_kernel<<<static_cast<unsigned>(blocks), bl::kBinThreads, 0, s>>>(w, N, k, ldw, bins);
-    if (launch_status() != BL_OK) return BL_ERR_CUDA;
-    bl::ternary_alpha_kernel<<<1, bl::kBins, 0, s>>>(bins, static_cast<unsigned long long>(N * K), alpha);
+    bl::ternary_bins_kernel<<<static_cast<unsigned>(blocks), bl::kBinThreads, 0, s>>>(w, N, k, ldw, bins, alpha);
     if (launch_status() != BL_OK) return BL_ERR_CUDA;
   }
   const int64_t total16 = N * (K / 16);
@@ -387,9 +385,7 @@ bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float 
     int64_t blocks = (total + bl::kBinThreads - 1) / bl::kBinThreads;
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
     if (blocks > cap) blocks = cap;
-    bl::ternary_bins_kernel<<<static_cast<unsigned>(blocks), bl::kBinThreads, 0, s>>>(w, N, k, ldw, bins);
-    if (launch_status() != BL_OK) return BL_ERR_CUDA;
-    bl::ternary_alpha_kernel<<<1, bl::kBins, 0, s>>>(bins, static_cast<unsigned long long>(N * K), alpha);
+    bl::ternary_bins_kernel<<<static_cast<unsigned>(blocks), bl::kBinThreads, 0, s>>>(w, N, k, ldw, bins, alpha);
     if (launch_status() != BL_OK) return BL_ERR_CUDA;
   }
   const int64_t total16 = N * (K / 16);

@@ -53,9 +53,15 @@ __device__ __forceinline__ void bins_flush(unsigned long long* sb, uint32_t ub, 
   }
 }
 
+__device__ void alpha_from_bins(const unsigned long long* gbins, unsigned long long D, float* alpha,
+                                unsigned long long* sb);
+
+// gbins (zeroed by the caller): bins 1..255 and, in bin 0, a count of finished
+// CTAs; the last CTA to finish computes alpha.
 __global__ void __launch_bounds__(kBinThreads) ternary_bins_kernel(const float* __restrict__ w, int64_t N, int K,
                                                                    int64_t ldw,
-                                                                   unsigned long long* __restrict__ gbins) {
+                                                                   unsigned long long* __restrict__ gbins,
+                                                                   float* __restrict__ alpha) {
   __shared__ unsigned long long sb[kBins];
   const int lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kBins; i += kBinThreads) sb[i] = 0ull;
@@ -112,6 +118,15 @@ __global__ void __launch_bounds__(kBinThreads) ternary_bins_kernel(const float* 
   __syncthreads();
   for (int b = threadIdx.x; b < kBins; b += kBinThreads)
     if (sb[b]) atomicAdd(&gbins[b], sb[b]);
+  // the last CTA to finish sees every CTA's bins and forms alpha
+  __threadfence();
+  __syncthreads();
+  __shared__ bool last;
+  if (threadIdx.x == 0) last = atomicAdd(&gbins[0], 1ull) == gridDim.x - 1u;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  alpha_from_bins(gbins, static_cast<unsigned long long>(N) * static_cast<unsigned long long>(K), alpha, sb);
 }
 
 // Multi-word unsigned integer, little-endian 32-bit limbs.
@@ -150,12 +165,13 @@ __device__ __forceinline__ unsigned long long big_window64(const uint32_t (&z)[k
   return bo ? ((lo >> bo) | (hi << (64 - bo))) : lo;
 }
 
-// alpha = RN_fp32( (Z * 2^-149) / D ),  Z = sum_e bins[e] << (e - 1); single thread.
-__global__ void __launch_bounds__(kBins) ternary_alpha_kernel(const unsigned long long* __restrict__ gbins,
-                                                               unsigned long long D, float* __restrict__ alpha) {
-  __shared__ unsigned long long sb[kBins];
+// alpha = RN_fp32( (Z * 2^-149) / D ),  Z = sum_e bins[e] << (e - 1), by the last
+// CTA of the binning kernel (bin 0 holds the CTA counter and is not a bin):
+// twelve threads form the limbs, thread 0 divides.
+__device__ void alpha_from_bins(const unsigned long long* gbins, unsigned long long D, float* alpha,
+                                unsigned long long* sb) {
   __shared__ unsigned long long limb_sum[kLimbs];
-  for (int e = threadIdx.x; e < kBins; e += blockDim.x) sb[e] = gbins[e];   // one round trip for all bins
+  for (int e = threadIdx.x; e < kBins; e += blockDim.x) sb[e] = e == 0 ? 0ull : __ldcg(gbins + e);
   __syncthreads();
   // thread l < kLimbs sums the 32-bit pieces of every shifted bin that fall in
   // limb l (at most 256 pieces < 2^32, so the sum stays below 2^40)
@@ -171,7 +187,7 @@ __global__ void __launch_bounds__(kBins) ternary_alpha_kernel(const unsigned lon
     limb_sum[l] = acc;
   }
   __syncthreads();
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  if (threadIdx.x != 0) return;
   uint32_t z[kLimbs];
   unsigned long long carry = 0;
   for (int i = 0; i < kLimbs; ++i) {
