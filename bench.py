@@ -179,8 +179,15 @@ class Layer:
         wts = synth.layer_weights(SHAPE, seed=3)
         self.w_lat = {k: dev_from(v) for k, v in wts.items()}
         del wts
-        self.w8 = {"qkv": T.empty((3 * d, d), dtype=u8, device=dev), "o": T.empty((d, d), dtype=u8, device=dev),
-                   "upgate": T.empty((2 * f, d), dtype=u8, device=dev), "down": T.empty((d, f), dtype=u8, device=dev)}
+        # QKV and Up|Gate take the INT4 inputs' int8 operand, or with FP4 inputs E2M1-coded weights
+        # (kind::mxf4 GEMM); O and Down always take the Top-K INT8 inputs and int8 weights
+        fp4 = afmt == "fp4"
+        kq = d // 2 if fp4 else d
+        self.wfmt_q = tba.BL_W_E2M1 if fp4 else tba.BL_W_I8
+        self.afmt_q = tba.BL_A_E2M1 if fp4 else tba.BL_A_I8
+        self.store_q = tba.BL_STORE_PACKED if fp4 else tba.BL_STORE_BYTES
+        self.w8 = {"qkv": T.empty((3 * d, kq), dtype=u8, device=dev), "o": T.empty((d, d), dtype=u8, device=dev),
+                   "upgate": T.empty((2 * f, kq), dtype=u8, device=dev), "down": T.empty((d, f), dtype=u8, device=dev)}
         self.alpha = T.zeros((8,), dtype=f32, device=dev)   # qkv, o, up, gate, down
         self.ws = T.empty((tba.workspace_size("pack_ternary") // 8,), dtype=T.int64, device=dev)
 
@@ -193,10 +200,10 @@ class Layer:
         self.x_sets = [[h.to(dev) for h in self.h_in] for _ in range(2)]
         self.x = self.x_sets[0]
 
-        qbytes = 1  # BL_STORE_BYTES: one int8 per element for the tensor-core operand
-        self.qa = T.empty((m, d * qbytes), dtype=u8, device=dev)
+        # BL_STORE_BYTES: one int8 per element; FP4: packed E2M1 nibbles
+        self.qa = T.empty((m, kq), dtype=u8, device=dev)
         self.qa_s = T.empty((m,), dtype=f32, device=dev)
-        self.qf = T.empty((m, d * qbytes), dtype=u8, device=dev)
+        self.qf = T.empty((m, kq), dtype=u8, device=dev)
         self.qf_s = T.empty((m,), dtype=f32, device=dev)
         self.o8 = T.empty((m, d), dtype=i8, device=dev)
         self.o8_s = T.empty((m,), dtype=f32, device=dev)
@@ -225,12 +232,16 @@ class Layer:
     def kernel_bytes(self):
         m, d, f, H, Dh = self.m, self.d, self.f, self.H, self.Dh
         kv_one = m * H * (2 * Dh + Dh * 3 // 8 + 4)
+        fp4 = self.afmt == "fp4"
+        qout = m * d // 2 if fp4 else m * d
+        wq = 4.5 if fp4 else 5      # fp32 read + E2M1 nibble or int8 written per weight
         return {
-            "quant_a4": 2 * (m * d * 2 + m * d + 4 * m),
+            "quant_a4": 2 * (m * d * 2 + qout + 4 * m),
             "sparsify_a8": m * d * 2 + m * d + 4 * m,
             "relu2_glu": m * f * 4 + m * f + 4 * m,
             "kv_quant3": 2 * kv_one,
-            "pack_ternary": sum(n * kk * 5 for n, kk in [(3 * d, d), (d, d), (2 * f, d), (d, f)]),
+            "pack_ternary": int(sum(n * kk * c for (n, kk), c in [((3 * d, d), wq), ((d, d), 5), ((2 * f, d), wq),
+                                                                  ((d, f), 5)])),
         }
 
     def step(self, ev=None):
@@ -253,18 +264,18 @@ class Layer:
 
         W, w8, al = self.w_lat, self.w8, self.alpha
         ws = self.ws
-        timed("pack_ternary", lambda: tba.pack_ternary(W["qkv"], al[0:1], w8["qkv"], tba.BL_W_I8, ws, eps=EPS))
+        wq, aq, sq = self.wfmt_q, self.afmt_q, self.store_q
+        timed("pack_ternary", lambda: tba.pack_ternary(W["qkv"], al[0:1], w8["qkv"], wq, ws, eps=EPS))
         timed("pack_ternary", lambda: tba.pack_ternary(W["o"], al[1:2], w8["o"], tba.BL_W_I8, ws, eps=EPS))
-        timed("pack_ternary", lambda: tba.pack_ternary(W["up"], al[2:3], w8["upgate"][:f], tba.BL_W_I8, ws, eps=EPS))
-        timed("pack_ternary", lambda: tba.pack_ternary(W["gate"], al[3:4], w8["upgate"][f:], tba.BL_W_I8, ws,
-                                                       eps=EPS))
+        timed("pack_ternary", lambda: tba.pack_ternary(W["up"], al[2:3], w8["upgate"][:f], wq, ws, eps=EPS))
+        timed("pack_ternary", lambda: tba.pack_ternary(W["gate"], al[3:4], w8["upgate"][f:], wq, ws, eps=EPS))
         timed("pack_ternary", lambda: tba.pack_ternary(W["down"], al[4:5], w8["down"], tba.BL_W_I8, ws, eps=EPS))
         q = tba.BL_QUANT_FP4_E2M1 if fp4 else tba.BL_QUANT_INT4
         x_attn, x_o, x_ffn = self.x
         # attention block
-        timed("quant_a4", lambda: tba.bitlinear_quant_a4(x_attn, self.qa, self.qa_s, q, tba.BL_STORE_BYTES, EPS))
+        timed("quant_a4", lambda: tba.bitlinear_quant_a4(x_attn, self.qa, self.qa_s, q, sq, EPS))
         timed("gemm_qkv", lambda: tba.bitlinear_gemm(self.qa, self.qa_s, w8["qkv"], al[0:1], m, 3 * d, d,
-                                                     y=self.y_qkv))
+                                                     y=self.y_qkv, afmt=aq, wfmt=wq))
         for i, off in enumerate((d, 2 * d)):     # K and V slices of the QKV output
             timed("kv_quant3", lambda off=off, i=i: tba.kv_quant3(self.y_qkv[:, off:], m, H, Dh, self.kv_codes[i],
                                                                   self.kv_scale[i], self.kv_bos[i], bits=3,
@@ -273,9 +284,9 @@ class Layer:
                                                                self.o8_s, None, EPS))
         timed("gemm_o", lambda: tba.bitlinear_gemm(self.o8, self.o8_s, w8["o"], al[1:2], m, d, d, y=self.y_o))
         # FFN block
-        timed("quant_a4", lambda: tba.bitlinear_quant_a4(x_ffn, self.qf, self.qf_s, q, tba.BL_STORE_BYTES, EPS))
+        timed("quant_a4", lambda: tba.bitlinear_quant_a4(x_ffn, self.qf, self.qf_s, q, sq, EPS))
         timed("gemm_upgate", lambda: tba.bitlinear_gemm(self.qf, self.qf_s, w8["upgate"], al[2:4], m, 2 * f, d,
-                                                        y=self.y_ug, alpha_group=f))
+                                                        y=self.y_ug, alpha_group=f, afmt=aq, wfmt=wq))
         timed("relu2_glu", lambda: tba.relu2_glu(self.y_ug[:, f:], self.y_ug[:, :f],
                                                  synth.k_keep(f, SHAPE.topk_pct_down), self.h8, self.h8_s, None,
                                                  EPS, M=m, F=f, ld=2 * f))
@@ -419,6 +430,12 @@ def run_gpu(args):
         burst = (clk.get("sm_mhz") or 0) >= 0.95 * (clk.get("sm_max_mhz") or 1e9)
         basis = "bf16_tflops" if burst else "bf16_tflops_sustained"
         peak_int8 = peaks[basis] * INT8_PER_BF16
+        if args.afmt == "fp4":
+            # QKV and Up|Gate run as kind::mxf4 (nominal dense fp4 = 2 x int8): the step's peak is
+            # the ops-weighted harmonic combination of the two rates
+            ops_f4 = layer.gemm_ops["qkv"] + layer.gemm_ops["upgate"]
+            ops_i8 = layer.gemm_ops["o"] + layer.gemm_ops["down"]
+            peak_int8 = (ops_f4 + ops_i8) / (ops_f4 / (2 * peak_int8) + ops_i8 / peak_int8)
         kb = layer.kernel_bytes()
         kernels = {}
         for k, v in per_kernel.items():
@@ -445,12 +462,13 @@ def run_gpu(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "int8",
+            "dtype": "int8" if args.afmt == "int4" else "fp4(e2m1)+int8",
             "data": "synthetic (seeded; Gaussian QKV/FFN inputs, Student-t nu=3 O input, N(0,0.02) latent weights)",
             "config": dict(workload_config(args.afmt, m), parallelism=f"replicas x{world}"),
             "roofline": {
                 "bound": "tensor",
-                "kernel": "gemm_tc2_kernel (tcgen05 kind::i8, CTA pairs)",
+                "kernel": "gemm_tc2_kernel (tcgen05 kind::i8, CTA pairs)" if args.afmt == "int4" else
+                          "gemm_tc2_kernel (tcgen05 kind::mxf4 for QKV/Up|Gate, kind::i8 for O/Down, CTA pairs)",
                 "achieved": round(tops, 1),
                 "peak": round(peak_int8, 1),
                 "unit": "TFLOP/s",
@@ -459,7 +477,8 @@ def run_gpu(args):
                 "traffic_note": "DRAM read+write bytes of the 4 GEMM launches of one step (ncu, one pass); "
                                 "algorithmic 3.75e9",
                 "peak_note": f"int8 = {INT8_PER_BF16:g} x {peaks['source']} {'burst' if burst else 'sustained'} "
-                             f"bf16 cuBLAS ({peaks[basis]} TFLOP/s; nominal dense int8:bf16 ratio)",
+                             f"bf16 cuBLAS ({peaks[basis]} TFLOP/s; nominal dense int8:bf16 ratio)" +
+                             ("; fp4 = 2 x int8, combined by the ops of each kind" if args.afmt == "fp4" else ""),
                 "work": "dense-equivalent 2*M*N*K over the 4 GEMM launches of a step / their summed event time",
             },
             "gemm": {"tops_dense": round(tops, 1), "tops_algorithmic": round(alg_ops / (gemm_ms / 1e3) / 1e12, 1),

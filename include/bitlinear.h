@@ -71,7 +71,9 @@ typedef enum {
 /* Ternary weight formats (both K-major: row n holds the K codes of output n). */
 typedef enum {
     BL_W_T2 = 0,              /* 2-bit codes, 4 per byte, element 4i in bits 0-1: 0->00, +1->01, -1->11 */
-    BL_W_I8 = 1               /* one int8 in {-1,0,1} per element (tensor-core operand layout) */
+    BL_W_I8 = 1,              /* one int8 in {-1,0,1} per element (tensor-core operand layout) */
+    BL_W_E2M1 = 2             /* E2M1 nibbles, element 2i in bits 0-3: 0 -> 0x0, +1 -> 0x2, -1 -> 0xA
+                                 (the FP4 tensor-core operand for BL_A_E2M1 activations) */
 } bl_wfmt;
 
 /*
@@ -125,7 +127,7 @@ BL_API bl_status bitlinear_sparsify_a8(const void* x_bf16, int64_t M, int64_t K,
  * is an IEEE fp32 division.
  * w: [N x K] fp32, row stride ldw.  alpha: one device float; read as the
  * input when alpha_given != 0, written otherwise.  w_out: BL_W_T2 -> N x K/4
- * bytes, BL_W_I8 -> N x K bytes (layouts in bl_wfmt).
+ * bytes, BL_W_I8 -> N x K bytes, BL_W_E2M1 -> N x K/2 bytes (layouts in bl_wfmt).
  * workspace: device scratch of bitlinear_workspace_size("pack_ternary", N, K, 0)
  * bytes (2 KiB; cleared by the call itself).  Not needed when alpha_given != 0.
  * Requires K % 16 == 0, ldw % 4 == 0, N * K < 2^31.
@@ -176,6 +178,10 @@ BL_API bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int6
  * tensor cores too, the 2-bit weights widened to int8 into tensor memory as the
  * MMA's A operand (the tokens are the MMA's N side); other operand formats and
  * fewer tokens run on a CUDA-core kernel that reads packed operands directly.
+ * BL_A_E2M1 x BL_W_E2M1 (any M) runs on the tensor cores as kind::mxf4 with
+ * unit block scales and fp32 accumulation, exact for these operands (every
+ * partial sum is a multiple of 1/2 below 2^24); acc_out holds 2 * the sum.
+ * BL_W_E2M1 weights take BL_A_E2M1 activations only.
  * Requires K % 64 == 0, ldy % 8 == 0, 1 <= alpha_group.
  */
 BL_API bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale,

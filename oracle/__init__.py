@@ -272,6 +272,15 @@ def pack_ternary2(t: np.ndarray) -> np.ndarray:
     return out.astype(np.uint8)
 
 
+def pack_ternary_e2m1(t: np.ndarray) -> np.ndarray:
+    """Ternary codes as E2M1 nibbles along K (the FP4 tensor-core weight layout):
+    0 -> 0x0 (+0), +1 -> 0x2 (exponent 1, mantissa 0), -1 -> 0xA (sign | 0x2);
+    element 2i in bits 0-3."""
+    c = np.asarray(t).astype(np.int16)
+    e = np.where(c > 0, 0x2, np.where(c < 0, 0xA, 0x0)).astype(np.int16)
+    return pack_nibbles(e)
+
+
 def pack_mask_bits(mask: np.ndarray) -> np.ndarray:
     """Mask bits per row in uint32 words: bit j of word w is element 32w + j;
     rows padded to a whole number of words."""

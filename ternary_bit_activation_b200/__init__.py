@@ -25,7 +25,7 @@ BL_ERR_CUDA = STATUS_NAMES.index("BL_ERR_CUDA")
 BL_QUANT_INT4, BL_QUANT_FP4_E2M1 = 0, 1
 BL_STORE_PACKED, BL_STORE_BYTES = 0, 1
 BL_A_I8, BL_A_I4, BL_A_E2M1 = 0, 1, 2
-BL_W_T2, BL_W_I8 = 0, 1
+BL_W_T2, BL_W_I8, BL_W_E2M1 = 0, 1, 2
 
 EXPORTED = ["bitlinear_quant_a4", "bitlinear_sparsify_a8", "pack_ternary", "pack_ternary_noalloc", "bitlinear_gemm",
             "relu2_glu",
@@ -115,7 +115,7 @@ def bitlinear_sparsify_a8(x, k_keep, codes, scale, mask=None, eps=1e-5, stream=N
 
 
 def pack_ternary(w, alpha, w_out, wfmt=BL_W_T2, workspace=None, alpha_given=False, eps=1e-5, stream=None):
-    """Absmean ternary quantization (Eq. 2) into the 2-bit or int8 layout."""
+    """Absmean ternary quantization (Eq. 2) into the 2-bit, int8 or E2M1 layout."""
     N, K = w.shape
     ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("pack_ternary", lib().pack_ternary(_ptr(w), N, K, w.stride(0), eps, 1 if alpha_given else 0, _ptr(alpha),

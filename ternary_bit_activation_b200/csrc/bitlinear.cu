@@ -112,8 +112,10 @@ bool tc_kernel_ready() {
     if (!cuda_ok(cudaFuncSetAttribute(bl::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(bl::kTcSmemBytes))))
       return false;
-    if (!cuda_ok(cudaFuncSetAttribute(bl::gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      static_cast<int>(bl::kT2SmemBytes))))
+    if (!cuda_ok(cudaFuncSetAttribute(bl::gemm_tc2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(bl::kT2SmemBytes))) ||
+        !cuda_ok(cudaFuncSetAttribute(bl::gemm_tc2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(bl::kF4SmemBytes))))
       return false;
     if (!cuda_ok(cudaFuncSetAttribute(bl::gemm_t2tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       227 * 1024)) ||
@@ -244,7 +246,7 @@ extern "C" {
 
 bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int64_t ldw, float eps, int alpha_given,
                                float* alpha, bl_wfmt wfmt, void* w_out, void* stream) {
-  if (wfmt != BL_W_T2 && wfmt != BL_W_I8) return BL_ERR_ARG;
+  if (wfmt != BL_W_T2 && wfmt != BL_W_I8 && wfmt != BL_W_E2M1) return BL_ERR_ARG;
   if (N < 0 || K < 16 || (K & 15) || ldw < K || (ldw & 3) || K > 0x7FFFFFFF) return BL_ERR_SHAPE;
   if (N > 0 && N * K >= kNoallocMaxElems) return BL_ERR_SHAPE;
   if (!(eps >= 0.f)) return BL_ERR_ARG;
@@ -270,9 +272,11 @@ bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int64_t ldw
   if (blocks > cap) blocks = cap;
   uint8_t* out = static_cast<uint8_t*>(w_out);
   if (wfmt == BL_W_T2)
-    bl::ternary_pack_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+    bl::ternary_pack_kernel<BL_W_T2><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+  else if (wfmt == BL_W_E2M1)
+    bl::ternary_pack_kernel<BL_W_E2M1><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
   else
-    bl::ternary_pack_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+    bl::ternary_pack_kernel<BL_W_I8><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
   return launch_status();
 }
 
@@ -366,7 +370,7 @@ bl_status relu2_glu(const void* gate_bf16, const void* up_bf16, int64_t M, int64
 
 bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float eps, int alpha_given, float* alpha,
                        bl_wfmt wfmt, void* w_out, void* workspace, size_t ws_bytes, void* stream) {
-  if (wfmt != BL_W_T2 && wfmt != BL_W_I8) return BL_ERR_ARG;
+  if (wfmt != BL_W_T2 && wfmt != BL_W_I8 && wfmt != BL_W_E2M1) return BL_ERR_ARG;
   if (N < 0 || K < 16 || (K & 15) || ldw < K || (ldw & 3)) return BL_ERR_SHAPE;
   if (N > 0 && (N * K >= bl::kMaxPackElems || K > 0x7FFFFFFF)) return BL_ERR_SHAPE;
   if (!(eps >= 0.f)) return BL_ERR_ARG;
@@ -394,9 +398,11 @@ bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float 
   if (blocks > cap) blocks = cap;
   uint8_t* out = static_cast<uint8_t*>(w_out);
   if (wfmt == BL_W_T2)
-    bl::ternary_pack_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+    bl::ternary_pack_kernel<BL_W_T2><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+  else if (wfmt == BL_W_E2M1)
+    bl::ternary_pack_kernel<BL_W_E2M1><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
   else
-    bl::ternary_pack_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+    bl::ternary_pack_kernel<BL_W_I8><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
   return launch_status();
 }
 
@@ -404,7 +410,7 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
                          const float* alpha, int64_t alpha_group, int64_t M, int64_t N, int64_t K, void* y_bf16,
                          int64_t ldy, int32_t* acc_out, void* stream) {
   if (afmt != BL_A_I8 && afmt != BL_A_I4 && afmt != BL_A_E2M1) return BL_ERR_ARG;
-  if (wfmt != BL_W_T2 && wfmt != BL_W_I8) return BL_ERR_ARG;
+  if (wfmt != BL_W_T2 && wfmt != BL_W_I8 && wfmt != BL_W_E2M1) return BL_ERR_ARG;
   if (alpha_group < 1 || alpha_group > 0x7FFFFFFFLL) return BL_ERR_ARG;
   if (M < 0 || N < 1 || K < 64 || (K & 63) || K > (1 << 20) || M > 0x7FFFFFFFLL || N > 0x7FFFFFFFLL)
     return BL_ERR_SHAPE;
@@ -421,6 +427,32 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
   const uint8_t* W = static_cast<const uint8_t*>(w);
   uint16_t* Y = static_cast<uint16_t*>(y_bf16);
 
+  if (wfmt == BL_W_E2M1) {
+    // FP4 x FP4-coded ternary on the tensor cores (kind::mxf4, CTA pairs)
+    if (afmt != BL_A_E2M1) return BL_ERR_ARG;
+    if (!tc_kernel_ready()) return BL_ERR_CUDA;
+    CUtensorMap ta, tb;
+    if (!make_i8_map(&ta, A, static_cast<uint64_t>(M), static_cast<uint64_t>(K / 2), 128, bl::kTcBK) ||
+        !make_i8_map(&tb, W, static_cast<uint64_t>(N), static_cast<uint64_t>(K / 2), bl::kF4BN / 2, bl::kTcBK))
+      return BL_ERR_CUDA;
+    bl::TcParams p;
+    p.a_scale = a_scale;
+    p.alpha = alpha;
+    p.alpha_group = alpha_group;
+    p.M = m;
+    p.N = n;
+    p.K = k;
+    p.y = Y;
+    p.ldy = ldy;
+    p.acc = acc_out;
+    p.num_m_blocks = (m + bl::kT2BM - 1) / bl::kT2BM;
+    p.num_n_blocks = (n + bl::kF4BN - 1) / bl::kF4BN;
+    p.num_tiles = p.num_m_blocks * p.num_n_blocks;
+    p.num_kb = (k / 2 + bl::kTcBK - 1) / bl::kTcBK;
+    const int pairs = p.num_tiles < sm_count() / 2 ? p.num_tiles : sm_count() / 2;
+    bl::gemm_tc2_kernel<true><<<2 * pairs, bl::kT2Threads, bl::kF4SmemBytes, s>>>(ta, tb, p);
+    return launch_status();
+  }
   if (afmt == BL_A_I8 && wfmt == BL_W_I8 && M > bl::kTcBM) {
     // CTA-pair kernel: 256 x 256 tiles over clusters of two CTAs
     if (!tc_kernel_ready()) return BL_ERR_CUDA;
@@ -443,7 +475,7 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
     p.num_tiles = p.num_m_blocks * p.num_n_blocks;
     p.num_kb = (k + bl::kTcBK - 1) / bl::kTcBK;
     const int pairs = p.num_tiles < sm_count() / 2 ? p.num_tiles : sm_count() / 2;
-    bl::gemm_tc2_kernel<<<2 * pairs, bl::kT2Threads, bl::kT2SmemBytes, s>>>(ta, tb, p);
+    bl::gemm_tc2_kernel<false><<<2 * pairs, bl::kT2Threads, bl::kT2SmemBytes, s>>>(ta, tb, p);
     return launch_status();
   }
   if (afmt == BL_A_I8 && wfmt == BL_W_I8) {

@@ -297,6 +297,25 @@ constexpr size_t kT2SmemBytes = 1024 + kT2Stages * (kT2StageA + kT2StageB) + 256
 constexpr uint32_t kT2Idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(kT2BN) >> 3) << 17) |
                               ((static_cast<uint32_t>(kT2BM) >> 4) << 24);
 
+// FP4 variant (E2M1 activations x E2M1-coded ternary weights, kind::mxf4): a
+// 128-byte stage row holds 256 values, an MMA takes K = 64 (32 bytes), so the
+// same ring moves twice the K of the int8 kernel.  The fp32 accumulator holds
+// the exact sum (every partial sum is a multiple of 1/2 far below 2^24).  Tiles
+// are 256 x 224 so that two accumulators (2 x 224 TMEM columns) and the block
+// scales (64 columns, every byte 2^0 in UE8M0) fit in the 512 columns.
+constexpr int kF4BN = 224;
+constexpr uint32_t kF4StageB = (kF4BN / 2) * kTcBK;
+constexpr size_t kF4SmemBytes = 1024 + kT2Stages * (kT2StageA + kF4StageB) + 256;
+constexpr uint32_t kF4SfCol = 2 * kF4BN;    // scale-factor columns 448..511
+constexpr uint32_t kF4Idesc = (1u << 7) | (1u << 10) | ((static_cast<uint32_t>(kF4BN) >> 3) << 17) | (1u << 23) |
+                              ((static_cast<uint32_t>(kT2BM) >> 4) << 24);   // E2M1 x E2M1, UE8M0 scales, K = 64
+
+template <bool FP4>
+struct PairCfg {
+  static constexpr int BN = FP4 ? kF4BN : kT2BN;
+  static constexpr uint32_t StageB = FP4 ? kF4StageB : kT2StageB;
+};
+
 __device__ __forceinline__ void t2_tile_coords(int tile, int nmb, int nnb, int& mb, int& nb) {
   const int group = tile / (kT2GroupM * nnb);
   const int first_m = group * kT2GroupM;
@@ -307,6 +326,9 @@ __device__ __forceinline__ void t2_tile_coords(int tile, int nmb, int nnb, int& 
 }
 
 // One row's 32 consecutive accumulators -> y (bf16, scaled) and/or acc (int32).
+// FP4: the accumulators are fp32 sums of E2M1 values (multiples of 1/2); acc
+// receives twice the sum.
+template <bool FP4 = false>
 __device__ __forceinline__ void epilogue_chunk(const TcParams& p, int row, int n0, float rs, const uint32_t (&r)[32]) {
   const int group = static_cast<int>(p.alpha_group);   // host keeps alpha_group < 2^31
   const int ga = n0 / group;
@@ -316,7 +338,7 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams& p, int row, int n
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
     const float cs = one_alpha ? cs_uniform : __fmul_rn(rs, p.alpha[min(n0 + j, p.N - 1) / group]);
-    yv[j] = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), cs);
+    yv[j] = __fmul_rn(FP4 ? __uint_as_float(r[j]) : __int2float_rn(static_cast<int>(r[j])), cs);
   }
   const bool full_chunk = n0 + 32 <= p.N;
   if (p.y != nullptr) {
@@ -342,28 +364,35 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams& p, int row, int n
     }
   }
   if (p.acc != nullptr) {
+    uint32_t iv[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      iv[j] = FP4 ? static_cast<uint32_t>(__float2int_rn(__fmul_rn(__uint_as_float(r[j]), 2.f))) : r[j];
     int32_t* ar = p.acc + static_cast<int64_t>(row) * p.N + n0;
     if (full_chunk && (p.N & 3) == 0) {
 #pragma unroll
       for (int q = 0; q < 8; ++q)
-        reinterpret_cast<uint4*>(ar)[q] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+        reinterpret_cast<uint4*>(ar)[q] = make_uint4(iv[4 * q], iv[4 * q + 1], iv[4 * q + 2], iv[4 * q + 3]);
     } else {
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        if (n0 + j < p.N) ar[j] = static_cast<int32_t>(r[j]);
+        if (n0 + j < p.N) ar[j] = static_cast<int32_t>(iv[j]);
     }
   }
 }
 
 constexpr int kT2Threads = 320;  // warp 0: TMA, warp 1: MMA (leader), warps 2-9: epilogue
 
+template <bool FP4>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT2Threads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcParams p) {
+  constexpr int BN = PairCfg<FP4>::BN;
+  constexpr uint32_t SB = PairCfg<FP4>::StageB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kT2Stages * kT2StageA;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kT2Stages * kT2StageB);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + kT2Stages * SB);
   uint64_t* full = bars;
   uint64_t* empty = bars + kT2Stages;
   uint64_t* tfull = bars + 2 * kT2Stages;
@@ -400,6 +429,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT2Threads, 1)
   cluster_sync_all();   // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  if constexpr (FP4) {
+    // block scales: every byte 0x7F (2^0 in UE8M0) in columns 448..511 of all 128 lanes
+    if (warp >= 2 && warp < 6) {
+      uint32_t ones[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) ones[j] = 0x7F7F7F7Fu;
+      const uint32_t lanes = static_cast<uint32_t>((warp & 3) * 32) << 16;
+      tmem_st_32x32b_x32(tmem_base + lanes + kF4SfCol, ones);
+      tmem_st_32x32b_x32(tmem_base + lanes + kF4SfCol + 32, ones);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    cluster_sync_all();   // scales in place in both CTAs before the first MMA
+    tc_fence_after();
+  }
   bool aborted = false;
 
   if (warp == 0) {
@@ -416,9 +460,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT2Threads, 1)
             break;
           }
           const uint32_t leader_full = mapa_shared(smem_u32(&full[s]), 0);
-          if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kT2StageA + kT2StageB));
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kT2StageA + SB));
           tma_load_2d_pair(&tmA, leader_full, sA + s * kT2StageA, kb * kTcBK, mb * kT2BM + rank * 128);
-          tma_load_2d_pair(&tmB, leader_full, sB + s * kT2StageB, kb * kTcBK, nb * kT2BN + rank * 128);
+          tma_load_2d_pair(&tmB, leader_full, sB + s * SB, kb * kTcBK, nb * BN + rank * (BN / 2));
           if (++s == kT2Stages) {
             s = 0;
             ph ^= 1u;
@@ -440,7 +484,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT2Threads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kT2BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait_bounded(&full[s], ph)) {
             aborted = true;
@@ -448,11 +492,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT2Threads, 1)
           }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * kT2StageA);
-          const uint32_t b0 = smem_u32(sB + s * kT2StageB);
+          const uint32_t b0 = smem_u32(sB + s * SB);
 #pragma unroll
           for (int kk = 0; kk < kTcBK / 32; ++kk) {
-            mma_i8_pair(d_tmem, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), kT2Idesc,
-                        (kb | kk) != 0 ? 1u : 0u);
+            if constexpr (FP4) {
+              mma_mxf4_pair(d_tmem, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), kF4Idesc,
+                            tmem_base + kF4SfCol, tmem_base + kF4SfCol + 32, (kb | kk) != 0 ? 1u : 0u);
+            } else {
+              mma_i8_pair(d_tmem, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), kT2Idesc,
+                          (kb | kk) != 0 ? 1u : 0u);
+            }
           }
           // free stage s in both CTAs once these MMAs have read it
           mma_commit_pair(mapa_shared(smem_u32(&empty[s]), 0));
@@ -469,10 +518,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT2Threads, 1)
     }
   } else {
     // ---------------- epilogue (warps 2-9 of both CTAs) ----------------
-    // Two warps per TMEM lane quadrant, 128 columns (4 chunks of 32) each; the
+    // Two warps per TMEM lane quadrant, up to 4 chunks of 32 columns each; the
     // TMEM load of the next chunk is in flight while the current one is stored.
     const int quad = warp & 3;
-    const int c0 = ((warp - 2) >> 2) * 4;
+    constexpr int kChunks = BN / 32;
+    const int c_begin = ((warp - 2) >> 2) * 4;
+    const int c_end = min(c_begin + 4, kChunks);
     int local = 0;
     for (int tile = pair; tile < p.num_tiles; tile += npairs, ++local) {
       const int buf = local & 1;
@@ -487,16 +538,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT2Threads, 1)
       const int row = mb * kT2BM + static_cast<int>(rank) * 128 + quad * 32 + lane;
       const bool row_ok = row < p.M;
       const float rs = row_ok ? p.a_scale[row] : 0.f;
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * kT2BN);
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * BN);
       uint32_t ra[32], rb[32];
-      tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(c0 * 32), ra);
-      tmem_wait_ld();
+      if (c_begin < c_end) {
+        tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(c_begin * 32), ra);
+        tmem_wait_ld();
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
+        const int c = c_begin + i;
+        if (c >= c_end) break;
         uint32_t(&r)[32] = (i & 1) ? rb : ra;
-        if (i + 1 < 4) tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((c0 + i + 1) * 32), (i & 1) ? ra : rb);
-        const int n0 = nb * kT2BN + (c0 + i) * 32;
-        if (row_ok && n0 < p.N) epilogue_chunk(p, row, n0, rs, r);
+        if (c + 1 < c_end) tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>((c + 1) * 32), (i & 1) ? ra : rb);
+        const int n0 = nb * BN + c * 32;
+        if (row_ok && n0 < p.N) epilogue_chunk<FP4>(p, row, n0, rs, r);
         tmem_wait_ld();
       }
       tc_fence_before();

@@ -264,9 +264,10 @@ __device__ __forceinline__ int ternary_code(float w, float d, float h, bool fast
 }
 
 // t = RoundClip(w / (alpha + eps), -1, 1); 16 weights per thread-step.
-//   T2: 4 bytes out (2-bit codes, element 4i in bits 0-1; 0->00, +1->01, -1->11)
-//   I8: 16 bytes out
-template <bool T2>
+//   WF = BL_W_T2:   4 bytes out (2-bit codes, element 4i in bits 0-1; 0->00, +1->01, -1->11)
+//   WF = BL_W_I8:   16 bytes out
+//   WF = BL_W_E2M1: 8 bytes out (E2M1 nibbles, element 2i in bits 0-3; 0->0x0, +1->0x2, -1->0xA)
+template <int WF>
 __global__ void __launch_bounds__(256) ternary_pack_kernel(const float* __restrict__ w, int64_t N, int K,
                                                            int64_t ldw, const float* __restrict__ alpha,
                                                            float eps, uint8_t* __restrict__ out) {
@@ -301,11 +302,19 @@ __global__ void __launch_bounds__(256) ternary_pack_kernel(const float* __restri
           c[4 * j + 2] = ternary_code(__uint_as_float(v[h2][j].z), d, h, fast);
           c[4 * j + 3] = ternary_code(__uint_as_float(v[h2][j].w), d, h, fast);
         }
-        if constexpr (T2) {
+        if constexpr (WF == BL_W_T2) {
           uint32_t word = 0;
 #pragma unroll
           for (int j = 0; j < 16; ++j) word |= (static_cast<uint32_t>(c[j]) & 3u) << (2 * j);
           reinterpret_cast<uint32_t*>(out + n * static_cast<int64_t>(K >> 2))[q] = word;
+        } else if constexpr (WF == BL_W_E2M1) {
+          uint32_t lo = 0, hi = 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            lo |= ((c[j] != 0 ? 2u : 0u) | (c[j] < 0 ? 8u : 0u)) << (4 * j);
+            hi |= ((c[8 + j] != 0 ? 2u : 0u) | (c[8 + j] < 0 ? 8u : 0u)) << (4 * j);
+          }
+          reinterpret_cast<uint2*>(out + n * static_cast<int64_t>(K >> 1))[q] = make_uint2(lo, hi);
         } else {
           uint32_t wd[4];
 #pragma unroll

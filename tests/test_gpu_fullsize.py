@@ -159,6 +159,35 @@ def test_gemm_tc_full_7b(name, N, K):
     assert bf16_rows_rel_err(host(y, np.uint16)[rows], exact) <= BF16_ROW_TOL
 
 
+def test_gemm_fp4_mxf4_full_7b_qkv(acts):
+    """The FP4 variant's QKV GEMM at full size: FP4 E2M1 activations x
+    E2M1-coded ternary weights on kind::mxf4; sampled rows against the oracle."""
+    x = acts[0]
+    N, K = 3 * D, D
+    w = synth.latent_weights_f32(synth.rng(91), N, K)
+    t_ref, a_ref = oracle.ternary_quantize(w, EPS)
+    codes = empty((M, K // 2), torch.uint8)
+    scale = empty((M,), torch.float32)
+    tba.bitlinear_quant_a4(to_dev(x), codes, scale, tba.BL_QUANT_FP4_E2M1, tba.BL_STORE_PACKED, EPS)
+    wdev = empty((N, K // 2), torch.uint8)
+    alpha = empty((1,), torch.float32)
+    ws = empty((tba.workspace_size("pack_ternary") // 8,), torch.int64)
+    tba.pack_ternary(to_dev(w), alpha, wdev, tba.BL_W_E2M1, ws, eps=EPS)
+    acc = empty((M, N), torch.int32)
+    y = empty((M, N), torch.int16)
+    tba.bitlinear_gemm(codes, scale, wdev, alpha, M, N, K, y=y, acc=acc, afmt=tba.BL_A_E2M1, wfmt=tba.BL_W_E2M1)
+    tba.sync_status()
+    assert np.array_equal(host(wdev), oracle.pack_ternary_e2m1(t_ref))
+    rows = sample_rows(M, 40, 4)
+    code4, twice, _, s_ref = oracle.quant_fp4(x[rows])
+    assert np.array_equal(host(codes)[rows], oracle.pack_nibbles(code4))
+    acc_scale = (s_ref.astype(np.float64) / 2).astype(np.float32)
+    acc_ref, _ = oracle.gemm(twice, acc_scale, t_ref, a_ref, want_y=False)
+    assert np.array_equal(host(acc)[rows], acc_ref)
+    exact = acc_ref.astype(np.float64) * acc_scale[:, None].astype(np.float64) * float(a_ref)
+    assert bf16_rows_rel_err(host(y, np.uint16)[rows], exact) <= BF16_ROW_TOL
+
+
 @pytest.mark.parametrize("m", [1, 8])
 def test_decode_gemm_full_7b_qkv(up_weights, m):
     # 2-bit weights of a 7B-size matrix against m INT4-packed tokens

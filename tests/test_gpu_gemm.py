@@ -19,7 +19,8 @@ EPS = 1e-5
 def run_pack(w, wfmt, alpha_in=None):
     N, K = w.shape
     wd = to_dev(w)
-    out = empty((N, K // 4 if wfmt == tba.BL_W_T2 else K), torch.uint8)
+    width = {tba.BL_W_T2: K // 4, tba.BL_W_E2M1: K // 2}.get(wfmt, K)
+    out = empty((N, width), torch.uint8)
     ws = empty((tba.workspace_size("pack_ternary", 0, N, K) // 8,), torch.int64)
     alpha = empty((1,), torch.float32)
     if alpha_in is not None:
@@ -250,6 +251,75 @@ def test_gemm_t2_tensor_core_alpha_groups_and_ldy():
     assert np.array_equal(acc, acc_ref)
     _, ex = exact_y(a, scale, t, alpha, F, np.arange(M))
     assert bf16_rows_rel_err(y, ex) <= BF16_ROW_TOL
+
+
+# FP4: E2M1 activations x E2M1-coded ternary weights on the tensor cores
+# (kind::mxf4, unit block scales, exact fp32 sums; acc holds twice the sum)
+@pytest.mark.parametrize("name,make", PACK_CASES[:4], ids=[c[0] for c in PACK_CASES[:4]])
+def test_pack_ternary_e2m1_parity(name, make):
+    w = make()
+    out, alpha = run_pack(w, tba.BL_W_E2M1)
+    t_ref, a_ref = oracle.ternary_quantize(w, EPS)
+    assert np.float32(alpha).view(np.uint32) == np.float32(a_ref).view(np.uint32)
+    assert np.array_equal(out, oracle.pack_ternary_e2m1(t_ref))
+
+
+GEMM_FP4_CASES = [
+    ("one_row", 1, 224, 128),
+    ("K_tail_130x300x320", 130, 300, 320),
+    ("two_pair_tiles_300x448x1024", 300, 448, 1024),
+    ("ragged_257x520x3200", 257, 520, 3200),
+    ("many_tiles_1300x2304x1024", 1300, 2304, 1024),
+    ("K11008_512x256", 512, 256, 11008),
+]
+
+
+@pytest.mark.parametrize("name,M,N,K", GEMM_FP4_CASES, ids=[c[0] for c in GEMM_FP4_CASES])
+def test_gemm_fp4_mxf4_parity(name, M, N, K):
+    g = synth.rng(M * 5 + N + K)
+    x = synth.gaussian_bf16(g, (M, K), outlier_channels=(3,), outlier_scale=8.0)
+    w = synth.latent_weights_f32(g, N, K)
+    t_ref, a_ref = oracle.ternary_quantize(w, EPS)
+    code4, twice, _, scale = oracle.quant_fp4(x)
+    acc, y = run_gemm(to_dev(oracle.pack_nibbles(code4)), tba.BL_A_E2M1, scale,
+                      to_dev(oracle.pack_ternary_e2m1(t_ref)), tba.BL_W_E2M1, a_ref, M, N, K)
+    acc_scale = (scale.astype(np.float64) / 2).astype(np.float32)
+    acc_ref, _ = oracle.gemm(twice, acc_scale, t_ref, a_ref, want_y=False)
+    assert np.array_equal(acc, acc_ref)
+    _, ex = exact_y(twice, acc_scale, t_ref, a_ref, N, np.arange(M))
+    assert bf16_rows_rel_err(y, ex) <= BF16_ROW_TOL
+
+
+def test_gemm_fp4_end_to_end_alpha_groups():
+    # FP4 quantizer -> packed codes -> stacked Up|Gate E2M1 weights, one alpha each
+    M, F, K = 200, 448, 1536
+    g = synth.rng(35)
+    x = synth.gaussian_bf16(g, (M, K))
+    wu, wg = synth.latent_weights_f32(g, F, K), synth.latent_weights_f32(g, F, K)
+    tu, au = oracle.ternary_quantize(wu, EPS)
+    tg, ag = oracle.ternary_quantize(wg, EPS)
+    codes = empty((M, K // 2), torch.uint8)
+    scale = empty((M,), torch.float32)
+    tba.bitlinear_quant_a4(to_dev(x), codes, scale, quant=tba.BL_QUANT_FP4_E2M1, store=tba.BL_STORE_PACKED, eps=EPS)
+    wdev = empty((2 * F, K // 2), torch.uint8)
+    alpha = empty((2,), torch.float32)
+    ws = empty((tba.workspace_size("pack_ternary") // 8,), torch.int64)
+    tba.pack_ternary(to_dev(wu), alpha[0:1], wdev[:F], tba.BL_W_E2M1, ws, eps=EPS)
+    tba.pack_ternary(to_dev(wg), alpha[1:2], wdev[F:], tba.BL_W_E2M1, ws, eps=EPS)
+    y = empty((M, 2 * F), torch.int16)
+    acc = empty((M, 2 * F), torch.int32)
+    tba.bitlinear_gemm(codes, scale, wdev, alpha, M, 2 * F, K, y=y, acc=acc, afmt=tba.BL_A_E2M1,
+                       wfmt=tba.BL_W_E2M1, alpha_group=F)
+    tba.sync_status()
+    code4, twice, _, s_ref = oracle.quant_fp4(x)
+    assert np.array_equal(host(codes), oracle.pack_nibbles(code4))
+    t = np.concatenate([tu, tg])
+    al = np.array([au, ag], np.float32)
+    acc_scale = (s_ref.astype(np.float64) / 2).astype(np.float32)
+    acc_ref, _ = oracle.gemm(twice, acc_scale, t, al, alpha_group=F, want_y=False)
+    assert np.array_equal(host(acc), acc_ref)
+    _, ex = exact_y(twice, acc_scale, t, al, F, np.arange(M))
+    assert bf16_rows_rel_err(host(y, np.uint16), ex) <= BF16_ROW_TOL
 
 
 def test_sync_status_clean():

@@ -384,6 +384,12 @@ def test_kv_ranges_and_roundtrip_bound():
 def test_pack_layouts():
     assert oracle.pack_nibbles(np.array([1, -2], np.int8)).tolist() == [0xE1]
     assert oracle.pack_ternary2(np.array([1, -1, 0, 1], np.int8)).tolist() == [0x4D]
+    # ternary as E2M1 (FP4 weight layout): +1 -> 0x2, -1 -> 0xA, 0 -> 0x0, element 2i low nibble
+    assert oracle.pack_ternary_e2m1(np.array([1, -1, 0, 1], np.int8)).tolist() == [0xA2, 0x20]
+    # the same codes are what the FP4 quantizer writes for +1, -1 and 0 (scale 2^0 when max|x| = 6)
+    code4, twice, _, _ = oracle.quant_fp4(synth.f32_to_bf16_bits(np.array([[1.0, -1.0, 0.0, 6.0]], np.float32)))
+    assert code4[0].tolist() == [0x2, 0xA, 0x0, 0x7]
+    assert twice[0].tolist() == [2, -2, 0, 12]
     m = np.zeros((1, 40), np.uint8)
     m[0, [0, 31, 32, 39]] = 1
     assert oracle.pack_mask_bits(m).tolist() == [[0x80000001, 0x81]]
