@@ -174,7 +174,8 @@ BL_API bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int6
  * y: [M x N] bf16 with row stride ldy (nullable).  acc_out: [M x N] int32,
  * row stride N (nullable; a test aid).
  * Kernels: BL_A_I8 x BL_W_I8 runs on the tcgen05 tensor cores (kind::i8,
- * TMA-fed, TMEM accumulators); BL_A_I8 x BL_W_T2 with M >= 8 runs on the
+ * TMA-fed, TMEM accumulators); BL_A_I8 x BL_W_T2 with M <= 2 runs on a GEMV
+ * that widens the 2-bit codes in registers; with M >= 8 it runs on the
  * tensor cores too, the 2-bit weights widened to int8 into tensor memory as the
  * MMA's A operand (the tokens are the MMA's N side); other operand formats and
  * fewer tokens run on a CUDA-core kernel that reads packed operands directly.

@@ -502,6 +502,29 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
     bl::gemm_tc_kernel<<<grid, bl::kTcThreads, bl::kTcSmemBytes, s>>>(ta, tb, p);
     return launch_status();
   }
+  if (afmt == BL_A_I8 && wfmt == BL_W_T2 && M <= 2 && M * K <= 65536) {
+    // one or two tokens: register-widening GEMV, one pass over the 2-bit weights
+    static bool attr_done[kMaxDevices] = {};
+    const int d = current_device();
+    if (d < 0 || d >= kMaxDevices) return BL_ERR_CUDA;
+    if (!attr_done[d]) {
+      if (!cuda_ok(cudaFuncSetAttribute(bl::gemv_t2_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536)) ||
+          !cuda_ok(cudaFuncSetAttribute(bl::gemv_t2_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536)))
+        return BL_ERR_CUDA;
+      attr_done[d] = true;
+    }
+    const int64_t warps = (N + bl::kGvRows - 1) / bl::kGvRows;
+    const int64_t need = (warps + bl::kGvThreads / 32 - 1) / (bl::kGvThreads / 32);
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    const unsigned grid = static_cast<unsigned>(need < cap ? need : cap);
+    const size_t smem = static_cast<size_t>(M) * static_cast<size_t>(K);
+    const int8_t* A8 = static_cast<const int8_t*>(a);
+    if (M == 1)
+      bl::gemv_t2_kernel<1><<<grid, bl::kGvThreads, smem, s>>>(A8, a_scale, W, alpha, alpha_group, n, k, Y, ldy, acc_out);
+    else
+      bl::gemv_t2_kernel<2><<<grid, bl::kGvThreads, smem, s>>>(A8, a_scale, W, alpha, alpha_group, n, k, Y, ldy, acc_out);
+    return launch_status();
+  }
   if (afmt == BL_A_I8 && wfmt == BL_W_T2 && M >= bl::kTsMinTokens) {
     // 2-bit weights widened into tensor memory; tokens on the MMA's N side
     if (!tc_kernel_ready()) return BL_ERR_CUDA;

@@ -11,10 +11,11 @@
 // gemm_t2tc_kernel -- 2-bit ternary weights x int8 activations for 8..256
 //                     tokens (decode): weights widened to int8 in registers
 //                     and stored into tensor memory as the MMA's A operand.
+// gemv_t2_kernel   -- 1 or 2 tokens x 2-bit weights: 2-bit codes widened in
+//                     registers, activations from shared memory, dp4a.
 // gemm_simt_kernel -- CUDA-core kernel that reads packed operands directly
 //                     (2-bit ternary weights, INT4 / E2M1 nibbles); decode of
-//                     fewer than 8 tokens, where the packed weight bytes and
-//                     the latency of a few tiles set the time.
+//                     3 to 7 tokens and the packed activation formats.
 #pragma once
 
 #include "common.cuh"
@@ -870,6 +871,123 @@ __global__ void __launch_bounds__(kTsThreads, 1)
     tmem_dealloc(tmem_base, 512);
   }
 }
+
+// ---------------------------------------------------------------------------
+// gemv_t2_kernel -- 1 or 2 tokens against 2-bit ternary weights (decode).  A
+// warp takes 4 weight rows at a time; in each round of 4096 codes lane l loads
+// 2 x 16 bytes of every row (words 4l..4l+3 and 128+4l..128+4l+3 of the round,
+// so each load instruction reads 512 contiguous bytes), widens the 16-code
+// words to int8 in registers (byte permutes, no table) and dot-products them
+// with the matching activation words, read once per round from shared memory
+// and reused by the 4 rows.  Partial sums are reduced by shuffles.
+// ---------------------------------------------------------------------------
+constexpr int kGvRows = 4;          // weight rows per warp and pass
+constexpr int kGvThreads = 256;
+
+template <int MT>
+__global__ void __launch_bounds__(kGvThreads) gemv_t2_kernel(const int8_t* __restrict__ a,
+                                                             const float* __restrict__ a_scale,
+                                                             const uint8_t* __restrict__ w,
+                                                             const float* __restrict__ alpha, int64_t alpha_group,
+                                                             int N, int K, uint16_t* __restrict__ y, int64_t ldy,
+                                                             int32_t* __restrict__ acc_out) {
+  extern __shared__ uint4 gv_act[];   // MT rows of K int8 codes
+  const int lane = threadIdx.x & 31;
+  const int kw16 = K >> 4;            // 16-code words per row (16 bytes of int8 activations each)
+  const int64_t wrow_bytes = K >> 2;
+  const int rounds = (kw16 + 255) >> 8;            // 256 words (4096 codes) per round
+  const int64_t warp_id = (static_cast<int64_t>(blockIdx.x) * kGvThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kGvThreads) >> 5;
+
+  // this lane's weight words of round rd for rows n0.. (2 pieces of 4 words)
+  auto load_round = [&](int64_t n0, int rd, uint4 (&wv)[kGvRows][2]) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int wq = (rd << 8) + h * 128 + 4 * lane;
+      const bool ok = wq < kw16;                  // kw16 is a multiple of 4 (K % 64 == 0)
+#pragma unroll
+      for (int r = 0; r < kGvRows; ++r) {
+        const int64_t n = n0 + r < N ? n0 + r : n0;
+        wv[r][h] = ok ? ld_global_nc_v4(w + n * wrow_bytes + static_cast<int64_t>(wq) * 4) : make_uint4(0, 0, 0, 0);
+      }
+    }
+  };
+  // the first weight loads go out before the activations are staged: the two
+  // latencies overlap
+  uint4 wv[kGvRows][2];
+  if (warp_id * kGvRows < N) load_round(warp_id * kGvRows, 0, wv);
+  for (int i = threadIdx.x; i < MT * kw16; i += blockDim.x) {
+    const int m = i / kw16, q = i - m * kw16;
+    gv_act[i] = ld_global_nc_v4(a + static_cast<int64_t>(m) * K + static_cast<int64_t>(q) * 16);
+  }
+  __syncthreads();
+  bool first = true;
+  for (int64_t n0 = warp_id * kGvRows; n0 < N; n0 += nwarps * kGvRows) {
+    int acc[kGvRows][MT];
+#pragma unroll
+    for (int r = 0; r < kGvRows; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc[r][m] = 0;
+    for (int rd = 0; rd < rounds; ++rd) {
+      int wq[2];
+      bool ok[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        wq[h] = (rd << 8) + h * 128 + 4 * lane;
+        ok[h] = wq[h] < kw16;
+      }
+      if (!first) load_round(n0, rd, wv);
+      first = false;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (!ok[h]) continue;
+        // activation words of the 4 T2 words: 4 x 16 bytes per token
+        uint4 av[MT][4];
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) av[m][j] = gv_act[m * kw16 + wq[h] + j];
+#pragma unroll
+        for (int r = 0; r < kGvRows; ++r) {
+          const uint32_t x4[4] = {wv[r][h].x, wv[r][h].y, wv[r][h].z, wv[r][h].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t t[4];
+            widen_t2_word(x4[j], t);
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+              acc[r][m] = __dp4a(static_cast<int>(t[0]), static_cast<int>(av[m][j].x), acc[r][m]);
+              acc[r][m] = __dp4a(static_cast<int>(t[1]), static_cast<int>(av[m][j].y), acc[r][m]);
+              acc[r][m] = __dp4a(static_cast<int>(t[2]), static_cast<int>(av[m][j].z), acc[r][m]);
+              acc[r][m] = __dp4a(static_cast<int>(t[3]), static_cast<int>(av[m][j].w), acc[r][m]);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kGvRows; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc[r][m] = __reduce_add_sync(0xFFFFFFFFu, acc[r][m]);
+    // lane r * MT + m writes output (row n0 + r, token m)
+#pragma unroll
+    for (int r = 0; r < kGvRows; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const int64_t n = n0 + r;
+        if (lane == r * MT + m && n < N) {
+          const int v = acc[r][m];
+          if (acc_out != nullptr) acc_out[static_cast<int64_t>(m) * N + n] = v;
+          if (y != nullptr) {
+            const float cs = __fmul_rn(a_scale[m], alpha[n / alpha_group]);
+            const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__int2float_rn(v), cs));
+            y[static_cast<int64_t>(m) * ldy + n] = *reinterpret_cast<const uint16_t*>(&b);
+          }
+        }
+      }
+  }
+}
+
 
 // ---------------------------------------------------------------------------
 // CUDA-core kernel for packed operands.  One warp per output column n (a row

@@ -322,5 +322,21 @@ def test_gemm_fp4_end_to_end_alpha_groups():
     assert bf16_rows_rel_err(host(y, np.uint16), ex) <= BF16_ROW_TOL
 
 
+# one or two tokens against 2-bit weights: the register-widening GEMV
+@pytest.mark.parametrize("M", [1, 2])
+@pytest.mark.parametrize("N,K", [(1, 64), (7, 320), (130, 4096), (258, 4160), (37, 11008), (96, 640)])
+def test_gemv_t2_parity(M, N, K):
+    g = synth.rng(M * 1000 + N + K)
+    a = g.integers(-128, 128, (M, K)).astype(np.int8)
+    t = g.integers(-1, 2, (N, K)).astype(np.int8)
+    scale = (g.random(M) * 0.1 + 1e-3).astype(np.float32)
+    alpha = np.float32(0.0211)
+    acc, y = run_gemm(to_dev(a), tba.BL_A_I8, scale, to_dev(oracle.pack_ternary2(t)), tba.BL_W_T2, alpha, M, N, K)
+    acc_ref, _ = oracle.gemm(a, scale, t, alpha, want_y=False)
+    assert np.array_equal(acc, acc_ref)
+    _, ex = exact_y(a, scale, t, alpha, N, np.arange(M))
+    assert bf16_rows_rel_err(y, ex) <= BF16_ROW_TOL
+
+
 def test_sync_status_clean():
     tba.sync_status()
