@@ -36,7 +36,34 @@ bool cuda_ok(cudaError_t e) {
   return false;
 }
 
-bl_status launch_status() { return cuda_ok(cudaGetLastError()) ? BL_OK : BL_ERR_CUDA; }
+// The error of the last launch_pdl call of this thread that failed and has not
+// yet been reported by launch_status.
+thread_local cudaError_t t_launch_error = cudaSuccess;
+
+bl_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = t_launch_error;
+  t_launch_error = cudaSuccess;
+  return cuda_ok(e) ? BL_OK : BL_ERR_CUDA;
+}
+
+// Launch with programmatic stream serialization (see pdl_wait / pdl_trigger):
+// the kernel may start while the previous kernel of the stream finishes.
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  if (e != cudaSuccess) t_launch_error = e;
+}
 
 int current_device() {
   int d = 0;
@@ -139,10 +166,10 @@ void launch_quant_a4_c(const uint16_t* x, int64_t M, int K, int64_t ldx, bool fp
   const int64_t need = (M + 1) / 2;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   const dim3 grid(static_cast<unsigned>(need < cap ? need : cap));
-  if (!fp4 && packed) bl::quant_a4_kernel<C, false, true><<<grid, 256, 0, s>>>(x, M, K, ldx, eps, codes, scale);
-  if (!fp4 && !packed) bl::quant_a4_kernel<C, false, false><<<grid, 256, 0, s>>>(x, M, K, ldx, eps, codes, scale);
-  if (fp4 && packed) bl::quant_a4_kernel<C, true, true><<<grid, 256, 0, s>>>(x, M, K, ldx, eps, codes, scale);
-  if (fp4 && !packed) bl::quant_a4_kernel<C, true, false><<<grid, 256, 0, s>>>(x, M, K, ldx, eps, codes, scale);
+  if (!fp4 && packed) launch_pdl(bl::quant_a4_kernel<C, false, true>, grid, 256, 0, s, x, M, K, ldx, eps, codes, scale);
+  if (!fp4 && !packed) launch_pdl(bl::quant_a4_kernel<C, false, false>, grid, 256, 0, s, x, M, K, ldx, eps, codes, scale);
+  if (fp4 && packed) launch_pdl(bl::quant_a4_kernel<C, true, true>, grid, 256, 0, s, x, M, K, ldx, eps, codes, scale);
+  if (fp4 && !packed) launch_pdl(bl::quant_a4_kernel<C, true, false>, grid, 256, 0, s, x, M, K, ldx, eps, codes, scale);
 }
 
 // Top-K rows: one 256-thread CTA per row, persistent grid sized by the occupancy
@@ -167,7 +194,7 @@ bl_status launch_topk_rows(const uint16_t* x, const uint16_t* up, int64_t M, int
     per_sm = 1;
   const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
   const unsigned grid = static_cast<unsigned>(M < cap ? M : cap);
-  kern<<<grid, bl::kTkThreads, smem, s>>>(x, up, M, K, ldx, keep, eps, codes, scale, mask);
+  launch_pdl(kern, grid, bl::kTkThreads, smem, s, x, up, M, K, ldx, keep, eps, codes, scale, mask);
   return launch_status();
 }
 
@@ -194,7 +221,7 @@ bool launch_simt_mu(const uint8_t* a, const float* sc, const uint8_t* w, const f
   const int64_t blocks_needed = (warps_needed + 7) / 8;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   const unsigned grid = static_cast<unsigned>(blocks_needed < cap ? blocks_needed : cap);
-  kern<<<grid, 256, smem, s>>>(a, sc, w, al, g, M, N, K, y, ldy, acc);
+  launch_pdl(kern, grid, 256, smem, s, a, sc, w, al, g, M, N, K, y, ldy, acc);
   return true;
 }
 
@@ -263,7 +290,7 @@ bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int64_t ldw
     int64_t blocks = (total + bl::kBinThreads - 1) / bl::kBinThreads;
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
     if (blocks > cap) blocks = cap;
-    bl::ternary_bins_kernel<<<static_cast<unsigned>(blocks), bl::kBinThreads, 0, s>>>(w, N, k, ldw, bins, alpha);
+    launch_pdl(bl::ternary_bins_kernel, static_cast<unsigned>(blocks), bl::kBinThreads, 0, s, w, N, k, ldw, bins, alpha);
     if (launch_status() != BL_OK) return BL_ERR_CUDA;
   }
   const int64_t total16 = N * (K / 16);
@@ -272,11 +299,11 @@ bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int64_t ldw
   if (blocks > cap) blocks = cap;
   uint8_t* out = static_cast<uint8_t*>(w_out);
   if (wfmt == BL_W_T2)
-    bl::ternary_pack_kernel<BL_W_T2><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+    launch_pdl(bl::ternary_pack_kernel<BL_W_T2>, static_cast<unsigned>(blocks), 256, 0, s, w, N, k, ldw, alpha, eps, out);
   else if (wfmt == BL_W_E2M1)
-    bl::ternary_pack_kernel<BL_W_E2M1><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+    launch_pdl(bl::ternary_pack_kernel<BL_W_E2M1>, static_cast<unsigned>(blocks), 256, 0, s, w, N, k, ldw, alpha, eps, out);
   else
-    bl::ternary_pack_kernel<BL_W_I8><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+    launch_pdl(bl::ternary_pack_kernel<BL_W_I8>, static_cast<unsigned>(blocks), 256, 0, s, w, N, k, ldw, alpha, eps, out);
   return launch_status();
 }
 
@@ -389,7 +416,7 @@ bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float 
     int64_t blocks = (total + bl::kBinThreads - 1) / bl::kBinThreads;
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
     if (blocks > cap) blocks = cap;
-    bl::ternary_bins_kernel<<<static_cast<unsigned>(blocks), bl::kBinThreads, 0, s>>>(w, N, k, ldw, bins, alpha);
+    launch_pdl(bl::ternary_bins_kernel, static_cast<unsigned>(blocks), bl::kBinThreads, 0, s, w, N, k, ldw, bins, alpha);
     if (launch_status() != BL_OK) return BL_ERR_CUDA;
   }
   const int64_t total16 = N * (K / 16);
@@ -398,11 +425,11 @@ bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float 
   if (blocks > cap) blocks = cap;
   uint8_t* out = static_cast<uint8_t*>(w_out);
   if (wfmt == BL_W_T2)
-    bl::ternary_pack_kernel<BL_W_T2><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+    launch_pdl(bl::ternary_pack_kernel<BL_W_T2>, static_cast<unsigned>(blocks), 256, 0, s, w, N, k, ldw, alpha, eps, out);
   else if (wfmt == BL_W_E2M1)
-    bl::ternary_pack_kernel<BL_W_E2M1><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+    launch_pdl(bl::ternary_pack_kernel<BL_W_E2M1>, static_cast<unsigned>(blocks), 256, 0, s, w, N, k, ldw, alpha, eps, out);
   else
-    bl::ternary_pack_kernel<BL_W_I8><<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, k, ldw, alpha, eps, out);
+    launch_pdl(bl::ternary_pack_kernel<BL_W_I8>, static_cast<unsigned>(blocks), 256, 0, s, w, N, k, ldw, alpha, eps, out);
   return launch_status();
 }
 
@@ -450,7 +477,7 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
     p.num_tiles = p.num_m_blocks * p.num_n_blocks;
     p.num_kb = (k / 2 + bl::kTcBK - 1) / bl::kTcBK;
     const int pairs = p.num_tiles < sm_count() / 2 ? p.num_tiles : sm_count() / 2;
-    bl::gemm_tc2_kernel<true><<<2 * pairs, bl::kT2Threads, bl::kF4SmemBytes, s>>>(ta, tb, p);
+    launch_pdl(bl::gemm_tc2_kernel<true>, 2 * pairs, bl::kT2Threads, bl::kF4SmemBytes, s, ta, tb, p);
     return launch_status();
   }
   if (afmt == BL_A_I8 && wfmt == BL_W_I8 && M > bl::kTcBM) {
@@ -475,7 +502,7 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
     p.num_tiles = p.num_m_blocks * p.num_n_blocks;
     p.num_kb = (k + bl::kTcBK - 1) / bl::kTcBK;
     const int pairs = p.num_tiles < sm_count() / 2 ? p.num_tiles : sm_count() / 2;
-    bl::gemm_tc2_kernel<false><<<2 * pairs, bl::kT2Threads, bl::kT2SmemBytes, s>>>(ta, tb, p);
+    launch_pdl(bl::gemm_tc2_kernel<false>, 2 * pairs, bl::kT2Threads, bl::kT2SmemBytes, s, ta, tb, p);
     return launch_status();
   }
   if (afmt == BL_A_I8 && wfmt == BL_W_I8) {
@@ -499,7 +526,7 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
     p.num_tiles = p.num_m_blocks * p.num_n_blocks;
     p.num_kb = (k + bl::kTcBK - 1) / bl::kTcBK;
     const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
-    bl::gemm_tc_kernel<<<grid, bl::kTcThreads, bl::kTcSmemBytes, s>>>(ta, tb, p);
+    launch_pdl(bl::gemm_tc_kernel, grid, bl::kTcThreads, bl::kTcSmemBytes, s, ta, tb, p);
     return launch_status();
   }
   if (afmt == BL_A_I8 && wfmt == BL_W_T2 && M <= 2 && M * K <= 65536) {
@@ -520,9 +547,9 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
     const size_t smem = static_cast<size_t>(M) * static_cast<size_t>(K);
     const int8_t* A8 = static_cast<const int8_t*>(a);
     if (M == 1)
-      bl::gemv_t2_kernel<1><<<grid, bl::kGvThreads, smem, s>>>(A8, a_scale, W, alpha, alpha_group, n, k, Y, ldy, acc_out);
+      launch_pdl(bl::gemv_t2_kernel<1>, grid, bl::kGvThreads, smem, s, A8, a_scale, W, alpha, alpha_group, n, k, Y, ldy, acc_out);
     else
-      bl::gemv_t2_kernel<2><<<grid, bl::kGvThreads, smem, s>>>(A8, a_scale, W, alpha, alpha_group, n, k, Y, ldy, acc_out);
+      launch_pdl(bl::gemv_t2_kernel<2>, grid, bl::kGvThreads, smem, s, A8, a_scale, W, alpha, alpha_group, n, k, Y, ldy, acc_out);
     return launch_status();
   }
   if (afmt == BL_A_I8 && wfmt == BL_W_T2 && M >= bl::kTsMinTokens) {
@@ -559,9 +586,9 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
     p.abufs = ab > static_cast<uint32_t>(bl::kTsMaxABufs) ? static_cast<uint32_t>(bl::kTsMaxABufs) : ab;
     const size_t smem = 1024 + static_cast<size_t>(p.stages) * per_stage + 512;   // + barriers
     const int grid = p.num_units < sm_count() ? p.num_units : sm_count();
-    if (sub == 4) bl::gemm_t2tc_kernel<4><<<grid, bl::kTsThreads, smem, s>>>(tx, tw, p);
-    else if (sub == 2) bl::gemm_t2tc_kernel<2><<<grid, bl::kTsThreads, smem, s>>>(tx, tw, p);
-    else bl::gemm_t2tc_kernel<1><<<grid, bl::kTsThreads, smem, s>>>(tx, tw, p);
+    if (sub == 4) launch_pdl(bl::gemm_t2tc_kernel<4>, grid, bl::kTsThreads, smem, s, tx, tw, p);
+    else if (sub == 2) launch_pdl(bl::gemm_t2tc_kernel<2>, grid, bl::kTsThreads, smem, s, tx, tw, p);
+    else launch_pdl(bl::gemm_t2tc_kernel<1>, grid, bl::kTsThreads, smem, s, tx, tw, p);
     return launch_status();
   }
   const bool t2 = wfmt == BL_W_T2;
@@ -608,10 +635,10 @@ bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D, int64_
   const int64_t bos = has_bos ? bos_pos : -1;
   const int h = static_cast<int>(H);
   switch (tpv) {
-    case 2: bl::kv_quant_kernel<2><<<grid, 256, 0, s>>>(kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
-    case 4: bl::kv_quant_kernel<4><<<grid, 256, 0, s>>>(kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
-    case 8: bl::kv_quant_kernel<8><<<grid, 256, 0, s>>>(kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
-    case 16: bl::kv_quant_kernel<16><<<grid, 256, 0, s>>>(kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
+    case 2: launch_pdl(bl::kv_quant_kernel<2>, grid, 256, 0, s, kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
+    case 4: launch_pdl(bl::kv_quant_kernel<4>, grid, 256, 0, s, kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
+    case 8: launch_pdl(bl::kv_quant_kernel<8>, grid, 256, 0, s, kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
+    case 16: launch_pdl(bl::kv_quant_kernel<16>, grid, 256, 0, s, kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
     default: return BL_ERR_SHAPE;
   }
   return launch_status();

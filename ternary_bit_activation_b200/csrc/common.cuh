@@ -25,6 +25,37 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ void raise_status(int code) { atomicCAS(&g_status, 0, code); }
 
+// Programmatic dependent launch: every kernel of this library is launched with
+// programmatic stream serialization.  pdl_wait blocks until the previous grid of
+// the stream has finished and its writes are visible; pdl_trigger lets the next
+// kernel start.  Each kernel does only on-chip setup (barriers, tensor memory)
+// and L2 prefetches before its wait, and triggers right after it, so the next
+// kernel's launch and prologue overlap this one while at most one kernel runs
+// ahead of its inputs.  (Both are no-ops without the launch attribute.)
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Loads of data that an earlier kernel of the stream may have written.  They are
+// volatile asm so that they stay behind pdl_wait: an ordinary load through a
+// const __restrict__ pointer counts as invariant for the whole kernel and may
+// be scheduled above the wait.
+__device__ __forceinline__ float ld_dep_f32(const float* p) {
+  float r;
+  asm volatile("ld.global.f32 %0, [%1];" : "=f"(r) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint4 ld_dep_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+// L2 prefetch hint (no data returned; safe on data a predecessor is still writing:
+// L2 is the point of coherence).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t h16) {
   return __uint_as_float(h16 << 16);
 }
@@ -162,6 +193,12 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* ba
           smem_u32(smem_dst)),
       "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
+}
+
+// L2 prefetch of the tile a tma_load_2d with the same map and coordinates would copy
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {

@@ -124,6 +124,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The next kernel may start once every CTA holds its tensor memory (a later
+  // allocation on this SM then waits for this CTA, never the reverse) and has
+  // passed its own wait (so at most one kernel runs ahead of its inputs).
+  pdl_wait();
+  pdl_trigger();
   bool aborted = false;
 
   if (warp == 0) {
@@ -203,7 +208,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_tile_coords(tile, p.num_m_blocks, p.num_n_blocks, mb, nb);
       const int row = mb * kTcBM + quad * 32 + lane;
       const bool row_ok = row < p.M;
-      const float rs = row_ok ? p.a_scale[row] : 0.f;
+      const float rs = row_ok ? ld_dep_f32(p.a_scale + row) : 0.f;
 #pragma unroll 1
       for (int c = 0; c < kTcBN / 32; ++c) {
         uint32_t r[32];
@@ -215,12 +220,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!row_ok || n0 >= p.N) continue;
         const int64_t ga = n0 / p.alpha_group;
         const bool one_alpha = ((n0 + 31) / p.alpha_group) == ga;
-        const float cs_uniform = __fmul_rn(rs, p.alpha[one_alpha ? ga : 0]);
+        const float cs_uniform = __fmul_rn(rs, ld_dep_f32(p.alpha + (one_alpha ? ga : 0)));
         float yv[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const float cs = one_alpha ? cs_uniform
-                                     : __fmul_rn(rs, p.alpha[min(static_cast<int64_t>(n0 + j), static_cast<int64_t>(p.N - 1)) / p.alpha_group]);
+                                     : __fmul_rn(rs, ld_dep_f32(p.alpha + min(static_cast<int64_t>(n0 + j), static_cast<int64_t>(p.N - 1)) / p.alpha_group));
           yv[j] = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), cs);
         }
         const bool full_chunk = n0 + 32 <= p.N;
@@ -334,11 +339,11 @@ __device__ __forceinline__ void epilogue_chunk(const TcParams& p, int row, int n
   const int group = static_cast<int>(p.alpha_group);   // host keeps alpha_group < 2^31
   const int ga = n0 / group;
   const bool one_alpha = (n0 + 31) / group == ga;
-  const float cs_uniform = __fmul_rn(rs, p.alpha[ga]);
+  const float cs_uniform = __fmul_rn(rs, ld_dep_f32(p.alpha + ga));
   float yv[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
-    const float cs = one_alpha ? cs_uniform : __fmul_rn(rs, p.alpha[min(n0 + j, p.N - 1) / group]);
+    const float cs = one_alpha ? cs_uniform : __fmul_rn(rs, ld_dep_f32(p.alpha + min(n0 + j, p.N - 1) / group));
     yv[j] = __fmul_rn(FP4 ? __uint_as_float(r[j]) : __int2float_rn(static_cast<int>(r[j])), cs);
   }
   const bool full_chunk = n0 + 32 <= p.N;
@@ -445,6 +450,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT2Threads, 1)
     cluster_sync_all();   // scales in place in both CTAs before the first MMA
     tc_fence_after();
   }
+  pdl_wait();
+  pdl_trigger();   // after the tensor-memory allocation and the wait, as in gemm_tc_kernel
   bool aborted = false;
 
   if (warp == 0) {
@@ -538,7 +545,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT2Threads, 1)
       t2_tile_coords(tile, p.num_m_blocks, p.num_n_blocks, mb, nb);
       const int row = mb * kT2BM + static_cast<int>(rank) * 128 + quad * 32 + lane;
       const bool row_ok = row < p.M;
-      const float rs = row_ok ? p.a_scale[row] : 0.f;
+      const float rs = row_ok ? ld_dep_f32(p.a_scale + row) : 0.f;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * BN);
       uint32_t ra[32], rb[32];
       if (c_begin < c_end) {
@@ -685,6 +692,13 @@ __global__ void __launch_bounds__(kTsThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t d_col = p.abufs * kTsACols;  // accumulators follow the A buffers
+  if (warp == 0 && lane == 0 && blockIdx.x < p.num_units) {
+    // pull the first unit's weight tiles into L2 while the previous kernel finishes
+    const int nb = blockIdx.x % p.num_n_tiles;
+    for (int kb = 0; kb < p.num_kb; ++kb) tma_prefetch_2d(&tmW, kb * (kRowBytes / 8), nb * kTsBN);
+  }
+  pdl_wait();
+  pdl_trigger();   // after the tensor-memory allocation and the wait, as in gemm_tc_kernel
   bool aborted = false;
 
   if (warp == 0) {
@@ -827,7 +841,7 @@ __global__ void __launch_bounds__(kTsThreads, 1)
       tc_fence_after();
       const int n = nb * kTsBN + trow;
       const bool n_ok = n < p.N;
-      const float al = n_ok ? p.alpha[n / p.alpha_group] : 0.f;
+      const float al = n_ok ? ld_dep_f32(p.alpha + n / p.alpha_group) : 0.f;
       for (int c = half; c < p.nt / 8; c += 2) {
         uint32_t r[8] = {0, 0, 0, 0, 0, 0, 0, 0};
         for (uint32_t slot = 0; slot < p.dslots; ++slot) {
@@ -847,7 +861,7 @@ __global__ void __launch_bounds__(kTsThreads, 1)
           const int v = static_cast<int>(r[j]);
           if (p.acc != nullptr) p.acc[static_cast<int64_t>(m) * p.N + n] = v;
           if (p.y != nullptr) {
-            const float cs = __fmul_rn(p.a_scale[m], al);
+            const float cs = __fmul_rn(ld_dep_f32(p.a_scale + m), al);
             const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__int2float_rn(v), cs));
             p.y[static_cast<int64_t>(m) * p.ldy + n] = *reinterpret_cast<const uint16_t*>(&b);
           }
@@ -912,6 +926,13 @@ __global__ void __launch_bounds__(kGvThreads) gemv_t2_kernel(const int8_t* __res
       }
     }
   };
+  // pull this warp's weight rows into L2 while the previous kernel finishes
+  for (int64_t n0 = warp_id * kGvRows; n0 < N; n0 += nwarps * kGvRows)
+    for (int r = 0; r < kGvRows && n0 + r < N; ++r)
+      for (int64_t b = static_cast<int64_t>(lane) * 128; b < wrow_bytes; b += 32 * 128)
+        prefetch_l2(w + (n0 + r) * wrow_bytes + b);
+  pdl_wait();
+  pdl_trigger();
   // the first weight loads go out before the activations are staged: the two
   // latencies overlap
   uint4 wv[kGvRows][2];
@@ -979,7 +1000,7 @@ __global__ void __launch_bounds__(kGvThreads) gemv_t2_kernel(const int8_t* __res
           const int v = acc[r][m];
           if (acc_out != nullptr) acc_out[static_cast<int64_t>(m) * N + n] = v;
           if (y != nullptr) {
-            const float cs = __fmul_rn(a_scale[m], alpha[n / alpha_group]);
+            const float cs = __fmul_rn(ld_dep_f32(a_scale + m), ld_dep_f32(alpha + n / alpha_group));
             const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__int2float_rn(v), cs));
             y[static_cast<int64_t>(m) * ldy + n] = *reinterpret_cast<const uint16_t*>(&b);
           }
@@ -1027,14 +1048,14 @@ __device__ __forceinline__ void load_a_unit(const uint8_t* a_row, int u, uint32_
     const uint4* p = reinterpret_cast<const uint4*>(a_row + static_cast<int64_t>(u) * 64);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint4 v = p[i];
+      const uint4 v = ld_dep_v4(p + i);
       out[4 * i] = v.x; out[4 * i + 1] = v.y; out[4 * i + 2] = v.z; out[4 * i + 3] = v.w;
     }
   } else {
     const uint4* p = reinterpret_cast<const uint4*>(a_row + static_cast<int64_t>(u) * 32);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      const uint4 v = p[i];
+      const uint4 v = ld_dep_v4(p + i);
       const uint32_t pk[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -1105,6 +1126,8 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const uint8_t* __restric
   const int64_t a_row_bytes = (AF == kSimtA_I8) ? K : (K >> 1);
   const int64_t w_row_bytes = WT2 ? (K >> 2) : K;
   const float unit_scale = (AF == kSimtA_E2M1) ? 0.5f : 1.0f;
+  pdl_wait();
+  pdl_trigger();
 
   for (int m0 = 0; m0 < M; m0 += MT) {
     __syncthreads();  // the previous tile's readers are done with sa
@@ -1190,7 +1213,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const uint8_t* __restric
               const int v = acc[r][m];
               if (acc_out != nullptr) acc_out[static_cast<int64_t>(mm) * N + n] = v;
               if (y != nullptr) {
-                const float cs = __fmul_rn(__fmul_rn(a_scale[mm], unit_scale), alpha[n / alpha_group]);
+                const float cs = __fmul_rn(__fmul_rn(ld_dep_f32(a_scale + mm), unit_scale), ld_dep_f32(alpha + n / alpha_group));
                 const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__int2float_rn(v), cs));
                 y[static_cast<int64_t>(mm) * ldy + n] = *reinterpret_cast<const uint16_t*>(&b);
               }

@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(256) kv_quant_kernel(const uint16_t* __restric
   p.t = group / uh;
   p.h = group - p.t * uh;
   uint4 v[kKvItems][2];
+  pdl_wait();
+  pdl_trigger();
   kv_load<TPV>(kv, p, dt, dh, ngroups, uh, nvec, ldt, sub, v);
   // rounds continue while the warp's first group has a vector left, so every
   // lane takes part in every shuffle (lanes past the end only skip their stores)

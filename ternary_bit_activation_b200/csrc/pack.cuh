@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(kBinThreads) ternary_bins_kernel(const float* 
   const int lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kBins; i += kBinThreads) sb[i] = 0ull;
   __syncthreads();
+  pdl_wait();
+  pdl_trigger();
   const int per_row = K >> 2;  // float4 per row
   const int64_t gwarp = (static_cast<int64_t>(blockIdx.x) * kBinThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kBinThreads) >> 5;
@@ -271,7 +273,9 @@ template <int WF>
 __global__ void __launch_bounds__(256) ternary_pack_kernel(const float* __restrict__ w, int64_t N, int K,
                                                            int64_t ldw, const float* __restrict__ alpha,
                                                            float eps, uint8_t* __restrict__ out) {
-  const float d = __fadd_rn(*alpha, eps);
+  pdl_wait();
+  pdl_trigger();
+  const float d = __fadd_rn(ld_dep_f32(alpha), eps);
   const bool fast = d >= 0x1p-125f && d <= 0x1p+127f;   // d/2 exact and normal
   const float h = __fmul_rn(d, 0.5f);
   const int per_row = K >> 4;   // 16 weights per thread-step

@@ -102,6 +102,8 @@ __global__ void __launch_bounds__(256) quant_a4_kernel(const uint16_t* __restric
   const int nchunk = K >> 3;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * 2;
   int64_t row = static_cast<int64_t>(blockIdx.x) * 2 + sub;
+  pdl_wait();
+  pdl_trigger();
 
   // rows of up to 4096 values prefetch the next row; longer rows would need too
   // many registers for two rows, so they load at the top of each iteration

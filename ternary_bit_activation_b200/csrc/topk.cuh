@@ -172,6 +172,8 @@ __global__ void __launch_bounds__(kTkThreads, F32 ? 2 : 4) topk_rows_kernel(
   };
 
   zero_counters();
+  pdl_wait();
+  pdl_trigger();
   int64_t row = blockIdx.x;
   prefetch(row, 0);
   int buf = 0;
