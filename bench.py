@@ -584,10 +584,18 @@ def run_reference(args):
 # decode: M tokens through the BitLinear path of DECODE_LAYERS distinct 7B-shape
 # layers (2-bit weights packed once, as at inference); the layers' weights
 # together exceed L2, so every layer streams its weights from HBM.  Activations
-# are INT4 / Top-K INT8 codes one byte each; the GEMM runs on the tensor cores
-# from 8 tokens and on the CUDA-core kernel below.
+# are INT4 / Top-K INT8 codes one byte each; the GEMM runs on the dp4a GEMV for
+# 1-2 tokens, the warp-MMA GEMV for 3-8 and the tensor cores beyond.
 # ---------------------------------------------------------------------------
 DECODE_LAYERS = 4   # 4 x 50.6 MB of 2-bit weights > the 126 MB L2
+
+
+def decode_gemm_kernel(m: int) -> str:
+    if m <= 2:
+        return "CUDA-core GEMV (dp4a on offset codes)"
+    if m <= 8:
+        return "warp-MMA GEMV (m16n8k32 u8 x s8)"
+    return "tcgen05 (2-bit weights widened into TMEM)"
 
 
 def run_decode(args):
@@ -696,7 +704,7 @@ def run_decode(args):
         gbs = weight_bytes / (gemm_ms / 1e3) / 1e9
         results.append({"tokens": m, "ms_per_layer": round(ms, 4), "tokens_per_s": round(m / (ms / 1e3), 1),
                         "gemm_ms_per_layer": round(gemm_ms, 4),
-                        "gemm_kernel": "tcgen05 (2-bit weights widened into TMEM)" if m >= 8 else "CUDA-core",
+                        "gemm_kernel": decode_gemm_kernel(m),
                         "weight_stream_gbs": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 3)})
     line = {"metric": "decode BitLinear layer latency (7B shapes, 2-bit weights; CUDA-graph replay)",
             "unit": "ms per layer",
@@ -718,7 +726,7 @@ PROFILE_CASES = {
     "relu2_glu": "ReLU^2-GLU + Top-K 50% + INT8, gate/up bf16 [16384 x 11008]",
     "kv_quant3": "3-bit KV, K bf16 [32768 x 32 x 128]",
     "pack_ternary": "ternary pack to int8, W fp32 [22016 x 4096]",
-    "gemm_decode": "CUDA-core GEMM, 2-bit W [12288 x 4096], 1 token",
+    "gemm_decode": "CUDA-core GEMV, 2-bit W [12288 x 4096], 1 token",
     "gemm_decode_tc": "tcgen05 GEMM, 2-bit W [12288 x 4096] widened into TMEM, 16 tokens",
 }
 

@@ -237,13 +237,21 @@ bool launch_simt_m(const uint8_t* a, const float* sc, const uint8_t* w, const fl
   return launch_simt_mu<AF, WT2, MT, 8>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
 }
 
-// Rows of A per staged tile (MT): up to 8 tokens share each streamed weight unit.
+// Rows of A per staged tile (MT): up to 8 tokens share each streamed weight
+// unit, fewer where MT rows of K codes would not fit in shared memory (the
+// kernel walks the rows of A in tiles of MT).
+constexpr size_t kSimtMaxSmem = 192 * 1024;
+constexpr int64_t kSimtMaxK = 196608;   // one row of A per tile still fits
+
 template <int AF, bool WT2>
 bool launch_simt(const uint8_t* a, const float* sc, const uint8_t* w, const float* al, int64_t g, int M, int N,
                  int K, uint16_t* y, int64_t ldy, int32_t* acc, cudaStream_t s) {
-  if (M <= 1) return launch_simt_m<AF, WT2, 1>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
-  if (M <= 2) return launch_simt_m<AF, WT2, 2>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
-  if (M <= 4) return launch_simt_m<AF, WT2, 4>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
+  const size_t row_bytes = static_cast<size_t>(((K >> 6) + 31) >> 5) * 32 * 16 * sizeof(uint32_t);
+  int mt = M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8));
+  while (mt > 1 && static_cast<size_t>(mt) * row_bytes > kSimtMaxSmem) mt >>= 1;
+  if (mt == 1) return launch_simt_m<AF, WT2, 1>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
+  if (mt == 2) return launch_simt_m<AF, WT2, 2>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
+  if (mt == 4) return launch_simt_m<AF, WT2, 4>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
   return launch_simt_m<AF, WT2, 8>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
 }
 
@@ -265,6 +273,98 @@ unsigned long long* noalloc_bins_ptr() {
     cached[d] = static_cast<unsigned long long*>(p);
   }
   return cached[d];
+}
+
+// GEMV for up to kGvMaxTokens tokens against 2-bit weights: token slots per
+// launch, and the limits that keep the staged activations in shared memory.
+constexpr int kGvMaxTokens = 8;
+constexpr int64_t kGvMaxK = 65536;                  // 16 rounds of 4096 codes: 512 threads
+constexpr int64_t kGvMaxActBytes = 144 * 1024;      // token slots x K int8 activations
+constexpr int kGvSmemLimit = 144 * 1024 + 8192;     // + round partial sums (two buffers)
+
+int64_t gv_tokens(int m) { return m <= 1 ? 1 : (m <= 2 ? 2 : (m <= 4 ? 4 : 8)); }
+
+template <int AF, int MT>
+bl_status launch_gemv_mt(const uint8_t* A, const float* a_scale, const uint8_t* W, const float* alpha,
+                         int64_t alpha_group, int m, int n, int k, uint16_t* Y, int64_t ldy, int32_t* acc_out,
+                         cudaStream_t s) {
+  static bool attr_done[kMaxDevices] = {};
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return BL_ERR_CUDA;
+  if (!attr_done[d]) {
+    if (!cuda_ok(cudaFuncSetAttribute(bl::gemv_t2_kernel<AF, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      kGvSmemLimit)))
+      return BL_ERR_CUDA;
+    attr_done[d] = true;
+  }
+  constexpr int R = bl::GvShape<MT>::R;
+  const int S = (k / 16 + 255) / 256;   // 4096-code rounds of a row, one warp each
+  const int G = S >= 8 ? 1 : 8 / S;     // row groups per CTA and pass
+  const int threads = 32 * G * S;
+  const int64_t groups = (static_cast<int64_t>(n) + R - 1) / R;
+  const size_t smem =
+      static_cast<size_t>(MT) * static_cast<size_t>(k) + 2 * static_cast<size_t>(G * S * R * MT) * sizeof(int);
+  // persistent CTAs: as many as are resident at once, at most one pass each
+  int per_sm = 0;
+  if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bl::gemv_t2_kernel<AF, MT>, threads, smem)))
+    return BL_ERR_CUDA;
+  if (per_sm < 1) per_sm = 1;
+  const int64_t passes = (groups + G - 1) / G;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
+  const unsigned grid = static_cast<unsigned>(passes < cap ? passes : cap);
+  launch_pdl(bl::gemv_t2_kernel<AF, MT>, grid, threads, smem, s, A, a_scale, W, alpha, alpha_group, m, n, k, S, G,
+             Y, ldy, acc_out);
+  return launch_status();
+}
+
+// Warp-MMA GEMV: all 8 token slots staged, so 8 x K activation bytes.  One
+// or two tokens run faster on the dp4a GEMV (the MMA's 8 columns mostly idle).
+constexpr int64_t kGmMaxK = kGvMaxActBytes / 8;
+constexpr int64_t kGmMinTokens = 3;
+constexpr int kGmSmemLimit = 144 * 1024 + 16384;    // + batch partial sums (two buffers)
+
+template <int AF>
+bl_status launch_gemv_mma(const uint8_t* A, const float* a_scale, const uint8_t* W, const float* alpha,
+                          int64_t alpha_group, int m, int n, int k, uint16_t* Y, int64_t ldy, int32_t* acc_out,
+                          cudaStream_t s) {
+  static bool attr_done[kMaxDevices] = {};
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return BL_ERR_CUDA;
+  if (!attr_done[d]) {
+    if (!cuda_ok(cudaFuncSetAttribute(bl::gemv_mma_t2_kernel<AF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      kGmSmemLimit)))
+      return BL_ERR_CUDA;
+    attr_done[d] = true;
+  }
+  const int batches = (k / 16 + bl::kGmBatchWords - 1) / bl::kGmBatchWords;   // 1024-code batches of a row
+  const int S = batches < 16 ? batches : 16;                                  // warps per 16-row tile
+  const int G = S >= 8 ? 1 : 8 / S;                                           // tiles per CTA and pass
+  const int threads = 32 * G * S;
+  const int64_t tiles = (static_cast<int64_t>(n) + 15) / 16;
+  const size_t smem = static_cast<size_t>(bl::kGmTokens) * static_cast<size_t>(k) +
+                      2 * static_cast<size_t>(G * S * 32) * sizeof(int4);
+  int per_sm = 0;
+  if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bl::gemv_mma_t2_kernel<AF>, threads, smem)))
+    return BL_ERR_CUDA;
+  if (per_sm < 1) per_sm = 1;
+  const int64_t passes = (tiles + G - 1) / G;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
+  const unsigned grid = static_cast<unsigned>(passes < cap ? passes : cap);
+  launch_pdl(bl::gemv_mma_t2_kernel<AF>, grid, threads, smem, s, A, a_scale, W, alpha, alpha_group, m, n, k, S, G, Y,
+             ldy, acc_out);
+  return launch_status();
+}
+
+template <int AF>
+bl_status launch_gemv(const uint8_t* A, const float* a_scale, const uint8_t* W, const float* alpha,
+                      int64_t alpha_group, int m, int n, int k, uint16_t* Y, int64_t ldy, int32_t* acc_out,
+                      cudaStream_t s) {
+  switch (gv_tokens(m)) {
+    case 1: return launch_gemv_mt<AF, 1>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+    case 2: return launch_gemv_mt<AF, 2>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+    case 4: return launch_gemv_mt<AF, 4>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+    default: return launch_gemv_mt<AF, 8>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+  }
 }
 
 }  // namespace
@@ -529,28 +629,17 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
     launch_pdl(bl::gemm_tc_kernel, grid, bl::kTcThreads, bl::kTcSmemBytes, s, ta, tb, p);
     return launch_status();
   }
-  if (afmt == BL_A_I8 && wfmt == BL_W_T2 && M <= 2 && M * K <= 65536) {
-    // one or two tokens: register-widening GEMV, one pass over the 2-bit weights
-    static bool attr_done[kMaxDevices] = {};
-    const int d = current_device();
-    if (d < 0 || d >= kMaxDevices) return BL_ERR_CUDA;
-    if (!attr_done[d]) {
-      if (!cuda_ok(cudaFuncSetAttribute(bl::gemv_t2_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536)) ||
-          !cuda_ok(cudaFuncSetAttribute(bl::gemv_t2_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536)))
-        return BL_ERR_CUDA;
-      attr_done[d] = true;
-    }
-    const int64_t warps = (N + bl::kGvRows - 1) / bl::kGvRows;
-    const int64_t need = (warps + bl::kGvThreads / 32 - 1) / (bl::kGvThreads / 32);
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
-    const unsigned grid = static_cast<unsigned>(need < cap ? need : cap);
-    const size_t smem = static_cast<size_t>(M) * static_cast<size_t>(K);
-    const int8_t* A8 = static_cast<const int8_t*>(a);
-    if (M == 1)
-      launch_pdl(bl::gemv_t2_kernel<1>, grid, bl::kGvThreads, smem, s, A8, a_scale, W, alpha, alpha_group, n, k, Y, ldy, acc_out);
-    else
-      launch_pdl(bl::gemv_t2_kernel<2>, grid, bl::kGvThreads, smem, s, A8, a_scale, W, alpha, alpha_group, n, k, Y, ldy, acc_out);
-    return launch_status();
+  if (wfmt == BL_W_T2 && M >= kGmMinTokens && M <= kGvMaxTokens && K <= kGmMaxK) {
+    // 3 to 8 tokens: warp-MMA GEMV, one pass over the 2-bit weights
+    if (afmt == BL_A_I8) return launch_gemv_mma<bl::kSimtA_I8>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+    if (afmt == BL_A_I4) return launch_gemv_mma<bl::kSimtA_I4>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+    return launch_gemv_mma<bl::kSimtA_E2M1>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+  }
+  if (wfmt == BL_W_T2 && M <= kGvMaxTokens && K <= kGvMaxK && gv_tokens(m) * K <= kGvMaxActBytes) {
+    // 1 or 2 tokens, or longer rows: dp4a GEMV staging only the token slots in use
+    if (afmt == BL_A_I8) return launch_gemv<bl::kSimtA_I8>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+    if (afmt == BL_A_I4) return launch_gemv<bl::kSimtA_I4>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+    return launch_gemv<bl::kSimtA_E2M1>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
   }
   if (afmt == BL_A_I8 && wfmt == BL_W_T2 && M >= bl::kTsMinTokens) {
     // 2-bit weights widened into tensor memory; tokens on the MMA's N side
@@ -591,6 +680,8 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
     else launch_pdl(bl::gemm_t2tc_kernel<1>, grid, bl::kTsThreads, smem, s, tx, tw, p);
     return launch_status();
   }
+  // CUDA-core kernel: one row of A per tile must fit in shared memory
+  if (K > kSimtMaxK) return BL_ERR_SHAPE;
   const bool t2 = wfmt == BL_W_T2;
   bool ok;
   switch (afmt) {

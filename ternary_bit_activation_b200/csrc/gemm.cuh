@@ -11,8 +11,11 @@
 // gemm_t2tc_kernel -- 2-bit ternary weights x int8 activations for 8..256
 //                     tokens (decode): weights widened to int8 in registers
 //                     and stored into tensor memory as the MMA's A operand.
-// gemv_t2_kernel   -- 1 or 2 tokens x 2-bit weights: 2-bit codes widened in
-//                     registers, activations from shared memory, dp4a.
+// gemv_t2_kernel   -- 1 to 8 tokens x 2-bit weights: offset codes c + 1
+//                     isolated per byte field, dp4a against transposed
+//                     activations in shared memory (long rows).
+// gemv_mma_t2_kernel -- the same offset codes fed to warp-level integer MMA
+//                     (16 weight rows x 8 token slots per instruction).
 // gemm_simt_kernel -- CUDA-core kernel that reads packed operands directly
 //                     (2-bit ternary weights, INT4 / E2M1 nibbles); decode of
 //                     3 to 7 tokens and the packed activation formats.
@@ -887,130 +890,6 @@ __global__ void __launch_bounds__(kTsThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// gemv_t2_kernel -- 1 or 2 tokens against 2-bit ternary weights (decode).  A
-// warp takes 4 weight rows at a time; in each round of 4096 codes lane l loads
-// 2 x 16 bytes of every row (words 4l..4l+3 and 128+4l..128+4l+3 of the round,
-// so each load instruction reads 512 contiguous bytes), widens the 16-code
-// words to int8 in registers (byte permutes, no table) and dot-products them
-// with the matching activation words, read once per round from shared memory
-// and reused by the 4 rows.  Partial sums are reduced by shuffles.
-// ---------------------------------------------------------------------------
-constexpr int kGvRows = 4;          // weight rows per warp and pass
-constexpr int kGvThreads = 256;
-
-template <int MT>
-__global__ void __launch_bounds__(kGvThreads) gemv_t2_kernel(const int8_t* __restrict__ a,
-                                                             const float* __restrict__ a_scale,
-                                                             const uint8_t* __restrict__ w,
-                                                             const float* __restrict__ alpha, int64_t alpha_group,
-                                                             int N, int K, uint16_t* __restrict__ y, int64_t ldy,
-                                                             int32_t* __restrict__ acc_out) {
-  extern __shared__ uint4 gv_act[];   // MT rows of K int8 codes
-  const int lane = threadIdx.x & 31;
-  const int kw16 = K >> 4;            // 16-code words per row (16 bytes of int8 activations each)
-  const int64_t wrow_bytes = K >> 2;
-  const int rounds = (kw16 + 255) >> 8;            // 256 words (4096 codes) per round
-  const int64_t warp_id = (static_cast<int64_t>(blockIdx.x) * kGvThreads + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kGvThreads) >> 5;
-
-  // this lane's weight words of round rd for rows n0.. (2 pieces of 4 words)
-  auto load_round = [&](int64_t n0, int rd, uint4 (&wv)[kGvRows][2]) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int wq = (rd << 8) + h * 128 + 4 * lane;
-      const bool ok = wq < kw16;                  // kw16 is a multiple of 4 (K % 64 == 0)
-#pragma unroll
-      for (int r = 0; r < kGvRows; ++r) {
-        const int64_t n = n0 + r < N ? n0 + r : n0;
-        wv[r][h] = ok ? ld_global_nc_v4(w + n * wrow_bytes + static_cast<int64_t>(wq) * 4) : make_uint4(0, 0, 0, 0);
-      }
-    }
-  };
-  // pull this warp's weight rows into L2 while the previous kernel finishes
-  for (int64_t n0 = warp_id * kGvRows; n0 < N; n0 += nwarps * kGvRows)
-    for (int r = 0; r < kGvRows && n0 + r < N; ++r)
-      for (int64_t b = static_cast<int64_t>(lane) * 128; b < wrow_bytes; b += 32 * 128)
-        prefetch_l2(w + (n0 + r) * wrow_bytes + b);
-  pdl_wait();
-  pdl_trigger();
-  // the first weight loads go out before the activations are staged: the two
-  // latencies overlap
-  uint4 wv[kGvRows][2];
-  if (warp_id * kGvRows < N) load_round(warp_id * kGvRows, 0, wv);
-  for (int i = threadIdx.x; i < MT * kw16; i += blockDim.x) {
-    const int m = i / kw16, q = i - m * kw16;
-    gv_act[i] = ld_global_nc_v4(a + static_cast<int64_t>(m) * K + static_cast<int64_t>(q) * 16);
-  }
-  __syncthreads();
-  bool first = true;
-  for (int64_t n0 = warp_id * kGvRows; n0 < N; n0 += nwarps * kGvRows) {
-    int acc[kGvRows][MT];
-#pragma unroll
-    for (int r = 0; r < kGvRows; ++r)
-#pragma unroll
-      for (int m = 0; m < MT; ++m) acc[r][m] = 0;
-    for (int rd = 0; rd < rounds; ++rd) {
-      int wq[2];
-      bool ok[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        wq[h] = (rd << 8) + h * 128 + 4 * lane;
-        ok[h] = wq[h] < kw16;
-      }
-      if (!first) load_round(n0, rd, wv);
-      first = false;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (!ok[h]) continue;
-        // activation words of the 4 T2 words: 4 x 16 bytes per token
-        uint4 av[MT][4];
-#pragma unroll
-        for (int m = 0; m < MT; ++m)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) av[m][j] = gv_act[m * kw16 + wq[h] + j];
-#pragma unroll
-        for (int r = 0; r < kGvRows; ++r) {
-          const uint32_t x4[4] = {wv[r][h].x, wv[r][h].y, wv[r][h].z, wv[r][h].w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t t[4];
-            widen_t2_word(x4[j], t);
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-              acc[r][m] = __dp4a(static_cast<int>(t[0]), static_cast<int>(av[m][j].x), acc[r][m]);
-              acc[r][m] = __dp4a(static_cast<int>(t[1]), static_cast<int>(av[m][j].y), acc[r][m]);
-              acc[r][m] = __dp4a(static_cast<int>(t[2]), static_cast<int>(av[m][j].z), acc[r][m]);
-              acc[r][m] = __dp4a(static_cast<int>(t[3]), static_cast<int>(av[m][j].w), acc[r][m]);
-            }
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < kGvRows; ++r)
-#pragma unroll
-      for (int m = 0; m < MT; ++m) acc[r][m] = __reduce_add_sync(0xFFFFFFFFu, acc[r][m]);
-    // lane r * MT + m writes output (row n0 + r, token m)
-#pragma unroll
-    for (int r = 0; r < kGvRows; ++r)
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        const int64_t n = n0 + r;
-        if (lane == r * MT + m && n < N) {
-          const int v = acc[r][m];
-          if (acc_out != nullptr) acc_out[static_cast<int64_t>(m) * N + n] = v;
-          if (y != nullptr) {
-            const float cs = __fmul_rn(ld_dep_f32(a_scale + m), ld_dep_f32(alpha + n / alpha_group));
-            const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__int2float_rn(v), cs));
-            y[static_cast<int64_t>(m) * ldy + n] = *reinterpret_cast<const uint16_t*>(&b);
-          }
-        }
-      }
-  }
-}
-
-
-// ---------------------------------------------------------------------------
 // CUDA-core kernel for packed operands.  One warp per output column n (a row
 // of W); lanes split K in units of 64 codes; MT rows of A per pass share the
 // expanded weight unit.  dp4a on int8x4 words.
@@ -1220,6 +1099,418 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const uint8_t* __restric
             }
           }
         }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// gemv_t2_kernel -- 1 to 8 tokens against 2-bit ternary weights (decode).
+//
+// A 16-code weight word x (code e in bits 2e..2e+1: 00 -> 0, 01 -> +1,
+// 11 -> -1) becomes offset codes c + 1 in {0, 1, 2} with one shift and one
+// three-input logic op,
+//     u = ~x & (0x55555555 | (x << 1))
+// (a field's low bit is set for code 0 only, its high bit for +1 only).  Field
+// j of every byte (code 4b + j of the word) is dotted with the activation
+// bytes a[4b + j] by dp4a (unsigned x signed).  For one token the field is
+// isolated in place by one AND, u & (0x03030303 << 2j) = 4^j (c + 1), into one
+// of four accumulators, each an exact multiple of 4^j:
+//     sum_k (c_k + 1) a_k  =  s_0 + s_1/4 + s_2/16 + s_3/64   (exact shifts);
+// for several tokens the fields are shifted down once per word and every token
+// keeps a single accumulator.  The token's sum_k a_k is subtracted at the end.
+//
+// The activations (INT8, INT4 or E2M1 codes; E2M1 as twice their value) are
+// staged once per CTA in shared memory as int8, the 16 bytes of each word
+// transposed field-major so that the four dp4a operands of a word are one
+// 16-byte load.  CTAs are persistent: G row groups of R rows per pass, warp w
+// taking group w / S and 4096-code round w % S of it; the S partial sums of a
+// row meet in shared memory.  Before its wait each warp issues L2 prefetches
+// for every weight byte it will read, so HBM streams the whole matrix while
+// the CTAs stage activations and compute.
+// ---------------------------------------------------------------------------
+// 16 activation codes -> the field-major word f (field j = bytes j of v[0..3])
+// and the sum of the codes
+__device__ __forceinline__ uint4 gv_transpose(const uint32_t (&v)[4], int& sum) {
+  const uint32_t t0 = __byte_perm(v[0], v[1], 0x5140), t1 = __byte_perm(v[0], v[1], 0x7362);
+  const uint32_t t2 = __byte_perm(v[2], v[3], 0x5140), t3 = __byte_perm(v[2], v[3], 0x7362);
+  const uint4 f = make_uint4(__byte_perm(t0, t2, 0x5410), __byte_perm(t0, t2, 0x7632),
+                             __byte_perm(t1, t3, 0x5410), __byte_perm(t1, t3, 0x7632));
+  int sv = __dp4a(static_cast<int>(f.x), 0x01010101, 0);
+  sv = __dp4a(static_cast<int>(f.y), 0x01010101, sv);
+  sv = __dp4a(static_cast<int>(f.z), 0x01010101, sv);
+  sum += __dp4a(static_cast<int>(f.w), 0x01010101, sv);
+  return f;
+}
+
+template <int MT>
+struct GvShape {
+  static constexpr int R = 4;   // weight rows per warp
+};
+constexpr int kGvMaxThreads = 512;
+
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// 16 activation codes of word q of row m as int8, element order (w[i] holds 4i..4i+3)
+template <int AF>
+__device__ __forceinline__ void gv_load_word(const uint8_t* a, int K, int m, int q, uint32_t (&w)[4]) {
+  if constexpr (AF == kSimtA_I8) {
+    const uint4 v = ld_dep_v4(a + static_cast<int64_t>(m) * K + static_cast<int64_t>(q) * 16);
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else {
+    const uint8_t* src = a + static_cast<int64_t>(m) * (K >> 1) + static_cast<int64_t>(q) * 8;
+    uint32_t p0, p1;
+    asm volatile("ld.global.v2.u32 {%0,%1}, [%2];" : "=r"(p0), "=r"(p1) : "l"(src));
+    uint32_t n[4];
+    split_nibbles(p0, n[0], n[1]);
+    split_nibbles(p1, n[2], n[3]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = AF == kSimtA_I4 ? sext_nibble_bytes(n[i]) : e2m1_bytes_to_twice(n[i]);
+  }
+}
+// Stage the activations of M tokens into shared memory as field-major int8
+// words (gv_transpose) at act[slot(q, m)], zeros for the token slots M..TOK-1,
+// and add each token's code sum to asum[m].  A thread's loads for all tokens of
+// a word are in flight together.
+template <int AF, int TOK, typename Slot>
+__device__ __forceinline__ void gv_stage(const uint8_t* a, int M, int K, uint4* act, Slot slot, int* asum) {
+  const int kw16 = K >> 4;
+  int tsum[TOK];
+#pragma unroll
+  for (int m = 0; m < TOK; ++m) tsum[m] = 0;
+  for (int q = threadIdx.x; q < kw16; q += blockDim.x) {
+    uint32_t v[TOK][4];
+#pragma unroll
+    for (int m = 0; m < TOK; ++m) {
+      v[m][0] = v[m][1] = v[m][2] = v[m][3] = 0u;
+      if (m < M) gv_load_word<AF>(a, K, m, q, v[m]);
+    }
+#pragma unroll
+    for (int m = 0; m < TOK; ++m) act[slot(q, m)] = gv_transpose(v[m], tsum[m]);
+  }
+#pragma unroll
+  for (int m = 0; m < TOK; ++m) {
+    const int v = __reduce_add_sync(0xFFFFFFFFu, tsum[m]);
+    if ((threadIdx.x & 31) == 0 && v != 0) atomicAdd(&asum[m], v);
+  }
+}
+
+template <int AF, int MT>
+__global__ void __launch_bounds__(kGvMaxThreads) gemv_t2_kernel(const uint8_t* __restrict__ a,
+                                                                const float* __restrict__ a_scale,
+                                                                const uint8_t* __restrict__ w,
+                                                                const float* __restrict__ alpha, int64_t alpha_group,
+                                                                int M, int N, int K, int S, int G,
+                                                                uint16_t* __restrict__ y, int64_t ldy,
+                                                                int32_t* __restrict__ acc_out) {
+  constexpr int R = GvShape<MT>::R;
+  extern __shared__ uint4 gv_smem[];
+  __shared__ int asum[MT];
+  const int kw16 = K >> 4;                              // 16-code words per row
+  const int kq = kw16 >> 2;                             // words per lane slot (kw16 % 4 == 0)
+  uint4* act = gv_smem;                                 // [MT][4][kw16 / 4], field-major bytes
+  int* part = reinterpret_cast<int*>(act + MT * kw16);  // [2][G][S][R][MT] partial sums
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int g = warp / S;
+  const int rd = warp - g * S;
+  const int64_t wrow_bytes = K >> 2;
+  const int64_t groups = (static_cast<int64_t>(N) + R - 1) / R;
+  const int64_t group_step = static_cast<int64_t>(gridDim.x) * G;
+
+  // every weight line this warp will read (R rows x its 1 KiB round per pass)
+  // into L2 while the previous kernel finishes
+  if (lane < 8 * R) {
+    const int r = lane >> 3;
+    const int64_t b = static_cast<int64_t>(rd) * 1024 + (lane & 7) * 128;
+    if (b < wrow_bytes)
+      for (int64_t gi = static_cast<int64_t>(blockIdx.x) * G + g; gi < groups; gi += group_step) {
+        const int64_t n = gi * R + r;
+        if (n < N) prefetch_l2(w + n * wrow_bytes + b);
+      }
+  }
+  if (threadIdx.x < MT) asum[threadIdx.x] = 0;
+  __syncthreads();
+  pdl_wait();
+  pdl_trigger();
+
+  // weights of a pass: lane l holds words 4l..4l+3 and 128+4l..128+4l+3 of the
+  // round; the first pass's loads go out before the activations are staged
+  uint4 wv[R][2];
+  auto load_weights = [&](int64_t gb) {
+    const int64_t n0 = (gb + g) * R;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int wq = rd * 256 + h * 128 + 4 * lane;
+      const bool ok = gb < groups && n0 < N && wq < kw16;   // kw16 is a multiple of 4
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int64_t n = n0 + r < N ? n0 + r : n0;
+        wv[r][h] = ok ? ld_global_nc_v4(w + n * wrow_bytes + static_cast<int64_t>(wq) * 4) : make_uint4(0, 0, 0, 0);
+      }
+    }
+  };
+  load_weights(static_cast<int64_t>(blockIdx.x) * G);
+
+  // stage the activations (zeros for token slots past M) and their sums
+  // word 4p + j of token m at [m][j][p]: the lanes of a warp read consecutive slots
+  gv_stage<AF, MT>(a, M, K, act, [kq](int q, int m) { return (m * 4 + (q & 3)) * kq + (q >> 2); }, asum);
+  __syncthreads();
+  const float unit_scale = (AF == kSimtA_E2M1) ? 0.5f : 1.0f;
+
+  int par = 0;
+  for (int64_t gb = static_cast<int64_t>(blockIdx.x) * G; gb < groups; gb += group_step, par ^= 1) {
+    const int64_t n0 = (gb + g) * R;
+    const bool rows_ok = n0 < N;
+    int tot[R][MT];
+    if constexpr (MT == 1) {
+      int acc[R][4];
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[r][j] = 0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int wq = rd * 256 + h * 128 + 4 * lane;
+        if (!rows_ok || wq >= kw16) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 av = act[j * kq + (wq >> 2)];
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            const uint32_t x = j == 0 ? wv[r][h].x : (j == 1 ? wv[r][h].y : (j == 2 ? wv[r][h].z : wv[r][h].w));
+            const uint32_t u = ~x & (0x55555555u | (x << 1));
+            acc[r][0] = dp4a_us(u & 0x03030303u, av.x, acc[r][0]);
+            acc[r][1] = dp4a_us(u & 0x0C0C0C0Cu, av.y, acc[r][1]);
+            acc[r][2] = dp4a_us(u & 0x30303030u, av.z, acc[r][2]);
+            acc[r][3] = dp4a_us(u & 0xC0C0C0C0u, av.w, acc[r][3]);
+          }
+        }
+      }
+      load_weights(gb + group_step);   // the next pass's loads overlap the reductions
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+        tot[r][0] = __reduce_add_sync(0xFFFFFFFFu, acc[r][0] + (acc[r][1] >> 2) + (acc[r][2] >> 4) + (acc[r][3] >> 6));
+    } else {
+      int acc[R][MT];
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[r][m] = 0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int wq = rd * 256 + h * 128 + 4 * lane;
+        if (!rows_ok || wq >= kw16) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t f[R][4];
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            const uint32_t x = j == 0 ? wv[r][h].x : (j == 1 ? wv[r][h].y : (j == 2 ? wv[r][h].z : wv[r][h].w));
+            const uint32_t u = ~x & (0x55555555u | (x << 1));
+            f[r][0] = u & 0x03030303u;
+            f[r][1] = (u >> 2) & 0x03030303u;
+            f[r][2] = (u >> 4) & 0x03030303u;
+            f[r][3] = (u >> 6) & 0x03030303u;
+          }
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            const uint4 av = act[(m * 4 + j) * kq + (wq >> 2)];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              int t = dp4a_us(f[r][0], av.x, acc[r][m]);
+              t = dp4a_us(f[r][1], av.y, t);
+              t = dp4a_us(f[r][2], av.z, t);
+              acc[r][m] = dp4a_us(f[r][3], av.w, t);
+            }
+          }
+        }
+      }
+      load_weights(gb + group_step);
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) tot[r][m] = __reduce_add_sync(0xFFFFFFFFu, acc[r][m]);
+    }
+    if (S > 1) {
+      // rounds of a row group meet in shared memory (two buffers: the readers
+      // of one pass are done before the pass after next writes it again)
+      int* pp = part + par * (G * S * R * MT);
+      if (lane == 0) {
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int m = 0; m < MT; ++m) pp[((g * S + rd) * R + r) * MT + m] = tot[r][m];
+      }
+      __syncthreads();
+      if (rd != 0) continue;
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+          for (int q = 1; q < S; ++q) tot[r][m] += pp[((g * S + q) * R + r) * MT + m];
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const int64_t n = n0 + r;
+        if (lane == r * MT + m && n < N && m < M) {
+          const int v = tot[r][m] - asum[m];
+          if (acc_out != nullptr) acc_out[static_cast<int64_t>(m) * N + n] = v;
+          if (y != nullptr) {
+            const float cs =
+                __fmul_rn(__fmul_rn(ld_dep_f32(a_scale + m), unit_scale), ld_dep_f32(alpha + n / alpha_group));
+            const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__int2float_rn(v), cs));
+            y[static_cast<int64_t>(m) * ldy + n] = *reinterpret_cast<const uint16_t*>(&b);
+          }
+        }
+      }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// gemv_mma_t2_kernel -- up to 8 tokens against 2-bit ternary weights (decode)
+// on warp-level integer MMA (m16n8k32, u8 x s8 -> s32): weight rows are the
+// MMA's 16 rows, the 8 token slots its 8 columns.  The MMA adds up 32 codes per
+// row and token whatever order they come in, so each lane feeds it the offset
+// codes c + 1 of the weight words it loaded itself (field j of a word, isolated
+// with a shift and an AND as in gemv_t2_kernel) and the B fragment holds the
+// activations of the same codes: the field-major activation words staged in
+// shared memory are exactly that.  Lane (g, t) of a warp (g = lane / 4,
+// t = lane % 4) loads 16 bytes (4 words, 64 codes) of rows g and g + 8 of the
+// warp's 16-row tile per 256-code step, word 4t + c of the step; per word pair
+// it issues two MMAs (fields 0, 1 and fields 2, 3).  The sums are of c + 1;
+// each token's sum_k a_k is subtracted at the end.  CTAs are persistent and
+// stage the activations once; K is split into 1024-code batches over S warps
+// per tile whose partial sums meet in shared memory; every weight line a warp
+// will read is prefetched into L2 before its wait.
+// ---------------------------------------------------------------------------
+constexpr int kGmTokens = 8;          // MMA columns: token slots
+constexpr int kGmBatchWords = 64;     // 16-code words per row and batch (4 steps of 16)
+
+__device__ __forceinline__ void mma_u8s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int AF>
+__global__ void __launch_bounds__(kGvMaxThreads) gemv_mma_t2_kernel(const uint8_t* __restrict__ a,
+                                                                    const float* __restrict__ a_scale,
+                                                                    const uint8_t* __restrict__ w,
+                                                                    const float* __restrict__ alpha,
+                                                                    int64_t alpha_group, int M, int N, int K, int S,
+                                                                    int G, uint16_t* __restrict__ y, int64_t ldy,
+                                                                    int32_t* __restrict__ acc_out) {
+  extern __shared__ uint4 gm_smem[];
+  __shared__ int asum[kGmTokens];
+  const int kw16 = K >> 4;      // 16-code words per row (a multiple of 4)
+  const int kq = kw16 >> 2;
+  // activation word 4p + c of token m at (p * 4 + c) * 8 + m: the 32 lanes of
+  // a B-fragment load hit 8 consecutive slots 4 times (no bank conflict)
+  uint4* act = gm_smem;
+  int4* part = reinterpret_cast<int4*>(act + static_cast<size_t>(kq) * 4 * kGmTokens);   // [2][G][S][32]
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int g = warp / S;
+  const int rd = warp - g * S;
+  const int grp = lane >> 2;
+  const int tig = lane & 3;
+  const int64_t wrow_bytes = K >> 2;
+  const int64_t tiles = (static_cast<int64_t>(N) + 15) >> 4;
+  const int64_t tile_step = static_cast<int64_t>(gridDim.x) * G;
+  const int batches = (kw16 + kGmBatchWords - 1) / kGmBatchWords;
+
+  // every weight line this warp will read into L2 while the previous kernel
+  // finishes: per tile and batch 16 rows x 256 bytes, one 128-byte line a lane
+  for (int64_t tile = static_cast<int64_t>(blockIdx.x) * G + g; tile < tiles; tile += tile_step)
+    for (int b = rd; b < batches; b += S) {
+      const int64_t n = tile * 16 + (lane & 15);
+      const int64_t off = static_cast<int64_t>(b) * (kGmBatchWords * 4) + (lane >> 4) * 128;
+      if (n < N && off < wrow_bytes) prefetch_l2(w + n * wrow_bytes + off);
+    }
+  if (threadIdx.x < kGmTokens) asum[threadIdx.x] = 0;
+  __syncthreads();
+  pdl_wait();
+  pdl_trigger();
+
+  // stage the activations (zeros for token slots past M) and their sums
+  gv_stage<AF, kGmTokens>(a, M, K, act, [](int q, int m) { return ((q >> 2) * 4 + (q & 3)) * kGmTokens + m; },
+                          asum);
+  __syncthreads();
+  const float unit_scale = (AF == kSimtA_E2M1) ? 0.5f : 1.0f;
+
+  int par = 0;
+  for (int64_t tb = static_cast<int64_t>(blockIdx.x) * G; tb < tiles; tb += tile_step, par ^= 1) {
+    const int64_t tile = tb + g;
+    const int64_t r0 = tile * 16 + grp;
+    const int64_t r1 = r0 + 8;
+    const bool ok0 = tile < tiles && r0 < N;
+    const bool ok1 = tile < tiles && r1 < N;
+    int c[4] = {0, 0, 0, 0};
+    for (int b = rd; b < batches; b += S) {
+      // words 4 tig .. 4 tig + 3 of rows r0 and r1 in each of the batch's 4 steps
+      uint4 w0[4], w1[4];
+#pragma unroll
+      for (int st = 0; st < 4; ++st) {
+        const int q = b * kGmBatchWords + st * 16 + 4 * tig;
+        const bool okq = q < kw16;
+        w0[st] = ok0 && okq ? ld_global_nc_v4(w + r0 * wrow_bytes + static_cast<int64_t>(q) * 4) : make_uint4(0, 0, 0, 0);
+        w1[st] = ok1 && okq ? ld_global_nc_v4(w + r1 * wrow_bytes + static_cast<int64_t>(q) * 4) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int st = 0; st < 4; ++st) {
+        const uint32_t x0[4] = {w0[st].x, w0[st].y, w0[st].z, w0[st].w};
+        const uint32_t x1[4] = {w1[st].x, w1[st].y, w1[st].z, w1[st].w};
+        const int q = b * kGmBatchWords + st * 16 + 4 * tig;
+        const bool okq = q < kw16;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          // words past K: zero activations (the weight side is then irrelevant)
+          const uint4 bv = okq ? act[((q >> 2) * 4 + cc) * kGmTokens + grp] : make_uint4(0, 0, 0, 0);
+          const uint32_t p0 = ~x0[cc] & (0x55555555u | (x0[cc] << 1));
+          const uint32_t p1 = ~x1[cc] & (0x55555555u | (x1[cc] << 1));
+          mma_u8s8_16832(c, p0 & 0x03030303u, p1 & 0x03030303u, (p0 >> 2) & 0x03030303u, (p1 >> 2) & 0x03030303u,
+                         bv.x, bv.y);
+          mma_u8s8_16832(c, (p0 >> 4) & 0x03030303u, (p1 >> 4) & 0x03030303u, (p0 >> 6) & 0x03030303u,
+                         (p1 >> 6) & 0x03030303u, bv.z, bv.w);
+        }
+      }
+    }
+    if (S > 1) {
+      // batches of a tile meet in shared memory (two buffers, as in gemv_t2_kernel)
+      int4* pp = part + static_cast<size_t>(par) * (G * S * 32);
+      pp[(g * S + rd) * 32 + lane] = make_int4(c[0], c[1], c[2], c[3]);
+      __syncthreads();
+      if (rd != 0) continue;
+      for (int q = 1; q < S; ++q) {
+        const int4 o = pp[(g * S + q) * 32 + lane];
+        c[0] += o.x;
+        c[1] += o.y;
+        c[2] += o.z;
+        c[3] += o.w;
+      }
+    }
+    // lane (grp, tig) holds rows r0 (c0, c1) and r1 (c2, c3), tokens 2 tig and 2 tig + 1
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int64_t n = e < 2 ? r0 : r1;
+      const int m = 2 * tig + (e & 1);
+      if ((e < 2 ? ok0 : ok1) && m < M) {
+        const int v = c[e] - asum[m];
+        if (acc_out != nullptr) acc_out[static_cast<int64_t>(m) * N + n] = v;
+        if (y != nullptr) {
+          const float cs =
+              __fmul_rn(__fmul_rn(ld_dep_f32(a_scale + m), unit_scale), ld_dep_f32(alpha + n / alpha_group));
+          const __nv_bfloat16 bb = __float2bfloat16_rn(__fmul_rn(__int2float_rn(v), cs));
+          y[static_cast<int64_t>(m) * ldy + n] = *reinterpret_cast<const uint16_t*>(&bb);
+        }
+      }
     }
   }
 }

@@ -206,11 +206,13 @@ def test_gemm_simt_parity(M, afmt, wfmt):
     assert bf16_rows_rel_err(y, ex) <= BF16_ROW_TOL
 
 
-# 2-bit weights x int8 activations on the tensor cores for M >= 8 (weights
-# widened into tensor memory; tokens on the MMA's N side: 8 for M = 8, else a
-# multiple of 16 up to 256 per token block); fewer tokens take the CUDA-core
-# kernel (test_gemm_simt_parity)
+# 2-bit weights x int8 activations on the tensor cores for M > 8 (weights
+# widened into tensor memory; tokens on the MMA's N side: a multiple of 16 up
+# to 256 per token block; 8 for M = 8 with rows too long for the GEMV's
+# staged activations).  The M = 8 cases with shorter rows run on the warp-MMA
+# GEMV.
 GEMM_T2TC_CASES = [
+    ("M8_long_K_20480_tc", 8, 136, 20480),
     ("M8_min_K", 8, 128, 64),
     ("M8_ragged_N_K_tail", 8, 300, 320),
     ("M8_two_tiles", 8, 256, 4096),
@@ -322,20 +324,94 @@ def test_gemm_fp4_end_to_end_alpha_groups():
     assert bf16_rows_rel_err(host(y, np.uint16), ex) <= BF16_ROW_TOL
 
 
-# one or two tokens against 2-bit weights: the register-widening GEMV
-@pytest.mark.parametrize("M", [1, 2])
-@pytest.mark.parametrize("N,K", [(1, 64), (7, 320), (130, 4096), (258, 4160), (37, 11008), (96, 640)])
-def test_gemv_t2_parity(M, N, K):
-    g = synth.rng(M * 1000 + N + K)
-    a = g.integers(-128, 128, (M, K)).astype(np.int8)
+# up to 8 tokens against 2-bit weights: the CUDA-core GEMV.  Rows of 4096
+# codes are split over warps (K = 11008: 3 rounds; K = 36864: 9 rounds, one
+# warp per row group), so the shapes cover one and many rounds, a ragged last
+# round, and N that fills no CTA; 8 token slots x K = 36864 exceeds the staged
+# activation limit and takes the tiled CUDA-core kernel instead.
+GEMV_SHAPES = [(1, 64), (7, 320), (130, 4096), (258, 4160), (37, 11008), (96, 640), (40, 36864)]
+
+
+def gemv_inputs(g, afmt, M, K):
+    """(device codes, afmt, the integer codes the sums use, scale passed, scale of those sums)"""
+    if afmt == "i8":
+        a = g.integers(-128, 128, (M, K)).astype(np.int8)
+        scale = (g.random(M) * 0.1 + 1e-3).astype(np.float32)
+        return to_dev(a), tba.BL_A_I8, a, scale, scale
+    x = synth.gaussian_bf16(g, (M, K))
+    if afmt == "i4":
+        c, _, scale = oracle.quant_int4(x, EPS)
+        return to_dev(oracle.pack_nibbles(c)), tba.BL_A_I4, c, scale, scale
+    code4, twice, _, scale = oracle.quant_fp4(x)
+    return (to_dev(oracle.pack_nibbles(code4)), tba.BL_A_E2M1, twice, scale,
+            (scale.astype(np.float64) / 2).astype(np.float32))
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8])
+@pytest.mark.parametrize("afmt", ["i8", "i4", "e2m1"])
+@pytest.mark.parametrize("N,K", GEMV_SHAPES)
+def test_gemv_t2_parity(M, afmt, N, K):
+    g = synth.rng(M * 1000 + N + K + len(afmt))
+    a_dev, af, codes, scale, sum_scale = gemv_inputs(g, afmt, M, K)
     t = g.integers(-1, 2, (N, K)).astype(np.int8)
-    scale = (g.random(M) * 0.1 + 1e-3).astype(np.float32)
     alpha = np.float32(0.0211)
+    acc, y = run_gemm(a_dev, af, scale, to_dev(oracle.pack_ternary2(t)), tba.BL_W_T2, alpha, M, N, K)
+    acc_ref, _ = oracle.gemm(codes, sum_scale, t, alpha, want_y=False)
+    assert np.array_equal(acc, acc_ref)
+    _, ex = exact_y(codes, sum_scale, t, alpha, N, np.arange(M))
+    assert bf16_rows_rel_err(y, ex) <= BF16_ROW_TOL
+
+
+# the largest sums the GEMV meets: every activation -128 against rows of all
+# +1, all -1, all 0 and random signs, at the longest K it takes
+@pytest.mark.parametrize("M,K", [(1, 65536), (2, 65536), (4, 32768), (8, 16384), (1, 16384), (3, 18432)])
+def test_gemv_t2_extreme_sums(M, K):
+    N = 12
+    g = synth.rng(M + K)
+    a = np.full((M, K), -128, np.int8)
+    t = np.zeros((N, K), np.int8)
+    t[0], t[1] = 1, -1
+    t[3:] = g.integers(-1, 2, (N - 3, K))
+    scale = np.full(M, 1e-6, np.float32)
+    alpha = np.float32(0.5)
     acc, y = run_gemm(to_dev(a), tba.BL_A_I8, scale, to_dev(oracle.pack_ternary2(t)), tba.BL_W_T2, alpha, M, N, K)
     acc_ref, _ = oracle.gemm(a, scale, t, alpha, want_y=False)
     assert np.array_equal(acc, acc_ref)
+    assert acc[0, 0] == -128 * K and acc[0, 1] == 128 * K and acc[0, 2] == 0
     _, ex = exact_y(a, scale, t, alpha, N, np.arange(M))
     assert bf16_rows_rel_err(y, ex) <= BF16_ROW_TOL
+
+
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_gemv_t2_alpha_groups_and_ldy(M):
+    F, K = 100, 4096
+    g = synth.rng(40 + M)
+    a_dev, af, codes, scale, sum_scale = gemv_inputs(g, "i4", M, K)
+    t = g.integers(-1, 2, (2 * F, K)).astype(np.int8)
+    alpha = np.array([0.0151, 0.0213], np.float32)
+    acc, y = run_gemm(a_dev, af, scale, to_dev(oracle.pack_ternary2(t)), tba.BL_W_T2, alpha, M, 2 * F, K,
+                      group=F, ldy=2 * F + 64)
+    acc_ref, _ = oracle.gemm(codes, sum_scale, t, alpha, alpha_group=F, want_y=False)
+    assert np.array_equal(acc, acc_ref)
+    _, ex = exact_y(codes, sum_scale, t, alpha, F, np.arange(M))
+    assert bf16_rows_rel_err(y, ex) <= BF16_ROW_TOL
+
+
+# past the GEMV's K limit the tiled CUDA-core kernel stages fewer rows of A
+# per tile; past its own limit the call is refused before any launch
+def test_gemm_t2_long_k_cuda_core():
+    M, N, K = 3, 16, 131072
+    g = synth.rng(77)
+    a_dev, af, codes, scale, sum_scale = gemv_inputs(g, "i4", M, K)
+    t = g.integers(-1, 2, (N, K)).astype(np.int8)
+    acc, y = run_gemm(a_dev, af, scale, to_dev(oracle.pack_ternary2(t)), tba.BL_W_T2, np.float32(0.02), M, N, K)
+    acc_ref, _ = oracle.gemm(codes, sum_scale, t, np.float32(0.02), want_y=False)
+    assert np.array_equal(acc, acc_ref)
+    K = 196608 + 64
+    with pytest.raises(tba.BitLinearError) as e:
+        run_gemm(to_dev(np.zeros((1, K), np.int8)), tba.BL_A_I8, np.ones(1, np.float32),
+                 to_dev(np.zeros((2, K // 4), np.uint8)), tba.BL_W_T2, np.float32(1.0), 1, 2, K)
+    assert tba.STATUS_NAMES[e.value.status] == "BL_ERR_SHAPE"
 
 
 def test_sync_status_clean():
