@@ -635,19 +635,28 @@ def run_decode(args):
         y_o = T.empty((m, d), dtype=T.int16, device=dev)
         y_ug = T.empty((m, 2 * f), dtype=T.int16, device=dev)
         y_down = T.empty((m, d), dtype=T.int16, device=dev)
+        qg_ws = T.empty((tba.workspace_size("quant_gemm", m, 2 * f, d) // 8 + 1,), dtype=T.int64, device=dev)
 
-        def layer(w2, alpha, gemms=True, others=True):
-            if others:
+        def layer(w2, alpha, gemms=True, others=True, fused=False):
+            # fused: the INT4 quantizer of the QKV and Up|Gate inputs runs inside
+            # the GEMM call (bitlinear_quant_gemm)
+            if fused:
+                tba.bitlinear_quant_gemm(x_attn, w2["qkv"], alpha[0:1], m, 3 * d, d, y=y_qkv, eps=EPS,
+                                         workspace=qg_ws)
+            if others and not fused:
                 tba.bitlinear_quant_a4(x_attn, qa, qa_s, tba.BL_QUANT_INT4, tba.BL_STORE_BYTES, EPS)
-            if gemms:
+            if gemms and not fused:
                 tba.bitlinear_gemm(qa, qa_s, w2["qkv"], alpha[0:1], m, 3 * d, d, y=y_qkv, wfmt=tba.BL_W_T2)
             if others:
                 tba.bitlinear_sparsify_a8(x_o, synth.k_keep(d, s.topk_pct_o), o8, o8_s, None, EPS)
             if gemms:
                 tba.bitlinear_gemm(o8, o8_s, w2["o"], alpha[1:2], m, d, d, y=y_o, wfmt=tba.BL_W_T2)
-            if others:
+            if fused:
+                tba.bitlinear_quant_gemm(x_ffn, w2["upgate"], alpha[2:4], m, 2 * f, d, y=y_ug, eps=EPS,
+                                         alpha_group=f, workspace=qg_ws)
+            if others and not fused:
                 tba.bitlinear_quant_a4(x_ffn, qa, qa_s, tba.BL_QUANT_INT4, tba.BL_STORE_BYTES, EPS)
-            if gemms:
+            if gemms and not fused:
                 tba.bitlinear_gemm(qa, qa_s, w2["upgate"], alpha[2:4], m, 2 * f, d, y=y_ug, wfmt=tba.BL_W_T2,
                                    alpha_group=f)
             if others:
@@ -659,6 +668,10 @@ def run_decode(args):
         def step():
             for w2, alpha in layers:
                 layer(w2, alpha)
+
+        def step_fused():
+            for w2, alpha in layers:
+                layer(w2, alpha, fused=True)
 
         def gemms_only():
             for w2, alpha in layers:
@@ -683,6 +696,7 @@ def run_decode(args):
             return graph
 
         g_step = capture(step)
+        g_fused = capture(step_fused)
         g_gemm = capture(gemms_only)
 
         def time_graph(graph):
@@ -698,18 +712,22 @@ def run_decode(args):
             return a_.elapsed_time(b_) / (args.steps * DECODE_LAYERS)
 
         ms = time_graph(g_step)
+        fused_ms = time_graph(g_fused)
         gemm_ms = time_graph(g_gemm)
         tba.sync_status()
-        del g_step, g_gemm
+        del g_step, g_fused, g_gemm
         gbs = weight_bytes / (gemm_ms / 1e3) / 1e9
         results.append({"tokens": m, "ms_per_layer": round(ms, 4), "tokens_per_s": round(m / (ms / 1e3), 1),
+                        "fused_quant_ms_per_layer": round(fused_ms, 4),
                         "gemm_ms_per_layer": round(gemm_ms, 4),
                         "gemm_kernel": decode_gemm_kernel(m),
                         "weight_stream_gbs": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 3)})
     line = {"metric": "decode BitLinear layer latency (7B shapes, 2-bit weights; CUDA-graph replay)",
             "unit": "ms per layer",
             "workload": f"7B-shape decoder layers, decode of M tokens through all four BitLinear matrices of "
-                        f"each of {DECODE_LAYERS} distinct layers (weights exceed L2)",
+                        f"each of {DECODE_LAYERS} distinct layers (weights exceed L2), separate quantizer and GEMM "
+                        f"calls; fused_quant_ms_per_layer: the QKV and Up|Gate INT4 quantizers fused into their "
+                        f"GEMMs (bitlinear_quant_gemm)",
             "weight_bytes_per_layer": weight_bytes, "hbm_peak_gbs": peaks["hbm_gbs"],
             "steps": args.steps, "warmup": args.warmup, "results": results}
     print(json.dumps(line), flush=True)

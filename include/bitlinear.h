@@ -195,6 +195,31 @@ BL_API bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scal
                          void* y_bf16, int64_t ldy, int32_t* acc_out, void* stream);
 
 /*
+ * bitlinear_quant_gemm -- bitlinear_quant_a4 fused into the BitLinear GEMM:
+ * y = bf16(Q(x) . t^T * scale[m] * alpha[n / alpha_group]) straight from the
+ * bf16 rows x (paper: §3.4, Eq. 6-7 / 8-9 followed by Y = Q_x(X) . Q_w(W)^T).
+ * The codes, the scale and acc_out are exactly those of bitlinear_quant_a4
+ * followed by bitlinear_gemm (for FP4, acc_out holds 2 * the sum, as for
+ * BL_A_E2M1 activations).
+ * With BL_W_T2 weights and a shape the decode GEMV takes (M <= 8; see
+ * bitlinear_gemm) the quantization runs in the GEMV's prologue: every CTA reads
+ * the M bf16 rows, reduces each token's statistic and quantizes into shared
+ * memory, so no codes reach global memory and there is one launch.  Otherwise
+ * it runs as bitlinear_quant_a4 (BL_STORE_BYTES) into `workspace` and then
+ * bitlinear_gemm with BL_A_I8 codes; `workspace` then needs
+ * bitlinear_workspace_size("quant_gemm", M, N, K) bytes (16-byte aligned) and
+ * may be NULL otherwise.
+ * x: [M x K] bf16, row stride ldx.  w: BL_W_T2 or BL_W_I8 (pack_ternary's
+ * output).  y / acc_out / alpha / alpha_group as in bitlinear_gemm.
+ * Requires K % 64 == 0, 64 <= K <= 16384, ldx % 8 == 0, ldy % 8 == 0.
+ */
+BL_API bl_status bitlinear_quant_gemm(const void* x_bf16, int64_t ldx, bl_quant quant, float eps,
+                               const void* w, bl_wfmt wfmt, const float* alpha, int64_t alpha_group,
+                               int64_t M, int64_t N, int64_t K,
+                               void* y_bf16, int64_t ldy, int32_t* acc_out,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * relu2_glu -- squared-ReLU GLU fused with the down projection's
  * sparsify-then-quantize step.
  * Paper: §3.4 "Squared ReLU Gating and Conditional Computation in the FFN",

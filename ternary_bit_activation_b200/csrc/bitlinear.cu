@@ -287,7 +287,7 @@ int64_t gv_tokens(int m) { return m <= 1 ? 1 : (m <= 2 ? 2 : (m <= 4 ? 4 : 8)); 
 template <int AF, int MT>
 bl_status launch_gemv_mt(const uint8_t* A, const float* a_scale, const uint8_t* W, const float* alpha,
                          int64_t alpha_group, int m, int n, int k, uint16_t* Y, int64_t ldy, int32_t* acc_out,
-                         cudaStream_t s) {
+                         cudaStream_t s, int64_t ldx, float eps) {
   static bool attr_done[kMaxDevices] = {};
   const int d = current_device();
   if (d < 0 || d >= kMaxDevices) return BL_ERR_CUDA;
@@ -313,7 +313,7 @@ bl_status launch_gemv_mt(const uint8_t* A, const float* a_scale, const uint8_t* 
   const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
   const unsigned grid = static_cast<unsigned>(passes < cap ? passes : cap);
   launch_pdl(bl::gemv_t2_kernel<AF, MT>, grid, threads, smem, s, A, a_scale, W, alpha, alpha_group, m, n, k, S, G,
-             Y, ldy, acc_out);
+             Y, ldy, acc_out, ldx, eps);
   return launch_status();
 }
 
@@ -326,7 +326,7 @@ constexpr int kGmSmemLimit = 144 * 1024 + 16384;    // + batch partial sums (two
 template <int AF>
 bl_status launch_gemv_mma(const uint8_t* A, const float* a_scale, const uint8_t* W, const float* alpha,
                           int64_t alpha_group, int m, int n, int k, uint16_t* Y, int64_t ldy, int32_t* acc_out,
-                          cudaStream_t s) {
+                          cudaStream_t s, int64_t ldx = 0, float eps = 0.f) {
   static bool attr_done[kMaxDevices] = {};
   const int d = current_device();
   if (d < 0 || d >= kMaxDevices) return BL_ERR_CUDA;
@@ -351,21 +351,43 @@ bl_status launch_gemv_mma(const uint8_t* A, const float* a_scale, const uint8_t*
   const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
   const unsigned grid = static_cast<unsigned>(passes < cap ? passes : cap);
   launch_pdl(bl::gemv_mma_t2_kernel<AF>, grid, threads, smem, s, A, a_scale, W, alpha, alpha_group, m, n, k, S, G, Y,
-             ldy, acc_out);
+             ldy, acc_out, ldx, eps);
   return launch_status();
 }
 
 template <int AF>
 bl_status launch_gemv(const uint8_t* A, const float* a_scale, const uint8_t* W, const float* alpha,
                       int64_t alpha_group, int m, int n, int k, uint16_t* Y, int64_t ldy, int32_t* acc_out,
-                      cudaStream_t s) {
+                      cudaStream_t s, int64_t ldx = 0, float eps = 0.f) {
   switch (gv_tokens(m)) {
-    case 1: return launch_gemv_mt<AF, 1>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
-    case 2: return launch_gemv_mt<AF, 2>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
-    case 4: return launch_gemv_mt<AF, 4>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
-    default: return launch_gemv_mt<AF, 8>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+    case 1: return launch_gemv_mt<AF, 1>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s, ldx, eps);
+    case 2: return launch_gemv_mt<AF, 2>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s, ldx, eps);
+    case 4: return launch_gemv_mt<AF, 4>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s, ldx, eps);
+    default: return launch_gemv_mt<AF, 8>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s, ldx, eps);
   }
 }
+
+// The decode GEMV applies to 2-bit weights and up to 8 tokens: the warp-MMA
+// kernel from 3 tokens, the dp4a kernel otherwise (and for longer rows).
+bool gemv_applies(int64_t M, int64_t K) {
+  if (M < 1 || M > kGvMaxTokens) return false;
+  if (M >= kGmMinTokens && K <= kGmMaxK) return true;
+  return K <= kGvMaxK && gv_tokens(static_cast<int>(M)) * K <= kGvMaxActBytes;
+}
+
+template <int AF>
+bl_status launch_gemv_any(const uint8_t* A, const float* a_scale, const uint8_t* W, const float* alpha,
+                          int64_t alpha_group, int m, int n, int k, uint16_t* Y, int64_t ldy, int32_t* acc_out,
+                          cudaStream_t s, int64_t ldx = 0, float eps = 0.f) {
+  if (m >= kGmMinTokens && k <= kGmMaxK)
+    return launch_gemv_mma<AF>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s, ldx, eps);
+  return launch_gemv<AF>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s, ldx, eps);
+}
+
+// Workspace of bitlinear_quant_gemm when it runs as two kernels: M x K int8
+// codes, then M fp32 scales, each 16-byte aligned.
+int64_t qg_codes_bytes(int64_t M, int64_t K) { return (M * K + 15) / 16 * 16; }
+int64_t qg_workspace_bytes(int64_t M, int64_t K) { return qg_codes_bytes(M, K) + (4 * M + 15) / 16 * 16; }
 
 }  // namespace
 
@@ -427,8 +449,10 @@ const char* bitlinear_status_string(bl_status st) {
 }
 
 size_t bitlinear_workspace_size(const char* op, int64_t M, int64_t N, int64_t K) {
-  (void)M; (void)N; (void)K;
+  (void)N;
   if (op != nullptr && strcmp(op, "pack_ternary") == 0) return bl::kBins * sizeof(unsigned long long);
+  if (op != nullptr && strcmp(op, "quant_gemm") == 0 && M > 0 && K > 0)
+    return static_cast<size_t>(qg_workspace_bytes(M, K));
   return 0;
 }
 
@@ -629,17 +653,11 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
     launch_pdl(bl::gemm_tc_kernel, grid, bl::kTcThreads, bl::kTcSmemBytes, s, ta, tb, p);
     return launch_status();
   }
-  if (wfmt == BL_W_T2 && M >= kGmMinTokens && M <= kGvMaxTokens && K <= kGmMaxK) {
-    // 3 to 8 tokens: warp-MMA GEMV, one pass over the 2-bit weights
-    if (afmt == BL_A_I8) return launch_gemv_mma<bl::kSimtA_I8>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
-    if (afmt == BL_A_I4) return launch_gemv_mma<bl::kSimtA_I4>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
-    return launch_gemv_mma<bl::kSimtA_E2M1>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
-  }
-  if (wfmt == BL_W_T2 && M <= kGvMaxTokens && K <= kGvMaxK && gv_tokens(m) * K <= kGvMaxActBytes) {
-    // 1 or 2 tokens, or longer rows: dp4a GEMV staging only the token slots in use
-    if (afmt == BL_A_I8) return launch_gemv<bl::kSimtA_I8>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
-    if (afmt == BL_A_I4) return launch_gemv<bl::kSimtA_I4>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
-    return launch_gemv<bl::kSimtA_E2M1>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+  if (wfmt == BL_W_T2 && gemv_applies(M, K)) {
+    // up to 8 tokens: one pass over the 2-bit weights (warp-MMA from 3 tokens, else dp4a)
+    if (afmt == BL_A_I8) return launch_gemv_any<bl::kSimtA_I8>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+    if (afmt == BL_A_I4) return launch_gemv_any<bl::kSimtA_I4>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+    return launch_gemv_any<bl::kSimtA_E2M1>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
   }
   if (afmt == BL_A_I8 && wfmt == BL_W_T2 && M >= bl::kTsMinTokens) {
     // 2-bit weights widened into tensor memory; tokens on the MMA's N side
@@ -700,6 +718,46 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
   }
   if (!ok) return BL_ERR_CUDA;
   return launch_status();
+}
+
+bl_status bitlinear_quant_gemm(const void* x_bf16, int64_t ldx, bl_quant quant, float eps, const void* w,
+                               bl_wfmt wfmt, const float* alpha, int64_t alpha_group, int64_t M, int64_t N, int64_t K,
+                               void* y_bf16, int64_t ldy, int32_t* acc_out, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  if (quant != BL_QUANT_INT4 && quant != BL_QUANT_FP4_E2M1) return BL_ERR_ARG;
+  if (wfmt != BL_W_T2 && wfmt != BL_W_I8) return BL_ERR_ARG;
+  if (alpha_group < 1 || alpha_group > 0x7FFFFFFFLL || !(eps >= 0.f)) return BL_ERR_ARG;
+  if (M < 0 || N < 1 || K < 64 || (K & 63) || K > 16384 || ldx < K || (ldx & 7) || M > 0x7FFFFFFELL ||
+      N > 0x7FFFFFFFLL)
+    return BL_ERR_SHAPE;
+  if (y_bf16 != nullptr && (ldy < N || (ldy & 7))) return BL_ERR_SHAPE;
+  if (M == 0) return BL_OK;
+  if (x_bf16 == nullptr || w == nullptr || alpha == nullptr) return BL_ERR_NULL;
+  if (y_bf16 == nullptr && acc_out == nullptr) return BL_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(w) || (y_bf16 && !aligned16(y_bf16)) || (acc_out && !aligned16(acc_out)) ||
+      (reinterpret_cast<uintptr_t>(alpha) & 3u))
+    return BL_ERR_ALIGN;
+  cudaStream_t s = as_stream(stream);
+  const bool fp4 = quant == BL_QUANT_FP4_E2M1;
+  if (wfmt == BL_W_T2 && gemv_applies(M, K)) {
+    // decode: each GEMV CTA quantizes the token rows itself
+    const uint8_t* X = static_cast<const uint8_t*>(x_bf16);
+    const uint8_t* W = static_cast<const uint8_t*>(w);
+    uint16_t* Y = static_cast<uint16_t*>(y_bf16);
+    const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+    if (fp4)
+      return launch_gemv_any<bl::kGvX_Fp4>(X, nullptr, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s, ldx, eps);
+    return launch_gemv_any<bl::kGvX_Int4>(X, nullptr, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s, ldx, eps);
+  }
+  // otherwise the quantizer writes int8 codes into the workspace for the GEMM
+  if (workspace == nullptr) return BL_ERR_NULL;
+  if (!aligned16(workspace)) return BL_ERR_ALIGN;
+  if (ws_bytes < static_cast<size_t>(qg_workspace_bytes(M, K))) return BL_ERR_WORKSPACE;
+  uint8_t* codes = static_cast<uint8_t*>(workspace);
+  float* scale = reinterpret_cast<float*>(codes + qg_codes_bytes(M, K));
+  const bl_status st = bitlinear_quant_a4(x_bf16, M, K, ldx, quant, BL_STORE_BYTES, eps, codes, scale, stream);
+  if (st != BL_OK) return st;
+  return bitlinear_gemm(codes, BL_A_I8, scale, w, wfmt, alpha, alpha_group, M, N, K, y_bf16, ldy, acc_out, stream);
 }
 
 bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D, int64_t ldt, int bits, int64_t bos_pos,

@@ -22,6 +22,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "quant.cuh"
 
 namespace bl {
 
@@ -895,6 +896,9 @@ __global__ void __launch_bounds__(kTsThreads, 1)
 // expanded weight unit.  dp4a on int8x4 words.
 // ---------------------------------------------------------------------------
 enum : int { kSimtA_I8 = 0, kSimtA_I4 = 1, kSimtA_E2M1 = 2 };
+// GEMV activation sources that are bf16 rows quantized in the kernel's prologue
+// (INT4 absmean, FP4 E2M1 MinMax as twice the value), bit-identical to quant_a4
+enum : int { kGvX_Int4 = 3, kGvX_Fp4 = 4 };
 
 // four 2-bit ternary codes (one byte) -> four int8 {-1,0,1} (two's-complement sign extension)
 __device__ __forceinline__ uint32_t expand_t2_byte(uint32_t b) {
@@ -1004,7 +1008,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const uint8_t* __restric
   const int units_hi = (units + 31) >> 5;
   const int64_t a_row_bytes = (AF == kSimtA_I8) ? K : (K >> 1);
   const int64_t w_row_bytes = WT2 ? (K >> 2) : K;
-  const float unit_scale = (AF == kSimtA_E2M1) ? 0.5f : 1.0f;
+  const float unit_scale = (AF == kSimtA_E2M1 || AF == kGvX_Fp4) ? 0.5f : 1.0f;
   pdl_wait();
   pdl_trigger();
 
@@ -1174,10 +1178,114 @@ __device__ __forceinline__ void gv_load_word(const uint8_t* a, int K, int m, int
 // Stage the activations of M tokens into shared memory as field-major int8
 // words (gv_transpose) at act[slot(q, m)], zeros for the token slots M..TOK-1,
 // and add each token's code sum to asum[m].  A thread's loads for all tokens of
-// a word are in flight together.
+// a word are in flight together.  For the bf16 sources (kGvX_*) the tokens are
+// quantized here as quant_a4 does it: a first pass over the rows reduces each
+// token's statistic (the exact fp64 sum of |x|, or max |x|) over the CTA
+// through red[warp][token], the second quantizes; s_scale[m] receives the
+// token's dequant scale.
+template <int AF>
+constexpr bool gv_fused() { return AF == kGvX_Int4 || AF == kGvX_Fp4; }
+
+constexpr int kGvMaxWarps = kGvMaxThreads / 32;
+
+// bf16 x 8 -> eight int8 codes in two words (INT4: the code; FP4: twice the value)
+template <int AF>
+__device__ __forceinline__ void gv_quant8(const uint4& h, float mult, int p, uint32_t& lo, uint32_t& hi) {
+  float f[8];
+  unpack_bf16x8(h, f);
+  uint32_t q[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    if constexpr (AF == kGvX_Int4) {
+      q[e] = q4_code_bits(f[e], mult);   // low byte: the code, two's complement
+    } else {
+      const float sv = mul_pow2(f[e], -p);
+      const int i = e2m1_index(fabsf(sv));
+      const int tv = (i <= 4) ? i : (i == 5 ? 6 : (i == 6 ? 8 : 12));
+      q[e] = static_cast<uint32_t>((sv < 0.f && i != 0) ? -tv : tv);
+    }
+  }
+  lo = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+  hi = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
+}
+
 template <int AF, int TOK, typename Slot>
-__device__ __forceinline__ void gv_stage(const uint8_t* a, int M, int K, uint4* act, Slot slot, int* asum) {
+__device__ __forceinline__ void gv_stage(const uint8_t* a, int64_t ldx, float eps, int M, int K, uint4* act,
+                                         Slot slot, int* asum, double (*red)[TOK], float* s_scale) {
   const int kw16 = K >> 4;
+  float mult[TOK];
+  int pexp[TOK];
+#pragma unroll
+  for (int m = 0; m < TOK; ++m) {
+    mult[m] = 0.f;
+    pexp[m] = 0;
+  }
+  if constexpr (gv_fused<AF>()) {
+    const uint16_t* x = reinterpret_cast<const uint16_t*>(a);
+    double ps[TOK];
+    uint32_t pm[TOK];
+#pragma unroll
+    for (int m = 0; m < TOK; ++m) {
+      ps[m] = 0.0;
+      pm[m] = 0u;
+    }
+    for (int q = threadIdx.x; q < kw16; q += blockDim.x) {
+#pragma unroll
+      for (int m = 0; m < TOK; ++m) {
+        if (m >= M) continue;
+        const uint16_t* src = x + static_cast<int64_t>(m) * ldx + static_cast<int64_t>(q) * 16;
+        const uint4 h[2] = {ld_dep_v4(src), ld_dep_v4(src + 8)};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          if constexpr (AF == kGvX_Int4) {
+            float f[8];
+            unpack_bf16x8(h[hh], f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ps[m] += static_cast<double>(fabsf(f[e]));
+          } else {
+            uint32_t k[8];
+            bf16x8_mag_keys(h[hh], k);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pm[m] = max(pm[m], k[e]);
+          }
+        }
+      }
+    }
+    const int warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int m = 0; m < TOK; ++m) {
+      if constexpr (AF == kGvX_Int4) {
+        double v = ps[m];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        if ((threadIdx.x & 31) == 0) red[warp][m] = v;
+      } else {
+        const uint32_t v = __reduce_max_sync(0xFFFFFFFFu, pm[m]);
+        if ((threadIdx.x & 31) == 0) red[warp][m] = static_cast<double>(v);
+      }
+    }
+    __syncthreads();
+    const int nw = static_cast<int>(blockDim.x >> 5);
+#pragma unroll
+    for (int m = 0; m < TOK; ++m) {
+      float sc;
+      if constexpr (AF == kGvX_Int4) {
+        // the sum of bf16 magnitudes in fp64 is exact, so the order of the
+        // partial sums does not change it (the same value as quant_a4's)
+        double S = 0.0;
+        for (int i = 0; i < nw; ++i) S += red[i][m];
+        const float beta = __double2float_rn(S / static_cast<double>(K));
+        mult[m] = __fdiv_rn(sqrt7_f32(), __fadd_rn(beta, eps));
+        sc = __fdiv_rn(beta, sqrt7_f32());
+      } else {
+        uint32_t mk = 0u;
+        for (int i = 0; i < nw; ++i) mk = max(mk, static_cast<uint32_t>(red[i][m]));
+        pexp[m] = fp4_scale_exponent(mk << 16);
+        sc = exact_pow2(pexp[m]);
+      }
+      if (threadIdx.x == m && m < M) s_scale[m] = sc;
+    }
+  }
   int tsum[TOK];
 #pragma unroll
   for (int m = 0; m < TOK; ++m) tsum[m] = 0;
@@ -1186,7 +1294,16 @@ __device__ __forceinline__ void gv_stage(const uint8_t* a, int M, int K, uint4* 
 #pragma unroll
     for (int m = 0; m < TOK; ++m) {
       v[m][0] = v[m][1] = v[m][2] = v[m][3] = 0u;
-      if (m < M) gv_load_word<AF>(a, K, m, q, v[m]);
+      if (m >= M) continue;
+      if constexpr (gv_fused<AF>()) {
+        const uint16_t* src =
+            reinterpret_cast<const uint16_t*>(a) + static_cast<int64_t>(m) * ldx + static_cast<int64_t>(q) * 16;
+        const uint4 h0 = ld_dep_v4(src), h1 = ld_dep_v4(src + 8);
+        gv_quant8<AF>(h0, mult[m], pexp[m], v[m][0], v[m][1]);
+        gv_quant8<AF>(h1, mult[m], pexp[m], v[m][2], v[m][3]);
+      } else {
+        gv_load_word<AF>(a, K, m, q, v[m]);
+      }
     }
 #pragma unroll
     for (int m = 0; m < TOK; ++m) act[slot(q, m)] = gv_transpose(v[m], tsum[m]);
@@ -1205,10 +1322,13 @@ __global__ void __launch_bounds__(kGvMaxThreads) gemv_t2_kernel(const uint8_t* _
                                                                 const float* __restrict__ alpha, int64_t alpha_group,
                                                                 int M, int N, int K, int S, int G,
                                                                 uint16_t* __restrict__ y, int64_t ldy,
-                                                                int32_t* __restrict__ acc_out) {
+                                                                int32_t* __restrict__ acc_out, int64_t ldx,
+                                                                float eps) {
   constexpr int R = GvShape<MT>::R;
   extern __shared__ uint4 gv_smem[];
   __shared__ int asum[MT];
+  __shared__ float s_scale[MT];
+  __shared__ double red[kGvMaxWarps][MT];
   const int kw16 = K >> 4;                              // 16-code words per row
   const int kq = kw16 >> 2;                             // words per lane slot (kw16 % 4 == 0)
   uint4* act = gv_smem;                                 // [MT][4][kw16 / 4], field-major bytes
@@ -1257,9 +1377,10 @@ __global__ void __launch_bounds__(kGvMaxThreads) gemv_t2_kernel(const uint8_t* _
 
   // stage the activations (zeros for token slots past M) and their sums
   // word 4p + j of token m at [m][j][p]: the lanes of a warp read consecutive slots
-  gv_stage<AF, MT>(a, M, K, act, [kq](int q, int m) { return (m * 4 + (q & 3)) * kq + (q >> 2); }, asum);
+  gv_stage<AF, MT>(a, ldx, eps, M, K, act, [kq](int q, int m) { return (m * 4 + (q & 3)) * kq + (q >> 2); }, asum,
+                   red, s_scale);
   __syncthreads();
-  const float unit_scale = (AF == kSimtA_E2M1) ? 0.5f : 1.0f;
+  const float unit_scale = (AF == kSimtA_E2M1 || AF == kGvX_Fp4) ? 0.5f : 1.0f;
 
   int par = 0;
   for (int64_t gb = static_cast<int64_t>(blockIdx.x) * G; gb < groups; gb += group_step, par ^= 1) {
@@ -1363,7 +1484,8 @@ __global__ void __launch_bounds__(kGvMaxThreads) gemv_t2_kernel(const uint8_t* _
           if (acc_out != nullptr) acc_out[static_cast<int64_t>(m) * N + n] = v;
           if (y != nullptr) {
             const float cs =
-                __fmul_rn(__fmul_rn(ld_dep_f32(a_scale + m), unit_scale), ld_dep_f32(alpha + n / alpha_group));
+                __fmul_rn(__fmul_rn(gv_fused<AF>() ? s_scale[m] : ld_dep_f32(a_scale + m), unit_scale),
+                        ld_dep_f32(alpha + n / alpha_group));
             const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__int2float_rn(v), cs));
             y[static_cast<int64_t>(m) * ldy + n] = *reinterpret_cast<const uint16_t*>(&b);
           }
@@ -1406,9 +1528,12 @@ __global__ void __launch_bounds__(kGvMaxThreads) gemv_mma_t2_kernel(const uint8_
                                                                     const float* __restrict__ alpha,
                                                                     int64_t alpha_group, int M, int N, int K, int S,
                                                                     int G, uint16_t* __restrict__ y, int64_t ldy,
-                                                                    int32_t* __restrict__ acc_out) {
+                                                                    int32_t* __restrict__ acc_out, int64_t ldx,
+                                                                    float eps) {
   extern __shared__ uint4 gm_smem[];
   __shared__ int asum[kGmTokens];
+  __shared__ float s_scale[kGmTokens];
+  __shared__ double red[kGvMaxWarps][kGmTokens];
   const int kw16 = K >> 4;      // 16-code words per row (a multiple of 4)
   const int kq = kw16 >> 2;
   // activation word 4p + c of token m at (p * 4 + c) * 8 + m: the 32 lanes of
@@ -1440,10 +1565,10 @@ __global__ void __launch_bounds__(kGvMaxThreads) gemv_mma_t2_kernel(const uint8_
   pdl_trigger();
 
   // stage the activations (zeros for token slots past M) and their sums
-  gv_stage<AF, kGmTokens>(a, M, K, act, [](int q, int m) { return ((q >> 2) * 4 + (q & 3)) * kGmTokens + m; },
-                          asum);
+  gv_stage<AF, kGmTokens>(a, ldx, eps, M, K, act,
+                          [](int q, int m) { return ((q >> 2) * 4 + (q & 3)) * kGmTokens + m; }, asum, red, s_scale);
   __syncthreads();
-  const float unit_scale = (AF == kSimtA_E2M1) ? 0.5f : 1.0f;
+  const float unit_scale = (AF == kSimtA_E2M1 || AF == kGvX_Fp4) ? 0.5f : 1.0f;
 
   int par = 0;
   for (int64_t tb = static_cast<int64_t>(blockIdx.x) * G; tb < tiles; tb += tile_step, par ^= 1) {
@@ -1506,7 +1631,8 @@ __global__ void __launch_bounds__(kGvMaxThreads) gemv_mma_t2_kernel(const uint8_
         if (acc_out != nullptr) acc_out[static_cast<int64_t>(m) * N + n] = v;
         if (y != nullptr) {
           const float cs =
-              __fmul_rn(__fmul_rn(ld_dep_f32(a_scale + m), unit_scale), ld_dep_f32(alpha + n / alpha_group));
+              __fmul_rn(__fmul_rn(gv_fused<AF>() ? s_scale[m] : ld_dep_f32(a_scale + m), unit_scale),
+                        ld_dep_f32(alpha + n / alpha_group));
           const __nv_bfloat16 bb = __float2bfloat16_rn(__fmul_rn(__int2float_rn(v), cs));
           y[static_cast<int64_t>(m) * ldy + n] = *reinterpret_cast<const uint16_t*>(&bb);
         }

@@ -46,6 +46,36 @@ def test_status_strings(L):
 def test_workspace_size(L):
     assert tba.workspace_size("pack_ternary", 0, 4096, 4096) == 2048
     assert tba.workspace_size("bitlinear_gemm", 128, 128, 128) == 0
+    # quant_gemm run as two kernels: M x K int8 codes, then M fp32 scales, each 16-byte aligned
+    assert tba.workspace_size("quant_gemm", 3, 64, 64) == 192 + 16
+    assert tba.workspace_size("quant_gemm", 32768, 4096, 4096) == 32768 * 4096 + 4 * 32768
+
+
+def test_quant_gemm_validation(L):
+    g = L.bitlinear_quant_gemm
+    ok = dict(x=A16, ldx=256, q=0, eps=1e-5, w=A16, wfmt=0, al=A16, grp=256, M=16, N=256, K=256, y=A16, ldy=256,
+              acc=None, ws=A16, wsb=1 << 20)
+
+    def call(**kw):
+        d = dict(ok, **kw)
+        return g(P(d["x"]), d["ldx"], d["q"], d["eps"], P(d["w"]), d["wfmt"], P(d["al"]), d["grp"], d["M"], d["N"],
+                 d["K"], P(d["y"]), d["ldy"], P(d["acc"]), P(d["ws"]), d["wsb"], None)
+
+    assert call(q=2) == 4
+    assert call(wfmt=2) == 4           # E2M1 weights: use the separate calls
+    assert call(eps=-1.0) == 4
+    assert call(K=100) == 3
+    assert call(K=16448) == 3          # the quantizer's row limit
+    assert call(ldx=200) == 3          # ldx < K
+    assert call(ldx=260) == 3          # ldx % 8
+    assert call(M=0) == 0
+    assert call(x=None) == 1
+    assert call(y=None, acc=None) == 1
+    assert call(x=MIS) == 2
+    # 16 tokens run as quantizer + GEMM: the workspace is checked before any launch
+    assert call(ws=None) == 1
+    assert call(ws=MIS) == 2
+    assert call(wsb=16 * 256) == 8
 
 
 # fake device addresses: validation rejects before anything dereferences them

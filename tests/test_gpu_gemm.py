@@ -414,5 +414,72 @@ def test_gemm_t2_long_k_cuda_core():
     assert tba.STATUS_NAMES[e.value.status] == "BL_ERR_SHAPE"
 
 
+# bitlinear_quant_gemm: the INT4 / FP4 quantizer fused into the GEMM.  Up to 8
+# tokens against 2-bit weights it runs in the decode GEMV's prologue (every CTA
+# quantizes the token rows itself); otherwise as quantizer + GEMM through the
+# workspace.  Either way the result must be the oracle's quantizer followed by
+# its matmul, and y must be bit-identical to the two separate calls.
+QG_CASES = [(1, 96, 640), (2, 130, 4096), (3, 37, 11008), (5, 258, 4160), (8, 40, 16384), (16, 136, 1024),
+            (40, 200, 4096)]
+
+
+@pytest.mark.parametrize("quant", ["int4", "fp4"])
+@pytest.mark.parametrize("wfmt", [tba.BL_W_T2, tba.BL_W_I8], ids=["t2", "i8w"])
+@pytest.mark.parametrize("M,N,K", QG_CASES)
+def test_quant_gemm_parity(quant, wfmt, M, N, K):
+    g = synth.rng(M * 31 + N + K + len(quant))
+    x = synth.gaussian_bf16(g, (M, K))
+    x[:, 5] = synth.f32_to_bf16_bits(synth.bf16_bits_to_f32(x[:, 5]) * 20)   # an outlier channel
+    if M >= 2:
+        x[1] = 0                                                               # an all-zero token
+    w = synth.latent_weights_f32(g, N, K)
+    t, a_ref = oracle.ternary_quantize(w, EPS)
+    wq = oracle.pack_ternary2(t) if wfmt == tba.BL_W_T2 else t.view(np.uint8)
+    q = tba.BL_QUANT_INT4 if quant == "int4" else tba.BL_QUANT_FP4_E2M1
+    if quant == "int4":
+        codes, _, scale = oracle.quant_int4(x, EPS)
+        sum_scale = scale
+    else:
+        _, codes, _, scale = oracle.quant_fp4(x)
+        sum_scale = (scale.astype(np.float64) / 2).astype(np.float32)
+    ldx = K + 64
+    xp = np.zeros((M, ldx), np.uint16)
+    xp[:, :K] = x
+    xd, wd = to_dev(xp), to_dev(wq)
+    al = to_dev(np.array([a_ref], np.float32))
+    ldy = (N + 7) // 8 * 8
+    y, acc = empty((M, ldy), torch.int16), empty((M, N), torch.int32)
+    ws = empty((tba.workspace_size("quant_gemm", M, N, K) // 8 + 1,), torch.int64)
+    tba.bitlinear_quant_gemm(xd, wd, al, M, N, K, y=y, acc=acc, quant=q, wfmt=wfmt, eps=EPS, ldx=ldx, workspace=ws)
+    tba.sync_status()
+    acc_ref, _ = oracle.gemm(codes, sum_scale, t, a_ref, want_y=False)
+    assert np.array_equal(host(acc), acc_ref)
+    _, ex = exact_y(codes, sum_scale, t, a_ref, N, np.arange(M))
+    y_fused = host(y, np.uint16)[:, :N]
+    assert bf16_rows_rel_err(y_fused, ex) <= BF16_ROW_TOL
+    # the same two steps as separate calls
+    c8, s8 = empty((M, K), torch.int8), empty((M,), torch.float32)
+    tba.bitlinear_quant_a4(xd, c8, s8, q, tba.BL_STORE_BYTES, EPS, M=M, K=K, ldx=ldx)
+    y2 = empty((M, ldy), torch.int16)
+    tba.bitlinear_gemm(c8, s8, wd, al, M, N, K, y=y2, wfmt=wfmt)
+    tba.sync_status()
+    assert np.array_equal(host(y2, np.uint16)[:, :N], y_fused)
+
+
+def test_quant_gemm_needs_workspace_beyond_the_gemv():
+    M, N, K = 16, 64, 256
+    x = to_dev(np.zeros((M, K), np.uint16))
+    w = to_dev(np.zeros((N, K // 4), np.uint8))
+    al = to_dev(np.ones(1, np.float32))
+    y = empty((M, N), torch.int16)
+    with pytest.raises(tba.BitLinearError) as e:
+        tba.bitlinear_quant_gemm(x, w, al, M, N, K, y=y)
+    assert tba.STATUS_NAMES[e.value.status] == "BL_ERR_NULL"
+    # the decode GEMV needs none
+    tba.bitlinear_quant_gemm(x[:4], w, al, 4, N, K, y=y[:4])
+    tba.sync_status()
+    assert np.array_equal(host(y[:4], np.uint16), np.zeros((4, N), np.uint16))
+
+
 def test_sync_status_clean():
     tba.sync_status()
