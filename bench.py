@@ -745,6 +745,7 @@ PROFILE_CASES = {
     "kv_quant3": "3-bit KV, K bf16 [32768 x 32 x 128]",
     "pack_ternary": "ternary pack to int8, W fp32 [22016 x 4096]",
     "gemm_decode": "CUDA-core GEMV, 2-bit W [12288 x 4096], 1 token",
+    "gemm_decode_mma": "warp-MMA GEMV, 2-bit W [12288 x 4096], 8 tokens",
     "gemm_decode_tc": "tcgen05 GEMM, 2-bit W [12288 x 4096] widened into TMEM, 16 tokens",
 }
 
@@ -769,8 +770,8 @@ def run_profile_case(name: str, launches: int):
         al = torch.full((1,), 0.0173, device=dev)
         y = torch.empty((M, N), dtype=torch.int16, device=dev)
         fn = lambda: tba.bitlinear_gemm(a, s, w, al, M, N, K, y=y)
-    elif name == "gemm_decode":
-        M, N, K = 1, 12288, 4096
+    elif name in ("gemm_decode", "gemm_decode_mma"):
+        M, N, K = (1 if name == "gemm_decode" else 8), 12288, 4096
         a = torch.randint(-8, 8, (M, K), generator=g, device=dev, dtype=torch.int8)
         w = torch.randint(0, 256, (N, K // 4), generator=g, device=dev, dtype=torch.int32).to(torch.uint8)
         s = torch.rand((M,), generator=g, device=dev)
