@@ -34,11 +34,13 @@ struct __align__(16) TkShared {
   uint32_t cnt[F32 ? 2048 : 4096];         // 256 bins x 16 columns (u32, or u16 pairs for fp32)
   uint32_t tot[256];                       // bin totals of the current pass
   uint32_t red[8][2];                      // per-warp max key / nonzero count
-  int32_t ties[8][kTkMaxSlots];            // ties at the threshold per (warp, slot)
+  uint32_t scan[8];                        // per-warp tie counts (rank scan)
   uint32_t sel[4];                         // selected digit, count above it, its count
   uint32_t hist[2][F32 ? 256 : 1];         // list passes (fp32 keys)
   uint32_t list_n;
   uint32_t list[F32 ? kTkListCap : 1];
+  uint32_t maskw[kTkMaxSlots * kTkThreads / 4];   // mask bits of the row, 8 per chunk
+  uint16_t tiec[F32 ? kTkMaxSlots * kTkThreads : 2];   // fp32 rows: ties per chunk, then their prefix
 };
 
 // Bytes of dynamic shared memory for rows of K values.
@@ -58,21 +60,27 @@ __device__ __forceinline__ void tk_count(uint32_t* cnt, uint32_t bin, int col, u
   }
 }
 
-// Sum of bin b over the 16 counter columns, the column order rotated so that
-// the 32 lanes of a warp read 32 banks (lanes 2m and 2m+1 share words for fp32).
+// Sum of bin b over the 16 counter columns: four 16-byte loads, the quarter
+// order rotated by (lane / 2) % 4 so that each 8-lane phase of a load covers 8
+// different 4-bank groups (lanes 2m and 2m+1 read the same words for fp32).
 template <bool F32>
 __device__ __forceinline__ uint32_t tk_bin_total(const uint32_t* cnt, uint32_t b, int lane) {
+  const int rot = (lane >> 1) & 3;
+  const uint4* w = reinterpret_cast<const uint4*>(cnt + ((F32 ? (b >> 1) : b) << 4));
   uint32_t s = 0;
-  const int rot = lane >> 1;
   if constexpr (F32) {
-    const uint32_t* w = cnt + ((b >> 1) << 4);
     const int sh = (b & 1u) ? 16 : 0;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) s += (w[(rot + j) & 15] >> sh) & 0xFFFFu;
+    for (int j = 0; j < 4; ++j) {
+      const uint4 v = w[(rot + j) & 3];
+      s += ((v.x >> sh) & 0xFFFFu) + ((v.y >> sh) & 0xFFFFu) + ((v.z >> sh) & 0xFFFFu) + ((v.w >> sh) & 0xFFFFu);
+    }
   } else {
-    const uint32_t* w = cnt + (b << 4);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) s += w[(rot + j) & 15];
+    for (int j = 0; j < 4; ++j) {
+      const uint4 v = w[(rot + j) & 3];
+      s += (v.x + v.y) + (v.z + v.w);
+    }
   }
   return s;
 }
@@ -149,10 +157,19 @@ __global__ void __launch_bounds__(kTkThreads, F32 ? 2 : 4) topk_rows_kernel(
   const int row_words = nchunk;
   const int stage_words = F32 ? 2 * row_words : row_words;
   uint4* stages = reinterpret_cast<uint4*>(tk_dyn + sizeof(TkShared<F32>));
+  // bf16 rows: thread t owns the contiguous chunks [q_begin, q_end), a run of the
+  // row in index order, so a tie's rank is one scan over threads.  fp32 rows
+  // (six or more chunks per thread at the FFN width) stride their chunks over
+  // the threads instead, which keeps the 16-byte shared-memory accesses free of
+  // bank conflicts; their rare tie ranks come from a scan in chunk order.
   const int slots = (nchunk + kTkThreads - 1) / kTkThreads;
+  const int q_begin = F32 ? tid : min(tid * slots, nchunk);
+  const int q_end = F32 ? nchunk : min(q_begin + slots, nchunk);
+  constexpr int q_step = F32 ? kTkThreads : 1;
   const int mwords = (K + 31) >> 5;
   constexpr int kCntWords = F32 ? 2048 : 4096;
   const int col = lane & 15;
+  uint8_t* maskb = reinterpret_cast<uint8_t*>(sm.maskw);
 
   auto prefetch = [&](int64_t r, int buf) {
     if (r < M) {
@@ -185,7 +202,7 @@ __global__ void __launch_bounds__(kTkThreads, F32 ? 2 : 4) topk_rows_kernel(
 
     // ---- sweep 1: max key; bf16 counts its first digit, fp32 writes h and counts nonzeros ----
     uint32_t mk = 0, nz = 0;
-    for (int q = tid; q < nchunk; q += kTkThreads) {
+    for (int q = q_begin; q < q_end; q += q_step) {
       if constexpr (F32) {
         const uint4 gv = st[q], uv = st[row_words + q];
         float g[8], u[8];
@@ -248,7 +265,9 @@ __global__ void __launch_bounds__(kTkThreads, F32 ? 2 : 4) topk_rows_kernel(
         const uint32_t dmask = shift == 0 ? 0x7Fu : 0xFFu;
         if (!listed) {
           if (!counted) {
-            for (int q = tid; q < nchunk; q += kTkThreads) {
+            // the candidates (keys with the digits fixed so far) count 1, the
+            // others 0: one branch-free atomic per value
+            for (int q = q_begin; q < q_end; q += q_step) {
               uint32_t k[8];
               float f[8];
               tk_keys<F32>(st, q, row_words, k, f);
@@ -297,7 +316,7 @@ __global__ void __launch_bounds__(kTkThreads, F32 ? 2 : 4) topk_rows_kernel(
           if (tid == 0) sm.list_n = 0;
           for (int i = tid; i < 512; i += kTkThreads) (&sm.hist[0][0])[i] = 0;
           __syncthreads();
-          for (int q = tid; q < nchunk; q += kTkThreads) {
+          for (int q = q_begin; q < q_end; q += q_step) {
             uint32_t k[8];
             float f[8];
             tk_keys<F32>(st, q, row_words, k, f);
@@ -321,94 +340,95 @@ __global__ void __launch_bounds__(kTkThreads, F32 ? 2 : 4) topk_rows_kernel(
     // the tied key is 0 without a mask: a kept zero and a dropped one both get code 0.
     const bool partial = !all_kept && take < tie_total && (thr != 0u || mask != nullptr);
 
+    // ---- ties before this thread's values (bf16: before its run) ----
+    uint32_t before = 0;
+    auto block_exclusive_scan = [&](uint32_t n) {
+      uint32_t inc = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+        if (lane >= o) inc += v;
+      }
+      if (lane == 31) sm.scan[wig] = inc;
+      __syncthreads();
+      uint32_t wb = 0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) wb += w < wig ? sm.scan[w] : 0u;
+      return wb + inc - n;
+    };
+    if (partial) {
+      if constexpr (F32) {
+        // ties per chunk, an exclusive scan in chunk (= index) order, read back per chunk
+        for (int q = q_begin; q < q_end; q += q_step) {
+          uint32_t k[8];
+          float f[8];
+          tk_keys<F32>(st, q, row_words, k, f);
+          uint32_t n = 0;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) n += k[e] == thr ? 1u : 0u;
+          sm.tiec[q] = static_cast<uint16_t>(n);
+        }
+        __syncthreads();
+        const int c0 = min(tid * slots, nchunk), c1 = min(c0 + slots, nchunk);
+        uint32_t n = 0;
+        for (int c = c0; c < c1; ++c) n += sm.tiec[c];
+        uint32_t run = block_exclusive_scan(n);
+        for (int c = c0; c < c1; ++c) {
+          const uint32_t t = sm.tiec[c];
+          sm.tiec[c] = static_cast<uint16_t>(run);   // ties before chunk c (< 2^16: K <= 16384)
+          run += t;
+        }
+        __syncthreads();
+      } else {
+        uint32_t n = 0;
+        for (int q = q_begin; q < q_end; q += q_step) {
+          uint32_t k[8];
+          float f[8];
+          tk_keys<F32>(st, q, row_words, k, f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) n += k[e] == thr ? 1u : 0u;
+        }
+        before = block_exclusive_scan(n);
+      }
+    }
+
     // ---- codes and mask ----
     const float gamma = F32 ? __uint_as_float(mk) : __uint_as_float(mk << 16);
     const float denom = __fadd_rn(gamma, eps);
     const float mult = denom > 0.f ? __fdiv_rn(127.f, denom) : 0.f;
     if (tid == 0) scale[row] = __fdiv_rn(gamma, 127.f);
-    if (partial) {
-      for (int c = 0; c < slots; ++c) {
-        const int q = tid + c * kTkThreads;
-        int n = 0;
-        if (q < nchunk) {
-          uint32_t k[8];
-          float f[8];
-          tk_keys<F32>(st, q, row_words, k, f);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) n += k[e] == thr ? 1 : 0;
-        }
-        n = __reduce_add_sync(0xFFFFFFFFu, n);
-        if (lane == 0) sm.ties[wig][c] = n;
-      }
-      __syncthreads();
-    }
-    uint32_t before = 0;   // ties in earlier slots, over the whole row
-    for (int c = 0; c < slots; ++c) {
-      const int q = tid + c * kTkThreads;
-      const bool ok = q < nchunk;
+    for (int q = q_begin; q < q_end; q += q_step) {
       uint32_t k[8];
       float f[8];
-      if (ok) {
-        tk_keys<F32>(st, q, row_words, k, f);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          k[e] = 0;
-          f[e] = 0.f;
-        }
-      }
+      tk_keys<F32>(st, q, row_words, k, f);
       uint32_t bits = 0;
       if (!partial) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) bits |= (k[e] >= thr ? 1u : 0u) << e;
       } else {
-        // ties in this chunk: all kept, all dropped, or ranked (the slot holding the cut)
-        uint32_t slot_total = 0, warps_before = 0;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          const uint32_t tw = static_cast<uint32_t>(sm.ties[w][c]);
-          slot_total += tw;
-          warps_before += w < wig ? tw : 0u;
-        }
-        const bool keep_all = before + slot_total <= take;
-        const bool drop_all = before >= take;
-        int rank = 0;
-        if (!keep_all && !drop_all) {
-          int mine = 0;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) mine += (ok && k[e] == thr) ? 1 : 0;
-          int inc = mine;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int other = __shfl_up_sync(0xFFFFFFFFu, inc, o);
-            if (lane >= o) inc += other;
-          }
-          rank = static_cast<int>(before + warps_before) + inc - mine;
-        }
-        const uint32_t tie_ok = keep_all ? 1u : 0u;
+        if constexpr (F32) before = sm.tiec[q];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const uint32_t eq = k[e] == thr ? 1u : 0u;
-          const uint32_t ranked = (!drop_all && rank < static_cast<int>(take)) ? 1u : 0u;
-          const uint32_t kp = (k[e] > thr ? 1u : 0u) | (eq & (tie_ok | ranked));
-          rank += static_cast<int>(eq);
+          const uint32_t kp = (k[e] > thr ? 1u : 0u) | (eq & (before < take ? 1u : 0u));
+          before += eq;
           bits |= kp << e;
         }
-        before += slot_total;
       }
-      if (!ok) bits = 0;
-      if (ok) {
-        uint32_t cb[8];
+      uint32_t cb[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) cb[e] = tk_code_bits(f[e], mult);
-        reinterpret_cast<uint2*>(codes + row * static_cast<int64_t>(K))[q] = tk_pack_codes(cb, bits);
-      }
-      if (mask != nullptr) {
-        // chunks q..q+3 (lanes 4i..4i+3 of one slot) form one 32-bit mask word
-        const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, bits, 1);
-        const uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, bits, 2);
-        const uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, bits, 3);
-        if (ok && (lane & 3) == 0) mask[row * mwords + (q >> 2)] = bits | (b1 << 8) | (b2 << 16) | (b3 << 24);
+      for (int e = 0; e < 8; ++e) cb[e] = tk_code_bits(f[e], mult);
+      reinterpret_cast<uint2*>(codes + row * static_cast<int64_t>(K))[q] = tk_pack_codes(cb, bits);
+      if (mask != nullptr) maskb[q] = static_cast<uint8_t>(bits);
+    }
+    if (mask != nullptr) {
+      __syncthreads();
+      for (int w = tid; w < mwords; w += kTkThreads) {
+        uint32_t v = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          if (4 * w + b < nchunk) v |= static_cast<uint32_t>(maskb[4 * w + b]) << (8 * b);
+        mask[row * mwords + w] = v;
       }
     }
     __syncthreads();   // the stage and the shared state are reused
