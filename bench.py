@@ -585,7 +585,7 @@ def run_reference(args):
 # layers (2-bit weights packed once, as at inference); the layers' weights
 # together exceed L2, so every layer streams its weights from HBM.  Activations
 # are INT4 / Top-K INT8 codes one byte each; the GEMM runs on the dp4a GEMV for
-# 1-2 tokens, the warp-MMA GEMV for 3-8 and the tensor cores beyond.
+# 1-2 tokens, the warp-MMA GEMV for 3-16 and the tensor cores beyond.
 # ---------------------------------------------------------------------------
 DECODE_LAYERS = 4   # 4 x 50.6 MB of 2-bit weights > the 126 MB L2
 
@@ -593,7 +593,7 @@ DECODE_LAYERS = 4   # 4 x 50.6 MB of 2-bit weights > the 126 MB L2
 def decode_gemm_kernel(m: int) -> str:
     if m <= 2:
         return "CUDA-core GEMV (dp4a on offset codes)"
-    if m <= 8:
+    if m <= 16:
         return "warp-MMA GEMV (m16n8k32 u8 x s8)"
     return "tcgen05 (2-bit weights widened into TMEM)"
 

@@ -174,14 +174,14 @@ BL_API bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int6
  * y: [M x N] bf16 with row stride ldy (nullable).  acc_out: [M x N] int32,
  * row stride N (nullable; a test aid).
  * Kernels: BL_A_I8 x BL_W_I8 runs on the tcgen05 tensor cores (kind::i8,
- * TMA-fed, TMEM accumulators).  BL_W_T2 with M <= 8 (decode) runs on a GEMV
+ * TMA-fed, TMEM accumulators).  BL_W_T2 with M <= 16 (decode) runs on a GEMV
  * that reads the 2-bit weights once, for any activation format: 1 or 2 tokens
- * (or K > 18432) with dp4a, 3 to 8 tokens on warp-level integer MMA (16 weight
- * rows x 8 token slots), both on the offset codes c + 1 with the token's code
- * sum subtracted; the GEMV needs K <= 65536 and (token slots, 1/2/4/8) x K
- * <= 147456.  BL_A_I8 x BL_W_T2 with M > 8 runs on the tensor cores, the 2-bit
- * weights widened to int8 into tensor memory as the MMA's A operand (the tokens
- * are the MMA's N side).  Other cases run on a CUDA-core kernel that reads
+ * with dp4a (token slots 1/2/4/8 x K <= 147456, K <= 65536), 3 to 16 tokens on
+ * warp-level integer MMA (16 weight rows x 8 or 16 token slots, slots x K <=
+ * 180224), both on the offset codes c + 1 with the token's code sum subtracted.
+ * BL_A_I8 x BL_W_T2 beyond those runs on the tensor cores, the 2-bit weights
+ * widened to int8 into tensor memory as the MMA's A operand (the tokens are the
+ * MMA's N side).  Other cases run on a CUDA-core kernel that reads
  * packed operands directly and needs K <= 196608 (BL_ERR_SHAPE beyond).
  * BL_A_E2M1 x BL_W_E2M1 (any M) runs on the tensor cores as kind::mxf4 with
  * unit block scales and fp32 accumulation, exact for these operands (every

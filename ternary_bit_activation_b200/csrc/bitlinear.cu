@@ -317,13 +317,20 @@ bl_status launch_gemv_mt(const uint8_t* A, const float* a_scale, const uint8_t* 
   return launch_status();
 }
 
-// Warp-MMA GEMV: all 8 token slots staged, so 8 x K activation bytes.  One
-// or two tokens run faster on the dp4a GEMV (the MMA's 8 columns mostly idle).
-constexpr int64_t kGmMaxK = kGvMaxActBytes / 8;
+// Warp-MMA GEMV: 8 or 16 token slots (NT) staged, so NT x K activation bytes.
+// One or two tokens run faster on the dp4a GEMV (the MMA's 8 columns mostly
+// idle); beyond 16 tokens the tcgen05 decode kernel takes over.
 constexpr int64_t kGmMinTokens = 3;
-constexpr int kGmSmemLimit = 144 * 1024 + 16384;    // + batch partial sums (two buffers)
+constexpr int64_t kGmMaxTokens = 16;
+constexpr int64_t kGmActBytes = 176 * 1024;
+constexpr int kGmSmemLimit = 176 * 1024 + 32768;    // + batch partial sums (two buffers)
 
-template <int AF>
+int64_t gm_slots(int64_t m) { return m <= 8 ? 8 : 16; }
+bool gm_applies(int64_t M, int64_t K) {
+  return M >= kGmMinTokens && M <= kGmMaxTokens && gm_slots(M) * K <= kGmActBytes;
+}
+
+template <int AF, int NT>
 bl_status launch_gemv_mma(const uint8_t* A, const float* a_scale, const uint8_t* W, const float* alpha,
                           int64_t alpha_group, int m, int n, int k, uint16_t* Y, int64_t ldy, int32_t* acc_out,
                           cudaStream_t s, int64_t ldx = 0, float eps = 0.f) {
@@ -331,7 +338,7 @@ bl_status launch_gemv_mma(const uint8_t* A, const float* a_scale, const uint8_t*
   const int d = current_device();
   if (d < 0 || d >= kMaxDevices) return BL_ERR_CUDA;
   if (!attr_done[d]) {
-    if (!cuda_ok(cudaFuncSetAttribute(bl::gemv_mma_t2_kernel<AF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (!cuda_ok(cudaFuncSetAttribute(bl::gemv_mma_t2_kernel<AF, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       kGmSmemLimit)))
       return BL_ERR_CUDA;
     attr_done[d] = true;
@@ -341,17 +348,17 @@ bl_status launch_gemv_mma(const uint8_t* A, const float* a_scale, const uint8_t*
   const int G = S >= 8 ? 1 : 8 / S;                                           // tiles per CTA and pass
   const int threads = 32 * G * S;
   const int64_t tiles = (static_cast<int64_t>(n) + 15) / 16;
-  const size_t smem = static_cast<size_t>(bl::kGmTokens) * static_cast<size_t>(k) +
-                      2 * static_cast<size_t>(G * S * 32) * sizeof(int4);
+  const size_t smem = static_cast<size_t>(NT) * static_cast<size_t>(k) +
+                      2 * static_cast<size_t>(G * S * (NT / 8) * 32) * sizeof(int4);
   int per_sm = 0;
-  if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bl::gemv_mma_t2_kernel<AF>, threads, smem)))
+  if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bl::gemv_mma_t2_kernel<AF, NT>, threads, smem)))
     return BL_ERR_CUDA;
   if (per_sm < 1) per_sm = 1;
   const int64_t passes = (tiles + G - 1) / G;
   const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
   const unsigned grid = static_cast<unsigned>(passes < cap ? passes : cap);
-  launch_pdl(bl::gemv_mma_t2_kernel<AF>, grid, threads, smem, s, A, a_scale, W, alpha, alpha_group, m, n, k, S, G, Y,
-             ldy, acc_out, ldx, eps);
+  launch_pdl(bl::gemv_mma_t2_kernel<AF, NT>, grid, threads, smem, s, A, a_scale, W, alpha, alpha_group, m, n, k, S, G,
+             Y, ldy, acc_out, ldx, eps);
   return launch_status();
 }
 
@@ -367,20 +374,24 @@ bl_status launch_gemv(const uint8_t* A, const float* a_scale, const uint8_t* W, 
   }
 }
 
-// The decode GEMV applies to 2-bit weights and up to 8 tokens: the warp-MMA
-// kernel from 3 tokens, the dp4a kernel otherwise (and for longer rows).
-bool gemv_applies(int64_t M, int64_t K) {
-  if (M < 1 || M > kGvMaxTokens) return false;
-  if (M >= kGmMinTokens && K <= kGmMaxK) return true;
-  return K <= kGvMaxK && gv_tokens(static_cast<int>(M)) * K <= kGvMaxActBytes;
+// The decode GEMVs apply to 2-bit weights and up to max_tokens tokens (16; 8
+// when they quantize bf16 rows themselves): the warp-MMA kernel from 3 tokens,
+// the dp4a kernel otherwise (and for rows too long to stage 8 or 16 slots).
+bool gemv_applies(int64_t M, int64_t K, int64_t max_tokens) {
+  if (M < 1 || M > max_tokens) return false;
+  if (gm_applies(M, K)) return true;
+  return M <= kGvMaxTokens && K <= kGvMaxK && gv_tokens(static_cast<int>(M)) * K <= kGvMaxActBytes;
 }
 
 template <int AF>
 bl_status launch_gemv_any(const uint8_t* A, const float* a_scale, const uint8_t* W, const float* alpha,
                           int64_t alpha_group, int m, int n, int k, uint16_t* Y, int64_t ldy, int32_t* acc_out,
                           cudaStream_t s, int64_t ldx = 0, float eps = 0.f) {
-  if (m >= kGmMinTokens && k <= kGmMaxK)
-    return launch_gemv_mma<AF>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s, ldx, eps);
+  if (gm_applies(m, k)) {
+    if (m <= 8) return launch_gemv_mma<AF, 8>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s, ldx, eps);
+    if constexpr (!bl::gv_fused<AF>())
+      return launch_gemv_mma<AF, 16>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s, ldx, eps);
+  }
   return launch_gemv<AF>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s, ldx, eps);
 }
 
@@ -653,8 +664,8 @@ bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, cons
     launch_pdl(bl::gemm_tc_kernel, grid, bl::kTcThreads, bl::kTcSmemBytes, s, ta, tb, p);
     return launch_status();
   }
-  if (wfmt == BL_W_T2 && gemv_applies(M, K)) {
-    // up to 8 tokens: one pass over the 2-bit weights (warp-MMA from 3 tokens, else dp4a)
+  if (wfmt == BL_W_T2 && gemv_applies(M, K, kGmMaxTokens)) {
+    // up to 16 tokens: one pass over the 2-bit weights (warp-MMA from 3 tokens, else dp4a)
     if (afmt == BL_A_I8) return launch_gemv_any<bl::kSimtA_I8>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
     if (afmt == BL_A_I4) return launch_gemv_any<bl::kSimtA_I4>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
     return launch_gemv_any<bl::kSimtA_E2M1>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
@@ -739,7 +750,7 @@ bl_status bitlinear_quant_gemm(const void* x_bf16, int64_t ldx, bl_quant quant, 
     return BL_ERR_ALIGN;
   cudaStream_t s = as_stream(stream);
   const bool fp4 = quant == BL_QUANT_FP4_E2M1;
-  if (wfmt == BL_W_T2 && gemv_applies(M, K)) {
+  if (wfmt == BL_W_T2 && gemv_applies(M, K, kGvMaxTokens)) {
     // decode: each GEMV CTA quantizes the token rows itself
     const uint8_t* X = static_cast<const uint8_t*>(x_bf16);
     const uint8_t* W = static_cast<const uint8_t*>(w);

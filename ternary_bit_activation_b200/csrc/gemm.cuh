@@ -1509,9 +1509,10 @@ __global__ void __launch_bounds__(kGvMaxThreads) gemv_t2_kernel(const uint8_t* _
 // each token's sum_k a_k is subtracted at the end.  CTAs are persistent and
 // stage the activations once; K is split into 1024-code batches over S warps
 // per tile whose partial sums meet in shared memory; every weight line a warp
-// will read is prefetched into L2 before its wait.
+// will read is prefetched into L2 before its wait.  With 16 token slots (NT)
+// every weight fragment feeds two MMAs, one per 8 tokens.
 // ---------------------------------------------------------------------------
-constexpr int kGmTokens = 8;          // MMA columns: token slots
+constexpr int kGmTokens = 8;          // MMA columns: token slots of one MMA
 constexpr int kGmBatchWords = 64;     // 16-code words per row and batch (4 steps of 16)
 
 __device__ __forceinline__ void mma_u8s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -1521,7 +1522,7 @@ __device__ __forceinline__ void mma_u8s8_16832(int (&d)[4], uint32_t a0, uint32_
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <int AF>
+template <int AF, int NT>
 __global__ void __launch_bounds__(kGvMaxThreads) gemv_mma_t2_kernel(const uint8_t* __restrict__ a,
                                                                     const float* __restrict__ a_scale,
                                                                     const uint8_t* __restrict__ w,
@@ -1531,15 +1532,17 @@ __global__ void __launch_bounds__(kGvMaxThreads) gemv_mma_t2_kernel(const uint8_
                                                                     int32_t* __restrict__ acc_out, int64_t ldx,
                                                                     float eps) {
   extern __shared__ uint4 gm_smem[];
-  __shared__ int asum[kGmTokens];
-  __shared__ float s_scale[kGmTokens];
-  __shared__ double red[kGvMaxWarps][kGmTokens];
+  static_assert(NT == 8 || NT == 16, "token slots");
+  constexpr int kH = NT / kGmTokens;   // MMAs per weight fragment
+  __shared__ int asum[NT];
+  __shared__ float s_scale[NT];
+  __shared__ double red[kGvMaxWarps][NT];
   const int kw16 = K >> 4;      // 16-code words per row (a multiple of 4)
   const int kq = kw16 >> 2;
   // activation word 4p + c of token m at (p * 4 + c) * 8 + m: the 32 lanes of
   // a B-fragment load hit 8 consecutive slots 4 times (no bank conflict)
   uint4* act = gm_smem;
-  int4* part = reinterpret_cast<int4*>(act + static_cast<size_t>(kq) * 4 * kGmTokens);   // [2][G][S][32]
+  int4* part = reinterpret_cast<int4*>(act + static_cast<size_t>(kq) * 4 * NT);   // [2][G][S][kH][32]
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int g = warp / S;
@@ -1559,14 +1562,14 @@ __global__ void __launch_bounds__(kGvMaxThreads) gemv_mma_t2_kernel(const uint8_
       const int64_t off = static_cast<int64_t>(b) * (kGmBatchWords * 4) + (lane >> 4) * 128;
       if (n < N && off < wrow_bytes) prefetch_l2(w + n * wrow_bytes + off);
     }
-  if (threadIdx.x < kGmTokens) asum[threadIdx.x] = 0;
+  if (threadIdx.x < NT) asum[threadIdx.x] = 0;
   __syncthreads();
   pdl_wait();
   pdl_trigger();
 
   // stage the activations (zeros for token slots past M) and their sums
-  gv_stage<AF, kGmTokens>(a, ldx, eps, M, K, act,
-                          [](int q, int m) { return ((q >> 2) * 4 + (q & 3)) * kGmTokens + m; }, asum, red, s_scale);
+  gv_stage<AF, NT>(a, ldx, eps, M, K, act, [](int q, int m) { return ((q >> 2) * 4 + (q & 3)) * NT + m; }, asum,
+                   red, s_scale);
   __syncthreads();
   const float unit_scale = (AF == kSimtA_E2M1 || AF == kGvX_Fp4) ? 0.5f : 1.0f;
 
@@ -1577,7 +1580,7 @@ __global__ void __launch_bounds__(kGvMaxThreads) gemv_mma_t2_kernel(const uint8_
     const int64_t r1 = r0 + 8;
     const bool ok0 = tile < tiles && r0 < N;
     const bool ok1 = tile < tiles && r1 < N;
-    int c[4] = {0, 0, 0, 0};
+    int c[kH][4] = {};
     for (int b = rd; b < batches; b += S) {
       // words 4 tig .. 4 tig + 3 of rows r0 and r1 in each of the batch's 4 steps
       uint4 w0[4], w1[4];
@@ -1596,38 +1599,47 @@ __global__ void __launch_bounds__(kGvMaxThreads) gemv_mma_t2_kernel(const uint8_
         const bool okq = q < kw16;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
-          // words past K: zero activations (the weight side is then irrelevant)
-          const uint4 bv = okq ? act[((q >> 2) * 4 + cc) * kGmTokens + grp] : make_uint4(0, 0, 0, 0);
           const uint32_t p0 = ~x0[cc] & (0x55555555u | (x0[cc] << 1));
           const uint32_t p1 = ~x1[cc] & (0x55555555u | (x1[cc] << 1));
-          mma_u8s8_16832(c, p0 & 0x03030303u, p1 & 0x03030303u, (p0 >> 2) & 0x03030303u, (p1 >> 2) & 0x03030303u,
-                         bv.x, bv.y);
-          mma_u8s8_16832(c, (p0 >> 4) & 0x03030303u, (p1 >> 4) & 0x03030303u, (p0 >> 6) & 0x03030303u,
-                         (p1 >> 6) & 0x03030303u, bv.z, bv.w);
+          const uint32_t f0 = p0 & 0x03030303u, f1 = p1 & 0x03030303u;
+          const uint32_t f2 = (p0 >> 2) & 0x03030303u, f3 = (p1 >> 2) & 0x03030303u;
+          const uint32_t f4 = (p0 >> 4) & 0x03030303u, f5 = (p1 >> 4) & 0x03030303u;
+          const uint32_t f6 = (p0 >> 6) & 0x03030303u, f7 = (p1 >> 6) & 0x03030303u;
+#pragma unroll
+          for (int hh = 0; hh < kH; ++hh) {
+            // words past K: zero activations (the weight side is then irrelevant)
+            const uint4 bv = okq ? act[((q >> 2) * 4 + cc) * NT + hh * kGmTokens + grp] : make_uint4(0, 0, 0, 0);
+            mma_u8s8_16832(c[hh], f0, f1, f2, f3, bv.x, bv.y);
+            mma_u8s8_16832(c[hh], f4, f5, f6, f7, bv.z, bv.w);
+          }
         }
       }
     }
     if (S > 1) {
       // batches of a tile meet in shared memory (two buffers, as in gemv_t2_kernel)
-      int4* pp = part + static_cast<size_t>(par) * (G * S * 32);
-      pp[(g * S + rd) * 32 + lane] = make_int4(c[0], c[1], c[2], c[3]);
+      int4* pp = part + static_cast<size_t>(par) * (G * S * kH * 32);
+#pragma unroll
+      for (int hh = 0; hh < kH; ++hh)
+        pp[((g * S + rd) * kH + hh) * 32 + lane] = make_int4(c[hh][0], c[hh][1], c[hh][2], c[hh][3]);
       __syncthreads();
       if (rd != 0) continue;
-      for (int q = 1; q < S; ++q) {
-        const int4 o = pp[(g * S + q) * 32 + lane];
-        c[0] += o.x;
-        c[1] += o.y;
-        c[2] += o.z;
-        c[3] += o.w;
-      }
-    }
-    // lane (grp, tig) holds rows r0 (c0, c1) and r1 (c2, c3), tokens 2 tig and 2 tig + 1
+      for (int q = 1; q < S; ++q)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int64_t n = e < 2 ? r0 : r1;
-      const int m = 2 * tig + (e & 1);
-      if ((e < 2 ? ok0 : ok1) && m < M) {
-        const int v = c[e] - asum[m];
+        for (int hh = 0; hh < kH; ++hh) {
+          const int4 o = pp[((g * S + q) * kH + hh) * 32 + lane];
+          c[hh][0] += o.x;
+          c[hh][1] += o.y;
+          c[hh][2] += o.z;
+          c[hh][3] += o.w;
+        }
+    }
+    // lane (grp, tig) holds rows r0 (c0, c1) and r1 (c2, c3), tokens 8 hh + 2 tig and 8 hh + 2 tig + 1
+#pragma unroll
+    for (int e = 0; e < 4 * kH; ++e) {
+      const int64_t n = (e & 3) < 2 ? r0 : r1;
+      const int m = (e >> 2) * kGmTokens + 2 * tig + (e & 1);
+      if (((e & 3) < 2 ? ok0 : ok1) && m < M) {
+        const int v = c[e >> 2][e & 3] - asum[m];
         if (acc_out != nullptr) acc_out[static_cast<int64_t>(m) * N + n] = v;
         if (y != nullptr) {
           const float cs =

@@ -206,13 +206,15 @@ def test_gemm_simt_parity(M, afmt, wfmt):
     assert bf16_rows_rel_err(y, ex) <= BF16_ROW_TOL
 
 
-# 2-bit weights x int8 activations on the tensor cores for M > 8 (weights
-# widened into tensor memory; tokens on the MMA's N side: a multiple of 16 up
-# to 256 per token block; 8 for M = 8 with rows too long for the GEMV's
-# staged activations).  The M = 8 cases with shorter rows run on the warp-MMA
-# GEMV.
+# 2-bit weights x int8 activations on the tensor cores beyond the decode GEMVs
+# (more than 16 tokens, or rows too long to stage the GEMV's token slots):
+# weights widened into tensor memory, tokens on the MMA's N side (8 for M = 8,
+# else a multiple of 16 up to 256 per token block).  The cases with up to 16
+# tokens and shorter rows run on the warp-MMA GEMV.
 GEMM_T2TC_CASES = [
-    ("M8_long_K_20480_tc", 8, 136, 20480),
+    ("M8_long_K_24576_tc", 8, 136, 24576),
+    ("M12_long_K_12288_tc", 12, 136, 12288),
+    ("M16_long_K_11328_tc", 16, 300, 11328),
     ("M8_min_K", 8, 128, 64),
     ("M8_ragged_N_K_tail", 8, 300, 320),
     ("M8_two_tiles", 8, 256, 4096),
@@ -324,11 +326,12 @@ def test_gemm_fp4_end_to_end_alpha_groups():
     assert bf16_rows_rel_err(host(y, np.uint16), ex) <= BF16_ROW_TOL
 
 
-# up to 8 tokens against 2-bit weights: the CUDA-core GEMV.  Rows of 4096
-# codes are split over warps (K = 11008: 3 rounds; K = 36864: 9 rounds, one
-# warp per row group), so the shapes cover one and many rounds, a ragged last
-# round, and N that fills no CTA; 8 token slots x K = 36864 exceeds the staged
-# activation limit and takes the tiled CUDA-core kernel instead.
+# up to 16 tokens against 2-bit weights: the decode GEMVs (dp4a for 1-2 tokens,
+# warp-level MMA with 8 or 16 token slots for 3-16).  Rows are split over warps
+# (K = 11008: 3 rounds / 11 batches; K = 36864: 9 rounds), so the shapes cover
+# one and many rounds, a ragged last round, and N that fills no CTA; token slots
+# x K = 36864 beyond the staged-activation limit take the tiled CUDA-core
+# kernel or, for INT8 activations and more than 8 tokens, the tensor cores.
 GEMV_SHAPES = [(1, 64), (7, 320), (130, 4096), (258, 4160), (37, 11008), (96, 640), (40, 36864)]
 
 
@@ -347,7 +350,7 @@ def gemv_inputs(g, afmt, M, K):
             (scale.astype(np.float64) / 2).astype(np.float32))
 
 
-@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 9, 16])
 @pytest.mark.parametrize("afmt", ["i8", "i4", "e2m1"])
 @pytest.mark.parametrize("N,K", GEMV_SHAPES)
 def test_gemv_t2_parity(M, afmt, N, K):
@@ -364,7 +367,7 @@ def test_gemv_t2_parity(M, afmt, N, K):
 
 # the largest sums the GEMV meets: every activation -128 against rows of all
 # +1, all -1, all 0 and random signs, at the longest K it takes
-@pytest.mark.parametrize("M,K", [(1, 65536), (2, 65536), (4, 32768), (8, 16384), (1, 16384), (3, 18432)])
+@pytest.mark.parametrize("M,K", [(1, 65536), (2, 65536), (4, 32768), (8, 16384), (1, 16384), (3, 18432), (16, 11264)])
 def test_gemv_t2_extreme_sums(M, K):
     N = 12
     g = synth.rng(M + K)
