@@ -374,6 +374,46 @@ bl_status launch_gemv(const uint8_t* A, const float* a_scale, const uint8_t* W, 
   }
 }
 
+// Streaming GEMV (1-2 tokens): one CTA per SM, at least two 32-row stages of
+// K / 4 bytes per row in its shared-memory ring next to the staged activations.
+constexpr size_t kGsSmemBudget = 200 * 1024;
+
+int gs_stages(int64_t M, int64_t K) {
+  const int64_t stage = 32 * (K / 4);
+  const int64_t st = (static_cast<int64_t>(kGsSmemBudget) - M * K) / stage;
+  return static_cast<int>(st > bl::kGsMaxStages ? bl::kGsMaxStages : st);
+}
+// Measured: it beats the dp4a GEMV when every CTA's rows fit one stage (the
+// 7B O and Down shapes); with several stages per CTA the dp4a GEMV's 24 warps
+// per SM win, so it is used only then.
+bool gs_applies(int64_t M, int64_t N, int64_t K) {
+  const int64_t groups_per_cta = ((N + 3) / 4 + sm_count() - 1) / sm_count();
+  return M >= 1 && M <= 2 && gs_stages(M, K) >= 2 && groups_per_cta <= bl::kGsConsumers;
+}
+
+template <int AF, int MT>
+bl_status launch_gemv_stream(const uint8_t* A, const float* a_scale, const uint8_t* W, const float* alpha,
+                             int64_t alpha_group, int m, int n, int k, uint16_t* Y, int64_t ldy, int32_t* acc_out,
+                             cudaStream_t s) {
+  static size_t attr_set[kMaxDevices] = {};
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return BL_ERR_CUDA;
+  const int stages = gs_stages(MT, k);
+  const size_t smem = static_cast<size_t>(stages) * 32 * static_cast<size_t>(k / 4) + static_cast<size_t>(MT) * k;
+  if (smem > attr_set[d]) {
+    if (!cuda_ok(cudaFuncSetAttribute(bl::gemv_stream_t2_kernel<AF, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(smem))))
+      return BL_ERR_CUDA;
+    attr_set[d] = smem;
+  }
+  const int64_t groups = (static_cast<int64_t>(n) + 3) / 4;
+  const int64_t sms = sm_count();
+  const unsigned grid = static_cast<unsigned>(groups < sms ? groups : sms);
+  launch_pdl(bl::gemv_stream_t2_kernel<AF, MT>, grid, bl::kGsThreads, smem, s, A, a_scale, W, alpha, alpha_group, m, n,
+             k, stages, Y, ldy, acc_out);
+  return launch_status();
+}
+
 // The decode GEMVs apply to 2-bit weights and up to max_tokens tokens (16; 8
 // when they quantize bf16 rows themselves): the warp-MMA kernel from 3 tokens,
 // the dp4a kernel otherwise (and for rows too long to stage 8 or 16 slots).
@@ -387,6 +427,12 @@ template <int AF>
 bl_status launch_gemv_any(const uint8_t* A, const float* a_scale, const uint8_t* W, const float* alpha,
                           int64_t alpha_group, int m, int n, int k, uint16_t* Y, int64_t ldy, int32_t* acc_out,
                           cudaStream_t s, int64_t ldx = 0, float eps = 0.f) {
+  if constexpr (!bl::gv_fused<AF>()) {
+    if (gs_applies(m, n, k)) {
+      if (m == 1) return launch_gemv_stream<AF, 1>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+      return launch_gemv_stream<AF, 2>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s);
+    }
+  }
   if (gm_applies(m, k)) {
     if (m <= 8) return launch_gemv_mma<AF, 8>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s, ldx, eps);
     if constexpr (!bl::gv_fused<AF>())

@@ -15,7 +15,9 @@
 //                     isolated per byte field, dp4a against transposed
 //                     activations in shared memory (long rows).
 // gemv_mma_t2_kernel -- the same offset codes fed to warp-level integer MMA
-//                     (16 weight rows x 8 token slots per instruction).
+//                     (16 weight rows x 8 or 16 token slots per instruction).
+// gemv_stream_t2_kernel -- 1-2 tokens, the CTA's contiguous weight range
+//                     streamed through shared memory by 1-D bulk copies.
 // gemm_simt_kernel -- CUDA-core kernel that reads packed operands directly
 //                     (2-bit ternary weights, INT4 / E2M1 nibbles); decode of
 //                     3 to 7 tokens and the packed activation formats.
@@ -1649,6 +1651,229 @@ __global__ void __launch_bounds__(kGvMaxThreads) gemv_mma_t2_kernel(const uint8_
           y[static_cast<int64_t>(m) * ldy + n] = *reinterpret_cast<const uint16_t*>(&bb);
         }
       }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// gemv_stream_t2_kernel -- 1 or 2 tokens against 2-bit ternary weights, the
+// weights streamed.  One CTA per SM owns a contiguous run of whole 4-row
+// groups, i.e. one contiguous byte range of the packed matrix.  Before its wait
+// the CTA asks L2 for the whole range; after it, one thread moves the range
+// through a ring of shared-memory stages (32 rows each) with 1-D bulk copies
+// that complete on mbarriers, so the copy engine keeps the CTA's bytes in
+// flight with no registers tied up.  Eight consumer warps take 4 rows of each
+// stage and compute as gemv_t2_kernel does (offset codes, dp4a against the
+// field-major activations staged once per CTA), reading the weights from
+// shared memory.  Every wait is bounded.
+// ---------------------------------------------------------------------------
+constexpr int kGsConsumers = 8;                            // consumer warps; the last warp copies
+constexpr int kGsThreads = (kGsConsumers + 1) * 32;
+constexpr int kGsStageRows = kGsConsumers * 4;             // 32 rows per stage
+constexpr int kGsMaxStages = 4;
+
+template <int AF, int MT>
+__global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_t2_kernel(const uint8_t* __restrict__ a,
+                                                                      const float* __restrict__ a_scale,
+                                                                      const uint8_t* __restrict__ w,
+                                                                      const float* __restrict__ alpha,
+                                                                      int64_t alpha_group, int M, int N, int K,
+                                                                      int stages, uint16_t* __restrict__ y,
+                                                                      int64_t ldy, int32_t* __restrict__ acc_out) {
+  constexpr int R = 4;
+  extern __shared__ __align__(128) uint8_t gs_smem[];
+  __shared__ __align__(8) uint64_t full[kGsMaxStages];
+  __shared__ __align__(8) uint64_t empty[kGsMaxStages];
+  __shared__ int asum[MT];
+  __shared__ float s_scale[MT];
+  __shared__ double red[kGvMaxWarps][MT];
+  __shared__ int s_abort;
+  const int kw16 = K >> 4;
+  const int kq = kw16 >> 2;
+  const uint32_t rowbytes = static_cast<uint32_t>(K >> 2);
+  const uint32_t stage_bytes = kGsStageRows * rowbytes;
+  uint8_t* ring = gs_smem;
+  uint4* act = reinterpret_cast<uint4*>(gs_smem + static_cast<size_t>(stages) * stage_bytes);   // [MT][4][kq]
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const bool producer = warp == kGsConsumers;
+
+  // this CTA's 4-row groups [g0, g1): rows [4 g0, min(4 g1, N)), contiguous bytes
+  const int64_t groups = (static_cast<int64_t>(N) + 3) / 4;
+  const int64_t g0 = groups * blockIdx.x / gridDim.x;
+  const int64_t g1 = groups * (blockIdx.x + 1) / gridDim.x;
+  const int64_t row0 = 4 * g0;
+  const int64_t row_end = min(4 * g1, static_cast<int64_t>(N));
+  const int nstage = static_cast<int>((g1 - g0 + kGsConsumers - 1) / kGsConsumers);
+  auto stage_rows = [&](int i) {
+    const int64_t r = row0 + static_cast<int64_t>(i) * kGsStageRows;
+    return static_cast<uint32_t>(min(static_cast<int64_t>(kGsStageRows), row_end - r));
+  };
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < stages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], kGsConsumers);
+    }
+    fence_mbarrier_init();
+    s_abort = 0;
+  }
+  if (threadIdx.x < MT) asum[threadIdx.x] = 0;
+  if (producer && lane == 0 && row_end > row0)
+    bulk_prefetch_l2(w + row0 * rowbytes, static_cast<uint32_t>(row_end - row0) * rowbytes);
+  __syncthreads();
+  pdl_wait();
+  pdl_trigger();
+
+  // the first stages go out before the activations are staged
+  if (producer && lane == 0) {
+    for (int i = 0; i < nstage && i < stages; ++i) {
+      const uint32_t bytes = stage_rows(i) * rowbytes;
+      mbar_arrive_expect_tx(&full[i], bytes);
+      bulk_load_1d(ring + static_cast<size_t>(i) * stage_bytes, w + (row0 + static_cast<int64_t>(i) * kGsStageRows) * rowbytes,
+                   bytes, &full[i]);
+    }
+  }
+  gv_stage<AF, MT>(a, 0, 0.f, M, K, act, [kq](int q, int m) { return (m * 4 + (q & 3)) * kq + (q >> 2); }, asum,
+                   red, s_scale);
+  __syncthreads();
+
+  if (producer) {
+    if (lane == 0) {
+      for (int i = stages; i < nstage; ++i) {
+        const int st = i % stages;
+        if (!mbar_wait_bounded(&empty[st], static_cast<uint32_t>((i / stages - 1) & 1))) {
+          s_abort = 1;
+          break;
+        }
+        const uint32_t bytes = stage_rows(i) * rowbytes;
+        mbar_arrive_expect_tx(&full[st], bytes);
+        bulk_load_1d(ring + static_cast<size_t>(st) * stage_bytes, w + (row0 + static_cast<int64_t>(i) * kGsStageRows) * rowbytes,
+                     bytes, &full[st]);
+      }
+    }
+  } else {
+    const float unit_scale = (AF == kSimtA_E2M1) ? 0.5f : 1.0f;
+    const int rounds = (kw16 + 255) >> 8;
+    for (int i = 0; i < nstage; ++i) {
+      const int st = i % stages;
+      if (!mbar_wait_bounded(&full[st], static_cast<uint32_t>((i / stages) & 1))) {
+        s_abort = 1;
+        break;
+      }
+      const int64_t n0 = row0 + static_cast<int64_t>(i) * kGsStageRows + warp * R;
+      const bool rows_ok = n0 < row_end;
+      const uint8_t* sw = ring + static_cast<size_t>(st) * stage_bytes + static_cast<size_t>(warp * R) * rowbytes;
+      int tot[R][MT];
+      if constexpr (MT == 1) {
+        int acc[R][4];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[r][j] = 0;
+        for (int rd = 0; rd < rounds; ++rd) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int wq = rd * 256 + h * 128 + 4 * lane;
+            if (!rows_ok || wq >= kw16) continue;
+            uint4 wv[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+              wv[r] = n0 + r < row_end ? *reinterpret_cast<const uint4*>(sw + r * rowbytes + wq * 4)
+                                       : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint4 av = act[j * kq + (wq >> 2)];
+#pragma unroll
+              for (int r = 0; r < R; ++r) {
+                const uint32_t x = j == 0 ? wv[r].x : (j == 1 ? wv[r].y : (j == 2 ? wv[r].z : wv[r].w));
+                const uint32_t u = ~x & (0x55555555u | (x << 1));
+                acc[r][0] = dp4a_us(u & 0x03030303u, av.x, acc[r][0]);
+                acc[r][1] = dp4a_us(u & 0x0C0C0C0Cu, av.y, acc[r][1]);
+                acc[r][2] = dp4a_us(u & 0x30303030u, av.z, acc[r][2]);
+                acc[r][3] = dp4a_us(u & 0xC0C0C0C0u, av.w, acc[r][3]);
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);   // this warp is done with the stage
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+          tot[r][0] =
+              __reduce_add_sync(0xFFFFFFFFu, acc[r][0] + (acc[r][1] >> 2) + (acc[r][2] >> 4) + (acc[r][3] >> 6));
+      } else {
+        int acc[R][MT];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int m = 0; m < MT; ++m) acc[r][m] = 0;
+        for (int rd = 0; rd < rounds; ++rd) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int wq = rd * 256 + h * 128 + 4 * lane;
+            if (!rows_ok || wq >= kw16) continue;
+            uint4 wv[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+              wv[r] = n0 + r < row_end ? *reinterpret_cast<const uint4*>(sw + r * rowbytes + wq * 4)
+                                       : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint32_t f[R][4];
+#pragma unroll
+              for (int r = 0; r < R; ++r) {
+                const uint32_t x = j == 0 ? wv[r].x : (j == 1 ? wv[r].y : (j == 2 ? wv[r].z : wv[r].w));
+                const uint32_t u = ~x & (0x55555555u | (x << 1));
+                f[r][0] = u & 0x03030303u;
+                f[r][1] = (u >> 2) & 0x03030303u;
+                f[r][2] = (u >> 4) & 0x03030303u;
+                f[r][3] = (u >> 6) & 0x03030303u;
+              }
+#pragma unroll
+              for (int m = 0; m < MT; ++m) {
+                const uint4 av = act[(m * 4 + j) * kq + (wq >> 2)];
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                  int t = dp4a_us(f[r][0], av.x, acc[r][m]);
+                  t = dp4a_us(f[r][1], av.y, t);
+                  t = dp4a_us(f[r][2], av.z, t);
+                  acc[r][m] = dp4a_us(f[r][3], av.w, t);
+                }
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int m = 0; m < MT; ++m) tot[r][m] = __reduce_add_sync(0xFFFFFFFFu, acc[r][m]);
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const int64_t n = n0 + r;
+          if (lane == r * MT + m && n < row_end && m < M) {
+            const int v = tot[r][m] - asum[m];
+            if (acc_out != nullptr) acc_out[static_cast<int64_t>(m) * N + n] = v;
+            if (y != nullptr) {
+              const float cs =
+                  __fmul_rn(__fmul_rn(ld_dep_f32(a_scale + m), unit_scale), ld_dep_f32(alpha + n / alpha_group));
+              const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__int2float_rn(v), cs));
+              y[static_cast<int64_t>(m) * ldy + n] = *reinterpret_cast<const uint16_t*>(&b);
+            }
+          }
+        }
+    }
+  }
+  __syncthreads();
+  if (s_abort) {
+    // let any copies still in flight land before the CTA's memory goes away
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) {
     }
   }
 }

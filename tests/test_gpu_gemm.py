@@ -332,7 +332,10 @@ def test_gemm_fp4_end_to_end_alpha_groups():
 # one and many rounds, a ragged last round, and N that fills no CTA; token slots
 # x K = 36864 beyond the staged-activation limit take the tiled CUDA-core
 # kernel or, for INT8 activations and more than 8 tokens, the tensor cores.
-GEMV_SHAPES = [(1, 64), (7, 320), (130, 4096), (258, 4160), (37, 11008), (96, 640), (40, 36864)]
+# For 1-2 tokens, rows up to K = 11328 and at most 32 rows per SM the
+# streaming GEMV runs (every shape here with N <= 4736).
+GEMV_SHAPES = [(1, 64), (7, 320), (130, 4096), (258, 4160), (37, 11008), (96, 640), (40, 36864), (4736, 640),
+               (23680, 640)]
 
 
 def gemv_inputs(g, afmt, M, K):
