@@ -57,6 +57,9 @@ def _load():
         sigs = {
             "orc_quant_int4": [P, I64, I64, I64, F, P, P, P],
             "orc_quant_fp4": [P, I64, I64, I64, P, P, P, P],
+            "orc_quant_int4_absmax": [P, I64, I64, I64, F, P, P, P],
+            "orc_quant_int4_absmean2": [P, I64, I64, I64, F, P, P, P],
+            "orc_quant_fp4_e1m2": [P, I64, I64, I64, P, P, P, P],
             "orc_sparsify_a8": [P, I64, I64, I64, I64, F, P, P, P, P],
             "orc_relu2_glu": [P, P, I64, I64, I64, I64, F, P, P, P, P, P],
             "orc_ternary_abs_bins": [P, I64, I64, I64, P],
@@ -120,6 +123,48 @@ def quant_fp4(x_bf16: np.ndarray):
     _check(_load().orc_quant_fp4(_ptr(x), M, K, K, _ptr(code4), _ptr(tv), _ptr(p), _ptr(scale)),
            "quant_fp4")
     return code4, tv, p, scale
+
+
+def quant_int4_absmax(x_bf16: np.ndarray, eps: float = EPS):
+    """INT4 absmax per token (the Fig. 6 ablation; reading: Eq. 1's absmax with
+    the 4-bit range).  Returns (codes int8 [M,K], gamma fp32 [M], scale =
+    gamma/7 fp32 [M])."""
+    x = _bf16_2d(x_bf16)
+    M, K = x.shape
+    codes = np.empty((M, K), np.int8)
+    gamma = np.empty(M, np.float32)
+    scale = np.empty(M, np.float32)
+    _check(_load().orc_quant_int4_absmax(_ptr(x), M, K, K, eps, _ptr(codes), _ptr(gamma), _ptr(scale)),
+           "quant_int4_absmax")
+    return codes, gamma, scale
+
+
+def quant_int4_absmean2(x_bf16: np.ndarray, eps: float = EPS):
+    """INT4 absmean with beta = 2 mean|x| per token (the Fig. 5 ablation).
+    Returns (codes int8 [M,K], beta fp32 [M], scale = beta/sqrt7 fp32 [M])."""
+    x = _bf16_2d(x_bf16)
+    M, K = x.shape
+    codes = np.empty((M, K), np.int8)
+    beta = np.empty(M, np.float32)
+    scale = np.empty(M, np.float32)
+    _check(_load().orc_quant_int4_absmean2(_ptr(x), M, K, K, eps, _ptr(codes), _ptr(beta), _ptr(scale)),
+           "quant_int4_absmean2")
+    return codes, beta, scale
+
+
+def quant_fp4_e1m2(x_bf16: np.ndarray):
+    """FP4 E1M2 MinMax per token (the Fig. 6 ablation; reading: magnitudes
+    {0,.25,...,1.75}, scale 2^p with max|x| <= 1.75*2^p).  Returns (code4 uint8
+    [M,K], four_value int8 [M,K], p int32 [M], scale = 2^p fp32 [M])."""
+    x = _bf16_2d(x_bf16)
+    M, K = x.shape
+    code4 = np.empty((M, K), np.uint8)
+    fv = np.empty((M, K), np.int8)
+    p = np.empty(M, np.int32)
+    scale = np.empty(M, np.float32)
+    _check(_load().orc_quant_fp4_e1m2(_ptr(x), M, K, K, _ptr(code4), _ptr(fv), _ptr(p), _ptr(scale)),
+           "quant_fp4_e1m2")
+    return code4, fv, p, scale
 
 
 def sparsify_a8(x_bf16: np.ndarray, keep: int, eps: float = EPS):

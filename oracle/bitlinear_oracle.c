@@ -172,6 +172,111 @@ int orc_quant_fp4(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
 }
 
 /* ---------------------------------------------------------------------------
+ * Quantizer variants of the ablation figures (Fig. 5: INT4 absmean with
+ * beta = 2 mean(|X|); Fig. 6: INT4 absmax and FP4 E1M2 beside INT4 absmean and
+ * FP4 E2M1).  The pages name them without formulas; the readings used:
+ *   INT4 absmax:   Q(X) = gamma/7 * RoundClip(7/(gamma+eps) * X, -8, 7),
+ *                  gamma = max|X| per token -- the absmax quantizer of Eq. 1
+ *                  with the 4-bit range (7 = 2^(4-1) - 1).
+ *   INT4 absmean, beta = 2 mean(|X|):  Eq. 6-7 with that beta.
+ *   FP4 E1M2:      1 exponent bit (bias 1, no inf/nan) and 2 mantissa bits,
+ *                  magnitudes {0, .25, .5, .75, 1, 1.25, 1.5, 1.75}; a per-token
+ *                  power-of-two scale 2^p, p the smallest integer with
+ *                  max|x| <= 1.75 * 2^p (the MinMax reading of the E2M1 case);
+ *                  x / 2^p rounded to the nearest magnitude, ties to the even
+ *                  encoding; code = sign bit 3 + magnitude index bits 0..2.
+ * ------------------------------------------------------------------------- */
+int orc_quant_int4_absmax(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float eps,
+                          int8_t* codes, float* gamma_out, float* scale_out) {
+    if (M < 0 || K <= 0 || ldx < K) return ORC_ERR_ARG;
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t* row = x + m * ldx;
+        float gamma = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float a = fabsf(bf16_value(row[k]));
+            if (!isfinite(a)) return ORC_ERR_NONFINITE;
+            if (a > gamma) gamma = a;
+        }
+        float mult = 7.0f / (gamma + eps);
+        for (int64_t k = 0; k < K; ++k) {
+            float v = bf16_value(row[k]) * mult;
+            codes[m * K + k] = (int8_t)round_clip(v, -8.0f, 7.0f);
+        }
+        gamma_out[m] = gamma;
+        scale_out[m] = gamma / 7.0f;
+    }
+    return ORC_OK;
+}
+
+int orc_quant_int4_absmean2(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float eps,
+                            int8_t* codes, float* beta_out, float* scale_out) {
+    if (M < 0 || K <= 0 || ldx < K) return ORC_ERR_ARG;
+    const float sqrt7 = (float)sqrt(7.0);
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t* row = x + m * ldx;
+        double s;
+        int rc = exact_abs_sum_bf16(row, K, &s);
+        if (rc) return rc;
+        float beta = (float)((2.0 * s) / (double)K);   /* beta = 2 mean|x| */
+        float mult = sqrt7 / (beta + eps);
+        for (int64_t k = 0; k < K; ++k) {
+            float v = bf16_value(row[k]) * mult;
+            codes[m * K + k] = (int8_t)round_clip(v, -8.0f, 7.0f);
+        }
+        beta_out[m] = beta;
+        scale_out[m] = beta / sqrt7;
+    }
+    return ORC_OK;
+}
+
+static const double e1m2_grid[8] = {0.0, 0.25, 0.5, 0.75, 1.0, 1.25, 1.5, 1.75};
+
+static int e1m2_nearest_index(double mag) {
+    /* nearest magnitude; an exact tie goes to the even index (mantissa bit 0) */
+    int best = 0;
+    double best_d = fabs(mag - e1m2_grid[0]);
+    for (int i = 1; i < 8; ++i) {
+        double d = fabs(mag - e1m2_grid[i]);
+        if (d < best_d || (d == best_d && (i % 2 == 0) && (best % 2 == 1))) {
+            best = i;
+            best_d = d;
+        }
+    }
+    return best;
+}
+
+/* Outputs: the 4-bit code, four times the value (an exact integer in [-7, 7]),
+ * p per row and the dequant scale 2^p of the code's value. */
+int orc_quant_fp4_e1m2(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                       uint8_t* code4, int8_t* four_value, int32_t* p_out, float* scale_out) {
+    if (M < 0 || K <= 0 || ldx < K) return ORC_ERR_ARG;
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t* row = x + m * ldx;
+        double g = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double a = fabs((double)bf16_value(row[k]));
+            if (!isfinite(a)) return ORC_ERR_NONFINITE;
+            if (a > g) g = a;
+        }
+        int p = 0;
+        if (g > 0.0) {
+            while (g > 1.75 * ldexp(1.0, p)) ++p;
+            while (g <= 1.75 * ldexp(1.0, p - 1)) --p;
+        }
+        for (int64_t k = 0; k < K; ++k) {
+            double v = (double)bf16_value(row[k]) * ldexp(1.0, -p);   /* exact */
+            int idx = e1m2_nearest_index(fabs(v));
+            int neg = (v < 0.0) && idx != 0;
+            code4[m * K + k] = (uint8_t)((neg ? 8 : 0) | idx);
+            four_value[m * K + k] = (int8_t)(neg ? -idx : idx);
+        }
+        p_out[m] = p;
+        scale_out[m] = (float)ldexp(1.0, p);
+    }
+    return ORC_OK;
+}
+
+/* ---------------------------------------------------------------------------
  * Top-K mask (§3.4 "Sparsification Pipeline", Eq. 1: M = Top_k(|X|)).
  * Exactly `keep` survivors per row; the ranking key is (|x| descending,
  * index ascending), so ties at the threshold go to the lower index.

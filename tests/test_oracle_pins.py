@@ -393,3 +393,112 @@ def test_pack_layouts():
     m = np.zeros((1, 40), np.uint8)
     m[0, [0, 31, 32, 39]] = 1
     assert oracle.pack_mask_bits(m).tolist() == [[0x80000001, 0x81]]
+
+
+# ----------------------------------------------------------------------------
+# Quantizer variants of the ablations (Fig. 5 / Fig. 6), as flags
+# ----------------------------------------------------------------------------
+def test_int4_absmax_hand_examples():
+    # gamma = max|x| = 4: mult = 7/(4+eps) = 1.7499956 -> 0.175, -0.350, 6.99998,
+    # 0.526 -> [0, 0, 7, 1] (the bf16 values of 0.1, -0.2, 0.3 are 0.10009766,
+    # -0.20019531, 0.30078125); scale = 4/7
+    codes, gamma, scale = oracle.quant_int4_absmax(bf16([[0.1, -0.2, 4.0, 0.3]]))
+    assert codes[0].tolist() == [0, 0, 7, 1]
+    assert gamma[0] == 4.0
+    assert scale[0] == np.float32(np.float32(4.0) / np.float32(7.0))
+    # gamma = 7: mult ~ 1 - 1.4e-6 -> the integers themselves
+    codes, gamma, scale = oracle.quant_int4_absmax(bf16([[1.0, -2.0, 3.0, -7.0]]))
+    assert codes[0].tolist() == [1, -2, 3, -7]
+    assert scale[0] == 1.0
+
+
+def test_int4_absmax_max_element_maps_to_7():
+    # the largest magnitude always lands on +-7 (7*g/(g+eps) rounds to 7 for g >> eps)
+    x = synth.gaussian_bf16(synth.rng(21), (6, 256))
+    codes, gamma, _ = oracle.quant_int4_absmax(x)
+    xf = bf16_val(x)
+    for m in range(6):
+        k = int(np.argmax(np.abs(xf[m])))
+        assert abs(int(codes[m, k])) == 7
+        assert gamma[m] == np.float32(np.abs(xf[m]).max())
+    assert codes.min() >= -7 and codes.max() <= 7
+
+
+def test_int4_absmax_brute_force_nearest_code():
+    x = synth.gaussian_bf16(synth.rng(22), (4, 96), outlier_channels=(7,), outlier_scale=9.0)
+    codes, gamma, _ = oracle.quant_int4_absmax(x)
+    xf = bf16_val(x).astype(np.float32)
+    for m in range(x.shape[0]):
+        mult = np.float32(np.float32(7.0) / (np.float32(gamma[m]) + np.float32(EPS)))
+        for k in range(x.shape[1]):
+            v = float(np.float32(xf[m, k] * mult))
+            best = min(range(-8, 8), key=lambda c: (abs(v - c), c % 2))
+            assert codes[m, k] == best
+
+
+def test_int4_absmean2_hand_example_and_relation():
+    # mean|x| = 2.5 -> beta = 5; mult = sqrt7/(5+eps) = 0.52915 -> 0.529, -1.058,
+    # 1.587, -2.117 -> [1, -1, 2, -2]; scale = 5/sqrt7
+    codes, beta, scale = oracle.quant_int4_absmean2(bf16([[1.0, -2.0, 3.0, -4.0]]))
+    assert codes[0].tolist() == [1, -1, 2, -2]
+    assert beta[0] == 5.0
+    assert scale[0] == np.float32(np.float32(5.0) / np.float32(math.sqrt(7)))
+    # beta is twice the absmean beta of the same row, which is twice the absmean
+    # beta of the halved row (halving bf16 values is exact)
+    x = synth.gaussian_bf16(synth.rng(23), (5, 512))
+    c2, b2, _ = oracle.quant_int4_absmean2(x, 0.0)
+    _, b1, _ = oracle.quant_int4(x, 0.0)
+    _, bh, _ = oracle.quant_int4(synth.f32_to_bf16_bits(bf16_val(x) / 2), 0.0)
+    assert np.array_equal(b2, 2 * b1) and np.array_equal(b2, 4 * bh)
+    # each code is the nearest INT4 value to x*sqrt7/(beta+eps), ties to even (brute force)
+    xf = bf16_val(x).astype(np.float32)
+    for m in range(2):
+        mult = np.float32(np.float32(math.sqrt(7)) / (np.float32(b2[m]) + np.float32(0.0)))
+        for k in range(64):
+            v = float(np.float32(xf[m, k] * mult))
+            assert c2[m, k] == min(range(-8, 8), key=lambda c: (abs(v - c), c % 2))
+
+
+def test_fp4_e1m2_hand_examples():
+    # max|x| = 5 = 1.25 * 2^2 -> p = 2; x/4 = 0.0752, -0.3008, 1.25, 0.0175 ->
+    # nearest of {0,.25,...,1.75}: indices 0, 1 (negative), 5, 0
+    code4, fv, p, scale = oracle.quant_fp4_e1m2(bf16([[0.3, -1.2, 5.0, 0.07]]))
+    assert p[0] == 2 and scale[0] == 4.0
+    assert code4[0].tolist() == [0, 8 | 1, 5, 0]
+    assert fv[0].tolist() == [0, -1, 5, 0]
+    # ties to the even encoding: 0.125 (between 0 and .25) -> 0, 0.375 -> .5,
+    # -0.625 (between .5 and .75) -> -.5; max 1.75 -> p = 0
+    code4, fv, p, _ = oracle.quant_fp4_e1m2(bf16([[0.125, 0.375, 1.75, -0.625]]))
+    assert p[0] == 0
+    assert code4[0].tolist() == [0, 2, 7, 8 | 2]
+    assert fv[0].tolist() == [0, 2, 7, -2]
+
+
+@pytest.mark.parametrize("gmax,p", [(1.75, 0), (1.765625, 1), (0.875, -1), (3.5, 1), (3.515625, 2),
+                                    (1.0, 0), (1e-3, -10)])
+def test_fp4_e1m2_scale_exponent_closed_form(gmax, p):
+    row = bf16([[gmax, -gmax / 4, 0.0, gmax / 3]])
+    g = float(bf16_val(row)[0, 0])
+    _, _, pp, scale = oracle.quant_fp4_e1m2(row)
+    assert pp[0] == p
+    assert g <= 1.75 * 2.0 ** p and g > 1.75 * 2.0 ** (p - 1)
+    assert scale[0] == np.float32(2.0 ** p)
+
+
+def test_fp4_e1m2_exhaustive_bf16_is_rint_of_4x():
+    # On the uniform 0.25 grid, nearest-with-ties-to-even-index is rint(4|x|):
+    # every finite bf16 magnitude up to 1.75 at p = 0
+    bits = np.arange(0, 0x8000, dtype=np.uint16)
+    vals = bf16_val(bits)
+    keep = np.isfinite(vals) & (vals <= 1.75)
+    bits = bits[keep]
+    for sign in (0, 0x8000):
+        b = (bits | sign).astype(np.uint16)
+        row = np.concatenate([b, bf16([1.75])]).reshape(1, -1)
+        code4, fv, p, _ = oracle.quant_fp4_e1m2(row)
+        assert p[0] == 0
+        v = bf16_val(b).astype(np.float64)
+        idx = np.rint(4 * np.abs(v)).astype(np.int64)
+        neg = (v < 0) & (idx != 0)
+        assert np.array_equal(fv[0, :-1].astype(np.int64), np.where(neg, -idx, idx))
+        assert np.array_equal(code4[0, :-1].astype(np.int64), idx | np.where(neg, 8, 0))
