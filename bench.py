@@ -598,6 +598,51 @@ def decode_gemm_kernel(m: int) -> str:
     return "tcgen05 (2-bit weights widened into TMEM)"
 
 
+def run_quant_variants(args):
+    """The 4-bit activation quantizer with each bl_quant variant (INT4 absmean,
+    FP4 E2M1, and the ablation variants INT4 absmax, INT4 absmean with beta =
+    2 mean|x|, FP4 E1M2) on the 7B QKV input, M = 32768 x K = 4096 bf16 (268 MB,
+    larger than L2), byte-layout codes; CUDA events around each launch."""
+    import torch
+
+    import ternary_bit_activation_b200 as tba
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    s = SHAPE
+    m, k = s.tokens, s.hidden
+    x = torch.from_numpy(synth.gaussian_bf16(synth.rng(500), (m, k)).view(np.int16)).to(dev)   # Gaussian QKV input
+    codes = torch.empty((m, k), dtype=torch.int8, device=dev)
+    scale = torch.empty((m,), dtype=torch.float32, device=dev)
+    peaks = load_peaks()
+    nbytes = m * (2 * k + k + 4)
+    variants = [("int4_absmean", tba.BL_QUANT_INT4), ("fp4_e2m1", tba.BL_QUANT_FP4_E2M1),
+                ("int4_absmax", tba.BL_QUANT_INT4_ABSMAX), ("int4_absmean_2beta", tba.BL_QUANT_INT4_ABSMEAN2),
+                ("fp4_e1m2", tba.BL_QUANT_FP4_E1M2)]
+    results = []
+    for name, q in variants:
+        fn = lambda: tba.bitlinear_quant_a4(x, codes, scale, q, tba.BL_STORE_BYTES, EPS)
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record()
+            fn()
+            b_.record()
+            torch.cuda.synchronize()
+            ts.append(a_.elapsed_time(b_))
+        tba.sync_status()
+        ms = sorted(ts)[len(ts) // 2]
+        gbs = nbytes / (ms / 1e3) / 1e9
+        results.append({"variant": name, "us": round(ms * 1e3, 1), "gbs": round(gbs, 1),
+                        "hbm_frac": round(gbs / peaks["hbm_gbs"], 3)})
+    line = {"metric": "4-bit activation quantizer GB/s per variant (7B QKV input)", "unit": "GB/s",
+            "workload": f"X bf16 [{m} x {k}] -> int8 codes + fp32 scale per token (median of {args.steps} launches)",
+            "algorithmic_bytes": nbytes, "hbm_peak_gbs": peaks["hbm_gbs"], "results": results}
+    print(json.dumps(line), flush=True)
+
+
 def run_decode(args):
     import torch
 
@@ -833,8 +878,9 @@ def main(argv=None):
     ap.add_argument("--cpu-tokens", type=int, default=32, help="token sample of the CPU baseline")
     ap.add_argument("--cpu-tokens-ref", type=int, default=8, help="token sample per step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["prefill", "decode"], default="prefill",
-                    help="prefill: the headline step; decode: per-token-batch latency sweep")
+    ap.add_argument("--workload", choices=["prefill", "decode", "quant-variants"], default="prefill",
+                    help="prefill: the headline step; decode: per-token-batch latency sweep; "
+                         "quant-variants: the 4-bit quantizer and its ablation variants at the 7B prefill input")
     ap.add_argument("--decode-tokens", type=int, nargs="+", default=synth.DECODE_TOKENS)
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), help="run one kernel's small case and exit")
     ap.add_argument("--launches", type=int, default=3, help="launches of --profile-case")
@@ -848,6 +894,8 @@ def main(argv=None):
         run_reference(args)
     elif args.workload == "decode":
         run_decode(args)
+    elif args.workload == "quant-variants":
+        run_quant_variants(args)
     else:
         run_gpu(args)
 

@@ -52,7 +52,11 @@ typedef enum {
 /* Quantizer choice for the 4-bit activation path. */
 typedef enum {
     BL_QUANT_INT4 = 0,        /* absmean INT4, Eq. 6-7 */
-    BL_QUANT_FP4_E2M1 = 1     /* MinMax FP4 E2M1, Eq. 8-9 */
+    BL_QUANT_FP4_E2M1 = 1,    /* MinMax FP4 E2M1, Eq. 8-9 */
+    /* the ablation variants of Fig. 5 / Fig. 6 (formulas are readings, see bitlinear_quant_a4) */
+    BL_QUANT_INT4_ABSMAX = 2,   /* INT4 absmax */
+    BL_QUANT_INT4_ABSMEAN2 = 3, /* INT4 absmean with beta = 2 mean|x| */
+    BL_QUANT_FP4_E1M2 = 4       /* MinMax FP4 E1M2 */
 } bl_quant;
 
 /* How 4-bit codes are stored. */
@@ -90,9 +94,21 @@ typedef enum {
  *     x * 2^-p is rounded to the nearest E2M1 value {0,.5,1,1.5,2,3,4,6}, ties
  *     to the even encoding; codes are sign bit 3 + value bits 0-2, a zero
  *     magnitude is always +0.  scale[m] = 2^p.
+ *   Ablation variants (Fig. 5, Fig. 6; the pages give no formulas, readings):
+ *   BL_QUANT_INT4_ABSMAX: gamma = max|x|, mult = 7 / (gamma + eps),
+ *     code = RoundClip(x * mult, -8, 7), scale[m] = gamma / 7 (Eq. 1's absmax
+ *     quantizer with the 4-bit range).
+ *   BL_QUANT_INT4_ABSMEAN2: BL_QUANT_INT4 with beta = 2 mean|x|.
+ *   BL_QUANT_FP4_E1M2: magnitudes {0,.25,...,1.75} (1 exponent bit with bias 1,
+ *     2 mantissa bits); p = the smallest integer with max|x| <= 1.75 * 2^p;
+ *     nearest magnitude, ties to the even encoding; codes as for E2M1 (sign
+ *     bit 3 + magnitude index bits 0-2); scale[m] = 2^p.
  * Storage: BL_STORE_PACKED writes M x K/2 bytes; BL_STORE_BYTES writes M x K
- *   int8 (INT4: the code itself; FP4: 2 * value, an exact integer in [-12, 12],
- *   with scale[m] = 2^(p-1) so that value * 2^p = byte * scale).
+ *   int8 (INT4: the code itself; FP4 E2M1: 2 * value, an exact integer in
+ *   [-12, 12], with scale[m] = 2^(p-1) so that value * 2^p = byte * scale;
+ *   FP4 E1M2: 4 * value in [-7, 7] with scale[m] = 2^(p-2)).  The GEMM takes
+ *   the bytes of every variant as BL_A_I8, the packed INT4 variants as
+ *   BL_A_I4 and packed E2M1 as BL_A_E2M1.
  * x: [M x K] bf16 with row stride ldx.  codes: contiguous rows.  scale: [M] fp32.
  * Requires K % 8 == 0, 8 <= K <= 16384, ldx % 8 == 0, 16-byte aligned pointers.
  */

@@ -22,7 +22,7 @@ BL_OK = 0
 STATUS_NAMES = ["BL_OK", "BL_ERR_NULL", "BL_ERR_ALIGN", "BL_ERR_SHAPE", "BL_ERR_ARG", "BL_ERR_UNSUPPORTED",
                 "BL_ERR_CUDA", "BL_ERR_TIMEOUT", "BL_ERR_WORKSPACE"]
 BL_ERR_CUDA = STATUS_NAMES.index("BL_ERR_CUDA")
-BL_QUANT_INT4, BL_QUANT_FP4_E2M1 = 0, 1
+BL_QUANT_INT4, BL_QUANT_FP4_E2M1, BL_QUANT_INT4_ABSMAX, BL_QUANT_INT4_ABSMEAN2, BL_QUANT_FP4_E1M2 = 0, 1, 2, 3, 4
 BL_STORE_PACKED, BL_STORE_BYTES = 0, 1
 BL_A_I8, BL_A_I4, BL_A_E2M1 = 0, 1, 2
 BL_W_T2, BL_W_I8, BL_W_E2M1 = 0, 1, 2

@@ -19,6 +19,11 @@
 
 namespace {
 
+static_assert(BL_QUANT_INT4 == bl::kQInt4 && BL_QUANT_FP4_E2M1 == bl::kQFp4 &&
+                  BL_QUANT_INT4_ABSMAX == bl::kQInt4Absmax && BL_QUANT_INT4_ABSMEAN2 == bl::kQInt4Absmean2 &&
+                  BL_QUANT_FP4_E1M2 == bl::kQFp4E1M2,
+              "bl_quant values are the quantizer kernel's variant ids");
+
 constexpr int kMaxDevices = 64;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -159,17 +164,29 @@ bool tc_kernel_ready() {
 // ---------------------------------------------------------------------------
 // launch helpers
 // ---------------------------------------------------------------------------
+template <int C, int VAR>
+void launch_quant_a4_cv(const uint16_t* x, int64_t M, int K, int64_t ldx, bool packed, float eps, uint8_t* codes,
+                        float* scale, cudaStream_t s, dim3 grid) {
+  if (packed) launch_pdl(bl::quant_a4_kernel<C, VAR, true>, grid, 256, 0, s, x, M, K, ldx, eps, codes, scale);
+  else launch_pdl(bl::quant_a4_kernel<C, VAR, false>, grid, 256, 0, s, x, M, K, ldx, eps, codes, scale);
+}
+
 template <int C>
-void launch_quant_a4_c(const uint16_t* x, int64_t M, int K, int64_t ldx, bool fp4, bool packed, float eps,
+void launch_quant_a4_c(const uint16_t* x, int64_t M, int K, int64_t ldx, int var, bool packed, float eps,
                        uint8_t* codes, float* scale, cudaStream_t s) {
   // persistent: two rows per CTA and iteration, eight CTAs per SM
   const int64_t need = (M + 1) / 2;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   const dim3 grid(static_cast<unsigned>(need < cap ? need : cap));
-  if (!fp4 && packed) launch_pdl(bl::quant_a4_kernel<C, false, true>, grid, 256, 0, s, x, M, K, ldx, eps, codes, scale);
-  if (!fp4 && !packed) launch_pdl(bl::quant_a4_kernel<C, false, false>, grid, 256, 0, s, x, M, K, ldx, eps, codes, scale);
-  if (fp4 && packed) launch_pdl(bl::quant_a4_kernel<C, true, true>, grid, 256, 0, s, x, M, K, ldx, eps, codes, scale);
-  if (fp4 && !packed) launch_pdl(bl::quant_a4_kernel<C, true, false>, grid, 256, 0, s, x, M, K, ldx, eps, codes, scale);
+  switch (var) {
+    case bl::kQInt4: launch_quant_a4_cv<C, bl::kQInt4>(x, M, K, ldx, packed, eps, codes, scale, s, grid); break;
+    case bl::kQFp4: launch_quant_a4_cv<C, bl::kQFp4>(x, M, K, ldx, packed, eps, codes, scale, s, grid); break;
+    case bl::kQInt4Absmax: launch_quant_a4_cv<C, bl::kQInt4Absmax>(x, M, K, ldx, packed, eps, codes, scale, s, grid); break;
+    case bl::kQInt4Absmean2:
+      launch_quant_a4_cv<C, bl::kQInt4Absmean2>(x, M, K, ldx, packed, eps, codes, scale, s, grid);
+      break;
+    default: launch_quant_a4_cv<C, bl::kQFp4E1M2>(x, M, K, ldx, packed, eps, codes, scale, s, grid); break;
+  }
 }
 
 // Top-K rows: one 256-thread CTA per row, persistent grid sized by the occupancy
@@ -527,7 +544,9 @@ bl_status bitlinear_sync_status(void* stream) {
 
 bl_status bitlinear_quant_a4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, bl_quant quant, bl_store store,
                              float eps, void* codes, float* scale, void* stream) {
-  if (quant != BL_QUANT_INT4 && quant != BL_QUANT_FP4_E2M1) return BL_ERR_ARG;
+  if (quant != BL_QUANT_INT4 && quant != BL_QUANT_FP4_E2M1 && quant != BL_QUANT_INT4_ABSMAX &&
+      quant != BL_QUANT_INT4_ABSMEAN2 && quant != BL_QUANT_FP4_E1M2)
+    return BL_ERR_ARG;
   if (store != BL_STORE_PACKED && store != BL_STORE_BYTES) return BL_ERR_ARG;
   if (M < 0 || K < 8 || K > 16384 || (K & 7) || ldx < K || (ldx & 7) || M > 0x7FFFFFFELL) return BL_ERR_SHAPE;
   if (M == 0) return BL_OK;
@@ -535,16 +554,17 @@ bl_status bitlinear_quant_a4(const void* x_bf16, int64_t M, int64_t K, int64_t l
   if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scale)) return BL_ERR_ALIGN;
   if (!(eps >= 0.f)) return BL_ERR_ARG;
   const int64_t c = (K / 8 + bl::kQ4ThreadsPerRow - 1) / bl::kQ4ThreadsPerRow;
-  const bool fp4 = quant == BL_QUANT_FP4_E2M1, packed = store == BL_STORE_PACKED;
+  const int var = static_cast<int>(quant);   // bl_quant values are the kernel's variant ids
+  const bool packed = store == BL_STORE_PACKED;
   const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
   uint8_t* out = static_cast<uint8_t*>(codes);
   cudaStream_t s = as_stream(stream);
   const int k = static_cast<int>(K);
-  if (c <= 1) launch_quant_a4_c<1>(x, M, k, ldx, fp4, packed, eps, out, scale, s);
-  else if (c <= 2) launch_quant_a4_c<2>(x, M, k, ldx, fp4, packed, eps, out, scale, s);
-  else if (c <= 4) launch_quant_a4_c<4>(x, M, k, ldx, fp4, packed, eps, out, scale, s);
-  else if (c <= 8) launch_quant_a4_c<8>(x, M, k, ldx, fp4, packed, eps, out, scale, s);
-  else launch_quant_a4_c<16>(x, M, k, ldx, fp4, packed, eps, out, scale, s);
+  if (c <= 1) launch_quant_a4_c<1>(x, M, k, ldx, var, packed, eps, out, scale, s);
+  else if (c <= 2) launch_quant_a4_c<2>(x, M, k, ldx, var, packed, eps, out, scale, s);
+  else if (c <= 4) launch_quant_a4_c<4>(x, M, k, ldx, var, packed, eps, out, scale, s);
+  else if (c <= 8) launch_quant_a4_c<8>(x, M, k, ldx, var, packed, eps, out, scale, s);
+  else launch_quant_a4_c<16>(x, M, k, ldx, var, packed, eps, out, scale, s);
   return launch_status();
 }
 

@@ -908,25 +908,6 @@ __device__ __forceinline__ uint32_t expand_t2_byte(uint32_t b) {
   return __vsub4(spread ^ 0x02020202u, 0x02020202u);
 }
 
-// eight nibbles of a word -> two words of four bytes each, in element order
-__device__ __forceinline__ void split_nibbles(uint32_t p, uint32_t& w0, uint32_t& w1) {
-  const uint32_t lo = p & 0x0F0F0F0Fu;
-  const uint32_t hi = (p >> 4) & 0x0F0F0F0Fu;
-  w0 = __byte_perm(lo, hi, 0x5140);
-  w1 = __byte_perm(lo, hi, 0x7362);
-}
-
-__device__ __forceinline__ uint32_t sext_nibble_bytes(uint32_t x) { return __vsub4(x ^ 0x08080808u, 0x08080808u); }
-
-// E2M1 codes in bytes -> twice their value as int8: magnitudes {0,1,2,3,4,6,8,12}
-__device__ __forceinline__ uint32_t e2m1_bytes_to_twice(uint32_t x) {
-  const uint32_t idx = x & 0x07070707u;
-  const uint32_t sel = (idx & 0x7u) | ((idx >> 4) & 0x70u) | ((idx >> 8) & 0x700u) | ((idx >> 12) & 0x7000u);
-  const uint32_t mag = __byte_perm(0x03020100u, 0x0C080604u, sel);
-  const uint32_t m = ((x & 0x08080808u) >> 3) * 0xFFu;
-  return (mag & ~m) | (__vsub4(0u, mag) & m);
-}
-
 template <int AF>
 __device__ __forceinline__ void load_a_unit(const uint8_t* a_row, int u, uint32_t (&out)[16]) {
   if constexpr (AF == kSimtA_I8) {

@@ -1,5 +1,7 @@
 // 4-bit activation quantizer of BitNet a4.8 (arXiv 2411.04965, §3.4):
-//   quant_a4_kernel -- INT4 absmean (Eq. 6-7) or FP4 E2M1 MinMax (Eq. 8-9)
+//   quant_a4_kernel -- INT4 absmean (Eq. 6-7) or FP4 E2M1 MinMax (Eq. 8-9), and
+//                      the ablation variants INT4 absmax, INT4 absmean with
+//                      beta = 2 mean|x|, FP4 E1M2 (Fig. 5 and 6)
 // An HBM-bound row kernel: one pass over coalesced 16-byte loads, the row held
 // in registers, reductions by warp shuffles and a few shared words.  (Top-K +
 // INT8 rows are in topk.cuh.)
@@ -43,6 +45,43 @@ __device__ __forceinline__ int fp4_scale_exponent(uint32_t gbits) {
     e = -126 - sh;
   }
   return (m24 <= 0xC00000u) ? e - 2 : e - 1;
+}
+
+// Smallest p with g <= 1.75 * 2^p (FP4 E1M2's largest magnitude is 1.75):
+// with g = m * 2^e, m in [1, 2), p = e when m <= 1.75, else e + 1.
+__device__ __forceinline__ int e1m2_scale_exponent(uint32_t gbits) {
+  if (gbits == 0) return 0;
+  const uint32_t E = gbits >> 23;
+  const uint32_t mant = gbits & 0x7FFFFFu;
+  int e;
+  uint32_t m24;
+  if (E != 0) {
+    e = static_cast<int>(E) - 127;
+    m24 = mant | 0x800000u;
+  } else {
+    const int lead = 31 - __clz(mant);
+    const int sh = 23 - lead;
+    m24 = mant << sh;
+    e = -126 - sh;
+  }
+  return (m24 <= 0xE00000u) ? e : e + 1;
+}
+
+// Eight fp32 -> eight E2M1 codes (element e in bits 4e..4e+3) by the hardware
+// conversion: round to nearest, ties to the even encoding, saturating at 6.  A
+// magnitude that rounds to zero is re-encoded as +0 (sign bit cleared).
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
+  uint32_t w;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(w)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  const uint32_t nz = (w | (w >> 1) | (w >> 2)) & 0x11111111u;   // per nibble: magnitude bits nonzero
+  return w & (0x77777777u | (nz << 3));
 }
 
 // Index of the nearest E2M1 magnitude {0,.5,1,1.5,2,3,4,6} to a (a >= 0),
@@ -89,7 +128,12 @@ __device__ __forceinline__ void q4_load(const uint16_t* x, int64_t row, int64_t 
   }
 }
 
-template <int CHUNKS, bool FP4, bool PACKED>
+// Quantizer variants (the values of bl_quant): absmean INT4 (Eq. 6-7), MinMax
+// FP4 E2M1 (Eq. 8-9), and the ablation variants INT4 absmax, INT4 absmean with
+// beta = 2 mean|x|, FP4 E1M2.
+enum : int { kQInt4 = 0, kQFp4 = 1, kQInt4Absmax = 2, kQInt4Absmean2 = 3, kQFp4E1M2 = 4 };
+
+template <int CHUNKS, int VAR, bool PACKED>
 __global__ void __launch_bounds__(256) quant_a4_kernel(const uint16_t* __restrict__ x, int64_t M, int K,
                                                        int64_t ldx, float eps, uint8_t* __restrict__ codes,
                                                        float* __restrict__ scale) {
@@ -118,10 +162,13 @@ __global__ void __launch_bounds__(256) quant_a4_kernel(const uint16_t* __restric
       q4_load<CHUNKS>(x, row, M, ldx, nchunk, t, v);
     }
     const int par = it & 1;
+    constexpr bool kSum = VAR == kQInt4 || VAR == kQInt4Absmean2;   // mean|x| statistic, else max|x|
+    constexpr bool kInt = VAR == kQInt4 || VAR == kQInt4Absmean2 || VAR == kQInt4Absmax;
 
-    if constexpr (!FP4) {
-      // beta = mean|x|: the fp64 sum of bf16 magnitudes is exact for in-contract
-      // rows, so the reduction order does not change it.
+    // ---- the row statistic ----
+    double S = 0.0;       // sum |x| (exact in fp64 for in-contract rows: order-free)
+    uint32_t mk = 0;      // max |x| as the largest 15-bit bf16 magnitude
+    if constexpr (kSum) {
       double acc = 0.0;
 #pragma unroll
       for (int c = 0; c < CHUNKS; ++c) {
@@ -133,10 +180,34 @@ __global__ void __launch_bounds__(256) quant_a4_kernel(const uint16_t* __restric
       acc = warp_sum_f64(acc);
       if (lane == 0) s_sum[par][sub][warp] = acc;
       q4_row_sync(sub);
-      const double S = (s_sum[par][sub][0] + s_sum[par][sub][1]) + (s_sum[par][sub][2] + s_sum[par][sub][3]);
-      const float beta = __double2float_rn(S / static_cast<double>(K));
-      const float mult = __fdiv_rn(sqrt7_f32(), __fadd_rn(beta, eps));
-      if (t == 0) scale[row] = __fdiv_rn(beta, sqrt7_f32());
+      S = (s_sum[par][sub][0] + s_sum[par][sub][1]) + (s_sum[par][sub][2] + s_sum[par][sub][3]);
+    } else {
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) {
+        uint32_t k[8];
+        bf16x8_mag_keys(v[c], k);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mk = max(mk, k[e]);
+      }
+      mk = __reduce_max_sync(0xFFFFFFFFu, mk);
+      if (lane == 0) s_max[par][sub][warp] = mk;
+      q4_row_sync(sub);
+      mk = max(max(s_max[par][sub][0], s_max[par][sub][1]), max(s_max[par][sub][2], s_max[par][sub][3]));
+    }
+
+    if constexpr (kInt) {
+      // ---- INT4 codes RoundClip(x * mult, -8, 7) ----
+      float mult;
+      if constexpr (VAR == kQInt4Absmax) {
+        const float gamma = __uint_as_float(mk << 16);   // max |x| (a bf16 value)
+        mult = __fdiv_rn(7.f, __fadd_rn(gamma, eps));
+        if (t == 0) scale[row] = __fdiv_rn(gamma, 7.f);
+      } else {
+        // beta = mean|x| (INT4) or 2 mean|x| (the doubling is exact)
+        const float beta = __double2float_rn((VAR == kQInt4Absmean2 ? 2.0 * S : S) / static_cast<double>(K));
+        mult = __fdiv_rn(sqrt7_f32(), __fadd_rn(beta, eps));
+        if (t == 0) scale[row] = __fdiv_rn(beta, sqrt7_f32());
+      }
 #pragma unroll
       for (int c = 0; c < CHUNKS; ++c) {
         const int idx = c * kQ4ThreadsPerRow + t;
@@ -160,41 +231,42 @@ __global__ void __launch_bounds__(256) quant_a4_kernel(const uint16_t* __restric
         }
       }
     } else {
-      // MinMax FP4: max|x| as the largest 15-bit bf16 magnitude.
-      uint32_t mk = 0;
-#pragma unroll
-      for (int c = 0; c < CHUNKS; ++c) {
-        uint32_t k[8];
-        bf16x8_mag_keys(v[c], k);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mk = max(mk, k[e]);
-      }
-      mk = __reduce_max_sync(0xFFFFFFFFu, mk);
-      if (lane == 0) s_max[par][sub][warp] = mk;
-      q4_row_sync(sub);
-      mk = max(max(s_max[par][sub][0], s_max[par][sub][1]), max(s_max[par][sub][2], s_max[par][sub][3]));
-      const int p = fp4_scale_exponent(mk << 16);
-      if (t == 0) scale[row] = exact_pow2(PACKED ? p : p - 1);
+      // ---- MinMax FP4: a power-of-two scale 2^p, the nearest grid magnitude ----
+      constexpr bool kE1M2 = VAR == kQFp4E1M2;
+      const int p = kE1M2 ? e1m2_scale_exponent(mk << 16) : fp4_scale_exponent(mk << 16);
+      // bytes hold 2 x the E2M1 value or 4 x the E1M2 value
+      if (t == 0) scale[row] = exact_pow2(PACKED ? p : (kE1M2 ? p - 2 : p - 1));
 #pragma unroll
       for (int c = 0; c < CHUNKS; ++c) {
         const int idx = c * kQ4ThreadsPerRow + t;
         if (idx >= nchunk) continue;
         float f[8];
         unpack_bf16x8(v[c], f);
+        float sv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sv[e] = mul_pow2(f[e], -p);   // exact
         uint32_t word = 0;
         uint2 w2 = make_uint2(0, 0);
+        if constexpr (!kE1M2) {
+          word = cvt_e2m1x8(sv);
+          if constexpr (!PACKED) {
+            // bytes: twice the E2M1 value {0,1,2,3,4,6,8,12} with its sign
+            uint32_t b0, b1;
+            split_nibbles(word, b0, b1);
+            w2 = make_uint2(e2m1_bytes_to_twice(b0), e2m1_bytes_to_twice(b1));
+          }
+        } else {
+          // the E1M2 magnitudes are the quarters 0..7/4: index = rint(4 |v|)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float s = mul_pow2(f[e], -p);
-          const int i = e2m1_index(fabsf(s));
-          const bool neg = (s < 0.f) && (i != 0);
-          if constexpr (PACKED) {
-            word |= (static_cast<uint32_t>(i) | (neg ? 8u : 0u)) << (4 * e);
-          } else {
-            // twice the E2M1 value: {0,1,2,3,4,6,8,12}[i]
-            const int tv = (i <= 4) ? i : (i == 5 ? 6 : (i == 6 ? 8 : 12));
-            const uint32_t b = static_cast<uint32_t>(neg ? -tv : tv) & 0xFFu;
-            if (e < 4) w2.x |= b << (8 * e); else w2.y |= b << (8 * (e - 4));
+          for (int e = 0; e < 8; ++e) {
+            const int i = min(__float2int_rn(__fmul_rn(fabsf(sv[e]), 4.f)), 7);
+            const bool neg = (sv[e] < 0.f) && (i != 0);
+            if constexpr (PACKED) {
+              word |= (static_cast<uint32_t>(i) | (neg ? 8u : 0u)) << (4 * e);
+            } else {
+              const uint32_t b = static_cast<uint32_t>(neg ? -i : i) & 0xFFu;
+              if (e < 4) w2.x |= b << (8 * e); else w2.y |= b << (8 * (e - 4));
+            }
           }
         }
         if constexpr (PACKED) {

@@ -65,6 +65,63 @@ def test_quant_fp4_parity(name, make, store):
         assert np.array_equal(scale.view(np.uint32), half.view(np.uint32))
 
 
+# the ablation variants (Fig. 5 / Fig. 6) as flags of the same quantizer
+@pytest.mark.parametrize("name,make", QUANT_CASES, ids=[c[0] for c in QUANT_CASES])
+@pytest.mark.parametrize("store", [tba.BL_STORE_PACKED, tba.BL_STORE_BYTES], ids=["packed", "bytes"])
+@pytest.mark.parametrize("variant", ["int4_absmax", "int4_absmean2"])
+def test_quant_int4_variant_parity(name, make, store, variant):
+    x = make()
+    quant = tba.BL_QUANT_INT4_ABSMAX if variant == "int4_absmax" else tba.BL_QUANT_INT4_ABSMEAN2
+    codes, scale = run_quant_a4(x, quant, store)
+    ref = oracle.quant_int4_absmax if variant == "int4_absmax" else oracle.quant_int4_absmean2
+    c_ref, _, s_ref = ref(x, EPS)
+    if store == tba.BL_STORE_PACKED:
+        assert np.array_equal(codes, oracle.pack_nibbles(c_ref))
+    else:
+        assert np.array_equal(codes.view(np.int8), c_ref)
+    assert np.array_equal(scale.view(np.uint32), s_ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("name,make", QUANT_CASES, ids=[c[0] for c in QUANT_CASES])
+@pytest.mark.parametrize("store", [tba.BL_STORE_PACKED, tba.BL_STORE_BYTES], ids=["packed", "bytes"])
+def test_quant_fp4_e1m2_parity(name, make, store):
+    x = make()
+    codes, scale = run_quant_a4(x, tba.BL_QUANT_FP4_E1M2, store)
+    code4, four, p, s_ref = oracle.quant_fp4_e1m2(x)
+    if store == tba.BL_STORE_PACKED:
+        assert np.array_equal(codes, oracle.pack_nibbles(code4))
+        assert np.array_equal(scale.view(np.uint32), s_ref.view(np.uint32))
+    else:
+        assert np.array_equal(codes.view(np.int8), four)
+        quarter = (s_ref.astype(np.float64) / 4).astype(np.float32)
+        assert np.array_equal(scale.view(np.uint32), quarter.view(np.uint32))
+
+
+def test_quant_fp4_e1m2_extreme_exponents_and_gemm():
+    vals = [1e-39, 3e-38, 1e-20, 0.011, 1.75, 1.765625, 1e4, 3e38]
+    rows = []
+    for v in vals:
+        r = synth.gaussian_bf16(synth.rng(8), (1, 64))
+        f = np.clip(synth.bf16_bits_to_f32(r), -4, 4) * np.float32(v / 8)
+        rows.append(synth.f32_to_bf16_bits(f))
+    x = np.concatenate(rows)
+    codes, scale = run_quant_a4(x, tba.BL_QUANT_FP4_E1M2, tba.BL_STORE_BYTES)
+    code4, four, p, s_ref = oracle.quant_fp4_e1m2(x)
+    assert np.array_equal(codes.view(np.int8), four)
+    # the bytes feed the INT8 GEMM: acc = sum of 4 * value * t
+    g = synth.rng(9)
+    M, K = x.shape
+    N = 48
+    t = g.integers(-1, 2, (N, K)).astype(np.int8)
+    y = empty((M, N), torch.int16)
+    acc = empty((M, N), torch.int32)
+    tba.bitlinear_gemm(to_dev(codes.view(np.int8)), to_dev(scale), to_dev(oracle.pack_ternary2(t)),
+                       to_dev(np.array([0.02], np.float32)), M, N, K, y=y, acc=acc, wfmt=tba.BL_W_T2)
+    tba.sync_status()
+    acc_ref, _ = oracle.gemm(four, scale, t, np.float32(0.02), want_y=False)
+    assert np.array_equal(host(acc), acc_ref)
+
+
 def test_quant_fp4_extreme_exponents():
     # rows whose max spans bf16's whole exponent range, subnormals included
     vals = [1e-39, 3e-38, 1e-20, 0.011, 6.0, 6.03125, 1e4, 3e38]
