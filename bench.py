@@ -682,7 +682,7 @@ def run_decode(args):
         y_down = T.empty((m, d), dtype=T.int16, device=dev)
         qg_ws = T.empty((tba.workspace_size("quant_gemm", m, 2 * f, d) // 8 + 1,), dtype=T.int64, device=dev)
 
-        def layer(w2, alpha, gemms=True, others=True, fused=False):
+        def layer(w2, alpha, gemms=True, others=True, fused=False, gated=False):
             # fused: the INT4 quantizer of the QKV and Up|Gate inputs runs inside
             # the GEMM call (bitlinear_quant_gemm)
             if fused:
@@ -701,9 +701,12 @@ def run_decode(args):
                                          alpha_group=f, workspace=qg_ws)
             if others and not fused:
                 tba.bitlinear_quant_a4(x_ffn, qa, qa_s, tba.BL_QUANT_INT4, tba.BL_STORE_BYTES, EPS)
-            if gemms and not fused:
+            if gemms and not fused and not gated:
                 tba.bitlinear_gemm(qa, qa_s, w2["upgate"], alpha[2:4], m, 2 * f, d, y=y_ug, wfmt=tba.BL_W_T2,
                                    alpha_group=f)
+            if gemms and gated:
+                # conditional Up: Gate rows first, Up rows only for channels with a positive gate
+                tba.bitlinear_gemm_gated(qa, qa_s, w2["upgate"], alpha[2:4], m, f, d, y_ug)
             if others:
                 tba.relu2_glu(y_ug[:, f:], y_ug[:, :f], synth.k_keep(f, s.topk_pct_down), h8, h8_s, None, EPS,
                               M=m, F=f, ld=2 * f)
@@ -717,6 +720,10 @@ def run_decode(args):
         def step_fused():
             for w2, alpha in layers:
                 layer(w2, alpha, fused=True)
+
+        def step_gated():
+            for w2, alpha in layers:
+                layer(w2, alpha, gated=True)
 
         def gemms_only():
             for w2, alpha in layers:
@@ -742,6 +749,7 @@ def run_decode(args):
 
         g_step = capture(step)
         g_fused = capture(step_fused)
+        g_gated = capture(step_gated) if m <= 2 else None
         g_gemm = capture(gemms_only)
 
         def time_graph(graph):
@@ -758,12 +766,14 @@ def run_decode(args):
 
         ms = time_graph(g_step)
         fused_ms = time_graph(g_fused)
+        gated_ms = time_graph(g_gated) if g_gated is not None else None
         gemm_ms = time_graph(g_gemm)
         tba.sync_status()
-        del g_step, g_fused, g_gemm
+        del g_step, g_fused, g_gated, g_gemm
         gbs = weight_bytes / (gemm_ms / 1e3) / 1e9
         results.append({"tokens": m, "ms_per_layer": round(ms, 4), "tokens_per_s": round(m / (ms / 1e3), 1),
                         "fused_quant_ms_per_layer": round(fused_ms, 4),
+                        "conditional_up_ms_per_layer": round(gated_ms, 4) if gated_ms is not None else None,
                         "gemm_ms_per_layer": round(gemm_ms, 4),
                         "gemm_kernel": decode_gemm_kernel(m),
                         "weight_stream_gbs": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 3)})
@@ -772,7 +782,8 @@ def run_decode(args):
             "workload": f"7B-shape decoder layers, decode of M tokens through all four BitLinear matrices of "
                         f"each of {DECODE_LAYERS} distinct layers (weights exceed L2), separate quantizer and GEMM "
                         f"calls; fused_quant_ms_per_layer: the QKV and Up|Gate INT4 quantizers fused into their "
-                        f"GEMMs (bitlinear_quant_gemm)",
+                        f"GEMMs (bitlinear_quant_gemm); conditional_up_ms_per_layer (1-2 tokens): the Up|Gate GEMM as "
+                        f"Gate first and Up only on channels with a positive gate (bitlinear_gemm_gated)",
             "weight_bytes_per_layer": weight_bytes, "hbm_peak_gbs": peaks["hbm_gbs"],
             "steps": args.steps, "warmup": args.warmup, "results": results}
     print(json.dumps(line), flush=True)

@@ -236,6 +236,28 @@ BL_API bl_status bitlinear_quant_gemm(const void* x_bf16, int64_t ldx, bl_quant 
                                void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * bitlinear_gemm_gated -- the conditional Up projection (paper: §3.4 "Squared
+ * ReLU Gating" and the FFN paragraph after Eq. 5: the Up projection only needs
+ * the channels where ReLU^2(gate) != 0).  w = [W_up; W_gate] as for the stacked
+ * Up|Gate bitlinear_gemm (F rows each, BL_W_T2), alpha = {alpha_up, alpha_gate}.
+ *   y[m, F + n] = the Gate output, exactly as bitlinear_gemm writes it;
+ *   y[m, n]     = the Up output where some token's gate output y[., F + n] is
+ *                 > 0, else +0 (the Up row's bytes are then never read);
+ *   acc_out likewise (0 for skipped Up entries).
+ * relu2_glu(y[:, F:], y[:, :F], ...) then produces the same codes, mask and
+ * scale as after the dense Up|Gate GEMM: h = up * max(0, gate)^2 is a zero on
+ * the skipped channels either way.
+ * a: M x K activation codes (afmt as for bitlinear_gemm); y: [M x ldy] bf16
+ * with ldy >= 2F; acc_out: [M x 2F] int32 (nullable).
+ * Requires K % 64 == 0.  Kernel: decode, M <= 2 and K <= 4096
+ * (BL_ERR_UNSUPPORTED otherwise); weights only in BL_W_T2.
+ */
+BL_API bl_status bitlinear_gemm_gated(const void* a, bl_afmt afmt, const float* a_scale,
+                               const void* w, bl_wfmt wfmt, const float* alpha,
+                               int64_t M, int64_t F, int64_t K,
+                               void* y_bf16, int64_t ldy, int32_t* acc_out, void* stream);
+
+/*
  * relu2_glu -- squared-ReLU GLU fused with the down projection's
  * sparsify-then-quantize step.
  * Paper: §3.4 "Squared ReLU Gating and Conditional Computation in the FFN",

@@ -28,7 +28,7 @@ BL_A_I8, BL_A_I4, BL_A_E2M1 = 0, 1, 2
 BL_W_T2, BL_W_I8, BL_W_E2M1 = 0, 1, 2
 
 EXPORTED = ["bitlinear_quant_a4", "bitlinear_sparsify_a8", "pack_ternary", "pack_ternary_noalloc", "bitlinear_gemm",
-            "bitlinear_quant_gemm", "relu2_glu",
+            "bitlinear_quant_gemm", "bitlinear_gemm_gated", "relu2_glu",
             "kv_quant3", "bitlinear_workspace_size", "bitlinear_sync_status", "bitlinear_status_string",
             "bitlinear_last_cuda_error", "bitlinear_version"]
 
@@ -59,6 +59,7 @@ def lib():
             "pack_ternary_noalloc": [P, I64, I64, I64, F, I, P, I, P, P],
             "bitlinear_gemm": [P, I, P, P, I, P, I64, I64, I64, I64, P, I64, P, P],
             "bitlinear_quant_gemm": [P, I64, I, F, P, I, P, I64, I64, I64, I64, P, I64, P, P, ctypes.c_size_t, P],
+            "bitlinear_gemm_gated": [P, I, P, P, I, P, I64, I64, I64, P, I64, P, P],
             "relu2_glu": [P, P, I64, I64, I64, I64, F, P, P, P, P],
             "kv_quant3": [P, I64, I64, I64, I64, I, I64, F, P, P, P, P],
             "bitlinear_sync_status": [P],
@@ -152,6 +153,15 @@ def bitlinear_quant_gemm(x, w, alpha, M, N, K, y=None, acc=None, quant=BL_QUANT_
     _check("bitlinear_quant_gemm", lib().bitlinear_quant_gemm(_ptr(x), ldx, quant, eps, _ptr(w), wfmt, _ptr(alpha),
                                                               group, M, N, K, _ptr(y), ldy, _ptr(acc),
                                                               _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def bitlinear_gemm_gated(a, a_scale, w, alpha, M, F, K, y, acc=None, afmt=BL_A_I8, wfmt=BL_W_T2, ldy=None,
+                         stream=None):
+    """Gate rows of [W_up; W_gate] first, Up rows only where some token's gate > 0."""
+    ldy = y.stride(0) if ldy is None else ldy
+    _check("bitlinear_gemm_gated", lib().bitlinear_gemm_gated(_ptr(a), afmt, _ptr(a_scale), _ptr(w), wfmt,
+                                                              _ptr(alpha), M, F, K, _ptr(y), ldy, _ptr(acc),
+                                                              _stream(stream)))
 
 
 def relu2_glu(gate, up, k_keep, codes, scale, mask=None, eps=1e-5, M=None, F=None, ld=None, stream=None):

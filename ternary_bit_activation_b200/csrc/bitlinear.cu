@@ -837,6 +837,41 @@ bl_status bitlinear_quant_gemm(const void* x_bf16, int64_t ldx, bl_quant quant, 
   return bitlinear_gemm(codes, BL_A_I8, scale, w, wfmt, alpha, alpha_group, M, N, K, y_bf16, ldy, acc_out, stream);
 }
 
+bl_status bitlinear_gemm_gated(const void* a, bl_afmt afmt, const float* a_scale, const void* w, bl_wfmt wfmt,
+                               const float* alpha, int64_t M, int64_t F, int64_t K, void* y_bf16, int64_t ldy,
+                               int32_t* acc_out, void* stream) {
+  if (afmt != BL_A_I8 && afmt != BL_A_I4 && afmt != BL_A_E2M1) return BL_ERR_ARG;
+  if (wfmt != BL_W_T2) return BL_ERR_UNSUPPORTED;
+  if (M < 0 || F < 1 || K < 64 || (K & 63) || F > 0x3FFFFFFFLL || ldy < 2 * F || (ldy & 7)) return BL_ERR_SHAPE;
+  if (M == 0) return BL_OK;
+  if (M > 2 || K > 4096) return BL_ERR_UNSUPPORTED;   // the decode kernel: one 4096-code round, 1-2 tokens
+  if (a == nullptr || a_scale == nullptr || w == nullptr || alpha == nullptr || y_bf16 == nullptr) return BL_ERR_NULL;
+  if (!aligned16(a) || !aligned16(w) || !aligned16(y_bf16) || (acc_out && !aligned16(acc_out)) ||
+      (reinterpret_cast<uintptr_t>(a_scale) & 3u) || (reinterpret_cast<uintptr_t>(alpha) & 3u))
+    return BL_ERR_ALIGN;
+  cudaStream_t s = as_stream(stream);
+  const int m = static_cast<int>(M), f = static_cast<int>(F), k = static_cast<int>(K);
+  const uint8_t* A = static_cast<const uint8_t*>(a);
+  const uint8_t* W = static_cast<const uint8_t*>(w);
+  uint16_t* Y = static_cast<uint16_t*>(y_bf16);
+  auto go = [&](auto kern, int mt) -> bl_status {
+    const size_t smem = static_cast<size_t>(mt) * static_cast<size_t>(k);
+    int per_sm = 0;
+    if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem))) return BL_ERR_CUDA;
+    if (per_sm < 1) per_sm = 1;
+    const int64_t passes = ((static_cast<int64_t>(f) + 3) / 4 + 7) / 8;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
+    const unsigned grid = static_cast<unsigned>(passes < cap ? passes : cap);
+    launch_pdl(kern, grid, 256, smem, s, A, a_scale, W, alpha, m, f, k, Y, ldy, acc_out);
+    return launch_status();
+  };
+  if (afmt == BL_A_I8) return m == 1 ? go(bl::gemv_gated_t2_kernel<bl::kSimtA_I8, 1>, 1)
+                                     : go(bl::gemv_gated_t2_kernel<bl::kSimtA_I8, 2>, 2);
+  if (afmt == BL_A_I4) return m == 1 ? go(bl::gemv_gated_t2_kernel<bl::kSimtA_I4, 1>, 1)
+                                     : go(bl::gemv_gated_t2_kernel<bl::kSimtA_I4, 2>, 2);
+  return m == 1 ? go(bl::gemv_gated_t2_kernel<bl::kSimtA_E2M1, 1>, 1) : go(bl::gemv_gated_t2_kernel<bl::kSimtA_E2M1, 2>, 2);
+}
+
 bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D, int64_t ldt, int bits, int64_t bos_pos,
                     float eps, uint8_t* codes, float* scale, uint8_t* bos_codes, void* stream) {
   if (bits != 3 && bits != 4) return BL_ERR_ARG;

@@ -18,6 +18,8 @@
 //                     (16 weight rows x 8 or 16 token slots per instruction).
 // gemv_stream_t2_kernel -- 1-2 tokens, the CTA's contiguous weight range
 //                     streamed through shared memory by 1-D bulk copies.
+// gemv_gated_t2_kernel -- the conditional Up projection (Gate rows first, Up
+//                     rows only for channels with a positive gate), 1-2 tokens.
 // gemm_simt_kernel -- CUDA-core kernel that reads packed operands directly
 //                     (2-bit ternary weights, INT4 / E2M1 nibbles); decode of
 //                     3 to 7 tokens and the packed activation formats.
@@ -1856,6 +1858,159 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_stream_t2_kernel(const uin
     const uint64_t t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 200000ull) {
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// gemv_gated_t2_kernel -- the conditional Up projection for 1 or 2 tokens
+// (the FFN's Gate first, Up only where it matters).  W holds [W_up; W_gate]
+// (F rows each, 2-bit).  A warp takes 4 channels n: it computes their Gate rows
+// (F + n) exactly as gemv_t2_kernel does and writes y[:, F + n]; a channel is
+// active when some token's bf16 gate output is > 0, and only then are its Up
+// row's bytes loaded and y[:, n] computed -- elsewhere y[:, n] = +0 (and acc 0):
+// ReLU^2 makes h = up * max(0, gate)^2 a zero there whatever up is, so the
+// ReLU^2-GLU quantizer gives the same codes, mask and scale.  Rows of up to
+// 4096 codes (one round per warp); persistent CTAs stage the activations once.
+// ---------------------------------------------------------------------------
+template <int AF, int MT>
+__global__ void __launch_bounds__(256) gemv_gated_t2_kernel(const uint8_t* __restrict__ a,
+                                                            const float* __restrict__ a_scale,
+                                                            const uint8_t* __restrict__ w,
+                                                            const float* __restrict__ alpha, int M, int F, int K,
+                                                            uint16_t* __restrict__ y, int64_t ldy,
+                                                            int32_t* __restrict__ acc_out) {
+  constexpr int R = 4;
+  extern __shared__ uint4 gg_smem[];
+  __shared__ int asum[MT];
+  __shared__ float s_scale[MT];
+  __shared__ double red[kGvMaxWarps][MT];
+  const int kw16 = K >> 4;                 // <= 256: one 4096-code round
+  const int kq = kw16 >> 2;
+  uint4* act = gg_smem;                    // [MT][4][kq]
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int64_t wrow_bytes = K >> 2;
+  const int64_t groups = (static_cast<int64_t>(F) + R - 1) / R;
+  const int64_t group_step = static_cast<int64_t>(gridDim.x) * 8;
+  const int64_t N2 = 2 * static_cast<int64_t>(F);
+
+  // the Gate rows this warp will read go to L2 before the wait (the Up rows
+  // are read only where the gate says so)
+  if (lane < 8 * R) {
+    const int r = lane >> 3;
+    const int64_t b = (lane & 7) * 128;
+    if (b < wrow_bytes)
+      for (int64_t gi = static_cast<int64_t>(blockIdx.x) * 8 + warp; gi < groups; gi += group_step) {
+        const int64_t n = gi * R + r;
+        if (n < F) prefetch_l2(w + (F + n) * wrow_bytes + b);
+      }
+  }
+  if (threadIdx.x < MT) asum[threadIdx.x] = 0;
+  __syncthreads();
+  pdl_wait();
+  pdl_trigger();
+  gv_stage<AF, MT>(a, 0, 0.f, M, K, act, [kq](int q, int m) { return (m * 4 + (q & 3)) * kq + (q >> 2); }, asum,
+                   red, s_scale);
+  __syncthreads();
+  const float unit_scale = (AF == kSimtA_E2M1) ? 0.5f : 1.0f;
+  float sc[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) sc[m] = m < M ? __fmul_rn(ld_dep_f32(a_scale + m), unit_scale) : 0.f;
+  const float al_up = ld_dep_f32(alpha), al_gate = ld_dep_f32(alpha + 1);
+
+  // one matrix row block: R rows starting at `row` (skipping rows whose bit in
+  // `use` is clear), sums of (c + 1) a over this lane's codes, reduced over the warp
+  auto row_sums = [&](int64_t row, int64_t nrows, uint32_t use, int (&tot)[R][MT]) {
+    uint4 wv[R][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int wq = h * 128 + 4 * lane;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const bool ok = wq < kw16 && r < nrows && ((use >> r) & 1u);
+        wv[r][h] = ok ? ld_global_nc_v4(w + (row + r) * wrow_bytes + static_cast<int64_t>(wq) * 4)
+                      : make_uint4(0, 0, 0, 0);
+      }
+    }
+    int acc[R][MT][4];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[r][m][j] = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int wq = h * 128 + 4 * lane;
+      if (wq >= kw16) continue;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint4 av[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) av[m] = act[(m * 4 + j) * kq + (wq >> 2)];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          if (!((use >> r) & 1u)) continue;
+          const uint32_t x = j == 0 ? wv[r][h].x : (j == 1 ? wv[r][h].y : (j == 2 ? wv[r][h].z : wv[r][h].w));
+          const uint32_t u = ~x & (0x55555555u | (x << 1));
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            acc[r][m][0] = dp4a_us(u & 0x03030303u, av[m].x, acc[r][m][0]);
+            acc[r][m][1] = dp4a_us(u & 0x0C0C0C0Cu, av[m].y, acc[r][m][1]);
+            acc[r][m][2] = dp4a_us(u & 0x30303030u, av[m].z, acc[r][m][2]);
+            acc[r][m][3] = dp4a_us(u & 0xC0C0C0C0u, av[m].w, acc[r][m][3]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+        tot[r][m] = __reduce_add_sync(0xFFFFFFFFu, acc[r][m][0] + (acc[r][m][1] >> 2) + (acc[r][m][2] >> 4) +
+                                                       (acc[r][m][3] >> 6));
+  };
+
+  for (int64_t gb = static_cast<int64_t>(blockIdx.x) * 8; gb < groups; gb += group_step) {
+    const int64_t n0 = (gb + warp) * R;
+    if (n0 >= F) continue;   // warp-uniform; no barrier follows
+    const int64_t nrows = min(static_cast<int64_t>(R), static_cast<int64_t>(F) - n0);
+    // ---- Gate rows ----
+    int tg[R][MT];
+    row_sums(F + n0, nrows, 0xFu, tg);
+    uint32_t pos = 0;   // lane r * MT + m: the gate output is > 0
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+        if (lane == r * MT + m && r < nrows && m < M) {
+          const int64_t n = F + n0 + r;
+          const int v = tg[r][m] - asum[m];
+          if (acc_out != nullptr) acc_out[static_cast<int64_t>(m) * N2 + n] = v;
+          const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__int2float_rn(v), __fmul_rn(sc[m], al_gate)));
+          const uint16_t bits = *reinterpret_cast<const uint16_t*>(&b);
+          y[static_cast<int64_t>(m) * ldy + n] = bits;
+          pos = (bits & 0x8000u) == 0u && bits != 0u;
+        }
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, pos != 0u);
+    uint32_t use = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) use |= (((bal >> (r * MT)) & ((1u << MT) - 1u)) != 0u ? 1u : 0u) << r;
+    // ---- Up rows of the active channels ----
+    int tu[R][MT];
+    row_sums(n0, nrows, use, tu);
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+        if (lane == r * MT + m && r < nrows && m < M) {
+          const int64_t n = n0 + r;
+          const bool on = (use >> r) & 1u;
+          const int v = on ? tu[r][m] - asum[m] : 0;
+          if (acc_out != nullptr) acc_out[static_cast<int64_t>(m) * N2 + n] = v;
+          const __nv_bfloat16 b = __float2bfloat16_rn(__fmul_rn(__int2float_rn(v), __fmul_rn(sc[m], al_up)));
+          y[static_cast<int64_t>(m) * ldy + n] = on ? *reinterpret_cast<const uint16_t*>(&b) : uint16_t(0);
+        }
   }
 }
 

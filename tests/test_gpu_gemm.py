@@ -487,5 +487,67 @@ def test_quant_gemm_needs_workspace_beyond_the_gemv():
     assert np.array_equal(host(y[:4], np.uint16), np.zeros((4, N), np.uint16))
 
 
+# the conditional Up projection: Gate rows first, Up rows only where some
+# token's gate output is > 0; ReLU^2-GLU must then give exactly what it gives
+# after the dense Up|Gate GEMM
+@pytest.mark.parametrize("M", [1, 2])
+@pytest.mark.parametrize("F,K,zero_frac", [(96, 640, 0.0), (1000, 4096, 0.0), (1000, 4096, 0.675), (37, 64, 0.0),
+                                           (2048, 1536, 1.0)])
+def test_gemm_gated_conditional_up(M, F, K, zero_frac):
+    g = synth.rng(M * 7 + F + K)
+    x = synth.gaussian_bf16(g, (M, K))
+    c, _, s_ref = oracle.quant_int4(x, EPS)
+    wu, wg = synth.latent_weights_f32(g, F, K), synth.latent_weights_f32(g, F, K)
+    tu, au = oracle.ternary_quantize(wu, EPS)
+    tg, ag = oracle.ternary_quantize(wg, EPS)
+    # all-zero Gate rows give exactly-zero gate outputs: inactive channels at a
+    # chosen share (0.675: the pages' Gate sparsity; 1.0: no Up row is read)
+    tg[g.random(F) < zero_frac] = 0
+    t = np.concatenate([tu, tg])
+    al = np.array([au, ag], np.float32)
+    a_dev, s_dev, w_dev, al_dev = to_dev(c), to_dev(s_ref), to_dev(oracle.pack_ternary2(t)), to_dev(al)
+    ldy = (2 * F + 15) // 8 * 8
+    # dense reference path: the stacked Up|Gate GEMM
+    y_dense = empty((M, ldy), torch.int16)
+    acc_dense = empty((M, 2 * F), torch.int32)
+    tba.bitlinear_gemm(a_dev, s_dev, w_dev, al_dev, M, 2 * F, K, y=y_dense, acc=acc_dense, wfmt=tba.BL_W_T2,
+                       alpha_group=F, ldy=ldy)
+    y_g = empty((M, ldy), torch.int16)
+    acc_g = empty((M, 2 * F), torch.int32)
+    tba.bitlinear_gemm_gated(a_dev, s_dev, w_dev, al_dev, M, F, K, y_g, acc=acc_g, ldy=ldy)
+    tba.sync_status()
+    yd, yg = host(y_dense, np.uint16)[:, :2 * F], host(y_g, np.uint16)[:, :2 * F]
+    ad, ag_ = host(acc_dense), host(acc_g)
+    acc_ref, _ = oracle.gemm(c, s_ref, t, al, alpha_group=F, want_y=False)
+    # the Gate half: exactly the dense GEMM's, and the oracle's sums
+    assert np.array_equal(yg[:, F:], yd[:, F:])
+    assert np.array_equal(ag_[:, F:], acc_ref[:, F:])
+    # the Up half: the oracle's sums on active channels, zeros elsewhere
+    gate_bits = yg[:, F:]
+    active = ((gate_bits & 0x8000) == 0) & (gate_bits != 0)
+    active = active.any(axis=0)
+    assert np.array_equal(ag_[:, :F], np.where(active[None, :], acc_ref[:, :F], 0))
+    assert np.array_equal(yg[:, :F], np.where(active[None, :], yd[:, :F], 0))
+    if zero_frac == 0.0:
+        assert 0 < active.sum() < F
+    if zero_frac == 1.0:
+        assert not active.any() and not ag_[:, :F].any()
+    # ReLU^2-GLU + Top-K 50% + INT8 gives identical codes, scale and mask (rows of
+    # a multiple of 8 values; F = 37 checks the ragged last channel group only)
+    if F % 8:
+        return
+    keep = synth.k_keep(F, 50)
+    outs = []
+    for y in (y_dense, y_g):
+        h8 = empty((M, F), torch.int8)
+        h8_s = empty((M,), torch.float32)
+        mask = empty((M, (F + 31) // 32), torch.int32)
+        tba.relu2_glu(y[:, F:2 * F], y[:, :F], keep, h8, h8_s, mask, EPS, M=M, F=F, ld=ldy)
+        tba.sync_status()
+        outs.append((host(h8), host(h8_s).view(np.uint32), host(mask)))
+    for u, v in zip(*outs):
+        assert np.array_equal(u, v)
+
+
 def test_sync_status_clean():
     tba.sync_status()
