@@ -19,9 +19,9 @@
 
 namespace {
 
-static_assert(BL_QUANT_INT4 == bl::kQInt4 && BL_QUANT_FP4_E2M1 == bl::kQFp4 &&
-                  BL_QUANT_INT4_ABSMAX == bl::kQInt4Absmax && BL_QUANT_INT4_ABSMEAN2 == bl::kQInt4Absmean2 &&
-                  BL_QUANT_FP4_E1M2 == bl::kQFp4E1M2,
+static_assert(int{BL_QUANT_INT4} == bl::kQInt4 && int{BL_QUANT_FP4_E2M1} == bl::kQFp4 &&
+                  int{BL_QUANT_INT4_ABSMAX} == bl::kQInt4Absmax &&
+                  int{BL_QUANT_INT4_ABSMEAN2} == bl::kQInt4Absmean2 && int{BL_QUANT_FP4_E1M2} == bl::kQFp4E1M2,
               "bl_quant values are the quantizer kernel's variant ids");
 
 constexpr int kMaxDevices = 64;

@@ -304,6 +304,10 @@ __global__ void __launch_bounds__(kTkThreads, F32 ? 2 : 4) topk_rows_kernel(
 #pragma unroll
             for (int i = 0; i < 8; ++i) t[i] = h[8 * lane + i];
             tk_select(t, r, lane, sm.sel);
+          } else {
+            // the other histogram (last used a pass ago) is cleared for the next pass
+            uint32_t* h2 = sm.hist[(pass + 1) & 1];
+            for (int i = tid - 32; i < 256; i += kTkThreads - 32) h2[i] = 0;
           }
         }
         __syncthreads();
@@ -311,8 +315,10 @@ __global__ void __launch_bounds__(kTkThreads, F32 ? 2 : 4) topk_rows_kernel(
         tie_total = sm.sel[2];
         prefix |= sm.sel[0] << shift;
         fixed |= dmask << shift;
-        if (F32 && pass == 1 && tie_total <= static_cast<uint32_t>(kTkListCap)) {
-          // two digits fixed: the remaining candidates go to the list
+        if (F32 && !listed && pass < kPasses - 1 && tie_total <= static_cast<uint32_t>(kTkListCap)) {
+          // few candidates left (ReLU^2 rows usually cut among their smallest
+          // nonzero values, one exponent bucket): they go to a list, and the
+          // remaining digits are counted over the list only
           if (tid == 0) sm.list_n = 0;
           for (int i = tid; i < 512; i += kTkThreads) (&sm.hist[0][0])[i] = 0;
           __syncthreads();
