@@ -802,6 +802,7 @@ PROFILE_CASES = {
     "pack_ternary": "ternary pack to int8, W fp32 [22016 x 4096]",
     "gemm_decode": "CUDA-core GEMV, 2-bit W [12288 x 4096], 1 token",
     "gemm_decode_mma": "warp-MMA GEMV, 2-bit W [12288 x 4096], 8 tokens",
+    "gemm_decode_stream": "streaming GEMV, 2-bit W [4096 x 11008] (Down), 1 token",
     "gemm_decode_tc": "tcgen05 GEMM, 2-bit W [12288 x 4096] widened into TMEM, 16 tokens",
 }
 
@@ -826,8 +827,9 @@ def run_profile_case(name: str, launches: int):
         al = torch.full((1,), 0.0173, device=dev)
         y = torch.empty((M, N), dtype=torch.int16, device=dev)
         fn = lambda: tba.bitlinear_gemm(a, s, w, al, M, N, K, y=y)
-    elif name in ("gemm_decode", "gemm_decode_mma"):
-        M, N, K = (1 if name == "gemm_decode" else 8), 12288, 4096
+    elif name in ("gemm_decode", "gemm_decode_mma", "gemm_decode_stream"):
+        M, N, K = {"gemm_decode": (1, 12288, 4096), "gemm_decode_mma": (8, 12288, 4096),
+                   "gemm_decode_stream": (1, 4096, 11008)}[name]
         a = torch.randint(-8, 8, (M, K), generator=g, device=dev, dtype=torch.int8)
         w = torch.randint(0, 256, (N, K // 4), generator=g, device=dev, dtype=torch.int32).to(torch.uint8)
         s = torch.rand((M,), generator=g, device=dev)
