@@ -288,7 +288,7 @@ BL_API bl_status relu2_glu(const void* gate_bf16, const void* up_bf16, int64_t M
  * When bits == 3 and 0 <= bos_pos < T, position bos_pos is quantized at 4 bits
  * into bos_codes ([H x D/2] bytes, nibble layout), its scale is gamma/7, and
  * its 3-bit slot in `codes` is zero-filled.  bos_pos = -1: no BOS row.
- * Requires D % 32 == 0, 32 <= D <= 256, ldt % 8 == 0, T * H < 2^29.
+ * Requires D in {32, 64, 128, 256}, ldt % 8 == 0, T * H < 2^29.
  */
 BL_API bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D, int64_t ldt, int bits,
                     int64_t bos_pos, float eps, uint8_t* codes, float* scale, uint8_t* bos_codes,

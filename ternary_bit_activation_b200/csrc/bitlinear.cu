@@ -875,7 +875,8 @@ bl_status bitlinear_gemm_gated(const void* a, bl_afmt afmt, const float* a_scale
 bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D, int64_t ldt, int bits, int64_t bos_pos,
                     float eps, uint8_t* codes, float* scale, uint8_t* bos_codes, void* stream) {
   if (bits != 3 && bits != 4) return BL_ERR_ARG;
-  if (T < 0 || H < 1 || D < 32 || D > 256 || (D & 31) || ldt < H * D || (ldt & 7)) return BL_ERR_SHAPE;
+  if (T < 0 || H < 1 || (D != 32 && D != 64 && D != 128 && D != 256) || ldt < H * D || (ldt & 7))
+    return BL_ERR_SHAPE;
   if (bos_pos < -1) return BL_ERR_ARG;
   if (!(eps >= 0.f)) return BL_ERR_ARG;
   if (T * H > 0x7FFFFFFFLL / 4 || H > 0x7FFFFFFF) return BL_ERR_SHAPE;   // 32-bit vector indices in the kernel
@@ -885,7 +886,7 @@ bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D, int64_
     return BL_ERR_NULL;
   if (!aligned16(kv_bf16) || !aligned16(codes) || !aligned16(scale) || (has_bos && !aligned16(bos_codes)))
     return BL_ERR_ALIGN;
-  const int tpv = static_cast<int>(D / 16);
+  const int tpv = static_cast<int>(D / 32);
   // persistent grid: eight CTAs per SM at most, each thread group kKvItems vectors per round
   const int64_t groups = (T * H + bl::kKvItems - 1) / bl::kKvItems;
   const int64_t need = (groups * tpv + 255) / 256;
@@ -896,10 +897,10 @@ bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D, int64_
   const int64_t bos = has_bos ? bos_pos : -1;
   const int h = static_cast<int>(H);
   switch (tpv) {
+    case 1: launch_pdl(bl::kv_quant_kernel<1>, grid, 256, 0, s, kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
     case 2: launch_pdl(bl::kv_quant_kernel<2>, grid, 256, 0, s, kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
     case 4: launch_pdl(bl::kv_quant_kernel<4>, grid, 256, 0, s, kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
     case 8: launch_pdl(bl::kv_quant_kernel<8>, grid, 256, 0, s, kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
-    case 16: launch_pdl(bl::kv_quant_kernel<16>, grid, 256, 0, s, kv, T, h, ldt, bits, bos, eps, codes, scale, bos_codes); break;
     default: return BL_ERR_SHAPE;
   }
   return launch_status();

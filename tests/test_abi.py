@@ -144,6 +144,7 @@ def test_pack_and_kv_validation(L):
     assert pn(P(A16), 8, 64, 64, 1e-5, 0, None, 0, P(A16), None) == 1
     kv = L.kv_quant3
     assert kv(P(A16), 8, 4, 100, 400, 3, 0, 1e-5, P(A16), P(A16), P(A16), None) == 3     # D % 32
+    assert kv(P(A16), 8, 4, 96, 384, 3, 0, 1e-5, P(A16), P(A16), P(A16), None) == 3      # D not a power of two
     assert kv(P(A16), 8, 4, 128, 512, 5, 0, 1e-5, P(A16), P(A16), P(A16), None) == 4     # bits
     assert kv(P(A16), 8, 4, 128, 512, 3, 0, 1e-5, P(A16), P(A16), None, None) == 1       # BOS buffer needed
 
