@@ -272,6 +272,22 @@ bool launch_simt(const uint8_t* a, const float* sc, const uint8_t* w, const floa
   return launch_simt_m<AF, WT2, 8>(a, sc, w, al, g, M, N, K, y, ldy, acc, s);
 }
 
+// CTAs of the exact-sum kernel resident per SM: its grid is one wave, so every
+// CTA streams to the end and flushes its bins once.
+int bins_ctas_per_sm() {
+  static int per_sm[kMaxDevices] = {};
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return 4;
+  if (per_sm[d] == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bl::ternary_bins_kernel, bl::kBinThreads, 0) != cudaSuccess ||
+        n < 1)
+      n = 1;
+    per_sm[d] = n;
+  }
+  return per_sm[d];
+}
+
 // Scratch of pack_ternary_noalloc: the exponent bins of the exact |W| sum, one
 // array per device that loads the library.  Host code only ever uses the device
 // address looked up below, never the symbol itself.
@@ -484,7 +500,7 @@ bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int64_t ldw
     if (!cuda_ok(cudaMemsetAsync(bins, 0, sizeof(g_noalloc_bins), s))) return BL_ERR_CUDA;
     const int64_t total = N * (K / 4);
     int64_t blocks = (total + bl::kBinThreads - 1) / bl::kBinThreads;
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * bins_ctas_per_sm();   // one resident wave
     if (blocks > cap) blocks = cap;
     launch_pdl(bl::ternary_bins_kernel, static_cast<unsigned>(blocks), bl::kBinThreads, 0, s, w, N, k, ldw, bins, alpha);
     if (launch_status() != BL_OK) return BL_ERR_CUDA;
@@ -615,7 +631,7 @@ bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float 
     if (!cuda_ok(cudaMemsetAsync(bins, 0, bl::kBins * sizeof(unsigned long long), s))) return BL_ERR_CUDA;
     const int64_t total = N * (K / 4);
     int64_t blocks = (total + bl::kBinThreads - 1) / bl::kBinThreads;
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * bins_ctas_per_sm();   // one resident wave
     if (blocks > cap) blocks = cap;
     launch_pdl(bl::ternary_bins_kernel, static_cast<unsigned>(blocks), bl::kBinThreads, 0, s, w, N, k, ldw, bins, alpha);
     if (launch_status() != BL_OK) return BL_ERR_CUDA;
