@@ -58,7 +58,7 @@ __device__ void alpha_from_bins(const unsigned long long* gbins, unsigned long l
 
 // gbins (zeroed by the caller): bins 1..255 and, in bin 0, a count of finished
 // CTAs; the last CTA to finish computes alpha.
-__global__ void __launch_bounds__(kBinThreads) ternary_bins_kernel(const float* __restrict__ w, int64_t N, int K,
+__global__ void __launch_bounds__(kBinThreads, 6) ternary_bins_kernel(const float* __restrict__ w, int64_t N, int K,
                                                                    int64_t ldw,
                                                                    unsigned long long* __restrict__ gbins,
                                                                    float* __restrict__ alpha) {
