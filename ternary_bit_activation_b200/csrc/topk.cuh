@@ -145,7 +145,7 @@ __device__ __forceinline__ void tk_keys(const uint4* st, int q, int row_words, u
 }
 
 template <bool F32>
-__global__ void __launch_bounds__(kTkThreads, F32 ? 2 : 4) topk_rows_kernel(
+__global__ void __launch_bounds__(kTkThreads, F32 ? 2 : 6) topk_rows_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ up, int64_t M, int K, int64_t ldx, int keep,
     float eps, int8_t* __restrict__ codes, float* __restrict__ scale, uint32_t* __restrict__ mask) {
   extern __shared__ __align__(16) uint8_t tk_dyn[];
