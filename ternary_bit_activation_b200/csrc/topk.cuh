@@ -3,10 +3,12 @@
 // ReLU^2-GLU output h = up * max(0, gate)^2 in fp32 (Eq. 5, relu2_glu).
 //
 // One 256-thread CTA owns one row at a time (persistent over rows).  Rows stream
-// through a double-buffered shared-memory stage (cp.async, 16 B per copy): the
-// next row is in flight while the current one is ranked and quantized, so HBM is
-// read once per element and stays busy.  For ReLU^2 rows the first sweep writes
-// h over the staged gate/up values of its own chunk, so later sweeps read h.
+// through a shared-memory stage (cp.async, 16 B per copy), so HBM is read once
+// per element.  bf16 rows are double-buffered: the next row is in flight while
+// the current one is ranked and quantized.  ReLU^2 rows (gate and up, 44 KB at
+// the 7B FFN width) take a single stage so that three CTAs fit on an SM; the
+// other CTAs' ranking covers each row's load.  For ReLU^2 rows the first sweep
+// writes h over the staged gate/up values of its own chunk, so later sweeps read h.
 //
 // Selection: exactly `keep` survivors ranked by magnitude, ties to the lower
 // index.  The keep-th largest magnitude key is found by an MSD radix select:
@@ -44,9 +46,13 @@ struct __align__(16) TkShared {
 };
 
 // Bytes of dynamic shared memory for rows of K values.
+// Row stages per CTA (see above).
+template <bool F32>
+constexpr int kTkStages = F32 ? 1 : 2;
+
 template <bool F32>
 inline size_t tk_smem_bytes(int K) {
-  return sizeof(TkShared<F32>) + 2 * static_cast<size_t>(F32 ? 2 : 1) * static_cast<size_t>(K) * 2;
+  return sizeof(TkShared<F32>) + kTkStages<F32> * static_cast<size_t>(F32 ? 2 : 1) * static_cast<size_t>(K) * 2;
 }
 
 // Counter update: `inc` (0 or 1) for digit `bin`.  Lanes l and l+16 share a
@@ -145,7 +151,7 @@ __device__ __forceinline__ void tk_keys(const uint4* st, int q, int row_words, u
 }
 
 template <bool F32>
-__global__ void __launch_bounds__(kTkThreads, F32 ? 2 : 6) topk_rows_kernel(
+__global__ void __launch_bounds__(kTkThreads, F32 ? 3 : 6) topk_rows_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ up, int64_t M, int K, int64_t ldx, int keep,
     float eps, int8_t* __restrict__ codes, float* __restrict__ scale, uint32_t* __restrict__ mask) {
   extern __shared__ __align__(16) uint8_t tk_dyn[];
@@ -194,9 +200,13 @@ __global__ void __launch_bounds__(kTkThreads, F32 ? 2 : 6) topk_rows_kernel(
   int64_t row = blockIdx.x;
   prefetch(row, 0);
   int buf = 0;
-  for (; row < M; row += gridDim.x, buf ^= 1) {
-    prefetch(row + gridDim.x, buf ^ 1);
-    asm volatile("cp.async.wait_group 1;" ::: "memory");
+  for (; row < M; row += gridDim.x, buf ^= kTkStages<F32> - 1) {
+    if constexpr (kTkStages<F32> == 2) {
+      prefetch(row + gridDim.x, buf ^ 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
     __syncthreads();
     uint4* st = stages + buf * stage_words;
 
@@ -438,6 +448,7 @@ __global__ void __launch_bounds__(kTkThreads, F32 ? 2 : 6) topk_rows_kernel(
       }
     }
     __syncthreads();   // the stage and the shared state are reused
+    if constexpr (kTkStages<F32> == 1) prefetch(row + gridDim.x, 0);
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
