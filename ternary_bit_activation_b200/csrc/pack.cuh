@@ -79,6 +79,14 @@ __global__ void __launch_bounds__(kBinThreads, 6) ternary_bins_kernel(const floa
   for (int64_t n = gwarp; n < N; n += nwarps) {
     const float* wrow = w + n * ldw;
     for (int q0 = 0; q0 < per_row; q0 += 32 * kLoads) {
+      // lane 0 asks L2 for the row's batch two ahead (and, at the row's start,
+      // the next one too), so each warp keeps three batches in flight
+      if (lane == 0) {
+        for (int qa = q0 == 0 ? 32 * kLoads : 64 * kLoads; qa <= 64 * kLoads; qa += 32 * kLoads)
+          if (q0 + qa < per_row)
+            bulk_prefetch_l2(wrow + static_cast<int64_t>(q0 + qa) * 4,
+                             static_cast<uint32_t>(min(32 * kLoads, per_row - q0 - qa)) * 16u);
+      }
       uint32_t u[4 * kLoads];
 #pragma unroll
       for (int j = 0; j < kLoads; ++j) {
