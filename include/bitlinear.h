@@ -20,6 +20,11 @@
  *   - Quantizers work per token (one row of X).  NaN/Inf inputs are outside the
  *     contract (results unspecified).
  *   - eps is the paper's "small constant" (1e-5 in the tests).
+ *   - Host threads: the first call that meets a kernel at a given shared-memory
+ *     size on a device raises that kernel's shared-memory limit and caches the
+ *     device's SM count; this setup is not synchronised between host threads.
+ *     Make calls from one host thread, or run each operation and shape once on
+ *     one thread before calling from several.
  */
 #ifndef BITLINEAR_H_
 #define BITLINEAR_H_
