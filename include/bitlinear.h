@@ -307,6 +307,15 @@ BL_API size_t bitlinear_workspace_size(const char* op, int64_t M, int64_t N, int
  * last call, BL_ERR_CUDA on a runtime error, BL_OK otherwise. */
 BL_API bl_status bitlinear_sync_status(void* stream);
 
+/* Diagnostic of the failure handling (no counterpart in the paper): enqueues
+ * one thread that waits, through the same bounded wait the tensor-core kernels
+ * and the streaming GEMV use, on an mbarrier that nothing completes.  After the
+ * wait limit (2 s) the thread gives up, records BL_ERR_TIMEOUT in the device
+ * status word and returns; the next bitlinear_sync_status() reports
+ * BL_ERR_TIMEOUT and clears it, and the context stays usable.  Returns the
+ * launch status. */
+BL_API bl_status bitlinear_selftest_timeout(void* stream);
+
 /* Human-readable name of a status code (static storage). */
 BL_API const char* bitlinear_status_string(bl_status status);
 

@@ -29,7 +29,7 @@ BL_W_T2, BL_W_I8, BL_W_E2M1 = 0, 1, 2
 
 EXPORTED = ["bitlinear_quant_a4", "bitlinear_sparsify_a8", "pack_ternary", "pack_ternary_noalloc", "bitlinear_gemm",
             "bitlinear_quant_gemm", "bitlinear_gemm_gated", "relu2_glu",
-            "kv_quant3", "bitlinear_workspace_size", "bitlinear_sync_status", "bitlinear_status_string",
+            "kv_quant3", "bitlinear_workspace_size", "bitlinear_sync_status", "bitlinear_selftest_timeout", "bitlinear_status_string",
             "bitlinear_last_cuda_error", "bitlinear_version"]
 
 _lib = None
@@ -63,6 +63,7 @@ def lib():
             "relu2_glu": [P, P, I64, I64, I64, I64, F, P, P, P, P],
             "kv_quant3": [P, I64, I64, I64, I64, I, I64, F, P, P, P, P],
             "bitlinear_sync_status": [P],
+            "bitlinear_selftest_timeout": [P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -187,6 +188,12 @@ def workspace_size(op: str, M: int = 0, N: int = 0, K: int = 0) -> int:
 def sync_status(stream=None):
     """Synchronize and raise if a kernel reported a timeout since the last check."""
     _check("bitlinear_sync_status", lib().bitlinear_sync_status(_stream(stream)))
+
+
+def selftest_timeout(stream=None):
+    """Enqueue a bounded wait that runs out (about 2 s); the next sync_status()
+    raises BitLinearError with status BL_ERR_TIMEOUT."""
+    _check("bitlinear_selftest_timeout", lib().bitlinear_selftest_timeout(_stream(stream)))
 
 
 def status_string(status: int) -> str:

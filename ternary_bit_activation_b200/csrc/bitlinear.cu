@@ -558,6 +558,11 @@ bl_status bitlinear_sync_status(void* stream) {
   return BL_OK;
 }
 
+bl_status bitlinear_selftest_timeout(void* stream) {
+  bl::bounded_wait_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>();
+  return launch_status();
+}
+
 bl_status bitlinear_quant_a4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, bl_quant quant, bl_store store,
                              float eps, void* codes, float* scale, void* stream) {
   if (quant != BL_QUANT_INT4 && quant != BL_QUANT_FP4_E2M1 && quant != BL_QUANT_INT4_ABSMAX &&

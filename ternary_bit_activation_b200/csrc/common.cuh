@@ -205,6 +205,17 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Self-test of the timeout path: one thread waits, through mbar_wait_bounded,
+// on an mbarrier that nothing ever completes.  The wait gives up after
+// kWaitLimitNs, raises BL_ERR_TIMEOUT, and the kernel returns normally.
+__global__ void bounded_wait_selftest_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbarrier_init();
+  mbar_wait_bounded(&bar, 0);
+}
+
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* smem_dst, int32_t x,
                                             int32_t y) {
   asm volatile(
