@@ -8,6 +8,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
+#ifndef BITLINEAR_NO_NVTX
+#include <nvtx3/nvToolsExt.h>
+#endif
 
 #include "bitlinear.h"
 #include "common.cuh"
@@ -27,6 +30,27 @@ static_assert(int{BL_QUANT_INT4} == bl::kQInt4 && int{BL_QUANT_FP4_E2M1} == bl::
 constexpr int kMaxDevices = 64;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// An NVTX range named after the entry point around every call that enqueues
+// work, so that a profiler groups each call's kernels under its name.  Without a
+// tool attached the push and pop are no-ops; -DBITLINEAR_NO_NVTX compiles them out.
+class NvtxRange {
+ public:
+  explicit NvtxRange(const char* name) {
+#ifndef BITLINEAR_NO_NVTX
+    nvtxRangePushA(name);
+#else
+    (void)name;
+#endif
+  }
+  ~NvtxRange() {
+#ifndef BITLINEAR_NO_NVTX
+    nvtxRangePop();
+#endif
+  }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -485,6 +509,7 @@ extern "C" {
 
 bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int64_t ldw, float eps, int alpha_given,
                                float* alpha, bl_wfmt wfmt, void* w_out, void* stream) {
+  NvtxRange nvtx_range("pack_ternary_noalloc");
   if (wfmt != BL_W_T2 && wfmt != BL_W_I8 && wfmt != BL_W_E2M1) return BL_ERR_ARG;
   if (N < 0 || K < 16 || (K & 15) || ldw < K || (ldw & 3) || K > 0x7FFFFFFF) return BL_ERR_SHAPE;
   if (N > 0 && N * K >= kNoallocMaxElems) return BL_ERR_SHAPE;
@@ -565,6 +590,7 @@ bl_status bitlinear_selftest_timeout(void* stream) {
 
 bl_status bitlinear_quant_a4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, bl_quant quant, bl_store store,
                              float eps, void* codes, float* scale, void* stream) {
+  NvtxRange nvtx_range("bitlinear_quant_a4");
   if (quant != BL_QUANT_INT4 && quant != BL_QUANT_FP4_E2M1 && quant != BL_QUANT_INT4_ABSMAX &&
       quant != BL_QUANT_INT4_ABSMEAN2 && quant != BL_QUANT_FP4_E1M2)
     return BL_ERR_ARG;
@@ -591,6 +617,7 @@ bl_status bitlinear_quant_a4(const void* x_bf16, int64_t M, int64_t K, int64_t l
 
 bl_status bitlinear_sparsify_a8(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, int64_t k_keep, float eps,
                                 int8_t* codes, float* scale, uint32_t* mask, void* stream) {
+  NvtxRange nvtx_range("bitlinear_sparsify_a8");
   if (M < 0 || K < 8 || K > 16384 || (K & 7) || ldx < K || (ldx & 7) || M > 0x7FFFFFFFLL) return BL_ERR_SHAPE;
   if (k_keep < 1 || k_keep > K) return BL_ERR_ARG;
   if (!(eps >= 0.f)) return BL_ERR_ARG;
@@ -603,6 +630,7 @@ bl_status bitlinear_sparsify_a8(const void* x_bf16, int64_t M, int64_t K, int64_
 
 bl_status relu2_glu(const void* gate_bf16, const void* up_bf16, int64_t M, int64_t F, int64_t ld, int64_t k_keep,
                     float eps, int8_t* codes, float* scale, uint32_t* mask, void* stream) {
+  NvtxRange nvtx_range("relu2_glu");
   if (M < 0 || F < 8 || F > 16384 || (F & 7) || ld < F || (ld & 7) || M > 0x7FFFFFFFLL) return BL_ERR_SHAPE;
   if (k_keep < 1 || k_keep > F) return BL_ERR_ARG;
   if (!(eps >= 0.f)) return BL_ERR_ARG;
@@ -619,6 +647,7 @@ bl_status relu2_glu(const void* gate_bf16, const void* up_bf16, int64_t M, int64
 
 bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float eps, int alpha_given, float* alpha,
                        bl_wfmt wfmt, void* w_out, void* workspace, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("pack_ternary");
   if (wfmt != BL_W_T2 && wfmt != BL_W_I8 && wfmt != BL_W_E2M1) return BL_ERR_ARG;
   if (N < 0 || K < 16 || (K & 15) || ldw < K || (ldw & 3)) return BL_ERR_SHAPE;
   if (N > 0 && (N * K >= bl::kMaxPackElems || K > 0x7FFFFFFF)) return BL_ERR_SHAPE;
@@ -658,6 +687,7 @@ bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float 
 bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scale, const void* w, bl_wfmt wfmt,
                          const float* alpha, int64_t alpha_group, int64_t M, int64_t N, int64_t K, void* y_bf16,
                          int64_t ldy, int32_t* acc_out, void* stream) {
+  NvtxRange nvtx_range("bitlinear_gemm");
   if (afmt != BL_A_I8 && afmt != BL_A_I4 && afmt != BL_A_E2M1) return BL_ERR_ARG;
   if (wfmt != BL_W_T2 && wfmt != BL_W_I8 && wfmt != BL_W_E2M1) return BL_ERR_ARG;
   if (alpha_group < 1 || alpha_group > 0x7FFFFFFFLL) return BL_ERR_ARG;
@@ -822,6 +852,7 @@ bl_status bitlinear_quant_gemm(const void* x_bf16, int64_t ldx, bl_quant quant, 
                                bl_wfmt wfmt, const float* alpha, int64_t alpha_group, int64_t M, int64_t N, int64_t K,
                                void* y_bf16, int64_t ldy, int32_t* acc_out, void* workspace, size_t ws_bytes,
                                void* stream) {
+  NvtxRange nvtx_range("bitlinear_quant_gemm");
   if (quant != BL_QUANT_INT4 && quant != BL_QUANT_FP4_E2M1) return BL_ERR_ARG;
   if (wfmt != BL_W_T2 && wfmt != BL_W_I8) return BL_ERR_ARG;
   if (alpha_group < 1 || alpha_group > 0x7FFFFFFFLL || !(eps >= 0.f)) return BL_ERR_ARG;
@@ -861,6 +892,7 @@ bl_status bitlinear_quant_gemm(const void* x_bf16, int64_t ldx, bl_quant quant, 
 bl_status bitlinear_gemm_gated(const void* a, bl_afmt afmt, const float* a_scale, const void* w, bl_wfmt wfmt,
                                const float* alpha, int64_t M, int64_t F, int64_t K, void* y_bf16, int64_t ldy,
                                int32_t* acc_out, void* stream) {
+  NvtxRange nvtx_range("bitlinear_gemm_gated");
   if (afmt != BL_A_I8 && afmt != BL_A_I4 && afmt != BL_A_E2M1) return BL_ERR_ARG;
   if (wfmt != BL_W_T2) return BL_ERR_UNSUPPORTED;
   if (M < 0 || F < 1 || K < 64 || (K & 63) || F > 0x3FFFFFFFLL || ldy < 2 * F || (ldy & 7)) return BL_ERR_SHAPE;
@@ -895,6 +927,7 @@ bl_status bitlinear_gemm_gated(const void* a, bl_afmt afmt, const float* a_scale
 
 bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D, int64_t ldt, int bits, int64_t bos_pos,
                     float eps, uint8_t* codes, float* scale, uint8_t* bos_codes, void* stream) {
+  NvtxRange nvtx_range("kv_quant3");
   if (bits != 3 && bits != 4) return BL_ERR_ARG;
   if (T < 0 || H < 1 || (D != 32 && D != 64 && D != 128 && D != 256) || ldt < H * D || (ldt & 7))
     return BL_ERR_SHAPE;
