@@ -44,3 +44,35 @@ def bf16_rows_rel_err(y_gpu_bits: np.ndarray, exact: np.ndarray) -> float:
 
 # bf16 outputs: relative error per row (max |err| over the row's fp64 norm)
 BF16_ROW_TOL = 1e-2
+
+
+# Out-of-bounds write check without a sanitizer: an output tensor sits inside a
+# larger byte buffer; the margins on both sides and the tensor itself start as
+# CANARY bytes, and after the call the margins must still hold them.
+CANARY = 0xA5
+CANARY_PAD = 4096       # bytes on each side; a multiple of 16 keeps the tensor aligned
+
+
+def canaried(shape, dtype, dev=None):
+    """(tensor of `shape` and `dtype`, the buffer around it), all bytes CANARY."""
+    dev = device() if dev is None else dev
+    nbytes = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+    buf = torch.full((2 * CANARY_PAD + nbytes,), CANARY, dtype=torch.uint8, device=dev)
+    return buf[CANARY_PAD:CANARY_PAD + nbytes].view(dtype).view(*shape), buf
+
+
+def canary_margins_intact(t: torch.Tensor, buf: torch.Tensor) -> bool:
+    """True if no byte of buf outside tensor t differs from CANARY."""
+    if buf.is_cuda:
+        torch.cuda.synchronize()
+    b = buf.cpu().numpy()
+    nbytes = t.numel() * t.element_size()
+    return bool(np.all(b[:CANARY_PAD] == CANARY) and np.all(b[CANARY_PAD + nbytes:] == CANARY))
+
+
+def canary_bytes(t: torch.Tensor) -> np.ndarray:
+    """The bytes of tensor t, row by row (uint8 [rows x row bytes])."""
+    if t.is_cuda:
+        torch.cuda.synchronize()
+    a = t.detach().cpu().contiguous().view(torch.uint8).numpy()
+    return a.reshape(t.shape[0], -1) if t.dim() > 1 else a.reshape(1, -1)
