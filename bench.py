@@ -354,6 +354,20 @@ class Layer:
                 sum(h.numel() * h.element_size() for h in self.h_out))
 
 
+def zero_fractions(torch, layer) -> dict:
+    """Per projection, the fraction of zero codes in its quantized input after
+    the last step, and the fraction of gate pre-activations that ReLU^2 zeroes:
+    the sparsity the paper tabulates per projection (here of synthetic data)."""
+    def frac(is_zero):
+        return round(float(is_zero.sum().item()) / is_zero.numel(), 4)
+    out = {"o_input": frac(layer.o8 == 0), "down_input": frac(layer.h8 == 0),
+           "gate_relu_zero": frac(layer.y_ug[:, layer.f:].view(torch.bfloat16) <= 0)}
+    if layer.afmt == "int4":   # byte layout: one code per byte
+        out["qkv_input"] = frac(layer.qa == 0)
+        out["upgate_input"] = frac(layer.qf == 0)
+    return out
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -489,6 +503,7 @@ def run_gpu(args):
                     "ms_per_step": round(e2e_ms / args.steps, 4)},
             "gpu_launches": layer.launches_per_step * args.steps,
             "clocks": clk,
+            "zero_fraction": zero_fractions(torch, layer),
         }
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(args.afmt, tokens_sample=args.cpu_tokens)

@@ -41,3 +41,25 @@ def test_weak_scaling_throughput():
     # 2 ranks x 32768 tokens x 10 steps in 1 s of the slowest rank
     assert bench.weak_scaling_throughput(2, 32768, 10, 1000.0) == pytest.approx(655360.0)
     assert bench.weak_scaling_throughput(1, 32768, 10, 2000.0) == pytest.approx(163840.0)
+
+
+def test_zero_fractions_of_a_step():
+    """bench.zero_fractions on CPU tensors shaped and typed like a Layer's
+    buffers: counts zero codes per projection input and non-positive gates."""
+    from types import SimpleNamespace
+    m, f, d = 4, 8, 16
+    o8 = torch.ones((m, d), dtype=torch.int8)
+    o8[:, ::2] = 0                                            # half zeros
+    h8 = torch.zeros((m, f), dtype=torch.int8)
+    h8[0, 0] = 5                                              # 31 of 32 zeros
+    up = torch.full((m, f), 1.0, dtype=torch.bfloat16)
+    gate = torch.tensor([[-1.0, 0.0, -0.0, 2.0] * 2] * m, dtype=torch.bfloat16)   # 3 of 4 zeroed by ReLU
+    y_ug = torch.cat([up, gate], dim=1).view(torch.int16)
+    qa = torch.zeros((m, d), dtype=torch.uint8)
+    qf = torch.full((m, d), 3, dtype=torch.uint8)
+    layer = SimpleNamespace(o8=o8, h8=h8, y_ug=y_ug, f=f, qa=qa, qf=qf, afmt="int4")
+    z = bench.zero_fractions(torch, layer)
+    assert z == {"o_input": 0.5, "down_input": round(31 / 32, 4), "gate_relu_zero": 0.75,
+                 "qkv_input": 1.0, "upgate_input": 0.0}
+    layer.afmt = "fp4"
+    assert set(bench.zero_fractions(torch, layer)) == {"o_input", "down_input", "gate_relu_zero"}
