@@ -28,8 +28,8 @@ BL_A_I8, BL_A_I4, BL_A_E2M1 = 0, 1, 2
 BL_W_T2, BL_W_I8, BL_W_E2M1 = 0, 1, 2
 
 EXPORTED = ["bitlinear_quant_a4", "bitlinear_sparsify_a8", "pack_ternary", "pack_ternary_noalloc", "bitlinear_gemm",
-            "bitlinear_quant_gemm", "bitlinear_gemm_gated", "relu2_glu",
-            "kv_quant3", "bitlinear_workspace_size", "bitlinear_sync_status", "bitlinear_selftest_timeout", "bitlinear_status_string",
+            "bitlinear_quant_gemm", "bitlinear_gemm_gated", "relu2_glu", "kv_quant3", "bitlinear_workspace_size",
+            "bitlinear_sync_status", "bitlinear_selftest_timeout", "bitlinear_status_string",
             "bitlinear_last_cuda_error", "bitlinear_version"]
 
 _lib = None
