@@ -171,8 +171,11 @@ BL_API bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw,
  * bit-identical); the scratch is cleared at the start of every call.
  * Limits: N * K < 2^31, so no 64-bit bin can overflow; larger tensors are
  * rejected with BL_ERR_SHAPE.  The first call on a device looks up the
- * array's device address (once per device); make that first call before any
- * stream capture.  Every call on a device shares the one array, so calls that
+ * array's device address (once per device) and caches it; make that first
+ * call before any stream capture.  The cached address belongs to the device's
+ * current primary context: after cudaDeviceReset() on that device it is stale,
+ * so do not call this function again in that process after a reset.  Every
+ * call on a device shares the one array, so calls that
  * can overlap on that GPU (different streams, no ordering between them) race
  * and must be serialized by the caller.  Allocates nothing.
  */

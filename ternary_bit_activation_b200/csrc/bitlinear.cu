@@ -319,7 +319,9 @@ static __device__ __align__(256) unsigned long long g_noalloc_bins[bl::kBins];
 constexpr int64_t kNoallocMaxElems = bl::kMaxPackElems;  // keeps every 64-bit bin below overflow
 
 // Device address of g_noalloc_bins on the current device, looked up once per
-// device (with that device current) and cached.
+// device (with that device current) and cached.  The cache outlives the
+// device's primary context: after a cudaDeviceReset the address is stale (the
+// header says so).
 unsigned long long* noalloc_bins_ptr() {
   static unsigned long long* cached[kMaxDevices] = {nullptr};
   const int d = current_device();
@@ -512,7 +514,8 @@ bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int64_t ldw
   NvtxRange nvtx_range("pack_ternary_noalloc");
   if (wfmt != BL_W_T2 && wfmt != BL_W_I8 && wfmt != BL_W_E2M1) return BL_ERR_ARG;
   if (N < 0 || K < 16 || (K & 15) || ldw < K || (ldw & 3) || K > 0x7FFFFFFF) return BL_ERR_SHAPE;
-  if (N > 0 && N * K >= kNoallocMaxElems) return BL_ERR_SHAPE;
+  // N * K >= limit, tested without forming the product (which can overflow)
+  if (N > 0 && N >= (kNoallocMaxElems + K - 1) / K) return BL_ERR_SHAPE;
   if (!(eps >= 0.f)) return BL_ERR_ARG;
   if (N == 0) return BL_OK;
   if (w == nullptr || alpha == nullptr || w_out == nullptr) return BL_ERR_NULL;
@@ -649,8 +652,9 @@ bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float 
                        bl_wfmt wfmt, void* w_out, void* workspace, size_t ws_bytes, void* stream) {
   NvtxRange nvtx_range("pack_ternary");
   if (wfmt != BL_W_T2 && wfmt != BL_W_I8 && wfmt != BL_W_E2M1) return BL_ERR_ARG;
-  if (N < 0 || K < 16 || (K & 15) || ldw < K || (ldw & 3)) return BL_ERR_SHAPE;
-  if (N > 0 && (N * K >= bl::kMaxPackElems || K > 0x7FFFFFFF)) return BL_ERR_SHAPE;
+  if (N < 0 || K < 16 || (K & 15) || ldw < K || (ldw & 3) || K > 0x7FFFFFFF) return BL_ERR_SHAPE;
+  // N * K >= limit, tested without forming the product (which can overflow)
+  if (N > 0 && N >= (bl::kMaxPackElems + K - 1) / K) return BL_ERR_SHAPE;
   if (!(eps >= 0.f)) return BL_ERR_ARG;
   if (N == 0) return BL_OK;
   if (w == nullptr || alpha == nullptr || w_out == nullptr) return BL_ERR_NULL;

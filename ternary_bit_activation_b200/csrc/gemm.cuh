@@ -278,13 +278,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   }
 
-  __syncthreads();
-  if (aborted) {
-    // let any copies or MMAs still in flight land before the CTA's memory goes away
+  // One decision for the whole CTA: if any thread gave up on a wait, every
+  // thread waits out the drain together, so the warp-wide dealloc below runs
+  // converged and only after copies or MMAs still in flight have landed.
+  if (__syncthreads_or(aborted ? 1 : 0)) {
     const uint64_t t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 200000ull) {
     }
   }
+  __syncwarp();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTcTmemCols);
@@ -576,12 +578,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT2Threads, 1)
     }
   }
 
-  __syncthreads();
-  if (aborted) {
+  // CTA-wide abort decision (see gemm_tc_kernel): the drain is taken by every
+  // thread or by none, before the aligned cluster barrier and the dealloc.
+  if (__syncthreads_or(aborted ? 1 : 0)) {
     const uint64_t t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 200000ull) {
     }
   }
+  __syncwarp();
   tc_fence_before();
   cluster_sync_all();   // no CTA leaves while its peer may still signal its barriers
   tc_fence_after();
@@ -881,13 +885,13 @@ __global__ void __launch_bounds__(kTsThreads, 1)
     }
   }
 
-  __syncthreads();
-  if (aborted) {
-    // let any copies or MMAs still in flight land before the CTA's memory goes away
+  // CTA-wide abort decision (see gemm_tc_kernel)
+  if (__syncthreads_or(aborted ? 1 : 0)) {
     const uint64_t t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 200000ull) {
     }
   }
+  __syncwarp();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);

@@ -140,6 +140,12 @@ def test_pack_and_kv_validation(L):
     assert pk(P(A16), 8, 64, 64, 1e-5, 0, P(A16), 5, P(A16), P(A16), 2048, None) == 4
     pn = L.pack_ternary_noalloc
     assert pn(P(A16), 1 << 16, 1 << 15, 1 << 15, 1e-5, 0, P(A16), 0, P(A16), None) == 3   # N*K >= 2^31
+    # a product N*K that wraps in 64 bits (2^62 * 64 = 2^68) must not slip past the limit
+    assert pn(P(A16), 1 << 62, 64, 64, 1e-5, 0, P(A16), 0, P(A16), None) == 3
+    assert pk(P(A16), 1 << 62, 64, 64, 1e-5, 0, P(A16), 0, P(A16), P(A16), 2048, None) == 3
+    # the largest accepted N for K = 16 is 2^27 - 1; 2^27 reaches 2^31 elements
+    assert pn(P(A16), 1 << 27, 16, 16, 1e-5, 0, P(A16), 0, P(A16), None) == 3
+    assert pk(P(A16), 1 << 27, 16, 16, 1e-5, 0, P(A16), 0, P(A16), P(A16), 2048, None) == 3
     assert pn(P(A16), 8, 24, 24, 1e-5, 0, P(A16), 0, P(A16), None) == 3                   # K % 16
     assert pn(P(A16), 8, 64, 64, 1e-5, 0, None, 0, P(A16), None) == 1
     kv = L.kv_quant3

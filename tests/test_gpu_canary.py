@@ -119,3 +119,72 @@ def test_gemm_in_bounds(M, N, K, wfmt):
     check(y, acc)
     # the columns between N and the row stride are not part of the output
     assert np.all(canary_bytes(y[0])[:, 2 * N:] == CANARY)
+
+
+def test_pack_ternary_noalloc_in_bounds():
+    N, K = 37, 336
+    w = (synth.rng(32).standard_normal((N, K)) * 0.02).astype(np.float32)
+    for wfmt, width in ((tba.BL_W_T2, 4), (tba.BL_W_E2M1, 2)):
+        out = canaried((N, K // width), torch.uint8)
+        alpha = canaried((1,), torch.float32)
+        tba.pack_ternary_noalloc(to_dev(w), alpha[0], out[0], wfmt, eps=EPS)
+        check(out, alpha)
+
+
+# (M, N, K): the fused-prologue decode GEMV (M <= 8, 2-bit weights) and the
+# quantizer-into-workspace path (M > 8, or int8 weights)
+QG_CASES = [(1, 300, 832, tba.BL_W_T2), (2, 37, 4096, tba.BL_W_T2), (7, 130, 640, tba.BL_W_T2),
+            (13, 300, 320, tba.BL_W_T2), (200, 300, 320, tba.BL_W_I8)]
+
+
+@pytest.mark.parametrize("quant", [tba.BL_QUANT_INT4, tba.BL_QUANT_FP4_E2M1], ids=["int4", "fp4"])
+@pytest.mark.parametrize("M,N,K,wfmt", QG_CASES, ids=[f"{c[0]}x{c[1]}x{c[2]}" for c in QG_CASES])
+def test_quant_gemm_in_bounds(quant, M, N, K, wfmt):
+    g = synth.rng(M * 11 + N + K)
+    x = synth.gaussian_bf16(g, (M, K))
+    t = g.integers(-1, 2, (N, K)).astype(np.int8)
+    w = oracle.pack_ternary2(t) if wfmt == tba.BL_W_T2 else t
+    ldy = (N + 7) // 8 * 8
+    y = canaried((M, ldy), torch.int16)
+    acc = canaried((M, N), torch.int32)
+    ws_bytes = tba.workspace_size("quant_gemm", M, N, K)
+    ws = canaried((ws_bytes,), torch.uint8)
+    al = to_dev(np.array([0.0211], np.float32))
+    tba.bitlinear_quant_gemm(to_dev(x), to_dev(w), al, M, N, K, y=y[0], acc=acc[0], quant=quant, wfmt=wfmt,
+                             eps=EPS, ldy=ldy, workspace=ws[0])
+    check(y, acc)
+    assert canary_margins_intact(*ws)
+    assert np.all(canary_bytes(y[0])[:, 2 * N:] == CANARY)
+
+
+@pytest.mark.parametrize("M,F,K", [(1, 37, 640), (2, 300, 4096), (2, 4, 64)])
+def test_gemm_gated_in_bounds(M, F, K):
+    g = synth.rng(M * 13 + F + K)
+    a = g.integers(-8, 8, (M, K)).astype(np.int8)
+    scale = (g.random(M) * 0.1 + 1e-3).astype(np.float32)
+    t = g.integers(-1, 2, (2 * F, K)).astype(np.int8)
+    ldy = (2 * F + 7) // 8 * 8 + 8
+    y = canaried((M, ldy), torch.int16)
+    acc = canaried((M, 2 * F), torch.int32)
+    al = to_dev(np.array([0.0211, 0.0187], np.float32))
+    tba.bitlinear_gemm_gated(to_dev(a), to_dev(scale), to_dev(oracle.pack_ternary2(t)), al, M, F, K, y[0],
+                             acc=acc[0], ldy=ldy)
+    check(y, acc)
+    assert np.all(canary_bytes(y[0])[:, 4 * F:] == CANARY)
+
+
+@pytest.mark.parametrize("M,N,K", [(200, 300, 320), (37, 230, 576), (300, 450, 4160)])
+def test_gemm_fp4_mxf4_in_bounds(M, N, K):
+    g = synth.rng(M * 17 + N + K)
+    x = synth.gaussian_bf16(g, (M, K))
+    codes, _, _, p2 = oracle.quant_fp4(x)
+    a = oracle.pack_nibbles(codes)
+    t = g.integers(-1, 2, (N, K)).astype(np.int8)
+    ldy = (N + 7) // 8 * 8
+    y = canaried((M, ldy), torch.int16)
+    acc = canaried((M, N), torch.int32)
+    al = to_dev(np.array([0.0211], np.float32))
+    tba.bitlinear_gemm(to_dev(a), to_dev(p2.astype(np.float32)), to_dev(oracle.pack_ternary_e2m1(t)), al, M, N, K,
+                       y=y[0], acc=acc[0], afmt=tba.BL_A_E2M1, wfmt=tba.BL_W_E2M1, ldy=ldy)
+    check(y, acc)
+    assert np.all(canary_bytes(y[0])[:, 2 * N:] == CANARY)

@@ -24,9 +24,13 @@ def _dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).to("cuda:0")
 
 
+def _width(wfmt):
+    return {tba.BL_W_T2: 4, tba.BL_W_E2M1: 2}.get(wfmt, 1)
+
+
 def _with_workspace(wd, wfmt):
     N, K = wd.shape
-    out = torch.empty((N, K // 4 if wfmt == tba.BL_W_T2 else K), dtype=torch.uint8, device=wd.device)
+    out = torch.empty((N, K // _width(wfmt)), dtype=torch.uint8, device=wd.device)
     alpha = torch.empty((1,), dtype=torch.float32, device=wd.device)
     ws = torch.empty((tba.workspace_size("pack_ternary") // 8,), dtype=torch.int64, device=wd.device)
     tba.pack_ternary(wd, alpha, out, wfmt=wfmt, workspace=ws)
@@ -34,12 +38,19 @@ def _with_workspace(wd, wfmt):
     return out.cpu().numpy(), alpha.cpu().numpy()
 
 
-def _no_alloc(wd, wfmt):
+def _no_alloc(wd, wfmt, alpha_in=None):
+    """Outputs are allocated first; the call itself must leave torch's caching
+    allocator exactly as it found it."""
     N, K = wd.shape
-    out = torch.empty((N, K // 4 if wfmt == tba.BL_W_T2 else K), dtype=torch.uint8, device=wd.device)
+    out = torch.empty((N, K // _width(wfmt)), dtype=torch.uint8, device=wd.device)
     alpha = torch.empty((1,), dtype=torch.float32, device=wd.device)
-    tba.pack_ternary_noalloc(wd, alpha, out, wfmt=wfmt)
+    if alpha_in is not None:
+        alpha.fill_(float(alpha_in))
+    torch.cuda.synchronize()
+    before = (torch.cuda.memory_allocated(), torch.cuda.memory_reserved())
+    tba.pack_ternary_noalloc(wd, alpha, out, wfmt=wfmt, alpha_given=alpha_in is not None)
     tba.sync_status()
+    assert (torch.cuda.memory_allocated(), torch.cuda.memory_reserved()) == before
     return out.cpu().numpy(), alpha.cpu().numpy()
 
 
@@ -59,3 +70,25 @@ def test_no_alloc_matches_workspace_variant_on_two_calls():
     second = _no_alloc(wd, tba.BL_W_I8)
     assert first[1].view(np.uint32)[0] == second[1].view(np.uint32)[0]
     assert np.array_equal(first[0], second[0])
+
+
+def test_no_alloc_e2m1_and_given_alpha_on_two_calls():
+    """The E2M1 weight layout (the FP4 tensor-core operand), and alpha_given,
+    which skips the static scratch altogether: both match pack_ternary."""
+    w = synth.latent_weights_f32(synth.rng(43), 1000, 4096)
+    wd = _dev(w)
+    ref_codes, ref_alpha = _with_workspace(wd, tba.BL_W_E2M1)
+    for _ in range(2):
+        codes, alpha = _no_alloc(wd, tba.BL_W_E2M1)
+        assert alpha.view(np.uint32)[0] == ref_alpha.view(np.uint32)[0]
+        assert np.array_equal(codes, ref_codes)
+    # a caller-given alpha: the codes follow it, the alpha is left as given
+    given = np.float32(ref_alpha[0] * np.float32(1.5))
+    ws_out = torch.empty((1000, 4096 // 4), dtype=torch.uint8, device="cuda:0")
+    al = torch.full((1,), float(given), dtype=torch.float32, device="cuda:0")
+    tba.pack_ternary(wd, al, ws_out, wfmt=tba.BL_W_T2, alpha_given=True)
+    tba.sync_status()
+    for _ in range(2):
+        codes, alpha = _no_alloc(wd, tba.BL_W_T2, alpha_in=given)
+        assert alpha.view(np.uint32)[0] == np.array([given], np.float32).view(np.uint32)[0]
+        assert np.array_equal(codes, ws_out.cpu().numpy())
