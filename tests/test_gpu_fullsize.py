@@ -292,3 +292,122 @@ def test_decode_layer_7b(decode_weights, m):
     assert np.array_equal(host(h8), c_h)
     assert np.array_equal(host(h8_s).view(np.uint32), s_h.view(np.uint32))
     gemm_stage(h8, tba.BL_A_I8, h8_s, "down", c_h, s_h, D, F)
+
+
+def test_gemm_upgate_full_7b(acts):
+    """The stacked Up|Gate GEMM as the benchmark runs it: N = 2F = 22016 rows
+    [W_up; W_gate] with one alpha per tensor (alpha_group = F), INT4 byte codes
+    of a Gaussian input, M = 32768; sampled rows against the oracle."""
+    x = acts[0]
+    wu = synth.latent_weights_f32(synth.rng(93), F, D)
+    wg = synth.latent_weights_f32(synth.rng(94), F, D)
+    t_up, a_up = oracle.ternary_quantize(wu, EPS)
+    t_gate, a_gate = oracle.ternary_quantize(wg, EPS)
+    w8 = empty((2 * F, D), torch.uint8)
+    alpha = empty((2,), torch.float32)
+    ws = empty((tba.workspace_size("pack_ternary") // 8,), torch.int64)
+    tba.pack_ternary(to_dev(wu), alpha[0:1], w8[:F], tba.BL_W_I8, ws, eps=EPS)
+    tba.pack_ternary(to_dev(wg), alpha[1:2], w8[F:], tba.BL_W_I8, ws, eps=EPS)
+    codes = empty((M, D), torch.uint8)
+    scale = empty((M,), torch.float32)
+    tba.bitlinear_quant_a4(to_dev(x), codes, scale, tba.BL_QUANT_INT4, tba.BL_STORE_BYTES, EPS)
+    y = empty((M, 2 * F), torch.int16)
+    acc = empty((M, 2 * F), torch.int32)
+    tba.bitlinear_gemm(codes, scale, w8, alpha, M, 2 * F, D, y=y, acc=acc, alpha_group=F)
+    tba.sync_status()
+    a_ref = np.array([a_up, a_gate], np.float32)
+    assert np.array_equal(host(alpha).view(np.uint32), a_ref.view(np.uint32))
+    rows = sample_rows(M, 24, 5)
+    c_ref, _, s_ref = oracle.quant_int4(x[rows], EPS)
+    assert np.array_equal(host(codes)[rows].view(np.int8), c_ref)
+    t_ref = np.concatenate([t_up, t_gate])
+    acc_ref, _ = oracle.gemm(c_ref, s_ref, t_ref, a_ref, alpha_group=F, want_y=False)
+    assert np.array_equal(host(acc)[rows], acc_ref)
+    al = np.repeat(a_ref.astype(np.float64), F)
+    exact = acc_ref.astype(np.float64) * s_ref[:, None].astype(np.float64) * al[None, :]
+    assert bf16_rows_rel_err(host(y, np.uint16)[rows], exact) <= BF16_ROW_TOL
+
+
+def test_gemm_o_full_7b_topk_codes(acts):
+    """The O GEMM as the benchmark runs it: the Top-K 50% INT8 codes of the
+    heavy-tailed O input (from the GPU quantizer) x int8 ternary weights,
+    M = 32768, N = K = 4096; sampled rows against the oracle."""
+    x = acts[1]
+    keep = synth.k_keep(D, S.topk_pct_o)
+    w = synth.latent_weights_f32(synth.rng(95), D, D)
+    t_ref, a_ref = oracle.ternary_quantize(w, EPS)
+    w8 = empty((D, D), torch.uint8)
+    alpha = empty((1,), torch.float32)
+    ws = empty((tba.workspace_size("pack_ternary") // 8,), torch.int64)
+    tba.pack_ternary(to_dev(w), alpha, w8, tba.BL_W_I8, ws, eps=EPS)
+    c8 = empty((M, D), torch.int8)
+    s8 = empty((M,), torch.float32)
+    tba.bitlinear_sparsify_a8(to_dev(x), keep, c8, s8, None, EPS)
+    y = empty((M, D), torch.int16)
+    acc = empty((M, D), torch.int32)
+    tba.bitlinear_gemm(c8, s8, w8, alpha, M, D, D, y=y, acc=acc)
+    tba.sync_status()
+    rows = sample_rows(M, 32, 6)
+    c_ref, _, _, s_ref = oracle.sparsify_a8(x[rows], keep, EPS)
+    assert np.array_equal(host(c8)[rows], c_ref)
+    acc_ref, _ = oracle.gemm(c_ref, s_ref, t_ref, a_ref, want_y=False)
+    assert np.array_equal(host(acc)[rows], acc_ref)
+    exact = acc_ref.astype(np.float64) * s_ref[:, None].astype(np.float64) * float(a_ref)
+    assert bf16_rows_rel_err(host(y, np.uint16)[rows], exact) <= BF16_ROW_TOL
+
+
+@pytest.mark.parametrize("m", [17, 32, 64, 128, 256])
+def test_decode_layer_7b_tensor_cores(decode_weights, m):
+    """Decode of 17-256 tokens as the decode benchmark runs it: one-byte INT4 /
+    Top-K INT8 codes against the 2-bit weights of all four 7B matrices, which
+    takes the tcgen05 kernel with the weights widened into tensor memory.
+    Every GPU stage reads the previous GPU stage's output; each product is
+    checked on a seeded sample of token rows (all N) against the oracle."""
+    ref, dev = decode_weights
+    x_attn, x_o, x_ffn = synth.layer_activations(S, seed=900 + m, tokens=m)
+    keep_o, keep_d = synth.k_keep(D, S.topk_pct_o), synth.k_keep(F, S.topk_pct_down)
+    rows = np.arange(m) if m <= 32 else sample_rows(m, 14, m)
+
+    def gemm_stage(a_dev, a_scale_dev, name, n, k, group=0):
+        acc = empty((m, n), torch.int32)
+        y = empty((m, n), torch.int16)
+        packed, alpha = dev[name]
+        tba.bitlinear_gemm(a_dev, a_scale_dev, packed, alpha, m, n, k, y=y, acc=acc, afmt=tba.BL_A_I8,
+                           wfmt=tba.BL_W_T2, alpha_group=group if group else n)
+        tba.sync_status()
+        t_ref, a_ref = ref[name]
+        a_codes = host(a_dev).view(np.int8)[rows]
+        a_scale = host(a_scale_dev)[rows]
+        acc_ref, _ = oracle.gemm(a_codes, a_scale, t_ref, a_ref, alpha_group=group, want_y=False)
+        assert np.array_equal(host(acc)[rows], acc_ref), name
+        al = np.repeat(a_ref.astype(np.float64), group if group else n)[:n]
+        exact = acc_ref.astype(np.float64) * a_scale[:, None].astype(np.float64) * al[None, :]
+        assert bf16_rows_rel_err(host(y, np.uint16)[rows], exact) <= BF16_ROW_TOL, name
+        return y
+
+    def quant4(x):
+        qa = empty((m, D), torch.int8)
+        qs = empty((m,), torch.float32)
+        tba.bitlinear_quant_a4(to_dev(x), qa, qs, tba.BL_QUANT_INT4, tba.BL_STORE_BYTES, EPS)
+        tba.sync_status()
+        c, _, s = oracle.quant_int4(x, EPS)
+        assert np.array_equal(host(qa), c)
+        assert np.array_equal(host(qs).view(np.uint32), s.view(np.uint32))
+        return qa, qs
+
+    qa, qs = quant4(x_attn)
+    gemm_stage(qa, qs, "qkv", 3 * D, D)
+    o8 = empty((m, D), torch.int8)
+    o8_s = empty((m,), torch.float32)
+    tba.bitlinear_sparsify_a8(to_dev(x_o), keep_o, o8, o8_s, None, EPS)
+    gemm_stage(o8, o8_s, "o", D, D)
+    qf, qfs = quant4(x_ffn)
+    y_ug = gemm_stage(qf, qfs, "upgate", 2 * F, D, group=F)
+    h8 = empty((m, F), torch.int8)
+    h8_s = empty((m,), torch.float32)
+    tba.relu2_glu(y_ug[:, F:], y_ug[:, :F], keep_d, h8, h8_s, None, EPS, M=m, F=F, ld=2 * F)
+    tba.sync_status()
+    ug = host(y_ug, np.uint16)[rows]
+    c_h, _, _, s_h = oracle.relu2_glu(np.ascontiguousarray(ug[:, F:]), np.ascontiguousarray(ug[:, :F]), keep_d, EPS)
+    assert np.array_equal(host(h8)[rows], c_h)
+    gemm_stage(h8, h8_s, "down", D, F)
