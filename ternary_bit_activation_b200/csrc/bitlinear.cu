@@ -239,6 +239,39 @@ bl_status launch_topk_rows(const uint16_t* x, const uint16_t* up, int64_t M, int
   return launch_status();
 }
 
+// Top-K rows of up to 4096 bf16 values: one warp per row (persistent, four warps
+// per CTA, as many CTAs as are resident); C = 16-byte chunks per lane.
+template <int C>
+bl_status launch_topk_warp_c(const uint16_t* x, int64_t M, int K, int64_t ldx, int keep, float eps, int8_t* codes,
+                             float* scale, uint32_t* mask, cudaStream_t s) {
+  auto kern = bl::topk_warp_kernel<C>;
+  constexpr size_t smem = bl::tw_smem_bytes<C>();
+  static int per_sm[kMaxDevices] = {};
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return BL_ERR_CUDA;
+  if (per_sm[d] == 0) {
+    if (!cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))))
+      return BL_ERR_CUDA;
+    int n = 0;
+    if (!cuda_ok(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * bl::kTwWarps, smem))) return BL_ERR_CUDA;
+    per_sm[d] = n < 1 ? 1 : n;
+  }
+  const int64_t need = (M + bl::kTwWarps - 1) / bl::kTwWarps;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm[d];
+  const unsigned grid = static_cast<unsigned>(need < cap ? need : cap);
+  launch_pdl(kern, grid, 32 * bl::kTwWarps, smem, s, x, M, K, ldx, keep, eps, codes, scale, mask);
+  return launch_status();
+}
+
+bl_status launch_topk_warp(const uint16_t* x, int64_t M, int K, int64_t ldx, int keep, float eps, int8_t* codes,
+                           float* scale, uint32_t* mask, cudaStream_t s) {
+  const int per_lane = (K / 8 + 31) / 32;
+  if (per_lane <= 1) return launch_topk_warp_c<1>(x, M, K, ldx, keep, eps, codes, scale, mask, s);
+  if (per_lane <= 2) return launch_topk_warp_c<2>(x, M, K, ldx, keep, eps, codes, scale, mask, s);
+  if (per_lane <= 4) return launch_topk_warp_c<4>(x, M, K, ldx, keep, eps, codes, scale, mask, s);
+  if (per_lane <= 8) return launch_topk_warp_c<8>(x, M, K, ldx, keep, eps, codes, scale, mask, s);
+  return launch_topk_warp_c<16>(x, M, K, ldx, keep, eps, codes, scale, mask, s);
+}
 
 template <int AF, bool WT2, int MT, int UPL>
 bool launch_simt_mu(const uint8_t* a, const float* sc, const uint8_t* w, const float* al, int64_t g, int M, int N,
@@ -627,6 +660,9 @@ bl_status bitlinear_sparsify_a8(const void* x_bf16, int64_t M, int64_t K, int64_
   if (M == 0) return BL_OK;
   if (x_bf16 == nullptr || codes == nullptr || scale == nullptr) return BL_ERR_NULL;
   if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scale) || (mask && !aligned16(mask))) return BL_ERR_ALIGN;
+  if (K <= bl::kTwMaxK)
+    return launch_topk_warp(static_cast<const uint16_t*>(x_bf16), M, static_cast<int>(K), ldx, static_cast<int>(k_keep),
+                            eps, codes, scale, mask, as_stream(stream));
   return launch_topk_rows<false>(static_cast<const uint16_t*>(x_bf16), nullptr, M, static_cast<int>(K), ldx,
                                  static_cast<int>(k_keep), eps, codes, scale, mask, as_stream(stream));
 }

@@ -454,3 +454,415 @@ __global__ void __launch_bounds__(kTkThreads, F32 ? 3 : 6) topk_rows_kernel(
 }
 
 }  // namespace bl
+
+namespace bl {
+
+// ---------------------------------------------------------------------------
+// Top-K + INT8 for bf16 rows of up to 4096 values: one warp per row, the row in
+// registers (lane l holds the 16-byte chunks 32q + l, q < C), no shared memory
+// and no block barrier.
+//
+// The keep-th largest magnitude key thr is found by counting probes: count(t) =
+// #{|x| >= t} over the row, one packed bf16x2 comparison per two values
+// (set.ge.u32.bf16x2 writes 0xFFFF per true half; the sum of those masks over a
+// lane's words still tells how many low and how many high halves were true),
+// summed over the warp.  count(0) = K and count(max + 1) = 0 bracket thr; the
+// first probes come from a sorted sample of 32 values at the target quantile,
+// the next ones interpolate the counts linearly between the bracket's ends, and
+// a probe that fails to halve the bracket makes the next one a bisection, so the
+// search ends (at most two probes per halving of the 15-bit key range) with
+// count(thr) >= keep > count(thr + 1).  Values above thr survive; of the values
+// equal to thr the first keep - count(thr + 1) in index order survive, ranked
+// by a warp scan over the chunks in index order.  Values past K (a ragged last
+// chunk round) are a bf16 NaN, which no comparison counts.
+// ---------------------------------------------------------------------------
+constexpr int kTwWarps = 4;                  // rows in flight per CTA
+constexpr int kTwMaxK = 4096;                // 16 chunks of 8 values per lane
+
+// Dynamic shared memory of topk_warp_kernel<C>: two row buffers per warp and
+// their mbarriers.
+template <int C>
+constexpr size_t tw_smem_bytes() {
+  return static_cast<size_t>(kTwWarps) * 2 * C * 32 * 16 + kTwWarps * 2 * 8;
+}
+
+// 0xFFFF in each 16-bit half where a >= b as bf16 values (a, b finite or NaN).
+__device__ __forceinline__ uint32_t bf2_ge_mask(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("set.ge.u32.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf2_gt_mask(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("set.gt.u32.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf2_eq_mask(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("set.eq.u32.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// 1.0 in each bf16 half where a >= b, else +0 (a, b finite or NaN).
+__device__ __forceinline__ uint32_t bf2_ge_one(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("set.ge.bf16x2.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+// Per-half bf16 sum (round to nearest; exact for the small counts added here).
+__device__ __forceinline__ uint32_t bf2_add(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+// Per-half bf16 maximum of two non-negative values.
+__device__ __forceinline__ uint32_t bf2_max(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// 1.0 in each bf16 half where a > b / a == b, else +0.
+__device__ __forceinline__ uint32_t bf2_gt_one(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("set.gt.bf16x2.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+// |a| per bf16 half (sign bits cleared; runs on the FMA pipe, not the ALU).
+__device__ __forceinline__ uint32_t bf2_abs(uint32_t a) {
+  uint32_t d;
+  asm("abs.bf16x2 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+// x * k - 0 in fp32 for the low (HI = false) or high bf16 halves of x and k:
+// with k = 1.0 or +0 this is x converted exactly, or a zero (one FMA-pipe
+// instruction for the conversion and the mask).
+template <bool HI>
+__device__ __forceinline__ float bf16_times_f32(uint32_t x, uint32_t k) {
+  float d;
+  if constexpr (HI)
+    asm("{\n\t.reg .b16 xl, xh, kl, kh;\n\tmov.b32 {xl, xh}, %1;\n\tmov.b32 {kl, kh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, xh, kh, 0f80000000;\n\t}"
+        : "=f"(d) : "r"(x), "r"(k));
+  else
+    asm("{\n\t.reg .b16 xl, xh, kl, kh;\n\tmov.b32 {xl, xh}, %1;\n\tmov.b32 {kl, kh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, xl, kl, 0f80000000;\n\t}"
+        : "=f"(d) : "r"(x), "r"(k));
+  return d;
+}
+// Four codes as bytes from the bit patterns b_i = bits(c_i + 1.5 * 2^23)
+// = 0x4B400000 + c_i (|c_i| <= 127): the sum of (c_i + 128) * 256^i has no carry
+// between bytes, and XOR 0x80 turns each c + 128 back into c's two's
+// complement byte.  Multiply-adds, so the work stays off the ALU.
+__device__ __forceinline__ uint32_t tw_pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  constexpr uint32_t kBias = 0u - 0x4B3FFF80u * 0x01010101u;   // -sum_i (0x4B400000 - 128) * 256^i
+  uint32_t wd = b0 + kBias;
+  wd = b1 * 0x100u + wd;
+  wd = b2 * 0x10000u + wd;
+  wd = b3 * 0x1000000u + wd;
+  return wd ^ 0x80808080u;
+}
+
+// PRMT with the selector's replicate bit: a selector nibble 8 + b yields 0xFF
+// if byte b of {b:a} has its top bit set, else 0 (__byte_perm ignores that bit).
+__device__ __forceinline__ uint32_t prmt_sign(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// s = the 32-bit sum of n per-half masks (each 0, 0xFFFF, 0xFFFF0000 or
+// 0xFFFFFFFF), n < 2^15: the number of true halves.  With A true low halves and
+// B true high halves, s = (A - B) * 2^16 - A (mod 2^32), so A = -s mod 2^16 and
+// A - B is the signed high half of s + A.
+__device__ __forceinline__ int tw_true_halves(uint32_t s) {
+  const uint32_t a = (0u - s) & 0xFFFFu;
+  const int d = static_cast<int16_t>(static_cast<uint16_t>((s + a) >> 16));
+  return 2 * static_cast<int>(a) - d;
+}
+
+// 16-byte load that bypasses L1 (volatile: stays behind pdl_wait).
+__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+// Four bytes that are 0 or 0xFF -> four bits (byte i -> bit i).
+__device__ __forceinline__ uint32_t tw_byte_bits(uint32_t m) { return ((m & 0x01010101u) * 0x01020408u) >> 24; }
+
+template <int C>
+__global__ void __launch_bounds__(32 * kTwWarps) topk_warp_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int K, int64_t ldx, int keep, float eps,
+    int8_t* __restrict__ codes, float* __restrict__ scale, uint32_t* __restrict__ mask) {
+  constexpr uint32_t kAbs = 0x7FFF7FFFu;
+  constexpr uint32_t kPadNaN = 0x7FC07FC0u;
+  // Two row buffers per warp: 1-D bulk copies bring the next row in while the
+  // current one is ranked and quantized.  The code pass reads the signed row
+  // from its buffer in a rolled loop (an unrolled one overflows the
+  // instruction cache); the probes read the |x| words from registers.
+  extern __shared__ __align__(128) uint4 tw_dyn[];
+  uint4 (*rowbuf)[2][C * 32] = reinterpret_cast<uint4 (*)[2][C * 32]>(tw_dyn);
+  uint64_t (*rowbar)[2] = reinterpret_cast<uint64_t (*)[2]>(tw_dyn + kTwWarps * 2 * C * 32);
+  const int lane = threadIdx.x & 31;
+  const int wig = threadIdx.x >> 5;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kTwWarps;
+  const int nchunk = K >> 3;
+  const int mbytes = ((K + 31) >> 5) * 4;
+  const uint32_t row_bytes = static_cast<uint32_t>(2 * K);
+  // the sample: word 0 of chunk round (lane % C), low half
+  const int qs = lane % C;
+  if (lane == 0) {
+    mbar_init(&rowbar[wig][0], 1);
+    mbar_init(&rowbar[wig][1], 1);
+    fence_mbarrier_init();
+  }
+  __syncwarp();
+  pdl_wait();
+  pdl_trigger();
+  int64_t row = static_cast<int64_t>(blockIdx.x) * kTwWarps + wig;
+  if (lane == 0 && row < M) {
+    mbar_arrive_expect_tx(&rowbar[wig][0], row_bytes);
+    bulk_load_1d(rowbuf[wig][0], x + row * ldx, row_bytes, &rowbar[wig][0]);
+  }
+  uint32_t phase = 0;                         // bit b: parity of buffer b's next completion
+  bool aborted = false;
+  for (int buf = 0; row < M; row += nwarps, buf ^= 1) {
+    if (lane == 0 && row + nwarps < M) {
+      // the other buffer was last read by the previous row (this warp, in order)
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive_expect_tx(&rowbar[wig][buf ^ 1], row_bytes);
+      bulk_load_1d(rowbuf[wig][buf ^ 1], x + (row + nwarps) * ldx, row_bytes, &rowbar[wig][buf ^ 1]);
+    }
+    // every lane waits for the copy; giving up is decided for the whole warp
+    if (__any_sync(0xFFFFFFFFu, !mbar_wait_bounded(&rowbar[wig][buf], (phase >> buf) & 1u))) {
+      aborted = true;
+      break;
+    }
+    phase ^= 1u << buf;
+    const uint4* rb = rowbuf[wig][buf];
+    // |x| words in registers (the probes' operand), NaN past K
+    uint32_t w[C][4];
+#pragma unroll
+    for (int q = 0; q < C; ++q) {
+      uint4 v = make_uint4(kPadNaN, kPadNaN, kPadNaN, kPadNaN);
+      if (32 * q + lane < nchunk) v = rb[32 * q + lane];
+      w[q][0] = bf2_abs(v.x);
+      w[q][1] = bf2_abs(v.y);
+      w[q][2] = bf2_abs(v.z);
+      w[q][3] = bf2_abs(v.w);
+    }
+    // row maximum of |x| (bf16 maxima of non-negative values order like the
+    // 15-bit keys; NaN padding excluded) and the sample; four independent
+    // partial results per lane keep the dependency chains short
+    uint32_t mxp[4] = {0, 0, 0, 0}, smp = 0;
+#pragma unroll
+    for (int q = 0; q < C; ++q) {
+      if (32 * q + lane < nchunk) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mxp[j] = bf2_max(mxp[j], w[q][j]);
+        if (q == qs) smp = w[q][0] & 0x7FFFu;
+      }
+    }
+    const uint32_t mx = bf2_max(bf2_max(mxp[0], mxp[1]), bf2_max(mxp[2], mxp[3]));
+    const uint32_t maxkey = __reduce_max_sync(0xFFFFFFFFu, max(mx & 0xFFFFu, mx >> 16));
+
+    // ---- threshold: count(thr) >= keep > count(thr + 1) ----
+    uint32_t lo = 0, hi = maxkey + 1;
+    int clo = K, chi = 0;
+    if (keep < K) {
+      // sorted sample (ascending over lanes, bitonic)
+#pragma unroll
+      for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+          const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, smp, j);
+          const bool take_min = ((lane & j) == 0) == ((lane & k) == 0);
+          smp = take_min ? min(smp, o) : max(smp, o);
+        }
+      }
+      // the target's position among 32 descending samples, and two steps either side
+      const int rs = static_cast<int>(((2 * static_cast<int64_t>(keep) - 1) * 32) / (2 * static_cast<int64_t>(K)));
+      const int ai = 31 - rs;
+      const uint32_t t_hi = __shfl_sync(0xFFFFFFFFu, smp, min(ai + 2, 31));
+      const uint32_t t_lo = __shfl_sync(0xFFFFFFFFu, smp, max(ai - 2, 0));
+      // count(t) for one or two thresholds in one pass over the row: packed
+      // compares give 1.0 / 0 per half, summed in bf16 on the FMA pipe in
+      // independent partial sums (at most 2C per half and sum: exact); the
+      // counts leave the bf16 sums through fp32 (exact) and the 2^23 trick
+      auto bf2_count = [](uint32_t a, uint32_t b) -> uint32_t {
+        const uint32_t sa = bf2_add(a, b);
+        const float f = __fadd_rn(__fadd_rn(__uint_as_float(sa << 16), __uint_as_float(sa & 0xFFFF0000u)), 8388608.f);
+        return static_cast<uint32_t>(__float_as_int(f) - 0x4B000000);
+      };
+      auto counts2 = [&](uint32_t t0, uint32_t t1, int& c0, int& c1) {
+        const uint32_t u0 = t0 | (t0 << 16), u1 = t1 | (t1 << 16);
+        uint32_t a[2] = {0, 0}, b[2] = {0, 0};
+#pragma unroll
+        for (int q = 0; q < C; ++q)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            a[j & 1] = bf2_add(a[j & 1], bf2_ge_one(w[q][j], u0));
+            b[j & 1] = bf2_add(b[j & 1], bf2_ge_one(w[q][j], u1));
+          }
+        const uint32_t r = __reduce_add_sync(0xFFFFFFFFu, bf2_count(a[0], a[1]) | (bf2_count(b[0], b[1]) << 16));
+        c0 = static_cast<int>(r & 0xFFFFu);   // two 16-bit sums (K <= 4096)
+        c1 = static_cast<int>(r >> 16);
+      };
+      auto count1 = [&](uint32_t t0) -> int {
+        const uint32_t u0 = t0 | (t0 << 16);
+        uint32_t a[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int q = 0; q < C; ++q)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) a[j] = bf2_add(a[j], bf2_ge_one(w[q][j], u0));
+        return static_cast<int>(
+            __reduce_add_sync(0xFFFFFFFFu, bf2_count(a[0], a[1]) + bf2_count(a[2], a[3])));
+      };
+      auto update = [&](uint32_t t, int c) {
+        if (t <= lo || t >= hi) return;
+        if (c >= keep) {
+          lo = t;
+          clo = c;
+        } else {
+          hi = t;
+          chi = c;
+        }
+      };
+      // the sample's two guesses in one pass
+      {
+        int c0, c1;
+        counts2(t_hi, t_lo, c0, c1);
+        update(t_hi, c0);
+        update(t_lo, c1);
+      }
+      bool bisect = false;
+#pragma unroll 1
+      while (hi - lo > 1) {
+        if (hi - lo <= 3) {
+          // the last one or two candidates in one pass
+          int c0, c1;
+          const uint32_t t0 = lo + 1, t1 = hi - 1;
+          counts2(t0, t1, c0, c1);
+          update(t0, c0);
+          update(t1, c1);
+          continue;
+        }
+        uint32_t t;
+        if (bisect) {
+          t = (lo + hi) >> 1;
+        } else {
+          // linear interpolation of the counts (any guess inside the bracket is correct)
+          const float f = __fdividef(static_cast<float>(clo) - (static_cast<float>(keep) - 0.5f),
+                                     static_cast<float>(clo - chi));
+          t = lo + static_cast<uint32_t>(__float2int_rn(f * static_cast<float>(hi - lo)));
+          t = min(max(t, lo + 1), hi - 1);
+        }
+        const uint32_t before = hi - lo;
+        update(t, count1(t));
+        bisect = 2 * (hi - lo) > before;
+      }
+    }
+    const uint32_t thr = lo;
+    const int take = keep - chi;            // ties at thr that survive
+    const bool partial = keep < K && take < clo - chi && (thr != 0u || mask != nullptr);
+
+    // ---- codes and mask, chunk rounds in index order ----
+    const float gamma = __uint_as_float(maxkey << 16);
+    const float denom = __fadd_rn(gamma, eps);
+    const float mult = denom > 0.f ? __fdiv_rn(127.f, denom) : 0.f;
+    if (lane == 0) scale[row] = __fdiv_rn(gamma, 127.f);
+    const uint32_t tt = thr | (thr << 16);
+    // the code of +thr and of -thr, four times over: every surviving tie has
+    // magnitude thr, so its code depends only on its sign
+    const uint32_t ct = tk_code_bits(__uint_as_float(thr << 16), mult) & 0xFFu;
+    const uint32_t ct_pos = ct * 0x01010101u, ct_neg = ((0u - ct) & 0xFFu) * 0x01010101u;
+    int8_t* crow = codes + row * static_cast<int64_t>(K);
+    uint8_t* mrow = mask != nullptr ? reinterpret_cast<uint8_t*>(mask) + row * static_cast<int64_t>(mbytes) : nullptr;
+    int running = 0;                         // ties in the rounds before
+#pragma unroll 1
+    for (int q = 0; q < C; ++q) {
+      const int c = 32 * q + lane;
+      const uint4 v = rb[c];
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+      uint32_t av[4], kp[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        av[j] = bf2_abs(wv[j]);
+        // 1.0 where the value survives for sure: above thr, or at thr when every tie does
+        kp[j] = partial ? bf2_gt_one(av[j], tt) : bf2_ge_one(av[j], tt);
+      }
+      // codes of the surviving values, zeros elsewhere (x * 1 or x * 0 in one instruction)
+      uint32_t cb[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        cb[2 * j] = tk_code_bits(bf16_times_f32<false>(wv[j], kp[j]), mult);
+        cb[2 * j + 1] = tk_code_bits(bf16_times_f32<true>(wv[j], kp[j]), mult);
+      }
+      uint32_t lo4 = tw_pack4(cb[0], cb[1], cb[2], cb[3]);
+      uint32_t hi4 = tw_pack4(cb[4], cb[5], cb[6], cb[7]);
+      uint32_t sel_lo = 0, sel_hi = 0;
+      if (partial && running < take) {
+        // ties at thr, taken in index order until `take` have survived
+        uint32_t eq[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) eq[j] = bf2_eq_mask(av[j], tt);
+        const uint32_t tl = __byte_perm(eq[0], eq[1], 0x6420), th = __byte_perm(eq[2], eq[3], 0x6420);
+        const int n = (__popc(tl) + __popc(th)) >> 3;
+        if (__ballot_sync(0xFFFFFFFFu, n != 0) != 0u) {
+          const int tot = static_cast<int>(__reduce_add_sync(0xFFFFFFFFu, static_cast<uint32_t>(n)));
+          if (running + tot <= take) {
+            sel_lo = tl;                       // every tie of this round survives
+            sel_hi = th;
+          } else {
+            // the round where the cut falls: ranks by a scan over the lanes
+            int incl = n;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const int u = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+              if (lane >= o) incl += u;
+            }
+            int nt = min(max(take - (running + incl - n), 0), n);
+            // the first nt tie bytes in element order
+            uint64_t tb = (static_cast<uint64_t>(th) << 32) | tl;
+            uint64_t sel = 0;
+            for (; nt > 0; --nt) {
+              const uint64_t byte = (tb & (0ull - tb)) * 0xFFull;
+              sel |= byte;
+              tb &= ~byte;
+            }
+            sel_lo = static_cast<uint32_t>(sel);
+            sel_hi = static_cast<uint32_t>(sel >> 32);
+          }
+          running += tot;
+          if ((sel_lo | sel_hi) != 0u) {
+            // sign bytes (0xFF where negative) pick the tie code
+            const uint32_t sg_lo = prmt_sign(wv[0], wv[1], 0xFDB9u), sg_hi = prmt_sign(wv[2], wv[3], 0xFDB9u);
+            lo4 |= ((sg_lo & ct_neg) | (~sg_lo & ct_pos)) & sel_lo;
+            hi4 |= ((sg_hi & ct_neg) | (~sg_hi & ct_pos)) & sel_hi;
+          }
+        }
+      }
+      if (c < nchunk) {
+        *reinterpret_cast<uint2*>(crow + 8 * c) = make_uint2(lo4, hi4);
+        if (mrow != nullptr) {
+          // kept: the 1.0 halves (byte 1 of a half is 0x3F) and the selected ties
+          const uint32_t kl = (((__byte_perm(kp[0], kp[1], 0x7531) + 0x7F7F7F7Fu) >> 7) & 0x01010101u) * 0xFFu | sel_lo;
+          const uint32_t kh = (((__byte_perm(kp[2], kp[3], 0x7531) + 0x7F7F7F7Fu) >> 7) & 0x01010101u) * 0xFFu | sel_hi;
+          mrow[c] = static_cast<uint8_t>(tw_byte_bits(kl) | (tw_byte_bits(kh) << 4));
+        }
+      } else if (mrow != nullptr && c < mbytes) {
+        mrow[c] = 0;                         // bits past K
+      }
+    }
+    __syncwarp();                            // the buffer is refilled two rows later
+  }
+  if (aborted) {
+    // a copy may still be in flight into this warp's buffers: let it land
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) {
+    }
+  }
+}
+
+}  // namespace bl

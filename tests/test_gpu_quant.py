@@ -204,6 +204,44 @@ def test_sparsify_a8_zero_and_constant_rows():
         check_topk(codes, scale, mask, oracle.sparsify_a8(x, keep, EPS))
 
 
+@pytest.mark.parametrize("K", [4096, 1000, 40])
+def test_sparsify_a8_subnormal_and_extreme_rows(K):
+    """Rows whose threshold falls among bf16 subnormals, on the subnormal /
+    normal boundary, or among values spread over the whole exponent range: the
+    magnitude ranking must order subnormals exactly (no flush to zero)."""
+    g = synth.rng(K + 5)
+    x = synth.student_t_bf16(g, (6, K))
+    sign = (g.integers(0, 2, (6, K)) << 15).astype(np.uint16)
+    x[0] = sign[0] | g.integers(1, 0x80, K).astype(np.uint16)                       # all subnormal
+    x[1] = sign[1] | np.where(g.random(K) < 0.5, g.integers(1, 0x80, K),
+                              g.integers(0x80, 0x100, K)).astype(np.uint16)       # subnormal and smallest normals
+    x[2] = sign[2] | g.integers(1, 0x7F7F, K).astype(np.uint16)                      # whole exponent range
+    x[3] = sign[3] | np.full(K, 0x0005, np.uint16)                                   # one subnormal value
+    x[3, ::7] = 0x0003
+    x[4, : K // 2] = 0x0001                                                          # smallest subnormal ties
+    for keep in sorted({1, K // 3, K // 2, K - 1}):
+        ref = oracle.sparsify_a8(x, keep, EPS)
+        codes, scale, mask = run_sparsify(x, keep)
+        check_topk(codes, scale, mask, ref)
+
+
+def test_sparsify_a8_without_mask():
+    """Without a mask the codes and scales are the same (dropped zeros among the
+    ties need no ranking then)."""
+    x = synth.student_t_bf16(synth.rng(24), (9, 4096))
+    x[1, ::2] = 0
+    x[2, :3000] = 0x8000
+    for keep in (1, 1500, 2048, 3000, 4095):
+        ref = oracle.sparsify_a8(x, keep, EPS)
+        xd = to_dev(x)
+        codes = empty(x.shape, torch.int8)
+        scale = empty((x.shape[0],), torch.float32)
+        tba.bitlinear_sparsify_a8(xd, keep, codes, scale, None, eps=EPS)
+        tba.sync_status()
+        assert np.array_equal(host(codes), ref[0])
+        assert np.array_equal(host(scale).view(np.uint32), ref[3].view(np.uint32))
+
+
 def run_relu2(gate, up, keep, ld_pad=0):
     M, F = gate.shape
     both = np.zeros((M, 2 * F + ld_pad), np.uint16)
