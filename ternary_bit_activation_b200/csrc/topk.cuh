@@ -479,11 +479,11 @@ namespace bl {
 constexpr int kTwWarps = 4;                  // rows in flight per CTA
 constexpr int kTwMaxK = 4096;                // 16 chunks of 8 values per lane
 
-// Dynamic shared memory of topk_warp_kernel<C>: two row buffers per warp and
-// their mbarriers.
+// Dynamic shared memory of topk_warp_kernel<C>: a row buffer per warp and its
+// mbarrier.
 template <int C>
 constexpr size_t tw_smem_bytes() {
-  return static_cast<size_t>(kTwWarps) * 2 * C * 32 * 16 + kTwWarps * 2 * 8;
+  return static_cast<size_t>(kTwWarps) * C * 32 * 16 + kTwWarps * 8;
 }
 
 // 0xFFFF in each 16-bit half where a >= b as bf16 values (a, b finite or NaN).
@@ -597,13 +597,15 @@ __global__ void __launch_bounds__(32 * kTwWarps) topk_warp_kernel(
     int8_t* __restrict__ codes, float* __restrict__ scale, uint32_t* __restrict__ mask) {
   constexpr uint32_t kAbs = 0x7FFF7FFFu;
   constexpr uint32_t kPadNaN = 0x7FC07FC0u;
-  // Two row buffers per warp: 1-D bulk copies bring the next row in while the
-  // current one is ranked and quantized.  The code pass reads the signed row
-  // from its buffer in a rolled loop (an unrolled one overflows the
-  // instruction cache); the probes read the |x| words from registers.
+  // One row buffer per warp, filled by a 1-D bulk copy.  The code pass reads the
+  // signed row from it in a rolled loop (an unrolled one overflows the
+  // instruction cache); the probes read the |x| words from registers.  The
+  // next row is prefetched into L2 when a row starts and copied in as soon as
+  // the code pass is done: a row keeps a warp busy far longer than a copy
+  // takes, and one buffer per warp leaves room for more warps per SM.
   extern __shared__ __align__(128) uint4 tw_dyn[];
-  uint4 (*rowbuf)[2][C * 32] = reinterpret_cast<uint4 (*)[2][C * 32]>(tw_dyn);
-  uint64_t (*rowbar)[2] = reinterpret_cast<uint64_t (*)[2]>(tw_dyn + kTwWarps * 2 * C * 32);
+  uint4 (*rowbuf)[C * 32] = reinterpret_cast<uint4 (*)[C * 32]>(tw_dyn);
+  uint64_t* rowbar = reinterpret_cast<uint64_t*>(tw_dyn + kTwWarps * C * 32);
   const int lane = threadIdx.x & 31;
   const int wig = threadIdx.x >> 5;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kTwWarps;
@@ -613,8 +615,7 @@ __global__ void __launch_bounds__(32 * kTwWarps) topk_warp_kernel(
   // the sample: word 0 of chunk round (lane % C), low half
   const int qs = lane % C;
   if (lane == 0) {
-    mbar_init(&rowbar[wig][0], 1);
-    mbar_init(&rowbar[wig][1], 1);
+    mbar_init(&rowbar[wig], 1);
     fence_mbarrier_init();
   }
   __syncwarp();
@@ -622,25 +623,20 @@ __global__ void __launch_bounds__(32 * kTwWarps) topk_warp_kernel(
   pdl_trigger();
   int64_t row = static_cast<int64_t>(blockIdx.x) * kTwWarps + wig;
   if (lane == 0 && row < M) {
-    mbar_arrive_expect_tx(&rowbar[wig][0], row_bytes);
-    bulk_load_1d(rowbuf[wig][0], x + row * ldx, row_bytes, &rowbar[wig][0]);
+    mbar_arrive_expect_tx(&rowbar[wig], row_bytes);
+    bulk_load_1d(rowbuf[wig], x + row * ldx, row_bytes, &rowbar[wig]);
   }
-  uint32_t phase = 0;                         // bit b: parity of buffer b's next completion
+  uint32_t phase = 0;
   bool aborted = false;
-  for (int buf = 0; row < M; row += nwarps, buf ^= 1) {
-    if (lane == 0 && row + nwarps < M) {
-      // the other buffer was last read by the previous row (this warp, in order)
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive_expect_tx(&rowbar[wig][buf ^ 1], row_bytes);
-      bulk_load_1d(rowbuf[wig][buf ^ 1], x + (row + nwarps) * ldx, row_bytes, &rowbar[wig][buf ^ 1]);
-    }
+  const uint4* rb = rowbuf[wig];
+  for (; row < M; row += nwarps) {
+    if (lane == 0 && row + nwarps < M) bulk_prefetch_l2(x + (row + nwarps) * ldx, row_bytes);
     // every lane waits for the copy; giving up is decided for the whole warp
-    if (__any_sync(0xFFFFFFFFu, !mbar_wait_bounded(&rowbar[wig][buf], (phase >> buf) & 1u))) {
+    if (__any_sync(0xFFFFFFFFu, !mbar_wait_bounded(&rowbar[wig], phase))) {
       aborted = true;
       break;
     }
-    phase ^= 1u << buf;
-    const uint4* rb = rowbuf[wig][buf];
+    phase ^= 1u;
     // |x| words in registers (the probes' operand), NaN past K
     uint32_t w[C][4];
 #pragma unroll
@@ -688,8 +684,9 @@ __global__ void __launch_bounds__(32 * kTwWarps) topk_warp_kernel(
       const uint32_t t_lo = __shfl_sync(0xFFFFFFFFu, smp, max(ai - 2, 0));
       // count(t) for one or two thresholds in one pass over the row: packed
       // compares give 1.0 / 0 per half, summed in bf16 on the FMA pipe in
-      // independent partial sums (at most 2C per half and sum: exact); the
-      // counts leave the bf16 sums through fp32 (exact) and the 2^23 trick
+      // independent partial sums (at most C per half and partial sum, 4C <= 64
+      // per lane: exact); the counts leave the bf16 sums through fp32 (exact)
+      // and the 2^23 trick
       auto bf2_count = [](uint32_t a, uint32_t b) -> uint32_t {
         const uint32_t sa = bf2_add(a, b);
         const float f = __fadd_rn(__fadd_rn(__uint_as_float(sa << 16), __uint_as_float(sa & 0xFFFF0000u)), 8388608.f);
@@ -697,15 +694,16 @@ __global__ void __launch_bounds__(32 * kTwWarps) topk_warp_kernel(
       };
       auto counts2 = [&](uint32_t t0, uint32_t t1, int& c0, int& c1) {
         const uint32_t u0 = t0 | (t0 << 16), u1 = t1 | (t1 << 16);
-        uint32_t a[2] = {0, 0}, b[2] = {0, 0};
+        uint32_t a[4] = {0, 0, 0, 0}, b[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int q = 0; q < C; ++q)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            a[j & 1] = bf2_add(a[j & 1], bf2_ge_one(w[q][j], u0));
-            b[j & 1] = bf2_add(b[j & 1], bf2_ge_one(w[q][j], u1));
+            a[j] = bf2_add(a[j], bf2_ge_one(w[q][j], u0));
+            b[j] = bf2_add(b[j], bf2_ge_one(w[q][j], u1));
           }
-        const uint32_t r = __reduce_add_sync(0xFFFFFFFFu, bf2_count(a[0], a[1]) | (bf2_count(b[0], b[1]) << 16));
+        const uint32_t r = __reduce_add_sync(0xFFFFFFFFu, (bf2_count(a[0], a[1]) + bf2_count(a[2], a[3])) |
+                                                              ((bf2_count(b[0], b[1]) + bf2_count(b[2], b[3])) << 16));
         c0 = static_cast<int>(r & 0xFFFFu);   // two 16-bit sums (K <= 4096)
         c1 = static_cast<int>(r >> 16);
       };
@@ -739,10 +737,10 @@ __global__ void __launch_bounds__(32 * kTwWarps) topk_warp_kernel(
       bool bisect = false;
 #pragma unroll 1
       while (hi - lo > 1) {
-        if (hi - lo <= 3) {
-          // the last one or two candidates in one pass
+        if (hi - lo == 3) {
+          // the last two candidates in one pass
           int c0, c1;
-          const uint32_t t0 = lo + 1, t1 = hi - 1;
+          const uint32_t t0 = lo + 1, t1 = lo + 2;
           counts2(t0, t1, c0, c1);
           update(t0, c0);
           update(t1, c1);
@@ -780,7 +778,7 @@ __global__ void __launch_bounds__(32 * kTwWarps) topk_warp_kernel(
     int8_t* crow = codes + row * static_cast<int64_t>(K);
     uint8_t* mrow = mask != nullptr ? reinterpret_cast<uint8_t*>(mask) + row * static_cast<int64_t>(mbytes) : nullptr;
     int running = 0;                         // ties in the rounds before
-#pragma unroll 1
+#pragma unroll 2
     for (int q = 0; q < C; ++q) {
       const int c = 32 * q + lane;
       const uint4 v = rb[c];
@@ -855,7 +853,12 @@ __global__ void __launch_bounds__(32 * kTwWarps) topk_warp_kernel(
         mrow[c] = 0;                         // bits past K
       }
     }
-    __syncwarp();                            // the buffer is refilled two rows later
+    __syncwarp();                            // the code pass is done with the buffer
+    if (lane == 0 && row + nwarps < M) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive_expect_tx(&rowbar[wig], row_bytes);
+      bulk_load_1d(rowbuf[wig], x + (row + nwarps) * ldx, row_bytes, &rowbar[wig]);
+    }
   }
   if (aborted) {
     // a copy may still be in flight into this warp's buffers: let it land
