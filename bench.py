@@ -28,6 +28,7 @@ token sample of the same workload, scaled to tokens/s.
 from __future__ import annotations
 
 import argparse
+import functools
 import json
 import os
 import statistics
@@ -50,11 +51,16 @@ EPS = 1e-5
 # measured B200 peaks of this machine (generated file), else the documented fallback
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 INT8_PER_BF16 = 2.0   # nominal dense int8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
-# DRAM bytes (read + write) of the four GEMM launches of one step, from a one-pass ncu
-# capture of this benchmark (profiles/gemm_tc2_kernel__int8_16384x12288x4096.md gives the
-# command); algorithmic bytes of the same launches: 3.75 GB (A and W read once, Y written once)
-GEMM_STEP_DRAM_BYTES = 549892096 + 763724544 + 196653568 + 224203520 + 962767872 + 1400955648 + \
-    1338792960 + 251956480
+FP4_PER_BF16 = 4.0    # nominal dense fp4 : bf16 (9 : 2.25 PFLOP/s)
+# DRAM bytes (read + write) of one launch of each of the step's four GEMM shapes at
+# 16384 tokens (`--profile-case gemm / gemm_o / gemm_upgate / gemm_down`, ncu
+# dram__bytes_read.sum + dram__bytes_write.sum, second launch), doubled for the
+# step's 32768 tokens: A and Y grow with the token count, the 202 MB of weights do
+# not, so the doubling overstates by at most 0.2 GB.  Algorithmic bytes of the same
+# launches at 32768 tokens: 3.75 GB (A and W read once, Y written once).
+GEMM_TRAFFIC_16K = {"qkv": 269529088 + 358346496, "o": 103798016 + 91663360,
+                    "upgate": 436135936 + 679412736, "down": 627190016 + 121038336}
+GEMM_STEP_DRAM_BYTES = 2 * sum(GEMM_TRAFFIC_16K.values())
 
 
 def load_peaks():
@@ -226,6 +232,13 @@ class Layer:
         self.gemm_ops = {k: 2.0 * m * n * kk for k, (n, kk) in N_K.items()}
         self.weights = sum(n * kk for n, kk in N_K.values())
         self.launches_per_step = 5 * 3 + 2 + 4 + 2 + 1 + 1
+
+    def alg_gemm_ops(self):
+        """2 N nnz(A) per step: QKV and Up|Gate dense, O and Down with the
+        Top-K survivors (k_keep of K per token)."""
+        m, d, f = self.m, self.d, self.f
+        keep_o, keep_d = synth.k_keep(d, SHAPE.topk_pct_o), synth.k_keep(f, SHAPE.topk_pct_down)
+        return (self.gemm_ops["qkv"] + self.gemm_ops["upgate"] + 2.0 * m * d * keep_o + 2.0 * m * d * keep_d)
 
     # kernel-by-kernel bytes each launch must move (algorithmic, per the formulas
     # of the path: read inputs once, write outputs once)
@@ -461,9 +474,10 @@ def run_gpu(args):
                 entry["gbs"] = round(kb[k] / (per_step / 1e3) / 1e9, 1)
                 entry["hbm_frac"] = round(entry["gbs"] / peaks["hbm_gbs"], 3)
             kernels[k] = entry
-        # algorithmic TOPS: the Top-K-50% inputs (O, Down) carry half the nonzeros
-        alg_ops = (layer.gemm_ops["qkv"] + layer.gemm_ops["upgate"] +
-                   0.5 * (layer.gemm_ops["o"] + layer.gemm_ops["down"])) * args.steps
+        # algorithmic ops: 2 N nnz(A) -- the INT4 / FP4 inputs are dense, the
+        # Top-K inputs of O and Down keep k_keep of their K values per token
+        alg_ops = layer.alg_gemm_ops() * args.steps
+        alg_tops = alg_ops / (gemm_ms / 1e3) / 1e12
         h2d, d2h = layer.io_bytes()
         line = {
             "metric": METRIC,
@@ -487,15 +501,20 @@ def run_gpu(args):
                 "peak": round(peak_int8, 1),
                 "unit": "TFLOP/s",
                 "frac": round(tops / peak_int8, 4),
+                "achieved_algorithmic": round(alg_tops, 1),
+                "frac_algorithmic": round(alg_tops / peak_int8, 4),
                 "traffic": GEMM_STEP_DRAM_BYTES if args.afmt == "int4" else None,
-                "traffic_note": "DRAM read+write bytes of the 4 GEMM launches of one step (ncu, one pass); "
-                                "algorithmic 3.75e9",
+                "traffic_note": "DRAM read+write bytes of the 4 GEMM shapes, each captured by ncu at 16384 "
+                                "tokens (--profile-case) and doubled for the step's 32768 (the weights do not "
+                                "double: overstates by <= 0.2e9); algorithmic 3.75e9",
                 "peak_note": f"int8 = {INT8_PER_BF16:g} x {peaks['source']} {'burst' if burst else 'sustained'} "
                              f"bf16 cuBLAS ({peaks[basis]} TFLOP/s; nominal dense int8:bf16 ratio)" +
                              ("; fp4 = 2 x int8, combined by the ops of each kind" if args.afmt == "fp4" else ""),
-                "work": "dense-equivalent 2*M*N*K over the 4 GEMM launches of a step / their summed event time",
+                "work": "achieved / frac: dense-equivalent 2*M*N*K over the 4 GEMM launches of a step / their "
+                        "summed event time; achieved_algorithmic / frac_algorithmic: 2*N*nnz(A), the O and Down "
+                        "inputs counted with their k_keep survivors per token",
             },
-            "gemm": {"tops_dense": round(tops, 1), "tops_algorithmic": round(alg_ops / (gemm_ms / 1e3) / 1e12, 1),
+            "gemm": {"tops_dense": round(tops, 1), "tops_algorithmic": round(alg_tops, 1),
                      "ms_per_step": round(gemm_ms / args.steps, 4)},
             "kernels": kernels,
             "e2e": {"value": round(world * m * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
@@ -505,8 +524,31 @@ def run_gpu(args):
             "clocks": clk,
             "zero_fraction": zero_fractions(torch, layer),
         }
+        if not args.no_extras and world == 1:
+            # the decode sweep (7B shapes, 1-256 tokens) and the FP4 variant's two
+            # GEMMs, on this GPU, after the timed regions
+            dec = decode_sweep(torch, tba, dev, synth.DECODE_TOKENS, steps=20, warmup=3, w_lat=layer.w_lat,
+                               variants=False)
+            line["decode"] = {"unit": "us per layer",
+                              "workload": f"M tokens through the BitLinear path (quantizers, Top-K, ReLU^2-GLU "
+                                          f"and the four GEMMs on 2-bit weights) of {DECODE_LAYERS} 7B-shape layers "
+                                          f"with their own weight buffers (together larger than L2); CUDA-graph "
+                                          f"replay; hbm_frac_layer = weight bytes / layer time / HBM peak",
+                              **dec}
+            f4 = fp4_gemm_key(torch, tba, layer, reps=10)
+            f4_peak = FP4_PER_BF16 * peaks[basis]
+            for v in f4.values():
+                v["frac"] = round(v["tops_dense"] / f4_peak, 4)
+            line["fp4"] = {"unit": "TFLOP/s", "peak": round(f4_peak, 1),
+                           "peak_note": f"fp4 = {FP4_PER_BF16:g} x {peaks['source']} "
+                                        f"{'burst' if burst else 'sustained'} bf16 cuBLAS (nominal dense 9 : 2.25 "
+                                        f"PFLOP/s)",
+                           "workload": "QKV [32768 x 4096] x [12288 x 4096]^T and Up|Gate [32768 x 4096] x "
+                                       "[22016 x 4096]^T, packed E2M1 activations x E2M1-coded ternary weights, "
+                                       "tcgen05 kind::mxf4; median of 10 launches",
+                           **f4}
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(args.afmt, tokens_sample=args.cpu_tokens)
+            line["cpu_baseline"] = cpu_baseline(args.afmt, args.cpu_tokens_per_core, args.cpu_tokens)
         print(json.dumps(line), flush=True)
     if distributed:
         dist.barrier()
@@ -516,55 +558,92 @@ def run_gpu(args):
 # ---------------------------------------------------------------------------
 # CPU oracle arm
 # ---------------------------------------------------------------------------
-def oracle_sample_seconds(afmt: str, tokens: int, pack: bool = True):
-    """Time the CPU oracle over the same step on `tokens` rows: per-token work
-    (quantizers, the four products, ReLU^2-GLU, KV) plus, if `pack`, the
-    once-per-step ternary quantization of all latent weights."""
+def host_cores() -> int:
+    """Host CPU threads this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+@functools.lru_cache(maxsize=1)
+def _oracle_weights():
+    """The layer's latent weights for the CPU oracle, generated once."""
+    return synth.layer_weights(SHAPE, seed=3)
+
+
+def oracle_sample_seconds(afmt: str, tokens: int, threads: int = 1):
+    """Time the CPU oracle over the same step on `tokens` rows: the ternary
+    quantization of all latent weights (the five tensors side by side), then
+    the per-token work (quantizers, the four products, ReLU^2-GLU, KV) with the
+    token rows split over `threads` threads.  The oracle's loops are C called
+    through ctypes, which releases the GIL, so the threads run in parallel.
+    Returns (pack seconds, token seconds), wall clock; input generation is
+    outside both."""
+    from concurrent.futures import ThreadPoolExecutor
+
     import oracle
+    oracle.build()
     s = SHAPE
     d, f = s.hidden, s.ffn
-    wts = synth.layer_weights(s, seed=3)
+    wts = _oracle_weights()
     x_attn, x_o, x_ffn = synth.layer_activations(s, seed=99, tokens=tokens)
-    t_pack = 0.0
-    t0 = time.perf_counter()
-    tq = {}
-    al = {}
-    for k, w in wts.items():
-        tq[k], al[k] = oracle.ternary_quantize(w, EPS)
-    t_pack = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    if afmt == "fp4":
-        _, qa, _, s_a = oracle.quant_fp4(x_attn)
-        s_a = (s_a / 2).astype(np.float32)
-    else:
-        qa, _, s_a = oracle.quant_int4(x_attn, EPS)
-    _, y_qkv = oracle.gemm(qa, s_a, tq["qkv"], al["qkv"])
-    kvin = np.ascontiguousarray(y_qkv[:, d:].reshape(tokens, 2, s.heads, s.head_dim).transpose(1, 0, 2, 3))
-    for i in range(2):
-        oracle.kv_quant(kvin[i], bits=3, bos_pos=0, eps=EPS)
-    c8, _, _, s8 = oracle.sparsify_a8(x_o, synth.k_keep(d, s.topk_pct_o), EPS)
-    oracle.gemm(c8, s8, tq["o"], al["o"])
-    if afmt == "fp4":
-        _, qf, _, s_f = oracle.quant_fp4(x_ffn)
-        s_f = (s_f / 2).astype(np.float32)
-    else:
-        qf, _, s_f = oracle.quant_int4(x_ffn, EPS)
-    _, y_up = oracle.gemm(qf, s_f, tq["up"], al["up"])
-    _, y_gate = oracle.gemm(qf, s_f, tq["gate"], al["gate"])
-    h8, _, _, sh = oracle.relu2_glu(y_gate, y_up, synth.k_keep(f, s.topk_pct_down), EPS)
-    oracle.gemm(h8, sh, tq["down"], al["down"])
-    t_tok = time.perf_counter() - t0
+    keep_o, keep_d = synth.k_keep(d, s.topk_pct_o), synth.k_keep(f, s.topk_pct_down)
+    with ThreadPoolExecutor(max_workers=max(threads, 1)) as pool:
+        t0 = time.perf_counter()
+        packed = dict(zip(wts, pool.map(lambda w: oracle.ternary_quantize(w, EPS), wts.values())))
+        t_pack = time.perf_counter() - t0
+        tq = {k: v[0] for k, v in packed.items()}
+        al = {k: v[1] for k, v in packed.items()}
+
+        def quant4(x):
+            if afmt == "fp4":
+                _, q, _, sc = oracle.quant_fp4(x)
+                return q, (sc / 2).astype(np.float32)
+            q, _, sc = oracle.quant_int4(x, EPS)
+            return q, sc
+
+        def rows(sl):
+            n = sl.stop - sl.start
+            qa, s_a = quant4(x_attn[sl])
+            _, y_qkv = oracle.gemm(qa, s_a, tq["qkv"], al["qkv"])
+            kvin = np.ascontiguousarray(y_qkv[:, d:].reshape(n, 2, s.heads, s.head_dim).transpose(1, 0, 2, 3))
+            for i in range(2):
+                oracle.kv_quant(kvin[i], bits=3, bos_pos=0, eps=EPS)
+            c8, _, _, s8 = oracle.sparsify_a8(x_o[sl], keep_o, EPS)
+            oracle.gemm(c8, s8, tq["o"], al["o"])
+            qf, s_f = quant4(x_ffn[sl])
+            _, y_up = oracle.gemm(qf, s_f, tq["up"], al["up"])
+            _, y_gate = oracle.gemm(qf, s_f, tq["gate"], al["gate"])
+            h8, _, _, sh = oracle.relu2_glu(y_gate, y_up, keep_d, EPS)
+            oracle.gemm(h8, sh, tq["down"], al["down"])
+
+        bounds = np.linspace(0, tokens, max(threads, 1) + 1).astype(int)
+        slices = [slice(a, b) for a, b in zip(bounds[:-1], bounds[1:]) if b > a]
+        t0 = time.perf_counter()
+        list(pool.map(rows, slices))
+        t_tok = time.perf_counter() - t0
     return t_pack, t_tok
 
 
-def cpu_baseline(afmt: str, tokens_sample: int):
-    t_pack, t_tok = oracle_sample_seconds(afmt, tokens_sample)
+def cpu_baseline(afmt: str, tokens_per_core: int, one_core_tokens: int):
+    """The oracle on all host cores (token rows split over one thread per core,
+    the five weight tensors quantized side by side) and on one core, each over
+    a bounded token sample scaled linearly to the step's token count."""
     m = SHAPE.tokens
-    step_s = t_pack + t_tok * (m / tokens_sample)
-    return {"value": round(m / step_s, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{tokens_sample} tokens of the 7B-shape layer through every step of the path, plus the "
-                      f"once-per-step ternary quantization of all 202M latent weights; per-token time scaled "
-                      f"linearly to {m} tokens (pack {t_pack:.2f} s, sample {t_tok:.2f} s, single-threaded C)"}
+    cores = host_cores()
+    n_all = tokens_per_core * cores
+    p_all, t_all = oracle_sample_seconds(afmt, n_all, threads=cores)
+    p_one, t_one = oracle_sample_seconds(afmt, one_core_tokens, threads=1)
+    v_all = m / (p_all + t_all * (m / n_all))
+    v_one = m / (p_one + t_one * (m / one_core_tokens))
+    return {"value": round(v_all, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "value_1core": round(v_one, 2),
+            "sample": f"all cores: {n_all} tokens ({tokens_per_core} per thread, {cores} threads) of the 7B-shape "
+                      f"layer through every step of the path, plus the ternary quantization of all 202M latent "
+                      f"weights (five tensors side by side): pack {p_all:.2f} s, tokens {t_all:.2f} s wall; one "
+                      f"core: {one_core_tokens} tokens, pack {p_one:.2f} s, tokens {t_one:.2f} s; per-token time "
+                      f"scaled linearly to {m} tokens (extrapolated); C oracle via ctypes"}
 
 
 def run_reference(args):
@@ -573,23 +652,29 @@ def run_reference(args):
     if rank != 0:
         return
     m = SHAPE.tokens
+    cores = host_cores()
+    n_tok = args.cpu_tokens_ref * cores
     for _ in range(args.warmup):
-        oracle_sample_seconds(args.afmt, args.cpu_tokens_ref, pack=True)
-    total = 0.0
+        oracle_sample_seconds(args.afmt, n_tok, threads=cores)
+    wall, full = 0.0, 0.0
     for _ in range(args.steps):
-        t_pack, t_tok = oracle_sample_seconds(args.afmt, args.cpu_tokens_ref, pack=True)
-        total += t_pack + t_tok * (m / args.cpu_tokens_ref)
-    value = args.steps * m / total
+        t_pack, t_tok = oracle_sample_seconds(args.afmt, n_tok, threads=cores)
+        wall += t_pack + t_tok
+        full += t_pack + t_tok * (m / n_tok)
+    value = args.steps * m / full
     line = {
         "impl": "reference",
         "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 1), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded)",
-        "config": dict(workload_config(args.afmt, m), parallelism="host CPU, rank 0 only"),
-        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"each step: {args.cpu_tokens_ref} tokens of the 7B-shape layer through the "
-                                   f"whole path plus the ternary quantization of all latent weights, per-token time "
-                                   f"scaled to {m} tokens; single-threaded C oracle"},
+        "warmup": args.warmup, "ms_per_step": round(1e3 * wall / args.steps, 1),
+        "extrapolated": True, "ms_per_step_full_workload": round(1e3 * full / args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8" if args.afmt == "int4" else "fp4(e2m1)+int8", "data": "synthetic (seeded)",
+        "config": dict(workload_config(args.afmt, m), parallelism=f"replicas x{world}"),
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: the ternary quantization of all latent weights plus {n_tok} tokens "
+                                   f"({args.cpu_tokens_ref} per thread, {cores} threads) of the 7B-shape layer "
+                                   f"through the whole path; ms_per_step is that sample's wall time, and value scales "
+                                   f"its per-token time linearly to {m} tokens (extrapolated)"},
         "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -658,12 +743,13 @@ def run_quant_variants(args):
     print(json.dumps(line), flush=True)
 
 
-def run_decode(args):
-    import torch
-
-    import ternary_bit_activation_b200 as tba
-    torch.cuda.set_device(0)
-    dev = torch.device("cuda", 0)
+def decode_sweep(torch, tba, dev, tokens_list, steps, warmup, w_lat=None, variants=True):
+    """Per M in tokens_list: CUDA-graph replay of M tokens through the BitLinear
+    path of DECODE_LAYERS distinct 7B-shape layers (2-bit weights packed once,
+    as at inference; together they exceed L2, so every layer streams its weights
+    from HBM).  w_lat: latent fp32 weights on the device to pack into each
+    layer's own buffers (else seeded weights per layer).  variants adds the
+    fused-quantizer and conditional-Up timings."""
     s = SHAPE
     d, f = s.hidden, s.ffn
     T = torch
@@ -671,18 +757,19 @@ def run_decode(args):
     layers = []
     ws = T.empty((tba.workspace_size("pack_ternary") // 8,), dtype=T.int64, device=dev)
     for li in range(DECODE_LAYERS):
-        wts = synth.layer_weights(s, seed=3 + li)
+        wts = w_lat if w_lat is not None else {k: T.from_numpy(v).to(dev)
+                                                for k, v in synth.layer_weights(s, seed=3 + li).items()}
         w2 = {k: T.empty((n, kk // 4), dtype=T.uint8, device=dev) for k, (n, kk) in shapes.items()}
         alpha = T.zeros((8,), dtype=T.float32, device=dev)
         for key, dst, ai in (("qkv", w2["qkv"], 0), ("o", w2["o"], 1), ("up", w2["upgate"][:f], 2),
                              ("gate", w2["upgate"][f:], 3), ("down", w2["down"], 4)):
-            tba.pack_ternary(T.from_numpy(wts[key]).to(dev), alpha[ai:ai + 1], dst, tba.BL_W_T2, ws)
+            tba.pack_ternary(wts[key], alpha[ai:ai + 1], dst, tba.BL_W_T2, ws)
         del wts
         layers.append((w2, alpha))
     weight_bytes = sum(n * kk // 4 for n, kk in shapes.values())
     peaks = load_peaks()
     results = []
-    for m in args.decode_tokens:
+    for m in tokens_list:
         x_attn, x_o, x_ffn = [T.from_numpy(a.view(np.int16)).to(dev)
                               for a in synth.layer_activations(s, seed=500 + m, tokens=m)]
         qa = T.empty((m, d), dtype=T.int8, device=dev)
@@ -728,24 +815,11 @@ def run_decode(args):
             if gemms:
                 tba.bitlinear_gemm(h8, h8_s, w2["down"], alpha[4:5], m, d, f, y=y_down, wfmt=tba.BL_W_T2)
 
-        def step():
-            for w2, alpha in layers:
-                layer(w2, alpha)
+        def all_layers(**kw):
+            return lambda: [layer(w2, alpha, **kw) for w2, alpha in layers]
 
-        def step_fused():
-            for w2, alpha in layers:
-                layer(w2, alpha, fused=True)
-
-        def step_gated():
-            for w2, alpha in layers:
-                layer(w2, alpha, gated=True)
-
-        def gemms_only():
-            for w2, alpha in layers:
-                layer(w2, alpha, others=False)
-
-        for _ in range(args.warmup):
-            step()
+        for _ in range(warmup):
+            all_layers()()
         tba.sync_status()
         torch.cuda.synchronize()
 
@@ -762,46 +836,99 @@ def run_decode(args):
                 fn()
             return graph
 
-        g_step = capture(step)
-        g_fused = capture(step_fused)
-        g_gated = capture(step_gated) if m <= 2 else None
-        g_gemm = capture(gemms_only)
-
         def time_graph(graph):
             for _ in range(3):
                 graph.replay()
             torch.cuda.synchronize()
             a_, b_ = T.cuda.Event(enable_timing=True), T.cuda.Event(enable_timing=True)
             a_.record()
-            for _ in range(args.steps):
+            for _ in range(steps):
                 graph.replay()
             b_.record()
             torch.cuda.synchronize()
-            return a_.elapsed_time(b_) / (args.steps * DECODE_LAYERS)
+            return a_.elapsed_time(b_) / (steps * DECODE_LAYERS)
 
-        ms = time_graph(g_step)
-        fused_ms = time_graph(g_fused)
-        gated_ms = time_graph(g_gated) if g_gated is not None else None
-        gemm_ms = time_graph(g_gemm)
+        graphs = {"step": capture(all_layers()), "gemm": capture(all_layers(others=False))}
+        if variants:
+            graphs["fused"] = capture(all_layers(fused=True))
+            if m <= 2:
+                graphs["gated"] = capture(all_layers(gated=True))
+        ms = {k: time_graph(g) for k, g in graphs.items()}
         tba.sync_status()
-        del g_step, g_fused, g_gated, g_gemm
-        gbs = weight_bytes / (gemm_ms / 1e3) / 1e9
-        results.append({"tokens": m, "ms_per_layer": round(ms, 4), "tokens_per_s": round(m / (ms / 1e3), 1),
-                        "fused_quant_ms_per_layer": round(fused_ms, 4),
-                        "conditional_up_ms_per_layer": round(gated_ms, 4) if gated_ms is not None else None,
-                        "gemm_ms_per_layer": round(gemm_ms, 4),
-                        "gemm_kernel": decode_gemm_kernel(m),
-                        "weight_stream_gbs": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 3)})
+        del graphs
+        gbs = weight_bytes / (ms["gemm"] / 1e3) / 1e9
+        r = {"tokens": m, "us_per_layer": round(1e3 * ms["step"], 2), "tokens_per_s": round(m / (ms["step"] / 1e3), 1),
+             "us_gemm_per_layer": round(1e3 * ms["gemm"], 2), "gemm_kernel": decode_gemm_kernel(m),
+             "weight_stream_gbs": round(gbs, 1), "hbm_frac_gemm": round(gbs / peaks["hbm_gbs"], 3),
+             "hbm_frac_layer": round(weight_bytes / (ms["step"] / 1e3) / 1e9 / peaks["hbm_gbs"], 3)}
+        if "fused" in ms:
+            r["fused_quant_us_per_layer"] = round(1e3 * ms["fused"], 2)
+        if "gated" in ms:
+            r["conditional_up_us_per_layer"] = round(1e3 * ms["gated"], 2)
+        results.append(r)
+    return {"weight_bytes_per_layer": weight_bytes, "layers": DECODE_LAYERS, "hbm_peak_gbs": peaks["hbm_gbs"],
+            "results": results}
+
+
+def run_decode(args):
+    import torch
+
+    import ternary_bit_activation_b200 as tba
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    sweep = decode_sweep(torch, tba, dev, args.decode_tokens, args.steps, args.warmup)
     line = {"metric": "decode BitLinear layer latency (7B shapes, 2-bit weights; CUDA-graph replay)",
-            "unit": "ms per layer",
+            "unit": "us per layer",
             "workload": f"7B-shape decoder layers, decode of M tokens through all four BitLinear matrices of "
                         f"each of {DECODE_LAYERS} distinct layers (weights exceed L2), separate quantizer and GEMM "
-                        f"calls; fused_quant_ms_per_layer: the QKV and Up|Gate INT4 quantizers fused into their "
-                        f"GEMMs (bitlinear_quant_gemm); conditional_up_ms_per_layer (1-2 tokens): the Up|Gate GEMM as "
+                        f"calls; fused_quant_us_per_layer: the QKV and Up|Gate INT4 quantizers fused into their "
+                        f"GEMMs (bitlinear_quant_gemm); conditional_up_us_per_layer (1-2 tokens): the Up|Gate GEMM as "
                         f"Gate first and Up only on channels with a positive gate (bitlinear_gemm_gated)",
-            "weight_bytes_per_layer": weight_bytes, "hbm_peak_gbs": peaks["hbm_gbs"],
-            "steps": args.steps, "warmup": args.warmup, "results": results}
+            "steps": args.steps, "warmup": args.warmup, **sweep}
     print(json.dumps(line), flush=True)
+
+
+def fp4_gemm_key(torch, tba, layer, reps: int):
+    """The FP4 activation variant's two tensor-core GEMMs at the step's size:
+    packed E2M1 activations (the step's QKV and FFN inputs, quantized) x
+    E2M1-coded ternary weights (the step's latent Q|K|V and Up|Gate weights) on
+    tcgen05 kind::mxf4; CUDA events around each launch, median of reps."""
+    T = torch
+    dev = layer.dev
+    m, d, f = layer.m, layer.d, layer.f
+    W = layer.w_lat
+    wq = T.empty((3 * d, d // 2), dtype=T.uint8, device=dev)
+    wug = T.empty((2 * f, d // 2), dtype=T.uint8, device=dev)
+    al = T.zeros((4,), dtype=T.float32, device=dev)
+    tba.pack_ternary(W["qkv"], al[0:1], wq, tba.BL_W_E2M1, layer.ws, eps=EPS)
+    tba.pack_ternary(W["up"], al[1:2], wug[:f], tba.BL_W_E2M1, layer.ws, eps=EPS)
+    tba.pack_ternary(W["gate"], al[2:3], wug[f:], tba.BL_W_E2M1, layer.ws, eps=EPS)
+    qa = T.empty((m, d // 2), dtype=T.uint8, device=dev)
+    qf = T.empty((m, d // 2), dtype=T.uint8, device=dev)
+    sa = T.empty((m,), dtype=T.float32, device=dev)
+    sf = T.empty((m,), dtype=T.float32, device=dev)
+    tba.bitlinear_quant_a4(layer.x[0], qa, sa, tba.BL_QUANT_FP4_E2M1, tba.BL_STORE_PACKED, EPS)
+    tba.bitlinear_quant_a4(layer.x[2], qf, sf, tba.BL_QUANT_FP4_E2M1, tba.BL_STORE_PACKED, EPS)
+    runs = {"qkv": (lambda: tba.bitlinear_gemm(qa, sa, wq, al[0:1], m, 3 * d, d, y=layer.y_qkv,
+                                                afmt=tba.BL_A_E2M1, wfmt=tba.BL_W_E2M1), 3 * d),
+            "upgate": (lambda: tba.bitlinear_gemm(qf, sf, wug, al[1:3], m, 2 * f, d, y=layer.y_ug, alpha_group=f,
+                                                   afmt=tba.BL_A_E2M1, wfmt=tba.BL_W_E2M1), 2 * f)}
+    out = {}
+    for name, (fn, n) in runs.items():
+        for _ in range(2):
+            fn()
+        ts = []
+        for _ in range(reps):
+            a_, b_ = T.cuda.Event(enable_timing=True), T.cuda.Event(enable_timing=True)
+            a_.record()
+            fn()
+            b_.record()
+            T.cuda.synchronize()
+            ts.append(a_.elapsed_time(b_))
+        ms = sorted(ts)[len(ts) // 2]
+        out[name] = {"us": round(1e3 * ms, 1), "tops_dense": round(2.0 * m * n * d / (ms / 1e3) / 1e12, 1)}
+    tba.sync_status()
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -810,6 +937,9 @@ def run_decode(args):
 # ---------------------------------------------------------------------------
 PROFILE_CASES = {
     "gemm": "tcgen05 GEMM, int8 A [16384 x 4096] x ternary int8 W [12288 x 4096]",
+    "gemm_o": "tcgen05 GEMM, int8 A [16384 x 4096] x ternary int8 W [4096 x 4096]",
+    "gemm_upgate": "tcgen05 GEMM, int8 A [16384 x 4096] x ternary int8 W [22016 x 4096]",
+    "gemm_down": "tcgen05 GEMM, int8 A [16384 x 11008] x ternary int8 W [4096 x 11008]",
     "quant_a4": "INT4 quantizer, X bf16 [32768 x 4096]",
     "sparsify_a8": "Top-K 50% + INT8, X bf16 [32768 x 4096]",
     "relu2_glu": "ReLU^2-GLU + Top-K 50% + INT8, gate/up bf16 [16384 x 11008]",
@@ -834,8 +964,9 @@ def run_profile_case(name: str, launches: int):
     def bf16(m, k, scale=1.0):
         return (torch.randn((m, k), generator=g, device=dev) * scale).to(torch.bfloat16).view(torch.int16)
 
-    if name == "gemm":
-        M, N, K = 16384, 12288, 4096
+    if name in ("gemm", "gemm_o", "gemm_upgate", "gemm_down"):
+        M, N, K = {"gemm": (16384, 12288, 4096), "gemm_o": (16384, 4096, 4096), "gemm_upgate": (16384, 22016, 4096),
+                   "gemm_down": (16384, 4096, 11008)}[name]
         a = torch.randint(-8, 8, (M, K), generator=g, device=dev, dtype=torch.int8)
         w = torch.randint(-1, 2, (N, K), generator=g, device=dev, dtype=torch.int8)
         s = torch.rand((M,), generator=g, device=dev)
@@ -903,9 +1034,11 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--afmt", choices=["int4", "fp4"], default="int4")
-    ap.add_argument("--cpu-tokens", type=int, default=32, help="token sample of the CPU baseline")
-    ap.add_argument("--cpu-tokens-ref", type=int, default=8, help="token sample per step of --impl reference")
+    ap.add_argument("--cpu-tokens", type=int, default=16, help="token sample of the one-core CPU baseline")
+    ap.add_argument("--cpu-tokens-per-core", type=int, default=4, help="tokens per thread of the all-core CPU baseline")
+    ap.add_argument("--cpu-tokens-ref", type=int, default=2, help="tokens per thread and step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the decode and FP4 keys of the prefill line")
     ap.add_argument("--workload", choices=["prefill", "decode", "quant-variants"], default="prefill",
                     help="prefill: the headline step; decode: per-token-batch latency sweep; "
                          "quant-variants: the 4-bit quantizer and its ablation variants at the 7B prefill input")
