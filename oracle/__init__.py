@@ -66,6 +66,9 @@ def _load():
             "orc_ternary_codes": [P, I64, I64, I64, F, F, P],
             "orc_gemm": [P, I64, P, P, P, I64, I64, I64, I64, P, I64, P, P],
             "orc_kv_quant": [P, I64, I64, I64, I64, ctypes.c_int, I64, F, P, P],
+            "orc_rmsnorm_sumsq": [P, I64, I64, I64, P, P],
+            "orc_rmsnorm_apply": [P, I64, I64, I64, P, P, F, P, P],
+            "orc_quant_int4_given_beta": [P, I64, I64, I64, F, F, P, P],
             "orc_rounding_is_nearest": [],
         }
         for name, args in sigs.items():
@@ -199,6 +202,66 @@ def relu2_glu(gate_bf16: np.ndarray, up_bf16: np.ndarray, keep: int, eps: float 
     _check(_load().orc_relu2_glu(_ptr(gate), _ptr(up), M, F, F, keep, eps, _ptr(codes), _ptr(mask),
                                  _ptr(h), _ptr(gamma), _ptr(scale)), "relu2_glu")
     return (codes, mask, gamma, scale, h) if want_h else (codes, mask, gamma, scale)
+
+
+# ---------------------------------------------------------------------------
+# RMSNorm ahead of the 4-bit quantizer (§3.2's data flow), and per-tensor INT4
+# ---------------------------------------------------------------------------
+def rmsnorm(x_bf16: np.ndarray, gamma=None, eps_norm: float = 1e-6):
+    """y = bf16((x * r) * g), r = 1 / sqrt(ms + eps_norm) per row, ms the exact
+    mean of x^2 rounded once to fp32, the rest single fp32 operations (see
+    bitlinear_oracle.c).  Returns (y bf16 bits uint16 [M,K], r fp32 [M])."""
+    x = _bf16_2d(x_bf16)
+    M, K = x.shape
+    g = None if gamma is None else np.ascontiguousarray(gamma, dtype=np.float32)
+    if g is not None and g.shape != (K,):
+        raise ValueError("gamma must have K entries")
+    if not eps_norm > 0:
+        raise ValueError("eps_norm must be positive")
+    hi = np.empty(M, np.float64)
+    lo = np.empty(M, np.float64)
+    _check(_load().orc_rmsnorm_sumsq(_ptr(x), M, K, K, _ptr(hi), _ptr(lo)), "rmsnorm_sumsq")
+    ms = np.array([round_fraction_to_f32((Fraction(float(h)) + Fraction(float(l))) / K) for h, l in zip(hi, lo)],
+                  np.float32)
+    y = np.empty((M, K), np.uint16)
+    r = np.empty(M, np.float32)
+    _check(_load().orc_rmsnorm_apply(_ptr(x), M, K, K, _ptr(ms), _ptr(g), np.float32(eps_norm), _ptr(y), _ptr(r)),
+           "rmsnorm_apply")
+    return y, r
+
+
+def rmsnorm_quant(x_bf16: np.ndarray, gamma=None, eps_norm: float = 1e-6, quant: str = "int4", eps: float = EPS):
+    """The 4-bit quantizer applied to the RMSNorm output: quant_int4 (returns
+    (codes, beta, scale)) or quant_fp4 (returns (code4, twice, p, scale)) of
+    rmsnorm(x)."""
+    y, _ = rmsnorm(x_bf16, gamma, eps_norm)
+    if quant == "int4":
+        return quant_int4(y, eps)
+    if quant == "fp4":
+        return quant_fp4(y)
+    raise ValueError(quant)
+
+
+def tensor_abs_mean_bf16(x_bf16: np.ndarray) -> np.float32:
+    """The exact mean of |x| over every entry of a bf16 tensor, rounded once to
+    fp32 (the bf16 values are exact in fp32, so the exponent-bin sum of
+    ternary_alpha applies unchanged)."""
+    x = _bf16_2d(x_bf16)
+    return ternary_alpha((x.astype(np.uint32) << 16).view(np.float32))
+
+
+def quant_int4_per_tensor(x_bf16: np.ndarray, eps: float = EPS):
+    """INT4 absmean with beta = mean|X| over the whole tensor (per-tensor
+    scaling).  Returns (codes int8 [M,K], beta fp32, scale fp32 [M], every
+    entry beta/sqrt7)."""
+    x = _bf16_2d(x_bf16)
+    M, K = x.shape
+    beta = tensor_abs_mean_bf16(x)
+    codes = np.empty((M, K), np.int8)
+    scale = np.empty(M, np.float32)
+    _check(_load().orc_quant_int4_given_beta(_ptr(x), M, K, K, np.float32(beta), eps, _ptr(codes), _ptr(scale)),
+           "quant_int4_given_beta")
+    return codes, beta, scale
 
 
 # ---------------------------------------------------------------------------

@@ -484,5 +484,109 @@ int orc_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D, int64_t ld
     return ORC_OK;
 }
 
+/* ---------------------------------------------------------------------------
+ * RMSNorm ahead of the 4-bit quantizer (§3.2's per-layer data flow: RMSNorm ->
+ * 4-bit quantize -> QKV / Up|Gate BitLinear).  The pages name the step without
+ * a formula; the reading used is the usual root-mean-square normalization with
+ * a per-channel weight, its output an activation tensor in bf16 like every
+ * other one:
+ *   ms = mean(x^2) over the row,  s = sqrt(ms + eps_n),  r = 1 / s,
+ *   y_k = bf16( (x_k * r) * g_k )      (g_k = 1 without a weight).
+ * The arithmetic is fixed so that it can be reproduced exactly: ms is the exact
+ * mean of the squares rounded once to fp32 (order-free); ms + eps_n, the square
+ * root, 1 / s and the two products are single IEEE fp32 operations, each
+ * rounded to nearest even; the last result is rounded once to bf16.
+ *
+ * orc_rmsnorm_sumsq gives the exact sum of squares of each row as an unevaluated
+ * pair hi + lo of doubles (the caller divides and rounds with exact rationals).
+ * Each x^2 is exact in fp64; the pair is a double-double accumulation whose
+ * every step is checked to be exact (TwoSum), and the row is rejected unless
+ * the squares, as multiples of the smallest one's last significant bit, stay
+ * below 2^106 in sum -- then every order of accumulation is exact as well.
+ * orc_rmsnorm_apply takes ms and forms y and r.
+ * ------------------------------------------------------------------------- */
+static void two_sum(double a, double b, double* s, double* e) {
+    double t = a + b;
+    double bp = t - a;
+    *e = (a - (t - bp)) + (b - bp);
+    *s = t;
+}
+
+int orc_rmsnorm_sumsq(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, double* hi_out, double* lo_out) {
+    if (M < 0 || K <= 0 || ldx < K) return ORC_ERR_ARG;
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t* row = x + m * ldx;
+        double hi = 0.0, lo = 0.0;
+        int lowbit = INT32_MAX;            /* exponent of the lowest significant bit over the squares */
+        for (int64_t k = 0; k < K; ++k) {
+            double v = (double)bf16_value(row[k]);
+            if (!isfinite(v)) return ORC_ERR_NONFINITE;
+            double a = v * v;              /* exact: an 8-bit significand squared, within fp64's range */
+            if (a != 0.0) {
+                int e;
+                double f = frexp(a, &e);   /* a = f * 2^e, f in [0.5, 1) */
+                int b = e - 53;            /* a = (f * 2^53) * 2^b with f * 2^53 an integer */
+                double n = ldexp(f, 53);
+                while (fmod(n, 2.0) == 0.0) { n /= 2.0; ++b; }
+                if (b < lowbit) lowbit = b;
+            }
+            double t, e1, e2;
+            two_sum(hi, a, &t, &e1);
+            two_sum(lo, e1, &lo, &e2);
+            if (e2 != 0.0) return ORC_ERR_INEXACT_SUM;
+            hi = t;
+        }
+        if (hi != 0.0) {
+            int e;
+            frexp(hi + lo, &e);            /* the sum is below 2^e (within a rounding) */
+            if (e + 1 - lowbit > 106) return ORC_ERR_INEXACT_SUM;
+        }
+        hi_out[m] = hi;
+        lo_out[m] = lo;
+    }
+    return ORC_OK;
+}
+
+int orc_rmsnorm_apply(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const float* ms, const float* g,
+                      float eps_n, uint16_t* y, float* r_out) {
+    if (M < 0 || K <= 0 || ldx < K || !(eps_n > 0.0f)) return ORC_ERR_ARG;
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t* row = x + m * ldx;
+        float s = sqrtf(ms[m] + eps_n);
+        float r = 1.0f / s;
+        for (int64_t k = 0; k < K; ++k) {
+            float t = bf16_value(row[k]) * r;
+            if (g) t = t * g[k];
+            y[m * K + k] = bf16_round((double)t);
+        }
+        r_out[m] = r;
+    }
+    return ORC_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * INT4 absmean with one scale for the whole tensor (the per-tensor scaling of
+ * the ablations, Fig. 5 / Fig. 6; also the literal reading of Eq. 6-7, whose
+ * mean runs over all entries of X): the same codes as orc_quant_int4 but with
+ * a given beta, the exact mean of |X| over all M*K entries rounded once to fp32
+ * (the caller forms it from orc_ternary_abs_bins on the exact fp32 values).
+ * ------------------------------------------------------------------------- */
+int orc_quant_int4_given_beta(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float beta, float eps,
+                              int8_t* codes, float* scale_out) {
+    if (M < 0 || K <= 0 || ldx < K) return ORC_ERR_ARG;
+    const float sqrt7 = (float)sqrt(7.0);
+    const float mult = sqrt7 / (beta + eps);
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t* row = x + m * ldx;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = bf16_value(row[k]);
+            if (!isfinite(v)) return ORC_ERR_NONFINITE;
+            codes[m * K + k] = (int8_t)round_clip(v * mult, -8.0f, 7.0f);
+        }
+        scale_out[m] = beta / sqrt7;
+    }
+    return ORC_OK;
+}
+
 /* The rounding mode every function above assumes. */
 int orc_rounding_is_nearest(void) { return fegetround() == FE_TONEAREST; }

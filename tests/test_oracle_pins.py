@@ -502,3 +502,110 @@ def test_fp4_e1m2_exhaustive_bf16_is_rint_of_4x():
         neg = (v < 0) & (idx != 0)
         assert np.array_equal(fv[0, :-1].astype(np.int64), np.where(neg, -idx, idx))
         assert np.array_equal(code4[0, :-1].astype(np.int64), idx | np.where(neg, 8, 0))
+
+
+# ----------------------------------------------------------------------------
+# RMSNorm ahead of the 4-bit quantizer (§3.2 data flow; formula a reading)
+# ----------------------------------------------------------------------------
+def test_rmsnorm_hand_examples():
+    g = read_golden("rmsnorm_hand.txt")
+    for xs, gs, ys in zip(g["x"], g["g"], g["y"]):
+        y, _ = oracle.rmsnorm(bf16([xs]), gamma=np.array(gs, np.float32), eps_norm=1e-8)
+        assert bf16_val(y)[0].tolist() == ys
+
+
+def test_rmsnorm_within_bf16_rounding_of_exact():
+    # y against the exact x * g / sqrt(mean(x^2) + eps) in fp64: within half a bf16
+    # ulp plus the few fp32 roundings before it (relative 2^-8 covers both)
+    g = synth.rng(61)
+    x = synth.student_t_bf16(g, (16, 1536))
+    w = (1.0 + 0.25 * g.standard_normal(1536)).astype(np.float32)
+    y, _ = oracle.rmsnorm(x, gamma=w, eps_norm=1e-6)
+    xf = bf16_val(x).astype(np.float64)
+    exact = xf * w.astype(np.float64) / np.sqrt((xf ** 2).mean(axis=1, keepdims=True) + 1e-6)
+    err = np.abs(bf16_val(y).astype(np.float64) - exact)
+    assert np.all(err <= 2.0 ** -8 * np.abs(exact) + 1e-30)
+
+
+def test_rmsnorm_constant_power_of_two_rows():
+    # x = c everywhere with c a power of two: mean(x^2) = c^2 exactly, sqrt exact,
+    # r = 1/|c| exactly, so y = sign(c) * g
+    w = np.array([1.5, -0.25, 3.0, 0.125] * 8, np.float32)
+    for c in (0.5, -4.0, 2.0 ** -20, 1024.0):
+        y, r = oracle.rmsnorm(bf16([[c] * 32]), gamma=w, eps_norm=1e-30)
+        assert float(r[0]) == 1.0 / abs(c)
+        assert bf16_val(y)[0].tolist() == (np.sign(c) * w).tolist()
+
+
+def test_rmsnorm_zero_row_and_eps():
+    y, r = oracle.rmsnorm(np.zeros((1, 8), np.uint16), eps_norm=0.25)
+    assert not y.any() and float(r[0]) == 2.0           # 1/sqrt(0 + 0.25)
+    with pytest.raises(ValueError):
+        oracle.rmsnorm(np.zeros((1, 8), np.uint16), eps_norm=0.0)
+
+
+def test_rmsnorm_quant_constant_row_codes():
+    # after the norm a constant row is all g; with g = 1, beta = 1 and every code is
+    # RoundClip(sqrt7 / (1 + eps)) = 3 (INT4); for FP4 the smallest p with 1 <= 6 * 2^p
+    # is -2, so every value is 1 * 2^2 = 4, E2M1 code 0b110
+    c, b, _ = oracle.rmsnorm_quant(bf16([[-6.0] * 64, [0.375] * 64]), quant="int4")
+    assert c.tolist() == [[-3] * 64, [3] * 64] and b.tolist() == [1.0, 1.0]
+    code4, _, p, _ = oracle.rmsnorm_quant(bf16([[0.375] * 64]), quant="fp4")
+    assert set(code4[0].tolist()) == {0x6} and p[0] == -2
+
+
+# ----------------------------------------------------------------------------
+# INT4 absmean with a per-tensor scale (ablations; Eq. 6-7 read over all of X)
+# ----------------------------------------------------------------------------
+def test_int4_per_tensor_hand_example():
+    g = read_golden("int4_per_tensor_hand.txt")
+    c, beta, scale = oracle.quant_int4_per_tensor(bf16(g["x"]))
+    assert c.tolist() == [[int(v) for v in row] for row in g["codes"]]
+    assert float(beta) == g["beta"][0][0]
+    assert np.all(scale == np.float32(beta) / np.float32(math.sqrt(7)))
+
+
+def test_int4_per_tensor_single_row_is_per_token():
+    # with one token the tensor mean is the token mean: the pinned per-token quantizer
+    x = synth.gaussian_bf16(synth.rng(62), (1, 3200))
+    c1, b1, s1 = oracle.quant_int4(x)
+    c2, b2, s2 = oracle.quant_int4_per_tensor(x)
+    assert np.array_equal(c1, c2) and float(b1[0]) == float(b2) and s1[0] == s2[0]
+
+
+def test_int4_per_tensor_beta_exact_mean_brute_force():
+    # beta is the exact rational mean of |x| rounded once to fp32 (checked with
+    # Fractions), and permuting the rows changes nothing but the row order
+    g = synth.rng(63)
+    x = synth.student_t_bf16(g, (7, 96))
+    x[0, :5] = bf16([1e-30, 3e30, -2.5e-38, 65504.0, -1e-3])
+    exact = sum(Fraction(float(abs(v))) for v in bf16_val(x).ravel()) / x.size
+    c, beta, _ = oracle.quant_int4_per_tensor(x)
+    assert float(beta) == float(oracle.round_fraction_to_f32(exact))
+    perm = g.permutation(7)
+    c2, beta2, _ = oracle.quant_int4_per_tensor(x[perm])
+    assert float(beta2) == float(beta) and np.array_equal(c2, c[perm])
+
+
+def test_int4_per_tensor_constant_tensor():
+    c, beta, _ = oracle.quant_int4_per_tensor(bf16([[-0.5] * 16] * 3))
+    assert float(beta) == 0.5 and set(c.ravel().tolist()) == {-3}
+
+
+def test_rmsnorm_mean_is_exact_and_rejects_wide_rows():
+    # ms is the exact mean of the squares rounded once: checked with Fractions on rows
+    # that defeat a plain fp64 sum (squares spanning ~80 bits); a row whose squares
+    # span beyond 106 bits is outside the contract and rejected
+    g = synth.rng(64)
+    x = synth.gaussian_bf16(g, (4, 512))
+    x[1, :3] = bf16([1e-6, 3e3, -7e-7])
+    y, r = oracle.rmsnorm(x, eps_norm=1e-6)
+    for i in range(4):
+        sq = sum(Fraction(float(v)) ** 2 for v in bf16_val(x[i]))
+        ms = oracle.round_fraction_to_f32(sq / 512)
+        s = np.sqrt(np.float32(ms) + np.float32(1e-6), dtype=np.float32)
+        assert float(r[i]) == float(np.float32(1.0) / s)
+    wide = np.zeros((1, 8), np.uint16)
+    wide[0, :2] = bf16([1e30, 1e-30])
+    with pytest.raises(ValueError):
+        oracle.rmsnorm(wide)
