@@ -718,9 +718,19 @@ def run_quant_variants(args):
     variants = [("int4_absmean", tba.BL_QUANT_INT4), ("fp4_e2m1", tba.BL_QUANT_FP4_E2M1),
                 ("int4_absmax", tba.BL_QUANT_INT4_ABSMAX), ("int4_absmean_2beta", tba.BL_QUANT_INT4_ABSMEAN2),
                 ("fp4_e1m2", tba.BL_QUANT_FP4_E1M2)]
+    gnorm = (1.0 + 0.3 * torch.randn((k,), device=dev)).float()
+    beta = torch.empty((1,), dtype=torch.float32, device=dev)
+    ws = torch.empty((tba.workspace_size("quant_a4_per_tensor") // 8,), dtype=torch.int64, device=dev)
+    calls = [(name, (lambda q=q: tba.bitlinear_quant_a4(x, codes, scale, q, tba.BL_STORE_BYTES, EPS)))
+             for name, q in variants]
+    # RMSNorm fused in front of INT4 (one read of x), and INT4 with one scale for the
+    # tensor (a pass for the exact mean |x|, then the quantizer: x is read twice)
+    calls.append(("rmsnorm_int4", lambda: tba.bitlinear_rmsnorm_quant_a4(x, codes, scale, gamma=gnorm, eps_norm=1e-6,
+                                                                         store=tba.BL_STORE_BYTES, eps=EPS)))
+    calls.append(("int4_per_tensor", lambda: tba.bitlinear_quant_a4_per_tensor(x, codes, scale, beta, ws,
+                                                                              store=tba.BL_STORE_BYTES, eps=EPS)))
     results = []
-    for name, q in variants:
-        fn = lambda: tba.bitlinear_quant_a4(x, codes, scale, q, tba.BL_STORE_BYTES, EPS)
+    for name, fn in calls:
         for _ in range(args.warmup):
             fn()
         torch.cuda.synchronize()
@@ -735,8 +745,11 @@ def run_quant_variants(args):
         tba.sync_status()
         ms = sorted(ts)[len(ts) // 2]
         gbs = nbytes / (ms / 1e3) / 1e9
-        results.append({"variant": name, "us": round(ms * 1e3, 1), "gbs": round(gbs, 1),
-                        "hbm_frac": round(gbs / peaks["hbm_gbs"], 3)})
+        r = {"variant": name, "us": round(ms * 1e3, 1), "gbs": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 3)}
+        if name == "int4_per_tensor":
+            moved = nbytes + m * 2 * k        # x is read by both passes
+            r["hbm_frac_bytes_moved"] = round(moved / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 3)
+        results.append(r)
     line = {"metric": "4-bit activation quantizer GB/s per variant (7B QKV input)", "unit": "GB/s",
             "workload": f"X bf16 [{m} x {k}] -> int8 codes + fp32 scale per token (median of {args.steps} launches)",
             "algorithmic_bytes": nbytes, "hbm_peak_gbs": peaks["hbm_gbs"], "results": results}

@@ -122,6 +122,47 @@ BL_API bl_status bitlinear_quant_a4(const void* x_bf16, int64_t M, int64_t K, in
                              void* codes, float* scale, void* stream);
 
 /*
+ * bitlinear_rmsnorm_quant_a4 -- RMSNorm fused into the 4-bit quantizer: the
+ * per-layer data flow puts an RMSNorm before each 4-bit quantization (paper:
+ * §3.2, "RMSNorm -> 4-bit quantize -> attention QKV" and "-> FFN Up/Gate"); this
+ * call reads x once and writes exactly the codes and scales that
+ * bitlinear_quant_a4 writes for y = RMSNorm(x).
+ * RMSNorm (the pages give no formula; reading used):
+ *   ms = mean(x^2) over the row -- the exact mean of the squares, rounded once
+ *        to fp32 (order-free; the contract covers rows whose squares, as
+ *        multiples of the smallest one's last significant bit, sum below 2^90,
+ *        true for ordinary data),
+ *   r  = 1 / sqrt(ms + eps_norm),  y_k = bf16((x_k * r) * gamma_k),
+ * each operation a single IEEE fp32 operation rounded to nearest even, the
+ * last to bf16; gamma NULL means gamma_k = 1 (then y_k = bf16(x_k * r)).
+ * Then quant as in bitlinear_quant_a4 (any bl_quant, either bl_store).
+ * x: [M x K] bf16, row stride ldx.  gamma: [K] fp32 (nullable, 16-byte
+ * aligned).  codes / scale as in bitlinear_quant_a4.
+ * Requires K % 8 == 0, 8 <= K <= 16384, ldx % 8 == 0, eps_norm > 0 (finite).
+ */
+BL_API bl_status bitlinear_rmsnorm_quant_a4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                                            const float* gamma, float eps_norm, bl_quant quant, bl_store store,
+                                            float eps, void* codes, float* scale, void* stream);
+
+/*
+ * bitlinear_quant_a4_per_tensor -- INT4 absmean with one scale for the whole
+ * tensor: beta = mean|X| over all M x K entries (the per-tensor scaling of the
+ * ablations, Fig. 5 / Fig. 6; also the literal reading of Eq. 6-7, whose mean
+ * runs over all entries of X).  beta is the exact mean rounded once to fp32
+ * (the exponent-bin sum of pack_ternary), then every row is quantized as by
+ * BL_QUANT_INT4 with that beta: code = RoundClip(x * fp32(sqrt7)/(beta + eps),
+ * -8, 7), scale[m] = beta / fp32(sqrt7) for every m.
+ * x: [M x K] bf16, row stride ldx.  codes / scale as in bitlinear_quant_a4
+ * (BL_STORE_PACKED or BL_STORE_BYTES).  beta: one device float, written.
+ * workspace: bitlinear_workspace_size("quant_a4_per_tensor", M, K, 0) bytes
+ * (2 KiB, 8-byte aligned, cleared by the call).
+ * Requires K % 8 == 0, 8 <= K <= 16384, ldx % 8 == 0, M * K < 2^31.
+ */
+BL_API bl_status bitlinear_quant_a4_per_tensor(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                                               bl_store store, float eps, void* codes, float* scale, float* beta,
+                                               void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * bitlinear_sparsify_a8 -- Top-K sparsification then INT8 absmax quantization
  * for the outlier-heavy inputs (attention-output and FFN-down inputs).
  * Paper: §3.4 "Sparsification Pipeline for Outlier-Heavy Intermediate States",
@@ -302,7 +343,8 @@ BL_API bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D,
                     int64_t bos_pos, float eps, uint8_t* codes, float* scale, uint8_t* bos_codes,
                     void* stream);
 
-/* Bytes of device workspace an operation needs ("pack_ternary"; 0 for the others). */
+/* Bytes of device workspace an operation needs ("pack_ternary", "quant_a4_per_tensor",
+ * "quant_gemm"; 0 for the others). */
 BL_API size_t bitlinear_workspace_size(const char* op, int64_t M, int64_t N, int64_t K);
 
 /* Synchronizes `stream`, then reads and clears the calling device's status

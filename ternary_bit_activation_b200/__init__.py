@@ -27,7 +27,8 @@ BL_STORE_PACKED, BL_STORE_BYTES = 0, 1
 BL_A_I8, BL_A_I4, BL_A_E2M1 = 0, 1, 2
 BL_W_T2, BL_W_I8, BL_W_E2M1 = 0, 1, 2
 
-EXPORTED = ["bitlinear_quant_a4", "bitlinear_sparsify_a8", "pack_ternary", "pack_ternary_noalloc", "bitlinear_gemm",
+EXPORTED = ["bitlinear_quant_a4", "bitlinear_rmsnorm_quant_a4", "bitlinear_quant_a4_per_tensor",
+            "bitlinear_sparsify_a8", "pack_ternary", "pack_ternary_noalloc", "bitlinear_gemm",
             "bitlinear_quant_gemm", "bitlinear_gemm_gated", "relu2_glu", "kv_quant3", "bitlinear_workspace_size",
             "bitlinear_sync_status", "bitlinear_selftest_timeout", "bitlinear_status_string",
             "bitlinear_last_cuda_error", "bitlinear_version"]
@@ -54,6 +55,8 @@ def lib():
         P, I64, F, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
         sig = {
             "bitlinear_quant_a4": [P, I64, I64, I64, I, I, F, P, P, P],
+            "bitlinear_rmsnorm_quant_a4": [P, I64, I64, I64, P, F, I, I, F, P, P, P],
+            "bitlinear_quant_a4_per_tensor": [P, I64, I64, I64, I, F, P, P, P, P, ctypes.c_size_t, P],
             "bitlinear_sparsify_a8": [P, I64, I64, I64, I64, F, P, P, P, P],
             "pack_ternary": [P, I64, I64, I64, F, I, P, I, P, P, ctypes.c_size_t, P],
             "pack_ternary_noalloc": [P, I64, I64, I64, F, I, P, I, P, P],
@@ -108,6 +111,26 @@ def bitlinear_quant_a4(x, codes, scale, quant=BL_QUANT_INT4, store=BL_STORE_PACK
     ldx = x.stride(0) if ldx is None else ldx
     _check("bitlinear_quant_a4", lib().bitlinear_quant_a4(_ptr(x), M, K, ldx, quant, store, eps, _ptr(codes),
                                                           _ptr(scale), _stream(stream)))
+
+
+def bitlinear_rmsnorm_quant_a4(x, codes, scale, gamma=None, eps_norm=1e-6, quant=BL_QUANT_INT4,
+                               store=BL_STORE_PACKED, eps=1e-5, ldx=None, stream=None):
+    """RMSNorm (x * r * gamma, r = 1/sqrt(mean(x^2) + eps_norm)) fused into the
+    4-bit quantizer: the codes and scales of bitlinear_quant_a4 on RMSNorm(x)."""
+    M, K = x.shape
+    ldx = x.stride(0) if ldx is None else ldx
+    _check("bitlinear_rmsnorm_quant_a4", lib().bitlinear_rmsnorm_quant_a4(
+        _ptr(x), M, K, ldx, _ptr(gamma), eps_norm, quant, store, eps, _ptr(codes), _ptr(scale), _stream(stream)))
+
+
+def bitlinear_quant_a4_per_tensor(x, codes, scale, beta, workspace, store=BL_STORE_PACKED, eps=1e-5, ldx=None,
+                                  stream=None):
+    """INT4 absmean with beta = the exact mean |x| over the whole tensor."""
+    M, K = x.shape
+    ldx = x.stride(0) if ldx is None else ldx
+    ws = workspace.numel() * workspace.element_size()
+    _check("bitlinear_quant_a4_per_tensor", lib().bitlinear_quant_a4_per_tensor(
+        _ptr(x), M, K, ldx, store, eps, _ptr(codes), _ptr(scale), _ptr(beta), _ptr(workspace), ws, _stream(stream)))
 
 
 def bitlinear_sparsify_a8(x, k_keep, codes, scale, mask=None, eps=1e-5, stream=None):

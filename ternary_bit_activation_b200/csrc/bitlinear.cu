@@ -188,29 +188,60 @@ bool tc_kernel_ready() {
 // ---------------------------------------------------------------------------
 // launch helpers
 // ---------------------------------------------------------------------------
+// The optional parts of a quantizer launch: the RMSNorm prologue (gnorm may be
+// NULL for a unit weight) and the tensor-wide beta of kQInt4Tensor.
+struct QuantExtra {
+  bool norm = false;
+  const float* gnorm = nullptr;
+  float eps_n = 0.f;
+  const float* beta = nullptr;
+};
+
 template <int C, int VAR>
 void launch_quant_a4_cv(const uint16_t* x, int64_t M, int K, int64_t ldx, bool packed, float eps, uint8_t* codes,
-                        float* scale, cudaStream_t s, dim3 grid) {
-  if (packed) launch_pdl(bl::quant_a4_kernel<C, VAR, true>, grid, 256, 0, s, x, M, K, ldx, eps, codes, scale);
-  else launch_pdl(bl::quant_a4_kernel<C, VAR, false>, grid, 256, 0, s, x, M, K, ldx, eps, codes, scale);
+                        float* scale, cudaStream_t s, dim3 grid, const QuantExtra& q) {
+  auto go = [&](auto kern) { launch_pdl(kern, grid, 256, 0, s, x, M, K, ldx, eps, codes, scale, q.gnorm, q.eps_n, q.beta); };
+  if (q.norm) {
+    if (packed) go(bl::quant_a4_kernel<C, VAR, true, true>);
+    else go(bl::quant_a4_kernel<C, VAR, false, true>);
+  } else {
+    if (packed) go(bl::quant_a4_kernel<C, VAR, true, false>);
+    else go(bl::quant_a4_kernel<C, VAR, false, false>);
+  }
 }
 
 template <int C>
 void launch_quant_a4_c(const uint16_t* x, int64_t M, int K, int64_t ldx, int var, bool packed, float eps,
-                       uint8_t* codes, float* scale, cudaStream_t s) {
+                       uint8_t* codes, float* scale, cudaStream_t s, const QuantExtra& q) {
   // persistent: two rows per CTA and iteration, eight CTAs per SM
   const int64_t need = (M + 1) / 2;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   const dim3 grid(static_cast<unsigned>(need < cap ? need : cap));
   switch (var) {
-    case bl::kQInt4: launch_quant_a4_cv<C, bl::kQInt4>(x, M, K, ldx, packed, eps, codes, scale, s, grid); break;
-    case bl::kQFp4: launch_quant_a4_cv<C, bl::kQFp4>(x, M, K, ldx, packed, eps, codes, scale, s, grid); break;
-    case bl::kQInt4Absmax: launch_quant_a4_cv<C, bl::kQInt4Absmax>(x, M, K, ldx, packed, eps, codes, scale, s, grid); break;
-    case bl::kQInt4Absmean2:
-      launch_quant_a4_cv<C, bl::kQInt4Absmean2>(x, M, K, ldx, packed, eps, codes, scale, s, grid);
+    case bl::kQInt4: launch_quant_a4_cv<C, bl::kQInt4>(x, M, K, ldx, packed, eps, codes, scale, s, grid, q); break;
+    case bl::kQFp4: launch_quant_a4_cv<C, bl::kQFp4>(x, M, K, ldx, packed, eps, codes, scale, s, grid, q); break;
+    case bl::kQInt4Absmax:
+      launch_quant_a4_cv<C, bl::kQInt4Absmax>(x, M, K, ldx, packed, eps, codes, scale, s, grid, q);
       break;
-    default: launch_quant_a4_cv<C, bl::kQFp4E1M2>(x, M, K, ldx, packed, eps, codes, scale, s, grid); break;
+    case bl::kQInt4Absmean2:
+      launch_quant_a4_cv<C, bl::kQInt4Absmean2>(x, M, K, ldx, packed, eps, codes, scale, s, grid, q);
+      break;
+    case bl::kQInt4Tensor:
+      launch_quant_a4_cv<C, bl::kQInt4Tensor>(x, M, K, ldx, packed, eps, codes, scale, s, grid, q);
+      break;
+    default: launch_quant_a4_cv<C, bl::kQFp4E1M2>(x, M, K, ldx, packed, eps, codes, scale, s, grid, q); break;
   }
+}
+
+// The quantizer launch for rows of K values (chunks of 8 per thread and row).
+void launch_quant_a4(const uint16_t* x, int64_t M, int K, int64_t ldx, int var, bool packed, float eps,
+                     uint8_t* codes, float* scale, cudaStream_t s, const QuantExtra& q) {
+  const int64_t c = (K / 8 + bl::kQ4ThreadsPerRow - 1) / bl::kQ4ThreadsPerRow;
+  if (c <= 1) launch_quant_a4_c<1>(x, M, K, ldx, var, packed, eps, codes, scale, s, q);
+  else if (c <= 2) launch_quant_a4_c<2>(x, M, K, ldx, var, packed, eps, codes, scale, s, q);
+  else if (c <= 4) launch_quant_a4_c<4>(x, M, K, ldx, var, packed, eps, codes, scale, s, q);
+  else if (c <= 8) launch_quant_a4_c<8>(x, M, K, ldx, var, packed, eps, codes, scale, s, q);
+  else launch_quant_a4_c<16>(x, M, K, ldx, var, packed, eps, codes, scale, s, q);
 }
 
 // Top-K rows: one 256-thread CTA per row, persistent grid sized by the occupancy
@@ -337,7 +368,7 @@ int bins_ctas_per_sm() {
   if (d < 0 || d >= kMaxDevices) return 4;
   if (per_sm[d] == 0) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bl::ternary_bins_kernel, bl::kBinThreads, 0) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bl::ternary_bins_kernel<false>, bl::kBinThreads, 0) != cudaSuccess ||
         n < 1)
       n = 1;
     per_sm[d] = n;
@@ -563,7 +594,8 @@ bl_status pack_ternary_noalloc(const float* w, int64_t N, int64_t K, int64_t ldw
     int64_t blocks = (total + bl::kBinThreads - 1) / bl::kBinThreads;
     const int64_t cap = static_cast<int64_t>(sm_count()) * bins_ctas_per_sm();   // one resident wave
     if (blocks > cap) blocks = cap;
-    launch_pdl(bl::ternary_bins_kernel, static_cast<unsigned>(blocks), bl::kBinThreads, 0, s, w, N, k, ldw, bins, alpha);
+    launch_pdl(bl::ternary_bins_kernel<false>, static_cast<unsigned>(blocks), bl::kBinThreads, 0, s,
+               static_cast<const void*>(w), N, k, ldw, bins, alpha);
     if (launch_status() != BL_OK) return BL_ERR_CUDA;
   }
   const int64_t total16 = N * (K / 16);
@@ -601,7 +633,8 @@ const char* bitlinear_status_string(bl_status st) {
 
 size_t bitlinear_workspace_size(const char* op, int64_t M, int64_t N, int64_t K) {
   (void)N;
-  if (op != nullptr && strcmp(op, "pack_ternary") == 0) return bl::kBins * sizeof(unsigned long long);
+  if (op != nullptr && (strcmp(op, "pack_ternary") == 0 || strcmp(op, "quant_a4_per_tensor") == 0))
+    return bl::kBins * sizeof(unsigned long long);
   if (op != nullptr && strcmp(op, "quant_gemm") == 0 && M > 0 && K > 0)
     return static_cast<size_t>(qg_workspace_bytes(M, K));
   return 0;
@@ -636,18 +669,66 @@ bl_status bitlinear_quant_a4(const void* x_bf16, int64_t M, int64_t K, int64_t l
   if (x_bf16 == nullptr || codes == nullptr || scale == nullptr) return BL_ERR_NULL;
   if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scale)) return BL_ERR_ALIGN;
   if (!(eps >= 0.f)) return BL_ERR_ARG;
-  const int64_t c = (K / 8 + bl::kQ4ThreadsPerRow - 1) / bl::kQ4ThreadsPerRow;
   const int var = static_cast<int>(quant);   // bl_quant values are the kernel's variant ids
-  const bool packed = store == BL_STORE_PACKED;
-  const uint16_t* x = static_cast<const uint16_t*>(x_bf16);
-  uint8_t* out = static_cast<uint8_t*>(codes);
+  launch_quant_a4(static_cast<const uint16_t*>(x_bf16), M, static_cast<int>(K), ldx, var, store == BL_STORE_PACKED,
+                  eps, static_cast<uint8_t*>(codes), scale, as_stream(stream), QuantExtra());
+  return launch_status();
+}
+
+bl_status bitlinear_rmsnorm_quant_a4(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, const float* gamma,
+                                     float eps_norm, bl_quant quant, bl_store store, float eps, void* codes,
+                                     float* scale, void* stream) {
+  NvtxRange nvtx_range("bitlinear_rmsnorm_quant_a4");
+  if (quant != BL_QUANT_INT4 && quant != BL_QUANT_FP4_E2M1 && quant != BL_QUANT_INT4_ABSMAX &&
+      quant != BL_QUANT_INT4_ABSMEAN2 && quant != BL_QUANT_FP4_E1M2)
+    return BL_ERR_ARG;
+  if (store != BL_STORE_PACKED && store != BL_STORE_BYTES) return BL_ERR_ARG;
+  if (M < 0 || K < 8 || K > 16384 || (K & 7) || ldx < K || (ldx & 7) || M > 0x7FFFFFFELL) return BL_ERR_SHAPE;
+  if (!(eps >= 0.f) || !(eps_norm > 0.f) || !(eps_norm < 3.4e38f)) return BL_ERR_ARG;
+  if (M == 0) return BL_OK;
+  if (x_bf16 == nullptr || codes == nullptr || scale == nullptr) return BL_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scale) || (gamma && !aligned16(gamma)))
+    return BL_ERR_ALIGN;
+  QuantExtra q;
+  q.norm = true;
+  q.gnorm = gamma;
+  q.eps_n = eps_norm;
+  launch_quant_a4(static_cast<const uint16_t*>(x_bf16), M, static_cast<int>(K), ldx, static_cast<int>(quant),
+                  store == BL_STORE_PACKED, eps, static_cast<uint8_t*>(codes), scale, as_stream(stream), q);
+  return launch_status();
+}
+
+bl_status bitlinear_quant_a4_per_tensor(const void* x_bf16, int64_t M, int64_t K, int64_t ldx, bl_store store,
+                                        float eps, void* codes, float* scale, float* beta, void* workspace,
+                                        size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("bitlinear_quant_a4_per_tensor");
+  if (store != BL_STORE_PACKED && store != BL_STORE_BYTES) return BL_ERR_ARG;
+  if (M < 0 || K < 8 || K > 16384 || (K & 7) || ldx < K || (ldx & 7)) return BL_ERR_SHAPE;
+  // M * K >= limit, tested without forming the product
+  if (M > 0 && M >= (bl::kMaxPackElems + K - 1) / K) return BL_ERR_SHAPE;
+  if (!(eps >= 0.f)) return BL_ERR_ARG;
+  if (M == 0) return BL_OK;
+  if (x_bf16 == nullptr || codes == nullptr || scale == nullptr || beta == nullptr || workspace == nullptr)
+    return BL_ERR_NULL;
+  if (ws_bytes < bl::kBins * sizeof(unsigned long long)) return BL_ERR_WORKSPACE;
+  if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scale) || (reinterpret_cast<uintptr_t>(beta) & 3u) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 7u))
+    return BL_ERR_ALIGN;
   cudaStream_t s = as_stream(stream);
-  const int k = static_cast<int>(K);
-  if (c <= 1) launch_quant_a4_c<1>(x, M, k, ldx, var, packed, eps, out, scale, s);
-  else if (c <= 2) launch_quant_a4_c<2>(x, M, k, ldx, var, packed, eps, out, scale, s);
-  else if (c <= 4) launch_quant_a4_c<4>(x, M, k, ldx, var, packed, eps, out, scale, s);
-  else if (c <= 8) launch_quant_a4_c<8>(x, M, k, ldx, var, packed, eps, out, scale, s);
-  else launch_quant_a4_c<16>(x, M, k, ldx, var, packed, eps, out, scale, s);
+  unsigned long long* bins = static_cast<unsigned long long*>(workspace);
+  if (!cuda_ok(cudaMemsetAsync(bins, 0, bl::kBins * sizeof(unsigned long long), s))) return BL_ERR_CUDA;
+  // the exact mean of |x| over the tensor (the bins kernel of pack_ternary on bf16 values)
+  const int64_t total = M * (K / 8);
+  int64_t blocks = (total + bl::kBinThreads - 1) / bl::kBinThreads;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * bins_ctas_per_sm();
+  if (blocks > cap) blocks = cap;
+  launch_pdl(bl::ternary_bins_kernel<true>, static_cast<unsigned>(blocks), bl::kBinThreads, 0, s, x_bf16, M,
+             static_cast<int>(K), ldx, bins, beta);
+  if (launch_status() != BL_OK) return BL_ERR_CUDA;
+  QuantExtra q;
+  q.beta = beta;
+  launch_quant_a4(static_cast<const uint16_t*>(x_bf16), M, static_cast<int>(K), ldx, bl::kQInt4Tensor,
+                  store == BL_STORE_PACKED, eps, static_cast<uint8_t*>(codes), scale, s, q);
   return launch_status();
 }
 
@@ -707,7 +788,8 @@ bl_status pack_ternary(const float* w, int64_t N, int64_t K, int64_t ldw, float 
     int64_t blocks = (total + bl::kBinThreads - 1) / bl::kBinThreads;
     const int64_t cap = static_cast<int64_t>(sm_count()) * bins_ctas_per_sm();   // one resident wave
     if (blocks > cap) blocks = cap;
-    launch_pdl(bl::ternary_bins_kernel, static_cast<unsigned>(blocks), bl::kBinThreads, 0, s, w, N, k, ldw, bins, alpha);
+    launch_pdl(bl::ternary_bins_kernel<false>, static_cast<unsigned>(blocks), bl::kBinThreads, 0, s,
+               static_cast<const void*>(w), N, k, ldw, bins, alpha);
     if (launch_status() != BL_OK) return BL_ERR_CUDA;
   }
   const int64_t total16 = N * (K / 16);

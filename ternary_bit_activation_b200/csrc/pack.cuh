@@ -57,8 +57,11 @@ __device__ void alpha_from_bins(const unsigned long long* gbins, unsigned long l
                                 unsigned long long* sb);
 
 // gbins (zeroed by the caller): bins 1..255 and, in bin 0, a count of finished
-// CTAs; the last CTA to finish computes alpha.
-__global__ void __launch_bounds__(kBinThreads, 6) ternary_bins_kernel(const float* __restrict__ w, int64_t N, int K,
+// CTAs; the last CTA to finish computes alpha.  BF16: w holds bf16 values (row
+// stride ldw in bf16 elements), each exact as an fp32 -- the same exact mean
+// of |x| for an activation tensor (the per-tensor INT4 scale).
+template <bool BF16>
+__global__ void __launch_bounds__(kBinThreads, 6) ternary_bins_kernel(const void* __restrict__ wv, int64_t N, int K,
                                                                    int64_t ldw,
                                                                    unsigned long long* __restrict__ gbins,
                                                                    float* __restrict__ alpha) {
@@ -68,7 +71,8 @@ __global__ void __launch_bounds__(kBinThreads, 6) ternary_bins_kernel(const floa
   __syncthreads();
   pdl_wait();
   pdl_trigger();
-  const int per_row = K >> 2;  // float4 per row
+  constexpr int kPer = BF16 ? 8 : 4;   // values per 16-byte load
+  const int per_row = K / kPer;        // 16-byte loads per row
   const int64_t gwarp = (static_cast<int64_t>(blockIdx.x) * kBinThreads + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kBinThreads) >> 5;
   constexpr int kLoads = 4;   // float4 loads per lane issued together (16 weights)
@@ -77,30 +81,39 @@ __global__ void __launch_bounds__(kBinThreads, 6) ternary_bins_kernel(const floa
   double acc = 0.0;
   int batches = 0;
   for (int64_t n = gwarp; n < N; n += nwarps) {
-    const float* wrow = w + n * ldw;
+    const uint8_t* wrow = static_cast<const uint8_t*>(wv) + n * ldw * (BF16 ? 2 : 4);
     for (int q0 = 0; q0 < per_row; q0 += 32 * kLoads) {
       // lane 0 asks L2 for the row's batch two ahead (and, at the row's start,
       // the next one too), so each warp keeps three batches in flight
       if (lane == 0) {
         for (int qa = q0 == 0 ? 32 * kLoads : 64 * kLoads; qa <= 64 * kLoads; qa += 32 * kLoads)
           if (q0 + qa < per_row)
-            bulk_prefetch_l2(wrow + static_cast<int64_t>(q0 + qa) * 4,
+            bulk_prefetch_l2(wrow + static_cast<int64_t>(q0 + qa) * 16,
                              static_cast<uint32_t>(min(32 * kLoads, per_row - q0 - qa)) * 16u);
       }
-      uint32_t u[4 * kLoads];
+      uint32_t u[kPer * kLoads];   // |w| as fp32 bit patterns
 #pragma unroll
       for (int j = 0; j < kLoads; ++j) {
         const int q = q0 + j * 32 + lane;
-        const uint4 v = q < per_row ? ld_global_nc_v4(wrow + static_cast<int64_t>(q) * 4) : make_uint4(0, 0, 0, 0);
-        u[4 * j] = v.x & 0x7FFFFFFFu;
-        u[4 * j + 1] = v.y & 0x7FFFFFFFu;
-        u[4 * j + 2] = v.z & 0x7FFFFFFFu;
-        u[4 * j + 3] = v.w & 0x7FFFFFFFu;
+        const uint4 v = q < per_row ? ld_global_nc_v4(wrow + static_cast<int64_t>(q) * 16) : make_uint4(0, 0, 0, 0);
+        if constexpr (BF16) {
+          const uint32_t hw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            u[8 * j + 2 * h] = (hw[h] << 16) & 0x7FFFFFFFu;
+            u[8 * j + 2 * h + 1] = hw[h] & 0x7FFF0000u;
+          }
+        } else {
+          u[4 * j] = v.x & 0x7FFFFFFFu;
+          u[4 * j + 1] = v.y & 0x7FFFFFFFu;
+          u[4 * j + 2] = v.z & 0x7FFFFFFFu;
+          u[4 * j + 3] = v.w & 0x7FFFFFFFu;
+        }
       }
       if (ub == 0) {
         uint32_t amax = 0;
 #pragma unroll
-        for (int i = 0; i < 4 * kLoads; ++i) amax = max(amax, u[i]);
+        for (int i = 0; i < kPer * kLoads; ++i) amax = max(amax, u[i]);
         if (amax != 0) {
           const int E = static_cast<int>(amax >> 23);
           ub = static_cast<uint32_t>(min(max(E - 12, 1), 223));
@@ -108,7 +121,7 @@ __global__ void __launch_bounds__(kBinThreads, 6) ternary_bins_kernel(const floa
         }
       }
 #pragma unroll
-      for (int i = 0; i < 4 * kLoads; ++i) {
+      for (int i = 0; i < kPer * kLoads; ++i) {
         const uint32_t a = u[i];
         if (a - lo_bits < (kWin << 23)) {
           acc += static_cast<double>(__uint_as_float(a));   // exact; 0 before the anchor
@@ -118,7 +131,7 @@ __global__ void __launch_bounds__(kBinThreads, 6) ternary_bins_kernel(const floa
           atomicAdd(&sb[E ? E : 1u], static_cast<unsigned long long>(m));
         }
       }
-      if (++batches == 16) {
+      if (++batches == 128 / kPer) {   // every 256 values per lane (the exact-sum bound above)
         bins_flush(sb, ub, acc);
         batches = 0;
       }

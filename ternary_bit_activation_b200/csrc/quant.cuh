@@ -130,15 +130,86 @@ __device__ __forceinline__ void q4_load(const uint16_t* x, int64_t row, int64_t 
 
 // Quantizer variants (the values of bl_quant): absmean INT4 (Eq. 6-7), MinMax
 // FP4 E2M1 (Eq. 8-9), and the ablation variants INT4 absmax, INT4 absmean with
-// beta = 2 mean|x|, FP4 E1M2.
-enum : int { kQInt4 = 0, kQFp4 = 1, kQInt4Absmax = 2, kQInt4Absmean2 = 3, kQFp4E1M2 = 4 };
+// beta = 2 mean|x|, FP4 E1M2; kQInt4Tensor is absmean INT4 with a beta given in
+// device memory (one for the whole tensor).
+enum : int { kQInt4 = 0, kQFp4 = 1, kQInt4Absmax = 2, kQInt4Absmean2 = 3, kQFp4E1M2 = 4, kQInt4Tensor = 5 };
 
-template <int CHUNKS, int VAR, bool PACKED>
+// ---------------------------------------------------------------------------
+// RMSNorm prologue: ms = the exact mean of x^2 over the row, rounded once to
+// fp32.  Each thread accumulates its squares (exact in fp64) as a double-double
+// hi + lo with TwoSum; the partial pairs are combined the same way.  For rows
+// whose squares, as multiples of the smallest one's last bit, sum below 2^90,
+// every one of these additions is exact, so the pair holds the exact sum
+// whatever the order (the error of a TwoSum is exact; lo stays below n * 2^-53
+// of the sum, n <= 16384, so its additions fit 53 bits).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void two_sum_f64(double a, double b, double& s, double& e) {
+  s = __dadd_rn(a, b);
+  const double bp = __dsub_rn(s, a);
+  e = __dadd_rn(__dsub_rn(a, __dsub_rn(s, bp)), __dsub_rn(b, bp));
+}
+__device__ __forceinline__ void dd_add(double& hi, double& lo, double a) {
+  double s, e;
+  two_sum_f64(hi, a, s, e);
+  hi = s;
+  lo = __dadd_rn(lo, e);
+}
+__device__ __forceinline__ void dd_add_dd(double& hi, double& lo, double h2, double l2) {
+  double s, e;
+  two_sum_f64(hi, h2, s, e);
+  hi = s;
+  lo = __dadd_rn(__dadd_rn(lo, l2), e);
+}
+
+// RN_fp32((hi + lo) / K) for an exact sum hi + lo >= 0: the fp32 nearest to
+// hi / K, then moved while the exact quotient lies beyond a midpoint to a
+// neighbour (at a midpoint: the even one).  A midpoint m has at most 25
+// significant bits and K at most 15, so K * m is exact in fp64, and the sign of
+// (hi - K m) + lo is the sign of the exact S - K m (exact subtraction when hi
+// and K m are within a factor of two, a difference much larger than lo
+// otherwise).
+__device__ __forceinline__ float dd_mean_f32(double hi, double lo, int K) {
+  if (hi == 0.0 && lo == 0.0) return 0.f;
+  const double dk = static_cast<double>(K);
+  float c = __double2float_rn(__ddiv_rn(hi, dk));
+  auto side = [&](float nb) -> int {   // sign of S/K - (c + nb)/2
+    const double mid = 0.5 * (static_cast<double>(c) + static_cast<double>(nb));
+    const double d = __dadd_rn(__dsub_rn(hi, __dmul_rn(mid, dk)), lo);
+    return d > 0.0 ? 1 : (d < 0.0 ? -1 : 0);
+  };
+#pragma unroll 1
+  for (int it = 0; it < 4; ++it) {
+    const bool odd = (__float_as_uint(c) & 1u) != 0u;
+    const float up = nextafterf(c, __int_as_float(0x7F800000));
+    const int su = side(up);
+    if (su > 0 || (su == 0 && odd)) {
+      c = up;
+      continue;
+    }
+    if (c > 0.f) {
+      const float dn = nextafterf(c, 0.f);
+      const int sd = side(dn);
+      if (sd < 0 || (sd == 0 && odd)) {
+        c = dn;
+        continue;
+      }
+    }
+    break;
+  }
+  return c;
+}
+
+// NORM: the row is first replaced by its RMSNorm, y = bf16((x * r) * g),
+// r = 1 / sqrt(ms + eps_n) (fp32 IEEE operations; g = gnorm, or 1 when NULL),
+// and the quantizer runs on y.  VAR == kQInt4Tensor reads beta from *beta_dev.
+template <int CHUNKS, int VAR, bool PACKED, bool NORM>
 __global__ void __launch_bounds__(256) quant_a4_kernel(const uint16_t* __restrict__ x, int64_t M, int K,
                                                        int64_t ldx, float eps, uint8_t* __restrict__ codes,
-                                                       float* __restrict__ scale) {
+                                                       float* __restrict__ scale, const float* __restrict__ gnorm,
+                                                       float eps_n, const float* __restrict__ beta_dev) {
   __shared__ double s_sum[2][2][4];
   __shared__ uint32_t s_max[2][2][4];
+  __shared__ double s_dd[NORM ? 2 : 1][2][4][2];
   const int sub = threadIdx.x >> 7;
   const int t = threadIdx.x & 127;
   const int warp = t >> 5;
@@ -163,7 +234,60 @@ __global__ void __launch_bounds__(256) quant_a4_kernel(const uint16_t* __restric
     }
     const int par = it & 1;
     constexpr bool kSum = VAR == kQInt4 || VAR == kQInt4Absmean2;   // mean|x| statistic, else max|x|
-    constexpr bool kInt = VAR == kQInt4 || VAR == kQInt4Absmean2 || VAR == kQInt4Absmax;
+    constexpr bool kInt = VAR == kQInt4 || VAR == kQInt4Absmean2 || VAR == kQInt4Absmax || VAR == kQInt4Tensor;
+
+    if constexpr (NORM) {
+      // ---- RMSNorm: the exact sum of squares, ms, r, and y in place of x ----
+      double hi = 0.0, lo = 0.0;
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) {
+        float f[8];
+        unpack_bf16x8(v[c], f);   // chunks past K hold zeros
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const double d = static_cast<double>(f[e]);
+          dd_add(hi, lo, __dmul_rn(d, d));
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+        dd_add_dd(hi, lo, __shfl_xor_sync(0xFFFFFFFFu, hi, o), __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+      if (lane == 0) {
+        s_dd[par][sub][warp][0] = hi;
+        s_dd[par][sub][warp][1] = lo;
+      }
+      q4_row_sync(sub);
+      hi = s_dd[par][sub][0][0];
+      lo = s_dd[par][sub][0][1];
+#pragma unroll
+      for (int w = 1; w < 4; ++w) dd_add_dd(hi, lo, s_dd[par][sub][w][0], s_dd[par][sub][w][1]);
+      const float ms = dd_mean_f32(hi, lo, K);
+      const float r = __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(ms, eps_n)));
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) {
+        const int idx = c * kQ4ThreadsPerRow + t;
+        if (idx >= nchunk) continue;
+        float f[8];
+        unpack_bf16x8(v[c], f);
+        float g[8];
+        if (gnorm != nullptr) {
+          const uint4 g0 = ld_global_nc_v4(gnorm + 8 * static_cast<int64_t>(idx));
+          const uint4 g1 = ld_global_nc_v4(gnorm + 8 * static_cast<int64_t>(idx) + 4);
+          g[0] = __uint_as_float(g0.x); g[1] = __uint_as_float(g0.y); g[2] = __uint_as_float(g0.z);
+          g[3] = __uint_as_float(g0.w); g[4] = __uint_as_float(g1.x); g[5] = __uint_as_float(g1.y);
+          g[6] = __uint_as_float(g1.z); g[7] = __uint_as_float(g1.w);
+        }
+        uint32_t hb[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float tv = __fmul_rn(f[e], r);
+          if (gnorm != nullptr) tv = __fmul_rn(tv, g[e]);
+          const __nv_bfloat16 b = __float2bfloat16_rn(tv);
+          hb[e] = *reinterpret_cast<const uint16_t*>(&b);
+        }
+        v[c] = make_uint4(hb[0] | (hb[1] << 16), hb[2] | (hb[3] << 16), hb[4] | (hb[5] << 16), hb[6] | (hb[7] << 16));
+      }
+    }
 
     // ---- the row statistic ----
     double S = 0.0;       // sum |x| (exact in fp64 for in-contract rows: order-free)
@@ -181,7 +305,7 @@ __global__ void __launch_bounds__(256) quant_a4_kernel(const uint16_t* __restric
       if (lane == 0) s_sum[par][sub][warp] = acc;
       q4_row_sync(sub);
       S = (s_sum[par][sub][0] + s_sum[par][sub][1]) + (s_sum[par][sub][2] + s_sum[par][sub][3]);
-    } else {
+    } else if constexpr (VAR != kQInt4Tensor) {
 #pragma unroll
       for (int c = 0; c < CHUNKS; ++c) {
         uint32_t k[8];
@@ -198,7 +322,11 @@ __global__ void __launch_bounds__(256) quant_a4_kernel(const uint16_t* __restric
     if constexpr (kInt) {
       // ---- INT4 codes RoundClip(x * mult, -8, 7) ----
       float mult;
-      if constexpr (VAR == kQInt4Absmax) {
+      if constexpr (VAR == kQInt4Tensor) {
+        const float beta = ld_dep_f32(beta_dev);   // the tensor's exact mean |x|
+        mult = __fdiv_rn(sqrt7_f32(), __fadd_rn(beta, eps));
+        if (t == 0) scale[row] = __fdiv_rn(beta, sqrt7_f32());
+      } else if constexpr (VAR == kQInt4Absmax) {
         const float gamma = __uint_as_float(mk << 16);   // max |x| (a bf16 value)
         mult = __fdiv_rn(7.f, __fadd_rn(gamma, eps));
         if (t == 0) scale[row] = __fdiv_rn(gamma, 7.f);

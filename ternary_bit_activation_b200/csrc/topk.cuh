@@ -595,7 +595,6 @@ template <int C>
 __global__ void __launch_bounds__(32 * kTwWarps) topk_warp_kernel(
     const uint16_t* __restrict__ x, int64_t M, int K, int64_t ldx, int keep, float eps,
     int8_t* __restrict__ codes, float* __restrict__ scale, uint32_t* __restrict__ mask) {
-  constexpr uint32_t kAbs = 0x7FFF7FFFu;
   constexpr uint32_t kPadNaN = 0x7FC07FC0u;
   // One row buffer per warp, filled by a 1-D bulk copy.  The code pass reads the
   // signed row from it in a rolled loop (an unrolled one overflows the

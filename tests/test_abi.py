@@ -121,6 +121,41 @@ def test_quant_validation(L):
     assert q(P(A16), 0, 64, 64, 0, 0, 1e-5, P(A16), P(A16), None) == 0
 
 
+def test_rmsnorm_quant_and_per_tensor_validation(L):
+    r = L.bitlinear_rmsnorm_quant_a4
+    ok = dict(x=A16, M=4, K=64, ldx=64, g=None, en=1e-6, q=0, st=0, eps=1e-5, c=A16, s=A16)
+
+    def call(**kw):
+        d = dict(ok, **kw)
+        return r(P(d["x"]), d["M"], d["K"], d["ldx"], P(d["g"]), d["en"], d["q"], d["st"], d["eps"], P(d["c"]),
+                 P(d["s"]), None)
+
+    assert call(en=0.0) == 4                 # eps_norm must be positive
+    assert call(en=float("inf")) == 4
+    assert call(K=100) == 3
+    assert call(K=16392, ldx=16392) == 3
+    assert call(q=9) == 4
+    assert call(g=MIS) == 2                  # the weight is read 16 bytes at a time
+    assert call(x=None) == 1
+    assert call(M=0) == 0
+    pt = L.bitlinear_quant_a4_per_tensor
+    okp = dict(x=A16, M=4, K=64, ldx=64, st=0, eps=1e-5, c=A16, s=A16, b=A16, ws=A16, wsb=2048)
+
+    def callp(**kw):
+        d = dict(okp, **kw)
+        return pt(P(d["x"]), d["M"], d["K"], d["ldx"], d["st"], d["eps"], P(d["c"]), P(d["s"]), P(d["b"]),
+                  P(d["ws"]), d["wsb"], None)
+
+    assert callp(wsb=1024) == 8
+    assert callp(ws=None) == 1
+    assert callp(b=None) == 1
+    assert callp(M=1 << 20, K=4096, ldx=4096) == 3      # M * K >= 2^31
+    assert callp(M=1 << 62, K=64) == 3                  # no overflowing product
+    assert callp(st=7) == 4
+    assert callp(M=0) == 0
+    assert tba.workspace_size("quant_a4_per_tensor") == 2048
+
+
 def test_topk_validation(L):
     s = L.bitlinear_sparsify_a8
     assert s(P(A16), 4, 64, 64, 0, 1e-5, P(A16), P(A16), None, None) == 4      # k_keep < 1
