@@ -954,6 +954,7 @@ PROFILE_CASES = {
     "gemm_upgate": "tcgen05 GEMM, int8 A [16384 x 4096] x ternary int8 W [22016 x 4096]",
     "gemm_down": "tcgen05 GEMM, int8 A [16384 x 11008] x ternary int8 W [4096 x 11008]",
     "quant_a4": "INT4 quantizer, X bf16 [32768 x 4096]",
+    "rmsnorm_quant_a4": "RMSNorm (with a weight) fused into the INT4 quantizer, X bf16 [32768 x 4096]",
     "sparsify_a8": "Top-K 50% + INT8, X bf16 [32768 x 4096]",
     "relu2_glu": "ReLU^2-GLU + Top-K 50% + INT8, gate/up bf16 [16384 x 11008]",
     "kv_quant3": "3-bit KV, K bf16 [32768 x 32 x 128]",
@@ -1008,6 +1009,12 @@ def run_profile_case(name: str, launches: int):
         c = torch.empty((32768, 4096), dtype=torch.uint8, device=dev)
         s = torch.empty((32768,), device=dev)
         fn = lambda: tba.bitlinear_quant_a4(x, c, s, tba.BL_QUANT_INT4, tba.BL_STORE_BYTES)
+    elif name == "rmsnorm_quant_a4":
+        x = bf16(32768, 4096)
+        c = torch.empty((32768, 4096), dtype=torch.uint8, device=dev)
+        s = torch.empty((32768,), device=dev)
+        gn = (1.0 + 0.3 * torch.randn((4096,), generator=g, device=dev)).float()
+        fn = lambda: tba.bitlinear_rmsnorm_quant_a4(x, c, s, gamma=gn, store=tba.BL_STORE_BYTES)
     elif name == "sparsify_a8":
         x = bf16(32768, 4096)
         c = torch.empty((32768, 4096), dtype=torch.int8, device=dev)

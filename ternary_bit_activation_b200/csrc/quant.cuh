@@ -161,6 +161,33 @@ __device__ __forceinline__ void dd_add_dd(double& hi, double& lo, double h2, dou
   lo = __dadd_rn(__dadd_rn(lo, l2), e);
 }
 
+// fp64 value of a bf16 magnitude key k (15 bits: exponent << 7 | mantissa),
+// built from its bits with one multiply-add (no conversion unit): exact for a
+// normal value (k >= 0x80); for a zero or subnormal key the result and the true
+// value are both below 2^-126, an absolute error the certificates below count.
+__device__ __forceinline__ double key_to_f64(uint32_t k) {
+  return __hiloint2double(static_cast<int>(k * 8192u + 0x38000000u), 0);
+}
+
+// Certified rounding: c = RN_fp32(q), and true when every value within err of
+// q rounds to the same fp32 (so c is the rounding of any quotient known to lie
+// within err of q; the quotients here are non-negative).
+__device__ __forceinline__ bool certify_f32(double q, double err, float& c) {
+  c = __double2float_rn(q);
+  const double up = 0.5 * (static_cast<double>(c) + static_cast<double>(nextafterf(c, __int_as_float(0x7F800000))));
+  if (!(__dadd_rn(q, err) < up)) return false;
+  if (c > 0.f) {
+    const double dn = 0.5 * (static_cast<double>(c) + static_cast<double>(nextafterf(c, 0.f)));
+    if (!(__dsub_rn(q, err) > dn)) return false;
+  }
+  return true;
+}
+
+// Relative error bound of an fp64 sum of n positive terms (at most n + 10
+// roundings along any path of the partial-sums-then-warp-then-CTA reduction),
+// with a factor of two to spare: 2 (n + 32) 2^-53.
+__device__ __forceinline__ double sum_rel_bound(int n) { return static_cast<double>(2 * n + 64) * 0x1p-53; }
+
 // RN_fp32((hi + lo) / K) for an exact sum hi + lo >= 0: the fp32 nearest to
 // hi / K, then moved while the exact quotient lies beyond a midpoint to a
 // neighbour (at a midpoint: the even one).  A midpoint m has at most 25
@@ -237,31 +264,61 @@ __global__ void __launch_bounds__(256) quant_a4_kernel(const uint16_t* __restric
     constexpr bool kInt = VAR == kQInt4 || VAR == kQInt4Absmean2 || VAR == kQInt4Absmax || VAR == kQInt4Tensor;
 
     if constexpr (NORM) {
-      // ---- RMSNorm: the exact sum of squares, ms, r, and y in place of x ----
-      double hi = 0.0, lo = 0.0;
+      // ---- RMSNorm: ms = RN_fp32(exact mean of x^2), r, and y in place of x ----
+      // Fast path: a plain fp64 sum of the squares (each exact; one rounding per
+      // addition, at most K + 8 of them in any order), so the sum is within
+      // (K + 8) * 2^-53 of the exact one, relatively.  If every quotient in that
+      // interval (and the division's own rounding) rounds to the same fp32, that
+      // fp32 is ms; otherwise -- a quotient within about K * 2^-53 of an fp32
+      // midpoint, one row in ~2^15 -- the row's sum is recomputed exactly as a
+      // double-double.  The decision is the same for every thread of the row.
+      double sp[4] = {0.0, 0.0, 0.0, 0.0};   // independent partial sums: short dependency chains
 #pragma unroll
       for (int c = 0; c < CHUNKS; ++c) {
-        float f[8];
-        unpack_bf16x8(v[c], f);   // chunks past K hold zeros
+        uint32_t k[8];
+        bf16x8_mag_keys(v[c], k);   // chunks past K hold zeros
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const double d = static_cast<double>(f[e]);
-          dd_add(hi, lo, __dmul_rn(d, d));
+          const double d = key_to_f64(k[e]);
+          sp[e & 3] = __fma_rn(d, d, sp[e & 3]);
         }
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1)
-        dd_add_dd(hi, lo, __shfl_xor_sync(0xFFFFFFFFu, hi, o), __shfl_xor_sync(0xFFFFFFFFu, lo, o));
-      if (lane == 0) {
-        s_dd[par][sub][warp][0] = hi;
-        s_dd[par][sub][warp][1] = lo;
-      }
+      double sa = warp_sum_f64((sp[0] + sp[1]) + (sp[2] + sp[3]));
+      if (lane == 0) s_dd[par][sub][warp][0] = sa;
       q4_row_sync(sub);
-      hi = s_dd[par][sub][0][0];
-      lo = s_dd[par][sub][0][1];
+      sa = (s_dd[par][sub][0][0] + s_dd[par][sub][1][0]) + (s_dd[par][sub][2][0] + s_dd[par][sub][3][0]);
+      const double q = __ddiv_rn(sa, static_cast<double>(K));
+      // zero and subnormal keys: each square off by less than 2^-252
+      float ms;
+      const bool certain = certify_f32(q, __dadd_rn(__dmul_rn(q, sum_rel_bound(K)), 0x1p-252), ms);
+      if (!certain) {
+        double hi = 0.0, lo = 0.0;
 #pragma unroll
-      for (int w = 1; w < 4; ++w) dd_add_dd(hi, lo, s_dd[par][sub][w][0], s_dd[par][sub][w][1]);
-      const float ms = dd_mean_f32(hi, lo, K);
+        for (int c = 0; c < CHUNKS; ++c) {
+          float f[8];
+          unpack_bf16x8(v[c], f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const double d = static_cast<double>(f[e]);
+            dd_add(hi, lo, __dmul_rn(d, d));
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+          dd_add_dd(hi, lo, __shfl_xor_sync(0xFFFFFFFFu, hi, o), __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+        // the fast-path words of this row slot were read by every thread before the barrier below
+        q4_row_sync(sub);
+        if (lane == 0) {
+          s_dd[par][sub][warp][0] = hi;
+          s_dd[par][sub][warp][1] = lo;
+        }
+        q4_row_sync(sub);
+        hi = s_dd[par][sub][0][0];
+        lo = s_dd[par][sub][0][1];
+#pragma unroll
+        for (int w = 1; w < 4; ++w) dd_add_dd(hi, lo, s_dd[par][sub][w][0], s_dd[par][sub][w][1]);
+        ms = dd_mean_f32(hi, lo, K);
+      }
       const float r = __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(ms, eps_n)));
 #pragma unroll
       for (int c = 0; c < CHUNKS; ++c) {
@@ -277,22 +334,68 @@ __global__ void __launch_bounds__(256) quant_a4_kernel(const uint16_t* __restric
           g[3] = __uint_as_float(g0.w); g[4] = __uint_as_float(g1.x); g[5] = __uint_as_float(g1.y);
           g[6] = __uint_as_float(g1.z); g[7] = __uint_as_float(g1.w);
         }
-        uint32_t hb[8];
+        float tv[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          float tv = __fmul_rn(f[e], r);
-          if (gnorm != nullptr) tv = __fmul_rn(tv, g[e]);
-          const __nv_bfloat16 b = __float2bfloat16_rn(tv);
-          hb[e] = *reinterpret_cast<const uint16_t*>(&b);
+          tv[e] = __fmul_rn(f[e], r);
+          if (gnorm != nullptr) tv[e] = __fmul_rn(tv[e], g[e]);
         }
-        v[c] = make_uint4(hb[0] | (hb[1] << 16), hb[2] | (hb[3] << 16), hb[4] | (hb[5] << 16), hb[6] | (hb[7] << 16));
+        // paired conversions (round to nearest even; no conversion-unit instruction)
+        uint32_t hb[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 b = __floats2bfloat162_rn(tv[2 * e], tv[2 * e + 1]);
+          hb[e] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+        v[c] = make_uint4(hb[0], hb[1], hb[2], hb[3]);
       }
     }
 
     // ---- the row statistic ----
     double S = 0.0;       // sum |x| (exact in fp64 for in-contract rows: order-free)
     uint32_t mk = 0;      // max |x| as the largest 15-bit bf16 magnitude
-    if constexpr (kSum) {
+    float beta_c = 0.f;   // beta, when the certified fast path settles it (RMSNorm rows)
+    bool beta_ok = false;
+    if constexpr (kSum && NORM) {
+      // beta = RN_fp32(RN_fp64(S / K)) with S the exact sum of |y| (exact in fp64
+      // for in-contract rows).  Fast path: doubles built from the bits, four
+      // partial sums, and a certificate; the exact sum only for rows the
+      // certificate cannot settle.  (Measured: faster here, where the norm
+      // already keeps the conversion unit busy; slower than the exact sum alone
+      // in the plain quantizer, which keeps that.)
+      double ap[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+      for (int c = 0; c < CHUNKS; ++c) {
+        uint32_t k[8];
+        bf16x8_mag_keys(v[c], k);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ap[e & 3] = __dadd_rn(ap[e & 3], key_to_f64(k[e]));
+      }
+      double acc = warp_sum_f64((ap[0] + ap[1]) + (ap[2] + ap[3]));
+      if (lane == 0) s_sum[par][sub][warp] = acc;
+      q4_row_sync(sub);
+      const double sa = (s_sum[par][sub][0] + s_sum[par][sub][1]) + (s_sum[par][sub][2] + s_sum[par][sub][3]);
+      const double two = VAR == kQInt4Absmean2 ? 2.0 : 1.0;   // exact doubling
+      const double q = __ddiv_rn(two * sa, static_cast<double>(K));
+      // + the fp64 division's own rounding (2^-53 relative, inside the bound) and
+      // zero / subnormal keys (each off by less than 2^-126)
+      beta_ok = certify_f32(q, __dadd_rn(__dmul_rn(q, sum_rel_bound(K)), two * 0x1p-126), beta_c);
+      if (!beta_ok) {
+        double ex = 0.0;
+#pragma unroll
+        for (int c = 0; c < CHUNKS; ++c) {
+          float f[8];
+          unpack_bf16x8(v[c], f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ex += static_cast<double>(fabsf(f[e]));
+        }
+        ex = warp_sum_f64(ex);
+        q4_row_sync(sub);   // every thread has read the fast-path words
+        if (lane == 0) s_sum[par][sub][warp] = ex;
+        q4_row_sync(sub);
+        S = (s_sum[par][sub][0] + s_sum[par][sub][1]) + (s_sum[par][sub][2] + s_sum[par][sub][3]);
+      }
+    } else if constexpr (kSum) {
       double acc = 0.0;
 #pragma unroll
       for (int c = 0; c < CHUNKS; ++c) {
@@ -332,7 +435,8 @@ __global__ void __launch_bounds__(256) quant_a4_kernel(const uint16_t* __restric
         if (t == 0) scale[row] = __fdiv_rn(gamma, 7.f);
       } else {
         // beta = mean|x| (INT4) or 2 mean|x| (the doubling is exact)
-        const float beta = __double2float_rn((VAR == kQInt4Absmean2 ? 2.0 * S : S) / static_cast<double>(K));
+        const float beta =
+            beta_ok ? beta_c : __double2float_rn((VAR == kQInt4Absmean2 ? 2.0 * S : S) / static_cast<double>(K));
         mult = __fdiv_rn(sqrt7_f32(), __fadd_rn(beta, eps));
         if (t == 0) scale[row] = __fdiv_rn(beta, sqrt7_f32());
       }
