@@ -502,7 +502,8 @@ int orc_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D, int64_t ld
  * Each x^2 is exact in fp64; the pair is a double-double accumulation whose
  * every step is checked to be exact (TwoSum), and the row is rejected unless
  * the squares, as multiples of the smallest one's last significant bit, stay
- * below 2^106 in sum -- then every order of accumulation is exact as well.
+ * below 2^90 in sum -- then a double-double accumulation in any order (and any
+ * grouping, up to 16384 terms) is exact as well.
  * orc_rmsnorm_apply takes ms and forms y and r.
  * ------------------------------------------------------------------------- */
 static void two_sum(double a, double b, double* s, double* e) {
@@ -539,7 +540,7 @@ int orc_rmsnorm_sumsq(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, doub
         if (hi != 0.0) {
             int e;
             frexp(hi + lo, &e);            /* the sum is below 2^e (within a rounding) */
-            if (e + 1 - lowbit > 106) return ORC_ERR_INEXACT_SUM;
+            if (e - lowbit > 90) return ORC_ERR_INEXACT_SUM;
         }
         hi_out[m] = hi;
         lo_out[m] = lo;
