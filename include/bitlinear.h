@@ -266,10 +266,12 @@ BL_API bl_status bitlinear_gemm(const void* a, bl_afmt afmt, const float* a_scal
  * The codes, the scale and acc_out are exactly those of bitlinear_quant_a4
  * followed by bitlinear_gemm (for FP4, acc_out holds 2 * the sum, as for
  * BL_A_E2M1 activations).
- * With BL_W_T2 weights and a shape the decode GEMV takes (M <= 8; see
+ * With BL_W_T2 weights and 1 or 2 tokens (a shape the decode GEMV takes; see
  * bitlinear_gemm) the quantization runs in the GEMV's prologue: every CTA reads
  * the M bf16 rows, reduces each token's statistic and quantizes into shared
- * memory, so no codes reach global memory and there is one launch.  Otherwise
+ * memory, so no codes reach global memory and there is one launch (measured
+ * faster there; from 3 tokens the repeated quantization in every CTA costs more
+ * than the separate launch, so those run as two kernels).  Otherwise
  * it runs as bitlinear_quant_a4 (BL_STORE_BYTES) into `workspace` and then
  * bitlinear_gemm with BL_A_I8 codes; `workspace` then needs
  * bitlinear_workspace_size("quant_gemm", M, N, K) bytes (16-byte aligned) and

@@ -564,6 +564,13 @@ bl_status launch_gemv_any(const uint8_t* A, const float* a_scale, const uint8_t*
   return launch_gemv<AF>(A, a_scale, W, alpha, alpha_group, m, n, k, Y, ldy, acc_out, s, ldx, eps);
 }
 
+// bitlinear_quant_gemm quantizes inside the decode GEMV for at most this many
+// tokens.  Measured on 7B decode shapes: the fused layer is ~1 us faster at 1-2
+// tokens, but 15-21 us slower at 4-8 (every CTA repeats the quantization, while
+// the separate quantizer already overlaps the GEMV's weight prefetch), so from 3
+// tokens the call runs the quantizer and the GEMM separately.
+constexpr int64_t kQgFusedMaxTokens = 2;
+
 // Workspace of bitlinear_quant_gemm when it runs as two kernels: M x K int8
 // codes, then M fp32 scales, each 16-byte aligned.
 int64_t qg_codes_bytes(int64_t M, int64_t K) { return (M * K + 15) / 16 * 16; }
@@ -990,8 +997,8 @@ bl_status bitlinear_quant_gemm(const void* x_bf16, int64_t ldx, bl_quant quant, 
     return BL_ERR_ALIGN;
   cudaStream_t s = as_stream(stream);
   const bool fp4 = quant == BL_QUANT_FP4_E2M1;
-  if (wfmt == BL_W_T2 && gemv_applies(M, K, kGvMaxTokens)) {
-    // decode: each GEMV CTA quantizes the token rows itself
+  if (wfmt == BL_W_T2 && M <= kQgFusedMaxTokens && gemv_applies(M, K, kGvMaxTokens)) {
+    // decode of 1-2 tokens: each GEMV CTA quantizes the token rows itself
     const uint8_t* X = static_cast<const uint8_t*>(x_bf16);
     const uint8_t* W = static_cast<const uint8_t*>(w);
     uint16_t* Y = static_cast<uint16_t*>(y_bf16);

@@ -420,7 +420,7 @@ def test_gemm_t2_long_k_cuda_core():
     assert tba.STATUS_NAMES[e.value.status] == "BL_ERR_SHAPE"
 
 
-# bitlinear_quant_gemm: the INT4 / FP4 quantizer fused into the GEMM.  Up to 8
+# bitlinear_quant_gemm: the INT4 / FP4 quantizer fused into the GEMM.  For 1-2
 # tokens against 2-bit weights it runs in the decode GEMV's prologue (every CTA
 # quantizes the token rows itself); otherwise as quantizer + GEMM through the
 # workspace.  Either way the result must be the oracle's quantizer followed by
@@ -481,10 +481,14 @@ def test_quant_gemm_needs_workspace_beyond_the_gemv():
     with pytest.raises(tba.BitLinearError) as e:
         tba.bitlinear_quant_gemm(x, w, al, M, N, K, y=y)
     assert tba.STATUS_NAMES[e.value.status] == "BL_ERR_NULL"
-    # the decode GEMV needs none
-    tba.bitlinear_quant_gemm(x[:4], w, al, 4, N, K, y=y[:4])
+    # from 3 tokens the quantizer runs separately, through the workspace
+    with pytest.raises(tba.BitLinearError) as e:
+        tba.bitlinear_quant_gemm(x[:3], w, al, 3, N, K, y=y[:3])
+    assert tba.STATUS_NAMES[e.value.status] == "BL_ERR_NULL"
+    # the decode GEMV with the quantizer in its prologue (1-2 tokens) needs none
+    tba.bitlinear_quant_gemm(x[:2], w, al, 2, N, K, y=y[:2])
     tba.sync_status()
-    assert np.array_equal(host(y[:4], np.uint16), np.zeros((4, N), np.uint16))
+    assert np.array_equal(host(y[:2], np.uint16), np.zeros((2, N), np.uint16))
 
 
 # the conditional Up projection: Gate rows first, Up rows only where some

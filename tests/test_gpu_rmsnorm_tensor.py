@@ -34,6 +34,14 @@ def rows(name):
         x[1] = synth.f32_to_bf16_bits(np.full(4096, 2.0 ** -60, np.float32))          # tiny constant row
         x[2, ::2] = 0
         return x
+    if name == "midpoint_rows":
+        # mean(x^2) exactly on an fp32 midpoint (6 + 2^-22 over 8 = 0.75 + 2^-25: ties to
+        # 0.75), just above it (+ 2^-60: rounds up), and the same with zeros past the
+        # squares: the fast sum cannot settle these, the exact path must
+        f = lambda v: synth.f32_to_bf16_bits(np.array([v], np.float32))
+        r = [f([1, 1, 1, 1, 1, 1, 2.0 ** -11, 0]), f([1, 1, 1, 1, 1, 1, 2.0 ** -11, 2.0 ** -30]),
+             f([-1, 1, -1, 1, -1, 1, -2.0 ** -11, 0]), f([0.5, 0.5, 0.5, 0.5, 0.5, 0.5, 2.0 ** -12, 0])]
+        return np.concatenate(r)
     if name == "zeros_consts":
         return np.concatenate([np.zeros((2, 256), np.uint16),
                                synth.f32_to_bf16_bits(np.full((2, 256), -0.75, np.float32)),
@@ -41,7 +49,8 @@ def rows(name):
     raise KeyError(name)
 
 
-ROWS = ["gauss_M37_K1536", "studentt_K3200", "K8_min", "K16384_max", "wide_in_contract", "zeros_consts"]
+ROWS = ["gauss_M37_K1536", "studentt_K3200", "K8_min", "K16384_max", "wide_in_contract", "midpoint_rows",
+        "zeros_consts"]
 
 
 def gamma_for(K, kind):
@@ -186,3 +195,14 @@ def test_new_quantizers_in_bounds(store, M, K):
     for t, buf in (codes, scale, beta):
         assert canary_margins_intact(t, buf) and np.any(canary_bytes(t) != CANARY)
     assert canary_margins_intact(*ws)
+
+
+def test_rmsnorm_midpoint_rows_take_the_exact_mean():
+    # the oracle's r for these rows follows ms = 0.75 (the tie to even) and 0.75 + 2^-24
+    y, r = oracle.rmsnorm(rows("midpoint_rows"), None, EPS_N)
+    s0 = np.sqrt(np.float32(0.75) + np.float32(EPS_N), dtype=np.float32)
+    s1 = np.sqrt(np.float32(0.75 + 2.0 ** -24) + np.float32(EPS_N), dtype=np.float32)
+    assert float(r[0]) == float(np.float32(1) / s0) and float(r[1]) == float(np.float32(1) / s1)
+    codes, scale = run_rmsnorm_quant(rows("midpoint_rows"), None, tba.BL_QUANT_INT4, tba.BL_STORE_BYTES)
+    c_ref, s_ref = expected(rows("midpoint_rows"), None, tba.BL_QUANT_INT4, tba.BL_STORE_BYTES)
+    assert np.array_equal(codes, c_ref) and np.array_equal(scale.view(np.uint32), s_ref.view(np.uint32))
