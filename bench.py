@@ -516,6 +516,10 @@ def run_gpu(args):
             },
             "gemm": {"tops_dense": round(tops, 1), "tops_algorithmic": round(alg_tops, 1),
                      "ms_per_step": round(gemm_ms / args.steps, 4)},
+            # the same step with the ternary weights packed once beforehand (as at
+            # inference): the step's time less its pack_ternary launches
+            "value_weights_packed_once": round(weak_scaling_throughput(
+                world, m, args.steps, elapsed_ms - sum(per_kernel.get("pack_ternary", []))), 1),
             "kernels": kernels,
             "e2e": {"value": round(world * m * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

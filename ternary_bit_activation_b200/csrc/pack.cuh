@@ -124,7 +124,13 @@ __global__ void __launch_bounds__(kBinThreads, 6) ternary_bins_kernel(const void
       for (int i = 0; i < kPer * kLoads; ++i) {
         const uint32_t a = u[i];
         if (a - lo_bits < (kWin << 23)) {
-          acc += static_cast<double>(__uint_as_float(a));   // exact; 0 before the anchor
+          // exact: inside the window a is a normal fp32 (biased exponent >= 1), so
+          // its fp64 is built from the bits -- exponent rebiased by 1023 - 127,
+          // significand shifted up by 29 -- with integer operations instead of
+          // the conversion unit; before the anchor a is 0 and so is the double
+          acc += a != 0u ? __hiloint2double(static_cast<int>((a >> 3) + ((1023u - 127u) << 20)),
+                                            static_cast<int>(a << 29))
+                         : 0.0;
         } else if (a != 0) {
           const uint32_t E = a >> 23;
           const uint32_t m = (a & 0x7FFFFFu) | (E ? 0x800000u : 0u);
