@@ -375,6 +375,17 @@ def zero_fractions(torch, layer) -> dict:
         return round(float(is_zero.sum().item()) / is_zero.numel(), 4)
     out = {"o_input": frac(layer.o8 == 0), "down_input": frac(layer.h8 == 0),
            "gate_relu_zero": frac(layer.y_ug[:, layer.f:].view(torch.bfloat16) <= 0)}
+    # what a sparse Down GEMM could skip: K columns that are zero in every row of a
+    # 128-row tile (the tensor-core GEMM's M tile), and groups of four codes with
+    # more than two nonzeros (which break the 2:4 pattern of a structured-sparse MMA)
+    nz = layer.h8 != 0
+    rows = (nz.shape[0] // 128) * 128
+    if rows:
+        tile_any = nz[:rows].view(rows // 128, 128, nz.shape[1]).any(dim=1)
+        out["down_all_zero_k_columns_per_128_rows"] = frac(~tile_any)
+    if nz.shape[1] % 4 == 0:
+        out["down_groups_over_2of4"] = frac(nz.view(nz.shape[0], -1, 4).sum(dim=-1) > 2)
+    del nz
     if layer.afmt == "int4":   # byte layout: one code per byte
         out["qkv_input"] = frac(layer.qa == 0)
         out["upgate_input"] = frac(layer.qf == 0)

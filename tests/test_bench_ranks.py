@@ -60,6 +60,18 @@ def test_zero_fractions_of_a_step():
     layer = SimpleNamespace(o8=o8, h8=h8, y_ug=y_ug, f=f, qa=qa, qf=qf, afmt="int4")
     z = bench.zero_fractions(torch, layer)
     assert z == {"o_input": 0.5, "down_input": round(31 / 32, 4), "gate_relu_zero": 0.75,
-                 "qkv_input": 1.0, "upgate_input": 0.0}
+                 "qkv_input": 1.0, "upgate_input": 0.0, "down_groups_over_2of4": 0.0}
     layer.afmt = "fp4"
-    assert set(bench.zero_fractions(torch, layer)) == {"o_input", "down_input", "gate_relu_zero"}
+    assert set(bench.zero_fractions(torch, layer)) == {"o_input", "down_input", "gate_relu_zero",
+                                                        "down_groups_over_2of4"}
+    # two 128-row tiles of 8 columns: tile 0 has nonzeros in columns 0, 1, 3 (row 5)
+    # and 6 (row 77), tile 1 in column 2 only (row 200), so 4 + 7 = 11 of the 16
+    # (tile, column) pairs are all zero; row 5's first group of four holds three
+    # nonzeros (1 of the 512 groups breaks 2:4)
+    layer.h8 = torch.zeros((256, 8), dtype=torch.int8)
+    layer.h8[5, 0], layer.h8[5, 1], layer.h8[5, 3] = -3, 1, 1
+    layer.h8[77, 6] = 9
+    layer.h8[200, 2] = 4
+    z = bench.zero_fractions(torch, layer)
+    assert z["down_all_zero_k_columns_per_128_rows"] == round(11 / 16, 4)
+    assert z["down_groups_over_2of4"] == round(1 / 512, 4)
