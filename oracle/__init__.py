@@ -12,7 +12,8 @@ written from the layout statements of the public C header.
 Equations follow arXiv 2411.04965 ("BitNet a4.8: 4-bit Activations for 1-bit
 LLMs"), §3.4: Eq. 2 (ternary weights), Eq. 6-7 (INT4 absmean), Eq. 8-9 (FP4
 MinMax), Eq. 1 with Q_INT8 (Top-K + INT8 absmax), Eq. 5 (ReLU^2-GLU) and the
-"Low-Bit KV Cache Quantization" paragraph.
+"Low-Bit KV Cache Quantization" paragraph (the KV quantizer, and the attention
+of 4-bit queries over the quantized cache).
 
 Every function here is pinned by ``tests/test_oracle_pins.py``.
 """
@@ -357,6 +358,61 @@ def kv_quant(kv_bf16: np.ndarray, bits: int = 3, bos_pos: int = 0, eps: float = 
     _check(_load().orc_kv_quant(_ptr(kv), T, H, D, H * D, bits, bos_pos, eps, _ptr(codes),
                                 _ptr(scale)), "kv_quant")
     return codes, scale
+
+
+# ---------------------------------------------------------------------------
+# Low-bit attention over the quantized cache
+# ---------------------------------------------------------------------------
+def attention_lowbit(q_codes_u: np.ndarray, q_scale: np.ndarray, k_codes_u: np.ndarray, k_scale: np.ndarray,
+                     v_codes_u: np.ndarray, v_scale: np.ndarray, kv_bits: int = 3, bos_pos: int = -1,
+                     softmax_scale=None, heads=None) -> np.ndarray:
+    """Attention of 4-bit queries over a 3- or 4-bit key/value cache, in fp64
+    (§3.4 "Low-Bit KV Cache Quantization": post-RoPE Q, K and V quantized by
+    absmax to unsigned integers; Table 3's "4-bit Q, 3-bit KV" and "4-bit QKV"
+    rows).  The pages give the quantizer, not the attention; the reading used is
+    softmax attention over the dequantized codes:
+
+      q_hat = (q_code - 8) * q_scale                      (4-bit Q)
+      k_hat_t = (k_code_t - 2^(b-1)) * k_scale_t          (b = kv_bits; the BOS
+      v_hat_t = (v_code_t - 2^(b-1)) * v_scale_t           position of a 3-bit
+                                                           cache is 4-bit: offset 8)
+      s_t = softmax_scale * <q_hat, k_hat_t>,  p = softmax(s) over the allowed t,
+      o = sum_t p_t * v_hat_t.
+
+    The M queries are the cache's last M positions: query m sits at position
+    T - M + m and attends positions 0 .. T - M + m (causal).
+    q_codes_u: [M, H, D] unsigned 4-bit codes; q_scale: [M, H].  k_codes_u,
+    v_codes_u: [T, H, D] unsigned codes as ``kv_quant`` returns them; k_scale,
+    v_scale: [T, H].  softmax_scale: fp32 value (default fp32(1/sqrt(D))).
+    heads: optional list of heads to compute (others are left NaN).
+    Returns o: fp64 [M, H, D]."""
+    q = np.asarray(q_codes_u)
+    k = np.asarray(k_codes_u)
+    v = np.asarray(v_codes_u)
+    M, H, D = q.shape
+    T = k.shape[0]
+    if k.shape != (T, H, D) or v.shape != (T, H, D) or kv_bits not in (3, 4) or not 1 <= M <= T:
+        raise ValueError("attention_lowbit: bad shapes or kv_bits")
+    if softmax_scale is None:
+        softmax_scale = np.float32(1.0 / np.sqrt(D))
+    sm = float(np.float32(softmax_scale))
+    offset = np.full(T, float(1 << (kv_bits - 1)))
+    if kv_bits == 3 and 0 <= bos_pos < T:
+        offset[bos_pos] = 8.0
+    qs = np.asarray(q_scale, np.float32).astype(np.float64)
+    ks = np.asarray(k_scale, np.float32).astype(np.float64)
+    vs = np.asarray(v_scale, np.float32).astype(np.float64)
+    out = np.full((M, H, D), np.nan)
+    for h in (range(H) if heads is None else heads):
+        k_hat = (k[:, h, :].astype(np.float64) - offset[:, None]) * ks[:, h, None]
+        v_hat = (v[:, h, :].astype(np.float64) - offset[:, None]) * vs[:, h, None]
+        for m in range(M):
+            last = T - M + m
+            q_hat = (q[m, h, :].astype(np.float64) - 8.0) * qs[m, h]
+            s = sm * (k_hat[:last + 1] @ q_hat)
+            e = np.exp(s - s.max())
+            out[m, h] = (e @ v_hat[:last + 1]) / e.sum()
+    return out
 
 
 # ---------------------------------------------------------------------------

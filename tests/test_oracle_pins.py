@@ -609,3 +609,136 @@ def test_rmsnorm_mean_is_exact_and_rejects_wide_rows():
     wide[0, :2] = bf16([1e30, 1e-30])
     with pytest.raises(ValueError):
         oracle.rmsnorm(wide)
+
+
+# ---------------------------------------------------------------------------
+# Low-bit attention over the quantized cache (§3.4 "Low-Bit KV Cache Quantization")
+# ---------------------------------------------------------------------------
+def _attention_case(g, c):
+    M, T, bits, bos = (int(v) for v in g[c + "_meta"][0])
+    D = len(g[c + "_q"][0])
+    q = np.array(g[c + "_q"], np.uint8).reshape(M, 1, D)
+    k = np.array(g[c + "_k"], np.uint8).reshape(T, 1, D)
+    v = np.array(g[c + "_v"], np.uint8).reshape(T, 1, D)
+    qs = np.array(g[c + "_qs"][0], np.float32).reshape(M, 1)
+    ks = np.array(g[c + "_ks"][0], np.float32).reshape(T, 1)
+    vs = np.array(g[c + "_vs"][0], np.float32).reshape(T, 1)
+    o = oracle.attention_lowbit(q, qs, k, ks, v, vs, kv_bits=bits, bos_pos=bos,
+                                softmax_scale=np.float32(g[c + "_sm"][0][0]))
+    return o[:, 0, :], np.array(g[c + "_o"])
+
+
+def test_attention_hand_examples():
+    g = read_golden("attention_hand.txt")
+    for c in ("c1", "c2", "c3"):
+        o, want = _attention_case(g, c)
+        np.testing.assert_allclose(o, want, rtol=0, atol=1e-6, err_msg=c)
+
+
+def _random_cache(g, T, H, D, bits):
+    k = g.integers(0, 1 << bits, (T, H, D)).astype(np.uint8)
+    v = g.integers(0, 1 << bits, (T, H, D)).astype(np.uint8)
+    ks = g.uniform(0.05, 2.0, (T, H)).astype(np.float32)
+    vs = g.uniform(0.05, 2.0, (T, H)).astype(np.float32)
+    return k, ks, v, vs
+
+
+def _dequant(codes, scale, offset):
+    return (codes.astype(np.float64) - offset) * scale.astype(np.float64)[..., None]
+
+
+def test_attention_single_position_is_v():
+    # softmax over one position is 1: the output is that position's dequantized V exactly
+    g = synth.rng(70)
+    for bits in (3, 4):
+        k, ks, v, vs = _random_cache(g, 1, 3, 16, bits)
+        q = g.integers(0, 16, (1, 3, 16)).astype(np.uint8)
+        qs = g.uniform(0.1, 1.0, (1, 3)).astype(np.float32)
+        o = oracle.attention_lowbit(q, qs, k, ks, v, vs, kv_bits=bits, bos_pos=-1)
+        assert np.array_equal(o[0], _dequant(v[0], vs[0], 1 << (bits - 1)))
+
+
+def test_attention_zero_query_is_the_mean_of_allowed_values():
+    # q_hat = 0 makes every score 0: uniform weights over the positions the query sees
+    g = synth.rng(71)
+    T, H, D, M = 9, 2, 16, 3
+    k, ks, v, vs = _random_cache(g, T, H, D, 3)
+    q = np.full((M, H, D), 8, np.uint8)
+    qs = np.ones((M, H), np.float32)
+    o = oracle.attention_lowbit(q, qs, k, ks, v, vs, kv_bits=3, bos_pos=2)
+    vh = _dequant(v, vs, 4.0)
+    vh[2] = _dequant(v[2], vs[2], 8.0)          # the BOS position is 4-bit
+    for m in range(M):
+        np.testing.assert_allclose(o[m], vh[:T - M + m + 1].mean(axis=0), rtol=1e-12, atol=1e-12)
+
+
+def test_attention_dominant_score_selects_its_value():
+    # one score above all others by far more than 745 (fp64 exp underflows to 0):
+    # the output is exactly that position's value; also checks that no overflow occurs
+    g = synth.rng(72)
+    T, H, D = 6, 1, 8
+    k = np.full((T, H, D), 4, np.uint8)
+    k[4, 0, 0] = 7                               # k_hat_4 = 3 e_0 * scale, the others 0
+    ks = np.full((T, H), 1000.0, np.float32)
+    v = g.integers(0, 8, (T, H, D)).astype(np.uint8)
+    vs = g.uniform(0.1, 2.0, (T, H)).astype(np.float32)
+    q = np.full((1, H, D), 8, np.uint8)
+    q[0, 0, 0] = 15                              # q_hat = 7 e_0
+    o = oracle.attention_lowbit(q, np.ones((1, H), np.float32), k, ks, v, vs, kv_bits=3, bos_pos=-1,
+                                softmax_scale=np.float32(1.0))
+    assert np.array_equal(o[0, 0], _dequant(v[4, 0], vs[4, 0], 4.0))
+
+
+def test_attention_causal_mask_and_last_query():
+    # query m sees positions 0..T-M+m: values at later positions do not move it, and
+    # the last of M queries equals a single query over the whole cache
+    g = synth.rng(73)
+    T, H, D, M = 12, 2, 16, 4
+    k, ks, v, vs = _random_cache(g, T, H, D, 3)
+    q = g.integers(0, 16, (M, H, D)).astype(np.uint8)
+    qs = g.uniform(0.1, 1.0, (M, H)).astype(np.float32)
+    o = oracle.attention_lowbit(q, qs, k, ks, v, vs, kv_bits=3, bos_pos=0)
+    k2, v2 = k.copy(), v.copy()
+    k2[T - M + 1:] = 7 - k2[T - M + 1:]
+    v2[T - M + 1:] = 7 - v2[T - M + 1:]
+    o2 = oracle.attention_lowbit(q, qs, k2, ks, v2, vs, kv_bits=3, bos_pos=0)
+    assert np.array_equal(o[0], o2[0]) and not np.array_equal(o[M - 1], o2[M - 1])
+    o1 = oracle.attention_lowbit(q[M - 1:], qs[M - 1:], k, ks, v, vs, kv_bits=3, bos_pos=0)
+    assert np.array_equal(o1[0], o[M - 1])
+
+
+def test_attention_is_a_convex_combination_and_order_free():
+    # every output lies between the smallest and largest allowed value per channel,
+    # and permuting the cache positions (one query sees all of them) changes nothing
+    g = synth.rng(74)
+    T, H, D = 40, 3, 32
+    k, ks, v, vs = _random_cache(g, T, H, D, 4)
+    q = g.integers(0, 16, (1, H, D)).astype(np.uint8)
+    qs = g.uniform(0.1, 1.0, (1, H)).astype(np.float32)
+    o = oracle.attention_lowbit(q, qs, k, ks, v, vs, kv_bits=4)
+    vh = _dequant(v, vs, 8.0)
+    assert np.all(o[0] >= vh.min(axis=0) - 1e-12) and np.all(o[0] <= vh.max(axis=0) + 1e-12)
+    perm = g.permutation(T)
+    op = oracle.attention_lowbit(q, qs, k[perm], ks[perm], v[perm], vs[perm], kv_bits=4)
+    np.testing.assert_allclose(op, o, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_of_quantized_cache_approaches_full_precision():
+    # with the cache quantized by the pinned kv_quant at 4 bits and a 4-bit query, the
+    # output stays within the quantization error of full-precision attention on the
+    # bf16 inputs (each dequantized value is off by at most half a step, gamma/(2*7))
+    g = synth.rng(75)
+    T, H, D = 64, 2, 32
+    x = synth.gaussian_bf16(g, (3 * T, H, D))
+    kc, ksc = oracle.kv_quant(x[:T], bits=4, bos_pos=-1)
+    vc, vsc = oracle.kv_quant(x[T:2 * T], bits=4, bos_pos=-1)
+    qc, qsc = oracle.kv_quant(x[2 * T:2 * T + 1], bits=4, bos_pos=-1)
+    o = oracle.attention_lowbit(qc, qsc, kc, ksc, vc, vsc, kv_bits=4)
+    xf = bf16_val(x).astype(np.float64)
+    K, V, Q = xf[:T], xf[T:2 * T], xf[2 * T]
+    for h in range(H):
+        s = (K[:, h, :] @ Q[h]) / np.sqrt(D)
+        p = np.exp(s - s.max())
+        ref = (p @ V[:, h, :]) / p.sum()
+        assert np.max(np.abs(o[0, h] - ref)) < 0.35    # loose: 4-bit Q and K move the weights too
+        assert np.corrcoef(o[0, h], ref)[0, 1] > 0.9
