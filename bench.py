@@ -562,6 +562,7 @@ def run_gpu(args):
                                        "[22016 x 4096]^T, packed E2M1 activations x E2M1-coded ternary weights, "
                                        "tcgen05 kind::mxf4; median of 10 launches",
                            **f4}
+            line["attention"] = attention_key(torch, tba, dev, peaks["hbm_gbs"])
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(args.afmt, args.cpu_tokens_per_core, args.cpu_tokens)
         print(json.dumps(line), flush=True)
@@ -959,6 +960,71 @@ def fp4_gemm_key(torch, tba, layer, reps: int):
     return out
 
 
+ATTN_SHAPE = (32768, 32, 128)   # positions x heads x head_dim of the 7B decode cache
+ATTN_CACHES = 4                 # 4 x 109 MB of codes and scales > the 126 MB L2
+
+
+def attention_key(torch, tba, dev, hbm_peak: float, queries=(1, 2, 4, 8), reps: int = 10):
+    """attention_lowbit in the 7B decode context: M 4-bit queries over a
+    32768-position cache of 32 heads of 128 (3-bit K and V, the BOS position at
+    4 bits).  ATTN_CACHES caches with their own buffers (together larger than L2)
+    are visited in turn, so every call streams its cache from HBM; CUDA events
+    around `reps` passes over the caches.  Algorithmic bytes per call: the K and
+    V codes and scales, 2 * T * H * (3 D / 8 + 4)."""
+    T = torch
+    Tn, H, D = ATTN_SHAPE
+    g = T.Generator(device=dev)
+    g.manual_seed(11)
+
+    def quant(x, bits, bos):
+        n = x.shape[0]
+        c = T.empty((n, H, D * bits // 8), dtype=T.uint8, device=dev)
+        sc = T.empty((n, H), dtype=T.float32, device=dev)
+        b = T.empty((H, D // 2), dtype=T.uint8, device=dev)
+        tba.kv_quant3(x, n, H, D, c, sc, bos_codes=b, bits=bits, bos_pos=bos, eps=EPS)
+        return c, sc, b
+
+    caches = []
+    for _ in range(ATTN_CACHES):
+        kx = T.randn((Tn, H * D), generator=g, device=dev).to(T.bfloat16).view(T.int16)
+        kc, ks, kb = quant(kx, 3, 0)
+        del kx
+        vx = T.randn((Tn, H * D), generator=g, device=dev).to(T.bfloat16).view(T.int16)
+        vc, vs, vb = quant(vx, 3, 0)
+        del vx
+        caches.append((kc, ks, kb, vc, vs, vb))
+    nbytes = 2 * Tn * H * (3 * D // 8 + 4)
+    results = []
+    for m in queries:
+        qx = T.randn((m, H * D), generator=g, device=dev).to(T.bfloat16).view(T.int16)
+        qc, qs, _ = quant(qx, 4, -1)
+        out = T.empty((m, H * D), dtype=T.int16, device=dev)
+        ws = T.empty((tba.workspace_size("attention_lowbit", m, H, D) // 4,), dtype=T.float32, device=dev)
+
+        def one_pass():
+            for kc, ks, kb, vc, vs, vb in caches:
+                tba.attention_lowbit(qc, qs, m, kc, ks, vc, vs, Tn, H, D, out, ws, k_bos=kb, v_bos=vb, kv_bits=3,
+                                     bos_pos=0)
+
+        for _ in range(3):
+            one_pass()
+        a_, b_ = T.cuda.Event(enable_timing=True), T.cuda.Event(enable_timing=True)
+        T.cuda.synchronize()
+        a_.record()
+        for _ in range(reps):
+            one_pass()
+        b_.record()
+        T.cuda.synchronize()
+        us = 1e3 * a_.elapsed_time(b_) / (reps * ATTN_CACHES)
+        gbs = nbytes / (us * 1e-6) / 1e9
+        results.append({"queries": m, "us": round(us, 2), "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm_peak, 3)})
+    tba.sync_status()
+    return {"unit": "us per call", "workload": f"attention_lowbit: M 4-bit queries over a {Tn}-position cache of {H} "
+                                               f"heads x {D} (3-bit K and V, BOS position at 4 bits); "
+                                               f"{ATTN_CACHES} caches visited in turn (larger than L2)",
+            "algorithmic_bytes": nbytes, "hbm_peak_gbs": hbm_peak, "results": results}
+
+
 # ---------------------------------------------------------------------------
 # single-kernel cases for profiler captures (small enough for ncu's replays;
 # inputs still larger than L2)
@@ -973,6 +1039,7 @@ PROFILE_CASES = {
     "sparsify_a8": "Top-K 50% + INT8, X bf16 [32768 x 4096]",
     "relu2_glu": "ReLU^2-GLU + Top-K 50% + INT8, gate/up bf16 [16384 x 11008]",
     "kv_quant3": "3-bit KV, K bf16 [32768 x 32 x 128]",
+    "attention": "low-bit attention, 1 4-bit query over a 3-bit cache [32768 x 32 x 128]",
     "pack_ternary": "ternary pack to int8, W fp32 [22016 x 4096]",
     "gemm_decode": "CUDA-core GEMV, 2-bit W [12288 x 4096], 1 token",
     "gemm_decode_mma": "warp-MMA GEMV, 2-bit W [12288 x 4096], 8 tokens",
@@ -1048,6 +1115,23 @@ def run_profile_case(name: str, launches: int):
         s = torch.empty((T, H), device=dev)
         b = torch.empty((H, D // 2), dtype=torch.uint8, device=dev)
         fn = lambda: tba.kv_quant3(kv, T, H, D, c, s, b, bits=3, bos_pos=0)
+    elif name == "attention":
+        T_, H, D = 32768, 32, 128
+
+        def quant(x, n, bits, bos):
+            c = torch.empty((n, H, D * bits // 8), dtype=torch.uint8, device=dev)
+            s = torch.empty((n, H), device=dev)
+            b = torch.empty((H, D // 2), dtype=torch.uint8, device=dev)
+            tba.kv_quant3(x, n, H, D, c, s, b, bits=bits, bos_pos=bos)
+            return c, s, b
+
+        kc, ks, kb = quant(bf16(T_, H * D), T_, 3, 0)
+        vc, vs, vb = quant(bf16(T_, H * D), T_, 3, 0)
+        qc, qs, _ = quant(bf16(1, H * D), 1, 4, -1)
+        out = torch.empty((1, H * D), dtype=torch.int16, device=dev)
+        ws = torch.empty((tba.workspace_size("attention_lowbit", 1, H, D) // 4,), device=dev)
+        fn = lambda: tba.attention_lowbit(qc, qs, 1, kc, ks, vc, vs, T_, H, D, out, ws, k_bos=kb, v_bos=vb,
+                                          kv_bits=3, bos_pos=0)
     elif name == "pack_ternary":
         w = torch.randn((22016, 4096), generator=g, device=dev) * 0.02
         o = torch.empty((22016, 4096), dtype=torch.uint8, device=dev)
@@ -1074,9 +1158,10 @@ def main(argv=None):
     ap.add_argument("--cpu-tokens-ref", type=int, default=2, help="tokens per thread and step of --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the decode and FP4 keys of the prefill line")
-    ap.add_argument("--workload", choices=["prefill", "decode", "quant-variants"], default="prefill",
+    ap.add_argument("--workload", choices=["prefill", "decode", "quant-variants", "attention"], default="prefill",
                     help="prefill: the headline step; decode: per-token-batch latency sweep; "
-                         "quant-variants: the 4-bit quantizer and its ablation variants at the 7B prefill input")
+                         "quant-variants: the 4-bit quantizer and its ablation variants at the 7B prefill input; "
+                         "attention: low-bit attention over the 7B decode cache")
     ap.add_argument("--decode-tokens", type=int, nargs="+", default=synth.DECODE_TOKENS)
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), help="run one kernel's small case and exit")
     ap.add_argument("--launches", type=int, default=3, help="launches of --profile-case")
@@ -1092,6 +1177,12 @@ def main(argv=None):
         run_decode(args)
     elif args.workload == "quant-variants":
         run_quant_variants(args)
+    elif args.workload == "attention":
+        import torch
+
+        import ternary_bit_activation_b200 as tba
+        torch.cuda.set_device(0)
+        print(json.dumps(attention_key(torch, tba, torch.device("cuda", 0), load_peaks()["hbm_gbs"])), flush=True)
     else:
         run_gpu(args)
 

@@ -345,8 +345,43 @@ BL_API bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D,
                     int64_t bos_pos, float eps, uint8_t* codes, float* scale, uint8_t* bos_codes,
                     void* stream);
 
+/*
+ * attention_lowbit -- softmax attention of 4-bit queries over the low-bit KV
+ * cache that kv_quant3 writes.
+ * Paper: §3.4 "Low-Bit KV Cache Quantization" (post-RoPE Q, K and V quantized
+ * by absmax to unsigned integers; 4-bit Q with 3-bit KV, the BOS position's
+ * heads at 4 bits) and Table 3's "4-bit Q, 3-bit KV" / "4-bit QKV" rows.  The
+ * pages give no attention formula; reading used (softmax over the dequantized
+ * codes):
+ *   q_hat = (q_code - 8) * q_scale,  k_hat_t = (k_code_t - 2^(b-1)) * k_scale_t,
+ *   v_hat_t likewise (b = kv_bits; offset 8 at the BOS position of a 3-bit cache),
+ *   s_t = softmax_scale * <q_hat, k_hat_t>,  out = sum_t softmax(s)_t * v_hat_t.
+ * The M queries are the cache's last M positions: query m sits at position
+ * T - M + m and attends positions 0 .. T - M + m (causal; M = 1 is decode).
+ * q_codes: [M x H x D/2] bytes, 4-bit codes c + 8 (kv_quant3 with bits = 4 on
+ * the query slice).  q_scale: [M x H] fp32.
+ * k_codes / v_codes, k_scale / v_scale, k_bos / v_bos: as kv_quant3 writes them
+ * for T positions (the BOS buffers are read only when kv_bits == 3 and
+ * 0 <= bos_pos < T; bos_pos is ignored for 4-bit caches).
+ * out: [M x ldo] bf16, row m holding head h's D values at h*D .. h*D + D-1
+ * (the O projection's input layout), each rounded once to bf16.
+ * Arithmetic: <q, k> exactly in integers, scores and the softmax in fp32 (base-2
+ * exponentials), fp32 sums; against the fp64 definition the result is within
+ * 2^-8 |out| + 2^-12 max_t |v_hat_t| per element.
+ * workspace: bitlinear_workspace_size("attention_lowbit", M, H, D) bytes,
+ * 16-byte aligned (partial results of the position chunks).
+ * Requires D in {64, 128}, H * D / 32 <= 256, 1 <= M <= min(T, 65535),
+ * T * H < 2^29, ldo >= H * D; k_codes / v_codes 16-byte aligned, the scales
+ * 4-byte aligned.  M = 0 is a no-op.
+ */
+BL_API bl_status attention_lowbit(const uint8_t* q_codes, const float* q_scale, int64_t M, const uint8_t* k_codes,
+                                  const float* k_scale, const uint8_t* k_bos, const uint8_t* v_codes,
+                                  const float* v_scale, const uint8_t* v_bos, int64_t T, int64_t H, int64_t D,
+                                  int kv_bits, int64_t bos_pos, float softmax_scale, void* out_bf16, int64_t ldo,
+                                  void* workspace, size_t ws_bytes, void* stream);
+
 /* Bytes of device workspace an operation needs ("pack_ternary", "quant_a4_per_tensor",
- * "quant_gemm"; 0 for the others). */
+ * "quant_gemm"; "attention_lowbit" with M queries, N = H heads, K = D; 0 for the others). */
 BL_API size_t bitlinear_workspace_size(const char* op, int64_t M, int64_t N, int64_t K);
 
 /* Synchronizes `stream`, then reads and clears the calling device's status

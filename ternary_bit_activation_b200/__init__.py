@@ -29,7 +29,8 @@ BL_W_T2, BL_W_I8, BL_W_E2M1 = 0, 1, 2
 
 EXPORTED = ["bitlinear_quant_a4", "bitlinear_rmsnorm_quant_a4", "bitlinear_quant_a4_per_tensor",
             "bitlinear_sparsify_a8", "pack_ternary", "pack_ternary_noalloc", "bitlinear_gemm",
-            "bitlinear_quant_gemm", "bitlinear_gemm_gated", "relu2_glu", "kv_quant3", "bitlinear_workspace_size",
+            "bitlinear_quant_gemm", "bitlinear_gemm_gated", "relu2_glu", "kv_quant3", "attention_lowbit",
+            "bitlinear_workspace_size",
             "bitlinear_sync_status", "bitlinear_selftest_timeout", "bitlinear_status_string",
             "bitlinear_last_cuda_error", "bitlinear_version"]
 
@@ -65,6 +66,8 @@ def lib():
             "bitlinear_gemm_gated": [P, I, P, P, I, P, I64, I64, I64, P, I64, P, P],
             "relu2_glu": [P, P, I64, I64, I64, I64, F, P, P, P, P],
             "kv_quant3": [P, I64, I64, I64, I64, I, I64, F, P, P, P, P],
+            "attention_lowbit": [P, P, I64, P, P, P, P, P, P, I64, I64, I64, I, I64, F, P, I64, P, ctypes.c_size_t,
+                                 P],
             "bitlinear_sync_status": [P],
             "bitlinear_selftest_timeout": [P],
         }
@@ -202,6 +205,22 @@ def kv_quant3(kv, T, H, D, codes, scale, bos_codes=None, bits=3, bos_pos=0, eps=
     ldt = H * D if ldt is None else ldt
     _check("kv_quant3", lib().kv_quant3(_ptr(kv), T, H, D, ldt, bits, bos_pos, eps, _ptr(codes), _ptr(scale),
                                         _ptr(bos_codes), _stream(stream)))
+
+
+def attention_lowbit(q_codes, q_scale, M, k_codes, k_scale, v_codes, v_scale, T, H, D, out, workspace,
+                     k_bos=None, v_bos=None, kv_bits=3, bos_pos=0, softmax_scale=None, ldo=None, ws_bytes=None,
+                     stream=None):
+    """Softmax attention of M 4-bit queries (the cache's last M positions) over
+    the kv_quant3 cache of T positions; out: [M x ldo] bf16."""
+    ldo = H * D if ldo is None else ldo
+    if softmax_scale is None:
+        softmax_scale = float(1.0 / (D ** 0.5))
+    if ws_bytes is None:
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("attention_lowbit", lib().attention_lowbit(_ptr(q_codes), _ptr(q_scale), M, _ptr(k_codes), _ptr(k_scale),
+                                                      _ptr(k_bos), _ptr(v_codes), _ptr(v_scale), _ptr(v_bos), T, H,
+                                                      D, kv_bits, bos_pos, softmax_scale, _ptr(out), ldo,
+                                                      _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def workspace_size(op: str, M: int = 0, N: int = 0, K: int = 0) -> int:

@@ -13,6 +13,7 @@
 #endif
 
 #include "bitlinear.h"
+#include "attn.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
 #include "kv.cuh"
@@ -576,6 +577,57 @@ constexpr int64_t kQgFusedMaxTokens = 2;
 int64_t qg_codes_bytes(int64_t M, int64_t K) { return (M * K + 15) / 16 * 16; }
 int64_t qg_workspace_bytes(int64_t M, int64_t K) { return qg_codes_bytes(M, K) + (4 * M + 15) / 16 * 16; }
 
+// ---------------------------------------------------------------------------
+// Low-bit attention: position chunks spread over one resident wave of CTAs
+// ---------------------------------------------------------------------------
+size_t attn_workspace_bytes(int64_t M, int64_t H, int64_t D) {
+  return static_cast<size_t>(bl::kAttnMaxChunks) * static_cast<size_t>(M) * static_cast<size_t>(H) *
+         static_cast<size_t>(D + 4) * sizeof(float);
+}
+
+template <int D, int BITS>
+bl_status launch_attention(bl::AttnParams a, cudaStream_t s) {
+  auto kern = bl::attn_partial_kernel<D, BITS>;
+  int group = bl::kAttnThreads / (a.H * (D / 32));
+  if (group > bl::kAttnMaxGroup) group = bl::kAttnMaxGroup;
+  if (group > a.M) group = a.M;
+  const int ngroups = (a.M + group - 1) / group;
+  const size_t smem = bl::attn_smem_bytes<D, BITS>(group, a.H);
+  // per device: the largest shared-memory size set so far, and the occupancy of the last size asked for
+  static int smem_set[kMaxDevices] = {};
+  static size_t occ_smem[kMaxDevices] = {};
+  static int occ_val[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return BL_ERR_CUDA;
+  if (static_cast<int>(smem) > smem_set[dev]) {
+    if (!cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))))
+      return BL_ERR_CUDA;
+    smem_set[dev] = static_cast<int>(smem);
+  }
+  if (occ_smem[dev] != smem || occ_val[dev] == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, bl::kAttnThreads, smem) != cudaSuccess || n < 1) n = 1;
+    occ_smem[dev] = smem;
+    occ_val[dev] = n;
+  }
+  int64_t target = static_cast<int64_t>(sm_count()) * occ_val[dev] / ngroups;
+  if (target < 1) target = 1;
+  if (target > bl::kAttnMaxChunks) target = bl::kAttnMaxChunks;
+  if (target > a.T) target = a.T;
+  const int chunk = static_cast<int>((a.T + target - 1) / target);
+  a.group = group;
+  a.chunk = chunk;
+  a.nchunks = (a.T + chunk - 1) / chunk;
+  const int nblk = (chunk + bl::kAttnMaxPos - 1) / bl::kAttnMaxPos;
+  a.blk = (chunk + nblk - 1) / nblk;
+  launch_pdl(kern, dim3(static_cast<unsigned>(a.nchunks), static_cast<unsigned>(ngroups)), bl::kAttnThreads, smem,
+             s, a);
+  if (launch_status() != BL_OK) return BL_ERR_CUDA;
+  launch_pdl(bl::attn_combine_kernel<D, BITS>, dim3(static_cast<unsigned>(a.H), static_cast<unsigned>(a.M)), D, 0,
+             s, a);
+  return launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -639,11 +691,12 @@ const char* bitlinear_status_string(bl_status st) {
 }
 
 size_t bitlinear_workspace_size(const char* op, int64_t M, int64_t N, int64_t K) {
-  (void)N;
   if (op != nullptr && (strcmp(op, "pack_ternary") == 0 || strcmp(op, "quant_a4_per_tensor") == 0))
     return bl::kBins * sizeof(unsigned long long);
   if (op != nullptr && strcmp(op, "quant_gemm") == 0 && M > 0 && K > 0)
     return static_cast<size_t>(qg_workspace_bytes(M, K));
+  if (op != nullptr && strcmp(op, "attention_lowbit") == 0 && M > 0 && N > 0 && K > 0)
+    return attn_workspace_bytes(M, N, K);
   return 0;
 }
 
@@ -1087,6 +1140,49 @@ bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D, int64_
     default: return BL_ERR_SHAPE;
   }
   return launch_status();
+}
+
+bl_status attention_lowbit(const uint8_t* q_codes, const float* q_scale, int64_t M, const uint8_t* k_codes,
+                           const float* k_scale, const uint8_t* k_bos, const uint8_t* v_codes, const float* v_scale,
+                           const uint8_t* v_bos, int64_t T, int64_t H, int64_t D, int kv_bits, int64_t bos_pos,
+                           float softmax_scale, void* out_bf16, int64_t ldo, void* workspace, size_t ws_bytes,
+                           void* stream) {
+  NvtxRange nvtx_range("attention_lowbit");
+  if (kv_bits != 3 && kv_bits != 4) return BL_ERR_ARG;
+  if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f) return BL_ERR_ARG;
+  if (bos_pos < -1) return BL_ERR_ARG;
+  if ((D != 64 && D != 128) || H < 1 || H * (D / 32) > bl::kAttnThreads) return BL_ERR_SHAPE;
+  if (T < 1 || M < 0 || M > T || M > 65535 || T > 0x7FFFFFFFLL / 4 / H || ldo < H * D) return BL_ERR_SHAPE;
+  if (M == 0) return BL_OK;
+  const bool has_bos = kv_bits == 3 && bos_pos >= 0 && bos_pos < T;
+  if (q_codes == nullptr || q_scale == nullptr || k_codes == nullptr || k_scale == nullptr || v_codes == nullptr ||
+      v_scale == nullptr || out_bf16 == nullptr || workspace == nullptr || (has_bos && (k_bos == nullptr || v_bos == nullptr)))
+    return BL_ERR_NULL;
+  if (!aligned16(k_codes) || !aligned16(v_codes) || !aligned16(workspace) ||
+      ((reinterpret_cast<uintptr_t>(q_scale) | reinterpret_cast<uintptr_t>(k_scale) |
+        reinterpret_cast<uintptr_t>(v_scale)) & 3u) || (reinterpret_cast<uintptr_t>(out_bf16) & 1u))
+    return BL_ERR_ALIGN;
+  if (ws_bytes < attn_workspace_bytes(M, H, D)) return BL_ERR_WORKSPACE;
+  bl::AttnParams a = {};
+  a.q = q_codes;
+  a.qs = q_scale;
+  a.k = k_codes;
+  a.ks = k_scale;
+  a.v = v_codes;
+  a.vs = v_scale;
+  a.kbos = k_bos;
+  a.vbos = v_bos;
+  a.M = static_cast<int>(M);
+  a.T = static_cast<int>(T);
+  a.H = static_cast<int>(H);
+  a.bos = has_bos ? static_cast<int>(bos_pos) : -1;
+  a.coef = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);   // log2(e)
+  a.part = static_cast<float*>(workspace);
+  a.out = static_cast<uint16_t*>(out_bf16);
+  a.ldo = ldo;
+  cudaStream_t s = as_stream(stream);
+  if (D == 128) return kv_bits == 3 ? launch_attention<128, 3>(a, s) : launch_attention<128, 4>(a, s);
+  return kv_bits == 3 ? launch_attention<64, 3>(a, s) : launch_attention<64, 4>(a, s);
 }
 
 }  // extern "C"

@@ -190,6 +190,39 @@ def test_pack_and_kv_validation(L):
     assert kv(P(A16), 8, 4, 128, 512, 3, 0, 1e-5, P(A16), P(A16), None, None) == 1       # BOS buffer needed
 
 
+def test_attention_validation(L):
+    at = L.attention_lowbit
+    ws = tba.workspace_size("attention_lowbit", 1, 32, 128)
+    assert ws == 512 * 32 * 132 * 4
+    ok = dict(q=A16, qs=A16, M=1, k=A16, ks=A16, kb=A16, v=A16, vs=A16, vb=A16, T=100, H=32, D=128, bits=3, bos=0,
+              sm=0.088, out=A16, ldo=4096, ws=A16, wsb=ws)
+
+    def call(**kw):
+        d = dict(ok, **kw)
+        return at(P(d["q"]), P(d["qs"]), d["M"], P(d["k"]), P(d["ks"]), P(d["kb"]), P(d["v"]), P(d["vs"]),
+                  P(d["vb"]), d["T"], d["H"], d["D"], d["bits"], d["bos"], d["sm"], P(d["out"]), d["ldo"],
+                  P(d["ws"]), d["wsb"], None)
+
+    assert call(bits=2) == 4
+    assert call(bos=-2) == 4
+    assert call(sm=float("nan")) == 4
+    assert call(D=32) == 3 and call(D=256) == 3
+    assert call(H=128, ldo=128 * 128) == 3          # H * D / 32 > 256
+    assert call(M=101) == 3                         # more queries than positions
+    assert call(ldo=4095) == 3
+    assert call(T=1 << 30) == 3
+    assert call(M=0) == 0
+    assert call(kb=None) == 1                       # a 3-bit cache with a BOS position needs its 4-bit row
+    # ... a 4-bit cache does not, nor one without a BOS position: the call gets past the
+    # null checks to the workspace check
+    assert call(kb=None, vb=None, bits=4, wsb=ws - 1) == 8
+    assert call(kb=None, vb=None, bos=-1, wsb=ws - 1) == 8
+    assert call(k=MIS) == 2
+    assert call(ws=MIS) == 2
+    assert call(wsb=ws - 1) == 8
+    assert call(ws=None) == 1
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(tba, "_lib", None)
     monkeypatch.setattr(tba, "LIB_PATH", str(tmp_path / "nope.so"))
