@@ -367,11 +367,12 @@ BL_API bl_status kv_quant3(const void* kv_bf16, int64_t T, int64_t H, int64_t D,
  * (the O projection's input layout), each rounded once to bf16.
  * Arithmetic: <q, k> exactly in integers, scores and the softmax in fp32 (base-2
  * exponentials), fp32 sums; against the fp64 definition the result is within
- * 2^-8 |out| + 2^-12 max_t |v_hat_t| per element.
+ * 2^-8 |out| + 2^-12 max_t |v_hat_t| per element.  The contract covers k_scale
+ * and v_scale values between 2^-40 and 2^40 (the V sums carry a 2^64 factor).
  * workspace: bitlinear_workspace_size("attention_lowbit", M, H, D) bytes,
  * 16-byte aligned (partial results of the position chunks).
- * Requires D in {64, 128}, H * D / 32 <= 256, 1 <= M <= min(T, 65535),
- * T * H < 2^29, ldo >= H * D; k_codes / v_codes 16-byte aligned, the scales
+ * Requires D in {64, 128}, H % 4 == 0, H * D / 32 <= 256, 1 <= M <= min(T, 65535),
+ * T * H < 2^29, ldo >= H * D; q_codes / k_codes / v_codes 16-byte aligned, the scales
  * 4-byte aligned.  M = 0 is a no-op.
  */
 BL_API bl_status attention_lowbit(const uint8_t* q_codes, const float* q_scale, int64_t M, const uint8_t* k_codes,

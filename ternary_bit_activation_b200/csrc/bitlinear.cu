@@ -585,14 +585,12 @@ size_t attn_workspace_bytes(int64_t M, int64_t H, int64_t D) {
          static_cast<size_t>(D + 4) * sizeof(float);
 }
 
-template <int D, int BITS>
-bl_status launch_attention(bl::AttnParams a, cudaStream_t s) {
-  auto kern = bl::attn_partial_kernel<D, BITS>;
-  int group = bl::kAttnThreads / (a.H * (D / 32));
-  if (group > bl::kAttnMaxGroup) group = bl::kAttnMaxGroup;
-  if (group > a.M) group = a.M;
+template <int D, int BITS, int HG, bool ONE>
+bl_status launch_attention_hg(bl::AttnParams a, int group, cudaStream_t s) {
+  auto kern = bl::attn_partial_kernel<D, BITS, HG, ONE>;
   const int ngroups = (a.M + group - 1) / group;
-  const size_t smem = bl::attn_smem_bytes<D, BITS>(group, a.H);
+  const int nheadgroups = a.H / HG;
+  const size_t smem = bl::AttnSmem<D, BITS, HG>(group).total;
   // per device: the largest shared-memory size set so far, and the occupancy of the last size asked for
   static int smem_set[kMaxDevices] = {};
   static size_t occ_smem[kMaxDevices] = {};
@@ -610,22 +608,46 @@ bl_status launch_attention(bl::AttnParams a, cudaStream_t s) {
     occ_smem[dev] = smem;
     occ_val[dev] = n;
   }
-  int64_t target = static_cast<int64_t>(sm_count()) * occ_val[dev] / ngroups;
+  // one resident wave of CTAs over (chunks, head groups, query groups); chunks are whole blocks
+  constexpr int kPos = bl::AttnSmem<D, BITS, HG>::kPos;
+  constexpr int kVB = bl::AttnShape<D, BITS>::kVecBytes;
+  CUtensorMap tk, tv, tks, tvs;
+  const uint64_t rows = static_cast<uint64_t>(a.T);
+  if (!make_u64_map(&tk, a.k, rows, static_cast<uint64_t>(a.H) * kVB, kPos, HG * kVB) ||
+      !make_u64_map(&tv, a.v, rows, static_cast<uint64_t>(a.H) * kVB, kPos, HG * kVB) ||
+      !make_u64_map(&tks, a.ks, rows, static_cast<uint64_t>(a.H) * 4, kPos, HG * 4) ||
+      !make_u64_map(&tvs, a.vs, rows, static_cast<uint64_t>(a.H) * 4, kPos, HG * 4))
+    return BL_ERR_CUDA;
+  int64_t target = static_cast<int64_t>(sm_count()) * occ_val[dev] / (static_cast<int64_t>(ngroups) * nheadgroups);
   if (target < 1) target = 1;
   if (target > bl::kAttnMaxChunks) target = bl::kAttnMaxChunks;
-  if (target > a.T) target = a.T;
-  const int chunk = static_cast<int>((a.T + target - 1) / target);
+  int64_t chunk = (a.T + target - 1) / target;
+  chunk = (chunk + kPos - 1) / kPos * kPos;
   a.group = group;
-  a.chunk = chunk;
-  a.nchunks = (a.T + chunk - 1) / chunk;
-  const int nblk = (chunk + bl::kAttnMaxPos - 1) / bl::kAttnMaxPos;
-  a.blk = (chunk + nblk - 1) / nblk;
-  launch_pdl(kern, dim3(static_cast<unsigned>(a.nchunks), static_cast<unsigned>(ngroups)), bl::kAttnThreads, smem,
-             s, a);
+  a.chunk = static_cast<int>(chunk);
+  a.nchunks = static_cast<int>((a.T + chunk - 1) / chunk);
+  launch_pdl(kern, dim3(static_cast<unsigned>(a.nchunks), static_cast<unsigned>(nheadgroups),
+                        static_cast<unsigned>(ngroups)),
+             bl::kAttnThreads, smem, s, tk, tv, tks, tvs, a);
   if (launch_status() != BL_OK) return BL_ERR_CUDA;
-  launch_pdl(bl::attn_combine_kernel<D, BITS>, dim3(static_cast<unsigned>(a.H), static_cast<unsigned>(a.M)), D, 0,
-             s, a);
+  launch_pdl(bl::attn_combine_kernel<D, BITS>,
+             dim3(static_cast<unsigned>(a.H), static_cast<unsigned>(a.M), static_cast<unsigned>(D / 32)),
+             bl::kAttnThreads, 0, s, a);
   return launch_status();
+}
+
+template <int D, int BITS, int HG>
+bl_status launch_attention_g(const bl::AttnParams& a, cudaStream_t s) {
+  int group = bl::kAttnThreads / (HG * (D / 32));
+  if (group > bl::kAttnMaxGroup) group = bl::kAttnMaxGroup;
+  if (group > a.M) group = a.M;
+  return group == 1 ? launch_attention_hg<D, BITS, HG, true>(a, 1, s)
+                    : launch_attention_hg<D, BITS, HG, false>(a, group, s);
+}
+
+template <int D, int BITS>
+bl_status launch_attention(const bl::AttnParams& a, cudaStream_t s) {
+  return (a.H % 8 == 0) ? launch_attention_g<D, BITS, 8>(a, s) : launch_attention_g<D, BITS, 4>(a, s);
 }
 
 }  // namespace
@@ -1151,14 +1173,14 @@ bl_status attention_lowbit(const uint8_t* q_codes, const float* q_scale, int64_t
   if (kv_bits != 3 && kv_bits != 4) return BL_ERR_ARG;
   if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f) return BL_ERR_ARG;
   if (bos_pos < -1) return BL_ERR_ARG;
-  if ((D != 64 && D != 128) || H < 1 || H * (D / 32) > bl::kAttnThreads) return BL_ERR_SHAPE;
+  if ((D != 64 && D != 128) || H < 4 || (H & 3) || H * (D / 32) > bl::kAttnThreads) return BL_ERR_SHAPE;
   if (T < 1 || M < 0 || M > T || M > 65535 || T > 0x7FFFFFFFLL / 4 / H || ldo < H * D) return BL_ERR_SHAPE;
   if (M == 0) return BL_OK;
   const bool has_bos = kv_bits == 3 && bos_pos >= 0 && bos_pos < T;
   if (q_codes == nullptr || q_scale == nullptr || k_codes == nullptr || k_scale == nullptr || v_codes == nullptr ||
       v_scale == nullptr || out_bf16 == nullptr || workspace == nullptr || (has_bos && (k_bos == nullptr || v_bos == nullptr)))
     return BL_ERR_NULL;
-  if (!aligned16(k_codes) || !aligned16(v_codes) || !aligned16(workspace) ||
+  if (!aligned16(q_codes) || !aligned16(k_codes) || !aligned16(v_codes) || !aligned16(workspace) ||
       ((reinterpret_cast<uintptr_t>(q_scale) | reinterpret_cast<uintptr_t>(k_scale) |
         reinterpret_cast<uintptr_t>(v_scale)) & 3u) || (reinterpret_cast<uintptr_t>(out_bf16) & 1u))
     return BL_ERR_ALIGN;
