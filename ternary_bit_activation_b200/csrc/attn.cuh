@@ -378,11 +378,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const uint8_t* vst = st + L::kCodes;
     const float* kss = reinterpret_cast<const float*>(st + 2 * L::kCodes);
     const float* vss = kss + NPAIR;
-    const bool ok = mbar_wait_bounded(&bars[b % NS], static_cast<uint32_t>((b / NS) & 1));
-    if (__syncthreads_or(ok ? 0 : 1)) {   // one decision for the CTA
-      aborted = true;
-      break;
-    }
+    // each thread waits for the block itself (a wait that runs out is noted and the
+    // CTA decides after the loop)
+    if (!mbar_wait_bounded(&bars[b % NS], static_cast<uint32_t>((b / NS) & 1))) aborted = true;
     {
       // scores of the two pairs for every query, and each warp's maximum per head
       uint32_t kw0[S::kVecWords], kw1[S::kVecWords];
@@ -490,9 +488,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     __syncthreads();   // the stage, the scores and the maxima are free again
     if (threadIdx.x == 0) issue(b + NS);
   }
-  if (aborted) {
-    // a wait ran out: let copies still in flight land before the CTA's shared
-    // memory is released, and write nothing (the status word reports the timeout)
+  // one decision for the CTA: after a wait ran out, let copies still in flight land
+  // before the CTA's shared memory is released, and write nothing (the status word
+  // reports the timeout)
+  if (__syncthreads_or(aborted ? 1 : 0)) {
     const uint64_t tw = globaltimer_ns();
     while (globaltimer_ns() - tw < 200000ull) {
     }
