@@ -305,6 +305,29 @@ def test_relu2_glu_ties_and_no_mask():
         assert np.array_equal(host(s2).view(np.uint32), ref[3].view(np.uint32))
 
 
+def test_relu2_glu_subnormal_cut():
+    # h = up * relu(gate)^2 subnormal in fp32 for part of each row, and the cut among
+    # those values: the selection's first digit (the exponent) is then 0, the digit
+    # the zero keys share, so the zeros stay candidates in the later digits
+    g = synth.rng(123)
+    M, F = 4, 2048
+    gate = np.where(g.random((M, F)) < 0.5, -1.0, 1.0) * g.uniform(0.5, 1.5, (M, F))
+    up = g.standard_normal((M, F))
+    small = g.random((M, F)) < 0.6                    # these positions get a subnormal h
+    gate = np.where(small, gate * 1e-15, gate)
+    up = np.where(small, up * 1e-10, up)
+    gate_b = synth.f32_to_bf16_bits(gate.astype(np.float32))
+    up_b = synth.f32_to_bf16_bits(up.astype(np.float32))
+    h = synth.bf16_bits_to_f32(up_b).astype(np.float32) * np.maximum(synth.bf16_bits_to_f32(gate_b), 0) ** 2
+    nz = (h != 0).sum(axis=1)
+    normal = (np.abs(h) >= np.float32(2.0 ** -126)).sum(axis=1)
+    keep = int(normal.max() + (nz.min() - normal.max()) // 2)   # between the normal and the nonzero counts
+    assert (normal < keep).all() and (nz > keep).all()
+    ref = oracle.relu2_glu(gate_b, up_b, keep, EPS)
+    codes, scale, mask = run_relu2(gate_b, up_b, keep)
+    check_topk(codes, scale, mask, ref)
+
+
 def run_kv(kv, bits, bos_pos, ldt_pad=0):
     T, H, D = kv.shape
     buf = np.zeros((T, H * D + ldt_pad), np.uint16)
