@@ -36,7 +36,7 @@
 
 namespace bl {
 
-constexpr int kAttnThreads = 256;     // also the (position, head) pairs of one block
+constexpr int kAttnThreads = 256;     // threads per CTA (two (position, head) pairs of a block each)
 constexpr int kAttnMaxGroup = 8;      // queries per CTA
 constexpr int kAttnMaxChunks = 512;   // position chunks per (query group, head group)
 constexpr int kAttnAcc = 34;          // per V thread: 32 sums, the weight sum, the probability sum
