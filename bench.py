@@ -231,7 +231,10 @@ class Layer:
         N_K = {"qkv": (3 * d, d), "o": (d, d), "upgate": (2 * f, d), "down": (d, f)}
         self.gemm_ops = {k: 2.0 * m * n * kk for k, (n, kk) in N_K.items()}
         self.weights = sum(n * kk for n, kk in N_K.values())
-        self.launches_per_step = 5 * 3 + 2 + 4 + 2 + 1 + 1
+        # kernels of this library per step: exact-sum + pack for each of the five weight
+        # tensors (each call also enqueues a 2 KiB workspace memset, not counted), two
+        # quantizers, four GEMMs, two KV quantizers, sparsify, ReLU^2-GLU
+        self.launches_per_step = 5 * 2 + 2 + 4 + 2 + 1 + 1
 
     def alg_gemm_ops(self):
         """2 N nnz(A) per step: QKV and Up|Gate dense, O and Down with the
