@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kBinThreads, 6) ternary_bins_kernel(const void
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kBinThreads) >> 5;
   constexpr int kLoads = 4;   // float4 loads per lane issued together (16 weights)
   uint32_t ub = 0;            // 0: not anchored yet
-  uint32_t lo_bits = 0;       // ub << 23
+  uint32_t lo_bits = 0x7F800000u;   // ub << 23 once anchored; before that no finite value is in the window
   double acc = 0.0;
   int batches = 0;
   for (int64_t n = gwarp; n < N; n += nwarps) {
@@ -124,13 +124,11 @@ __global__ void __launch_bounds__(kBinThreads, 6) ternary_bins_kernel(const void
       for (int i = 0; i < kPer * kLoads; ++i) {
         const uint32_t a = u[i];
         if (a - lo_bits < (kWin << 23)) {
-          // exact: inside the window a is a normal fp32 (biased exponent >= 1), so
-          // its fp64 is built from the bits -- exponent rebiased by 1023 - 127,
+          // exact: inside the window a is a normal fp32 (biased exponent >= ub >= 1),
+          // so its fp64 is built from the bits -- exponent rebiased by 1023 - 127,
           // significand shifted up by 29 -- with integer operations instead of
-          // the conversion unit; before the anchor a is 0 and so is the double
-          acc += a != 0u ? __hiloint2double(static_cast<int>((a >> 3) + ((1023u - 127u) << 20)),
-                                            static_cast<int>(a << 29))
-                         : 0.0;
+          // the conversion unit
+          acc += __hiloint2double(static_cast<int>((a >> 3) + ((1023u - 127u) << 20)), static_cast<int>(a << 29));
         } else if (a != 0) {
           const uint32_t E = a >> 23;
           const uint32_t m = (a & 0x7FFFFFu) | (E ? 0x800000u : 0u);
