@@ -87,6 +87,13 @@ def test_attention_pipeline_parity(D, bits, bos_pos, T, H, M):
     pipeline_case(11 + T + D, T, H, D, M, bits, bos_pos)
 
 
+@pytest.mark.parametrize("bits,bos_pos", [(3, 0), (4, -1)])
+@pytest.mark.parametrize("M", [1, 5])
+def test_attention_700m_heads(bits, bos_pos, M):
+    # the 700M shape: 12 heads of 128 (d = 1536), so head groups of 4 heads, three of them
+    pipeline_case(53 + M, 2500, 12, 128, M, bits, bos_pos)
+
+
 @pytest.mark.parametrize("bits", [3, 4])
 def test_attention_peaked_scores(bits):
     # large softmax scale: a few positions dominate (scores spread over tens of units)
